@@ -1,0 +1,206 @@
+"""Float64 CPU oracle for Flint decode attention (test infrastructure only).
+
+Only ``tests/``, ``__graft_entry__.smoke()`` and the CPU-baseline leg of
+``bench.py`` may import this package.  The product path (the CUDA library and
+its Python binding) never imports it and shares no code with it.
+
+``flint_oracle.c`` holds the arithmetic; this module builds it with gcc and
+marshals numpy arrays through ctypes.  bf16 values travel as uint16 bit
+patterns.  Every function is pinned by tests in ``tests/test_oracle_pins.py``.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import subprocess
+import threading
+
+import numpy as np
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_SRC = os.path.join(_HERE, "flint_oracle.c")
+_LIB_PATH = os.path.join(_HERE, "libflint_oracle.so")
+_lock = threading.Lock()
+_lib = None
+
+# Storage layouts of the oracle's own cache model.
+CONTIGUOUS, RING, PAGED = 0, 1, 2
+
+
+def build(force: bool = False) -> str:
+    """Compile flint_oracle.c into libflint_oracle.so (plain -O2, IEEE math)."""
+    if force or not os.path.exists(_LIB_PATH) or (
+            os.path.getmtime(_LIB_PATH) < os.path.getmtime(_SRC)):
+        tmp = _LIB_PATH + f".{os.getpid()}.tmp"
+        subprocess.run(["gcc", "-O2", "-std=c11", "-fPIC", "-shared", "-fopenmp",
+                        "-o", tmp, _SRC, "-lm"], check=True)
+        os.replace(tmp, _LIB_PATH)
+    return _LIB_PATH
+
+
+def _load():
+    global _lib
+    with _lock:
+        if _lib is None:
+            lib = ctypes.CDLL(build())
+            P = ctypes.c_void_p
+            I, L, D = ctypes.c_int, ctypes.c_long, ctypes.c_double
+            lib.fo_bf16_to_f64_array.argtypes = [P, P, L]
+            lib.fo_f64_to_bf16_array.argtypes = [P, P, L]
+            lib.fo_rmsnorm_rows.argtypes = [P, I, I, P, D, P]
+            lib.fo_rope_rows.argtypes = [P, I, I, L, D]
+            lib.fo_qk_norm_rope.argtypes = [P, P, P, P, I, I, I, L, D, D, I, P, P, P]
+            lib.fo_storage_row.argtypes = [I, L, I, P, I]
+            lib.fo_storage_row.restype = L
+            lib.fo_kv_append.argtypes = [P, P, I, I, P, I, I, I, L, P, P]
+            lib.fo_attn_decode.argtypes = [P, I, I, I, P, P, I, I, P, I, L, I, P, P, I]
+            lib.fo_attn_decode.restype = I
+            lib.fo_decode_layer.argtypes = [P, P, P, P, P, P, I, I, I, P, P, I, I, P,
+                                            I, L, I, I, D, D, P, I]
+            lib.fo_decode_layer.restype = I
+            lib.fo_kv_bytes.argtypes = [L, I, I, I, I, I, I]
+            lib.fo_kv_bytes.restype = D
+            lib.fo_num_threads.restype = I
+            _lib = lib
+    return _lib
+
+
+def _u16(a) -> np.ndarray:
+    a = np.asarray(a)
+    if a.dtype != np.uint16:
+        raise TypeError(f"expected bf16 bit patterns as uint16, got {a.dtype}")
+    return np.ascontiguousarray(a)
+
+
+def _f64(a) -> np.ndarray:
+    return np.ascontiguousarray(np.asarray(a, dtype=np.float64))
+
+
+def _ptr(a):
+    return None if a is None else a.ctypes.data_as(ctypes.c_void_p)
+
+
+def num_threads() -> int:
+    return _load().fo_num_threads()
+
+
+def bf16_to_f64(bits) -> np.ndarray:
+    b = _u16(bits)
+    out = np.empty(b.shape, np.float64)
+    _load().fo_bf16_to_f64_array(_ptr(b), _ptr(out), b.size)
+    return out
+
+
+def f64_to_bf16(x) -> np.ndarray:
+    x = _f64(x)
+    out = np.empty(x.shape, np.uint16)
+    _load().fo_f64_to_bf16_array(_ptr(x), _ptr(out), x.size)
+    return out
+
+
+def rmsnorm(x, w=None, eps: float = 1e-6) -> np.ndarray:
+    """x [rows, d] float64, w [d] float64 or None."""
+    x = _f64(x)
+    rows, d = x.shape
+    w = None if w is None else _f64(w)
+    y = np.empty_like(x)
+    _load().fo_rmsnorm_rows(_ptr(x), rows, d, _ptr(w), eps, _ptr(y))
+    return y
+
+
+def rope(x, pos: int, theta: float = 10000.0) -> np.ndarray:
+    """Rotate-half RoPE of rows x [rows, d] at absolute position pos."""
+    y = _f64(x).copy()
+    rows, d = y.shape
+    _load().fo_rope_rows(_ptr(y), rows, d, int(pos), float(theta))
+    return y
+
+
+def qk_norm_rope(q_raw, k_raw, w_q, w_k, pos: int, eps: float = 1e-6,
+                 theta: float = 10000.0, apply_rope: bool = True):
+    """Returns (q f64 [nq,d], k f64 [nkv,d], k bf16 bits [nkv,d])."""
+    q_raw, k_raw = _u16(q_raw), _u16(k_raw)
+    w_q = None if w_q is None else _u16(w_q)
+    w_k = None if w_k is None else _u16(w_k)
+    nq, d = q_raw.shape
+    nkv = k_raw.shape[0]
+    q = np.empty((nq, d), np.float64)
+    k = np.empty((nkv, d), np.float64)
+    kb = np.empty((nkv, d), np.uint16)
+    _load().fo_qk_norm_rope(_ptr(q_raw), _ptr(k_raw), _ptr(w_q), _ptr(w_k), nq, nkv, d,
+                            int(pos), float(eps), float(theta), int(bool(apply_rope)),
+                            _ptr(q), _ptr(k), _ptr(kb))
+    return q, k, kb
+
+
+def storage_row(layout: int, pos: int, capacity: int = 0, block_table=None,
+                block_size: int = 64) -> int:
+    bt = None if block_table is None else np.ascontiguousarray(block_table, np.int32)
+    return _load().fo_storage_row(layout, int(pos), int(capacity), _ptr(bt), int(block_size))
+
+
+def kv_append(k_cache, v_cache, layout: int, pos: int, k, v, capacity: int = 0,
+              block_table=None, block_size: int = 64):
+    """In place: writes k, v [nkv, d] bf16 bits at pos of uint16 caches whose
+    trailing dims are [nkv, d]."""
+    for c in (k_cache, v_cache):
+        if c.dtype != np.uint16 or not c.flags["C_CONTIGUOUS"]:
+            raise TypeError("caches must be C-contiguous uint16 arrays")
+    k, v = _u16(k), _u16(v)
+    nkv, d = k.shape
+    bt = None if block_table is None else np.ascontiguousarray(block_table, np.int32)
+    _load().fo_kv_append(_ptr(k_cache), _ptr(v_cache), layout, int(capacity), _ptr(bt),
+                         int(block_size), nkv, d, int(pos), _ptr(k), _ptr(v))
+
+
+def attn_decode(q, k_cache, v_cache, L: int, sinks, window: int = 0,
+                layout: int = CONTIGUOUS, capacity: int = 0, block_table=None,
+                block_size: int = 64, nthreads: int = 0) -> np.ndarray:
+    """One request's decode attention; q [nq, d] float64 (or bf16 bits),
+    caches uint16 with trailing dims [nkv, d]; returns float64 [nq, d]."""
+    q = bf16_to_f64(q) if np.asarray(q).dtype == np.uint16 else _f64(q)
+    nq, d = q.shape
+    k_cache, v_cache = _u16(k_cache), _u16(v_cache)
+    nkv = k_cache.shape[-2]
+    if k_cache.shape[-1] != d:
+        raise ValueError("head_dim mismatch")
+    sinks = _f64(sinks)
+    bt = None if block_table is None else np.ascontiguousarray(block_table, np.int32)
+    out = np.empty((nq, d), np.float64)
+    rc = _load().fo_attn_decode(_ptr(q), nq, nkv, d, _ptr(k_cache), _ptr(v_cache), layout,
+                                int(capacity), _ptr(bt), int(block_size), int(L), int(window),
+                                _ptr(sinks), _ptr(out), int(nthreads))
+    if rc != 0:
+        raise ValueError("oracle rejected the arguments")
+    return out
+
+
+def decode_layer(q_raw, k_raw, v_raw, w_q, w_k, sinks, k_cache, v_cache, L: int,
+                 window: int, apply_rope: bool, layout: int = CONTIGUOUS,
+                 capacity: int = 0, block_table=None, block_size: int = 64,
+                 eps: float = 1e-6, theta: float = 10000.0, nthreads: int = 0):
+    """norm (+RoPE) -> append at L-1 -> attend; modifies the caches in place."""
+    q_raw, k_raw, v_raw = _u16(q_raw), _u16(k_raw), _u16(v_raw)
+    w_q = None if w_q is None else _u16(w_q)
+    w_k = None if w_k is None else _u16(w_k)
+    for c in (k_cache, v_cache):
+        if c.dtype != np.uint16 or not c.flags["C_CONTIGUOUS"]:
+            raise TypeError("caches must be C-contiguous uint16 arrays")
+    nq, d = q_raw.shape
+    nkv = k_raw.shape[0]
+    sinks = _f64(sinks)
+    bt = None if block_table is None else np.ascontiguousarray(block_table, np.int32)
+    out = np.empty((nq, d), np.float64)
+    rc = _load().fo_decode_layer(_ptr(q_raw), _ptr(k_raw), _ptr(v_raw), _ptr(w_q), _ptr(w_k),
+                                 _ptr(sinks), nq, nkv, d, _ptr(k_cache), _ptr(v_cache), layout,
+                                 int(capacity), _ptr(bt), int(block_size), int(L), int(window),
+                                 int(bool(apply_rope)), float(eps), float(theta), _ptr(out),
+                                 int(nthreads))
+    if rc != 0:
+        raise ValueError("oracle rejected the arguments")
+    return out
+
+
+def kv_bytes(ctx: int, n_full: int = 14, n_window: int = 35, window: int = 513,
+             nkv: int = 4, d: int = 128, elem_bytes: int = 2) -> float:
+    return _load().fo_kv_bytes(int(ctx), n_full, n_window, window, nkv, d, elem_bytes)

@@ -1,0 +1,352 @@
+"""Pins of the float64 oracle against things other than itself.
+
+Each test ties one oracle function to a library routine (torch's RMSNorm and
+SDPA, the rotate-half RoPE of transformers' Llama code, torch's bf16
+conversion), to a closed form, to an invariant, or to the numbers printed by
+the "Recursive Flint" model JSON.  A dropped term, a wrong sign, a swapped
+index or a transposed operand in the oracle fails at least one of them.
+"""
+import math
+import os
+
+import numpy as np
+import pytest
+import torch
+import torch.nn.functional as F
+
+import oracle
+from long_context_decode_flash_b200 import inputs as I
+
+GOLDEN = os.path.join(os.path.dirname(__file__), "golden")
+rng = np.random.default_rng(7)
+
+
+def bf16_bits(shape, seed, mean=0.0, std=1.0):
+    return I.bits(I.bf16_normal(shape, seed, mean, std))
+
+
+def f64(bits):
+    return torch.from_numpy(bits.astype(np.uint16).view(np.int16).copy()).view(
+        torch.bfloat16).to(torch.float64).numpy()
+
+
+# ---------------------------------------------------------------- bf16 -----
+
+def test_bf16_widening_matches_torch():
+    b = rng.integers(0, 1 << 16, size=20000, dtype=np.uint16)
+    b = b[(b & 0x7f80) != 0x7f80]  # drop inf / nan patterns
+    assert np.array_equal(oracle.bf16_to_f64(b), f64(b))
+
+
+def test_bf16_rounding_matches_torch_rne_on_float32_values():
+    x = np.concatenate([
+        rng.standard_normal(20000).astype(np.float32),
+        (rng.standard_normal(2000) * 1e-39).astype(np.float32),   # subnormals
+        (rng.standard_normal(2000) * 1e30).astype(np.float32),
+    ])
+    want = torch.from_numpy(x).to(torch.bfloat16).view(torch.int16).numpy().view(np.uint16)
+    assert np.array_equal(oracle.f64_to_bf16(x.astype(np.float64)), want)
+
+
+def test_bf16_rounding_ties_go_to_even():
+    # 1 + 2^-8 is halfway between 1 and 1 + 2^-7: the even neighbour is 1.0.
+    # 1 + 3*2^-8 is halfway between 1 + 2^-7 and 1 + 2^-6: the even one is 1 + 2^-6.
+    got = oracle.f64_to_bf16(np.array([1 + 2 ** -8, 1 + 3 * 2 ** -8, -(1 + 2 ** -8)]))
+    assert list(got) == [0x3f80, 0x3f82, 0xbf80]
+
+
+# ------------------------------------------------------------- RMSNorm -----
+
+def test_rmsnorm_matches_torch_rms_norm():
+    x = rng.standard_normal((36, 128)) * 3.0
+    w = 1.0 + 0.1 * rng.standard_normal(128)
+    want = F.rms_norm(torch.from_numpy(x), (128,), torch.from_numpy(w), eps=1e-6).numpy()
+    np.testing.assert_allclose(oracle.rmsnorm(x, w, 1e-6), want, rtol=1e-13, atol=1e-13)
+
+
+def test_rmsnorm_closed_form_unit_weight():
+    # with w = 1, mean(y^2) = ms / (ms + eps) for ms = mean(x^2)
+    x = rng.standard_normal((5, 128)) * 1e-3
+    eps = 1e-6
+    y = oracle.rmsnorm(x, None, eps)
+    ms = (x ** 2).mean(axis=1)
+    np.testing.assert_allclose((y ** 2).mean(axis=1), ms / (ms + eps), rtol=1e-12)
+
+
+# ---------------------------------------------------------------- RoPE -----
+
+def _hf_rope(x, pos):
+    from transformers import LlamaConfig
+    from transformers.models.llama.modeling_llama import (LlamaRotaryEmbedding,
+                                                          apply_rotary_pos_emb)
+    cfg = LlamaConfig(hidden_size=4096, num_attention_heads=32, head_dim=128,
+                      rope_parameters={"rope_type": "default", "rope_theta": 10000.0})
+    emb = LlamaRotaryEmbedding(cfg)
+    xt = torch.from_numpy(x)[None, :, None, :]            # [1, rows, seq=1, d]
+    cos, sin = emb(xt, torch.tensor([[pos]]))
+    y, _ = apply_rotary_pos_emb(xt, xt, cos, sin, unsqueeze_dim=1)
+    return y[0, :, 0, :].numpy()
+
+
+@pytest.mark.parametrize("pos", [0, 1, 7, 63])
+def test_rope_matches_transformers_rotate_half(pos):
+    # transformers forms its angles in float32: use positions where that is exact
+    # to ~1e-5 and compare at that tolerance.
+    x = rng.standard_normal((6, 128))
+    np.testing.assert_allclose(oracle.rope(x, pos), _hf_rope(x, pos), rtol=0, atol=3e-5)
+
+
+@pytest.mark.parametrize("i,freq", [(0, 1.0), (16, 0.1), (32, 0.01), (48, 0.001)])
+def test_rope_closed_form_at_long_context(i, freq):
+    # theta^(-2i/128) with theta = 10^4 is 10^(-i/16): exactly these decades.
+    pos = 99_999
+    e = np.zeros((1, 128))
+    e[0, i] = 1.0
+    y = oracle.rope(e, pos)
+    a = pos * freq
+    assert abs(y[0, i] - math.cos(a)) < 1e-9
+    assert abs(y[0, i + 64] - math.sin(a)) < 1e-9
+    e2 = np.zeros((1, 128))
+    e2[0, i + 64] = 1.0
+    y2 = oracle.rope(e2, pos)
+    assert abs(y2[0, i] + math.sin(a)) < 1e-9
+    assert abs(y2[0, i + 64] - math.cos(a)) < 1e-9
+
+
+def test_rope_invariants():
+    q = rng.standard_normal((3, 128))
+    k = rng.standard_normal((3, 128))
+    np.testing.assert_array_equal(oracle.rope(q, 0), q)
+    qr = oracle.rope(q, 123_456)
+    np.testing.assert_allclose(np.linalg.norm(qr, axis=1), np.linalg.norm(q, axis=1), rtol=1e-13)
+    # the score depends only on the distance m - n
+    a = (oracle.rope(q, 100_000) * oracle.rope(k, 99_500)).sum(axis=1)
+    b = (oracle.rope(q, 600) * oracle.rope(k, 100)).sum(axis=1)
+    np.testing.assert_allclose(a, b, rtol=0, atol=1e-9)
+
+
+# ----------------------------------------------------------- attention -----
+
+def _logical(cache, layout, L, capacity=0, table=None, bs=64):
+    """Gather positions 0..L-1 by plain numpy indexing."""
+    pos = np.arange(L)
+    if layout == oracle.CONTIGUOUS:
+        return cache[pos]
+    if layout == oracle.RING:
+        return cache[pos % capacity]
+    flat = cache.reshape((-1,) + cache.shape[2:])
+    return flat[np.asarray(table)[pos // bs] * bs + pos % bs]
+
+
+def sdpa_with_sink(q, K, V, sinks, lo, hi):
+    """Library route: torch SDPA in float64 over keys lo..hi-1 plus one extra
+    key with zero key and zero value whose logit is set to sink_h through an
+    additive mask; q [nq,d], K/V [n,nkv,d] float64."""
+    nq, d = q.shape
+    nkv = K.shape[1]
+    Kt = torch.from_numpy(K[lo:hi]).permute(1, 0, 2)        # [nkv, n, d]
+    Vt = torch.from_numpy(V[lo:hi]).permute(1, 0, 2)
+    Kt = torch.repeat_interleave(Kt, nq // nkv, dim=0)      # [nq, n, d]
+    Vt = torch.repeat_interleave(Vt, nq // nkv, dim=0)
+    zero = torch.zeros(nq, 1, d, dtype=torch.float64)
+    Kx, Vx = torch.cat([Kt, zero], 1), torch.cat([Vt, zero], 1)
+    mask = torch.zeros(nq, 1, hi - lo + 1, dtype=torch.float64)
+    mask[:, 0, -1] = torch.from_numpy(np.asarray(sinks, np.float64))
+    out = F.scaled_dot_product_attention(torch.from_numpy(q)[:, None, :], Kx, Vx,
+                                         attn_mask=mask, scale=1.0 / math.sqrt(d))
+    return out[:, 0, :].numpy()
+
+
+@pytest.mark.parametrize("L,window", [(1, 0), (5, 0), (700, 0), (700, 513), (513, 513),
+                                      (514, 513), (3, 513)])
+def test_attention_matches_torch_sdpa_contiguous(L, window):
+    q = rng.standard_normal((32, 128))
+    kc = bf16_bits((L, 4, 128), 11)
+    vc = bf16_bits((L, 4, 128), 12)
+    sinks = rng.standard_normal(32) * 2
+    got = oracle.attn_decode(q, kc, vc, L, sinks, window)
+    lo = max(0, L - window) if window else 0
+    want = sdpa_with_sink(q, f64(kc), f64(vc), sinks, lo, L)
+    np.testing.assert_allclose(got, want, rtol=1e-10, atol=1e-12)
+
+
+def test_attention_ring_matches_sdpa_over_logical_window():
+    L, cap = 2000, 513
+    ring = bf16_bits((cap, 4, 128), 21)
+    vring = bf16_bits((cap, 4, 128), 22)
+    q = rng.standard_normal((32, 128))
+    sinks = rng.standard_normal(32)
+    got = oracle.attn_decode(q, ring, vring, L, sinks, 513, layout=oracle.RING, capacity=cap)
+    K = _logical(ring, oracle.RING, L, cap)
+    V = _logical(vring, oracle.RING, L, cap)
+    want = sdpa_with_sink(q, f64(K), f64(V), sinks, L - 513, L)
+    np.testing.assert_allclose(got, want, rtol=1e-10, atol=1e-12)
+
+
+def test_attention_paged_permuted_equals_contiguous_exactly():
+    L, bs = 1000, 64
+    nb = -(-L // bs)
+    kc = bf16_bits((nb * bs, 4, 128), 31)
+    vc = bf16_bits((nb * bs, 4, 128), 32)
+    perm = np.random.default_rng(3).permutation(nb + 5)[:nb].astype(np.int32)
+    kp = np.zeros((nb + 5, bs, 4, 128), np.uint16)
+    vp = np.zeros_like(kp)
+    for j in range(nb):
+        kp[perm[j]] = kc[j * bs:(j + 1) * bs]
+        vp[perm[j]] = vc[j * bs:(j + 1) * bs]
+    q = rng.standard_normal((32, 128))
+    sinks = rng.standard_normal(32)
+    for window in (0, 513):
+        a = oracle.attn_decode(q, kc, vc, L, sinks, window)
+        b = oracle.attn_decode(q, kp, vp, L, sinks, window, layout=oracle.PAGED,
+                               block_table=perm, block_size=bs)
+        np.testing.assert_array_equal(a, b)
+
+
+def test_sink_to_minus_infinity_is_plain_softmax_attention():
+    L = 300
+    q = rng.standard_normal((32, 128))
+    kc = bf16_bits((L, 4, 128), 41)
+    vc = bf16_bits((L, 4, 128), 42)
+    got = oracle.attn_decode(q, kc, vc, L, np.full(32, -np.inf))
+    K = torch.from_numpy(f64(kc)).permute(1, 0, 2)
+    V = torch.from_numpy(f64(vc)).permute(1, 0, 2)
+    want = F.scaled_dot_product_attention(torch.from_numpy(q)[None, :, None, :],
+                                          K[None], V[None], enable_gqa=True)[0, :, 0].numpy()
+    np.testing.assert_allclose(got, want, rtol=1e-10, atol=1e-12)
+
+
+def test_window_at_least_context_equals_full():
+    q = rng.standard_normal((32, 128))
+    sinks = rng.standard_normal(32)
+    for L in (1, 200, 513):
+        kc = bf16_bits((L, 4, 128), 51)
+        vc = bf16_bits((L, 4, 128), 52)
+        np.testing.assert_array_equal(oracle.attn_decode(q, kc, vc, L, sinks, 513),
+                                      oracle.attn_decode(q, kc, vc, L, sinks, 0))
+
+
+def test_gqa_equals_explicitly_repeated_kv_heads():
+    L = 257
+    q = rng.standard_normal((32, 128))
+    sinks = rng.standard_normal(32)
+    kc = bf16_bits((L, 4, 128), 61)
+    vc = bf16_bits((L, 4, 128), 62)
+    a = oracle.attn_decode(q, kc, vc, L, sinks)
+    kr = np.ascontiguousarray(np.repeat(kc, 8, axis=1))   # [L, 32, 128]
+    vr = np.ascontiguousarray(np.repeat(vc, 8, axis=1))
+    b = oracle.attn_decode(q, kr, vr, L, sinks)
+    np.testing.assert_array_equal(a, b)
+
+
+def test_constant_v_gives_v_times_one_minus_sink_weight():
+    L = 400
+    q = rng.standard_normal((32, 128))
+    sinks = rng.standard_normal(32) + 3.0
+    kc = bf16_bits((L, 4, 128), 71)
+    c = np.float32(0.71875)                                  # exact in bf16
+    vc = np.full((L, 4, 128), np.frombuffer(np.float32(c).tobytes(), np.uint16)[1], np.uint16)
+    got = oracle.attn_decode(q, kc, vc, L, sinks)
+    K = f64(kc)
+    from scipy.special import logsumexp
+    for h in range(32):
+        s = K[:, h // 8, :] @ q[h] / math.sqrt(128)
+        w_sink = math.exp(sinks[h] - logsumexp(np.append(s, sinks[h])))
+        np.testing.assert_allclose(got[h], float(c) * (1.0 - w_sink), rtol=1e-12)
+
+
+# --------------------------------------------------- append and layers -----
+
+def test_append_placement_all_layouts():
+    k = bf16_bits((4, 128), 81)
+    v = bf16_bits((4, 128), 82)
+    # contiguous: row t
+    kc = bf16_bits((50, 4, 128), 83)
+    vc = bf16_bits((50, 4, 128), 84)
+    k0, v0 = kc.copy(), vc.copy()
+    oracle.kv_append(kc, vc, oracle.CONTIGUOUS, 37, k, v)
+    assert np.array_equal(kc[37], k) and np.array_equal(vc[37], v)
+    mask = np.ones(50, bool)
+    mask[37] = False
+    assert np.array_equal(kc[mask], k0[mask]) and np.array_equal(vc[mask], v0[mask])
+    # ring: row t mod 513
+    kr = bf16_bits((513, 4, 128), 85)
+    vr = bf16_bits((513, 4, 128), 86)
+    kr0 = kr.copy()
+    oracle.kv_append(kr, vr, oracle.RING, 99_999, k, v, capacity=513)
+    assert np.array_equal(kr[99_999 % 513], k) and np.array_equal(vr[99_999 % 513], v)
+    mask = np.ones(513, bool)
+    mask[99_999 % 513] = False
+    assert np.array_equal(kr[mask], kr0[mask])
+    # paged: block_table[t // 64] * 64 + t % 64
+    table = np.array([5, 2, 7, 0], np.int32)
+    kp = bf16_bits((8, 64, 4, 128), 87)
+    vp = bf16_bits((8, 64, 4, 128), 88)
+    kp0 = kp.copy()
+    oracle.kv_append(kp, vp, oracle.PAGED, 150, k, v, block_table=table)
+    assert np.array_equal(kp[7, 150 - 128], k) and np.array_equal(vp[7, 22], v)
+    kp0[7, 22] = k
+    assert np.array_equal(kp, kp0)
+
+
+def test_qk_norm_rope_chain_matches_library_pipeline():
+    # torch rms_norm then transformers' rotate-half RoPE, at a position where
+    # the library's float32 angles are accurate
+    pos = 9
+    q_raw = bf16_bits((32, 128), 91)
+    k_raw = bf16_bits((4, 128), 92)
+    w_q = bf16_bits((128,), 93, 1.0, 0.1)
+    w_k = bf16_bits((128,), 94, 1.0, 0.1)
+    q, k, kb = oracle.qk_norm_rope(q_raw, k_raw, w_q, w_k, pos)
+    qn = F.rms_norm(torch.from_numpy(f64(q_raw)), (128,), torch.from_numpy(f64(w_q)), 1e-6)
+    kn = F.rms_norm(torch.from_numpy(f64(k_raw)), (128,), torch.from_numpy(f64(w_k)), 1e-6)
+    np.testing.assert_allclose(q, _hf_rope(qn.numpy(), pos), atol=3e-5)
+    np.testing.assert_allclose(k, _hf_rope(kn.numpy(), pos), atol=3e-5)
+    want_kb = torch.from_numpy(k.astype(np.float32)).to(torch.bfloat16)
+    # bf16 of the f64 value: compare by value within half a bf16 ulp
+    np.testing.assert_allclose(f64(kb), k, rtol=2 ** -8)
+    assert np.mean(f64(kb) == want_kb.to(torch.float64).numpy()) > 0.99
+    # no RoPE, no norm: identity on the bf16 inputs
+    q2, k2, _ = oracle.qk_norm_rope(q_raw, k_raw, None, None, pos, apply_rope=False)
+    np.testing.assert_array_equal(q2, f64(q_raw))
+    np.testing.assert_array_equal(k2, f64(k_raw))
+
+
+def test_decode_layer_is_append_then_attend_over_library_reference():
+    L = 600
+    lay = I.make_layer(9, 0, L, 513, True, ring=True)
+    kc, vc = I.bits(lay.k_cache).copy(), I.bits(lay.v_cache).copy()
+    out = oracle.decode_layer(I.bits(lay.q_raw), I.bits(lay.k_raw), I.bits(lay.v_raw),
+                              I.bits(lay.w_q), I.bits(lay.w_k), lay.sinks.numpy(),
+                              kc, vc, L, 513, True, layout=oracle.RING, capacity=513)
+    # the appended row is the oracle's own k rounded to bf16, and v_raw as is
+    q, _, kb = oracle.qk_norm_rope(I.bits(lay.q_raw), I.bits(lay.k_raw), I.bits(lay.w_q),
+                                   I.bits(lay.w_k), L - 1)
+    slot = (L - 1) % 513
+    assert np.array_equal(kc[slot], kb) and np.array_equal(vc[slot], I.bits(lay.v_raw))
+    K = _logical(kc, oracle.RING, L, 513)
+    V = _logical(vc, oracle.RING, L, 513)
+    want = sdpa_with_sink(q, f64(K), f64(V), lay.sinks.numpy().astype(np.float64), L - 513, L)
+    np.testing.assert_allclose(out, want, rtol=1e-10, atol=1e-12)
+
+
+# ---------------------------------------------------------------- sizes ----
+
+def _golden_kv():
+    rows = []
+    with open(os.path.join(GOLDEN, "kv_cache_gib_per_request.txt")) as f:
+        for line in f:
+            if line.strip() and not line.startswith("#"):
+                c, b, e = line.split()
+                rows.append((int(c), float(b), float(e)))
+    return rows
+
+
+def test_kv_bytes_reproduce_the_model_json_table():
+    rows = _golden_kv()
+    assert len(rows) == 4
+    for ctx, gib_bf16, gib_fp8 in rows:
+        assert round(oracle.kv_bytes(ctx, elem_bytes=2) / 2 ** 30, 3) == gib_bf16
+        assert round(oracle.kv_bytes(ctx, elem_bytes=1) / 2 ** 30, 3) == gib_fp8
+    # "28 KiB per token" over the full layers (Model architecture)
+    assert oracle.kv_bytes(1000, n_window=0) - oracle.kv_bytes(999, n_window=0) == 28 * 1024
