@@ -1,0 +1,374 @@
+"""Benchmark: one decode step of Flint's 49-layer attention stack at context
+100,000, batch 1 (35 sliding-window RoPE layers + 14 full NoPE layers, each
+with its own bf16 KV cache), on B200s.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl flint|reference]
+                    [--workload stack|full100k|swa100k|paged32]
+
+Prints one JSON line (rank 0).  A step is one call of flint_attn_stack: for
+every layer the fused Q/K RMSNorm (+RoPE), KV append at position 99,999 and
+split-KV decode with sinks, in one kernel launch.  `value` is device time per
+decoded token (CUDA events on the launching stream, L2 flushed by a 256 MiB
+write before every step, max over ranks / tokens of all ranks).  Under
+torchrun each rank decodes its own independent token (weak scaling; there is
+no data-path collective).  `--impl reference` times the float64 CPU oracle on
+the host cores instead (bounded sample, scaled to the same unit).
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "49-layer decode-attention µs/token @100K ctx bs=1; achieved HBM GB/s vs peak"
+CONTEXT = 100_000
+NOMINAL_HBM_GBS = 8000.0
+FALLBACK_HBM_GBS = 6650.0
+
+
+def parse():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=50)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", default="flint", choices=["flint", "reference"])
+    ap.add_argument("--workload", default="stack", choices=["stack", "full100k", "swa100k", "paged32"])
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-e2e", action="store_true")
+    return ap.parse_args()
+
+
+def measured_peak():
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+            return float(json.load(f)["hbm_gbs"]), "measured"
+    except Exception:
+        return FALLBACK_HBM_GBS, "fallback"
+
+
+# ------------------------------------------------------------ CPU oracle ---
+
+def oracle_sample(layers_full, layers_window, nthreads):
+    """Time the oracle on some layers of the stack; returns (us per token for
+    the 14+35 stack, seconds spent, description)."""
+    import numpy as np
+    import oracle
+    from long_context_decode_flash_b200 import inputs as I
+
+    def one(lay):
+        kc, vc = I.bits(lay.k_cache).copy(), I.bits(lay.v_cache).copy()
+        t0 = time.perf_counter()
+        oracle.decode_layer(I.bits(lay.q_raw), I.bits(lay.k_raw), I.bits(lay.v_raw),
+                            I.bits(lay.w_q), I.bits(lay.w_k), lay.sinks.numpy().astype(np.float64),
+                            kc, vc, lay.L, lay.window, lay.rope, layout=lay.layout,
+                            capacity=lay.capacity, nthreads=nthreads)
+        return time.perf_counter() - t0
+
+    tf = [one(l) for l in layers_full]
+    tw = [one(l) for l in layers_window]
+    per_full = sum(tf) / len(tf)
+    per_win = sum(tw) / len(tw)
+    us = (14 * per_full + 35 * per_win) * 1e6
+    desc = (f"{len(layers_full)} full layer(s) + {len(layers_window)} window layer(s) of the "
+            f"stack at context {CONTEXT}, all 32 heads, scaled to 14 + 35 layers")
+    return us, sum(tf) + sum(tw), desc
+
+
+def run_reference(args, rank):
+    """The float64 oracle on the host cores, same metric and unit."""
+    if rank != 0:
+        return
+    import oracle
+    from long_context_decode_flash_b200 import inputs as I
+
+    oracle.build()
+    nthreads = os.cpu_count() or 1
+    kinds = I.layer_kinds()
+    full_i = kinds.index(True)
+    layers_full = [I.make_layer(I.W_STACK_100K, full_i, CONTEXT, 0, False, ring=False)]
+    layers_win = [I.make_layer(I.W_STACK_100K, 0, CONTEXT, 513, True, ring=True)]
+    for _ in range(args.warmup):
+        oracle_sample(layers_full, layers_win[:1], nthreads)
+    vals = [oracle_sample(layers_full, layers_win, nthreads)[0] for _ in range(args.steps)]
+    us = statistics.mean(vals)
+    sample = (f"per step: 1 full layer + 1 window layer of the stack at context {CONTEXT}, "
+              f"all heads, scaled to 14 + 35 layers")
+    line = {
+        "impl": "reference", "metric": METRIC, "value": us, "unit": "us/token",
+        "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": us / 1000.0, "higher_is_better": False, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": workload_config("stack"),
+        "cpu_baseline": {"value": us, "unit": "us/token", "cores": nthreads, "kind": "oracle",
+                         "sample": sample},
+        "e2e": {"value": us, "unit": "us/token", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+# ------------------------------------------------------------- GPU side ----
+
+def workload_config(name):
+    base = {"l2": "flushed before every step (256 MiB write)", "batch": 1}
+    if name == "stack":
+        return dict(base, workload="49-layer decode-attention stack for one token: 35 sliding-window "
+                    "(513, RoPE) + 14 full-context NoPE layers, GQA 32q/4kv x 128, sinks",
+                    context=CONTEXT, layers=49, kv_layout="ring(513) + contiguous")
+    if name == "full100k":
+        return dict(base, workload="one full-context NoPE decode layer", context=CONTEXT, layers=1,
+                    kv_layout="contiguous")
+    if name == "swa100k":
+        return dict(base, workload="one sliding-window RoPE layer with norm+RoPE+append",
+                    context=CONTEXT, layers=1, kv_layout="ring(513)")
+    return dict(base, workload="32 paged requests, log-uniform lengths in [4096, 131072], "
+                "full-context layer", batch=32, kv_layout="paged(64)")
+
+
+class ClockSampler:
+    """nvidia-smi samples during the timed region."""
+
+    def __init__(self, index):
+        self.index = index
+        self.rows = []
+        self.proc = None
+
+    def __enter__(self):
+        q = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.hw_slowdown,"
+             "clocks_event_reasons.hw_thermal_slowdown,clocks_event_reasons.sw_thermal_slowdown,"
+             "clocks_event_reasons.sw_power_cap")
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.index), f"--query-gpu={q}", "--format=csv,noheader,nounits",
+                 "-lms", "100"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self.thread = threading.Thread(target=self._read, daemon=True)
+            self.thread.start()
+        except Exception:
+            self.proc = None
+        return self
+
+    def _read(self):
+        for line in self.proc.stdout:
+            parts = [p.strip() for p in line.split(",")]
+            if len(parts) == 7:
+                self.rows.append(parts)
+
+    def __exit__(self, *exc):
+        if self.proc:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except Exception:
+                self.proc.kill()
+
+    def summary(self):
+        if not self.rows:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unsampled"]}
+        sm = [float(r[0]) for r in self.rows if r[0].replace(".", "").isdigit()]
+        mx = [float(r[1]) for r in self.rows if r[1].replace(".", "").isdigit()]
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({n for r in self.rows for n, v in zip(names, r[3:]) if v == "Active"})
+        return {"sm_mhz": statistics.median(sm) if sm else None,
+                "sm_max_mhz": max(mx) if mx else None, "reasons": reasons, "samples": len(self.rows)}
+
+
+def build_stack_device(torch, flint, I, layers):
+    """Device copies; the per-token inputs (q_raw, k_raw, v_raw of all layers)
+    live in one packed buffer so a step's inputs arrive with one copy."""
+    n = len(layers)
+    per = (32 + 4 + 4) * 128
+    packed = torch.empty((n, per), dtype=torch.bfloat16, device="cuda")
+
+    class Dev:
+        pass
+
+    dls = []
+    for i, lay in enumerate(layers):
+        d = Dev()
+        row = packed[i]
+        d.q_raw = row[:32 * 128].view(32, 128)
+        d.k_raw = row[32 * 128:36 * 128].view(4, 128)
+        d.v_raw = row[36 * 128:].view(4, 128)
+        d.q_raw.copy_(lay.q_raw)
+        d.k_raw.copy_(lay.k_raw)
+        d.v_raw.copy_(lay.v_raw)
+        d.w_q, d.w_k, d.sinks = lay.w_q.cuda(), lay.w_k.cuda(), lay.sinks.cuda()
+        d.k_cache, d.v_cache = lay.k_cache.cuda(), lay.v_cache.cuda()
+        d.window, d.rope = lay.window, lay.rope
+        d.cache = flint.kv_cache(d.k_cache, d.v_cache, lay.layout, capacity=lay.capacity)
+        dls.append(d)
+    host_in = torch.cat([torch.cat([l.q_raw.reshape(-1), l.k_raw.reshape(-1), l.v_raw.reshape(-1)])
+                         for l in layers]).reshape(n, per).pin_memory()
+    return dls, packed, host_in
+
+
+def main():
+    args = parse()
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if args.impl == "reference":
+        run_reference(args, rank)
+        return
+
+    import torch
+    import numpy as np
+    from long_context_decode_flash_b200 import flint
+    from long_context_decode_flash_b200 import inputs as I
+
+    # Host inputs first; the CPU baseline runs before any CUDA call.
+    if args.workload == "stack":
+        layers = I.make_stack(CONTEXT)
+        algo_bytes = flint.flint_kv_bytes(CONTEXT)
+    elif args.workload == "full100k":
+        layers = [I.make_layer(I.W_FULL_100K, 0, CONTEXT, 0, False, ring=False)]
+        algo_bytes = CONTEXT * 2048
+    elif args.workload == "swa100k":
+        layers = [I.make_layer(I.W_SWA_100K, 0, CONTEXT, 513, True, ring=True)]
+        algo_bytes = 513 * 2048
+    else:
+        layers = None
+        pb = I.make_paged_batch()
+        algo_bytes = sum(pb.seq_lens) * 2048
+
+    cpu_baseline = None
+    if rank == 0 and world == 1 and args.workload == "stack" and not args.no_cpu_baseline:
+        import oracle
+        oracle.build()
+        kinds = I.layer_kinds()
+        full = [layers[kinds.index(True)]]
+        win = [layers[0], layers[1]]
+        nthreads = os.cpu_count() or 1
+        us, spent, desc = oracle_sample(full, win, nthreads)
+        cpu_baseline = {"value": us, "unit": "us/token", "cores": nthreads, "kind": "oracle",
+                        "sample": desc + f" ({spent:.1f} s of CPU wall time)"}
+
+    if world > 1:
+        torch.distributed.init_process_group("nccl", timeout=__import__("datetime").timedelta(seconds=120))
+    torch.cuda.set_device(local)
+    dev_index = torch.cuda.current_device()
+    stream = torch.cuda.current_stream()
+
+    flush = torch.empty(256 * 1024 * 1024 // 4, dtype=torch.float32, device="cuda")
+    err = torch.zeros(1, dtype=torch.int32, device="cuda")
+
+    if layers is not None:
+        dls, packed, host_in = build_stack_device(torch, flint, I, layers)
+        pos = CONTEXT - 1
+        out = torch.empty((len(dls), 32, 128), dtype=torch.float32, device="cuda")
+        ws = flint.workspace(len(dls))
+        arr = flint.stack_layers(dls)
+
+        def step():
+            flint.flint_attn_stack(arr, pos, out, ws, dev_err=err)
+        h2d = host_in.numel() * host_in.element_size()
+    else:
+        q, k, v = pb.q.cuda(), pb.k_pool.cuda(), pb.v_pool.cuda()
+        table, sinks = pb.block_table.cuda(), pb.sinks.cuda()
+        cache = flint.kv_cache(k, v, flint.PAGED, block_table=table, num_blocks=pb.k_pool.shape[0])
+        out = torch.empty((len(pb.seq_lens), 32, 128), dtype=torch.float32, device="cuda")
+        ws = flint.workspace(len(pb.seq_lens))
+        host_in = pb.q.pin_memory()
+        packed = q
+
+        def step():
+            flint.flint_attn_decode(q, cache, pb.seq_lens, sinks, 0, out, ws, dev_err=err)
+        h2d = host_in.numel() * host_in.element_size()
+    host_out = torch.empty(out.shape, dtype=torch.float32).pin_memory()
+    d2h = host_out.numel() * 4
+
+    for _ in range(max(args.warmup, 3)):
+        flush.fill_(1.0)
+        step()
+    torch.cuda.synchronize()
+    if int(err.item()) != 0:
+        raise SystemExit(f"device error {int(err.item())} during warm-up")
+
+    starts = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    ends = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    if world > 1:
+        torch.distributed.barrier()
+    torch.cuda.synchronize()
+    with ClockSampler(dev_index) as clocks:
+        t_wall = time.perf_counter()
+        for i in range(args.steps):
+            flush.fill_(float(i))
+            starts[i].record(stream)
+            step()
+            ends[i].record(stream)
+        torch.cuda.synchronize()
+        t_wall = time.perf_counter() - t_wall
+    if world > 1:
+        torch.distributed.barrier()
+    per_step_ms = [s.elapsed_time(e) for s, e in zip(starts, ends)]
+    ms = statistics.mean(per_step_ms)
+    if int(err.item()) != 0:
+        raise SystemExit(f"device error {int(err.item())} in the timed region")
+
+    # end to end through the public API: pinned host inputs in, result out
+    e2e = None
+    if not args.no_e2e:
+        e_s = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+        e_e = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+        if world > 1:
+            torch.distributed.barrier()
+        torch.cuda.synchronize()
+        for i in range(args.steps):
+            flush.fill_(float(i))
+            e_s[i].record(stream)
+            packed.copy_(host_in, non_blocking=True)
+            step()
+            host_out.copy_(out, non_blocking=True)
+            e_e[i].record(stream)
+        torch.cuda.synchronize()
+        e2e_ms = statistics.mean(s.elapsed_time(e) for s, e in zip(e_s, e_e))
+        if world > 1:
+            t = torch.tensor([e2e_ms], device="cuda")
+            torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+            e2e_ms = float(t.item())
+        e2e = {"value": e2e_ms * 1000.0 / world, "unit": "us/token" if layers is not None else "us/step",
+               "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h)}
+
+    if world > 1:
+        t = torch.tensor([ms], device="cuda")
+        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+        ms = float(t.item())
+
+    peak, peak_kind = measured_peak()
+    achieved = algo_bytes / (ms * 1e-3) / 1e9
+    line = {
+        "metric": METRIC if args.workload == "stack" else f"{args.workload} decode-attention us/step",
+        "value": ms * 1000.0 / world,
+        "unit": "us/token" if args.workload == "stack" else "us/step",
+        "n_gpus": world, "steps": args.steps, "warmup": max(args.warmup, 3),
+        "ms_per_step": ms, "higher_is_better": False, "scaling": "weak", "vs_baseline": None,
+        "dtype": "bf16", "data": "synthetic (seeded bf16 N(0,1) q/k/v/KV, N(0,1) sinks, 1+N(0,0.1) norm weights)",
+        "config": dict(workload_config(args.workload), parallelism=f"replicas x{world}"),
+        "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
+                     "frac": achieved / peak, "peak_kind": peak_kind,
+                     "frac_of_nominal_8000": achieved / NOMINAL_HBM_GBS,
+                     "algorithmic_bytes": int(algo_bytes), "kernel": "flint decode_kernel",
+                     "traffic": None},
+        "cpu_baseline": cpu_baseline,
+        "e2e": e2e,
+        "gpu_launches": args.steps,
+        "clocks": clocks.summary(),
+        "per_step_us": {"min": min(per_step_ms) * 1000.0, "median": statistics.median(per_step_ms) * 1000.0,
+                        "max": max(per_step_ms) * 1000.0},
+        "timed_region_wall_s": t_wall,
+    }
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        torch.distributed.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,211 @@
+/*
+ * flint.h -- C ABI of libflint.so: one decode step of Flint attention on a
+ * B200 (sm_100a), batch 1 or a batch of paged requests.
+ *
+ * Model facts the operations follow (page title, section):
+ *   - "Day-0 Support for Flint on vLLM" (hnkhoi.com/news/1467), "Model
+ *     architecture": 49 layers; 35 attend a 513-token sliding window with
+ *     RoPE, 14 attend the full context with no positional encoding; only the
+ *     14 keep KV for the whole sequence; learned attention sinks; GQA with 32
+ *     query and 4 KV heads; per-head Q/K RMSNorm.
+ *   - "Recursive Flint" model JSON (studiotvai.com/api/models/flint.json):
+ *     `architecture` "GQA 4 KV x 128" (head_dim 128), `maxContext` 262144,
+ *     `kvCacheGiBPerRequest` (checked by flint_kv_bytes).
+ *   - "Day-0 Support for Flint on vLLM" (newruntime.com), "What happened":
+ *     BF16 KV cache; fused normalization, rotary-position and cache
+ *     operations; a low-latency decode path for small batches; "Why it
+ *     matters": one Blackwell GPU, tensor parallelism 1.
+ * The pages print no formulas.  Definitions adopted here:
+ *   score_j = q_h . K_j / sqrt(128); out_h = sum_j e^(score_j - M) V_j /
+ *   (sum_j e^(score_j - M) + e^(sink_h - M)), M = max(max_j score_j, sink_h):
+ *   the sink logit joins the softmax but carries no value.  Query head h reads
+ *   KV head h / 8.  A window layer at position t attends max(0, t-512) .. t.
+ *   RMSNorm: y = x * w / sqrt(mean(x^2) + eps).  RoPE: rotate-half over all
+ *   128 dims, pairs (i, i+64), angle t * theta^(-2i/128), absolute position.
+ *
+ * Conventions for every call:
+ *   - Device pointers are CUDA device memory owned by the caller; host
+ *     pointers are read during the call only.  The library allocates no
+ *     memory and never synchronises; work is queued on `stream` (a
+ *     cudaStream_t, NULL = legacy default stream) and runs asynchronously.
+ *   - bf16 tensors are passed as uint16_t bit patterns.  All shapes are
+ *     row-major and densely packed unless a stride says otherwise; every
+ *     device pointer must be 16-byte aligned.
+ *   - Errors found on the host (bad pointer, shape, size, index) return
+ *     synchronously with nothing queued: FLINT_ERR_INVALID_ARG or
+ *     FLINT_ERR_UNSUPPORTED.  A failed launch returns FLINT_ERR_CUDA.  The
+ *     detail of the last error on the calling thread is in flint_last_error().
+ *   - Problems found on the device (a paged block id out of range, a pipeline
+ *     wait that ran past its time limit) are written to *dev_err as a
+ *     flint_status value if dev_err is not NULL (first error wins; the caller
+ *     zeroes it).  No kernel traps or spins without a limit.
+ */
+#ifndef FLINT_H
+#define FLINT_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#define FLINT_NUM_Q_HEADS 32
+#define FLINT_NUM_KV_HEADS 4
+#define FLINT_HEAD_DIM 128
+#define FLINT_WINDOW 513          /* sliding-window length (tokens) */
+#define FLINT_BLOCK_SIZE 64       /* paged-cache block length (tokens) */
+#define FLINT_MAX_CONTEXT 262144  /* "maxContext" of the model JSON */
+#define FLINT_MAX_BATCH 64        /* requests per flint_attn_decode launch */
+#define FLINT_MAX_LAYERS 49       /* layers per flint_attn_stack call */
+
+typedef enum {
+    FLINT_OK = 0,
+    FLINT_ERR_INVALID_ARG = 1,
+    FLINT_ERR_UNSUPPORTED = 2,
+    FLINT_ERR_WORKSPACE = 3,
+    FLINT_ERR_CUDA = 4,
+    FLINT_ERR_TIMEOUT = 5
+} flint_status;
+
+typedef enum {
+    FLINT_KV_CONTIGUOUS = 0, /* K/V [B][capacity][4][128]; position t in slot t     */
+    FLINT_KV_RING = 1,       /* K/V [B][513][4][128]; position t in slot t mod 513   */
+    FLINT_KV_PAGED = 2       /* K/V [num_blocks][64][4][128]; position t in block
+                                block_table[b][t / 64], row t mod 64                 */
+} flint_kv_layout;
+
+/* One layer's KV cache for a batch of requests.  k and v are bf16 device
+ * buffers of identical geometry. */
+typedef struct {
+    void* k;
+    void* v;
+    int32_t layout;              /* flint_kv_layout */
+    int32_t capacity;            /* CONTIGUOUS: slots per request; RING: 513; PAGED: 0 */
+    int64_t req_stride;          /* CONTIGUOUS/RING: elements between requests
+                                    (0 = capacity*4*128); multiple of 8 */
+    const int32_t* block_table;  /* PAGED: device int32 [B][max_blocks_per_req] */
+    int32_t max_blocks_per_req;  /* PAGED */
+    int32_t block_size;          /* PAGED: must be 64 */
+    int32_t num_blocks;          /* PAGED: blocks in the pool */
+} flint_kv_cache;
+
+/* One layer of one decoded token, for flint_attn_stack (batch 1). */
+typedef struct {
+    const uint16_t* q_raw;   /* bf16 [32][128], before norm/RoPE */
+    const uint16_t* k_raw;   /* bf16 [4][128] */
+    const uint16_t* v_raw;   /* bf16 [4][128], appended as is */
+    const uint16_t* w_q;     /* bf16 [128] RMSNorm weight for q (shared by heads) */
+    const uint16_t* w_k;     /* bf16 [128] RMSNorm weight for k */
+    const float* sinks;      /* fp32 [32] sink logits */
+    flint_kv_cache cache;    /* this layer's cache (request 0 only) */
+    int32_t window;          /* 0 = full context, 513 = sliding window */
+    int32_t rope;            /* 1 = apply RoPE (window layers), 0 = NoPE */
+} flint_layer;
+
+/* Short English name of a status code (static storage). */
+const char* flint_status_string(flint_status s);
+
+/* Detail of the last error returned on the calling thread ("" if none). */
+const char* flint_last_error(void);
+
+/* KV-cache bytes per request of a model with n_full full-context layers and
+ * n_window window layers at context ctx_len: every token of a full layer, and
+ * min(ctx_len, window) tokens of a window layer, each 2*4*128 values of
+ * elem_bytes bytes ("Recursive Flint" model JSON, kvCacheGiBPerRequest).
+ * Pure host arithmetic; returns 0 for negative arguments. */
+uint64_t flint_kv_bytes(int64_t ctx_len, int32_t n_full, int32_t n_window,
+                        int32_t window, int32_t elem_bytes);
+
+/* Per-head Q/K RMSNorm, optional RoPE, optional KV append for B requests
+ * ("Model architecture": per-head Q/K RMSNorm, RoPE on window layers;
+ * "What happened": fused normalization, rotary-position and cache ops).
+ *   q_raw  bf16 [B][32][128], k_raw bf16 [B][4][128]          (device, in)
+ *   v_raw  bf16 [B][4][128] (device, in); only read when cache != NULL
+ *   w_q, w_k  bf16 [128] (device, in); the norm weight, shared by all heads
+ *   pos    host int32 [B]: absolute position of each request's new token
+ *   eps    RMSNorm epsilon (1e-6); theta  RoPE base (10000)
+ *   apply_rope  0 or 1
+ *   q_out  fp32 [B][32][128] (device, out) or NULL
+ *   k_out  bf16 [B][4][128]  (device, out) or NULL: k after norm/RoPE,
+ *          rounded to nearest even
+ *   cache  NULL, or the cache to append k (as in k_out) and v_raw to, at
+ *          position pos[b] (slot per the layout; PAGED reads block_table on
+ *          the device, an out-of-range block id skips the write and sets
+ *          *dev_err = FLINT_ERR_INVALID_ARG)
+ * B in [1, FLINT_MAX_BATCH]. */
+flint_status flint_qk_norm_rope(const uint16_t* q_raw, const uint16_t* k_raw,
+                                const uint16_t* v_raw, const uint16_t* w_q,
+                                const uint16_t* w_k, const int32_t* pos, int32_t B,
+                                float eps, double theta, int32_t apply_rope,
+                                float* q_out, uint16_t* k_out,
+                                const flint_kv_cache* cache, int32_t* dev_err,
+                                void* stream);
+
+/* Bit-exact append of already final k, v (bf16 [B][4][128], device) at host
+ * positions pos[B] of `cache` ("Model architecture": only full layers keep
+ * the whole sequence, window layers keep a 513-slot ring).  Untouched slots
+ * are not written.  Same device-side error rule as flint_qk_norm_rope. */
+flint_status flint_kv_append(const uint16_t* k, const uint16_t* v, const int32_t* pos,
+                             int32_t B, const flint_kv_cache* cache, int32_t* dev_err,
+                             void* stream);
+
+/* Bytes of device workspace that flint_attn_decode / flint_attn_stack need
+ * for n_problems (requests, or layers) on a grid of num_ctas CTAs (0 = the
+ * current device's default).  The workspace holds split partials and
+ * per-head arrival counters; it must be zero-filled before its first use and
+ * is left zeroed by every call that completes without a device error.
+ * Returns 0 for invalid arguments. */
+size_t flint_attn_workspace_bytes(int32_t n_problems, int32_t num_ctas);
+
+/* Split-KV flash-decode over a batch of B requests of one layer: q already
+ * normed (and roped).  The new token is already in the cache; request b
+ * attends positions [max(0, L_b - window), L_b) (window 513) or [0, L_b)
+ * (window 0), L_b = seq_lens[b].
+ *   q         bf16 or fp32 [B][32][128] (device); q_is_fp32 selects
+ *   cache     any layout; RING requires window == 513 and capacity 513
+ *   seq_lens  HOST int32 [B], 1 <= L_b <= FLINT_MAX_CONTEXT (and <= capacity
+ *             for CONTIGUOUS, <= max_blocks_per_req*64 for PAGED); the split
+ *             plan is built from them on the host
+ *   sinks     fp32 [32] (device), shared by the batch; -INFINITY drops a sink
+ *   out       fp32 [B][32][128] (device)
+ *   workspace device, >= flint_attn_workspace_bytes(B, num_ctas) bytes
+ *   num_ctas  0 = one CTA per SM (the tuned default)
+ * B in [1, FLINT_MAX_BATCH].  Result is deterministic run to run. */
+flint_status flint_attn_decode(const void* q, int32_t q_is_fp32,
+                               const flint_kv_cache* cache, const int32_t* seq_lens,
+                               int32_t B, const float* sinks, int32_t window,
+                               float* out, void* workspace, size_t ws_bytes,
+                               int32_t num_ctas, int32_t* dev_err, void* stream);
+
+/* One decoded token through n_layers attention layers in ONE launch: for each
+ * layer, per-head Q/K RMSNorm (+RoPE if layer.rope), append of k and v_raw at
+ * position pos, and decode attention over the layer's window, all scheduled
+ * together across the GPU (the layers are independent problems here).
+ *   layers    HOST array [n_layers], 1 <= n_layers <= FLINT_MAX_LAYERS;
+ *             window layers usually RING caches, full layers CONTIGUOUS
+ *   pos       position of the new token (context pos + 1 after the append)
+ *   out       fp32 [n_layers][32][128] (device)
+ *   workspace >= flint_attn_workspace_bytes(n_layers, num_ctas) bytes */
+flint_status flint_attn_stack(const flint_layer* layers, int32_t n_layers, int32_t pos,
+                              float eps, double theta, float* out, void* workspace,
+                              size_t ws_bytes, int32_t num_ctas, int32_t* dev_err,
+                              void* stream);
+
+/* The split planner behind both attention calls (pure host code, exposed for
+ * tests).  Work is n_segs segments (one per problem and KV head) of
+ * seg_tiles[s] 64-token tiles; it is cut into items (segment, tile range)
+ * laid over num_ctas CTAs so that tiles + item_cost per item are level.
+ * Outputs: item_seg/item_t0/item_t1 [max_items], cta_begin [num_ctas+1]
+ * (items of CTA c are cta_begin[c] .. cta_begin[c+1]-1; the items of one
+ * segment are consecutive).  Returns the item count, or -1 on bad
+ * arguments / too many items. */
+int32_t flint_plan_items(const int32_t* seg_tiles, int32_t n_segs, int32_t num_ctas,
+                         int32_t item_cost, int32_t* item_seg, int32_t* item_t0,
+                         int32_t* item_t1, int32_t* cta_begin, int32_t max_items);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* FLINT_H */

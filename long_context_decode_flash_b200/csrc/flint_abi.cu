@@ -1,0 +1,495 @@
+// flint_abi.cu -- the extern "C" entry points of libflint.so: argument
+// validation, split planning, TMA tensor maps and launches.  No entry point
+// allocates, frees or synchronises; everything is queued on the caller's
+// stream.
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <stdarg.h>
+#include <stdio.h>
+#include <string.h>
+
+#include <algorithm>
+#include <mutex>
+#include <string>
+
+#include "flint_internal.h"
+
+using namespace flint;
+
+namespace {
+
+thread_local std::string g_last_error;
+
+flint_status fail(flint_status s, const char* fmt, ...) {
+  char buf[512];
+  va_list ap;
+  va_start(ap, fmt);
+  vsnprintf(buf, sizeof buf, fmt, ap);
+  va_end(ap);
+  g_last_error = buf;
+  return s;
+}
+
+flint_status ok() {
+  g_last_error.clear();
+  return FLINT_OK;
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+constexpr int kItemCost = 2;  // per-item overhead in tile units (planner cost model)
+
+// ---- device properties (cached per device) --------------------------------
+
+int device_num_sms(int* out) {
+  static std::mutex mu;
+  static int sms[64] = {0};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return -1;
+  std::lock_guard<std::mutex> lock(mu);
+  if (sms[dev] == 0) {
+    int v = 0;
+    if (cudaDeviceGetAttribute(&v, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || v <= 0)
+      return -1;
+    sms[dev] = v;
+  }
+  *out = sms[dev];
+  return 0;
+}
+
+// ---- TMA tensor maps --------------------------------------------------------
+
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                  const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                  const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                  CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(p);
+  });
+  return fn;
+}
+
+// A K or V cache seen as a 4-D bf16 tensor (dims innermost first):
+//   CONTIGUOUS/RING: [128 dims][4 heads][capacity tokens][B requests]
+//   PAGED:           [128 dims][4 heads][64 tokens][num_blocks]
+// read in boxes of 64 dims x 1 head x 64 tokens x 1 with the 128-byte swizzle.
+flint_status encode_cache_map(CUtensorMap* map, void* base, const flint_kv_cache& c, int B) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) return fail(FLINT_ERR_CUDA, "cuTensorMapEncodeTiled is not available from the driver");
+  cuuint64_t dims[4], strides[3];
+  dims[0] = kDim;
+  dims[1] = kKvHeads;
+  strides[0] = kDim * 2;
+  strides[1] = kKvHeads * kDim * 2;
+  if (c.layout == FLINT_KV_PAGED) {
+    dims[2] = kBlock;
+    dims[3] = static_cast<cuuint64_t>(c.num_blocks);
+    strides[2] = static_cast<cuuint64_t>(kBlock) * kKvHeads * kDim * 2;
+  } else {
+    const int64_t rs = c.req_stride ? c.req_stride : static_cast<int64_t>(c.capacity) * kKvHeads * kDim;
+    dims[2] = static_cast<cuuint64_t>(c.capacity);
+    dims[3] = static_cast<cuuint64_t>(B);
+    strides[2] = static_cast<cuuint64_t>(rs) * 2;
+  }
+  const cuuint32_t box[4] = {64, 1, static_cast<cuuint32_t>(kTile), 1};
+  const cuuint32_t estr[4] = {1, 1, 1, 1};
+  CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, base, dims, strides, box, estr,
+                  CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                  CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) return fail(FLINT_ERR_CUDA, "cuTensorMapEncodeTiled failed (CUresult %d)", (int)r);
+  return FLINT_OK;
+}
+
+// ---- validation -------------------------------------------------------------
+
+flint_status check_cache(const flint_kv_cache* c, int B, const char* who) {
+  if (!c) return fail(FLINT_ERR_INVALID_ARG, "%s: cache is NULL", who);
+  if (!c->k || !c->v) return fail(FLINT_ERR_INVALID_ARG, "%s: cache k/v is NULL", who);
+  if (!aligned16(c->k) || !aligned16(c->v))
+    return fail(FLINT_ERR_INVALID_ARG, "%s: cache k/v must be 16-byte aligned", who);
+  switch (c->layout) {
+    case FLINT_KV_CONTIGUOUS:
+    case FLINT_KV_RING: {
+      if (c->capacity < 1 || c->capacity > FLINT_MAX_CONTEXT)
+        return fail(FLINT_ERR_INVALID_ARG, "%s: capacity %d out of range", who, c->capacity);
+      if (c->layout == FLINT_KV_RING && c->capacity != kWindow)
+        return fail(FLINT_ERR_UNSUPPORTED, "%s: a ring cache must have %d slots", who, kWindow);
+      const int64_t dense = static_cast<int64_t>(c->capacity) * kKvHeads * kDim;
+      if (c->req_stride != 0 && (c->req_stride < dense || c->req_stride % 8 != 0))
+        return fail(FLINT_ERR_INVALID_ARG, "%s: req_stride %lld must be 0 or a multiple of 8 >= %lld",
+                    who, (long long)c->req_stride, (long long)dense);
+      (void)B;
+      return FLINT_OK;
+    }
+    case FLINT_KV_PAGED:
+      if (!c->block_table) return fail(FLINT_ERR_INVALID_ARG, "%s: block_table is NULL", who);
+      if (c->block_size != kBlock)
+        return fail(FLINT_ERR_UNSUPPORTED, "%s: block_size must be %d", who, kBlock);
+      if (c->max_blocks_per_req < 1 || c->num_blocks < 1)
+        return fail(FLINT_ERR_INVALID_ARG, "%s: max_blocks_per_req and num_blocks must be >= 1", who);
+      return FLINT_OK;
+    default:
+      return fail(FLINT_ERR_INVALID_ARG, "%s: unknown cache layout %d", who, c->layout);
+  }
+}
+
+// Attended range of one request in storage coordinates, plus its tiles.
+struct Range {
+  int lo, hi, tile_base, tiles;
+};
+
+Range attended_range(const flint_kv_cache& c, int L, int window) {
+  Range r;
+  if (c.layout == FLINT_KV_RING) {
+    r.lo = 0;
+    r.hi = std::min(L, c.capacity);
+    r.tile_base = 0;
+  } else {
+    r.lo = window > 0 ? std::max(0, L - window) : 0;
+    r.hi = L;
+    r.tile_base = c.layout == FLINT_KV_PAGED ? (r.lo / kBlock) * kBlock : r.lo;
+  }
+  r.tiles = (r.hi - r.tile_base + kTile - 1) / kTile;
+  return r;
+}
+
+flint_status check_len(const flint_kv_cache& c, int L, int window, const char* who, int idx) {
+  if (L < 1 || L > FLINT_MAX_CONTEXT)
+    return fail(FLINT_ERR_INVALID_ARG, "%s: length %d of item %d outside [1, %d]", who, L, idx,
+                FLINT_MAX_CONTEXT);
+  if (c.layout == FLINT_KV_CONTIGUOUS && L > c.capacity)
+    return fail(FLINT_ERR_INVALID_ARG, "%s: length %d of item %d exceeds capacity %d", who, L, idx,
+                c.capacity);
+  if (c.layout == FLINT_KV_RING && window != kWindow)
+    return fail(FLINT_ERR_UNSUPPORTED, "%s: a ring cache needs window %d", who, kWindow);
+  if (c.layout == FLINT_KV_PAGED &&
+      static_cast<int64_t>(L) > static_cast<int64_t>(c.max_blocks_per_req) * kBlock)
+    return fail(FLINT_ERR_INVALID_ARG, "%s: length %d of item %d exceeds the block table (%d blocks)",
+                who, L, idx, c.max_blocks_per_req);
+  return FLINT_OK;
+}
+
+size_t workspace_bytes(int n_problems, int num_ctas) {
+  const int64_t items = std::min<int64_t>(kMaxItems, num_ctas + static_cast<int64_t>(n_problems) * kKvHeads);
+  return kCounterBytes + static_cast<size_t>(items) * kPartialFloats * sizeof(float);
+}
+
+// Fill plan fields of P from the problems' tile counts; returns the grid.
+flint_status plan(DecodeParams& P, const int* tiles, int n_problems, int num_ctas, int* grid) {
+  int sms = num_ctas;
+  if (sms == 0 && device_num_sms(&sms) != 0)
+    return fail(FLINT_ERR_CUDA, "cannot query the SM count of the current device");
+  sms = std::min(sms, kMaxCtas);
+  int32_t seg_tiles[kMaxSegs];
+  int64_t total = 0;
+  for (int p = 0; p < n_problems; ++p)
+    for (int g = 0; g < kKvHeads; ++g) {
+      seg_tiles[p * kKvHeads + g] = tiles[p];
+      total += tiles[p];
+    }
+  const int n_segs = n_problems * kKvHeads;
+  // at least two tiles of work per CTA, never more CTAs than the device's SMs
+  const int G = static_cast<int>(std::max<int64_t>(1, std::min<int64_t>(sms, (total + 1) / 2)));
+  int32_t seg[kMaxItems], t0[kMaxItems], t1[kMaxItems], cb[kMaxCtas + 1];
+  const int n = flint_plan_items(seg_tiles, n_segs, G, kItemCost, seg, t0, t1, cb, kMaxItems);
+  if (n < 0) return fail(FLINT_ERR_UNSUPPORTED, "split plan does not fit one launch");
+  for (int i = 0; i < n; ++i) {
+    P.items[i].seg = static_cast<int16_t>(seg[i]);
+    P.items[i].t0 = static_cast<int16_t>(t0[i]);
+    P.items[i].t1 = static_cast<int16_t>(t1[i]);
+    P.items[i].pad = 0;
+  }
+  int last = 0;  // CTAs past the last one with work are not launched
+  for (int c = 0; c < G; ++c) {
+    P.cta_item_begin[c] = static_cast<int16_t>(cb[c]);
+    if (cb[c + 1] > cb[c]) last = c + 1;
+  }
+  P.cta_item_begin[G] = static_cast<int16_t>(cb[G]);
+  for (int s = 0, i = 0; s <= n_segs; ++s) {
+    while (i < n && seg[i] < s) ++i;
+    P.seg_item_begin[s] = static_cast<int16_t>(i);
+  }
+  *grid = last;
+  return FLINT_OK;
+}
+
+flint_status launch_result(cudaError_t e, const char* who) {
+  if (e != cudaSuccess) return fail(FLINT_ERR_CUDA, "%s: launch failed: %s", who, cudaGetErrorString(e));
+  return ok();
+}
+
+}  // namespace
+
+extern "C" {
+
+const char* flint_status_string(flint_status s) {
+  switch (s) {
+    case FLINT_OK: return "ok";
+    case FLINT_ERR_INVALID_ARG: return "invalid argument";
+    case FLINT_ERR_UNSUPPORTED: return "unsupported";
+    case FLINT_ERR_WORKSPACE: return "workspace too small";
+    case FLINT_ERR_CUDA: return "CUDA error";
+    case FLINT_ERR_TIMEOUT: return "device wait timed out";
+  }
+  return "unknown status";
+}
+
+const char* flint_last_error(void) { return g_last_error.c_str(); }
+
+uint64_t flint_kv_bytes(int64_t ctx_len, int32_t n_full, int32_t n_window, int32_t window,
+                        int32_t elem_bytes) {
+  if (ctx_len < 0 || n_full < 0 || n_window < 0 || window < 0 || elem_bytes < 0) return 0;
+  const uint64_t per_tok = 2ull * kKvHeads * kDim * static_cast<uint64_t>(elem_bytes);
+  const uint64_t kept = static_cast<uint64_t>(std::min<int64_t>(ctx_len, window));
+  return per_tok * (static_cast<uint64_t>(n_full) * static_cast<uint64_t>(ctx_len) +
+                    static_cast<uint64_t>(n_window) * kept);
+}
+
+flint_status flint_qk_norm_rope(const uint16_t* q_raw, const uint16_t* k_raw, const uint16_t* v_raw,
+                                const uint16_t* w_q, const uint16_t* w_k, const int32_t* pos,
+                                int32_t B, float eps, double theta, int32_t apply_rope,
+                                float* q_out, uint16_t* k_out, const flint_kv_cache* cache,
+                                int32_t* dev_err, void* stream) {
+  const char* who = "flint_qk_norm_rope";
+  if (!q_raw || !k_raw || !w_q || !w_k || !pos)
+    return fail(FLINT_ERR_INVALID_ARG, "%s: NULL input pointer", who);
+  if (B < 1 || B > FLINT_MAX_BATCH) return fail(FLINT_ERR_INVALID_ARG, "%s: B=%d outside [1, %d]", who, B, FLINT_MAX_BATCH);
+  if (apply_rope != 0 && apply_rope != 1) return fail(FLINT_ERR_INVALID_ARG, "%s: apply_rope must be 0 or 1", who);
+  if (!(eps >= 0.f) || !(theta > 0.0)) return fail(FLINT_ERR_INVALID_ARG, "%s: eps must be >= 0, theta > 0", who);
+  if (!q_out && !k_out && !cache) return fail(FLINT_ERR_INVALID_ARG, "%s: no output requested", who);
+  const void* ptrs[] = {q_raw, k_raw, w_q, w_k, q_out, k_out, v_raw};
+  for (const void* p : ptrs)
+    if (p && !aligned16(p)) return fail(FLINT_ERR_INVALID_ARG, "%s: pointers must be 16-byte aligned", who);
+  PrepParams p;
+  memset(&p, 0, sizeof p);
+  p.q_raw = q_raw;
+  p.k_raw = k_raw;
+  p.v_raw = v_raw;
+  p.w_q = w_q;
+  p.w_k = w_k;
+  p.q_out = q_out;
+  p.k_out = k_out;
+  p.eps = eps;
+  p.theta = theta;
+  p.apply_rope = apply_rope;
+  p.do_norm = 1;
+  p.dev_err = dev_err;
+  for (int b = 0; b < B; ++b) {
+    if (pos[b] < 0 || pos[b] >= FLINT_MAX_CONTEXT)
+      return fail(FLINT_ERR_INVALID_ARG, "%s: pos[%d]=%d outside [0, %d)", who, b, pos[b], FLINT_MAX_CONTEXT);
+    p.pos[b] = pos[b];
+  }
+  if (cache) {
+    if (!v_raw) return fail(FLINT_ERR_INVALID_ARG, "%s: appending needs v_raw", who);
+    flint_status s = check_cache(cache, B, who);
+    if (s != FLINT_OK) return s;
+    for (int b = 0; b < B; ++b) {
+      const flint_kv_cache& c = *cache;
+      if (c.layout == FLINT_KV_CONTIGUOUS && pos[b] >= c.capacity)
+        return fail(FLINT_ERR_INVALID_ARG, "%s: pos[%d]=%d outside the cache capacity %d", who, b, pos[b], c.capacity);
+      if (c.layout == FLINT_KV_PAGED && pos[b] / kBlock >= c.max_blocks_per_req)
+        return fail(FLINT_ERR_INVALID_ARG, "%s: pos[%d]=%d outside the block table", who, b, pos[b]);
+    }
+    p.k_rows = static_cast<uint16_t*>(cache->k);
+    p.v_rows = static_cast<uint16_t*>(cache->v);
+    p.table = cache->block_table;
+    p.layout = cache->layout;
+    p.capacity = cache->capacity;
+    p.req_stride = cache->req_stride ? cache->req_stride
+                                     : static_cast<int64_t>(cache->capacity) * kKvHeads * kDim;
+    p.max_blocks = cache->max_blocks_per_req;
+    p.num_blocks = cache->num_blocks;
+  }
+  return launch_result(launch_prep(p, B, static_cast<cudaStream_t>(stream)), who);
+}
+
+flint_status flint_kv_append(const uint16_t* k, const uint16_t* v, const int32_t* pos, int32_t B,
+                             const flint_kv_cache* cache, int32_t* dev_err, void* stream) {
+  const char* who = "flint_kv_append";
+  if (!k || !v || !pos) return fail(FLINT_ERR_INVALID_ARG, "%s: NULL input pointer", who);
+  if (!aligned16(k) || !aligned16(v)) return fail(FLINT_ERR_INVALID_ARG, "%s: k/v must be 16-byte aligned", who);
+  if (B < 1 || B > FLINT_MAX_BATCH) return fail(FLINT_ERR_INVALID_ARG, "%s: B=%d outside [1, %d]", who, B, FLINT_MAX_BATCH);
+  flint_status s = check_cache(cache, B, who);
+  if (s != FLINT_OK) return s;
+  PrepParams p;
+  memset(&p, 0, sizeof p);
+  p.k_raw = k;
+  p.v_raw = v;
+  p.dev_err = dev_err;
+  p.do_norm = 0;
+  p.apply_rope = 0;
+  for (int b = 0; b < B; ++b) {
+    if (pos[b] < 0 || pos[b] >= FLINT_MAX_CONTEXT)
+      return fail(FLINT_ERR_INVALID_ARG, "%s: pos[%d]=%d outside [0, %d)", who, b, pos[b], FLINT_MAX_CONTEXT);
+    if (cache->layout == FLINT_KV_CONTIGUOUS && pos[b] >= cache->capacity)
+      return fail(FLINT_ERR_INVALID_ARG, "%s: pos[%d]=%d outside the cache capacity %d", who, b, pos[b], cache->capacity);
+    if (cache->layout == FLINT_KV_PAGED && pos[b] / kBlock >= cache->max_blocks_per_req)
+      return fail(FLINT_ERR_INVALID_ARG, "%s: pos[%d]=%d outside the block table", who, b, pos[b]);
+    p.pos[b] = pos[b];
+  }
+  p.k_rows = static_cast<uint16_t*>(cache->k);
+  p.v_rows = static_cast<uint16_t*>(cache->v);
+  p.table = cache->block_table;
+  p.layout = cache->layout;
+  p.capacity = cache->capacity;
+  p.req_stride = cache->req_stride ? cache->req_stride
+                                   : static_cast<int64_t>(cache->capacity) * kKvHeads * kDim;
+  p.max_blocks = cache->max_blocks_per_req;
+  p.num_blocks = cache->num_blocks;
+  return launch_result(launch_prep(p, B, static_cast<cudaStream_t>(stream)), who);
+}
+
+size_t flint_attn_workspace_bytes(int32_t n_problems, int32_t num_ctas) {
+  if (n_problems < 1 || n_problems > kMaxProblems || num_ctas < 0 || num_ctas > kMaxCtas) return 0;
+  int g = num_ctas;
+  if (g == 0 && device_num_sms(&g) != 0) g = kMaxCtas;
+  return workspace_bytes(n_problems, std::min(g, kMaxCtas));
+}
+
+flint_status flint_attn_decode(const void* q, int32_t q_is_fp32, const flint_kv_cache* cache,
+                               const int32_t* seq_lens, int32_t B, const float* sinks,
+                               int32_t window, float* out, void* workspace, size_t ws_bytes,
+                               int32_t num_ctas, int32_t* dev_err, void* stream) {
+  const char* who = "flint_attn_decode";
+  if (!q || !seq_lens || !sinks || !out || !workspace)
+    return fail(FLINT_ERR_INVALID_ARG, "%s: NULL pointer argument", who);
+  if (B < 1 || B > FLINT_MAX_BATCH) return fail(FLINT_ERR_INVALID_ARG, "%s: B=%d outside [1, %d]", who, B, FLINT_MAX_BATCH);
+  if (q_is_fp32 != 0 && q_is_fp32 != 1) return fail(FLINT_ERR_INVALID_ARG, "%s: q_is_fp32 must be 0 or 1", who);
+  if (window != 0 && window != kWindow) return fail(FLINT_ERR_UNSUPPORTED, "%s: window must be 0 or %d", who, kWindow);
+  if (num_ctas < 0 || num_ctas > kMaxCtas) return fail(FLINT_ERR_INVALID_ARG, "%s: num_ctas %d outside [0, %d]", who, num_ctas, kMaxCtas);
+  if (!aligned16(q) || !aligned16(out) || !aligned16(workspace) || (reinterpret_cast<uintptr_t>(sinks) & 3u))
+    return fail(FLINT_ERR_INVALID_ARG, "%s: q/out/workspace must be 16-byte aligned", who);
+  flint_status s = check_cache(cache, B, who);
+  if (s != FLINT_OK) return s;
+  int tiles[kMaxProblems];
+  static thread_local DecodeParams P;
+  memset(&P, 0, sizeof P);
+  for (int b = 0; b < B; ++b) {
+    s = check_len(*cache, seq_lens[b], window, who, b);
+    if (s != FLINT_OK) return s;
+    const Range r = attended_range(*cache, seq_lens[b], window);
+    Problem& pb = P.prob[b];
+    pb.q = static_cast<const uint8_t*>(q) + static_cast<size_t>(b) * kHeads * kDim * (q_is_fp32 ? 4 : 2);
+    pb.sinks = sinks;
+    pb.out = out + static_cast<size_t>(b) * kHeads * kDim;
+    pb.table = cache->layout == FLINT_KV_PAGED
+                   ? cache->block_table + static_cast<size_t>(b) * cache->max_blocks_per_req
+                   : nullptr;
+    pb.lo = r.lo;
+    pb.hi = r.hi;
+    pb.tile_base = r.tile_base;
+    pb.append_tok = -1;
+    pb.pos = seq_lens[b] - 1;
+    pb.num_blocks = cache->num_blocks;
+    pb.map_k = 0;
+    pb.map_v = 1;
+    pb.req = static_cast<int16_t>(cache->layout == FLINT_KV_PAGED ? 0 : b);
+    pb.layout = static_cast<int8_t>(cache->layout);
+    pb.q_fp32 = static_cast<int8_t>(q_is_fp32);
+    tiles[b] = r.tiles;
+  }
+  int grid = 0;
+  s = plan(P, tiles, B, num_ctas, &grid);
+  if (s != FLINT_OK) return s;
+  if (ws_bytes < workspace_bytes(B, grid))
+    return fail(FLINT_ERR_WORKSPACE, "%s: workspace of %zu bytes is below the %zu needed", who, ws_bytes,
+                workspace_bytes(B, grid));
+  s = encode_cache_map(&P.maps[0], cache->k, *cache, B);
+  if (s != FLINT_OK) return s;
+  s = encode_cache_map(&P.maps[1], cache->v, *cache, B);
+  if (s != FLINT_OK) return s;
+  P.counters = static_cast<int32_t*>(workspace);
+  P.partials = reinterpret_cast<float*>(static_cast<uint8_t*>(workspace) + kCounterBytes);
+  P.dev_err = dev_err;
+  P.n_problems = B;
+  P.prep = 0;
+  P.eps = 0.f;
+  P.theta = 0.0;
+  return launch_result(launch_decode(P, grid, static_cast<cudaStream_t>(stream)), who);
+}
+
+flint_status flint_attn_stack(const flint_layer* layers, int32_t n_layers, int32_t pos, float eps,
+                              double theta, float* out, void* workspace, size_t ws_bytes,
+                              int32_t num_ctas, int32_t* dev_err, void* stream) {
+  const char* who = "flint_attn_stack";
+  if (!layers || !out || !workspace) return fail(FLINT_ERR_INVALID_ARG, "%s: NULL pointer argument", who);
+  if (n_layers < 1 || n_layers > FLINT_MAX_LAYERS)
+    return fail(FLINT_ERR_INVALID_ARG, "%s: n_layers=%d outside [1, %d]", who, n_layers, FLINT_MAX_LAYERS);
+  if (pos < 0 || pos >= FLINT_MAX_CONTEXT) return fail(FLINT_ERR_INVALID_ARG, "%s: pos=%d outside [0, %d)", who, pos, FLINT_MAX_CONTEXT);
+  if (!(eps >= 0.f) || !(theta > 0.0)) return fail(FLINT_ERR_INVALID_ARG, "%s: eps must be >= 0, theta > 0", who);
+  if (num_ctas < 0 || num_ctas > kMaxCtas) return fail(FLINT_ERR_INVALID_ARG, "%s: num_ctas %d outside [0, %d]", who, num_ctas, kMaxCtas);
+  if (!aligned16(out) || !aligned16(workspace)) return fail(FLINT_ERR_INVALID_ARG, "%s: out/workspace must be 16-byte aligned", who);
+  const int L = pos + 1;
+  int tiles[kMaxProblems];
+  static thread_local DecodeParams P;
+  memset(&P, 0, sizeof P);
+  for (int i = 0; i < n_layers; ++i) {
+    const flint_layer& ly = layers[i];
+    if (!ly.q_raw || !ly.k_raw || !ly.v_raw || !ly.w_q || !ly.w_k || !ly.sinks)
+      return fail(FLINT_ERR_INVALID_ARG, "%s: layer %d has a NULL pointer", who, i);
+    const void* ptrs[] = {ly.q_raw, ly.k_raw, ly.v_raw, ly.w_q, ly.w_k};
+    for (const void* p : ptrs)
+      if (!aligned16(p)) return fail(FLINT_ERR_INVALID_ARG, "%s: layer %d pointers must be 16-byte aligned", who, i);
+    if (ly.window != 0 && ly.window != kWindow)
+      return fail(FLINT_ERR_UNSUPPORTED, "%s: layer %d window must be 0 or %d", who, i, kWindow);
+    if (ly.rope != 0 && ly.rope != 1) return fail(FLINT_ERR_INVALID_ARG, "%s: layer %d rope must be 0 or 1", who, i);
+    flint_status s = check_cache(&ly.cache, 1, who);
+    if (s != FLINT_OK) return s;
+    s = check_len(ly.cache, L, ly.window, who, i);
+    if (s != FLINT_OK) return s;
+    const Range r = attended_range(ly.cache, L, ly.window);
+    Problem& pb = P.prob[i];
+    pb.q = ly.q_raw;
+    pb.k_raw = ly.k_raw;
+    pb.v_raw = ly.v_raw;
+    pb.w_q = ly.w_q;
+    pb.w_k = ly.w_k;
+    pb.sinks = ly.sinks;
+    pb.out = out + static_cast<size_t>(i) * kHeads * kDim;
+    pb.k_rows = static_cast<uint16_t*>(ly.cache.k);
+    pb.v_rows = static_cast<uint16_t*>(ly.cache.v);
+    pb.table = ly.cache.layout == FLINT_KV_PAGED ? ly.cache.block_table : nullptr;
+    pb.lo = r.lo;
+    pb.hi = r.hi;
+    pb.tile_base = r.tile_base;
+    pb.pos = pos;
+    pb.append_tok = ly.cache.layout == FLINT_KV_RING ? pos % ly.cache.capacity : pos;
+    pb.num_blocks = ly.cache.num_blocks;
+    pb.map_k = static_cast<int16_t>(2 * i);
+    pb.map_v = static_cast<int16_t>(2 * i + 1);
+    pb.req = 0;
+    pb.layout = static_cast<int8_t>(ly.cache.layout);
+    pb.q_fp32 = 0;
+    pb.rope = static_cast<int8_t>(ly.rope);
+    tiles[i] = r.tiles;
+    s = encode_cache_map(&P.maps[2 * i], ly.cache.k, ly.cache, 1);
+    if (s != FLINT_OK) return s;
+    s = encode_cache_map(&P.maps[2 * i + 1], ly.cache.v, ly.cache, 1);
+    if (s != FLINT_OK) return s;
+  }
+  int grid = 0;
+  flint_status s = plan(P, tiles, n_layers, num_ctas, &grid);
+  if (s != FLINT_OK) return s;
+  if (ws_bytes < workspace_bytes(n_layers, grid))
+    return fail(FLINT_ERR_WORKSPACE, "%s: workspace of %zu bytes is below the %zu needed", who, ws_bytes,
+                workspace_bytes(n_layers, grid));
+  P.counters = static_cast<int32_t*>(workspace);
+  P.partials = reinterpret_cast<float*>(static_cast<uint8_t*>(workspace) + kCounterBytes);
+  P.dev_err = dev_err;
+  P.n_problems = n_layers;
+  P.prep = 1;
+  P.eps = eps;
+  P.theta = theta;
+  return launch_result(launch_decode(P, grid, static_cast<cudaStream_t>(stream)), who);
+}
+
+}  // extern "C"

@@ -1,0 +1,510 @@
+// flint_decode.cu -- split-KV flash-decode for Flint's grouped-query attention
+// with a per-head sink logit, on sm_100a.
+//
+// What is computed (page "Day-0 Support for Flint on vLLM", hnkhoi.com,
+// "Model architecture": GQA 32 query / 4 KV heads, learned attention sinks,
+// 513-token sliding window or full context): for query head h of KV group
+// g = h / 8 and its token range R,
+//     out_h = sum_{j in R} e^(s_j - M) V_j / (sum_{j in R} e^(s_j - M) + e^(sink_h - M)),
+//     s_j = q_h . K_j / sqrt(128),  M = max(max_j s_j, sink_h).
+//
+// How (one persistent launch for every problem of the call):
+//   * The host cuts each (problem, KV head) token range into 64-token tiles and
+//     lays the tiles over one CTA per SM (split-KV); each CTA walks its list
+//     of items (segment, tile range).
+//   * Warp 4 is the producer: it streams K and V tiles with TMA (4-D tensor
+//     maps, 128-byte swizzle) into a 6-stage ring of 32 KiB stages guarded by
+//     mbarriers.  In the fused layer-stack mode it also writes the new token's
+//     k (RMSNorm + RoPE) and v into the cache just before loading that tile.
+//   * Warps 0-3 consume tiles round-robin.  All 8 query heads of the group
+//     share every K/V tile: S^T = [q_hi; q_lo] K^T and O += [P_hi; P_lo] V run
+//     on bf16 mma.sync m16n8k16, where the 16 rows of A are the 8 heads' hi
+//     and lo bf16 parts (fp32 values split in two), so the products carry ~16
+//     significant bits while K/V stay exact bf16.  Softmax runs in fp32 in
+//     log2 units with quad shuffles; the running max is only moved when it
+//     grows by more than 2^8, so rescales are rare.
+//   * Item end: the four warps' (m, l, O) merge in shared memory.  A segment
+//     covered by one item is finished on the spot (sink folded in); otherwise
+//     the CTA stores a partial and the last CTA to arrive (atomic counter, no
+//     spinning) merges all partials of the segment in a fixed order and folds
+//     in the sink, so results are deterministic.
+// Every mbarrier wait is bounded in time; on timeout the kernel records
+// FLINT_ERR_TIMEOUT, lets its loads land and returns.
+#include <math.h>
+
+#include "flint_device.cuh"
+
+namespace flint {
+
+namespace {
+
+constexpr float kLog2e = 1.4426950408889634f;
+// log2(e) / sqrt(128): scores come out of the tensor cores in log2 units.
+constexpr float kQScale = static_cast<float>(1.4426950408889634 * 0.08838834764831845);
+constexpr float kRescaleSlack = 8.0f;
+constexpr int kXchStride = kDim + 2;  // per head: 128 O values, m, l
+constexpr int kXchFloats = kConsumerWarps * kGroup * kXchStride;
+
+struct Smem {
+  uint8_t* stages;
+  uint64_t* full;
+  uint64_t* empty;
+  float* xch;
+  float2* cs;
+  volatile int* flags;  // [0] abort, [1] last-arrival broadcast
+};
+
+__device__ __forceinline__ Smem carve(uint8_t* raw) {
+  Smem s;
+  uint8_t* base = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(raw) + 1023) & ~uintptr_t(1023));
+  s.stages = base;
+  s.full = reinterpret_cast<uint64_t*>(base + kStages * kStageBytes);
+  s.empty = s.full + kStages;
+  s.xch = reinterpret_cast<float*>(s.empty + kStages);
+  s.cs = reinterpret_cast<float2*>(s.xch + kXchFloats);
+  s.flags = reinterpret_cast<volatile int*>(s.cs + 64);
+  return s;
+}
+
+__device__ __forceinline__ void consumer_bar() {
+  asm volatile("bar.sync 1, %0;" ::"n"(kConsumerWarps * 32) : "memory");
+}
+
+// Raise the CTA abort flag after a failed wait (timeout unless already aborted).
+__device__ __forceinline__ void abort_cta(const DecodeParams& P, const Smem& S) {
+  if (!S.flags[0]) report_error(P.dev_err, FLINT_ERR_TIMEOUT);
+  S.flags[0] = 1;
+}
+
+// Storage offset (elements, from the cache base the problem names) of row
+// (position pos, KV head g); -1 if a paged block id is out of range.
+__device__ __forceinline__ long long append_offset(const Problem& pb, int g) {
+  if (pb.layout == FLINT_KV_PAGED) {
+    const int blk = pb.table[pb.pos / kBlock];
+    if (blk < 0 || blk >= pb.num_blocks) return -1;
+    return ((static_cast<long long>(blk) * kBlock + pb.pos % kBlock) * kKvHeads + g) * kDim;
+  }
+  return (static_cast<long long>(pb.append_tok) * kKvHeads + g) * kDim;
+}
+
+// Producer-warp side of the fused stack: norm (+RoPE) the new token's k for
+// KV head g, round to bf16 and write it and v_raw into the cache.
+__device__ void append_new_token(const DecodeParams& P, const Problem& pb, int g, int lane,
+                                 const float2* cs) {
+  float y[4];
+  norm_rope_row_warp(pb.k_raw + g * kDim, pb.w_k, P.eps, true, pb.rope != 0, cs, lane, y);
+  const long long off = append_offset(pb, g);
+  if (off < 0) {
+    if (lane == 0) report_error(P.dev_err, FLINT_ERR_INVALID_ARG);
+    return;
+  }
+  uint32_t* kd = reinterpret_cast<uint32_t*>(pb.k_rows + off);
+  uint32_t* vd = reinterpret_cast<uint32_t*>(pb.v_rows + off);
+  const uint32_t* vs = reinterpret_cast<const uint32_t*>(pb.v_raw + g * kDim);
+  kd[lane] = pack_bf16x2(y[0], y[1]);
+  kd[32 + lane] = pack_bf16x2(y[2], y[3]);
+  vd[lane] = vs[lane];
+  vd[32 + lane] = vs[32 + lane];
+  fence_proxy_async_global();
+}
+
+// Returns the number of tiles whose loads were issued.
+__device__ int run_producer(const DecodeParams& P, const Smem& S, int it0, int it1, int lane) {
+  int seq = 0;
+  for (int it = it0; it < it1; ++it) {
+    const Item item = P.items[it];
+    const Problem& pb = P.prob[item.seg >> 2];
+    const int g = item.seg & 3;
+    const CUtensorMap* mk = &P.maps[pb.map_k];
+    const CUtensorMap* mv = &P.maps[pb.map_v];
+    const bool paged = pb.layout == FLINT_KV_PAGED;
+    const int app_tile = (P.prep && pb.append_tok >= 0) ? (pb.append_tok - pb.tile_base) / kTile : -1;
+    for (int t = item.t0; t < item.t1; t += 32) {
+      const int n = min(32, item.t1 - t);
+      int blk = 0;
+      if (paged && lane < n) {
+        blk = __ldg(pb.table + pb.tile_base / kBlock + t + lane);
+        // An out-of-range coordinate makes TMA fill zeros; flag it for the caller.
+        if (blk < 0 || blk >= pb.num_blocks) report_error(P.dev_err, FLINT_ERR_INVALID_ARG);
+      }
+      for (int j = 0; j < n; ++j, ++seq) {
+        const int b = __shfl_sync(0xffffffffu, blk, j);
+        const int stage = seq % kStages;
+        const uint32_t phase = static_cast<uint32_t>(seq / kStages) & 1u;
+        bool ok = true;
+        if (lane == 0) ok = mbar_wait(smem_u32(&S.empty[stage]), phase ^ 1u, S.flags);
+        ok = __shfl_sync(0xffffffffu, ok, 0);
+        if (!ok) {
+          if (lane == 0) abort_cta(P, S);
+          return seq;
+        }
+        const int tile = t + j;
+        if (tile == app_tile) {
+          append_new_token(P, pb, g, lane, S.cs);
+          __syncwarp();
+        }
+        if (lane == 0) {
+          const uint32_t fb = smem_u32(&S.full[stage]);
+          const uint32_t dst = smem_u32(S.stages + stage * kStageBytes);
+          const int c2 = paged ? 0 : pb.tile_base + tile * kTile;
+          const int c3 = paged ? b : pb.req;
+          mbar_expect_tx(fb, kStageBytes);
+          tma_load_4d(dst, mk, fb, 0, g, c2, c3);
+          tma_load_4d(dst + kHalfBytes, mk, fb, 64, g, c2, c3);
+          tma_load_4d(dst + 2 * kHalfBytes, mv, fb, 0, g, c2, c3);
+          tma_load_4d(dst + 3 * kHalfBytes, mv, fb, 64, g, c2, c3);
+        }
+        __syncwarp();
+      }
+    }
+  }
+  return seq;
+}
+
+// q fragments for query head h: thread (g = lane/4, c = lane%4) holds dims
+// 16kk + 2c + {0,1} and 16kk + 2c + 8 + {0,1} for kk = 0..7 as the A operand
+// rows g (bf16 hi part) and g + 8 (bf16 lo part), prescaled by log2(e)/sqrt(128).
+__device__ __forceinline__ void load_q(const DecodeParams& P, const Problem& pb, int h, int c,
+                                       const float2* cs, uint32_t (&qa)[8][4]) {
+  float x[8][4];
+  if (P.prep || !pb.q_fp32) {
+    const uint16_t* q = static_cast<const uint16_t*>(pb.q) + h * kDim;
+#pragma unroll
+    for (int kk = 0; kk < 8; ++kk) {
+      const uint32_t a = *reinterpret_cast<const uint32_t*>(q + 16 * kk + 2 * c);
+      const uint32_t b = *reinterpret_cast<const uint32_t*>(q + 16 * kk + 2 * c + 8);
+      x[kk][0] = bf16_lo(a);
+      x[kk][1] = bf16_hi(a);
+      x[kk][2] = bf16_lo(b);
+      x[kk][3] = bf16_hi(b);
+    }
+  } else {
+    const float* q = static_cast<const float*>(pb.q) + h * kDim;
+#pragma unroll
+    for (int kk = 0; kk < 8; ++kk) {
+      const float2 a = *reinterpret_cast<const float2*>(q + 16 * kk + 2 * c);
+      const float2 b = *reinterpret_cast<const float2*>(q + 16 * kk + 2 * c + 8);
+      x[kk][0] = a.x;
+      x[kk][1] = a.y;
+      x[kk][2] = b.x;
+      x[kk][3] = b.y;
+    }
+  }
+  if (P.prep) {
+    // per-head RMSNorm over the quad's 128 values, then RoPE pairs (i, i+64),
+    // which sit in the same thread at kk and kk + 4
+    float ss = 0.f;
+#pragma unroll
+    for (int kk = 0; kk < 8; ++kk)
+#pragma unroll
+      for (int e = 0; e < 4; ++e) ss += x[kk][e] * x[kk][e];
+    ss += __shfl_xor_sync(0xffffffffu, ss, 1);
+    ss += __shfl_xor_sync(0xffffffffu, ss, 2);
+    const float r = 1.0f / sqrtf(ss * (1.0f / kDim) + P.eps);
+#pragma unroll
+    for (int kk = 0; kk < 8; ++kk) {
+      const uint32_t a = *reinterpret_cast<const uint32_t*>(pb.w_q + 16 * kk + 2 * c);
+      const uint32_t b = *reinterpret_cast<const uint32_t*>(pb.w_q + 16 * kk + 2 * c + 8);
+      x[kk][0] = x[kk][0] * r * bf16_lo(a);
+      x[kk][1] = x[kk][1] * r * bf16_hi(a);
+      x[kk][2] = x[kk][2] * r * bf16_lo(b);
+      x[kk][3] = x[kk][3] * r * bf16_hi(b);
+    }
+    if (pb.rope) {
+#pragma unroll
+      for (int kk = 0; kk < 4; ++kk)
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          const float2 t = cs[16 * kk + 2 * c + (e & 1) + ((e >> 1) << 3)];
+          const float a = x[kk][e], b = x[kk + 4][e];
+          x[kk][e] = a * t.x - b * t.y;
+          x[kk + 4][e] = b * t.x + a * t.y;
+        }
+    }
+  }
+#pragma unroll
+  for (int kk = 0; kk < 8; ++kk) {
+    split_bf16x2(x[kk][0] * kQScale, x[kk][1] * kQScale, qa[kk][0], qa[kk][1]);
+    split_bf16x2(x[kk][2] * kQScale, x[kk][3] * kQScale, qa[kk][2], qa[kk][3]);
+  }
+}
+
+// One 64-token tile for this warp's 8 heads: online-softmax update of
+// (m_run, l_run, o).  tok0 is the storage token of the tile's first row.
+__device__ __forceinline__ void consume_tile(uint32_t sK, int tok0, int lo, int hi, int lane,
+                                             const uint32_t (&qa)[8][4], float& m_run,
+                                             float& l_run, float (&o)[16][4]) {
+  const int c = lane & 3;
+  const int l7 = lane & 7;
+  const bool whole = (tok0 >= lo) && (tok0 + kTile <= hi);
+
+  // S^T = [q_hi; q_lo] * K^T: 8 n-tiles of 8 tokens, 8 k-steps of 16 dims.
+  float sc[16];
+#pragma unroll
+  for (int j = 0; j < 8; ++j) {
+    float acc[4] = {0.f, 0.f, 0.f, 0.f};
+    const uint32_t row = sK + (8 * j + l7) * 128;
+#pragma unroll
+    for (int kk = 0; kk < 8; kk += 2) {
+      const int u = 2 * kk + (lane >> 3);  // 16-byte unit along the 128 dims
+      uint32_t b0, b1, b2, b3;
+      ldsm_x4(row + (u >> 3) * kHalfBytes + (((u & 7) ^ l7) << 4), b0, b1, b2, b3);
+      mma_bf16_16816(acc, qa[kk], b0, b1);
+      mma_bf16_16816(acc, qa[kk + 1], b2, b3);
+    }
+    sc[2 * j] = acc[0] + acc[2];
+    sc[2 * j + 1] = acc[1] + acc[3];
+  }
+  if (!whole) {
+#pragma unroll
+    for (int j = 0; j < 8; ++j)
+#pragma unroll
+      for (int e = 0; e < 2; ++e) {
+        const int tok = tok0 + 8 * j + 2 * c + e;
+        if (tok < lo || tok >= hi) sc[2 * j + e] = -INFINITY;
+      }
+  }
+
+  float mx = sc[0];
+#pragma unroll
+  for (int i = 1; i < 16; ++i) mx = fmaxf(mx, sc[i]);
+  mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 1));
+  mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 2));
+  if (mx > m_run + kRescaleSlack) {  // also taken on the first valid tile
+    const float alpha = exp2f(m_run - mx);
+    l_run *= alpha;
+#pragma unroll
+    for (int n = 0; n < 16; ++n)
+#pragma unroll
+      for (int e = 0; e < 4; ++e) o[n][e] *= alpha;
+    m_run = mx;
+  }
+  const float mu = (m_run == -INFINITY) ? 0.f : m_run;
+
+  // P = 2^(s - m) split into bf16 hi/lo rows of the A operand.
+  uint32_t pa[4][4];
+#pragma unroll
+  for (int ks = 0; ks < 4; ++ks) {
+    const float p0 = exp2f(sc[4 * ks] - mu), p1 = exp2f(sc[4 * ks + 1] - mu);
+    const float p2 = exp2f(sc[4 * ks + 2] - mu), p3 = exp2f(sc[4 * ks + 3] - mu);
+    l_run += (p0 + p1) + (p2 + p3);
+    split_bf16x2(p0, p1, pa[ks][0], pa[ks][1]);
+    split_bf16x2(p2, p3, pa[ks][2], pa[ks][3]);
+  }
+
+  // O += [P_hi; P_lo] * V: 4 k-steps of 16 tokens, 16 n-tiles of 8 dims.
+  const uint32_t sV = sK + 2 * kHalfBytes;
+#pragma unroll
+  for (int ks = 0; ks < 4; ++ks) {
+    uint32_t m01 = 0xffffffffu, m23 = 0xffffffffu;
+    if (!whole) {
+      const int t = tok0 + 16 * ks + 2 * c;
+      m01 = ((t >= lo && t < hi) ? 0x0000ffffu : 0u) | ((t + 1 >= lo && t + 1 < hi) ? 0xffff0000u : 0u);
+      m23 = ((t + 8 >= lo && t + 8 < hi) ? 0x0000ffffu : 0u) |
+            ((t + 9 >= lo && t + 9 < hi) ? 0xffff0000u : 0u);
+    }
+    const uint32_t row = sV + (16 * ks + ((lane >> 3) & 1) * 8 + l7) * 128;
+#pragma unroll
+    for (int np = 0; np < 8; ++np) {
+      const int nt = 2 * np + (lane >> 4);
+      uint32_t v0, v1, v2, v3;
+      ldsm_x4_t(row + (nt >> 3) * kHalfBytes + (((nt & 7) ^ l7) << 4), v0, v1, v2, v3);
+      if (!whole) {  // rows outside the range may hold anything (even NaN)
+        v0 &= m01;
+        v2 &= m01;
+        v1 &= m23;
+        v3 &= m23;
+      }
+      mma_bf16_16816(o[2 * np], pa[ks], v0, v1);
+      mma_bf16_16816(o[2 * np + 1], pa[ks], v2, v3);
+    }
+  }
+}
+
+// Final normalisation with the sink logit of head kvh*8 + hh folded in.
+__device__ __forceinline__ void finish_head(const Problem& pb, int kvh, int hh, int d0, float M,
+                                            float L, const float (&acc)[8]) {
+  const int head = kvh * kGroup + hh;
+  const float s2 = pb.sinks[head] * kLog2e;
+  const float Mf = fmaxf(M, s2);
+  const float a = (M == -INFINITY) ? 0.f : exp2f(M - Mf);
+  const float inv = 1.0f / (L * a + exp2f(s2 - Mf));
+  float4* dst = reinterpret_cast<float4*>(pb.out + head * kDim + d0);
+  dst[0] = make_float4(acc[0] * a * inv, acc[1] * a * inv, acc[2] * a * inv, acc[3] * a * inv);
+  dst[1] = make_float4(acc[4] * a * inv, acc[5] * a * inv, acc[6] * a * inv, acc[7] * a * inv);
+}
+
+__device__ void run_consumer(const DecodeParams& P, const Smem& S, int it0, int it1, int warp,
+                             int lane) {
+  const int g = lane >> 2, c = lane & 3;
+  const int t = threadIdx.x;              // 0..127 within the consumer warps
+  const int hh = t >> 4, d0 = (t & 15) * 8;  // merge role: head, 8 dims
+  int seq = 0;
+  for (int it = it0; it < it1; ++it) {
+    const Item item = P.items[it];
+    const Problem& pb = P.prob[item.seg >> 2];
+    const int kvh = item.seg & 3;
+
+    uint32_t qa[8][4];
+    load_q(P, pb, kvh * kGroup + g, c, S.cs, qa);
+
+    float m_run = -INFINITY, l_run = 0.f;
+    float o[16][4];
+#pragma unroll
+    for (int n = 0; n < 16; ++n)
+#pragma unroll
+      for (int e = 0; e < 4; ++e) o[n][e] = 0.f;
+
+    const int ntiles = item.t1 - item.t0;
+    for (int k = 0; k < ntiles; ++k, ++seq) {
+      if (seq % kConsumerWarps != warp) continue;
+      const int stage = seq % kStages;
+      const uint32_t phase = static_cast<uint32_t>(seq / kStages) & 1u;
+      bool ok = true;
+      if (lane == 0) ok = mbar_wait(smem_u32(&S.full[stage]), phase, S.flags);
+      ok = __shfl_sync(0xffffffffu, ok, 0);
+      if (!ok) {
+        if (lane == 0) abort_cta(P, S);
+        continue;  // keep walking so that every warp meets the same barriers
+      }
+      const int tok0 = pb.tile_base + (item.t0 + k) * kTile;
+      consume_tile(smem_u32(S.stages + stage * kStageBytes), tok0, pb.lo, pb.hi, lane, qa, m_run,
+                   l_run, o);
+      __syncwarp();
+      if (lane == 0) mbar_arrive(smem_u32(&S.empty[stage]));
+    }
+
+    // ---- merge the four warps' states for this item
+    l_run += __shfl_xor_sync(0xffffffffu, l_run, 1);
+    l_run += __shfl_xor_sync(0xffffffffu, l_run, 2);
+    float* xw = S.xch + (warp * kGroup + g) * kXchStride;
+#pragma unroll
+    for (int n = 0; n < 16; ++n)
+      *reinterpret_cast<float2*>(xw + 8 * n + 2 * c) = make_float2(o[n][0] + o[n][2], o[n][1] + o[n][3]);
+    if (c == 0) {
+      xw[kDim] = m_run;
+      xw[kDim + 1] = l_run;
+    }
+    consumer_bar();
+
+    float M = -INFINITY;
+#pragma unroll
+    for (int w = 0; w < kConsumerWarps; ++w) M = fmaxf(M, S.xch[(w * kGroup + hh) * kXchStride + kDim]);
+    float L = 0.f, acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+    for (int w = 0; w < kConsumerWarps; ++w) {
+      const float* xr = S.xch + (w * kGroup + hh) * kXchStride;
+      const float mw = xr[kDim];
+      const float sw = (mw == -INFINITY) ? 0.f : exp2f(mw - M);
+      L += sw * xr[kDim + 1];
+#pragma unroll
+      for (int i = 0; i < 8; ++i) acc[i] += sw * xr[d0 + i];
+    }
+
+    const int seg = item.seg;
+    const int s0 = P.seg_item_begin[seg], s1 = P.seg_item_begin[seg + 1];
+    if (s1 - s0 == 1) {
+      finish_head(pb, kvh, hh, d0, M, L, acc);
+    } else {
+      float* part = P.partials + static_cast<size_t>(it) * kPartialFloats;
+      float4* pd = reinterpret_cast<float4*>(part + hh * kDim + d0);
+      pd[0] = make_float4(acc[0], acc[1], acc[2], acc[3]);
+      pd[1] = make_float4(acc[4], acc[5], acc[6], acc[7]);
+      if ((t & 15) == 0) {
+        part[kGroup * kDim + hh] = M;
+        part[kGroup * kDim + kGroup + hh] = L;
+      }
+      __threadfence();
+      consumer_bar();
+      if (t == 0) {
+        const int prev = atomicAdd(P.counters + seg, 1);
+        S.flags[1] = (prev == s1 - s0 - 1) ? 1 : 0;
+      }
+      consumer_bar();
+      if (S.flags[1]) {
+        // last arrival: merge every partial of the segment, in item order
+        __threadfence();
+        float M2 = -INFINITY;
+        for (int i = s0; i < s1; ++i)
+          M2 = fmaxf(M2, __ldcg(P.partials + static_cast<size_t>(i) * kPartialFloats + kGroup * kDim + hh));
+        float L2 = 0.f, acc2[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+        for (int i = s0; i < s1; ++i) {
+          const float* pi = P.partials + static_cast<size_t>(i) * kPartialFloats;
+          const float mi = __ldcg(pi + kGroup * kDim + hh);
+          const float si = (mi == -INFINITY) ? 0.f : exp2f(mi - M2);
+          L2 += si * __ldcg(pi + kGroup * kDim + kGroup + hh);
+          const float4 a = __ldcg(reinterpret_cast<const float4*>(pi + hh * kDim + d0));
+          const float4 b = __ldcg(reinterpret_cast<const float4*>(pi + hh * kDim + d0 + 4));
+          acc2[0] += si * a.x; acc2[1] += si * a.y; acc2[2] += si * a.z; acc2[3] += si * a.w;
+          acc2[4] += si * b.x; acc2[5] += si * b.y; acc2[6] += si * b.z; acc2[7] += si * b.w;
+        }
+        finish_head(pb, kvh, hh, d0, M2, L2, acc2);
+        if (t == 0) P.counters[seg] = 0;  // ready for the next call
+      }
+    }
+    consumer_bar();  // the exchange area and flags[1] are reused by the next item
+  }
+}
+
+__global__ void __launch_bounds__(kThreads, 1) decode_kernel(const __grid_constant__ DecodeParams P) {
+  extern __shared__ uint8_t smem_raw[];
+  const Smem S = carve(smem_raw);
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int it0 = P.cta_item_begin[blockIdx.x], it1 = P.cta_item_begin[blockIdx.x + 1];
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < kStages; ++s) {
+      mbar_init(smem_u32(&S.full[s]), 1);
+      mbar_init(smem_u32(&S.empty[s]), 1);
+    }
+    S.flags[0] = 0;
+    S.flags[1] = 0;
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+  }
+  if (P.prep && threadIdx.x < 64) S.cs[threadIdx.x] = rope_cos_sin(threadIdx.x, P.prob[0].pos, P.theta);
+  __syncthreads();
+
+  int issued = 0;
+  if (warp == kConsumerWarps) {
+    issued = run_producer(P, S, it0, it1, lane);
+  } else {
+    run_consumer(P, S, it0, it1, warp, lane);
+  }
+  __syncthreads();
+  // After an abort, let every issued load land before the CTA's shared memory
+  // goes away (bounded as well; a normal run returns at once).
+  if (warp == kConsumerWarps && lane == 0) {
+    const int first = issued > kStages ? issued - kStages : 0;
+    for (int s = first; s < issued; ++s) {
+      const unsigned long long t0 = globaltimer_ns();
+      while (!mbar_try_wait(smem_u32(&S.full[s % kStages]), static_cast<uint32_t>(s / kStages) & 1u)) {
+        if (globaltimer_ns() - t0 > kWaitLimitNs) break;
+      }
+    }
+  }
+}
+
+}  // namespace
+
+size_t decode_smem_bytes() {
+  return 1024 + static_cast<size_t>(kStages) * kStageBytes + 2 * kStages * sizeof(uint64_t) +
+         kXchFloats * sizeof(float) + 64 * sizeof(float2) + 4 * sizeof(int);
+}
+
+cudaError_t launch_decode(const DecodeParams& p, int grid, cudaStream_t stream) {
+  static int configured_device = -1;
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  if (configured_device != dev) {
+    e = cudaFuncSetAttribute(decode_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             static_cast<int>(decode_smem_bytes()));
+    if (e != cudaSuccess) return e;
+    configured_device = dev;
+  }
+  decode_kernel<<<grid, kThreads, decode_smem_bytes(), stream>>>(p);
+  return cudaGetLastError();
+}
+
+}  // namespace flint

@@ -1,0 +1,189 @@
+// flint_device.cuh -- device helpers: inline PTX for TMA, mbarriers,
+// ldmatrix and bf16 mma.sync, bounded waits, and the per-row Q/K norm+RoPE.
+#pragma once
+
+#include <cuda_bf16.h>
+#include <stdint.h>
+
+#include "flint_internal.h"
+
+namespace flint {
+
+// A pipeline wait gives up after this long (the whole decode step takes well
+// under a millisecond); the kernel then reports FLINT_ERR_TIMEOUT.
+constexpr unsigned long long kWaitLimitNs = 2000000000ull;
+
+__device__ __forceinline__ uint32_t smem_u32(const void* p) {
+  return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+}
+
+__device__ __forceinline__ unsigned long long globaltimer_ns() {
+  unsigned long long t;
+  asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+  return t;
+}
+
+__device__ __forceinline__ void report_error(int32_t* dev_err, int code) {
+  if (dev_err) atomicCAS(dev_err, 0, code);
+}
+
+// ---- mbarrier -------------------------------------------------------------
+
+__device__ __forceinline__ void mbar_init(uint32_t bar, uint32_t count) {
+  asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(bar), "r"(count) : "memory");
+}
+
+__device__ __forceinline__ void mbar_expect_tx(uint32_t bar, uint32_t bytes) {
+  asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(bar), "r"(bytes)
+               : "memory");
+}
+
+__device__ __forceinline__ void mbar_arrive(uint32_t bar) {
+  asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(bar) : "memory");
+}
+
+__device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(bar), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+
+// Wait for the phase with the given parity to complete.  Returns false if the
+// CTA's abort flag is raised or the time limit passes.
+__device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity,
+                                          const volatile int* abort_flag) {
+  if (mbar_try_wait(bar, parity)) return true;
+  const unsigned long long t0 = globaltimer_ns();
+  for (;;) {
+#pragma unroll 1
+    for (int i = 0; i < 32; ++i)
+      if (mbar_try_wait(bar, parity)) return true;
+    if (*abort_flag) return false;
+    if (globaltimer_ns() - t0 > kWaitLimitNs) return false;
+  }
+}
+
+// ---- TMA ------------------------------------------------------------------
+
+__device__ __forceinline__ void tma_load_4d(uint32_t dst, const CUtensorMap* map, uint32_t bar,
+                                            int c0, int c1, int c2, int c3) {
+  asm volatile(
+      "cp.async.bulk.tensor.4d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
+      " [%0], [%1, {%3, %4, %5, %6}], [%2];" ::"r"(dst),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(bar), "r"(c0), "r"(c1), "r"(c2), "r"(c3)
+      : "memory");
+}
+
+__device__ __forceinline__ void prefetch_tensormap(const CUtensorMap* map) {
+  asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(map)) : "memory");
+}
+
+// Order this thread's generic-proxy global writes before later async-proxy
+// (TMA) reads of the same addresses.
+__device__ __forceinline__ void fence_proxy_async_global() {
+  asm volatile("fence.proxy.async.global;" ::: "memory");
+}
+
+// ---- ldmatrix / mma.sync ---------------------------------------------------
+
+__device__ __forceinline__ void ldsm_x4(uint32_t addr, uint32_t& r0, uint32_t& r1, uint32_t& r2,
+                                        uint32_t& r3) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0,%1,%2,%3}, [%4];"
+               : "=r"(r0), "=r"(r1), "=r"(r2), "=r"(r3)
+               : "r"(addr));
+}
+
+__device__ __forceinline__ void ldsm_x4_t(uint32_t addr, uint32_t& r0, uint32_t& r1,
+                                          uint32_t& r2, uint32_t& r3) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0,%1,%2,%3}, [%4];"
+               : "=r"(r0), "=r"(r1), "=r"(r2), "=r"(r3)
+               : "r"(addr));
+}
+
+// D (16x8 fp32) += A (16x16 bf16, row) * B (16x8 bf16, col).
+__device__ __forceinline__ void mma_bf16_16816(float (&d)[4], const uint32_t (&a)[4], uint32_t b0,
+                                               uint32_t b1) {
+  asm("mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 "
+      "{%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, {%0,%1,%2,%3};"
+      : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+      : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
+}
+
+// ---- bf16 helpers ----------------------------------------------------------
+
+__device__ __forceinline__ float bf16_lo(uint32_t packed) {
+  return __uint_as_float(packed << 16);
+}
+__device__ __forceinline__ float bf16_hi(uint32_t packed) {
+  return __uint_as_float(packed & 0xffff0000u);
+}
+
+// Two floats -> packed bf16x2 (first in the low half), round to nearest even.
+__device__ __forceinline__ uint32_t pack_bf16x2(float a, float b) {
+  __nv_bfloat162 v = __floats2bfloat162_rn(a, b);
+  return *reinterpret_cast<uint32_t*>(&v);
+}
+
+// x = hi + lo with hi = bf16(x), lo = bf16(x - hi): a two-term bf16 split that
+// carries ~16 significant bits into a bf16 tensor-core product.
+__device__ __forceinline__ void split_bf16x2(float a, float b, uint32_t& hi, uint32_t& lo) {
+  __nv_bfloat162 h = __floats2bfloat162_rn(a, b);
+  float2 hf = __bfloat1622float2(h);
+  __nv_bfloat162 l = __floats2bfloat162_rn(a - hf.x, b - hf.y);
+  hi = *reinterpret_cast<uint32_t*>(&h);
+  lo = *reinterpret_cast<uint32_t*>(&l);
+}
+
+// ---- per-head RMSNorm (+RoPE) of one 128-wide row by one warp ---------------
+// Lane l holds dims (2l, 2l+1, 64+2l, 65+2l): RoPE pairs (i, i+64) stay in one
+// lane.  y = x * w / sqrt(mean(x^2) + eps), then for i < 64 the pair
+// (y_i, y_{i+64}) turns by the angle whose cos/sin are cs[i].
+__device__ __forceinline__ void norm_rope_row_warp(const uint16_t* __restrict__ x_row,
+                                                   const uint16_t* __restrict__ w, float eps,
+                                                   bool do_norm, bool rope, const float2* cs,
+                                                   int lane, float (&y)[4]) {
+  const uint32_t xa = reinterpret_cast<const uint32_t*>(x_row)[lane];
+  const uint32_t xb = reinterpret_cast<const uint32_t*>(x_row + 64)[lane];
+  y[0] = bf16_lo(xa);
+  y[1] = bf16_hi(xa);
+  y[2] = bf16_lo(xb);
+  y[3] = bf16_hi(xb);
+  if (do_norm) {
+    float ss = y[0] * y[0] + y[1] * y[1] + y[2] * y[2] + y[3] * y[3];
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
+    const float r = 1.0f / sqrtf(ss * (1.0f / kDim) + eps);
+    const uint32_t wa = reinterpret_cast<const uint32_t*>(w)[lane];
+    const uint32_t wb = reinterpret_cast<const uint32_t*>(w + 64)[lane];
+    y[0] = y[0] * r * bf16_lo(wa);
+    y[1] = y[1] * r * bf16_hi(wa);
+    y[2] = y[2] * r * bf16_lo(wb);
+    y[3] = y[3] * r * bf16_hi(wb);
+  }
+  if (rope) {
+#pragma unroll
+    for (int e = 0; e < 2; ++e) {
+      const float2 t = cs[2 * lane + e];
+      const float a = y[e], b = y[2 + e];
+      y[e] = a * t.x - b * t.y;
+      y[2 + e] = b * t.x + a * t.y;
+    }
+  }
+}
+
+// cos/sin of pos * theta^(-2i/128) for i < 64, angle formed and reduced in
+// double precision (an fp32 angle near position 1e5 would be off by ~1e-2 rad).
+__device__ __forceinline__ float2 rope_cos_sin(int i, int pos, double theta) {
+  const double inv_freq = pow(theta, -2.0 * i / kDim);
+  double s, c;
+  sincos(static_cast<double>(pos) * inv_freq, &s, &c);
+  return make_float2(static_cast<float>(c), static_cast<float>(s));
+}
+
+}  // namespace flint

@@ -1,0 +1,112 @@
+// flint_internal.h -- constants, kernel-parameter layout and launcher
+// declarations shared by the CUDA sources of libflint.so.
+#pragma once
+
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "../../include/flint.h"
+
+namespace flint {
+
+constexpr int kHeads = FLINT_NUM_Q_HEADS;     // 32 query heads
+constexpr int kKvHeads = FLINT_NUM_KV_HEADS;  // 4 KV heads
+constexpr int kDim = FLINT_HEAD_DIM;          // 128
+constexpr int kGroup = kHeads / kKvHeads;     // 8 query heads share a KV head
+constexpr int kWindow = FLINT_WINDOW;         // 513
+constexpr int kBlock = FLINT_BLOCK_SIZE;      // 64
+
+// Decode pipeline geometry.
+constexpr int kTile = 64;                     // tokens per pipeline stage
+constexpr int kHalfBytes = kTile * 64 * 2;    // one 64-dim half of a K or V tile: 8 KiB
+constexpr int kStageBytes = 4 * kHalfBytes;   // K lo/hi + V lo/hi: 32 KiB
+constexpr int kStages = 6;
+constexpr int kConsumerWarps = 4;
+constexpr int kThreads = (kConsumerWarps + 1) * 32;
+
+// Limits of one launch (bounded by the 32 KiB kernel-parameter space).
+constexpr int kMaxProblems = 64;
+constexpr int kMaxSegs = kMaxProblems * kKvHeads;
+constexpr int kMaxMaps = 2 * FLINT_MAX_LAYERS;
+constexpr int kMaxItems = 512;
+constexpr int kMaxCtas = 296;
+
+// One split partial: O [8][128], m [8], l [8] (fp32, m in log2 units).
+constexpr int kPartialFloats = kGroup * kDim + 2 * kGroup;
+constexpr size_t kCounterBytes = 4096;
+
+// One attention problem: one request of one layer.
+struct Problem {
+  const void* q;            // q (bf16 or fp32, normed) or q_raw (bf16) when prep
+  const uint16_t* k_raw;    // prep: bf16 [4][128]
+  const uint16_t* v_raw;    // prep: bf16 [4][128]
+  const uint16_t* w_q;      // prep: bf16 [128]
+  const uint16_t* w_k;      // prep: bf16 [128]
+  const float* sinks;       // fp32 [32]
+  float* out;               // fp32 [32][128]
+  uint16_t* k_rows;         // append target: this request's cache base (or the pool)
+  uint16_t* v_rows;
+  const int32_t* table;     // PAGED: this request's block-table row
+  int32_t lo, hi;           // attended tokens [lo, hi) in storage coordinates
+  int32_t tile_base;        // token of tile 0 (CONTIGUOUS/RING) or block index (PAGED)
+  int32_t append_tok;       // storage-coordinate token of the new token, or -1
+  int32_t pos;              // logical position of the new token (RoPE, paged append)
+  int32_t num_blocks;       // PAGED pool size
+  int16_t map_k, map_v;     // tensor-map indices
+  int16_t req;              // 4th tensor coordinate (request) for CONTIGUOUS/RING
+  int8_t layout, q_fp32, rope, pad;
+};
+
+struct Item {
+  int16_t seg;              // problem * 4 + kv head
+  int16_t t0, t1;           // tile range within the segment
+  int16_t pad;
+};
+
+struct DecodeParams {
+  CUtensorMap maps[kMaxMaps];
+  Problem prob[kMaxProblems];
+  Item items[kMaxItems];
+  int16_t cta_item_begin[kMaxCtas + 1];
+  int16_t seg_item_begin[kMaxSegs + 1];
+  int32_t* counters;        // workspace: per-segment arrival counters
+  float* partials;          // workspace: one partial per item
+  int32_t* dev_err;
+  double theta;
+  float eps;
+  int32_t n_problems;
+  int32_t prep;             // 1: q/k norm (+RoPE) and append fused in (layer stack)
+};
+
+static_assert(sizeof(DecodeParams) <= 32000, "kernel parameters exceed 32 KiB");
+
+struct PrepParams {
+  const uint16_t* q_raw;
+  const uint16_t* k_raw;
+  const uint16_t* v_raw;
+  const uint16_t* w_q;
+  const uint16_t* w_k;
+  float* q_out;
+  uint16_t* k_out;
+  // append target (k_rows == nullptr: no append)
+  uint16_t* k_rows;
+  uint16_t* v_rows;
+  const int32_t* table;
+  int64_t req_stride;
+  int32_t layout, capacity, max_blocks, num_blocks;
+  int32_t pos[kMaxProblems];
+  int32_t* dev_err;
+  double theta;
+  float eps;
+  int32_t apply_rope;
+  int32_t do_norm;          // 0: k is already final (plain append)
+};
+
+// Launchers (return cudaGetLastError() after the launch).
+cudaError_t launch_decode(const DecodeParams& p, int grid, cudaStream_t stream);
+cudaError_t launch_prep(const PrepParams& p, int B, cudaStream_t stream);
+
+size_t decode_smem_bytes();
+
+}  // namespace flint

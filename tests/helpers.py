@@ -1,0 +1,81 @@
+"""Shared pieces of the GPU parity tests: device copies of the seeded inputs,
+the parity bar, and oracle wrappers for the synthetic layers."""
+import numpy as np
+import torch
+
+import oracle
+from long_context_decode_flash_b200 import flint
+from long_context_decode_flash_b200 import inputs as I
+
+# Parity bar for fp32 outputs against the float64 oracle.
+MAX_ABS = 2e-3
+REL_L2 = 1e-3
+
+
+def dev(t: torch.Tensor) -> torch.Tensor:
+    return t.to("cuda", non_blocking=False).contiguous()
+
+
+def parity(got, want, what=""):
+    """Max-abs and relative-L2 bar over the whole output and per head."""
+    got = np.asarray(got, np.float64).reshape(-1, want.shape[-1])
+    want = np.asarray(want, np.float64).reshape(-1, want.shape[-1])
+    assert np.isfinite(got).all(), f"{what}: non-finite output"
+    err = np.abs(got - want)
+    rel = np.linalg.norm(got - want) / np.linalg.norm(want)
+    rel_head = np.linalg.norm(got - want, axis=1) / np.linalg.norm(want, axis=1)
+    assert err.max() <= MAX_ABS, f"{what}: max abs err {err.max():.3e}"
+    assert rel <= REL_L2, f"{what}: rel L2 err {rel:.3e}"
+    assert rel_head.max() <= REL_L2, f"{what}: worst head rel L2 {rel_head.max():.3e}"
+    return float(err.max()), float(rel)
+
+
+def bf16_ulp_diff(a_bits: np.ndarray, b_bits: np.ndarray) -> np.ndarray:
+    """|a - b| in bf16 ulps for finite bf16 bit patterns of the same sign."""
+    def ordered(x):
+        x = x.astype(np.int32)
+        return np.where(x & 0x8000, 0x8000 - (x & 0x7fff), 0x8000 + (x & 0x7fff))
+    return np.abs(ordered(a_bits) - ordered(b_bits))
+
+
+def oracle_layer(layer: I.Layer, nthreads: int = 0):
+    """Oracle for one synthetic layer: norm (+RoPE) -> append -> attend.
+    Returns (out f64 [32,128], k cache bits, v cache bits) after the append."""
+    kc = I.bits(layer.k_cache).copy()
+    vc = I.bits(layer.v_cache).copy()
+    out = oracle.decode_layer(I.bits(layer.q_raw), I.bits(layer.k_raw), I.bits(layer.v_raw),
+                              I.bits(layer.w_q), I.bits(layer.w_k),
+                              layer.sinks.numpy().astype(np.float64), kc, vc, layer.L,
+                              layer.window, layer.rope, layout=layer.layout,
+                              capacity=layer.capacity, nthreads=nthreads)
+    return out, kc, vc
+
+
+class DeviceLayer:
+    """Device copies of a synthetic layer, in the shape flint.stack_layers wants."""
+
+    def __init__(self, layer: I.Layer):
+        self.src = layer
+        self.q_raw = dev(layer.q_raw)
+        self.k_raw = dev(layer.k_raw)
+        self.v_raw = dev(layer.v_raw)
+        self.w_q = dev(layer.w_q)
+        self.w_k = dev(layer.w_k)
+        self.sinks = dev(layer.sinks)
+        self.k_cache = dev(layer.k_cache)
+        self.v_cache = dev(layer.v_cache)
+        self.window = layer.window
+        self.rope = layer.rope
+        self.cache = flint.kv_cache(self.k_cache, self.v_cache, layer.layout,
+                                    capacity=layer.capacity)
+
+
+def stack_on_gpu(layers, pos, num_ctas=0):
+    dl = [DeviceLayer(l) for l in layers]
+    out = torch.empty((len(dl), 32, 128), dtype=torch.float32, device="cuda")
+    ws = flint.workspace(len(dl), num_ctas)
+    err = torch.zeros(1, dtype=torch.int32, device="cuda")
+    flint.flint_attn_stack(dl, pos, out, ws, num_ctas=num_ctas, dev_err=err)
+    torch.cuda.synchronize()
+    assert int(err.item()) == 0, f"device error {int(err.item())}"
+    return out.cpu().numpy(), dl
