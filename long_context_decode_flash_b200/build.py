@@ -37,14 +37,19 @@ def up_to_date() -> bool:
     return all(os.path.getmtime(f) <= t for f in _inputs())
 
 
-def build(force: bool = False, verbose: bool = False, ptxas_info: bool = False) -> str:
-    if not force and up_to_date():
+def build(force: bool = False, verbose: bool = False, ptxas_info: bool = False,
+          debug_checks: bool = False) -> str:
+    """debug_checks compiles the kernels' self-checks in (bounds and alignment
+    checks that record the first failure in dev_err[2..7] and skip the access)."""
+    if not force and not debug_checks and up_to_date():
         return LIB
     tmp = LIB + f".{os.getpid()}.tmp"
     cmd = [nvcc(), "-O3", "-std=c++17", *ARCH, "-lineinfo", "-Xcompiler", "-fPIC", "-shared",
            "-I", os.path.join(ROOT, "include"), "-o", tmp]
     if ptxas_info:
         cmd += ["-Xptxas", "-v"]
+    if debug_checks:
+        cmd += ["-DFLINT_DEBUG_CHECKS"]
     cmd += [os.path.join(CSRC, s) for s in SOURCES]
     if verbose:
         print(" ".join(cmd), flush=True)
@@ -54,4 +59,5 @@ def build(force: bool = False, verbose: bool = False, ptxas_info: bool = False) 
 
 
 if __name__ == "__main__":
-    build(force="--force" in sys.argv, verbose=True, ptxas_info="--ptxas-info" in sys.argv)
+    build(force="--force" in sys.argv, verbose=True, ptxas_info="--ptxas-info" in sys.argv,
+          debug_checks="--debug-checks" in sys.argv)

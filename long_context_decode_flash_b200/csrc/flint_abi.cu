@@ -208,6 +208,7 @@ flint_status plan(DecodeParams& P, const int* tiles, int n_problems, int num_cta
     P.items[i].t1 = static_cast<int16_t>(t1[i]);
     P.items[i].pad = 0;
   }
+  P.n_items = n;
   int last = 0;  // CTAs past the last one with work are not launched
   for (int c = 0; c < G; ++c) {
     P.cta_item_begin[c] = static_cast<int16_t>(cb[c]);
@@ -390,6 +391,9 @@ flint_status flint_attn_decode(const void* q, int32_t q_is_fp32, const flint_kv_
     pb.append_tok = -1;
     pb.pos = seq_lens[b] - 1;
     pb.num_blocks = cache->num_blocks;
+    pb.ext2 = cache->layout == FLINT_KV_PAGED ? kBlock : cache->capacity;
+    pb.ext3 = cache->layout == FLINT_KV_PAGED ? cache->num_blocks : B;
+    pb.table_len = cache->layout == FLINT_KV_PAGED ? cache->max_blocks_per_req : 0;
     pb.map_k = 0;
     pb.map_v = 1;
     pb.req = static_cast<int16_t>(cache->layout == FLINT_KV_PAGED ? 0 : b);
@@ -407,6 +411,8 @@ flint_status flint_attn_decode(const void* q, int32_t q_is_fp32, const flint_kv_
   if (s != FLINT_OK) return s;
   s = encode_cache_map(&P.maps[1], cache->v, *cache, B);
   if (s != FLINT_OK) return s;
+  P.ws_items = static_cast<int32_t>(std::min<size_t>((ws_bytes - kCounterBytes) / (kPartialFloats * sizeof(float)), 1 << 30));
+  P.smem_bytes = static_cast<int32_t>(decode_smem_bytes());
   P.counters = static_cast<int32_t*>(workspace);
   P.partials = reinterpret_cast<float*>(static_cast<uint8_t*>(workspace) + kCounterBytes);
   P.dev_err = dev_err;
@@ -464,6 +470,9 @@ flint_status flint_attn_stack(const flint_layer* layers, int32_t n_layers, int32
     pb.pos = pos;
     pb.append_tok = ly.cache.layout == FLINT_KV_RING ? pos % ly.cache.capacity : pos;
     pb.num_blocks = ly.cache.num_blocks;
+    pb.ext2 = ly.cache.layout == FLINT_KV_PAGED ? kBlock : ly.cache.capacity;
+    pb.ext3 = ly.cache.layout == FLINT_KV_PAGED ? ly.cache.num_blocks : 1;
+    pb.table_len = ly.cache.layout == FLINT_KV_PAGED ? ly.cache.max_blocks_per_req : 0;
     pb.map_k = static_cast<int16_t>(2 * i);
     pb.map_v = static_cast<int16_t>(2 * i + 1);
     pb.req = 0;
@@ -482,6 +491,8 @@ flint_status flint_attn_stack(const flint_layer* layers, int32_t n_layers, int32
   if (ws_bytes < workspace_bytes(n_layers, grid))
     return fail(FLINT_ERR_WORKSPACE, "%s: workspace of %zu bytes is below the %zu needed", who, ws_bytes,
                 workspace_bytes(n_layers, grid));
+  P.ws_items = static_cast<int32_t>(std::min<size_t>((ws_bytes - kCounterBytes) / (kPartialFloats * sizeof(float)), 1 << 30));
+  P.smem_bytes = static_cast<int32_t>(decode_smem_bytes());
   P.counters = static_cast<int32_t*>(workspace);
   P.partials = reinterpret_cast<float*>(static_cast<uint8_t*>(workspace) + kCounterBytes);
   P.dev_err = dev_err;

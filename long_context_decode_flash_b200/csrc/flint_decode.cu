@@ -16,8 +16,9 @@
 //     maps, 128-byte swizzle) into a 6-stage ring of 32 KiB stages guarded by
 //     mbarriers.  In the fused layer-stack mode it also writes the new token's
 //     k (RMSNorm + RoPE) and v into the cache just before loading that tile.
-//   * Warps 0-3 consume tiles round-robin.  All 8 query heads of the group
-//     share every K/V tile: S^T = [q_hi; q_lo] K^T and O += [P_hi; P_lo] V run
+//   * Warps 0-3 each take a 16-token slice of every tile (so every warp waits
+//     on the stages' phases in order).  All 8 query heads of the group share
+//     every K/V tile: S^T = [q_hi; q_lo] K^T and O += [P_hi; P_lo] V run
 //     on bf16 mma.sync m16n8k16, where the 16 rows of A are the 8 heads' hi
 //     and lo bf16 parts (fp32 values split in two), so the products carry ~16
 //     significant bits while K/V stay exact bf16.  Softmax runs in fp32 in
@@ -110,6 +111,8 @@ __device__ void append_new_token(const DecodeParams& P, const Problem& pb, int g
 
 // Returns the number of tiles whose loads were issued.
 __device__ int run_producer(const DecodeParams& P, const Smem& S, int it0, int it1, int lane) {
+  int32_t* rec = P.dev_err;
+  (void)rec;
   int seq = 0;
   for (int it = it0; it < it1; ++it) {
     const Item item = P.items[it];
@@ -123,7 +126,8 @@ __device__ int run_producer(const DecodeParams& P, const Smem& S, int it0, int i
       const int n = min(32, item.t1 - t);
       int blk = 0;
       if (paged && lane < n) {
-        blk = __ldg(pb.table + pb.tile_base / kBlock + t + lane);
+        const int idx = pb.tile_base / kBlock + t + lane;
+        if (FLINT_CHECK(rec, idx >= 0 && idx < pb.table_len, 3, idx, pb.table_len, it)) blk = __ldg(pb.table + idx);
         // An out-of-range coordinate makes TMA fill zeros; flag it for the caller.
         if (blk < 0 || blk >= pb.num_blocks) report_error(P.dev_err, FLINT_ERR_INVALID_ARG);
       }
@@ -131,9 +135,8 @@ __device__ int run_producer(const DecodeParams& P, const Smem& S, int it0, int i
         const int b = __shfl_sync(0xffffffffu, blk, j);
         const int stage = seq % kStages;
         const uint32_t phase = static_cast<uint32_t>(seq / kStages) & 1u;
-        bool ok = true;
-        if (lane == 0) ok = mbar_wait(smem_u32(&S.empty[stage]), phase ^ 1u, S.flags);
-        ok = __shfl_sync(0xffffffffu, ok, 0);
+        bool ok = mbar_wait(smem_u32(&S.empty[stage]), phase ^ 1u, S.flags);
+        ok = __all_sync(0xffffffffu, ok);
         if (!ok) {
           if (lane == 0) abort_cta(P, S);
           return seq;
@@ -148,11 +151,18 @@ __device__ int run_producer(const DecodeParams& P, const Smem& S, int it0, int i
           const uint32_t dst = smem_u32(S.stages + stage * kStageBytes);
           const int c2 = paged ? 0 : pb.tile_base + tile * kTile;
           const int c3 = paged ? b : pb.req;
-          mbar_expect_tx(fb, kStageBytes);
-          tma_load_4d(dst, mk, fb, 0, g, c2, c3);
-          tma_load_4d(dst + kHalfBytes, mk, fb, 64, g, c2, c3);
-          tma_load_4d(dst + 2 * kHalfBytes, mv, fb, 0, g, c2, c3);
-          tma_load_4d(dst + 3 * kHalfBytes, mv, fb, 64, g, c2, c3);
+          bool fine = FLINT_CHECK(rec, (dst & 1023u) == 0 && dst + kStageBytes <= smem_u32(S.full), 6,
+                                  static_cast<int>(dst), stage, seq);
+          fine = fine && FLINT_CHECK(rec, c2 >= 0 && c2 < pb.ext2 && c3 >= 0 && c3 < pb.ext3, 5, c2, c3, it);
+          if (fine) {
+            mbar_expect_tx(fb, kStageBytes);
+            tma_load_4d(dst, mk, fb, 0, g, c2, c3);
+            tma_load_4d(dst + kHalfBytes, mk, fb, 64, g, c2, c3);
+            tma_load_4d(dst + 2 * kHalfBytes, mv, fb, 0, g, c2, c3);
+            tma_load_4d(dst + 3 * kHalfBytes, mv, fb, 64, g, c2, c3);
+          } else {
+            mbar_arrive(fb);  // complete the phase without data so nobody waits forever
+          }
         }
         __syncwarp();
       }
@@ -229,21 +239,23 @@ __device__ __forceinline__ void load_q(const DecodeParams& P, const Problem& pb,
   }
 }
 
-// One 64-token tile for this warp's 8 heads: online-softmax update of
-// (m_run, l_run, o).  tok0 is the storage token of the tile's first row.
-__device__ __forceinline__ void consume_tile(uint32_t sK, int tok0, int lo, int hi, int lane,
-                                             const uint32_t (&qa)[8][4], float& m_run,
-                                             float& l_run, float (&o)[16][4]) {
+// This warp's 16-token slice [tok0, tok0 + 16) of a 64-token tile, for the
+// 8 heads of the group: online-softmax update of (m_run, l_run, o).  sK is the
+// stage (K rows 0..63 in two swizzled 64-dim halves, then V likewise) and
+// r0 = 16 * warp is the slice's first row in it.
+__device__ __forceinline__ void consume_slice(uint32_t sK, int r0, int tok0, int lo, int hi,
+                                              int lane, const uint32_t (&qa)[8][4], float& m_run,
+                                              float& l_run, float (&o)[16][4]) {
   const int c = lane & 3;
   const int l7 = lane & 7;
-  const bool whole = (tok0 >= lo) && (tok0 + kTile <= hi);
+  const bool whole = (tok0 >= lo) && (tok0 + 16 <= hi);
 
-  // S^T = [q_hi; q_lo] * K^T: 8 n-tiles of 8 tokens, 8 k-steps of 16 dims.
-  float sc[16];
+  // S^T = [q_hi; q_lo] * K^T: 2 n-tiles of 8 tokens, 8 k-steps of 16 dims.
+  float sc[4];
 #pragma unroll
-  for (int j = 0; j < 8; ++j) {
+  for (int jj = 0; jj < 2; ++jj) {
     float acc[4] = {0.f, 0.f, 0.f, 0.f};
-    const uint32_t row = sK + (8 * j + l7) * 128;
+    const uint32_t row = sK + (r0 + 8 * jj + l7) * 128;
 #pragma unroll
     for (int kk = 0; kk < 8; kk += 2) {
       const int u = 2 * kk + (lane >> 3);  // 16-byte unit along the 128 dims
@@ -252,72 +264,64 @@ __device__ __forceinline__ void consume_tile(uint32_t sK, int tok0, int lo, int 
       mma_bf16_16816(acc, qa[kk], b0, b1);
       mma_bf16_16816(acc, qa[kk + 1], b2, b3);
     }
-    sc[2 * j] = acc[0] + acc[2];
-    sc[2 * j + 1] = acc[1] + acc[3];
+    sc[2 * jj] = acc[0] + acc[2];  // token tok0 + 8jj + 2c (+1)
+    sc[2 * jj + 1] = acc[1] + acc[3];
   }
   if (!whole) {
 #pragma unroll
-    for (int j = 0; j < 8; ++j)
-#pragma unroll
-      for (int e = 0; e < 2; ++e) {
-        const int tok = tok0 + 8 * j + 2 * c + e;
-        if (tok < lo || tok >= hi) sc[2 * j + e] = -INFINITY;
-      }
+    for (int i = 0; i < 4; ++i) {
+      const int tok = tok0 + 8 * (i >> 1) + 2 * c + (i & 1);
+      if (tok < lo || tok >= hi) sc[i] = -INFINITY;
+    }
   }
 
-  float mx = sc[0];
-#pragma unroll
-  for (int i = 1; i < 16; ++i) mx = fmaxf(mx, sc[i]);
+  float mx = fmaxf(fmaxf(sc[0], sc[1]), fmaxf(sc[2], sc[3]));
   mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 1));
   mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 2));
-  if (mx > m_run + kRescaleSlack) {  // also taken on the first valid tile
-    const float alpha = exp2f(m_run - mx);
+  // The running max moves only when a head's max grows by more than the
+  // slack (always on its first valid slice); the branch is warp-uniform.
+  const bool grow = mx > m_run + kRescaleSlack;
+  if (__any_sync(0xffffffffu, grow)) {
+    const float alpha = grow ? exp2f(m_run - mx) : 1.0f;
     l_run *= alpha;
 #pragma unroll
     for (int n = 0; n < 16; ++n)
 #pragma unroll
       for (int e = 0; e < 4; ++e) o[n][e] *= alpha;
-    m_run = mx;
+    if (grow) m_run = mx;
   }
   const float mu = (m_run == -INFINITY) ? 0.f : m_run;
 
-  // P = 2^(s - m) split into bf16 hi/lo rows of the A operand.
-  uint32_t pa[4][4];
-#pragma unroll
-  for (int ks = 0; ks < 4; ++ks) {
-    const float p0 = exp2f(sc[4 * ks] - mu), p1 = exp2f(sc[4 * ks + 1] - mu);
-    const float p2 = exp2f(sc[4 * ks + 2] - mu), p3 = exp2f(sc[4 * ks + 3] - mu);
-    l_run += (p0 + p1) + (p2 + p3);
-    split_bf16x2(p0, p1, pa[ks][0], pa[ks][1]);
-    split_bf16x2(p2, p3, pa[ks][2], pa[ks][3]);
-  }
+  // P = 2^(s - m) split into the bf16 hi/lo rows of the A operand.
+  const float p0 = exp2f(sc[0] - mu), p1 = exp2f(sc[1] - mu);
+  const float p2 = exp2f(sc[2] - mu), p3 = exp2f(sc[3] - mu);
+  l_run += (p0 + p1) + (p2 + p3);
+  uint32_t pa[4];
+  split_bf16x2(p0, p1, pa[0], pa[1]);
+  split_bf16x2(p2, p3, pa[2], pa[3]);
 
-  // O += [P_hi; P_lo] * V: 4 k-steps of 16 tokens, 16 n-tiles of 8 dims.
-  const uint32_t sV = sK + 2 * kHalfBytes;
+  // O += [P_hi; P_lo] * V: one k-step of 16 tokens, 16 n-tiles of 8 dims.
+  uint32_t m01 = 0xffffffffu, m23 = 0xffffffffu;
+  if (!whole) {
+    const int t = tok0 + 2 * c;
+    m01 = ((t >= lo && t < hi) ? 0x0000ffffu : 0u) | ((t + 1 >= lo && t + 1 < hi) ? 0xffff0000u : 0u);
+    m23 = ((t + 8 >= lo && t + 8 < hi) ? 0x0000ffffu : 0u) |
+          ((t + 9 >= lo && t + 9 < hi) ? 0xffff0000u : 0u);
+  }
+  const uint32_t row = sK + 2 * kHalfBytes + (r0 + ((lane >> 3) & 1) * 8 + l7) * 128;
 #pragma unroll
-  for (int ks = 0; ks < 4; ++ks) {
-    uint32_t m01 = 0xffffffffu, m23 = 0xffffffffu;
-    if (!whole) {
-      const int t = tok0 + 16 * ks + 2 * c;
-      m01 = ((t >= lo && t < hi) ? 0x0000ffffu : 0u) | ((t + 1 >= lo && t + 1 < hi) ? 0xffff0000u : 0u);
-      m23 = ((t + 8 >= lo && t + 8 < hi) ? 0x0000ffffu : 0u) |
-            ((t + 9 >= lo && t + 9 < hi) ? 0xffff0000u : 0u);
+  for (int np = 0; np < 8; ++np) {
+    const int nt = 2 * np + (lane >> 4);
+    uint32_t v0, v1, v2, v3;
+    ldsm_x4_t(row + (nt >> 3) * kHalfBytes + (((nt & 7) ^ l7) << 4), v0, v1, v2, v3);
+    if (!whole) {  // rows outside the range may hold anything (even NaN)
+      v0 &= m01;
+      v2 &= m01;
+      v1 &= m23;
+      v3 &= m23;
     }
-    const uint32_t row = sV + (16 * ks + ((lane >> 3) & 1) * 8 + l7) * 128;
-#pragma unroll
-    for (int np = 0; np < 8; ++np) {
-      const int nt = 2 * np + (lane >> 4);
-      uint32_t v0, v1, v2, v3;
-      ldsm_x4_t(row + (nt >> 3) * kHalfBytes + (((nt & 7) ^ l7) << 4), v0, v1, v2, v3);
-      if (!whole) {  // rows outside the range may hold anything (even NaN)
-        v0 &= m01;
-        v2 &= m01;
-        v1 &= m23;
-        v3 &= m23;
-      }
-      mma_bf16_16816(o[2 * np], pa[ks], v0, v1);
-      mma_bf16_16816(o[2 * np + 1], pa[ks], v2, v3);
-    }
+    mma_bf16_16816(o[2 * np], pa, v0, v1);
+    mma_bf16_16816(o[2 * np + 1], pa, v2, v3);
   }
 }
 
@@ -355,21 +359,22 @@ __device__ void run_consumer(const DecodeParams& P, const Smem& S, int it0, int 
 #pragma unroll
       for (int e = 0; e < 4; ++e) o[n][e] = 0.f;
 
+    // Every consumer warp takes part in every tile (its own 16-token slice),
+    // so each warp waits on the stages' phases strictly in order.
     const int ntiles = item.t1 - item.t0;
     for (int k = 0; k < ntiles; ++k, ++seq) {
-      if (seq % kConsumerWarps != warp) continue;
       const int stage = seq % kStages;
       const uint32_t phase = static_cast<uint32_t>(seq / kStages) & 1u;
-      bool ok = true;
-      if (lane == 0) ok = mbar_wait(smem_u32(&S.full[stage]), phase, S.flags);
-      ok = __shfl_sync(0xffffffffu, ok, 0);
+      // every lane observes the phase completion (acquire) before reading the stage
+      bool ok = mbar_wait(smem_u32(&S.full[stage]), phase, S.flags);
+      ok = __all_sync(0xffffffffu, ok);
       if (!ok) {
         if (lane == 0) abort_cta(P, S);
         continue;  // keep walking so that every warp meets the same barriers
       }
-      const int tok0 = pb.tile_base + (item.t0 + k) * kTile;
-      consume_tile(smem_u32(S.stages + stage * kStageBytes), tok0, pb.lo, pb.hi, lane, qa, m_run,
-                   l_run, o);
+      const int tok0 = pb.tile_base + (item.t0 + k) * kTile + 16 * warp;
+      consume_slice(smem_u32(S.stages + stage * kStageBytes), 16 * warp, tok0, pb.lo, pb.hi, lane, qa,
+                    m_run, l_run, o);
       __syncwarp();
       if (lane == 0) mbar_arrive(smem_u32(&S.empty[stage]));
     }
@@ -385,6 +390,7 @@ __device__ void run_consumer(const DecodeParams& P, const Smem& S, int it0, int 
       xw[kDim] = m_run;
       xw[kDim + 1] = l_run;
     }
+    __syncwarp();
     consumer_bar();
 
     float M = -INFINITY;
@@ -407,19 +413,25 @@ __device__ void run_consumer(const DecodeParams& P, const Smem& S, int it0, int 
       finish_head(pb, kvh, hh, d0, M, L, acc);
     } else {
       float* part = P.partials + static_cast<size_t>(it) * kPartialFloats;
-      float4* pd = reinterpret_cast<float4*>(part + hh * kDim + d0);
-      pd[0] = make_float4(acc[0], acc[1], acc[2], acc[3]);
-      pd[1] = make_float4(acc[4], acc[5], acc[6], acc[7]);
-      if ((t & 15) == 0) {
-        part[kGroup * kDim + hh] = M;
-        part[kGroup * kDim + kGroup + hh] = L;
+      if (FLINT_CHECK(P.dev_err, it < P.ws_items && s0 >= 0 && s1 <= P.n_items, 7, it, s0, s1)) {
+        float4* pd = reinterpret_cast<float4*>(part + hh * kDim + d0);
+        pd[0] = make_float4(acc[0], acc[1], acc[2], acc[3]);
+        pd[1] = make_float4(acc[4], acc[5], acc[6], acc[7]);
+        if ((t & 15) == 0) {
+          part[kGroup * kDim + hh] = M;
+          part[kGroup * kDim + kGroup + hh] = L;
+        }
       }
       __threadfence();
+      __syncwarp();
       consumer_bar();
       if (t == 0) {
-        const int prev = atomicAdd(P.counters + seg, 1);
+        int prev = 0;
+        if (FLINT_CHECK(P.dev_err, seg >= 0 && seg < kMaxSegs, 8, seg, 0, 0))
+          prev = atomicAdd(P.counters + seg, 1);
         S.flags[1] = (prev == s1 - s0 - 1) ? 1 : 0;
       }
+      __syncwarp();
       consumer_bar();
       if (S.flags[1]) {
         // last arrival: merge every partial of the segment, in item order
@@ -442,6 +454,7 @@ __device__ void run_consumer(const DecodeParams& P, const Smem& S, int it0, int 
         if (t == 0) P.counters[seg] = 0;  // ready for the next call
       }
     }
+    __syncwarp();
     consumer_bar();  // the exchange area and flags[1] are reused by the next item
   }
 }
@@ -450,12 +463,16 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const __grid_consta
   extern __shared__ uint8_t smem_raw[];
   const Smem S = carve(smem_raw);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int it0 = P.cta_item_begin[blockIdx.x], it1 = P.cta_item_begin[blockIdx.x + 1];
+  int it0 = P.cta_item_begin[blockIdx.x], it1 = P.cta_item_begin[blockIdx.x + 1];
+  if (!FLINT_CHECK(P.dev_err, 0 <= it0 && it0 <= it1 && it1 <= P.n_items, 1, it0, it1, P.n_items)) it1 = it0;
+  const int smem_end = static_cast<int>(smem_u32(const_cast<int*>(S.flags) + 4) - smem_u32(smem_raw));
+  if (!FLINT_CHECK(P.dev_err, smem_end <= P.smem_bytes, 2, smem_end, P.smem_bytes, 0)) it1 = it0;
+  (void)smem_end;
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < kStages; ++s) {
       mbar_init(smem_u32(&S.full[s]), 1);
-      mbar_init(smem_u32(&S.empty[s]), 1);
+      mbar_init(smem_u32(&S.empty[s]), kConsumerWarps);
     }
     S.flags[0] = 0;
     S.flags[1] = 0;

@@ -27,6 +27,25 @@ __device__ __forceinline__ void report_error(int32_t* dev_err, int code) {
   if (dev_err) atomicCAS(dev_err, 0, code);
 }
 
+// ---- self-checks (FLINT_DEBUG_CHECKS builds only) ---------------------------
+// A failed check records (code, block, thread, a, b, c) in dev_err[2..7] once
+// and the caller skips the access; release builds compile the checks away.
+#ifdef FLINT_DEBUG_CHECKS
+static __device__ __noinline__ void debug_record(int32_t* rec, int code, int a, int b, int c) {
+  if (rec && atomicCAS(rec + 2, 0, code) == 0) {
+    rec[3] = blockIdx.x;
+    rec[4] = threadIdx.x;
+    rec[5] = a;
+    rec[6] = b;
+    rec[7] = c;
+  }
+}
+#define FLINT_CHECK(rec, cond, code, a, b, c) \
+  ((cond) ? true : (::flint::debug_record((rec), (code), (a), (b), (c)), false))
+#else
+#define FLINT_CHECK(rec, cond, code, a, b, c) true
+#endif
+
 // ---- mbarrier -------------------------------------------------------------
 
 __device__ __forceinline__ void mbar_init(uint32_t bar, uint32_t count) {

@@ -53,6 +53,8 @@ struct Problem {
   int32_t append_tok;       // storage-coordinate token of the new token, or -1
   int32_t pos;              // logical position of the new token (RoPE, paged append)
   int32_t num_blocks;       // PAGED pool size
+  int32_t ext2, ext3;       // tensor extents along tokens and requests/blocks
+  int32_t table_len;        // PAGED: entries in this request's block-table row
   int16_t map_k, map_v;     // tensor-map indices
   int16_t req;              // 4th tensor coordinate (request) for CONTIGUOUS/RING
   int8_t layout, q_fp32, rope, pad;
@@ -72,11 +74,14 @@ struct DecodeParams {
   int16_t seg_item_begin[kMaxSegs + 1];
   int32_t* counters;        // workspace: per-segment arrival counters
   float* partials;          // workspace: one partial per item
-  int32_t* dev_err;
+  int32_t* dev_err;         // [0] status; debug builds also record a failed check in [2..7]
   double theta;
   float eps;
   int32_t n_problems;
   int32_t prep;             // 1: q/k norm (+RoPE) and append fused in (layer stack)
+  int32_t n_items;          // items in the plan
+  int32_t ws_items;         // partial slots in the workspace
+  int32_t smem_bytes;       // dynamic shared memory of the launch
 };
 
 static_assert(sizeof(DecodeParams) <= 32000, "kernel parameters exceed 32 KiB");
