@@ -37,10 +37,12 @@ FALLBACK_HBM_GBS = 6650.0
 def parse():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=50)
-    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--warmup", type=int, default=10)
     ap.add_argument("--impl", default="flint", choices=["flint", "reference"])
     ap.add_argument("--workload", default="stack", choices=["stack", "full100k", "swa100k", "paged32"])
+    ap.add_argument("--context", type=int, default=100_000,
+                    help="context length (the benchmark's figure is 100,000; smaller ones serve profiling)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     return ap.parse_args()
@@ -56,15 +58,20 @@ def measured_peak():
 
 # ------------------------------------------------------------ CPU oracle ---
 
-def oracle_sample(layers_full, layers_window, nthreads):
-    """Time the oracle on some layers of the stack; returns (us per token for
-    the 14+35 stack, seconds spent, description)."""
+def oracle_sample(layers_full, layers_window, nthreads, budget_s=10.0):
+    """Time the oracle on layers of the stack, repeating full layers for about
+    80% and window layers for about 20% of budget_s; returns (us per token
+    scaled to 14 full + 35 window layers, seconds spent, description)."""
     import numpy as np
     import oracle
     from long_context_decode_flash_b200 import inputs as I
 
+    caches = {}
+
     def one(lay):
-        kc, vc = I.bits(lay.k_cache).copy(), I.bits(lay.v_cache).copy()
+        if id(lay) not in caches:   # appending again at the same position is idempotent
+            caches[id(lay)] = (I.bits(lay.k_cache).copy(), I.bits(lay.v_cache).copy())
+        kc, vc = caches[id(lay)]
         t0 = time.perf_counter()
         oracle.decode_layer(I.bits(lay.q_raw), I.bits(lay.k_raw), I.bits(lay.v_raw),
                             I.bits(lay.w_q), I.bits(lay.w_k), lay.sinks.numpy().astype(np.float64),
@@ -72,13 +79,17 @@ def oracle_sample(layers_full, layers_window, nthreads):
                             capacity=lay.capacity, nthreads=nthreads)
         return time.perf_counter() - t0
 
-    tf = [one(l) for l in layers_full]
-    tw = [one(l) for l in layers_window]
-    per_full = sum(tf) / len(tf)
-    per_win = sum(tw) / len(tw)
-    us = (14 * per_full + 35 * per_win) * 1e6
-    desc = (f"{len(layers_full)} full layer(s) + {len(layers_window)} window layer(s) of the "
-            f"stack at context {CONTEXT}, all 32 heads, scaled to 14 + 35 layers")
+    def repeat(layers, budget):
+        times, t_end = [], time.perf_counter() + budget
+        while not times or time.perf_counter() < t_end:
+            times.append(one(layers[len(times) % len(layers)]))
+        return times
+
+    tf = repeat(layers_full, 0.8 * budget_s)
+    tw = repeat(layers_window, 0.2 * budget_s)
+    us = (14 * statistics.mean(tf) + 35 * statistics.mean(tw)) * 1e6
+    desc = (f"{len(tf)} full-layer and {len(tw)} window-layer oracle runs (context {CONTEXT}, "
+            f"all 32 heads, norm+RoPE+append+attend), mean times scaled to 14 + 35 layers")
     return us, sum(tf) + sum(tw), desc
 
 
@@ -95,12 +106,14 @@ def run_reference(args, rank):
     full_i = kinds.index(True)
     layers_full = [I.make_layer(I.W_STACK_100K, full_i, CONTEXT, 0, False, ring=False)]
     layers_win = [I.make_layer(I.W_STACK_100K, 0, CONTEXT, 513, True, ring=True)]
-    for _ in range(args.warmup):
-        oracle_sample(layers_full, layers_win[:1], nthreads)
-    vals = [oracle_sample(layers_full, layers_win, nthreads)[0] for _ in range(args.steps)]
+    oracle_sample(layers_full, layers_win, nthreads, budget_s=1.0)  # warm-up
+    # each step is a bounded sample; the whole run stays within a few minutes
+    budget = max(2.0, min(20.0, 120.0 / max(1, args.steps)))
+    vals = []
+    for _ in range(args.steps):
+        us_step, _, sample = oracle_sample(layers_full, layers_win, nthreads, budget_s=budget)
+        vals.append(us_step)
     us = statistics.mean(vals)
-    sample = (f"per step: 1 full layer + 1 window layer of the stack at context {CONTEXT}, "
-              f"all heads, scaled to 14 + 35 layers")
     line = {
         "impl": "reference", "metric": METRIC, "value": us, "unit": "us/token",
         "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
@@ -133,50 +146,63 @@ def workload_config(name):
 
 
 class ClockSampler:
-    """nvidia-smi samples during the timed region."""
+    """SM clock, power and throttle reasons sampled through NVML (about every
+    millisecond) while the timed region runs."""
 
-    def __init__(self, index):
-        self.index = index
-        self.rows = []
-        self.proc = None
+    REASONS = (("hw_slowdown", 0x8), ("hw_thermal_slowdown", 0x40),
+               ("sw_thermal_slowdown", 0x20), ("sw_power_cap", 0x4),
+               ("hw_power_brake_slowdown", 0x80))
+
+    def __init__(self, torch_device):
+        self.dev = torch_device
+        self.samples = []
+        self.stop = threading.Event()
+        self.handle = None
+        self.max_mhz = None
 
     def __enter__(self):
-        q = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.hw_slowdown,"
-             "clocks_event_reasons.hw_thermal_slowdown,clocks_event_reasons.sw_thermal_slowdown,"
-             "clocks_event_reasons.sw_power_cap")
         try:
-            self.proc = subprocess.Popen(
-                ["nvidia-smi", "-i", str(self.index), f"--query-gpu={q}", "--format=csv,noheader,nounits",
-                 "-lms", "100"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
-            self.thread = threading.Thread(target=self._read, daemon=True)
+            import pynvml
+            import torch
+            pynvml.nvmlInit()
+            p = torch.cuda.get_device_properties(self.dev)
+            bus = f"{p.pci_domain_id:08X}:{p.pci_bus_id:02X}:{p.pci_device_id:02X}.0"
+            try:
+                self.handle = pynvml.nvmlDeviceGetHandleByPciBusId(bus)
+            except Exception:
+                self.handle = pynvml.nvmlDeviceGetHandleByIndex(self.dev)
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self.handle, pynvml.NVML_CLOCK_SM)
+            self.nvml = pynvml
+            self.thread = threading.Thread(target=self._run, daemon=True)
             self.thread.start()
         except Exception:
-            self.proc = None
+            self.handle = None
         return self
 
-    def _read(self):
-        for line in self.proc.stdout:
-            parts = [p.strip() for p in line.split(",")]
-            if len(parts) == 7:
-                self.rows.append(parts)
+    def _run(self):
+        n = self.nvml
+        while not self.stop.is_set():
+            try:
+                sm = n.nvmlDeviceGetClockInfo(self.handle, n.NVML_CLOCK_SM)
+                reasons = n.nvmlDeviceGetCurrentClocksEventReasons(self.handle)
+                power = n.nvmlDeviceGetPowerUsage(self.handle) / 1000.0
+                self.samples.append((sm, reasons, power))
+            except Exception:
+                pass
+            time.sleep(0.001)
 
     def __exit__(self, *exc):
-        if self.proc:
-            self.proc.terminate()
-            try:
-                self.proc.wait(timeout=5)
-            except Exception:
-                self.proc.kill()
+        self.stop.set()
+        if self.handle is not None:
+            self.thread.join(timeout=2)
 
     def summary(self):
-        if not self.rows:
-            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unsampled"]}
-        sm = [float(r[0]) for r in self.rows if r[0].replace(".", "").isdigit()]
-        mx = [float(r[1]) for r in self.rows if r[1].replace(".", "").isdigit()]
-        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
-        reasons = sorted({n for r in self.rows for n, v in zip(names, r[3:]) if v == "Active"})
-        return {"sm_mhz": statistics.median(sm) if sm else None,
-                "sm_max_mhz": max(mx) if mx else None, "reasons": reasons, "samples": len(self.rows)}
+        if not self.samples:
+            return {"sm_mhz": None, "sm_max_mhz": self.max_mhz, "reasons": ["unsampled"], "samples": 0}
+        reasons = sorted({name for _, r, _ in self.samples for name, bit in self.REASONS if r & bit})
+        return {"sm_mhz": statistics.median(s for s, _, _ in self.samples), "sm_max_mhz": self.max_mhz,
+                "reasons": reasons, "samples": len(self.samples),
+                "power_w_max": max(p for _, _, p in self.samples), "source": "NVML, ~1 ms"}
 
 
 def build_stack_device(torch, flint, I, layers):
@@ -224,29 +250,30 @@ def main():
     from long_context_decode_flash_b200 import inputs as I
 
     # Host inputs first; the CPU baseline runs before any CUDA call.
+    ctx = args.context
     if args.workload == "stack":
-        layers = I.make_stack(CONTEXT)
-        algo_bytes = flint.flint_kv_bytes(CONTEXT)
+        layers = I.make_stack(ctx)
+        algo_bytes = flint.flint_kv_bytes(ctx)
     elif args.workload == "full100k":
-        layers = [I.make_layer(I.W_FULL_100K, 0, CONTEXT, 0, False, ring=False)]
-        algo_bytes = CONTEXT * 2048
+        layers = [I.make_layer(I.W_FULL_100K, 0, ctx, 0, False, ring=False)]
+        algo_bytes = ctx * 2048
     elif args.workload == "swa100k":
-        layers = [I.make_layer(I.W_SWA_100K, 0, CONTEXT, 513, True, ring=True)]
-        algo_bytes = 513 * 2048
+        layers = [I.make_layer(I.W_SWA_100K, 0, ctx, 513, True, ring=True)]
+        algo_bytes = min(ctx, 513) * 2048
     else:
         layers = None
         pb = I.make_paged_batch()
         algo_bytes = sum(pb.seq_lens) * 2048
 
     cpu_baseline = None
-    if rank == 0 and world == 1 and args.workload == "stack" and not args.no_cpu_baseline:
+    if rank == 0 and world == 1 and args.workload == "stack" and ctx == CONTEXT and not args.no_cpu_baseline:
         import oracle
         oracle.build()
         kinds = I.layer_kinds()
         full = [layers[kinds.index(True)]]
         win = [layers[0], layers[1]]
         nthreads = os.cpu_count() or 1
-        us, spent, desc = oracle_sample(full, win, nthreads)
+        us, spent, desc = oracle_sample(full, win, nthreads, budget_s=10.0)
         cpu_baseline = {"value": us, "unit": "us/token", "cores": nthreads, "kind": "oracle",
                         "sample": desc + f" ({spent:.1f} s of CPU wall time)"}
 
@@ -261,7 +288,7 @@ def main():
 
     if layers is not None:
         dls, packed, host_in = build_stack_device(torch, flint, I, layers)
-        pos = CONTEXT - 1
+        pos = ctx - 1
         out = torch.empty((len(dls), 32, 128), dtype=torch.float32, device="cuda")
         ws = flint.workspace(len(dls))
         arr = flint.stack_layers(dls)
@@ -350,7 +377,7 @@ def main():
         "n_gpus": world, "steps": args.steps, "warmup": max(args.warmup, 3),
         "ms_per_step": ms, "higher_is_better": False, "scaling": "weak", "vs_baseline": None,
         "dtype": "bf16", "data": "synthetic (seeded bf16 N(0,1) q/k/v/KV, N(0,1) sinks, 1+N(0,0.1) norm weights)",
-        "config": dict(workload_config(args.workload), parallelism=f"replicas x{world}"),
+        "config": dict(workload_config(args.workload), context=ctx, parallelism=f"replicas x{world}"),
         "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
                      "frac": achieved / peak, "peak_kind": peak_kind,
                      "frac_of_nominal_8000": achieved / NOMINAL_HBM_GBS,

@@ -104,7 +104,8 @@ flint_status encode_cache_map(CUtensorMap* map, void* base, const flint_kv_cache
   const cuuint32_t estr[4] = {1, 1, 1, 1};
   CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, base, dims, strides, box, estr,
                   CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
-                  CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+                  static_cast<CUtensorMapL2promotion>(FLINT_L2_PROMOTION),
+                  CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   if (r != CUDA_SUCCESS) return fail(FLINT_ERR_CUDA, "cuTensorMapEncodeTiled failed (CUresult %d)", (int)r);
   return FLINT_OK;
 }
@@ -156,7 +157,8 @@ Range attended_range(const flint_kv_cache& c, int L, int window) {
   } else {
     r.lo = window > 0 ? std::max(0, L - window) : 0;
     r.hi = L;
-    r.tile_base = c.layout == FLINT_KV_PAGED ? (r.lo / kBlock) * kBlock : r.lo;
+    // paged tiles must not straddle a block: start them on a multiple of kTile
+    r.tile_base = c.layout == FLINT_KV_PAGED ? (r.lo / kTile) * kTile : r.lo;
   }
   r.tiles = (r.hi - r.tile_base + kTile - 1) / kTile;
   return r;
@@ -179,7 +181,7 @@ flint_status check_len(const flint_kv_cache& c, int L, int window, const char* w
 }
 
 size_t workspace_bytes(int n_problems, int num_ctas) {
-  const int64_t items = std::min<int64_t>(kMaxItems, num_ctas + static_cast<int64_t>(n_problems) * kKvHeads);
+  const int64_t items = std::min<int64_t>(kMaxItems, num_ctas + static_cast<int64_t>(n_problems));
   return kCounterBytes + static_cast<size_t>(items) * kPartialFloats * sizeof(float);
 }
 
@@ -191,12 +193,11 @@ flint_status plan(DecodeParams& P, const int* tiles, int n_problems, int num_cta
   sms = std::min(sms, kMaxCtas);
   int32_t seg_tiles[kMaxSegs];
   int64_t total = 0;
-  for (int p = 0; p < n_problems; ++p)
-    for (int g = 0; g < kKvHeads; ++g) {
-      seg_tiles[p * kKvHeads + g] = tiles[p];
-      total += tiles[p];
-    }
-  const int n_segs = n_problems * kKvHeads;
+  for (int p = 0; p < n_problems; ++p) {
+    seg_tiles[p] = tiles[p];
+    total += tiles[p];
+  }
+  const int n_segs = n_problems;
   // at least two tiles of work per CTA, never more CTAs than the device's SMs
   const int G = static_cast<int>(std::max<int64_t>(1, std::min<int64_t>(sms, (total + 1) / 2)));
   int32_t seg[kMaxItems], t0[kMaxItems], t1[kMaxItems], cb[kMaxCtas + 1];

@@ -9,26 +9,31 @@
 //     s_j = q_h . K_j / sqrt(128),  M = max(max_j s_j, sink_h).
 //
 // How (one persistent launch for every problem of the call):
-//   * The host cuts each (problem, KV head) token range into 64-token tiles and
-//     lays the tiles over one CTA per SM (split-KV); each CTA walks its list
-//     of items (segment, tile range).
-//   * Warp 4 is the producer: it streams K and V tiles with TMA (4-D tensor
-//     maps, 128-byte swizzle) into a 6-stage ring of 32 KiB stages guarded by
-//     mbarriers.  In the fused layer-stack mode it also writes the new token's
-//     k (RMSNorm + RoPE) and v into the cache just before loading that tile.
-//   * Warps 0-3 each take a 16-token slice of every tile (so every warp waits
-//     on the stages' phases in order).  All 8 query heads of the group share
-//     every K/V tile: S^T = [q_hi; q_lo] K^T and O += [P_hi; P_lo] V run
-//     on bf16 mma.sync m16n8k16, where the 16 rows of A are the 8 heads' hi
-//     and lo bf16 parts (fp32 values split in two), so the products carry ~16
-//     significant bits while K/V stay exact bf16.  Softmax runs in fp32 in
-//     log2 units with quad shuffles; the running max is only moved when it
-//     grows by more than 2^8, so rescales are rare.
-//   * Item end: the four warps' (m, l, O) merge in shared memory.  A segment
-//     covered by one item is finished on the spot (sink folded in); otherwise
-//     the CTA stores a partial and the last CTA to arrive (atomic counter, no
-//     spinning) merges all partials of the segment in a fixed order and folds
-//     in the sink, so results are deterministic.
+//   * The host cuts each problem's token range into 16-token tiles and lays
+//     the tiles of all problems over one CTA per SM (split-KV); each CTA walks
+//     its list of items (problem, tile range).
+//   * The last warp is the producer: per 32-token tile it loads K and V of all
+//     four KV heads with 16 TMA boxes (4-D tensor maps, 128-byte swizzle,
+//     issued by lanes 0-15) into a 3-stage ring of 64 KiB stages guarded by
+//     mbarriers, so the CTA reads whole 1 KiB token rows of the cache.  In the fused layer-stack
+//     mode it first writes the new token's k (RMSNorm + RoPE) and v into the
+//     cache, just before loading the tile that holds it.
+//   * Consumer warps come in two groups of four; warp w of a group serves KV
+//     head w and its 8 query heads, group q on the q-th 16-token half of
+//     every tile, so every warp waits on every stage's phases in order (two
+//     consumer warps per scheduler hide the MMA/softmax latency).  At an
+//     item's end group 1 hands its state to group 0 through shared memory.
+//     S^T = [q_hi; q_lo] K^T and O += [P_hi; P_lo] V run on bf16 mma.sync
+//     m16n8k16, where the 16 rows of A are the 8 heads' hi and lo bf16 parts
+//     (fp32 values split in two): the products carry ~16 significant bits
+//     while K/V stay exact bf16.  Softmax runs in fp32 in log2 units with
+//     quad shuffles; the running max moves only when it grows by more than 8
+//     (warp-uniform branch), so rescales are rare.
+//   * Item end: a problem covered by one item is finished on the spot (sink
+//     folded in); otherwise the CTA stores a partial (m, l, O for 32 heads)
+//     and the last CTA to arrive (atomic counter, no spinning) merges all
+//     partials of the problem in item order and folds in the sinks, so
+//     results are deterministic.
 // Every mbarrier wait is bounded in time; on timeout the kernel records
 // FLINT_ERR_TIMEOUT, lets its loads land and returns.
 #include <math.h>
@@ -43,16 +48,19 @@ constexpr float kLog2e = 1.4426950408889634f;
 // log2(e) / sqrt(128): scores come out of the tensor cores in log2 units.
 constexpr float kQScale = static_cast<float>(1.4426950408889634 * 0.08838834764831845);
 constexpr float kRescaleSlack = 8.0f;
-constexpr int kXchStride = kDim + 2;  // per head: 128 O values, m, l
-constexpr int kXchFloats = kConsumerWarps * kGroup * kXchStride;
+
+// Per-thread state a consumer group hands to group 0 at an item's end:
+// 32 O values, m, l.
+constexpr int kXchFloats = 34;
+constexpr int kXchSize = (kConsumerGroups - 1) * kKvHeads * 32 * kXchFloats;
 
 struct Smem {
   uint8_t* stages;
   uint64_t* full;
   uint64_t* empty;
-  float* xch;
   float2* cs;
   volatile int* flags;  // [0] abort, [1] last-arrival broadcast
+  float* xch;           // group hand-over area
 };
 
 __device__ __forceinline__ Smem carve(uint8_t* raw) {
@@ -61,10 +69,15 @@ __device__ __forceinline__ Smem carve(uint8_t* raw) {
   s.stages = base;
   s.full = reinterpret_cast<uint64_t*>(base + kStages * kStageBytes);
   s.empty = s.full + kStages;
-  s.xch = reinterpret_cast<float*>(s.empty + kStages);
-  s.cs = reinterpret_cast<float2*>(s.xch + kXchFloats);
+  s.cs = reinterpret_cast<float2*>(s.empty + kStages);
   s.flags = reinterpret_cast<volatile int*>(s.cs + 64);
+  s.xch = reinterpret_cast<float*>(s.cs + 64) + 4;
   return s;
+}
+
+// Byte offset of box (kv: 0 = K, 1 = V; head; dim half) inside a stage.
+__device__ __forceinline__ uint32_t box_offset(int kv, int head, int half) {
+  return static_cast<uint32_t>(((kv * kKvHeads + head) * 2 + half) * kBoxBytes);
 }
 
 __device__ __forceinline__ void consumer_bar() {
@@ -77,57 +90,58 @@ __device__ __forceinline__ void abort_cta(const DecodeParams& P, const Smem& S) 
   S.flags[0] = 1;
 }
 
-// Storage offset (elements, from the cache base the problem names) of row
-// (position pos, KV head g); -1 if a paged block id is out of range.
-__device__ __forceinline__ long long append_offset(const Problem& pb, int g) {
+// Element offset, from the cache base the problem names, of the new token's
+// row (all 4 heads); -1 if a paged block id is out of range.
+__device__ __forceinline__ long long append_row(const Problem& pb) {
   if (pb.layout == FLINT_KV_PAGED) {
     const int blk = pb.table[pb.pos / kBlock];
     if (blk < 0 || blk >= pb.num_blocks) return -1;
-    return ((static_cast<long long>(blk) * kBlock + pb.pos % kBlock) * kKvHeads + g) * kDim;
+    return (static_cast<long long>(blk) * kBlock + pb.pos % kBlock) * kKvHeads * kDim;
   }
-  return (static_cast<long long>(pb.append_tok) * kKvHeads + g) * kDim;
+  return static_cast<long long>(pb.append_tok) * kKvHeads * kDim;
 }
 
 // Producer-warp side of the fused stack: norm (+RoPE) the new token's k for
-// KV head g, round to bf16 and write it and v_raw into the cache.
-__device__ void append_new_token(const DecodeParams& P, const Problem& pb, int g, int lane,
+// every KV head, round to bf16 and write it and v_raw into the cache.
+__device__ void append_new_token(const DecodeParams& P, const Problem& pb, int lane,
                                  const float2* cs) {
-  float y[4];
-  norm_rope_row_warp(pb.k_raw + g * kDim, pb.w_k, P.eps, true, pb.rope != 0, cs, lane, y);
-  const long long off = append_offset(pb, g);
-  if (off < 0) {
+  const long long row = append_row(pb);
+  if (row < 0) {
     if (lane == 0) report_error(P.dev_err, FLINT_ERR_INVALID_ARG);
     return;
   }
-  uint32_t* kd = reinterpret_cast<uint32_t*>(pb.k_rows + off);
-  uint32_t* vd = reinterpret_cast<uint32_t*>(pb.v_rows + off);
-  const uint32_t* vs = reinterpret_cast<const uint32_t*>(pb.v_raw + g * kDim);
-  kd[lane] = pack_bf16x2(y[0], y[1]);
-  kd[32 + lane] = pack_bf16x2(y[2], y[3]);
-  vd[lane] = vs[lane];
-  vd[32 + lane] = vs[32 + lane];
+#pragma unroll 1
+  for (int g = 0; g < kKvHeads; ++g) {
+    float y[4];
+    norm_rope_row_warp(pb.k_raw + g * kDim, pb.w_k, P.eps, true, pb.rope != 0, cs, lane, y);
+    uint32_t* kd = reinterpret_cast<uint32_t*>(pb.k_rows + row + g * kDim);
+    uint32_t* vd = reinterpret_cast<uint32_t*>(pb.v_rows + row + g * kDim);
+    const uint32_t* vs = reinterpret_cast<const uint32_t*>(pb.v_raw + g * kDim);
+    kd[lane] = pack_bf16x2(y[0], y[1]);
+    kd[32 + lane] = pack_bf16x2(y[2], y[3]);
+    vd[lane] = vs[lane];
+    vd[32 + lane] = vs[32 + lane];
+  }
   fence_proxy_async_global();
 }
 
 // Returns the number of tiles whose loads were issued.
 __device__ int run_producer(const DecodeParams& P, const Smem& S, int it0, int it1, int lane) {
-  int32_t* rec = P.dev_err;
-  (void)rec;
   int seq = 0;
+  // lane i < 16 issues box i: K/V (i >> 3), head ((i >> 1) & 3), dim half (i & 1)
+  const int my_kv = (lane >> 3) & 1, my_head = (lane >> 1) & 3, my_half = lane & 1;
   for (int it = it0; it < it1; ++it) {
     const Item item = P.items[it];
-    const Problem& pb = P.prob[item.seg >> 2];
-    const int g = item.seg & 3;
-    const CUtensorMap* mk = &P.maps[pb.map_k];
-    const CUtensorMap* mv = &P.maps[pb.map_v];
+    const Problem& pb = P.prob[item.seg];
+    const CUtensorMap* map = &P.maps[my_kv ? pb.map_v : pb.map_k];
     const bool paged = pb.layout == FLINT_KV_PAGED;
     const int app_tile = (P.prep && pb.append_tok >= 0) ? (pb.append_tok - pb.tile_base) / kTile : -1;
     for (int t = item.t0; t < item.t1; t += 32) {
       const int n = min(32, item.t1 - t);
       int blk = 0;
       if (paged && lane < n) {
-        const int idx = pb.tile_base / kBlock + t + lane;
-        if (FLINT_CHECK(rec, idx >= 0 && idx < pb.table_len, 3, idx, pb.table_len, it)) blk = __ldg(pb.table + idx);
+        const int idx = (pb.tile_base + (t + lane) * kTile) / kBlock;
+        if (FLINT_CHECK(P.dev_err, idx >= 0 && idx < pb.table_len, 3, idx, pb.table_len, it)) blk = __ldg(pb.table + idx);
         // An out-of-range coordinate makes TMA fill zeros; flag it for the caller.
         if (blk < 0 || blk >= pb.num_blocks) report_error(P.dev_err, FLINT_ERR_INVALID_ARG);
       }
@@ -143,27 +157,28 @@ __device__ int run_producer(const DecodeParams& P, const Smem& S, int it0, int i
         }
         const int tile = t + j;
         if (tile == app_tile) {
-          append_new_token(P, pb, g, lane, S.cs);
+          append_new_token(P, pb, lane, S.cs);
           __syncwarp();
         }
+        const uint32_t fb = smem_u32(&S.full[stage]);
+        const uint32_t base = smem_u32(S.stages + stage * kStageBytes);
+        const int tok = pb.tile_base + tile * kTile;
+        const int c2 = paged ? tok % kBlock : tok;
+        const int c3 = paged ? b : pb.req;
+        bool fine = true;
         if (lane == 0) {
-          const uint32_t fb = smem_u32(&S.full[stage]);
-          const uint32_t dst = smem_u32(S.stages + stage * kStageBytes);
-          const int c2 = paged ? 0 : pb.tile_base + tile * kTile;
-          const int c3 = paged ? b : pb.req;
-          bool fine = FLINT_CHECK(rec, (dst & 1023u) == 0 && dst + kStageBytes <= smem_u32(S.full), 6,
-                                  static_cast<int>(dst), stage, seq);
-          fine = fine && FLINT_CHECK(rec, c2 >= 0 && c2 < pb.ext2 && c3 >= 0 && c3 < pb.ext3, 5, c2, c3, it);
-          if (fine) {
+          fine = FLINT_CHECK(P.dev_err, (base & 1023u) == 0 && base + kStageBytes <= smem_u32(S.full), 6,
+                             static_cast<int>(base), stage, seq);
+          fine = fine && FLINT_CHECK(P.dev_err, c2 >= 0 && c2 < pb.ext2 && c3 >= 0 && c3 < pb.ext3, 5, c2, c3, it);
+          if (fine)
             mbar_expect_tx(fb, kStageBytes);
-            tma_load_4d(dst, mk, fb, 0, g, c2, c3);
-            tma_load_4d(dst + kHalfBytes, mk, fb, 64, g, c2, c3);
-            tma_load_4d(dst + 2 * kHalfBytes, mv, fb, 0, g, c2, c3);
-            tma_load_4d(dst + 3 * kHalfBytes, mv, fb, 64, g, c2, c3);
-          } else {
+          else
             mbar_arrive(fb);  // complete the phase without data so nobody waits forever
-          }
         }
+        fine = __shfl_sync(0xffffffffu, fine, 0);
+        __syncwarp();
+        if (fine && lane < kBoxes)
+          tma_load_4d(base + box_offset(my_kv, my_head, my_half), map, fb, 64 * my_half, my_head, c2, c3);
         __syncwarp();
       }
     }
@@ -239,33 +254,35 @@ __device__ __forceinline__ void load_q(const DecodeParams& P, const Problem& pb,
   }
 }
 
-// This warp's 16-token slice [tok0, tok0 + 16) of a 64-token tile, for the
-// 8 heads of the group: online-softmax update of (m_run, l_run, o).  sK is the
-// stage (K rows 0..63 in two swizzled 64-dim halves, then V likewise) and
-// r0 = 16 * warp is the slice's first row in it.
-__device__ __forceinline__ void consume_slice(uint32_t sK, int r0, int tok0, int lo, int hi,
+// One 16-token slice of a tile for KV head w and its 8 query heads: online-
+// softmax update of (m_run, l_run, o).  sK / sV point at row r0 of the head's
+// 64-dim K / V boxes (kTile rows of 128 bytes each, 128-byte swizzle, r0 a
+// multiple of 8); tok0 is the storage token of that row.
+__device__ __forceinline__ void consume_slice(uint32_t sK, uint32_t sV, int tok0, int lo, int hi,
                                               int lane, const uint32_t (&qa)[8][4], float& m_run,
                                               float& l_run, float (&o)[16][4]) {
   const int c = lane & 3;
   const int l7 = lane & 7;
-  const bool whole = (tok0 >= lo) && (tok0 + 16 <= hi);
+  const bool whole = (tok0 >= lo) && (tok0 + kSlice <= hi);
 
   // S^T = [q_hi; q_lo] * K^T: 2 n-tiles of 8 tokens, 8 k-steps of 16 dims.
+  // (two accumulators per n-tile keep the dependent MMA chains short)
   float sc[4];
 #pragma unroll
   for (int jj = 0; jj < 2; ++jj) {
-    float acc[4] = {0.f, 0.f, 0.f, 0.f};
-    const uint32_t row = sK + (r0 + 8 * jj + l7) * 128;
+    float a0[4] = {0.f, 0.f, 0.f, 0.f}, a1[4] = {0.f, 0.f, 0.f, 0.f};
+    const uint32_t row = sK + (8 * jj + l7) * 128;
 #pragma unroll
     for (int kk = 0; kk < 8; kk += 2) {
       const int u = 2 * kk + (lane >> 3);  // 16-byte unit along the 128 dims
       uint32_t b0, b1, b2, b3;
-      ldsm_x4(row + (u >> 3) * kHalfBytes + (((u & 7) ^ l7) << 4), b0, b1, b2, b3);
-      mma_bf16_16816(acc, qa[kk], b0, b1);
-      mma_bf16_16816(acc, qa[kk + 1], b2, b3);
+      ldsm_x4(row + (u >> 3) * kBoxBytes + (((u & 7) ^ l7) << 4), b0, b1, b2, b3);
+      mma_bf16_16816(a0, qa[kk], b0, b1);
+      mma_bf16_16816(a1, qa[kk + 1], b2, b3);
     }
-    sc[2 * jj] = acc[0] + acc[2];  // token tok0 + 8jj + 2c (+1)
-    sc[2 * jj + 1] = acc[1] + acc[3];
+    // rows g (q hi part) and g + 8 (q lo part): token tok0 + 8jj + 2c (+1)
+    sc[2 * jj] = (a0[0] + a1[0]) + (a0[2] + a1[2]);
+    sc[2 * jj + 1] = (a0[1] + a1[1]) + (a0[3] + a1[3]);
   }
   if (!whole) {
 #pragma unroll
@@ -279,7 +296,7 @@ __device__ __forceinline__ void consume_slice(uint32_t sK, int r0, int tok0, int
   mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 1));
   mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 2));
   // The running max moves only when a head's max grows by more than the
-  // slack (always on its first valid slice); the branch is warp-uniform.
+  // slack (always on its first valid tile); the branch is warp-uniform.
   const bool grow = mx > m_run + kRescaleSlack;
   if (__any_sync(0xffffffffu, grow)) {
     const float alpha = grow ? exp2f(m_run - mx) : 1.0f;
@@ -308,12 +325,12 @@ __device__ __forceinline__ void consume_slice(uint32_t sK, int r0, int tok0, int
     m23 = ((t + 8 >= lo && t + 8 < hi) ? 0x0000ffffu : 0u) |
           ((t + 9 >= lo && t + 9 < hi) ? 0xffff0000u : 0u);
   }
-  const uint32_t row = sK + 2 * kHalfBytes + (r0 + ((lane >> 3) & 1) * 8 + l7) * 128;
+  const uint32_t row = sV + (((lane >> 3) & 1) * 8 + l7) * 128;
 #pragma unroll
   for (int np = 0; np < 8; ++np) {
     const int nt = 2 * np + (lane >> 4);
     uint32_t v0, v1, v2, v3;
-    ldsm_x4_t(row + (nt >> 3) * kHalfBytes + (((nt & 7) ^ l7) << 4), v0, v1, v2, v3);
+    ldsm_x4_t(row + (nt >> 3) * kBoxBytes + (((nt & 7) ^ l7) << 4), v0, v1, v2, v3);
     if (!whole) {  // rows outside the range may hold anything (even NaN)
       v0 &= m01;
       v2 &= m01;
@@ -325,32 +342,37 @@ __device__ __forceinline__ void consume_slice(uint32_t sK, int r0, int tok0, int
   }
 }
 
-// Final normalisation with the sink logit of head kvh*8 + hh folded in.
-__device__ __forceinline__ void finish_head(const Problem& pb, int kvh, int hh, int d0, float M,
-                                            float L, const float (&acc)[8]) {
-  const int head = kvh * kGroup + hh;
+// Offset (floats) of consumer thread (head, c)'s 32 O values inside a partial.
+__device__ __forceinline__ int partial_o(int head, int c) { return (head * 4 + c) * 32; }
+
+// out[head][8n + 2c + e] = O * 2^(M - Mf) / (L 2^(M - Mf) + 2^(sink - Mf)), the
+// sink logit of this head folded into the softmax; thread (g, c) owns dims
+// 8n + 2c + {0,1} of head `head`.
+__device__ __forceinline__ void finish_head(const Problem& pb, int head, int c, float M, float L,
+                                            const float (&v)[32]) {
   const float s2 = pb.sinks[head] * kLog2e;
   const float Mf = fmaxf(M, s2);
   const float a = (M == -INFINITY) ? 0.f : exp2f(M - Mf);
-  const float inv = 1.0f / (L * a + exp2f(s2 - Mf));
-  float4* dst = reinterpret_cast<float4*>(pb.out + head * kDim + d0);
-  dst[0] = make_float4(acc[0] * a * inv, acc[1] * a * inv, acc[2] * a * inv, acc[3] * a * inv);
-  dst[1] = make_float4(acc[4] * a * inv, acc[5] * a * inv, acc[6] * a * inv, acc[7] * a * inv);
+  const float scale = a / (L * a + exp2f(s2 - Mf));
+  float* dst = pb.out + head * kDim + 2 * c;
+#pragma unroll
+  for (int n = 0; n < 16; ++n)
+    *reinterpret_cast<float2*>(dst + 8 * n) = make_float2(v[2 * n] * scale, v[2 * n + 1] * scale);
 }
 
 __device__ void run_consumer(const DecodeParams& P, const Smem& S, int it0, int it1, int warp,
                              int lane) {
   const int g = lane >> 2, c = lane & 3;
-  const int t = threadIdx.x;              // 0..127 within the consumer warps
-  const int hh = t >> 4, d0 = (t & 15) * 8;  // merge role: head, 8 dims
+  const int kvh = warp % kKvHeads;      // the KV head this warp serves
+  const int group = warp / kKvHeads;    // its consumer group
+  const int head = kvh * kGroup + g;    // the query head this thread's quad serves
   int seq = 0;
   for (int it = it0; it < it1; ++it) {
     const Item item = P.items[it];
-    const Problem& pb = P.prob[item.seg >> 2];
-    const int kvh = item.seg & 3;
+    const Problem& pb = P.prob[item.seg];
 
     uint32_t qa[8][4];
-    load_q(P, pb, kvh * kGroup + g, c, S.cs, qa);
+    load_q(P, pb, head, c, S.cs, qa);
 
     float m_run = -INFINITY, l_run = 0.f;
     float o[16][4];
@@ -359,8 +381,6 @@ __device__ void run_consumer(const DecodeParams& P, const Smem& S, int it0, int 
 #pragma unroll
       for (int e = 0; e < 4; ++e) o[n][e] = 0.f;
 
-    // Every consumer warp takes part in every tile (its own 16-token slice),
-    // so each warp waits on the stages' phases strictly in order.
     const int ntiles = item.t1 - item.t0;
     for (int k = 0; k < ntiles; ++k, ++seq) {
       const int stage = seq % kStages;
@@ -372,90 +392,108 @@ __device__ void run_consumer(const DecodeParams& P, const Smem& S, int it0, int 
         if (lane == 0) abort_cta(P, S);
         continue;  // keep walking so that every warp meets the same barriers
       }
-      const int tok0 = pb.tile_base + (item.t0 + k) * kTile + 16 * warp;
-      consume_slice(smem_u32(S.stages + stage * kStageBytes), 16 * warp, tok0, pb.lo, pb.hi, lane, qa,
-                    m_run, l_run, o);
+      const uint32_t base = smem_u32(S.stages + stage * kStageBytes);
+      const int r0 = group * kSlice;
+      const int tok0 = pb.tile_base + (item.t0 + k) * kTile + r0;
+      consume_slice(base + box_offset(0, kvh, 0) + r0 * 128, base + box_offset(1, kvh, 0) + r0 * 128,
+                    tok0, pb.lo, pb.hi, lane, qa, m_run, l_run, o);
       __syncwarp();
       if (lane == 0) mbar_arrive(smem_u32(&S.empty[stage]));
     }
 
-    // ---- merge the four warps' states for this item
+    // ---- item end: this warp holds (m, l, O) of its 8 heads over the item
     l_run += __shfl_xor_sync(0xffffffffu, l_run, 1);
     l_run += __shfl_xor_sync(0xffffffffu, l_run, 2);
-    float* xw = S.xch + (warp * kGroup + g) * kXchStride;
+    float v[32];
 #pragma unroll
-    for (int n = 0; n < 16; ++n)
-      *reinterpret_cast<float2*>(xw + 8 * n + 2 * c) = make_float2(o[n][0] + o[n][2], o[n][1] + o[n][3]);
-    if (c == 0) {
-      xw[kDim] = m_run;
-      xw[kDim + 1] = l_run;
+    for (int n = 0; n < 16; ++n) {
+      v[2 * n] = o[n][0] + o[n][2];
+      v[2 * n + 1] = o[n][1] + o[n][3];
+    }
+    if (kConsumerGroups > 1) {
+      // the other groups hand their states to group 0, which merges them
+      float* mine = S.xch + ((group - 1) * kKvHeads * 32 + kvh * 32 + lane) * kXchFloats;
+      if (group > 0) {
+#pragma unroll
+        for (int e = 0; e < 32; ++e) mine[e] = v[e];
+        mine[32] = m_run;
+        mine[33] = l_run;
+      }
+      __syncwarp();
+      consumer_bar();
+      if (group == 0) {
+#pragma unroll 1
+        for (int q = 1; q < kConsumerGroups; ++q) {
+          const float* other = S.xch + ((q - 1) * kKvHeads * 32 + kvh * 32 + lane) * kXchFloats;
+          const float mo = other[32], lo_ = other[33];
+          const float M = fmaxf(m_run, mo);
+          const float sa = (m_run == -INFINITY) ? 0.f : exp2f(m_run - M);
+          const float sb = (mo == -INFINITY) ? 0.f : exp2f(mo - M);
+#pragma unroll
+          for (int e = 0; e < 32; ++e) v[e] = v[e] * sa + other[e] * sb;
+          l_run = l_run * sa + lo_ * sb;
+          m_run = M;
+        }
+      }
+    }
+    const int s0 = P.seg_item_begin[item.seg], s1 = P.seg_item_begin[item.seg + 1];
+    if (s1 - s0 == 1) {
+      if (group == 0) finish_head(pb, head, c, m_run, l_run, v);
+      __syncwarp();
+      consumer_bar();  // the hand-over area is reused by the next item
+      continue;
+    }
+    float* part = P.partials + static_cast<size_t>(it) * kPartialFloats;
+    if (group == 0 &&
+        FLINT_CHECK(P.dev_err, it < P.ws_items && s0 >= 0 && s1 <= P.n_items, 7, it, s0, s1)) {
+      float4* pd = reinterpret_cast<float4*>(part + partial_o(head, c));
+#pragma unroll
+      for (int i = 0; i < 8; ++i) pd[i] = make_float4(v[4 * i], v[4 * i + 1], v[4 * i + 2], v[4 * i + 3]);
+      if (c == 0) {
+        part[kHeads * kDim + head] = m_run;
+        part[kHeads * kDim + kHeads + head] = l_run;
+      }
+    }
+    __threadfence();
+    __syncwarp();
+    consumer_bar();
+    if (threadIdx.x == 0) {
+      int prev = 0;
+      if (FLINT_CHECK(P.dev_err, item.seg < kMaxSegs, 8, item.seg, 0, 0))
+        prev = atomicAdd(P.counters + item.seg, 1);
+      S.flags[1] = (prev == s1 - s0 - 1) ? 1 : 0;
     }
     __syncwarp();
     consumer_bar();
-
-    float M = -INFINITY;
-#pragma unroll
-    for (int w = 0; w < kConsumerWarps; ++w) M = fmaxf(M, S.xch[(w * kGroup + hh) * kXchStride + kDim]);
-    float L = 0.f, acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
-#pragma unroll
-    for (int w = 0; w < kConsumerWarps; ++w) {
-      const float* xr = S.xch + (w * kGroup + hh) * kXchStride;
-      const float mw = xr[kDim];
-      const float sw = (mw == -INFINITY) ? 0.f : exp2f(mw - M);
-      L += sw * xr[kDim + 1];
-#pragma unroll
-      for (int i = 0; i < 8; ++i) acc[i] += sw * xr[d0 + i];
-    }
-
-    const int seg = item.seg;
-    const int s0 = P.seg_item_begin[seg], s1 = P.seg_item_begin[seg + 1];
-    if (s1 - s0 == 1) {
-      finish_head(pb, kvh, hh, d0, M, L, acc);
-    } else {
-      float* part = P.partials + static_cast<size_t>(it) * kPartialFloats;
-      if (FLINT_CHECK(P.dev_err, it < P.ws_items && s0 >= 0 && s1 <= P.n_items, 7, it, s0, s1)) {
-        float4* pd = reinterpret_cast<float4*>(part + hh * kDim + d0);
-        pd[0] = make_float4(acc[0], acc[1], acc[2], acc[3]);
-        pd[1] = make_float4(acc[4], acc[5], acc[6], acc[7]);
-        if ((t & 15) == 0) {
-          part[kGroup * kDim + hh] = M;
-          part[kGroup * kDim + kGroup + hh] = L;
-        }
-      }
+    if (S.flags[1] && group == 0) {
+      // last arrival: merge every partial of the problem, in item order
       __threadfence();
-      __syncwarp();
-      consumer_bar();
-      if (t == 0) {
-        int prev = 0;
-        if (FLINT_CHECK(P.dev_err, seg >= 0 && seg < kMaxSegs, 8, seg, 0, 0))
-          prev = atomicAdd(P.counters + seg, 1);
-        S.flags[1] = (prev == s1 - s0 - 1) ? 1 : 0;
-      }
-      __syncwarp();
-      consumer_bar();
-      if (S.flags[1]) {
-        // last arrival: merge every partial of the segment, in item order
-        __threadfence();
-        float M2 = -INFINITY;
-        for (int i = s0; i < s1; ++i)
-          M2 = fmaxf(M2, __ldcg(P.partials + static_cast<size_t>(i) * kPartialFloats + kGroup * kDim + hh));
-        float L2 = 0.f, acc2[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
-        for (int i = s0; i < s1; ++i) {
-          const float* pi = P.partials + static_cast<size_t>(i) * kPartialFloats;
-          const float mi = __ldcg(pi + kGroup * kDim + hh);
-          const float si = (mi == -INFINITY) ? 0.f : exp2f(mi - M2);
-          L2 += si * __ldcg(pi + kGroup * kDim + kGroup + hh);
-          const float4 a = __ldcg(reinterpret_cast<const float4*>(pi + hh * kDim + d0));
-          const float4 b = __ldcg(reinterpret_cast<const float4*>(pi + hh * kDim + d0 + 4));
-          acc2[0] += si * a.x; acc2[1] += si * a.y; acc2[2] += si * a.z; acc2[3] += si * a.w;
-          acc2[4] += si * b.x; acc2[5] += si * b.y; acc2[6] += si * b.z; acc2[7] += si * b.w;
+      float M = -INFINITY;
+      for (int i = s0; i < s1; ++i)
+        M = fmaxf(M, __ldcg(P.partials + static_cast<size_t>(i) * kPartialFloats + kHeads * kDim + head));
+      float L = 0.f;
+#pragma unroll
+      for (int e = 0; e < 32; ++e) v[e] = 0.f;
+      for (int i = s0; i < s1; ++i) {
+        const float* pi = P.partials + static_cast<size_t>(i) * kPartialFloats;
+        const float mi = __ldcg(pi + kHeads * kDim + head);
+        const float si = (mi == -INFINITY) ? 0.f : exp2f(mi - M);
+        L += si * __ldcg(pi + kHeads * kDim + kHeads + head);
+        const float4* po = reinterpret_cast<const float4*>(pi + partial_o(head, c));
+#pragma unroll
+        for (int q = 0; q < 8; ++q) {
+          const float4 a = __ldcg(po + q);
+          v[4 * q] += si * a.x;
+          v[4 * q + 1] += si * a.y;
+          v[4 * q + 2] += si * a.z;
+          v[4 * q + 3] += si * a.w;
         }
-        finish_head(pb, kvh, hh, d0, M2, L2, acc2);
-        if (t == 0) P.counters[seg] = 0;  // ready for the next call
       }
+      finish_head(pb, head, c, M, L, v);
+      if (threadIdx.x == 0) P.counters[item.seg] = 0;  // ready for the next call
     }
     __syncwarp();
-    consumer_bar();  // the exchange area and flags[1] are reused by the next item
+    consumer_bar();  // flags[1] is reused by the next item
   }
 }
 
@@ -465,7 +503,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const __grid_consta
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   int it0 = P.cta_item_begin[blockIdx.x], it1 = P.cta_item_begin[blockIdx.x + 1];
   if (!FLINT_CHECK(P.dev_err, 0 <= it0 && it0 <= it1 && it1 <= P.n_items, 1, it0, it1, P.n_items)) it1 = it0;
-  const int smem_end = static_cast<int>(smem_u32(const_cast<int*>(S.flags) + 4) - smem_u32(smem_raw));
+  const int smem_end = static_cast<int>(smem_u32(S.xch + kXchSize) - smem_u32(smem_raw));
   if (!FLINT_CHECK(P.dev_err, smem_end <= P.smem_bytes, 2, smem_end, P.smem_bytes, 0)) it1 = it0;
   (void)smem_end;
 
@@ -506,7 +544,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const __grid_consta
 
 size_t decode_smem_bytes() {
   return 1024 + static_cast<size_t>(kStages) * kStageBytes + 2 * kStages * sizeof(uint64_t) +
-         kXchFloats * sizeof(float) + 64 * sizeof(float2) + 4 * sizeof(int);
+         64 * sizeof(float2) + 4 * sizeof(int) + kXchSize * sizeof(float);
 }
 
 cudaError_t launch_decode(const DecodeParams& p, int grid, cudaStream_t stream) {

@@ -43,7 +43,7 @@ static __device__ __noinline__ void debug_record(int32_t* rec, int code, int a, 
 #define FLINT_CHECK(rec, cond, code, a, b, c) \
   ((cond) ? true : (::flint::debug_record((rec), (code), (a), (b), (c)), false))
 #else
-#define FLINT_CHECK(rec, cond, code, a, b, c) true
+#define FLINT_CHECK(rec, cond, code, a, b, c) ((void)(rec), true)
 #endif
 
 // ---- mbarrier -------------------------------------------------------------

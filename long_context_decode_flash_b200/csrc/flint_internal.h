@@ -6,7 +6,7 @@
 #include <cuda_runtime.h>
 #include <stdint.h>
 
-#include "../../include/flint.h"
+#include "flint.h"
 
 namespace flint {
 
@@ -17,23 +17,44 @@ constexpr int kGroup = kHeads / kKvHeads;     // 8 query heads share a KV head
 constexpr int kWindow = FLINT_WINDOW;         // 513
 constexpr int kBlock = FLINT_BLOCK_SIZE;      // 64
 
-// Decode pipeline geometry.
-constexpr int kTile = 64;                     // tokens per pipeline stage
-constexpr int kHalfBytes = kTile * 64 * 2;    // one 64-dim half of a K or V tile: 8 KiB
-constexpr int kStageBytes = 4 * kHalfBytes;   // K lo/hi + V lo/hi: 32 KiB
-constexpr int kStages = 6;
-constexpr int kConsumerWarps = 4;
+// Decode pipeline geometry: a stage holds K and V of kTile tokens for all 4
+// KV heads, as 16 TMA boxes of kTile rows x 64 dims (one per head, dim half
+// and K/V), so a CTA reads whole 1 KiB token rows of the cache.  Taller boxes
+// stream faster (measured: 32 rows ~4% above 16 rows).
+#ifndef FLINT_TILE
+#define FLINT_TILE 32
+#endif
+#ifndef FLINT_L2_PROMOTION
+#define FLINT_L2_PROMOTION 3                  // CU_TENSOR_MAP_L2_PROMOTION_L2_256B
+#endif
+constexpr int kTile = FLINT_TILE;             // tokens per pipeline stage
+constexpr int kBoxBytes = kTile * 64 * 2;     // one box: 2 KiB
+constexpr int kBoxes = 2 * kKvHeads * 2;      // K/V x heads x dim halves = 16
+constexpr int kStageBytes = kBoxes * kBoxBytes;  // 64 KiB at 32 tokens
+#ifndef FLINT_STAGES
+#define FLINT_STAGES 3
+#endif
+constexpr int kStages = FLINT_STAGES;
+// Consumer warps come in groups of 4 (warp w of a group serves KV head w);
+// every group takes part in every stage, group q on the q-th 16-token slice
+// of the tile, so every warp waits on every stage's phases in order.  Two
+// groups put two consumer warps on every scheduler.
+constexpr int kSlice = 16;                    // tokens per consumer warp per stage
+constexpr int kConsumerGroups = kTile / kSlice;
+constexpr int kConsumerWarps = kKvHeads * kConsumerGroups;
 constexpr int kThreads = (kConsumerWarps + 1) * 32;
+static_assert(kTile % kSlice == 0, "a tile splits into 16-token slices");
 
 // Limits of one launch (bounded by the 32 KiB kernel-parameter space).
 constexpr int kMaxProblems = 64;
-constexpr int kMaxSegs = kMaxProblems * kKvHeads;
+constexpr int kMaxSegs = kMaxProblems;         // one segment per problem
 constexpr int kMaxMaps = 2 * FLINT_MAX_LAYERS;
 constexpr int kMaxItems = 512;
 constexpr int kMaxCtas = 296;
 
-// One split partial: O [8][128], m [8], l [8] (fp32, m in log2 units).
-constexpr int kPartialFloats = kGroup * kDim + 2 * kGroup;
+// One split partial of a problem: O for 32 heads (stored so that each
+// consumer thread's 32 values are contiguous), m [32] (log2 units), l [32].
+constexpr int kPartialFloats = kHeads * kDim + 2 * kHeads;
 constexpr size_t kCounterBytes = 4096;
 
 // One attention problem: one request of one layer.
@@ -49,7 +70,7 @@ struct Problem {
   uint16_t* v_rows;
   const int32_t* table;     // PAGED: this request's block-table row
   int32_t lo, hi;           // attended tokens [lo, hi) in storage coordinates
-  int32_t tile_base;        // token of tile 0 (CONTIGUOUS/RING) or block index (PAGED)
+  int32_t tile_base;        // storage token of tile 0 (a multiple of 16 for PAGED)
   int32_t append_tok;       // storage-coordinate token of the new token, or -1
   int32_t pos;              // logical position of the new token (RoPE, paged append)
   int32_t num_blocks;       // PAGED pool size
@@ -61,8 +82,8 @@ struct Problem {
 };
 
 struct Item {
-  int16_t seg;              // problem * 4 + kv head
-  int16_t t0, t1;           // tile range within the segment
+  int16_t seg;              // problem
+  int16_t t0, t1;           // tile range within the problem's token range
   int16_t pad;
 };
 

@@ -9,7 +9,7 @@
 // items and the items of one segment sit on consecutive CTAs.
 #include <stdint.h>
 
-#include "../../include/flint.h"
+#include "flint.h"
 
 namespace {
 constexpr int kMinPiece = 2;

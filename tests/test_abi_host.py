@@ -153,24 +153,22 @@ def check_plan(seg_tiles, G, cost=2):
 
 
 def test_plan_single_full_layer_at_100k():
-    items, cb, loads = check_plan([1563] * 4, 148)
-    assert len(items) <= 148 + 4
-    assert min(l for l in loads if l) >= 40
+    # one problem of 100,000 tokens = 6,250 tiles of 16 tokens (all 4 KV heads)
+    items, cb, loads = check_plan([6250], 148)
+    assert len(items) == 148
+    assert min(loads) >= 40
 
 
 def test_plan_layer_stack_at_100k():
-    tiles = []
-    for i in range(49):
-        full = (i % 7) in (3, 6)
-        tiles += [1563 if full else 9] * 4
+    tiles = [6250 if (i % 7) in (3, 6) else 33 for i in range(49)]
     items, cb, loads = check_plan(tiles, 148)
-    assert len(items) <= 512
+    assert len(items) <= 148 + 49
 
 
 def test_plan_random_cases():
     r = random.Random(5)
     for _ in range(200):
-        n = r.randint(1, 256)
+        n = r.randint(1, 64)
         tiles = [r.choice([1, 2, 3, 9, r.randint(1, 4096)]) for _ in range(n)]
         G = r.randint(1, 296)
         try:

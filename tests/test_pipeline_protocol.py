@@ -11,15 +11,18 @@ This test replays the protocol under many random interleavings and random
 TMA landing times, and asserts that (a) a consumer only reads a stage after
 the exact tile it expects has landed, (b) the producer never re-arms a
 stage whose previous load is still in flight.  The kernel's scheme (every
-consumer warp takes a slice of every tile) passes; the earlier round-robin
-scheme (tile i to warp i mod 4 with 6 stages) is shown to fail.
+consumer warp takes a slice of every tile, so every warp waits on every
+stage in order) passes for 4 or 8 consumer warps and 3 or 6 stages, as do
+groups that take alternate tiles when the group count divides the stage
+count; the earlier round-robin scheme (tile i to warp i mod 4 with 6 stages)
+is shown to fail.
 """
 import random
 
 import pytest
 
 STAGES = 6
-WARPS = 4
+WARPS = 4     # warps per consumer group in the model
 
 
 class Barrier:
@@ -49,17 +52,32 @@ class Barrier:
             self.pending = self.count
 
 
-def simulate(n_tiles, scheme, rng):
+def simulate(n_tiles, scheme, rng, groups=1, warps=None, stages=None):
+    """scheme "all_warps": `groups` groups of WARPS warps; group q takes the
+    tiles i with i % groups == q and all its warps take part in each of them.
+    scheme "round_robin": whole tiles to single warps, i % WARPS."""
+    global STAGES, WARPS
+    saved = STAGES, WARPS
+    STAGES = stages or STAGES
+    WARPS = warps or WARPS
+    try:
+        return _simulate(n_tiles, scheme, rng, groups)
+    finally:
+        STAGES, WARPS = saved
+
+
+def _simulate(n_tiles, scheme, rng, groups):
     full = [Barrier(1) for _ in range(STAGES)]
     empty = [Barrier(WARPS if scheme == "all_warps" else 1) for _ in range(STAGES)]
     in_flight = []          # (stage, tile) loads not landed yet
     landed_tile = [None] * STAGES
     prod = 0
     if scheme == "all_warps":
-        work = [list(range(n_tiles)) for _ in range(WARPS)]
+        work = [[i for i in range(n_tiles) if i % groups == w // WARPS] for w in range(WARPS * groups)]
     else:
         work = [[i for i in range(n_tiles) if i % WARPS == w] for w in range(WARPS)]
-    pos = [0] * WARPS
+    nw = len(work)
+    pos = [0] * nw
     while True:
         actions = []
         if prod < n_tiles:
@@ -68,7 +86,7 @@ def simulate(n_tiles, scheme, rng):
                 actions.append("produce")
         if in_flight:
             actions.append("land")
-        for w in range(WARPS):
+        for w in range(nw):
             if pos[w] < len(work[w]):
                 i = work[w][pos[w]]
                 if full[i % STAGES].parity_done((i // STAGES) & 1):
@@ -95,16 +113,34 @@ def simulate(n_tiles, scheme, rng):
                 return f"warp {w} read stage {s} for tile {i} but it holds tile {landed_tile[s]}"
             empty[s].arrive()
             pos[w] += 1
-    if prod != n_tiles or any(pos[w] != len(work[w]) for w in range(WARPS)):
+    if prod != n_tiles or any(pos[w] != len(work[w]) for w in range(nw)):
         return "deadlock"
     return None
 
 
-def test_kernel_scheme_is_safe_under_random_interleavings():
-    rng = random.Random(1)
-    for trial in range(400):
-        err = simulate(rng.randint(1, 200), "all_warps", rng)
+@pytest.mark.parametrize("warps,stages", [(4, 6), (8, 3), (8, 6)])
+def test_every_warp_on_every_stage_is_safe(warps, stages):
+    rng = random.Random(warps * 10 + stages)
+    for trial in range(300):
+        err = simulate(rng.randint(1, 200), "all_warps", rng, warps=warps, stages=stages)
         assert err is None, f"trial {trial}: {err}"
+
+
+@pytest.mark.parametrize("groups", [1, 2, 3])
+def test_kernel_scheme_is_safe_under_random_interleavings(groups):
+    # the kernel needs STAGES % groups == 0 so that a stage always belongs to
+    # the same group
+    assert STAGES % groups == 0
+    rng = random.Random(groups)
+    for trial in range(300):
+        err = simulate(rng.randint(1, 200), "all_warps", rng, groups=groups)
+        assert err is None, f"trial {trial}: {err}"
+
+
+def test_groups_that_do_not_divide_the_stages_are_unsafe():
+    rng = random.Random(4)
+    errors = [simulate(200, "all_warps", rng, groups=4) for _ in range(100)]
+    assert any(e is not None for e in errors)
 
 
 def test_round_robin_scheme_is_unsafe():
