@@ -45,6 +45,7 @@ def parse():
                     help="context length (the benchmark's figure is 100,000; smaller ones serve profiling)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-graph", action="store_true", help="time direct launches instead of graph replays")
     return ap.parse_args()
 
 
@@ -318,6 +319,34 @@ def main():
     if int(err.item()) != 0:
         raise SystemExit(f"device error {int(err.item())} during warm-up")
 
+    # The device-timed steps replay the step captured in a CUDA graph (its
+    # launch parameters are fixed for a given token position), as a decode
+    # loop would; the e2e figure below goes through the direct API calls.
+    launch = "cuda graph replay"
+    graph = None
+    if not args.no_graph:
+        try:
+            graph = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(graph):
+                step()
+            torch.cuda.synchronize()
+        except Exception as e:  # capture unsupported: time direct launches
+            graph = None
+            launch = f"direct launches (graph capture failed: {str(e)[:80]})"
+    else:
+        launch = "direct launches"
+    run = graph.replay if graph is not None else step
+    for _ in range(3):
+        flush.fill_(1.0)
+        run()
+    torch.cuda.synchronize()
+    # host cost of one public-API call (argument marshalling, plan, launch)
+    t0 = time.perf_counter()
+    for _ in range(20):
+        step()
+    host_us = (time.perf_counter() - t0) / 20 * 1e6
+    torch.cuda.synchronize()
+
     starts = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
     ends = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
     if world > 1:
@@ -328,7 +357,7 @@ def main():
         for i in range(args.steps):
             flush.fill_(float(i))
             starts[i].record(stream)
-            step()
+            run()
             ends[i].record(stream)
         torch.cuda.synchronize()
         t_wall = time.perf_counter() - t_wall
@@ -377,7 +406,8 @@ def main():
         "n_gpus": world, "steps": args.steps, "warmup": max(args.warmup, 3),
         "ms_per_step": ms, "higher_is_better": False, "scaling": "weak", "vs_baseline": None,
         "dtype": "bf16", "data": "synthetic (seeded bf16 N(0,1) q/k/v/KV, N(0,1) sinks, 1+N(0,0.1) norm weights)",
-        "config": dict(workload_config(args.workload), context=ctx, parallelism=f"replicas x{world}"),
+        "config": dict(workload_config(args.workload), context=ctx, parallelism=f"replicas x{world}",
+                       launch=launch),
         "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
                      "frac": achieved / peak, "peak_kind": peak_kind,
                      "frac_of_nominal_8000": achieved / NOMINAL_HBM_GBS,
@@ -386,6 +416,7 @@ def main():
         "cpu_baseline": cpu_baseline,
         "e2e": e2e,
         "gpu_launches": args.steps,
+        "host_us_per_call": host_us,
         "clocks": clocks.summary(),
         "per_step_us": {"min": min(per_step_ms) * 1000.0, "median": statistics.median(per_step_ms) * 1000.0,
                         "max": max(per_step_ms) * 1000.0},

@@ -152,9 +152,11 @@ flint_status flint_kv_append(const uint16_t* k, const uint16_t* v, const int32_t
 
 /* Bytes of device workspace that flint_attn_decode / flint_attn_stack need
  * for n_problems (requests, or layers) on a grid of num_ctas CTAs (0 = the
- * current device's default).  The workspace holds split partials and
- * per-head arrival counters; it must be zero-filled before its first use and
- * is left zeroed by every call that completes without a device error.
+ * current device's default).  The workspace holds split partials, per-problem
+ * arrival counters and a grid-barrier word; it must be zero-filled before its
+ * first use, and every call that completes without a device error leaves it
+ * ready for the next call (counters back at zero).  After a device error,
+ * zero it again.  Calls that share a workspace must not overlap in time.
  * Returns 0 for invalid arguments. */
 size_t flint_attn_workspace_bytes(int32_t n_problems, int32_t num_ctas);
 

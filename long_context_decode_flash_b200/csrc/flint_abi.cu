@@ -11,6 +11,7 @@
 #include <algorithm>
 #include <mutex>
 #include <string>
+#include <unordered_map>
 
 #include "flint_internal.h"
 
@@ -78,6 +79,25 @@ EncodeTiledFn encode_fn() {
   return fn;
 }
 
+// Encoded maps are kept per (device, base, geometry): a decode loop calls with
+// the same caches every token, so encoding happens once.
+struct MapKey {
+  int dev;
+  uintptr_t base;
+  int64_t d2, d3, stride2;
+  bool operator==(const MapKey& o) const {
+    return dev == o.dev && base == o.base && d2 == o.d2 && d3 == o.d3 && stride2 == o.stride2;
+  }
+};
+struct MapKeyHash {
+  size_t operator()(const MapKey& k) const {
+    size_t h = std::hash<uintptr_t>()(k.base);
+    h ^= std::hash<int64_t>()(k.d2 * 1000003 + k.d3) + 0x9e3779b97f4a7c15ull + (h << 6) + (h >> 2);
+    h ^= std::hash<int64_t>()(k.stride2 * 31 + k.dev) + 0x9e3779b97f4a7c15ull + (h << 6) + (h >> 2);
+    return h;
+  }
+};
+
 // A K or V cache seen as a 4-D bf16 tensor (dims innermost first):
 //   CONTIGUOUS/RING: [128 dims][4 heads][capacity tokens][B requests]
 //   PAGED:           [128 dims][4 heads][64 tokens][num_blocks]
@@ -100,6 +120,20 @@ flint_status encode_cache_map(CUtensorMap* map, void* base, const flint_kv_cache
     dims[3] = static_cast<cuuint64_t>(B);
     strides[2] = static_cast<cuuint64_t>(rs) * 2;
   }
+  static std::mutex mu;
+  static std::unordered_map<MapKey, CUtensorMap, MapKeyHash> cache;
+  int dev = 0;
+  cudaGetDevice(&dev);
+  const MapKey key{dev, reinterpret_cast<uintptr_t>(base), static_cast<int64_t>(dims[2]),
+                   static_cast<int64_t>(dims[3]), static_cast<int64_t>(strides[2])};
+  {
+    std::lock_guard<std::mutex> lock(mu);
+    auto it = cache.find(key);
+    if (it != cache.end()) {
+      *map = it->second;
+      return FLINT_OK;
+    }
+  }
   const cuuint32_t box[4] = {64, 1, static_cast<cuuint32_t>(kTile), 1};
   const cuuint32_t estr[4] = {1, 1, 1, 1};
   CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, base, dims, strides, box, estr,
@@ -107,6 +141,9 @@ flint_status encode_cache_map(CUtensorMap* map, void* base, const flint_kv_cache
                   static_cast<CUtensorMapL2promotion>(FLINT_L2_PROMOTION),
                   CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   if (r != CUDA_SUCCESS) return fail(FLINT_ERR_CUDA, "cuTensorMapEncodeTiled failed (CUresult %d)", (int)r);
+  std::lock_guard<std::mutex> lock(mu);
+  if (cache.size() >= 4096) cache.clear();
+  cache.emplace(key, *map);
   return FLINT_OK;
 }
 
@@ -220,6 +257,13 @@ flint_status plan(DecodeParams& P, const int* tiles, int n_problems, int num_cta
     while (i < n && seg[i] < s) ++i;
     P.seg_item_begin[s] = static_cast<int16_t>(i);
   }
+  P.n_deferred = 0;
+  for (int s = 0; s < n_segs; ++s) {
+    const bool deferred = P.seg_item_begin[s + 1] - P.seg_item_begin[s] > kInlineMergeMax;
+    P.prob[s].deferred = deferred ? 1 : 0;
+    if (deferred) P.deferred[P.n_deferred++] = static_cast<int16_t>(s);
+  }
+  P.grid_merge = P.n_deferred > 0 ? 1 : 0;
   *grid = last;
   return FLINT_OK;
 }

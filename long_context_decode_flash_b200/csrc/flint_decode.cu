@@ -32,8 +32,10 @@
 //   * Item end: a problem covered by one item is finished on the spot (sink
 //     folded in); otherwise the CTA stores a partial (m, l, O for 32 heads)
 //     and the last CTA to arrive (atomic counter, no spinning) merges all
-//     partials of the problem in item order and folds in the sinks, so
-//     results are deterministic.
+//     partials of the problem in item order and folds in the sinks.  A
+//     problem split over many CTAs (more than kInlineMergeMax items) is
+//     instead merged after a grid barrier (cooperative launch) by every warp
+//     of the grid.  Merge orders are fixed, so results are deterministic.
 // Every mbarrier wait is bounded in time; on timeout the kernel records
 // FLINT_ERR_TIMEOUT, lets its loads land and returns.
 #include <math.h>
@@ -54,13 +56,28 @@ constexpr float kRescaleSlack = 8.0f;
 constexpr int kXchFloats = 34;
 constexpr int kXchSize = (kConsumerGroups - 1) * kKvHeads * 32 * kXchFloats;
 
+// Small per-item inputs staged in shared memory one item ahead by the
+// producer (bulk copies), so that neither the q set-up nor the new-token
+// append waits on DRAM while the cache stream saturates it.
+constexpr int kInQ = 0;          // q (bf16 [32][128]) or q_raw in the layer stack
+constexpr int kInWq = 8192;      // w_q  bf16 [128]
+constexpr int kInK = 8448;       // k_raw bf16 [4][128]
+constexpr int kInV = 9472;       // v_raw bf16 [4][128]
+constexpr int kInWk = 10496;     // w_k  bf16 [128]
+constexpr int kInBytes = 10752;
+constexpr int kAppendWarp = kConsumerWarps - 1;  // the consumer warp that appends
+
 struct Smem {
   uint8_t* stages;
   uint64_t* full;
   uint64_t* empty;
+  uint64_t* in_full;    // item inputs landed
+  uint64_t* in_empty;   // item inputs consumed
   float2* cs;
-  volatile int* flags;  // [0] abort, [1] last-arrival broadcast
+  volatile int* flags;  // [0] abort, [1] last-arrival broadcast, [2] grid barrier,
+                        // [3] item whose new token is in the cache (+1)
   float* xch;           // group hand-over area
+  uint8_t* in;          // item inputs
 };
 
 __device__ __forceinline__ Smem carve(uint8_t* raw) {
@@ -69,9 +86,12 @@ __device__ __forceinline__ Smem carve(uint8_t* raw) {
   s.stages = base;
   s.full = reinterpret_cast<uint64_t*>(base + kStages * kStageBytes);
   s.empty = s.full + kStages;
-  s.cs = reinterpret_cast<float2*>(s.empty + kStages);
+  s.in_full = s.empty + kStages;
+  s.in_empty = s.in_full + 1;
+  s.cs = reinterpret_cast<float2*>(s.in_empty + 1);
   s.flags = reinterpret_cast<volatile int*>(s.cs + 64);
   s.xch = reinterpret_cast<float*>(s.cs + 64) + 4;
+  s.in = reinterpret_cast<uint8_t*>(s.xch + kXchSize);  // 16-byte aligned
   return s;
 }
 
@@ -101,28 +121,52 @@ __device__ __forceinline__ long long append_row(const Problem& pb) {
   return static_cast<long long>(pb.append_tok) * kKvHeads * kDim;
 }
 
-// Producer-warp side of the fused stack: norm (+RoPE) the new token's k for
-// every KV head, round to bf16 and write it and v_raw into the cache.
-__device__ void append_new_token(const DecodeParams& P, const Problem& pb, int lane,
-                                 const float2* cs) {
+// Fused layer stack, new token: norm (+RoPE) its k for every KV head from the
+// staged inputs, round to bf16 and write it and v_raw into the cache; then
+// order the writes before later TMA reads of those rows (async proxy).
+__device__ void append_new_token(const DecodeParams& P, const Problem& pb, const uint8_t* in,
+                                 int lane, const float2* cs) {
   const long long row = append_row(pb);
   if (row < 0) {
     if (lane == 0) report_error(P.dev_err, FLINT_ERR_INVALID_ARG);
     return;
   }
-#pragma unroll 1
+  const uint16_t* k_raw = reinterpret_cast<const uint16_t*>(in + kInK);
+  const uint16_t* w_k = reinterpret_cast<const uint16_t*>(in + kInWk);
+  const uint32_t* v_raw = reinterpret_cast<const uint32_t*>(in + kInV);
+#pragma unroll
   for (int g = 0; g < kKvHeads; ++g) {
     float y[4];
-    norm_rope_row_warp(pb.k_raw + g * kDim, pb.w_k, P.eps, true, pb.rope != 0, cs, lane, y);
+    norm_rope_row_warp(k_raw + g * kDim, w_k, P.eps, true, pb.rope != 0, cs, lane, y);
     uint32_t* kd = reinterpret_cast<uint32_t*>(pb.k_rows + row + g * kDim);
     uint32_t* vd = reinterpret_cast<uint32_t*>(pb.v_rows + row + g * kDim);
-    const uint32_t* vs = reinterpret_cast<const uint32_t*>(pb.v_raw + g * kDim);
     kd[lane] = pack_bf16x2(y[0], y[1]);
     kd[32 + lane] = pack_bf16x2(y[2], y[3]);
-    vd[lane] = vs[lane];
-    vd[32 + lane] = vs[32 + lane];
+    vd[lane] = v_raw[g * 64 + lane];
+    vd[32 + lane] = v_raw[g * 64 + 32 + lane];
   }
   fence_proxy_async_global();
+}
+
+// Producer: stage an item's small inputs (q or q_raw, norm weights, k_raw,
+// v_raw) in shared memory with bulk copies completing on in_full.
+__device__ __forceinline__ void issue_item_inputs(const DecodeParams& P, const Problem& pb,
+                                                  const Smem& S) {
+  const uint32_t fb = smem_u32(S.in_full);
+  const uint32_t dst = smem_u32(S.in);
+  if (P.prep) {
+    mbar_expect_tx(fb, kInBytes);
+    bulk_copy_g2s(dst + kInQ, pb.q, 8192, fb);
+    bulk_copy_g2s(dst + kInWq, pb.w_q, 256, fb);
+    bulk_copy_g2s(dst + kInK, pb.k_raw, 1024, fb);
+    bulk_copy_g2s(dst + kInV, pb.v_raw, 1024, fb);
+    bulk_copy_g2s(dst + kInWk, pb.w_k, 256, fb);
+  } else if (!pb.q_fp32) {
+    mbar_expect_tx(fb, 8192);
+    bulk_copy_g2s(dst + kInQ, pb.q, 8192, fb);
+  } else {
+    mbar_arrive(fb);  // fp32 q is read from global memory
+  }
 }
 
 // Returns the number of tiles whose loads were issued.
@@ -136,6 +180,17 @@ __device__ int run_producer(const DecodeParams& P, const Smem& S, int it0, int i
     const CUtensorMap* map = &P.maps[my_kv ? pb.map_v : pb.map_k];
     const bool paged = pb.layout == FLINT_KV_PAGED;
     const int app_tile = (P.prep && pb.append_tok >= 0) ? (pb.append_tok - pb.tile_base) / kTile : -1;
+    {  // stage this item's small inputs once the consumers released the last ones
+      const uint32_t ph = static_cast<uint32_t>(it - it0) & 1u;
+      bool ok = mbar_wait(smem_u32(S.in_empty), ph ^ 1u, S.flags);
+      ok = __all_sync(0xffffffffu, ok);
+      if (!ok) {
+        if (lane == 0) abort_cta(P, S);
+        return seq;
+      }
+      if (lane == 0) issue_item_inputs(P, pb, S);
+      __syncwarp();
+    }
     for (int t = item.t0; t < item.t1; t += 32) {
       const int n = min(32, item.t1 - t);
       int blk = 0;
@@ -157,8 +212,23 @@ __device__ int run_producer(const DecodeParams& P, const Smem& S, int it0, int i
         }
         const int tile = t + j;
         if (tile == app_tile) {
-          append_new_token(P, pb, lane, S.cs);
-          __syncwarp();
+          // the new token's rows are written by a consumer warp: wait for them
+          bool done = true;
+          if (lane == 0) {
+            const unsigned long long t0 = globaltimer_ns();
+            while (S.flags[3] != it + 1) {
+              if (S.flags[0] || globaltimer_ns() - t0 > kWaitLimitNs) {
+                done = false;
+                break;
+              }
+            }
+            __threadfence_block();
+          }
+          done = __shfl_sync(0xffffffffu, done, 0);
+          if (!done) {
+            if (lane == 0) abort_cta(P, S);
+            return seq;
+          }
         }
         const uint32_t fb = smem_u32(&S.full[stage]);
         const uint32_t base = smem_u32(S.stages + stage * kStageBytes);
@@ -189,11 +259,11 @@ __device__ int run_producer(const DecodeParams& P, const Smem& S, int it0, int i
 // q fragments for query head h: thread (g = lane/4, c = lane%4) holds dims
 // 16kk + 2c + {0,1} and 16kk + 2c + 8 + {0,1} for kk = 0..7 as the A operand
 // rows g (bf16 hi part) and g + 8 (bf16 lo part), prescaled by log2(e)/sqrt(128).
-__device__ __forceinline__ void load_q(const DecodeParams& P, const Problem& pb, int h, int c,
-                                       const float2* cs, uint32_t (&qa)[8][4]) {
+__device__ __forceinline__ void load_q(const DecodeParams& P, const Problem& pb, const uint8_t* in,
+                                       int h, int c, const float2* cs, uint32_t (&qa)[8][4]) {
   float x[8][4];
   if (P.prep || !pb.q_fp32) {
-    const uint16_t* q = static_cast<const uint16_t*>(pb.q) + h * kDim;
+    const uint16_t* q = reinterpret_cast<const uint16_t*>(in + kInQ) + h * kDim;
 #pragma unroll
     for (int kk = 0; kk < 8; ++kk) {
       const uint32_t a = *reinterpret_cast<const uint32_t*>(q + 16 * kk + 2 * c);
@@ -228,8 +298,9 @@ __device__ __forceinline__ void load_q(const DecodeParams& P, const Problem& pb,
     const float r = 1.0f / sqrtf(ss * (1.0f / kDim) + P.eps);
 #pragma unroll
     for (int kk = 0; kk < 8; ++kk) {
-      const uint32_t a = *reinterpret_cast<const uint32_t*>(pb.w_q + 16 * kk + 2 * c);
-      const uint32_t b = *reinterpret_cast<const uint32_t*>(pb.w_q + 16 * kk + 2 * c + 8);
+      const uint16_t* w_q = reinterpret_cast<const uint16_t*>(in + kInWq);
+      const uint32_t a = *reinterpret_cast<const uint32_t*>(w_q + 16 * kk + 2 * c);
+      const uint32_t b = *reinterpret_cast<const uint32_t*>(w_q + 16 * kk + 2 * c + 8);
       x[kk][0] = x[kk][0] * r * bf16_lo(a);
       x[kk][1] = x[kk][1] * r * bf16_hi(a);
       x[kk][2] = x[kk][2] * r * bf16_lo(b);
@@ -372,7 +443,26 @@ __device__ void run_consumer(const DecodeParams& P, const Smem& S, int it0, int 
     const Problem& pb = P.prob[item.seg];
 
     uint32_t qa[8][4];
-    load_q(P, pb, head, c, S.cs, qa);
+    {
+      const uint32_t ph = static_cast<uint32_t>(it - it0) & 1u;
+      bool ok = mbar_wait(smem_u32(S.in_full), ph, S.flags);
+      ok = __all_sync(0xffffffffu, ok);
+      if (!ok && lane == 0) abort_cta(P, S);
+      load_q(P, pb, S.in, head, c, S.cs, qa);
+      if (P.prep && warp == kAppendWarp && pb.append_tok >= 0) {
+        const int app_tile = (pb.append_tok - pb.tile_base) / kTile;
+        if (app_tile >= item.t0 && app_tile < item.t1) {
+          append_new_token(P, pb, S.in, lane, S.cs);
+          __syncwarp();
+          if (lane == 0) {
+            __threadfence_block();
+            S.flags[3] = it + 1;
+          }
+        }
+      }
+      __syncwarp();
+      if (lane == 0) mbar_arrive(smem_u32(S.in_empty));
+    }
 
     float m_run = -INFINITY, l_run = 0.f;
     float o[16][4];
@@ -455,6 +545,11 @@ __device__ void run_consumer(const DecodeParams& P, const Smem& S, int it0, int 
       }
     }
     __threadfence();
+    if (pb.deferred) {  // merged by the whole grid after the grid barrier
+      __syncwarp();
+      consumer_bar();
+      continue;
+    }
     __syncwarp();
     consumer_bar();
     if (threadIdx.x == 0) {
@@ -466,7 +561,8 @@ __device__ void run_consumer(const DecodeParams& P, const Smem& S, int it0, int 
     __syncwarp();
     consumer_bar();
     if (S.flags[1] && group == 0) {
-      // last arrival: merge every partial of the problem, in item order
+      // last arrival: merge every partial of the problem, in item order,
+      // four partials' loads in flight at a time
       __threadfence();
       float M = -INFINITY;
       for (int i = s0; i < s1; ++i)
@@ -474,19 +570,30 @@ __device__ void run_consumer(const DecodeParams& P, const Smem& S, int it0, int 
       float L = 0.f;
 #pragma unroll
       for (int e = 0; e < 32; ++e) v[e] = 0.f;
-      for (int i = s0; i < s1; ++i) {
-        const float* pi = P.partials + static_cast<size_t>(i) * kPartialFloats;
-        const float mi = __ldcg(pi + kHeads * kDim + head);
-        const float si = (mi == -INFINITY) ? 0.f : exp2f(mi - M);
-        L += si * __ldcg(pi + kHeads * kDim + kHeads + head);
-        const float4* po = reinterpret_cast<const float4*>(pi + partial_o(head, c));
+      for (int i0 = s0; i0 < s1; i0 += 4) {
+        float sw[4], lw[4];
+        float4 ow[4][8];
 #pragma unroll
-        for (int q = 0; q < 8; ++q) {
-          const float4 a = __ldcg(po + q);
-          v[4 * q] += si * a.x;
-          v[4 * q + 1] += si * a.y;
-          v[4 * q + 2] += si * a.z;
-          v[4 * q + 3] += si * a.w;
+        for (int j = 0; j < 4; ++j) {
+          const int i = min(i0 + j, s1 - 1);
+          const float* pi = P.partials + static_cast<size_t>(i) * kPartialFloats;
+          const float mi = __ldcg(pi + kHeads * kDim + head);
+          sw[j] = (i0 + j >= s1 || mi == -INFINITY) ? 0.f : exp2f(mi - M);
+          lw[j] = __ldcg(pi + kHeads * kDim + kHeads + head);
+          const float4* po = reinterpret_cast<const float4*>(pi + partial_o(head, c));
+#pragma unroll
+          for (int q = 0; q < 8; ++q) ow[j][q] = __ldcg(po + q);
+        }
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+          L += sw[j] * lw[j];
+#pragma unroll
+          for (int q = 0; q < 8; ++q) {
+            v[4 * q] += sw[j] * ow[j][q].x;
+            v[4 * q + 1] += sw[j] * ow[j][q].y;
+            v[4 * q + 2] += sw[j] * ow[j][q].z;
+            v[4 * q + 3] += sw[j] * ow[j][q].w;
+          }
         }
       }
       finish_head(pb, head, c, M, L, v);
@@ -497,13 +604,128 @@ __device__ void run_consumer(const DecodeParams& P, const Smem& S, int it0, int 
   }
 }
 
+// Grid-wide barrier for a cooperative launch: block 0 adds 2^31 - (G - 1),
+// the others add 1, so bit 31 of the word flips once all G blocks arrived and
+// its low bits return to their start value (zero in a fresh workspace).
+// Bounded: returns false after the time limit.
+__device__ bool grid_barrier(unsigned int* bar, const Smem& S) {
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    __threadfence();
+    const unsigned int add = blockIdx.x == 0 ? 0x80000000u - (gridDim.x - 1) : 1u;
+    const unsigned int old = atomicAdd(bar, add);
+    const unsigned long long t0 = globaltimer_ns();
+    int ok = 1;
+    for (;;) {
+      unsigned int cur;
+      asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(cur) : "l"(bar) : "memory");
+      if ((cur ^ old) & 0x80000000u) break;
+      if (globaltimer_ns() - t0 > kWaitLimitNs) {
+        ok = 0;
+        break;
+      }
+      __nanosleep(64);
+    }
+    __threadfence();
+    S.flags[2] = ok;
+  }
+  __syncthreads();
+  return S.flags[2] != 0;
+}
+
+// Merge of the deferred problems by the whole grid: one CTA per (problem,
+// head, quarter c) unit, every thread folding in its own partials (one or two:
+// a problem has at most one partial per CTA), so all loads of a unit are in
+// flight at once; then a block reduction.  Value k of a quarter is dim
+// 8(k/2) + 2c + (k & 1) of the head.
+__device__ void grid_merge(const DecodeParams& P, const Smem& S) {
+  constexpr int kWarps = kThreads / 32;
+  const int t = threadIdx.x, lane = t & 31, warp = t >> 5;
+  float* red = S.xch;  // [kWarps][34] scratch (the hand-over area is free now)
+  const int units = P.n_deferred * kHeads * 4;
+  for (int u = blockIdx.x; u < units; u += gridDim.x) {
+    const int p = P.deferred[u / (kHeads * 4)];
+    const int head = (u / 4) % kHeads, c = u % 4;
+    const Problem& pb = P.prob[p];
+    const int s0 = P.seg_item_begin[p], s1 = P.seg_item_begin[p + 1];
+    float m = -INFINITY, l = 0.f, v[32];
+#pragma unroll
+    for (int e = 0; e < 32; ++e) v[e] = 0.f;
+    for (int i = s0 + t; i < s1; i += kThreads) {
+      const float* pi = P.partials + static_cast<size_t>(i) * kPartialFloats;
+      const float mi = __ldcg(pi + kHeads * kDim + head);
+      const float li = __ldcg(pi + kHeads * kDim + kHeads + head);
+      const float4* po = reinterpret_cast<const float4*>(pi + partial_o(head, c));
+      float4 ov[8];
+#pragma unroll
+      for (int q = 0; q < 8; ++q) ov[q] = __ldcg(po + q);
+      const float mn = fmaxf(m, mi);
+      const float sa = (m == -INFINITY) ? 0.f : exp2f(m - mn);
+      const float sb = (mi == -INFINITY) ? 0.f : exp2f(mi - mn);
+#pragma unroll
+      for (int q = 0; q < 8; ++q) {
+        v[4 * q] = v[4 * q] * sa + ov[q].x * sb;
+        v[4 * q + 1] = v[4 * q + 1] * sa + ov[q].y * sb;
+        v[4 * q + 2] = v[4 * q + 2] * sa + ov[q].z * sb;
+        v[4 * q + 3] = v[4 * q + 3] * sa + ov[q].w * sb;
+      }
+      l = l * sa + li * sb;
+      m = mn;
+    }
+    // block max of m
+    float M = m;
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, o));
+    if (lane == 0) red[warp] = M;
+    __syncthreads();
+    M = red[0];
+#pragma unroll
+    for (int w = 1; w < kWarps; ++w) M = fmaxf(M, red[w]);
+    __syncthreads();
+    const float sc = (m == -INFINITY) ? 0.f : exp2f(m - M);
+    l *= sc;
+#pragma unroll
+    for (int e = 0; e < 32; ++e) v[e] *= sc;
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) l += __shfl_xor_sync(0xffffffffu, l, o);
+    // warp reduce-scatter: afterwards lane k holds the warp's sum of value k
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) {
+      const bool up = (lane & o) != 0;
+#pragma unroll
+      for (int j = 0; j < o; ++j) {
+        const float send = up ? v[j] : v[j + o];
+        const float keep = up ? v[j + o] : v[j];
+        v[j] = keep + __shfl_xor_sync(0xffffffffu, send, o);
+      }
+    }
+    red[warp * 34 + lane] = v[0];
+    if (lane == 0) red[warp * 34 + 32] = l;
+    __syncthreads();
+    if (t < 32) {
+      float sum = 0.f, L = 0.f;
+#pragma unroll
+      for (int w = 0; w < kWarps; ++w) {
+        sum += red[w * 34 + t];
+        L += red[w * 34 + 32];
+      }
+      const float s2 = pb.sinks[head] * kLog2e;
+      const float Mf = fmaxf(M, s2);
+      const float a = (M == -INFINITY) ? 0.f : exp2f(M - Mf);
+      const float scale = a / (L * a + exp2f(s2 - Mf));
+      pb.out[head * kDim + 8 * (t >> 1) + 2 * c + (t & 1)] = sum * scale;
+    }
+    __syncthreads();  // red is reused by the next unit
+  }
+}
+
 __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const __grid_constant__ DecodeParams P) {
   extern __shared__ uint8_t smem_raw[];
   const Smem S = carve(smem_raw);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   int it0 = P.cta_item_begin[blockIdx.x], it1 = P.cta_item_begin[blockIdx.x + 1];
   if (!FLINT_CHECK(P.dev_err, 0 <= it0 && it0 <= it1 && it1 <= P.n_items, 1, it0, it1, P.n_items)) it1 = it0;
-  const int smem_end = static_cast<int>(smem_u32(S.xch + kXchSize) - smem_u32(smem_raw));
+  const int smem_end = static_cast<int>(smem_u32(S.in + kInBytes) - smem_u32(smem_raw));
   if (!FLINT_CHECK(P.dev_err, smem_end <= P.smem_bytes, 2, smem_end, P.smem_bytes, 0)) it1 = it0;
   (void)smem_end;
 
@@ -512,8 +734,11 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const __grid_consta
       mbar_init(smem_u32(&S.full[s]), 1);
       mbar_init(smem_u32(&S.empty[s]), kConsumerWarps);
     }
+    mbar_init(smem_u32(S.in_full), 1);
+    mbar_init(smem_u32(S.in_empty), kConsumerWarps);
     S.flags[0] = 0;
     S.flags[1] = 0;
+    S.flags[3] = 0;
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
     asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
   }
@@ -530,6 +755,12 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const __grid_consta
   // After an abort, let every issued load land before the CTA's shared memory
   // goes away (bounded as well; a normal run returns at once).
   if (warp == kConsumerWarps && lane == 0) {
+    if (it1 > it0) {  // the last staged inputs
+      const unsigned long long t0 = globaltimer_ns();
+      while (!mbar_try_wait(smem_u32(S.in_full), static_cast<uint32_t>(it1 - it0 - 1) & 1u)) {
+        if (globaltimer_ns() - t0 > kWaitLimitNs) break;
+      }
+    }
     const int first = issued > kStages ? issued - kStages : 0;
     for (int s = first; s < issued; ++s) {
       const unsigned long long t0 = globaltimer_ns();
@@ -538,13 +769,21 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const __grid_consta
       }
     }
   }
+  if (P.grid_merge) {
+    if (grid_barrier(reinterpret_cast<unsigned int*>(P.counters + kMaxSegs), S)) {
+      grid_merge(P, S);
+    } else if (threadIdx.x == 0) {
+      report_error(P.dev_err, FLINT_ERR_TIMEOUT);
+    }
+  }
 }
 
 }  // namespace
 
 size_t decode_smem_bytes() {
   return 1024 + static_cast<size_t>(kStages) * kStageBytes + 2 * kStages * sizeof(uint64_t) +
-         64 * sizeof(float2) + 4 * sizeof(int) + kXchSize * sizeof(float);
+         2 * sizeof(uint64_t) + 64 * sizeof(float2) + 4 * sizeof(int) + kXchSize * sizeof(float) +
+         kInBytes;
 }
 
 cudaError_t launch_decode(const DecodeParams& p, int grid, cudaStream_t stream) {
@@ -558,7 +797,15 @@ cudaError_t launch_decode(const DecodeParams& p, int grid, cudaStream_t stream) 
     if (e != cudaSuccess) return e;
     configured_device = dev;
   }
-  decode_kernel<<<grid, kThreads, decode_smem_bytes(), stream>>>(p);
+  if (p.grid_merge) {
+    // the grid barrier needs every CTA resident at once
+    void* args[] = {const_cast<DecodeParams*>(&p)};
+    e = cudaLaunchCooperativeKernel(reinterpret_cast<const void*>(decode_kernel), dim3(grid),
+                                    dim3(kThreads), args, decode_smem_bytes(), stream);
+    if (e != cudaSuccess) return e;
+  } else {
+    decode_kernel<<<grid, kThreads, decode_smem_bytes(), stream>>>(p);
+  }
   return cudaGetLastError();
 }
 

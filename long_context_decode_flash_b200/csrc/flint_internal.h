@@ -52,6 +52,11 @@ constexpr int kMaxMaps = 2 * FLINT_MAX_LAYERS;
 constexpr int kMaxItems = 512;
 constexpr int kMaxCtas = 296;
 
+// A problem split into more than kInlineMergeMax items is not merged by its
+// last-arriving CTA (one CTA reading every partial would be the tail of the
+// launch) but by all warps of the grid after a grid barrier.
+constexpr int kInlineMergeMax = 16;
+
 // One split partial of a problem: O for 32 heads (stored so that each
 // consumer thread's 32 values are contiguous), m [32] (log2 units), l [32].
 constexpr int kPartialFloats = kHeads * kDim + 2 * kHeads;
@@ -78,7 +83,8 @@ struct Problem {
   int32_t table_len;        // PAGED: entries in this request's block-table row
   int16_t map_k, map_v;     // tensor-map indices
   int16_t req;              // 4th tensor coordinate (request) for CONTIGUOUS/RING
-  int8_t layout, q_fp32, rope, pad;
+  int8_t layout, q_fp32, rope;
+  int8_t deferred;          // 1: merged by the whole grid after a grid barrier
 };
 
 struct Item {
@@ -101,6 +107,9 @@ struct DecodeParams {
   int32_t n_problems;
   int32_t prep;             // 1: q/k norm (+RoPE) and append fused in (layer stack)
   int32_t n_items;          // items in the plan
+  int32_t grid_merge;       // 1: some problem is deferred (cooperative launch)
+  int16_t deferred[kMaxProblems];  // the deferred problems
+  int32_t n_deferred;
   int32_t ws_items;         // partial slots in the workspace
   int32_t smem_bytes;       // dynamic shared memory of the launch
 };
@@ -130,7 +139,7 @@ struct PrepParams {
 };
 
 // Launchers (return cudaGetLastError() after the launch).
-cudaError_t launch_decode(const DecodeParams& p, int grid, cudaStream_t stream);
+cudaError_t launch_decode(const DecodeParams& p, int grid, cudaStream_t stream);  // cooperative if p.grid_merge
 cudaError_t launch_prep(const PrepParams& p, int B, cudaStream_t stream);
 
 size_t decode_smem_bytes();
