@@ -58,6 +58,7 @@ extern "C" {
 #define FLINT_MAX_CONTEXT 262144  /* "maxContext" of the model JSON */
 #define FLINT_MAX_BATCH 64        /* requests per flint_attn_decode launch */
 #define FLINT_MAX_LAYERS 49       /* layers per flint_attn_stack call */
+#define FLINT_NOALLOC_SCRATCH_BYTES (4u << 20)  /* flint_attn_stack_noalloc's fixed scratch */
 
 typedef enum {
     FLINT_OK = 0,
@@ -193,6 +194,27 @@ flint_status flint_attn_stack(const flint_layer* layers, int32_t n_layers, int32
                               float eps, double theta, float* out, void* workspace,
                               size_t ws_bytes, int32_t num_ctas, int32_t* dev_err,
                               void* stream);
+
+/* flint_attn_stack without a workspace argument, for callers that cannot
+ * allocate device memory (a runtime that owns all of it through its own pool,
+ * a plug-in handed buffers but no allocator).  No counterpart in the paper: it
+ * changes where the scratch lives, not what is computed; the results are
+ * those of flint_attn_stack.
+ *   Scratch: the library holds one FLINT_NOALLOC_SCRATCH_BYTES array in the
+ *   device memory of every device its device code is loaded on, until the
+ *   process exits.  Calls needing more, i.e. whenever
+ *   flint_attn_workspace_bytes(n_layers, num_ctas) exceeds it, are refused
+ *   with FLINT_ERR_WORKSPACE (49 layers fit with up to 202 CTAs).
+ *   Set-up: the first call on a device, with that device current, looks up the
+ *   scratch's address; make it before any stream capture.
+ *   Sharing: every call on a device uses the same scratch, which keeps the last
+ *   call's contents; each call clears the counters it needs on `stream` first.
+ *   Calls that overlap on the GPU (other streams, other threads) race.
+ * Allocates nothing: no cudaMalloc, cudaFree or allocating library routine.
+ * Other arguments, errors and the append are those of flint_attn_stack. */
+flint_status flint_attn_stack_noalloc(const flint_layer* layers, int32_t n_layers,
+                                      int32_t pos, float eps, double theta, float* out,
+                                      int32_t num_ctas, int32_t* dev_err, void* stream);
 
 /* The split planner behind both attention calls (pure host code, exposed for
  * tests).  Work is n_segs segments (one per problem and KV head) of

@@ -275,6 +275,20 @@ flint_status launch_result(cudaError_t e, const char* who) {
 
 }  // namespace
 
+namespace flint {
+
+flint_status record_error(flint_status s, const char* fmt, ...) {
+  char buf[512];
+  va_list ap;
+  va_start(ap, fmt);
+  vsnprintf(buf, sizeof buf, fmt, ap);
+  va_end(ap);
+  g_last_error = buf;
+  return s;
+}
+
+}  // namespace flint
+
 extern "C" {
 
 const char* flint_status_string(flint_status s) {

@@ -144,4 +144,7 @@ cudaError_t launch_prep(const PrepParams& p, int B, cudaStream_t stream);
 
 size_t decode_smem_bytes();
 
+// Sets the message that flint_last_error() returns on this thread; returns s.
+flint_status record_error(flint_status s, const char* fmt, ...);
+
 }  // namespace flint
