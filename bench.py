@@ -8,8 +8,9 @@ with its own bf16 KV cache), on B200s.
 Prints one JSON line (rank 0).  A step is one call of flint_attn_stack: for
 every layer the fused Q/K RMSNorm (+RoPE), KV append at position 99,999 and
 split-KV decode with sinks, in one kernel launch.  `value` is device time per
-decoded token (CUDA events on the launching stream, L2 flushed by a 256 MiB
-write before every step, max over ranks / tokens of all ranks).  Under
+decoded token (CUDA events on the launching stream; before every step the L2
+is flushed by a 256 MiB write and a 256 MiB read of another buffer; max over
+ranks / tokens of all ranks).  Under
 torchrun each rank decodes its own independent token (weak scaling; there is
 no data-path collective).  `--impl reference` times the float64 CPU oracle on
 the host cores instead (bounded sample, scaled to the same unit).
@@ -31,6 +32,29 @@ sys.path.insert(0, ROOT)
 METRIC = "49-layer decode-attention µs/token @100K ctx bs=1; achieved HBM GB/s vs peak"
 CONTEXT = 100_000
 NOMINAL_HBM_GBS = 8000.0
+
+# DRAM traffic (dram__bytes_read.sum + dram__bytes_write.sum) of one decode_kernel
+# launch from a full-size, one-pass ncu capture of the stack at context 100,000
+# (profiles/decode_kernel_stack100k_traffic.md), with the hash of the CUDA
+# sources it was taken on; reported only while the sources still hash the same.
+TRAFFIC = {("stack", 100_000): (2_910_000_000 + 4_770_000, "f04e15c1a173b08e")}
+
+
+def kernel_sources_hash() -> str:
+    import hashlib
+    d = os.path.join(ROOT, "long_context_decode_flash_b200", "csrc")
+    m = hashlib.sha256()
+    for f in sorted(os.listdir(d)):
+        if f.endswith((".cu", ".cuh", ".h", ".cpp")):
+            m.update(f.encode())
+            with open(os.path.join(d, f), "rb") as fh:
+                m.update(fh.read())
+    return m.hexdigest()[:16]
+
+
+def traffic_for(workload: str, ctx: int):
+    t = TRAFFIC.get((workload, ctx))
+    return t[0] if t is not None and t[1] == kernel_sources_hash() else None
 FALLBACK_HBM_GBS = 6650.0
 
 
@@ -131,7 +155,8 @@ def run_reference(args, rank):
 # ------------------------------------------------------------- GPU side ----
 
 def workload_config(name):
-    base = {"l2": "flushed before every step (256 MiB write)", "batch": 1}
+    base = {"l2": "flushed before every step (256 MiB write, then 256 MiB read of another buffer)",
+            "batch": 1}
     if name == "stack":
         return dict(base, workload="49-layer decode-attention stack for one token: 35 sliding-window "
                     "(513, RoPE) + 14 full-context NoPE layers, GQA 32q/4kv x 128, sinks",
@@ -284,7 +309,17 @@ def main():
     dev_index = torch.cuda.current_device()
     stream = torch.cuda.current_stream()
 
+    # L2 flush between steps: a 256 MiB write (twice the L2), then a 256 MiB
+    # read of a second buffer, so that the L2 holds only clean lines of
+    # unrelated data when a step starts; without the read, the write-back of
+    # the dirty flush lines would land inside the next timed step.
     flush = torch.empty(256 * 1024 * 1024 // 4, dtype=torch.float32, device="cuda")
+    flush_rd = torch.ones(256 * 1024 * 1024 // 4, dtype=torch.float32, device="cuda")
+    flush_acc = torch.zeros(1, dtype=torch.float32, device="cuda")
+
+    def flush_l2(i):
+        flush.fill_(float(i))
+        torch.sum(flush_rd, dim=0, keepdim=True, out=flush_acc)
     err = torch.zeros(1, dtype=torch.int32, device="cuda")
 
     if layers is not None:
@@ -313,7 +348,7 @@ def main():
     d2h = host_out.numel() * 4
 
     for _ in range(max(args.warmup, 3)):
-        flush.fill_(1.0)
+        flush_l2(1)
         step()
     torch.cuda.synchronize()
     if int(err.item()) != 0:
@@ -337,7 +372,7 @@ def main():
         launch = "direct launches"
     run = graph.replay if graph is not None else step
     for _ in range(3):
-        flush.fill_(1.0)
+        flush_l2(1)
         run()
     torch.cuda.synchronize()
     # host cost of one public-API call (argument marshalling, plan, launch)
@@ -355,7 +390,7 @@ def main():
     with ClockSampler(dev_index) as clocks:
         t_wall = time.perf_counter()
         for i in range(args.steps):
-            flush.fill_(float(i))
+            flush_l2(i)
             starts[i].record(stream)
             run()
             ends[i].record(stream)
@@ -377,7 +412,7 @@ def main():
             torch.distributed.barrier()
         torch.cuda.synchronize()
         for i in range(args.steps):
-            flush.fill_(float(i))
+            flush_l2(i)
             e_s[i].record(stream)
             packed.copy_(host_in, non_blocking=True)
             step()
@@ -412,7 +447,7 @@ def main():
                      "frac": achieved / peak, "peak_kind": peak_kind,
                      "frac_of_nominal_8000": achieved / NOMINAL_HBM_GBS,
                      "algorithmic_bytes": int(algo_bytes), "kernel": "flint decode_kernel",
-                     "traffic": None},
+                     "traffic": traffic_for(args.workload, ctx)},
         "cpu_baseline": cpu_baseline,
         "e2e": e2e,
         "gpu_launches": args.steps,

@@ -217,8 +217,8 @@ flint_status flint_attn_stack_noalloc(const flint_layer* layers, int32_t n_layer
                                       int32_t num_ctas, int32_t* dev_err, void* stream);
 
 /* The split planner behind both attention calls (pure host code, exposed for
- * tests).  Work is n_segs segments (one per problem and KV head) of
- * seg_tiles[s] 64-token tiles; it is cut into items (segment, tile range)
+ * tests).  Work is n_segs segments (one per problem, all four KV heads
+ * together) of seg_tiles[s] 32-token tiles; it is cut into items (segment, tile range)
  * laid over num_ctas CTAs so that tiles + item_cost per item are level.
  * Outputs: item_seg/item_t0/item_t1 [max_items], cta_begin [num_ctas+1]
  * (items of CTA c are cta_begin[c] .. cta_begin[c+1]-1; the items of one

@@ -101,7 +101,8 @@ struct MapKeyHash {
 // A K or V cache seen as a 4-D bf16 tensor (dims innermost first):
 //   CONTIGUOUS/RING: [128 dims][4 heads][capacity tokens][B requests]
 //   PAGED:           [128 dims][4 heads][64 tokens][num_blocks]
-// read in boxes of 64 dims x 1 head x 64 tokens x 1 with the 128-byte swizzle.
+// read in boxes of 64 dims x 1 head x kTile (32) tokens x 1 with the 128-byte
+// swizzle.
 flint_status encode_cache_map(CUtensorMap* map, void* base, const flint_kv_cache& c, int B) {
   EncodeTiledFn fn = encode_fn();
   if (!fn) return fail(FLINT_ERR_CUDA, "cuTensorMapEncodeTiled is not available from the driver");

@@ -1,7 +1,7 @@
 // flint_plan.cpp -- the split-KV work planner (pure host code).
 //
-// Work arrives as segments: one per (problem, KV head), each a run of 64-token
-// tiles.  The planner lays the concatenated segments over the CTAs of one
+// Work arrives as segments: one per problem (a layer, or a request), each a
+// run of 32-token tiles that cover all four KV heads.  The planner lays the concatenated segments over the CTAs of one
 // launch so that every CTA carries the same cost, where an item (a tile range
 // of one segment on one CTA) costs its tiles plus a fixed per-item overhead
 // (q set-up, merge, partial write).  Segments are cut only at CTA boundaries
