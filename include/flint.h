@@ -151,14 +151,17 @@ flint_status flint_kv_append(const uint16_t* k, const uint16_t* v, const int32_t
                              int32_t B, const flint_kv_cache* cache, int32_t* dev_err,
                              void* stream);
 
-/* Bytes of device workspace that flint_attn_decode / flint_attn_stack need
- * for n_problems (requests, or layers) on a grid of num_ctas CTAs (0 = the
- * current device's default).  The workspace holds split partials, per-problem
- * arrival counters and a grid-barrier word; it must be zero-filled before its
- * first use, and every call that completes without a device error leaves it
- * ready for the next call (counters back at zero).  After a device error,
- * zero it again.  Calls that share a workspace must not overlap in time.
- * Returns 0 for invalid arguments. */
+/* Bytes of device workspace for flint_attn_decode / flint_attn_stack with
+ * n_problems (requests, or layers) on num_ctas CTAs (0 = one per SM): room
+ * for the full split plan, 4096 + 640 * 16640 bytes (10.6 MB).  A call also
+ * runs with less, down to 4096 + (CTAs + n_problems) * 16640 bytes, with a
+ * coarser run-time balancing queue; below that it returns
+ * FLINT_ERR_WORKSPACE.  The workspace holds split partials, per-problem
+ * arrival counters, a grid-barrier word and the queue head; it must be
+ * zero-filled before its first use, and every call that completes without a
+ * device error leaves it ready for the next call (counters back at zero).
+ * After a device error, zero it again.  Calls that share a workspace must not
+ * overlap in time.  Returns 0 for invalid arguments. */
 size_t flint_attn_workspace_bytes(int32_t n_problems, int32_t num_ctas);
 
 /* Split-KV flash-decode over a batch of B requests of one layer: q already
@@ -174,7 +177,9 @@ size_t flint_attn_workspace_bytes(int32_t n_problems, int32_t num_ctas);
  *   out       fp32 [B][32][128] (device)
  *   workspace device, >= flint_attn_workspace_bytes(B, num_ctas) bytes
  *   num_ctas  0 = one CTA per SM (the tuned default)
- * B in [1, FLINT_MAX_BATCH].  Result is deterministic run to run. */
+ * B in [1, FLINT_MAX_BATCH].  Result is deterministic run to run for a given
+ * workspace size and num_ctas: queued chunks have fixed bounds, whichever CTA
+ * takes them, and partials are merged in a fixed order. */
 flint_status flint_attn_decode(const void* q, int32_t q_is_fp32,
                                const flint_kv_cache* cache, const int32_t* seq_lens,
                                int32_t B, const float* sinks, int32_t window,
@@ -202,9 +207,11 @@ flint_status flint_attn_stack(const flint_layer* layers, int32_t n_layers, int32
  * those of flint_attn_stack.
  *   Scratch: the library holds one FLINT_NOALLOC_SCRATCH_BYTES array in the
  *   device memory of every device its device code is loaded on, until the
- *   process exits.  Calls needing more, i.e. whenever
- *   flint_attn_workspace_bytes(n_layers, num_ctas) exceeds it, are refused
- *   with FLINT_ERR_WORKSPACE (49 layers fit with up to 202 CTAs).
+ *   process exits.  Calls whose smallest workspace,
+ *   4096 + (CTAs + n_layers) * 16640 bytes, exceeds it are refused with
+ *   FLINT_ERR_WORKSPACE (49 layers fit with up to 202 CTAs).  The scratch is
+ *   below flint_attn_workspace_bytes, so the run-time balancing queue is
+ *   coarser than with a full workspace (same results up to rounding order).
  *   Set-up: the first call on a device, with that device current, looks up the
  *   scratch's address; make it before any stream capture.
  *   Sharing: every call on a device uses the same scratch, which keeps the last
@@ -227,6 +234,24 @@ flint_status flint_attn_stack_noalloc(const flint_layer* layers, int32_t n_layer
 int32_t flint_plan_items(const int32_t* seg_tiles, int32_t n_segs, int32_t num_ctas,
                          int32_t item_cost, int32_t* item_seg, int32_t* item_t0,
                          int32_t* item_t1, int32_t* cta_begin, int32_t max_items);
+
+/* The full plan of one attention launch (pure host code, exposed for tests):
+ * when there are at least 64 tiles per CTA, the static plan of
+ * flint_plan_items over the first ~88 % of every segment of at least 64
+ * tiles (smaller ones stay whole), plus a queue of chunks that
+ * cut the remaining tails, in guided sizes (ceil(remaining tiles / num_ctas),
+ * at least 8), which CTAs claim at run time once their static lists are done.
+ * Coarser queues, then none, are used when max_items is too small; with
+ * fewer tiles per CTA the plan is static only.
+ * Outputs: item_seg/item_t0/item_t1 [max_items], sorted by (segment, t0);
+ * order [max_items] and cta_begin [num_ctas + 1]: the static items of CTA c
+ * are order[cta_begin[c] .. cta_begin[c+1]-1] and the queue is
+ * order[cta_begin[num_ctas] .. n-1].  Returns n, the item count, or -1 on bad
+ * arguments / no plan within max_items. */
+int32_t flint_plan_split(const int32_t* seg_tiles, int32_t n_segs, int32_t num_ctas,
+                         int32_t item_cost, int32_t max_items, int32_t* item_seg,
+                         int32_t* item_t0, int32_t* item_t1, int32_t* order,
+                         int32_t* cta_begin);
 
 #ifdef __cplusplus
 }

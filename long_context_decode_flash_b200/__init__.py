@@ -9,7 +9,7 @@ _BINDING_NAMES = (
     "flint_kv_bytes", "flint_qk_norm_rope", "flint_kv_append",
     "flint_attn_workspace_bytes", "flint_attn_decode", "flint_attn_stack",
     "flint_attn_stack_noalloc",
-    "flint_plan_items", "KVCache", "StackLayer",
+    "flint_plan_items", "flint_plan_split", "KVCache", "StackLayer",
 )
 
 __all__ = list(_BINDING_NAMES) + ["inputs"]

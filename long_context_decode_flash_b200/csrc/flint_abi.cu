@@ -39,6 +39,9 @@ flint_status ok() {
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
 constexpr int kItemCost = 2;  // per-item overhead in tile units (planner cost model)
+// A deferred problem with more partials than this is merged a CTA per unit
+// (thread per partial) instead of a warp per unit.
+constexpr int kWideMergeItems = 64;
 
 // ---- device properties (cached per device) --------------------------------
 
@@ -218,16 +221,20 @@ flint_status check_len(const flint_kv_cache& c, int L, int window, const char* w
   return FLINT_OK;
 }
 
-size_t workspace_bytes(int n_problems, int num_ctas) {
-  const int64_t items = std::min<int64_t>(kMaxItems, num_ctas + static_cast<int64_t>(n_problems));
-  return kCounterBytes + static_cast<size_t>(items) * kPartialFloats * sizeof(float);
-}
+constexpr size_t kPartialBytes = kPartialFloats * sizeof(float);
 
-// Fill plan fields of P from the problems' tile counts; returns the grid.
-flint_status plan(DecodeParams& P, const int* tiles, int n_problems, int num_ctas, int* grid) {
+// Fill plan fields of P from the problems' tile counts; returns the grid.  The
+// workspace must hold the static plan (at most G + n_problems - 1 items); the
+// run-time queue gets what the rest of it (and kMaxItems) allows.
+flint_status plan(DecodeParams& P, const int* tiles, int n_problems, int num_ctas, size_t ws_bytes,
+                  const char* who, int* grid) {
   int sms = num_ctas;
   if (sms == 0 && device_num_sms(&sms) != 0)
     return fail(FLINT_ERR_CUDA, "cannot query the SM count of the current device");
+  // One CTA fits an SM, and a launch that ends in a grid barrier needs all of
+  // them resident: never more CTAs than the device has SMs.
+  int dev_sms = 0;
+  if (num_ctas > 0 && device_num_sms(&dev_sms) == 0) sms = std::min(sms, dev_sms);
   sms = std::min(sms, kMaxCtas);
   int32_t seg_tiles[kMaxSegs];
   int64_t total = 0;
@@ -238,17 +245,26 @@ flint_status plan(DecodeParams& P, const int* tiles, int n_problems, int num_cta
   const int n_segs = n_problems;
   // at least two tiles of work per CTA, never more CTAs than the device's SMs
   const int G = static_cast<int>(std::max<int64_t>(1, std::min<int64_t>(sms, (total + 1) / 2)));
-  int32_t seg[kMaxItems], t0[kMaxItems], t1[kMaxItems], cb[kMaxCtas + 1];
-  const int n = flint_plan_items(seg_tiles, n_segs, G, kItemCost, seg, t0, t1, cb, kMaxItems);
-  if (n < 0) return fail(FLINT_ERR_UNSUPPORTED, "split plan does not fit one launch");
+  const size_t need = kCounterBytes + static_cast<size_t>(std::min(kMaxItems, G + n_problems)) * kPartialBytes;
+  if (ws_bytes < need)
+    return fail(FLINT_ERR_WORKSPACE, "%s: workspace of %zu bytes is below the %zu needed", who, ws_bytes, need);
+  const int cap = static_cast<int>(std::min<size_t>(kMaxItems, (ws_bytes - kCounterBytes) / kPartialBytes));
+  int32_t seg[kMaxItems], t0[kMaxItems], t1[kMaxItems], order[kMaxItems], cb[kMaxCtas + 1];
+  const int n = flint_plan_split(seg_tiles, n_segs, G, kItemCost, cap, seg, t0, t1, order, cb);
+  if (n < 0) return fail(FLINT_ERR_UNSUPPORTED, "%s: split plan does not fit one launch", who);
+  bool queued[kMaxSegs] = {};
   for (int i = 0; i < n; ++i) {
     P.items[i].seg = static_cast<int16_t>(seg[i]);
     P.items[i].t0 = static_cast<int16_t>(t0[i]);
     P.items[i].t1 = static_cast<int16_t>(t1[i]);
     P.items[i].pad = 0;
+    P.order[i] = static_cast<int16_t>(order[i]);
   }
   P.n_items = n;
-  int last = 0;  // CTAs past the last one with work are not launched
+  P.queue_begin = cb[G];
+  P.n_queue = n - cb[G];
+  for (int q = P.queue_begin; q < n; ++q) queued[seg[order[q]]] = true;
+  int last = 0;  // with no queue, CTAs past the last one with work are not launched
   for (int c = 0; c < G; ++c) {
     P.cta_item_begin[c] = static_cast<int16_t>(cb[c]);
     if (cb[c + 1] > cb[c]) last = c + 1;
@@ -258,14 +274,22 @@ flint_status plan(DecodeParams& P, const int* tiles, int n_problems, int num_cta
     while (i < n && seg[i] < s) ++i;
     P.seg_item_begin[s] = static_cast<int16_t>(i);
   }
+  // Problems with queued chunks, or split more widely than kInlineMergeMax,
+  // are merged by the whole grid after the grid barrier: their last items
+  // finish near the end of the launch, where one CTA merging alone would be
+  // the tail.
   P.n_deferred = 0;
+  P.merge_wide = 0;
   for (int s = 0; s < n_segs; ++s) {
-    const bool deferred = P.seg_item_begin[s + 1] - P.seg_item_begin[s] > kInlineMergeMax;
+    const int items = P.seg_item_begin[s + 1] - P.seg_item_begin[s];
+    const bool deferred = queued[s] || items > kInlineMergeMax;
     P.prob[s].deferred = deferred ? 1 : 0;
     if (deferred) P.deferred[P.n_deferred++] = static_cast<int16_t>(s);
+    if (deferred && items > kWideMergeItems) P.merge_wide = 1;
   }
-  P.grid_merge = P.n_deferred > 0 ? 1 : 0;
-  *grid = last;
+  P.grid_merge = (P.n_deferred > 0 || P.n_queue > 0) ? 1 : 0;
+  P.ws_items = cap;
+  *grid = P.n_queue > 0 ? G : last;
   return FLINT_OK;
 }
 
@@ -277,6 +301,14 @@ flint_status launch_result(cudaError_t e, const char* who) {
 }  // namespace
 
 namespace flint {
+
+size_t workspace_min_bytes(int n_problems, int num_ctas) {
+  if (n_problems < 1 || n_problems > kMaxProblems || num_ctas < 0 || num_ctas > kMaxCtas) return 0;
+  int g = num_ctas;
+  if (g == 0 && device_num_sms(&g) != 0) g = kMaxCtas;
+  g = std::min(g, kMaxCtas);
+  return kCounterBytes + static_cast<size_t>(std::min(kMaxItems, g + n_problems)) * kPartialBytes;
+}
 
 flint_status record_error(flint_status s, const char* fmt, ...) {
   char buf[512];
@@ -411,9 +443,7 @@ flint_status flint_kv_append(const uint16_t* k, const uint16_t* v, const int32_t
 
 size_t flint_attn_workspace_bytes(int32_t n_problems, int32_t num_ctas) {
   if (n_problems < 1 || n_problems > kMaxProblems || num_ctas < 0 || num_ctas > kMaxCtas) return 0;
-  int g = num_ctas;
-  if (g == 0 && device_num_sms(&g) != 0) g = kMaxCtas;
-  return workspace_bytes(n_problems, std::min(g, kMaxCtas));
+  return kCounterBytes + static_cast<size_t>(kMaxItems) * kPartialBytes;
 }
 
 flint_status flint_attn_decode(const void* q, int32_t q_is_fp32, const flint_kv_cache* cache,
@@ -462,16 +492,12 @@ flint_status flint_attn_decode(const void* q, int32_t q_is_fp32, const flint_kv_
     tiles[b] = r.tiles;
   }
   int grid = 0;
-  s = plan(P, tiles, B, num_ctas, &grid);
+  s = plan(P, tiles, B, num_ctas, ws_bytes, who, &grid);
   if (s != FLINT_OK) return s;
-  if (ws_bytes < workspace_bytes(B, grid))
-    return fail(FLINT_ERR_WORKSPACE, "%s: workspace of %zu bytes is below the %zu needed", who, ws_bytes,
-                workspace_bytes(B, grid));
   s = encode_cache_map(&P.maps[0], cache->k, *cache, B);
   if (s != FLINT_OK) return s;
   s = encode_cache_map(&P.maps[1], cache->v, *cache, B);
   if (s != FLINT_OK) return s;
-  P.ws_items = static_cast<int32_t>(std::min<size_t>((ws_bytes - kCounterBytes) / (kPartialFloats * sizeof(float)), 1 << 30));
   P.smem_bytes = static_cast<int32_t>(decode_smem_bytes());
   P.counters = static_cast<int32_t*>(workspace);
   P.partials = reinterpret_cast<float*>(static_cast<uint8_t*>(workspace) + kCounterBytes);
@@ -546,12 +572,8 @@ flint_status flint_attn_stack(const flint_layer* layers, int32_t n_layers, int32
     if (s != FLINT_OK) return s;
   }
   int grid = 0;
-  flint_status s = plan(P, tiles, n_layers, num_ctas, &grid);
+  flint_status s = plan(P, tiles, n_layers, num_ctas, ws_bytes, who, &grid);
   if (s != FLINT_OK) return s;
-  if (ws_bytes < workspace_bytes(n_layers, grid))
-    return fail(FLINT_ERR_WORKSPACE, "%s: workspace of %zu bytes is below the %zu needed", who, ws_bytes,
-                workspace_bytes(n_layers, grid));
-  P.ws_items = static_cast<int32_t>(std::min<size_t>((ws_bytes - kCounterBytes) / (kPartialFloats * sizeof(float)), 1 << 30));
   P.smem_bytes = static_cast<int32_t>(decode_smem_bytes());
   P.counters = static_cast<int32_t*>(workspace);
   P.partials = reinterpret_cast<float*>(static_cast<uint8_t*>(workspace) + kCounterBytes);

@@ -9,9 +9,11 @@
 //     s_j = q_h . K_j / sqrt(128),  M = max(max_j s_j, sink_h).
 //
 // How (one persistent launch for every problem of the call):
-//   * The host cuts each problem's token range into 16-token tiles and lays
-//     the tiles of all problems over one CTA per SM (split-KV); each CTA walks
-//     its list of items (problem, tile range).
+//   * The host cuts each problem's token range into 32-token tiles and lays
+//     most of them over one CTA per SM as static item lists (problem, tile
+//     range; split-KV).  The tails of large problems are cut into chunks that
+//     CTAs claim from a queue (atomic head in the workspace) once their own
+//     lists are done, which evens out SMs that stream at different rates.
 //   * The last warp is the producer: per 32-token tile it loads K and V of all
 //     four KV heads with 16 TMA boxes (4-D tensor maps, 128-byte swizzle,
 //     issued by lanes 0-15) into a 3-stage ring of 64 KiB stages guarded by
@@ -75,7 +77,9 @@ struct Smem {
   uint64_t* in_empty;   // item inputs consumed
   float2* cs;
   volatile int* flags;  // [0] abort, [1] last-arrival broadcast, [2] grid barrier,
-                        // [3] item whose new token is in the cache (+1)
+                        // [3] item whose new token is in the cache (+1),
+                        // [4] item whose inputs are staged (producer -> consumers),
+                        // [5] that item as consumer warp 0 saw it (-1: stop)
   float* xch;           // group hand-over area
   uint8_t* in;          // item inputs
 };
@@ -90,7 +94,7 @@ __device__ __forceinline__ Smem carve(uint8_t* raw) {
   s.in_empty = s.in_full + 1;
   s.cs = reinterpret_cast<float2*>(s.in_empty + 1);
   s.flags = reinterpret_cast<volatile int*>(s.cs + 64);
-  s.xch = reinterpret_cast<float*>(s.cs + 64) + 4;
+  s.xch = reinterpret_cast<float*>(s.cs + 64) + 8;
   s.in = reinterpret_cast<uint8_t*>(s.xch + kXchSize);  // 16-byte aligned
   return s;
 }
@@ -169,28 +173,53 @@ __device__ __forceinline__ void issue_item_inputs(const DecodeParams& P, const P
   }
 }
 
-// Returns the number of tiles whose loads were issued.
-__device__ int run_producer(const DecodeParams& P, const Smem& S, int it0, int it1, int lane) {
+// The next item of this CTA: its k-th static item, else a claim on the queue;
+// -1 when there is no more work.
+__device__ __forceinline__ int next_item(const DecodeParams& P, int k, int c0, int c1, bool claim) {
+  if (c0 + k < c1) return P.order[c0 + k];
+  if (!claim || P.n_queue <= 0) return -1;
+  const int q = atomicAdd(P.counters + kQueueHead, 1);
+  return q < P.n_queue ? P.order[P.queue_begin + q] : -1;
+}
+
+struct ProducerCount {
+  int issued;  // tiles whose loads were issued
+  int staged;  // in_full phases armed
+};
+
+__device__ ProducerCount run_producer(const DecodeParams& P, const Smem& S, int c0, int c1, bool claim,
+                                      int lane) {
   int seq = 0;
   // lane i < 16 issues box i: K/V (i >> 3), head ((i >> 1) & 3), dim half (i & 1)
   const int my_kv = (lane >> 3) & 1, my_head = (lane >> 1) & 3, my_half = lane & 1;
-  for (int it = it0; it < it1; ++it) {
+  for (int k = 0;; ++k) {
+    int it = -1;
+    {  // pick the next item once the consumers released the last inputs, and
+       // stage its small inputs (or, with no item left, tell them to stop)
+      bool ok = mbar_wait(smem_u32(S.in_empty), (static_cast<uint32_t>(k) & 1u) ^ 1u, S.flags);
+      ok = __all_sync(0xffffffffu, ok);
+      if (!ok) {
+        if (lane == 0) abort_cta(P, S);
+        return {seq, k};
+      }
+      if (lane == 0) {
+        it = next_item(P, k, c0, c1, claim);
+        if (!FLINT_CHECK(P.dev_err, it < P.n_items, 9, it, P.n_items, k)) it = -1;
+        S.flags[4] = it;  // published by the arrive below (release)
+        if (it >= 0)
+          issue_item_inputs(P, P.prob[P.items[it].seg], S);
+        else
+          mbar_arrive(smem_u32(S.in_full));
+      }
+      it = __shfl_sync(0xffffffffu, it, 0);
+      __syncwarp();
+      if (it < 0) return {seq, k + 1};
+    }
     const Item item = P.items[it];
     const Problem& pb = P.prob[item.seg];
     const CUtensorMap* map = &P.maps[my_kv ? pb.map_v : pb.map_k];
     const bool paged = pb.layout == FLINT_KV_PAGED;
     const int app_tile = (P.prep && pb.append_tok >= 0) ? (pb.append_tok - pb.tile_base) / kTile : -1;
-    {  // stage this item's small inputs once the consumers released the last ones
-      const uint32_t ph = static_cast<uint32_t>(it - it0) & 1u;
-      bool ok = mbar_wait(smem_u32(S.in_empty), ph ^ 1u, S.flags);
-      ok = __all_sync(0xffffffffu, ok);
-      if (!ok) {
-        if (lane == 0) abort_cta(P, S);
-        return seq;
-      }
-      if (lane == 0) issue_item_inputs(P, pb, S);
-      __syncwarp();
-    }
     for (int t = item.t0; t < item.t1; t += 32) {
       const int n = min(32, item.t1 - t);
       int blk = 0;
@@ -208,7 +237,7 @@ __device__ int run_producer(const DecodeParams& P, const Smem& S, int it0, int i
         ok = __all_sync(0xffffffffu, ok);
         if (!ok) {
           if (lane == 0) abort_cta(P, S);
-          return seq;
+          return {seq, k + 1};
         }
         const int tile = t + j;
         if (tile == app_tile) {
@@ -227,7 +256,7 @@ __device__ int run_producer(const DecodeParams& P, const Smem& S, int it0, int i
           done = __shfl_sync(0xffffffffu, done, 0);
           if (!done) {
             if (lane == 0) abort_cta(P, S);
-            return seq;
+            return {seq, k + 1};
           }
         }
         const uint32_t fb = smem_u32(&S.full[stage]);
@@ -253,7 +282,6 @@ __device__ int run_producer(const DecodeParams& P, const Smem& S, int it0, int i
       }
     }
   }
-  return seq;
 }
 
 // q fragments for query head h: thread (g = lane/4, c = lane%4) holds dims
@@ -431,23 +459,29 @@ __device__ __forceinline__ void finish_head(const Problem& pb, int head, int c, 
     *reinterpret_cast<float2*>(dst + 8 * n) = make_float2(v[2 * n] * scale, v[2 * n + 1] * scale);
 }
 
-__device__ void run_consumer(const DecodeParams& P, const Smem& S, int it0, int it1, int warp,
-                             int lane) {
+__device__ void run_consumer(const DecodeParams& P, const Smem& S, int warp, int lane) {
   const int g = lane >> 2, c = lane & 3;
   const int kvh = warp % kKvHeads;      // the KV head this warp serves
   const int group = warp / kKvHeads;    // its consumer group
   const int head = kvh * kGroup + g;    // the query head this thread's quad serves
   int seq = 0;
-  for (int it = it0; it < it1; ++it) {
+  for (int k = 0;; ++k) {
+    uint32_t qa[8][4];
+    // Every consumer warp waits for the staged inputs itself; all of them
+    // then take the item as warp 0 saw it, so they agree on when to stop and
+    // meet the same barriers.  Warp 0 rewrites flags[5] only once the next
+    // inputs are staged, which needs every warp's in_empty arrival below,
+    // made after its read (and the item-end barriers come in between too).
+    bool ok = mbar_wait(smem_u32(S.in_full), static_cast<uint32_t>(k) & 1u, S.flags);
+    ok = __all_sync(0xffffffffu, ok);
+    if (!ok && lane == 0) abort_cta(P, S);
+    if (warp == 0 && lane == 0) S.flags[5] = ok ? S.flags[4] : -1;
+    consumer_bar();
+    const int it = S.flags[5];
+    if (it < 0) break;
     const Item item = P.items[it];
     const Problem& pb = P.prob[item.seg];
-
-    uint32_t qa[8][4];
     {
-      const uint32_t ph = static_cast<uint32_t>(it - it0) & 1u;
-      bool ok = mbar_wait(smem_u32(S.in_full), ph, S.flags);
-      ok = __all_sync(0xffffffffu, ok);
-      if (!ok && lane == 0) abort_cta(P, S);
       load_q(P, pb, S.in, head, c, S.cs, qa);
       if (P.prep && warp == kAppendWarp && pb.append_tok >= 0) {
         const int app_tile = (pb.append_tok - pb.tile_base) / kTile;
@@ -633,72 +667,110 @@ __device__ bool grid_barrier(unsigned int* bar, const Smem& S) {
   return S.flags[2] != 0;
 }
 
-// Merge of the deferred problems by the whole grid: one CTA per (problem,
-// head, quarter c) unit, every thread folding in its own partials (one or two:
-// a problem has at most one partial per CTA), so all loads of a unit are in
-// flight at once; then a block reduction.  Value k of a quarter is dim
-// 8(k/2) + 2c + (k & 1) of the head.
+// Folds partials i = s0 + r, s0 + r + stride, ... (< s1) of (head, quarter c)
+// into a running (m, l, v), in increasing i.
+__device__ __forceinline__ void fold_partials(const DecodeParams& P, int s0, int s1, int r, int stride,
+                                              int head, int c, float& m, float& l, float (&v)[32]) {
+  for (int i = s0 + r; i < s1; i += stride) {
+    const float* pi = P.partials + static_cast<size_t>(i) * kPartialFloats;
+    const float mi = __ldcg(pi + kHeads * kDim + head);
+    const float li = __ldcg(pi + kHeads * kDim + kHeads + head);
+    const float4* po = reinterpret_cast<const float4*>(pi + partial_o(head, c));
+    float4 ov[8];
+#pragma unroll
+    for (int q = 0; q < 8; ++q) ov[q] = __ldcg(po + q);
+    const float mn = fmaxf(m, mi);
+    const float sa = (m == -INFINITY) ? 0.f : exp2f(m - mn);
+    const float sb = (mi == -INFINITY) ? 0.f : exp2f(mi - mn);
+#pragma unroll
+    for (int q = 0; q < 8; ++q) {
+      v[4 * q] = v[4 * q] * sa + ov[q].x * sb;
+      v[4 * q + 1] = v[4 * q + 1] * sa + ov[q].y * sb;
+      v[4 * q + 2] = v[4 * q + 2] * sa + ov[q].z * sb;
+      v[4 * q + 3] = v[4 * q + 3] * sa + ov[q].w * sb;
+    }
+    l = l * sa + li * sb;
+    m = mn;
+  }
+}
+
+// Rescales a lane's (m, l, v) to the common max M, then sums l over the warp
+// and reduce-scatters v: afterwards lane k holds the warp's sum of value k.
+__device__ __forceinline__ void warp_sum_at(float m, float M, float& l, float (&v)[32], int lane) {
+  const float sc = (m == -INFINITY) ? 0.f : exp2f(m - M);
+  l *= sc;
+#pragma unroll
+  for (int e = 0; e < 32; ++e) v[e] *= sc;
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) l += __shfl_xor_sync(0xffffffffu, l, o);
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) {
+    const bool up = (lane & o) != 0;
+#pragma unroll
+    for (int j = 0; j < o; ++j) {
+      const float send = up ? v[j] : v[j + o];
+      const float keep = up ? v[j + o] : v[j];
+      v[j] = keep + __shfl_xor_sync(0xffffffffu, send, o);
+    }
+  }
+}
+
+__device__ __forceinline__ float warp_max(float x) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) x = fmaxf(x, __shfl_xor_sync(0xffffffffu, x, o));
+  return x;
+}
+
+// Value t of quarter c of a head, with the sink folded in.
+__device__ __forceinline__ void write_merged(const Problem& pb, int head, int c, int t, float M, float L,
+                                             float sum) {
+  const float s2 = pb.sinks[head] * kLog2e;
+  const float Mf = fmaxf(M, s2);
+  const float a = (M == -INFINITY) ? 0.f : exp2f(M - Mf);
+  const float scale = a / (L * a + exp2f(s2 - Mf));
+  pb.out[head * kDim + 8 * (t >> 1) + 2 * c + (t & 1)] = sum * scale;
+}
+
+// Merge of the deferred problems by the whole grid after the grid barrier, in
+// units of (problem, head, quarter c); value k of a quarter is dim
+// 8(k/2) + 2c + (k & 1) of the head.  Problems with few partials take one
+// warp per unit (lane j folds partials j, j + 32, ...); with many partials
+// (a lone long problem split over every CTA) a unit takes a whole CTA, one
+// thread per partial, so that all of a unit's loads are in flight at once.
 __device__ void grid_merge(const DecodeParams& P, const Smem& S) {
   constexpr int kWarps = kThreads / 32;
   const int t = threadIdx.x, lane = t & 31, warp = t >> 5;
-  float* red = S.xch;  // [kWarps][34] scratch (the hand-over area is free now)
   const int units = P.n_deferred * kHeads * 4;
+  if (!P.merge_wide) {
+    for (int u = blockIdx.x * kWarps + warp; u < units; u += gridDim.x * kWarps) {
+      const int p = P.deferred[u / (kHeads * 4)];
+      const int head = (u / 4) % kHeads, c = u % 4;
+      float m = -INFINITY, l = 0.f, v[32];
+#pragma unroll
+      for (int e = 0; e < 32; ++e) v[e] = 0.f;
+      fold_partials(P, P.seg_item_begin[p], P.seg_item_begin[p + 1], lane, 32, head, c, m, l, v);
+      const float M = warp_max(m);
+      warp_sum_at(m, M, l, v, lane);
+      write_merged(P.prob[p], head, c, lane, M, l, v[0]);
+    }
+    return;
+  }
+  float* red = S.xch;  // [kWarps][34] scratch (the hand-over area is free now)
   for (int u = blockIdx.x; u < units; u += gridDim.x) {
     const int p = P.deferred[u / (kHeads * 4)];
     const int head = (u / 4) % kHeads, c = u % 4;
-    const Problem& pb = P.prob[p];
-    const int s0 = P.seg_item_begin[p], s1 = P.seg_item_begin[p + 1];
     float m = -INFINITY, l = 0.f, v[32];
 #pragma unroll
     for (int e = 0; e < 32; ++e) v[e] = 0.f;
-    for (int i = s0 + t; i < s1; i += kThreads) {
-      const float* pi = P.partials + static_cast<size_t>(i) * kPartialFloats;
-      const float mi = __ldcg(pi + kHeads * kDim + head);
-      const float li = __ldcg(pi + kHeads * kDim + kHeads + head);
-      const float4* po = reinterpret_cast<const float4*>(pi + partial_o(head, c));
-      float4 ov[8];
-#pragma unroll
-      for (int q = 0; q < 8; ++q) ov[q] = __ldcg(po + q);
-      const float mn = fmaxf(m, mi);
-      const float sa = (m == -INFINITY) ? 0.f : exp2f(m - mn);
-      const float sb = (mi == -INFINITY) ? 0.f : exp2f(mi - mn);
-#pragma unroll
-      for (int q = 0; q < 8; ++q) {
-        v[4 * q] = v[4 * q] * sa + ov[q].x * sb;
-        v[4 * q + 1] = v[4 * q + 1] * sa + ov[q].y * sb;
-        v[4 * q + 2] = v[4 * q + 2] * sa + ov[q].z * sb;
-        v[4 * q + 3] = v[4 * q + 3] * sa + ov[q].w * sb;
-      }
-      l = l * sa + li * sb;
-      m = mn;
-    }
-    // block max of m
-    float M = m;
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, o));
+    fold_partials(P, P.seg_item_begin[p], P.seg_item_begin[p + 1], t, kThreads, head, c, m, l, v);
+    float M = warp_max(m);
     if (lane == 0) red[warp] = M;
     __syncthreads();
     M = red[0];
 #pragma unroll
     for (int w = 1; w < kWarps; ++w) M = fmaxf(M, red[w]);
     __syncthreads();
-    const float sc = (m == -INFINITY) ? 0.f : exp2f(m - M);
-    l *= sc;
-#pragma unroll
-    for (int e = 0; e < 32; ++e) v[e] *= sc;
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) l += __shfl_xor_sync(0xffffffffu, l, o);
-    // warp reduce-scatter: afterwards lane k holds the warp's sum of value k
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) {
-      const bool up = (lane & o) != 0;
-#pragma unroll
-      for (int j = 0; j < o; ++j) {
-        const float send = up ? v[j] : v[j + o];
-        const float keep = up ? v[j + o] : v[j];
-        v[j] = keep + __shfl_xor_sync(0xffffffffu, send, o);
-      }
-    }
+    warp_sum_at(m, M, l, v, lane);
     red[warp * 34 + lane] = v[0];
     if (lane == 0) red[warp * 34 + 32] = l;
     __syncthreads();
@@ -709,11 +781,7 @@ __device__ void grid_merge(const DecodeParams& P, const Smem& S) {
         sum += red[w * 34 + t];
         L += red[w * 34 + 32];
       }
-      const float s2 = pb.sinks[head] * kLog2e;
-      const float Mf = fmaxf(M, s2);
-      const float a = (M == -INFINITY) ? 0.f : exp2f(M - Mf);
-      const float scale = a / (L * a + exp2f(s2 - Mf));
-      pb.out[head * kDim + 8 * (t >> 1) + 2 * c + (t & 1)] = sum * scale;
+      write_merged(P.prob[p], head, c, t, M, L, sum);
     }
     __syncthreads();  // red is reused by the next unit
   }
@@ -723,10 +791,18 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const __grid_consta
   extern __shared__ uint8_t smem_raw[];
   const Smem S = carve(smem_raw);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  int it0 = P.cta_item_begin[blockIdx.x], it1 = P.cta_item_begin[blockIdx.x + 1];
-  if (!FLINT_CHECK(P.dev_err, 0 <= it0 && it0 <= it1 && it1 <= P.n_items, 1, it0, it1, P.n_items)) it1 = it0;
+  int c0 = P.cta_item_begin[blockIdx.x], c1 = P.cta_item_begin[blockIdx.x + 1];
+  bool claim = true;
+  if (!FLINT_CHECK(P.dev_err, 0 <= c0 && c0 <= c1 && c1 <= P.queue_begin && P.queue_begin + P.n_queue <= P.n_items,
+                   1, c0, c1, P.n_items)) {
+    c1 = c0;
+    claim = false;
+  }
   const int smem_end = static_cast<int>(smem_u32(S.in + kInBytes) - smem_u32(smem_raw));
-  if (!FLINT_CHECK(P.dev_err, smem_end <= P.smem_bytes, 2, smem_end, P.smem_bytes, 0)) it1 = it0;
+  if (!FLINT_CHECK(P.dev_err, smem_end <= P.smem_bytes, 2, smem_end, P.smem_bytes, 0)) {
+    c1 = c0;
+    claim = false;
+  }
   (void)smem_end;
 
   if (threadIdx.x == 0) {
@@ -736,33 +812,33 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const __grid_consta
     }
     mbar_init(smem_u32(S.in_full), 1);
     mbar_init(smem_u32(S.in_empty), kConsumerWarps);
-    S.flags[0] = 0;
-    S.flags[1] = 0;
-    S.flags[3] = 0;
+    for (int f = 0; f < 8; ++f) S.flags[f] = 0;
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
     asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
   }
   if (P.prep && threadIdx.x < 64) S.cs[threadIdx.x] = rope_cos_sin(threadIdx.x, P.prob[0].pos, P.theta);
   __syncthreads();
 
-  int issued = 0;
+  ProducerCount pc{0, 0};
   if (warp == kConsumerWarps) {
-    issued = run_producer(P, S, it0, it1, lane);
+    pc = run_producer(P, S, c0, c1, claim, lane);
   } else {
-    run_consumer(P, S, it0, it1, warp, lane);
+    run_consumer(P, S, warp, lane);
   }
   __syncthreads();
-  // After an abort, let every issued load land before the CTA's shared memory
-  // goes away (bounded as well; a normal run returns at once).
+  // After an abort, let every issued copy land before the CTA's shared memory
+  // goes away (bounded as well; a normal run returns at once).  Only the last
+  // armed input phase can still have copies in flight: the producer arms the
+  // next one only after the consumers saw this one complete.
   if (warp == kConsumerWarps && lane == 0) {
-    if (it1 > it0) {  // the last staged inputs
+    if (pc.staged > 0) {
       const unsigned long long t0 = globaltimer_ns();
-      while (!mbar_try_wait(smem_u32(S.in_full), static_cast<uint32_t>(it1 - it0 - 1) & 1u)) {
+      while (!mbar_try_wait(smem_u32(S.in_full), static_cast<uint32_t>(pc.staged - 1) & 1u)) {
         if (globaltimer_ns() - t0 > kWaitLimitNs) break;
       }
     }
-    const int first = issued > kStages ? issued - kStages : 0;
-    for (int s = first; s < issued; ++s) {
+    const int first = pc.issued > kStages ? pc.issued - kStages : 0;
+    for (int s = first; s < pc.issued; ++s) {
       const unsigned long long t0 = globaltimer_ns();
       while (!mbar_try_wait(smem_u32(&S.full[s % kStages]), static_cast<uint32_t>(s / kStages) & 1u)) {
         if (globaltimer_ns() - t0 > kWaitLimitNs) break;
@@ -770,7 +846,9 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const __grid_consta
     }
   }
   if (P.grid_merge) {
-    if (grid_barrier(reinterpret_cast<unsigned int*>(P.counters + kMaxSegs), S)) {
+    if (grid_barrier(reinterpret_cast<unsigned int*>(P.counters + kBarrierWord), S)) {
+      // every CTA has made its last claim: ready the queue for the next call
+      if (blockIdx.x == 0 && threadIdx.x == 0) P.counters[kQueueHead] = 0;
       grid_merge(P, S);
     } else if (threadIdx.x == 0) {
       report_error(P.dev_err, FLINT_ERR_TIMEOUT);
@@ -782,7 +860,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const __grid_consta
 
 size_t decode_smem_bytes() {
   return 1024 + static_cast<size_t>(kStages) * kStageBytes + 2 * kStages * sizeof(uint64_t) +
-         2 * sizeof(uint64_t) + 64 * sizeof(float2) + 4 * sizeof(int) + kXchSize * sizeof(float) +
+         2 * sizeof(uint64_t) + 64 * sizeof(float2) + 8 * sizeof(int) + kXchSize * sizeof(float) +
          kInBytes;
 }
 

@@ -49,7 +49,7 @@ static_assert(kTile % kSlice == 0, "a tile splits into 16-token slices");
 constexpr int kMaxProblems = 64;
 constexpr int kMaxSegs = kMaxProblems;         // one segment per problem
 constexpr int kMaxMaps = 2 * FLINT_MAX_LAYERS;
-constexpr int kMaxItems = 512;
+constexpr int kMaxItems = 640;
 constexpr int kMaxCtas = 296;
 
 // A problem split into more than kInlineMergeMax items is not merged by its
@@ -61,6 +61,10 @@ constexpr int kInlineMergeMax = 16;
 // consumer thread's 32 values are contiguous), m [32] (log2 units), l [32].
 constexpr int kPartialFloats = kHeads * kDim + 2 * kHeads;
 constexpr size_t kCounterBytes = 4096;
+// int32 slots of the workspace's counter area: [0, kMaxSegs) per-problem
+// arrival counters, then the grid-barrier word and the run-time queue head.
+constexpr int kBarrierWord = kMaxSegs;
+constexpr int kQueueHead = kMaxSegs + 1;
 
 // One attention problem: one request of one layer.
 struct Problem {
@@ -96,9 +100,12 @@ struct Item {
 struct DecodeParams {
   CUtensorMap maps[kMaxMaps];
   Problem prob[kMaxProblems];
-  Item items[kMaxItems];
-  int16_t cta_item_begin[kMaxCtas + 1];
-  int16_t seg_item_begin[kMaxSegs + 1];
+  Item items[kMaxItems];          // sorted by (problem, first tile)
+  int16_t order[kMaxItems];       // static lists of the CTAs, then the run-time queue
+  int16_t cta_item_begin[kMaxCtas + 1];  // CTA c's static items: order[begin[c] .. begin[c+1])
+  int16_t seg_item_begin[kMaxSegs + 1];  // problem p's items: items[begin[p] .. begin[p+1])
+  int32_t queue_begin;            // the queue is order[queue_begin .. queue_begin + n_queue)
+  int32_t n_queue;
   int32_t* counters;        // workspace: per-segment arrival counters
   float* partials;          // workspace: one partial per item
   int32_t* dev_err;         // [0] status; debug builds also record a failed check in [2..7]
@@ -107,9 +114,11 @@ struct DecodeParams {
   int32_t n_problems;
   int32_t prep;             // 1: q/k norm (+RoPE) and append fused in (layer stack)
   int32_t n_items;          // items in the plan
-  int32_t grid_merge;       // 1: some problem is deferred (cooperative launch)
+  int32_t grid_merge;       // 1: a grid barrier ends the launch (cooperative launch):
+                            // some problem is deferred or the queue is not empty
   int16_t deferred[kMaxProblems];  // the deferred problems
   int32_t n_deferred;
+  int32_t merge_wide;       // 1: a deferred problem has many partials: a CTA per merge unit
   int32_t ws_items;         // partial slots in the workspace
   int32_t smem_bytes;       // dynamic shared memory of the launch
 };
@@ -143,6 +152,10 @@ cudaError_t launch_decode(const DecodeParams& p, int grid, cudaStream_t stream);
 cudaError_t launch_prep(const PrepParams& p, int B, cudaStream_t stream);
 
 size_t decode_smem_bytes();
+
+// Smallest workspace a launch of n_problems on num_ctas CTAs (0: one per SM)
+// can run with: the counters and one partial per static item; 0 if invalid.
+size_t workspace_min_bytes(int n_problems, int num_ctas);
 
 // Sets the message that flint_last_error() returns on this thread; returns s.
 flint_status record_error(flint_status s, const char* fmt, ...);

@@ -69,8 +69,9 @@ extern "C" flint_status flint_attn_stack_noalloc(const flint_layer* layers, int3
                                                  int32_t pos, float eps, double theta, float* out,
                                                  int32_t num_ctas, int32_t* dev_err, void* stream) {
   const char* who = "flint_attn_stack_noalloc";
-  // Size check first: the scratch cannot grow.
-  const size_t need = flint_attn_workspace_bytes(n_layers, num_ctas);
+  // Size check first: the scratch cannot grow.  It must hold the static plan;
+  // the run-time queue then gets the part of it that is left.
+  const size_t need = workspace_min_bytes(n_layers, num_ctas);
   if (need == 0)
     return record_error(FLINT_ERR_INVALID_ARG, "%s: n_layers=%d or num_ctas=%d out of range", who, n_layers, num_ctas);
   if (need > FLINT_NOALLOC_SCRATCH_BYTES)

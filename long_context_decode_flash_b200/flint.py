@@ -31,7 +31,7 @@ MAX_BATCH, MAX_LAYERS = 64, 49
 EXPORTED = (
     "flint_status_string", "flint_last_error", "flint_kv_bytes", "flint_qk_norm_rope",
     "flint_kv_append", "flint_attn_workspace_bytes", "flint_attn_decode", "flint_attn_stack",
-    "flint_attn_stack_noalloc", "flint_plan_items",
+    "flint_attn_stack_noalloc", "flint_plan_items", "flint_plan_split",
 )
 
 
@@ -87,6 +87,8 @@ def load_library() -> ctypes.CDLL:
                                                      P, I32, P, P]
             lib.flint_plan_items.argtypes = [P, I32, I32, I32, P, P, P, P, I32]
             lib.flint_plan_items.restype = I32
+            lib.flint_plan_split.argtypes = [P, I32, I32, I32, I32, P, P, P, P, P]
+            lib.flint_plan_split.restype = I32
             for name in ("flint_qk_norm_rope", "flint_kv_append", "flint_attn_decode",
                          "flint_attn_stack", "flint_attn_stack_noalloc"):
                 getattr(lib, name).restype = ctypes.c_int
@@ -240,3 +242,23 @@ def flint_plan_items(seg_tiles: Sequence[int], num_ctas: int, item_cost: int = 2
     if k < 0:
         raise FlintError(FLINT_ERR_INVALID_ARG, "planner rejected the arguments")
     return [(seg[i], t0[i], t1[i]) for i in range(k)], list(cb)
+
+
+def flint_plan_split(seg_tiles: Sequence[int], num_ctas: int, item_cost: int = 2,
+                     max_items: int = 640):
+    """Returns (items [(seg, t0, t1)] sorted by segment, static lists [[item
+    index, ...] per CTA], queue [item index, ...]) from the C planner."""
+    n = len(seg_tiles)
+    st = _i32_host(seg_tiles)
+    seg = (ctypes.c_int32 * max_items)()
+    t0 = (ctypes.c_int32 * max_items)()
+    t1 = (ctypes.c_int32 * max_items)()
+    order = (ctypes.c_int32 * max_items)()
+    cb = (ctypes.c_int32 * (num_ctas + 1))()
+    k = load_library().flint_plan_split(st, n, num_ctas, item_cost, max_items, seg, t0, t1, order, cb)
+    if k < 0:
+        raise FlintError(FLINT_ERR_INVALID_ARG, "planner rejected the arguments")
+    items = [(seg[i], t0[i], t1[i]) for i in range(k)]
+    lists = [[order[j] for j in range(cb[c], cb[c + 1])] for c in range(num_ctas)]
+    queue = [order[j] for j in range(cb[num_ctas], k)]
+    return items, lists, queue

@@ -120,9 +120,23 @@ def test_stack_and_prep_reject_bad_arguments_on_the_host():
 def test_workspace_bytes_bounds():
     assert flint.flint_attn_workspace_bytes(0, 148) == 0
     assert flint.flint_attn_workspace_bytes(65, 148) == 0
-    a = flint.flint_attn_workspace_bytes(1, 148)
-    b = flint.flint_attn_workspace_bytes(49, 148)
-    assert 0 < a < b
+    # room for the largest plan: 640 partials of (32*128 + 2*32) floats
+    full = 4096 + 640 * 16640
+    assert flint.flint_attn_workspace_bytes(1, 148) == full
+    assert flint.flint_attn_workspace_bytes(49, 148) == full
+
+
+def test_workspace_below_the_static_plan_is_refused_on_the_host():
+    # 4 requests of 4,096 tokens (128 tiles each) on 148 CTAs need at least
+    # 4096 + (148 + 4) * 16640 bytes; the check comes before any CUDA call
+    lib = flint.load_library()
+    cache = _fake_cache()
+    seq = (ctypes.c_int32 * 4)(*[4096] * 4)
+    need = 4096 + (148 + 4) * 16640
+    args = (ctypes.c_void_p(0x30000), 0, ctypes.byref(cache), seq, 4, ctypes.c_void_p(0x60000), 0,
+            ctypes.c_void_p(0x40000), ctypes.c_void_p(0x50000))
+    assert lib.flint_attn_decode(*args, need - 1, 148, None, None) == flint.FLINT_ERR_WORKSPACE
+    assert str(need) in flint.flint_last_error()
 
 
 # ------------------------------------------------------------ planner -----
@@ -153,14 +167,14 @@ def check_plan(seg_tiles, G, cost=2):
 
 
 def test_plan_single_full_layer_at_100k():
-    # one problem of 100,000 tokens = 6,250 tiles of 16 tokens (all 4 KV heads)
-    items, cb, loads = check_plan([6250], 148)
+    # one problem of 100,000 tokens = 3,125 tiles of 32 tokens (all 4 KV heads)
+    items, cb, loads = check_plan([3125], 148)
     assert len(items) == 148
-    assert min(loads) >= 40
+    assert min(loads) >= 20
 
 
 def test_plan_layer_stack_at_100k():
-    tiles = [6250 if (i % 7) in (3, 6) else 33 for i in range(49)]
+    tiles = [3125 if (i % 7) in (3, 6) else 17 for i in range(49)]
     items, cb, loads = check_plan(tiles, 148)
     assert len(items) <= 148 + 49
 
@@ -183,3 +197,87 @@ def test_plan_rejects_bad_arguments():
         flint.flint_plan_items([], 4)
     with pytest.raises(flint.FlintError):
         flint.flint_plan_items([0, 3], 4)
+
+
+# ------------------------------------------------- planner with a queue -----
+
+def check_split(seg_tiles, G, max_items=640, cost=2):
+    items, lists, queue = flint.flint_plan_split(seg_tiles, G, cost, max_items)
+    n = len(items)
+    assert n <= max_items
+    # items sorted by (segment, t0) and tiling every segment exactly
+    assert items == sorted(items)
+    if sum(seg_tiles) < 64 * G:
+        assert queue == []
+    for s, T in enumerate(seg_tiles):
+        rs = [(t0, t1) for q, t0, t1 in items if q == s]
+        assert rs[0][0] == 0 and rs[-1][1] == T
+        assert all(a[1] == b[0] and a[0] < a[1] for a, b in zip(rs, rs[1:]))
+    # the static lists and the queue name every item exactly once
+    named = [i for l in lists for i in l] + queue
+    assert sorted(named) == list(range(n))
+    # a segment's static items come before its queued chunks, and small
+    # segments are never queued
+    qset = set(queue)
+    for i, (s, t0, t1) in enumerate(items):
+        if i in qset:
+            assert seg_tiles[s] >= 64
+            assert all(items[j][1] < t0 for j in range(n) if items[j][0] == s and j not in qset)
+    # the static part is the static planner's plan of the shortened segments
+    st = list(seg_tiles)
+    for i in queue:
+        s, t0, t1 = items[i]
+        st[s] -= t1 - t0
+    ref_items, ref_cb = flint.flint_plan_items(st, G, cost, max_items)
+    static = [[items[i] for i in l] for l in lists]
+    assert static == [ref_items[ref_cb[c]:ref_cb[c + 1]] for c in range(G)]
+    return items, lists, queue
+
+
+def test_split_stack_at_100k_queues_the_full_layers_tails():
+    tiles = [3125 if (i % 7) in (3, 6) else 17 for i in range(49)]
+    items, lists, queue = check_split(tiles, 148)
+    queued = sum(items[i][2] - items[i][1] for i in queue)
+    assert queued == 14 * (3125 * 120 // 1000)
+    # guided sizes: ceil(remaining / 148), at least 8, largest first
+    rem, prev = queued, None
+    for i in queue:
+        size = items[i][2] - items[i][1]
+        want = max(8, -(-rem // 148))
+        assert size <= want
+        rem -= size
+    sizes = [items[i][2] - items[i][1] for i in queue]
+    assert sizes[0] == -(-queued // 148) and min(sizes) >= 1
+    assert len(items) <= 640
+
+
+def test_split_keeps_short_launches_static():
+    # one 100K layer on 148 CTAs is 21 tiles per CTA: no queue
+    items, lists, queue = check_split([3125], 148)
+    assert queue == [] and len(items) == 148
+    # 64 tiles per CTA and more: queued
+    assert check_split([64 * 148], 148)[2] != []
+    assert check_split([64 * 148 - 1], 148)[2] == []
+
+
+def test_split_falls_back_to_coarser_queues_then_none():
+    tiles = [3125 if (i % 7) in (3, 6) else 17 for i in range(49)]
+    full = check_split(tiles, 148)
+    small = check_split(tiles, 148, max_items=251)      # the no-alloc scratch
+    assert 0 < len(small[2]) < len(full[2])
+    static_only = check_split(tiles, 148, max_items=148 + 49)
+    assert static_only[2] == []
+
+
+def test_split_random_cases_and_determinism():
+    r = random.Random(11)
+    for _ in range(150):
+        n = r.randint(1, 64)
+        tiles = [r.choice([1, 2, 17, 63, 64, r.randint(1, 8192)]) for _ in range(n)]
+        G = r.randint(1, 296)
+        try:
+            a = check_split(tiles, G)
+        except flint.FlintError:
+            assert n + G > 640
+            continue
+        assert a == flint.flint_plan_split(tiles, G)

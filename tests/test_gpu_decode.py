@@ -25,8 +25,9 @@ def run_decode(q, k, v, seq_lens, sinks, window, layout=flint.CONTIGUOUS, capaci
                             dev_err=err)
     torch.cuda.synchronize()
     assert int(err.item()) == 0
-    # the library leaves the per-problem arrival counters at zero after a clean
-    # call (the grid-barrier word after them keeps only a generation bit)
+    # the library leaves the per-problem arrival counters and the queue head at
+    # zero after a clean call (the grid-barrier word between them keeps only a
+    # generation bit)
     assert int(ws[:256].view(torch.int32).abs().sum().item()) == 0
     assert int(ws[256:4096].view(torch.int32)[1:].abs().sum().item()) == 0
     return out.cpu().numpy()

@@ -50,6 +50,35 @@ def test_stack_split_invariance_and_determinism():
         np.testing.assert_allclose(o, outs[0], rtol=1e-4, atol=1e-5)
 
 
+def test_stack_workspace_sizes_agree_with_the_oracle():
+    """The run-time queue is sized by the workspace: the full workspace, the
+    no-alloc scratch's 251 partials and the static-plan minimum (no queue) give
+    three different plans; each agrees with the oracle, and with the others to
+    rounding."""
+    L = 20_000
+    layers = I.make_stack(L, workload=I.W_STACK_100K + 12)
+    dl = [DeviceLayer(l) for l in layers]
+    arr = flint.stack_layers(dl)
+    err = torch.zeros(1, dtype=torch.int32, device="cuda")
+    G = 148
+    outs = []
+    for items in (640, 251, G + 49):
+        ws = torch.zeros(4096 + items * 16640, dtype=torch.uint8, device="cuda")
+        out = torch.full((49, 32, 128), float("nan"), dtype=torch.float32, device="cuda")
+        flint.flint_attn_stack(arr, L - 1, out, ws, num_ctas=G, dev_err=err)
+        torch.cuda.synchronize()
+        assert int(err.item()) == 0
+        outs.append(out.cpu().numpy())
+    kinds = I.layer_kinds()
+    full = [i for i, f in enumerate(kinds) if f]
+    for o in outs:
+        for i in (full[0], full[-1], 0):
+            want, _, _ = oracle_layer(layers[i])
+            parity(o[i], want, f"layer {i}")
+    for o in outs[1:]:
+        np.testing.assert_allclose(o, outs[0], rtol=1e-4, atol=1e-5)
+
+
 def test_stack_100k_sampled_layers():
     """The full 49-layer stack at context 100,000, launched as the benchmark
     launches it; the oracle checks two full layers and three window layers

@@ -147,3 +147,130 @@ def test_round_robin_scheme_is_unsafe():
     rng = random.Random(2)
     errors = [simulate(200, "round_robin", rng) for _ in range(200)]
     assert any(e is not None for e in errors)
+
+
+# ---------------------------------------------------------------------------
+# The item hand-over: the producer picks each item (its static list, then
+# claims on the run-time queue), writes its index to a shared slot, and arms
+# the staged-input barrier; consumer warp 0 copies the slot to a second shared
+# word once its wait succeeds, all consumer warps meet at a named barrier and
+# read that word, and -1 tells them to stop.  In the kernel two things keep
+# warp 0 from rewriting that word while a warp still has to read it: every
+# warp reads it before it releases the inputs (arrive on in_empty), so the
+# next phase cannot be armed before, and an item's end includes another named
+# barrier.  The model checks, under random interleavings and random landing
+# times of the staged copies, that every warp reads the item the producer
+# chose for that phase, that the producer never rewrites the slot before warp
+# 0 copied it and that nobody deadlocks: with either protection alone, and
+# that with neither a warp can read the wrong item.
+
+def simulate_handover(items, rng, warps=8, item_end_barrier=True, release_after_read=True):
+    in_full, in_empty = Barrier(1), Barrier(warps)
+    slot, cur = None, None
+    landing = []              # staged copies in flight (phase k)
+    # producer state
+    pk, p_done, p_waiting_arm = 0, False, False
+    # consumer state per warp: phase k, step
+    ck = [0] * warps
+    step = ["wait"] * warps   # wait -> bar1 -> read -> (item) -> bar2 -> wait
+    seen = [[] for _ in range(warps)]
+    bar_count = {"b1": 0, "b2": 0}
+    bar_gen = {"b1": 0, "b2": 0}
+    at_bar = [None] * warps   # (name, gen) a warp is blocked at
+    plan = list(items) + [-1]
+    for _ in range(100000):
+        acts = []
+        if not p_done and in_empty.parity_done((pk & 1) ^ 1):
+            acts.append("produce")
+        if landing:
+            acts.append("land")
+        for w in range(warps):
+            st = step[w]
+            if st == "wait" and in_full.parity_done(ck[w] & 1):
+                acts.append(("wait", w))
+            elif st in ("bar1", "bar2"):
+                name, gen = at_bar[w]
+                if bar_gen[name] > gen:
+                    acts.append((st, w))
+            elif st in ("read", "item"):
+                acts.append((st, w))
+        if not acts:
+            break
+        a = rng.choice(acts)
+        if a == "produce":
+            it = plan[pk]
+            if slot is not None and cur != slot and pk > 0:
+                return f"slot rewritten at phase {pk} before warp 0 copied it"
+            slot = it
+            if it >= 0:
+                in_full.arrive(tx=1)
+                landing.append(pk)
+            else:
+                in_full.arrive()
+                p_done = True
+            pk += 1
+        elif a == "land":
+            landing.pop(rng.randrange(len(landing)))
+            in_full.complete_tx(1)
+        else:
+            kind, w = a
+            if kind == "wait":
+                if w == 0:
+                    cur = slot
+                if not release_after_read and plan[ck[w]] >= 0:
+                    in_empty.arrive()
+                step[w] = "bar1"
+                at_bar[w] = ("b1", bar_gen["b1"])
+                bar_count["b1"] += 1
+                if bar_count["b1"] == warps:
+                    bar_count["b1"] = 0
+                    bar_gen["b1"] += 1
+            elif kind == "bar1":
+                step[w] = "read"
+            elif kind == "read":
+                it = cur
+                seen[w].append(it)
+                if it != plan[ck[w]]:
+                    return f"warp {w} read item {it} for phase {ck[w]}, expected {plan[ck[w]]}"
+                if it < 0:
+                    step[w] = "done"
+                else:
+                    if release_after_read:
+                        in_empty.arrive()
+                    step[w] = "item"
+            elif kind == "item":
+                ck[w] += 1
+                if item_end_barrier:
+                    step[w] = "bar2"
+                    at_bar[w] = ("b2", bar_gen["b2"])
+                    bar_count["b2"] += 1
+                    if bar_count["b2"] == warps:
+                        bar_count["b2"] = 0
+                        bar_gen["b2"] += 1
+                else:
+                    step[w] = "wait"
+            elif kind == "bar2":
+                step[w] = "wait"
+    if not p_done or any(s != "done" for s in step):
+        return "deadlock"
+    if any(s != plan for s in seen):
+        return "a warp missed an item"
+    return None
+
+
+@pytest.mark.parametrize("item_end_barrier,release_after_read", [(True, True), (True, False), (False, True)])
+def test_item_handover_is_safe_under_random_interleavings(item_end_barrier, release_after_read):
+    rng = random.Random(7)
+    for trial in range(300):
+        items = [rng.randrange(600) for _ in range(rng.randint(0, 30))]
+        err = simulate_handover(items, rng, item_end_barrier=item_end_barrier,
+                                release_after_read=release_after_read)
+        assert err is None, f"trial {trial}: {err}"
+
+
+def test_item_handover_with_neither_protection_is_unsafe():
+    rng = random.Random(8)
+    errors = [simulate_handover([rng.randrange(600) for _ in range(20)], rng, item_end_barrier=False,
+                                release_after_read=False)
+              for _ in range(300)]
+    assert any(e is not None for e in errors)
