@@ -153,7 +153,7 @@ flint_status flint_kv_append(const uint16_t* k, const uint16_t* v, const int32_t
 
 /* Bytes of device workspace for flint_attn_decode / flint_attn_stack with
  * n_problems (requests, or layers) on num_ctas CTAs (0 = one per SM): room
- * for the full split plan, 4096 + 640 * 16640 bytes (10.6 MB).  A call also
+ * for the full split plan, 4096 + 768 * 16640 bytes (12.8 MB).  A call also
  * runs with less, down to 4096 + (CTAs + n_problems) * 16640 bytes, with a
  * coarser run-time balancing queue; below that it returns
  * FLINT_ERR_WORKSPACE.  The workspace holds split partials, per-problem
@@ -237,12 +237,13 @@ int32_t flint_plan_items(const int32_t* seg_tiles, int32_t n_segs, int32_t num_c
 
 /* The full plan of one attention launch (pure host code, exposed for tests):
  * when there are at least 64 tiles per CTA, the static plan of
- * flint_plan_items over the first ~88 % of every segment of at least 64
+ * flint_plan_items over the first ~80 % of every segment of at least 64
  * tiles (smaller ones stay whole), plus a queue of chunks that
  * cut the remaining tails, in guided sizes (ceil(remaining tiles / num_ctas),
  * at least 8), which CTAs claim at run time once their static lists are done.
- * Coarser queues, then none, are used when max_items is too small; with
- * fewer tiles per CTA the plan is static only.
+ * Coarser queues (chunks of at least 16 or 32 tiles, never above an eighth
+ * of a CTA's share), then none, are used when max_items is too small; with
+ * fewer than 64 tiles per CTA the plan is static only.
  * Outputs: item_seg/item_t0/item_t1 [max_items], sorted by (segment, t0);
  * order [max_items] and cta_begin [num_ctas + 1]: the static items of CTA c
  * are order[cta_begin[c] .. cta_begin[c+1]-1] and the queue is

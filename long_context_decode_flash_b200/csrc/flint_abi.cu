@@ -9,6 +9,7 @@
 #include <string.h>
 
 #include <algorithm>
+#include <cmath>
 #include <mutex>
 #include <string>
 #include <unordered_map>
@@ -40,8 +41,8 @@ bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) ==
 
 constexpr int kItemCost = 2;  // per-item overhead in tile units (planner cost model)
 // A deferred problem with more partials than this is merged a CTA per unit
-// (thread per partial) instead of a warp per unit.
-constexpr int kWideMergeItems = 64;
+// (thread per partial) instead of a warp per unit (lane per partial).
+constexpr int kWideMergeItems = 96;
 
 // ---- device properties (cached per device) --------------------------------
 
@@ -279,13 +280,15 @@ flint_status plan(DecodeParams& P, const int* tiles, int n_problems, int num_cta
   // finish near the end of the launch, where one CTA merging alone would be
   // the tail.
   P.n_deferred = 0;
-  P.merge_wide = 0;
-  for (int s = 0; s < n_segs; ++s) {
-    const int items = P.seg_item_begin[s + 1] - P.seg_item_begin[s];
-    const bool deferred = queued[s] || items > kInlineMergeMax;
-    P.prob[s].deferred = deferred ? 1 : 0;
-    if (deferred) P.deferred[P.n_deferred++] = static_cast<int16_t>(s);
-    if (deferred && items > kWideMergeItems) P.merge_wide = 1;
+  P.n_wide = 0;
+  for (int wide = 1; wide >= 0; --wide) {
+    for (int s = 0; s < n_segs; ++s) {
+      const int items = P.seg_item_begin[s + 1] - P.seg_item_begin[s];
+      const bool deferred = queued[s] || items > kInlineMergeMax;
+      P.prob[s].deferred = deferred ? 1 : 0;
+      if (deferred && (items > kWideMergeItems) == (wide == 1)) P.deferred[P.n_deferred++] = static_cast<int16_t>(s);
+    }
+    if (wide) P.n_wide = P.n_deferred;
   }
   P.grid_merge = (P.n_deferred > 0 || P.n_queue > 0) ? 1 : 0;
   P.ws_items = cap;
@@ -505,7 +508,6 @@ flint_status flint_attn_decode(const void* q, int32_t q_is_fp32, const flint_kv_
   P.n_problems = B;
   P.prep = 0;
   P.eps = 0.f;
-  P.theta = 0.0;
   return launch_result(launch_decode(P, grid, static_cast<cudaStream_t>(stream)), who);
 }
 
@@ -581,7 +583,12 @@ flint_status flint_attn_stack(const flint_layer* layers, int32_t n_layers, int32
   P.n_problems = n_layers;
   P.prep = 1;
   P.eps = eps;
-  P.theta = theta;
+  // RoPE angles of the new token, pos * theta^(-2i/128) for i < 64, in double
+  // on the host (one position for every layer of the call)
+  for (int i = 0; i < kDim / 2; ++i) {
+    const double a = static_cast<double>(pos) * std::pow(theta, -2.0 * i / kDim);
+    P.rope_cs[i] = make_float2(static_cast<float>(std::cos(a)), static_cast<float>(std::sin(a)));
+  }
   return launch_result(launch_decode(P, grid, static_cast<cudaStream_t>(stream)), who);
 }
 

@@ -192,6 +192,9 @@ __device__ ProducerCount run_producer(const DecodeParams& P, const Smem& S, int 
   int seq = 0;
   // lane i < 16 issues box i: K/V (i >> 3), head ((i >> 1) & 3), dim half (i & 1)
   const int my_kv = (lane >> 3) & 1, my_head = (lane >> 1) & 3, my_half = lane & 1;
+#if FLINT_KV_EVICT_FIRST
+  const uint64_t kv_policy = l2_policy_evict_first();
+#endif
   for (int k = 0;; ++k) {
     int it = -1;
     {  // pick the next item once the consumers released the last inputs, and
@@ -276,8 +279,14 @@ __device__ ProducerCount run_producer(const DecodeParams& P, const Smem& S, int 
         }
         fine = __shfl_sync(0xffffffffu, fine, 0);
         __syncwarp();
-        if (fine && lane < kBoxes)
+        if (fine && lane < kBoxes) {
+#if FLINT_KV_EVICT_FIRST
+          tma_load_4d_hint(base + box_offset(my_kv, my_head, my_half), map, fb, 64 * my_half, my_head, c2,
+                           c3, kv_policy);
+#else
           tma_load_4d(base + box_offset(my_kv, my_head, my_half), map, fb, 64 * my_half, my_head, c2, c3);
+#endif
+        }
         __syncwarp();
       }
     }
@@ -441,15 +450,20 @@ __device__ __forceinline__ void consume_slice(uint32_t sK, uint32_t sV, int tok0
   }
 }
 
-// Offset (floats) of consumer thread (head, c)'s 32 O values inside a partial.
-__device__ __forceinline__ int partial_o(int head, int c) { return (head * 4 + c) * 32; }
+// Float4 slot of values 4q..4q+3 of consumer thread (head, c)'s 32 O values
+// inside a partial.  The 32 threads of a KV head's warp (lane = 4(head % 8) + c)
+// hold chunk q in 512 consecutive bytes, so a warp's load or store of one
+// chunk touches 4 cache lines, not 32.
+__device__ __forceinline__ int partial_f4(int head, int c, int q) {
+  return ((head >> 3) * 8 + q) * 32 + (head & 7) * 4 + c;
+}
 
 // out[head][8n + 2c + e] = O * 2^(M - Mf) / (L 2^(M - Mf) + 2^(sink - Mf)), the
 // sink logit of this head folded into the softmax; thread (g, c) owns dims
 // 8n + 2c + {0,1} of head `head`.
 __device__ __forceinline__ void finish_head(const Problem& pb, int head, int c, float M, float L,
-                                            const float (&v)[32]) {
-  const float s2 = pb.sinks[head] * kLog2e;
+                                            const float (&v)[32], float sink) {
+  const float s2 = sink * kLog2e;
   const float Mf = fmaxf(M, s2);
   const float a = (M == -INFINITY) ? 0.f : exp2f(M - Mf);
   const float scale = a / (L * a + exp2f(s2 - Mf));
@@ -457,6 +471,79 @@ __device__ __forceinline__ void finish_head(const Problem& pb, int head, int c, 
 #pragma unroll
   for (int n = 0; n < 16; ++n)
     *reinterpret_cast<float2*>(dst + 8 * n) = make_float2(v[2 * n] * scale, v[2 * n + 1] * scale);
+}
+
+// Folds partials i = s0 + r, s0 + r + stride, ... (< s1) of (head, quarter c)
+// into a running (m, l, v), in increasing i.
+__device__ __forceinline__ void fold_partials(const DecodeParams& P, int s0, int s1, int r, int stride,
+                                              int head, int c, float& m, float& l, float (&v)[32]) {
+  // two partials per round, both loaded before either is folded
+  for (int i = s0 + r; i < s1; i += 2 * stride) {
+    float mi[2], li[2];
+    float4 ov[2][8];
+#pragma unroll
+    for (int j = 0; j < 2; ++j) {
+      const int ij = i + j * stride;
+      const float* pi = P.partials + static_cast<size_t>(ij < s1 ? ij : i) * kPartialFloats;
+      mi[j] = ij < s1 ? __ldcg(pi + kHeads * kDim + head) : -INFINITY;
+      li[j] = __ldcg(pi + kHeads * kDim + kHeads + head);
+      const float4* po = reinterpret_cast<const float4*>(pi);
+#pragma unroll
+      for (int q = 0; q < 8; ++q) ov[j][q] = __ldcg(po + partial_f4(head, c, q));
+    }
+#pragma unroll
+    for (int j = 0; j < 2; ++j) {
+      const float mn = fmaxf(m, mi[j]);
+      const float sa = (m == -INFINITY) ? 0.f : exp2f(m - mn);
+      const float sb = (mi[j] == -INFINITY) ? 0.f : exp2f(mi[j] - mn);
+#pragma unroll
+      for (int q = 0; q < 8; ++q) {
+        v[4 * q] = v[4 * q] * sa + ov[j][q].x * sb;
+        v[4 * q + 1] = v[4 * q + 1] * sa + ov[j][q].y * sb;
+        v[4 * q + 2] = v[4 * q + 2] * sa + ov[j][q].z * sb;
+        v[4 * q + 3] = v[4 * q + 3] * sa + ov[j][q].w * sb;
+      }
+      l = l * sa + li[j] * sb;
+      m = mn;
+    }
+  }
+}
+
+// Rescales a lane's (m, l, v) to the common max M, then sums l over the warp
+// and reduce-scatters v: afterwards lane k holds the warp's sum of value k.
+__device__ __forceinline__ void warp_sum_at(float m, float M, float& l, float (&v)[32], int lane) {
+  const float sc = (m == -INFINITY) ? 0.f : exp2f(m - M);
+  l *= sc;
+#pragma unroll
+  for (int e = 0; e < 32; ++e) v[e] *= sc;
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) l += __shfl_xor_sync(0xffffffffu, l, o);
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) {
+    const bool up = (lane & o) != 0;
+#pragma unroll
+    for (int j = 0; j < o; ++j) {
+      const float send = up ? v[j] : v[j + o];
+      const float keep = up ? v[j + o] : v[j];
+      v[j] = keep + __shfl_xor_sync(0xffffffffu, send, o);
+    }
+  }
+}
+
+__device__ __forceinline__ float warp_max(float x) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) x = fmaxf(x, __shfl_xor_sync(0xffffffffu, x, o));
+  return x;
+}
+
+// Value t of quarter c of a head, with the sink folded in.
+__device__ __forceinline__ void write_merged(const Problem& pb, int head, int c, int t, float M, float L,
+                                             float sum, float sink) {
+  const float s2 = sink * kLog2e;
+  const float Mf = fmaxf(M, s2);
+  const float a = (M == -INFINITY) ? 0.f : exp2f(M - Mf);
+  const float scale = a / (L * a + exp2f(s2 - Mf));
+  pb.out[head * kDim + 8 * (t >> 1) + 2 * c + (t & 1)] = sum * scale;
 }
 
 __device__ void run_consumer(const DecodeParams& P, const Smem& S, int warp, int lane) {
@@ -481,6 +568,8 @@ __device__ void run_consumer(const DecodeParams& P, const Smem& S, int warp, int
     if (it < 0) break;
     const Item item = P.items[it];
     const Problem& pb = P.prob[item.seg];
+    // this head's sink logit, needed only at the item's end: load it now
+    const float sink = pb.sinks[head];
     {
       load_q(P, pb, S.in, head, c, S.cs, qa);
       if (P.prep && warp == kAppendWarp && pb.append_tok >= 0) {
@@ -562,7 +651,7 @@ __device__ void run_consumer(const DecodeParams& P, const Smem& S, int warp, int
     }
     const int s0 = P.seg_item_begin[item.seg], s1 = P.seg_item_begin[item.seg + 1];
     if (s1 - s0 == 1) {
-      if (group == 0) finish_head(pb, head, c, m_run, l_run, v);
+      if (group == 0) finish_head(pb, head, c, m_run, l_run, v, sink);
       __syncwarp();
       consumer_bar();  // the hand-over area is reused by the next item
       continue;
@@ -570,71 +659,61 @@ __device__ void run_consumer(const DecodeParams& P, const Smem& S, int warp, int
     float* part = P.partials + static_cast<size_t>(it) * kPartialFloats;
     if (group == 0 &&
         FLINT_CHECK(P.dev_err, it < P.ws_items && s0 >= 0 && s1 <= P.n_items, 7, it, s0, s1)) {
-      float4* pd = reinterpret_cast<float4*>(part + partial_o(head, c));
+      float4* pd = reinterpret_cast<float4*>(part);
 #pragma unroll
-      for (int i = 0; i < 8; ++i) pd[i] = make_float4(v[4 * i], v[4 * i + 1], v[4 * i + 2], v[4 * i + 3]);
+      for (int q = 0; q < 8; ++q)
+        pd[partial_f4(head, c, q)] = make_float4(v[4 * q], v[4 * q + 1], v[4 * q + 2], v[4 * q + 3]);
       if (c == 0) {
         part[kHeads * kDim + head] = m_run;
         part[kHeads * kDim + kHeads + head] = l_run;
       }
     }
-    __threadfence();
-    if (pb.deferred) {  // merged by the whole grid after the grid barrier
-      __syncwarp();
-      consumer_bar();
-      continue;
-    }
     __syncwarp();
     consumer_bar();
+    // A deferred problem is merged after the grid barrier, whose fence
+    // releases these partials.  Otherwise one thread releases them (the
+    // barrier above orders every consumer's stores before its fence) and
+    // counts the arrival; the last CTA to arrive merges.
+    if (pb.deferred) continue;
     if (threadIdx.x == 0) {
       int prev = 0;
+      __threadfence();
       if (FLINT_CHECK(P.dev_err, item.seg < kMaxSegs, 8, item.seg, 0, 0))
         prev = atomicAdd(P.counters + item.seg, 1);
+      __threadfence();
       S.flags[1] = (prev == s1 - s0 - 1) ? 1 : 0;
     }
-    __syncwarp();
     consumer_bar();
-    if (S.flags[1] && group == 0) {
-      // last arrival: merge every partial of the problem, in item order,
-      // four partials' loads in flight at a time
-      __threadfence();
-      float M = -INFINITY;
-      for (int i = s0; i < s1; ++i)
-        M = fmaxf(M, __ldcg(P.partials + static_cast<size_t>(i) * kPartialFloats + kHeads * kDim + head));
-      float L = 0.f;
+    if (S.flags[1]) {
+      // last arrival: both groups fold half of the problem's partials each
+      // (items s0 + group, s0 + group + 2, ...; two loads in flight per
+      // thread), then group 1 hands its state to group 0, which finishes
+      float mm = -INFINITY, ll = 0.f;
 #pragma unroll
       for (int e = 0; e < 32; ++e) v[e] = 0.f;
-      for (int i0 = s0; i0 < s1; i0 += 4) {
-        float sw[4], lw[4];
-        float4 ow[4][8];
+      fold_partials(P, s0, s1, group, kConsumerGroups, head, c, mm, ll, v);
+      float* mine = S.xch + (kvh * 32 + lane) * kXchFloats;
+      if (group == 1) {
 #pragma unroll
-        for (int j = 0; j < 4; ++j) {
-          const int i = min(i0 + j, s1 - 1);
-          const float* pi = P.partials + static_cast<size_t>(i) * kPartialFloats;
-          const float mi = __ldcg(pi + kHeads * kDim + head);
-          sw[j] = (i0 + j >= s1 || mi == -INFINITY) ? 0.f : exp2f(mi - M);
-          lw[j] = __ldcg(pi + kHeads * kDim + kHeads + head);
-          const float4* po = reinterpret_cast<const float4*>(pi + partial_o(head, c));
-#pragma unroll
-          for (int q = 0; q < 8; ++q) ow[j][q] = __ldcg(po + q);
-        }
-#pragma unroll
-        for (int j = 0; j < 4; ++j) {
-          L += sw[j] * lw[j];
-#pragma unroll
-          for (int q = 0; q < 8; ++q) {
-            v[4 * q] += sw[j] * ow[j][q].x;
-            v[4 * q + 1] += sw[j] * ow[j][q].y;
-            v[4 * q + 2] += sw[j] * ow[j][q].z;
-            v[4 * q + 3] += sw[j] * ow[j][q].w;
-          }
-        }
+        for (int e = 0; e < 32; ++e) mine[e] = v[e];
+        mine[32] = mm;
+        mine[33] = ll;
       }
-      finish_head(pb, head, c, M, L, v);
-      if (threadIdx.x == 0) P.counters[item.seg] = 0;  // ready for the next call
+      __syncwarp();
+      consumer_bar();
+      if (group == 0) {
+        const float mo = mine[32], lo_ = mine[33];
+        const float M = fmaxf(mm, mo);
+        const float sa = (mm == -INFINITY) ? 0.f : exp2f(mm - M);
+        const float sb = (mo == -INFINITY) ? 0.f : exp2f(mo - M);
+#pragma unroll
+        for (int e = 0; e < 32; ++e) v[e] = v[e] * sa + mine[e] * sb;
+        finish_head(pb, head, c, M, ll * sa + lo_ * sb, v, sink);
+        if (threadIdx.x == 0) P.counters[item.seg] = 0;  // ready for the next call
+      }
     }
     __syncwarp();
-    consumer_bar();  // flags[1] is reused by the next item
+    consumer_bar();  // flags[1] and the hand-over area are reused by the next item
   }
 }
 
@@ -658,7 +737,7 @@ __device__ bool grid_barrier(unsigned int* bar, const Smem& S) {
         ok = 0;
         break;
       }
-      __nanosleep(64);
+      __nanosleep(20);
     }
     __threadfence();
     S.flags[2] = ok;
@@ -667,98 +746,77 @@ __device__ bool grid_barrier(unsigned int* bar, const Smem& S) {
   return S.flags[2] != 0;
 }
 
-// Folds partials i = s0 + r, s0 + r + stride, ... (< s1) of (head, quarter c)
-// into a running (m, l, v), in increasing i.
-__device__ __forceinline__ void fold_partials(const DecodeParams& P, int s0, int s1, int r, int stride,
-                                              int head, int c, float& m, float& l, float (&v)[32]) {
-  for (int i = s0 + r; i < s1; i += stride) {
-    const float* pi = P.partials + static_cast<size_t>(i) * kPartialFloats;
-    const float mi = __ldcg(pi + kHeads * kDim + head);
-    const float li = __ldcg(pi + kHeads * kDim + kHeads + head);
-    const float4* po = reinterpret_cast<const float4*>(pi + partial_o(head, c));
-    float4 ov[8];
-#pragma unroll
-    for (int q = 0; q < 8; ++q) ov[q] = __ldcg(po + q);
-    const float mn = fmaxf(m, mi);
-    const float sa = (m == -INFINITY) ? 0.f : exp2f(m - mn);
-    const float sb = (mi == -INFINITY) ? 0.f : exp2f(mi - mn);
-#pragma unroll
-    for (int q = 0; q < 8; ++q) {
-      v[4 * q] = v[4 * q] * sa + ov[q].x * sb;
-      v[4 * q + 1] = v[4 * q + 1] * sa + ov[q].y * sb;
-      v[4 * q + 2] = v[4 * q + 2] * sa + ov[q].z * sb;
-      v[4 * q + 3] = v[4 * q + 3] * sa + ov[q].w * sb;
-    }
-    l = l * sa + li * sb;
-    m = mn;
-  }
-}
+// Merge of the deferred problems by the whole grid after the grid barrier.
+//   * Most problems: one warp per (problem, KV head g, chunk q) unit.  Lane
+//     (h, c) of the warp owns values 4q..4q+3 of head 8g + h, quarter c (the
+//     layout the consumer warps wrote), so one warp load reads 512
+//     consecutive bytes of a partial; each lane folds every partial of the
+//     problem, kMergeBatch loads in flight at a time, in item order.
+//   * A problem with many partials (a lone long problem split over every
+//     CTA) takes a whole CTA per (head, quarter c) unit instead, one thread
+//     per partial, then a block reduction; value k of a quarter is dim
+//     8(k/2) + 2c + (k & 1) of the head.
+constexpr int kMergeBatch = 16;
 
-// Rescales a lane's (m, l, v) to the common max M, then sums l over the warp
-// and reduce-scatters v: afterwards lane k holds the warp's sum of value k.
-__device__ __forceinline__ void warp_sum_at(float m, float M, float& l, float (&v)[32], int lane) {
-  const float sc = (m == -INFINITY) ? 0.f : exp2f(m - M);
-  l *= sc;
-#pragma unroll
-  for (int e = 0; e < 32; ++e) v[e] *= sc;
-#pragma unroll
-  for (int o = 16; o > 0; o >>= 1) l += __shfl_xor_sync(0xffffffffu, l, o);
-#pragma unroll
-  for (int o = 16; o > 0; o >>= 1) {
-    const bool up = (lane & o) != 0;
-#pragma unroll
-    for (int j = 0; j < o; ++j) {
-      const float send = up ? v[j] : v[j + o];
-      const float keep = up ? v[j + o] : v[j];
-      v[j] = keep + __shfl_xor_sync(0xffffffffu, send, o);
-    }
-  }
-}
-
-__device__ __forceinline__ float warp_max(float x) {
-#pragma unroll
-  for (int o = 16; o > 0; o >>= 1) x = fmaxf(x, __shfl_xor_sync(0xffffffffu, x, o));
-  return x;
-}
-
-// Value t of quarter c of a head, with the sink folded in.
-__device__ __forceinline__ void write_merged(const Problem& pb, int head, int c, int t, float M, float L,
-                                             float sum) {
-  const float s2 = pb.sinks[head] * kLog2e;
-  const float Mf = fmaxf(M, s2);
-  const float a = (M == -INFINITY) ? 0.f : exp2f(M - Mf);
-  const float scale = a / (L * a + exp2f(s2 - Mf));
-  pb.out[head * kDim + 8 * (t >> 1) + 2 * c + (t & 1)] = sum * scale;
-}
-
-// Merge of the deferred problems by the whole grid after the grid barrier, in
-// units of (problem, head, quarter c); value k of a quarter is dim
-// 8(k/2) + 2c + (k & 1) of the head.  Problems with few partials take one
-// warp per unit (lane j folds partials j, j + 32, ...); with many partials
-// (a lone long problem split over every CTA) a unit takes a whole CTA, one
-// thread per partial, so that all of a unit's loads are in flight at once.
 __device__ void grid_merge(const DecodeParams& P, const Smem& S) {
   constexpr int kWarps = kThreads / 32;
   const int t = threadIdx.x, lane = t & 31, warp = t >> 5;
-  const int units = P.n_deferred * kHeads * 4;
-  if (!P.merge_wide) {
+  {
+    const int units = (P.n_deferred - P.n_wide) * kKvHeads * 8;
     for (int u = blockIdx.x * kWarps + warp; u < units; u += gridDim.x * kWarps) {
-      const int p = P.deferred[u / (kHeads * 4)];
-      const int head = (u / 4) % kHeads, c = u % 4;
-      float m = -INFINITY, l = 0.f, v[32];
+      const int p = P.deferred[P.n_wide + u / (kKvHeads * 8)];
+      const int kvh = (u / 8) % kKvHeads, q = u % 8;
+      const int head = kvh * kGroup + (lane >> 2), c = lane & 3;
+      const Problem& pb = P.prob[p];
+      const float sink = pb.sinks[head];  // in flight with the partials
+      const int s0 = P.seg_item_begin[p], s1 = P.seg_item_begin[p + 1];
+      float m = -INFINITY, l = 0.f;
+      float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+      for (int i0 = s0; i0 < s1; i0 += kMergeBatch) {
+        float mi[kMergeBatch], li[kMergeBatch];
+        float4 vi[kMergeBatch];
 #pragma unroll
-      for (int e = 0; e < 32; ++e) v[e] = 0.f;
-      fold_partials(P, P.seg_item_begin[p], P.seg_item_begin[p + 1], lane, 32, head, c, m, l, v);
-      const float M = warp_max(m);
-      warp_sum_at(m, M, l, v, lane);
-      write_merged(P.prob[p], head, c, lane, M, l, v[0]);
+        for (int j = 0; j < kMergeBatch; ++j) {
+          const int i = min(i0 + j, s1 - 1);
+          const float* pi = P.partials + static_cast<size_t>(i) * kPartialFloats;
+          mi[j] = i0 + j < s1 ? __ldcg(pi + kHeads * kDim + head) : -INFINITY;
+          li[j] = __ldcg(pi + kHeads * kDim + kHeads + head);
+          vi[j] = __ldcg(reinterpret_cast<const float4*>(pi) + partial_f4(head, c, q));
+        }
+        float mn = m;
+#pragma unroll
+        for (int j = 0; j < kMergeBatch; ++j) mn = fmaxf(mn, mi[j]);
+        const float sa = (m == -INFINITY) ? 0.f : exp2f(m - mn);
+        l *= sa;
+        acc = make_float4(acc.x * sa, acc.y * sa, acc.z * sa, acc.w * sa);
+        m = mn;
+#pragma unroll
+        for (int j = 0; j < kMergeBatch; ++j) {
+          const float sb = (mi[j] == -INFINITY) ? 0.f : exp2f(mi[j] - m);
+          l += sb * li[j];
+          acc.x += sb * vi[j].x;
+          acc.y += sb * vi[j].y;
+          acc.z += sb * vi[j].z;
+          acc.w += sb * vi[j].w;
+        }
+      }
+      // values 4q..4q+3 of thread (head, c) are dims 16q + 2c + {0, 1} and
+      // 16q + 8 + 2c + {0, 1}; fold in the sink as finish_head does
+      const float s2 = sink * kLog2e;
+      const float Mf = fmaxf(m, s2);
+      const float a = (m == -INFINITY) ? 0.f : exp2f(m - Mf);
+      const float scale = a / (l * a + exp2f(s2 - Mf));
+      float* o = pb.out + head * kDim + 16 * q + 2 * c;
+      *reinterpret_cast<float2*>(o) = make_float2(acc.x * scale, acc.y * scale);
+      *reinterpret_cast<float2*>(o + 8) = make_float2(acc.z * scale, acc.w * scale);
     }
-    return;
   }
   float* red = S.xch;  // [kWarps][34] scratch (the hand-over area is free now)
+  const int units = P.n_wide * kHeads * 4;
   for (int u = blockIdx.x; u < units; u += gridDim.x) {
     const int p = P.deferred[u / (kHeads * 4)];
     const int head = (u / 4) % kHeads, c = u % 4;
+    const float sink = P.prob[p].sinks[head];  // in flight with the partials
     float m = -INFINITY, l = 0.f, v[32];
 #pragma unroll
     for (int e = 0; e < 32; ++e) v[e] = 0.f;
@@ -781,7 +839,7 @@ __device__ void grid_merge(const DecodeParams& P, const Smem& S) {
         sum += red[w * 34 + t];
         L += red[w * 34 + 32];
       }
-      write_merged(P.prob[p], head, c, t, M, L, sum);
+      write_merged(P.prob[p], head, c, t, M, L, sum, sink);
     }
     __syncthreads();  // red is reused by the next unit
   }
@@ -816,7 +874,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const __grid_consta
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
     asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
   }
-  if (P.prep && threadIdx.x < 64) S.cs[threadIdx.x] = rope_cos_sin(threadIdx.x, P.prob[0].pos, P.theta);
+  if (P.prep && threadIdx.x < kDim / 2) S.cs[threadIdx.x] = P.rope_cs[threadIdx.x];
   __syncthreads();
 
   ProducerCount pc{0, 0};

@@ -24,6 +24,9 @@ constexpr int kBlock = FLINT_BLOCK_SIZE;      // 64
 #ifndef FLINT_TILE
 #define FLINT_TILE 32
 #endif
+#ifndef FLINT_KV_EVICT_FIRST
+#define FLINT_KV_EVICT_FIRST 1                // KV tiles loaded with an L2 evict-first hint
+#endif
 #ifndef FLINT_L2_PROMOTION
 #define FLINT_L2_PROMOTION 3                  // CU_TENSOR_MAP_L2_PROMOTION_L2_256B
 #endif
@@ -49,7 +52,7 @@ static_assert(kTile % kSlice == 0, "a tile splits into 16-token slices");
 constexpr int kMaxProblems = 64;
 constexpr int kMaxSegs = kMaxProblems;         // one segment per problem
 constexpr int kMaxMaps = 2 * FLINT_MAX_LAYERS;
-constexpr int kMaxItems = 640;
+constexpr int kMaxItems = 768;
 constexpr int kMaxCtas = 296;
 
 // A problem split into more than kInlineMergeMax items is not merged by its
@@ -57,8 +60,9 @@ constexpr int kMaxCtas = 296;
 // launch) but by all warps of the grid after a grid barrier.
 constexpr int kInlineMergeMax = 16;
 
-// One split partial of a problem: O for 32 heads (stored so that each
-// consumer thread's 32 values are contiguous), m [32] (log2 units), l [32].
+// One split partial of a problem: O for 32 heads (in the order the consumer
+// warps hold it, chunk-interleaved across each warp's lanes), m [32] (log2
+// units), l [32].
 constexpr int kPartialFloats = kHeads * kDim + 2 * kHeads;
 constexpr size_t kCounterBytes = 4096;
 // int32 slots of the workspace's counter area: [0, kMaxSegs) per-problem
@@ -109,16 +113,16 @@ struct DecodeParams {
   int32_t* counters;        // workspace: per-segment arrival counters
   float* partials;          // workspace: one partial per item
   int32_t* dev_err;         // [0] status; debug builds also record a failed check in [2..7]
-  double theta;
+  float2 rope_cs[kDim / 2]; // prep: cos, sin of pos * theta^(-2i/128), from the host in double
   float eps;
   int32_t n_problems;
   int32_t prep;             // 1: q/k norm (+RoPE) and append fused in (layer stack)
   int32_t n_items;          // items in the plan
   int32_t grid_merge;       // 1: a grid barrier ends the launch (cooperative launch):
                             // some problem is deferred or the queue is not empty
-  int16_t deferred[kMaxProblems];  // the deferred problems
+  int16_t deferred[kMaxProblems];  // the deferred problems, those with many partials first
   int32_t n_deferred;
-  int32_t merge_wide;       // 1: a deferred problem has many partials: a CTA per merge unit
+  int32_t n_wide;           // deferred[0, n_wide): merged a CTA per unit, the rest a warp per unit
   int32_t ws_items;         // partial slots in the workspace
   int32_t smem_bytes;       // dynamic shared memory of the launch
 };

@@ -80,7 +80,7 @@ extern "C" int32_t flint_plan_items(const int32_t* seg_tiles, int32_t n_segs, in
 // A static plan fixes every CTA's work before the launch, but CTAs do not
 // stream at the same rate (on B200 a fixed set of SMs reads ~10 % slower than
 // the rest while all of them stream), so the fast ones idle at the end.  Here
-// each large segment keeps only its first ~88 % of tiles in the static plan;
+// each large segment keeps only its first ~80 % of tiles in the static plan;
 // its tail is cut into chunks that CTAs claim from a shared queue once their
 // static lists are done.  Chunk sizes follow guided self-scheduling over the
 // whole pool (ceil(remaining / CTAs), never below a floor), so early claims are
@@ -104,7 +104,9 @@ struct Variant {
   int chunk_min;  // smallest chunk, tiles
 };
 // Tried in order until the plan fits max_items; the last one is static only.
-constexpr Variant kVariants[] = {{120, 8}, {120, 16}, {120, 32}, {120, 64}, {60, 64}, {0, 0}};
+// A variant whose smallest chunk exceeds an eighth of a CTA's share is
+// skipped: a chunk that large taken late would itself be the tail.
+constexpr Variant kVariants[] = {{200, 8}, {200, 16}, {200, 32}, {100, 32}, {0, 0}};
 
 }  // namespace
 
@@ -126,7 +128,7 @@ extern "C" int32_t flint_plan_split(const int32_t* seg_tiles, int32_t n_segs, in
   };
   constexpr int32_t kQueue = 1 << 20;
   for (const Variant& v : kVariants) {
-    if (!queue_pays && v.permille > 0) continue;
+    if (v.permille > 0 && (!queue_pays || static_cast<int64_t>(v.chunk_min) * 8 * num_ctas > total)) continue;
     int64_t pool = 0;
     for (int32_t s = 0; s < n_segs; ++s) {
       const int32_t d = (v.permille > 0 && seg_tiles[s] >= kDynMinTiles)

@@ -245,7 +245,7 @@ def flint_plan_items(seg_tiles: Sequence[int], num_ctas: int, item_cost: int = 2
 
 
 def flint_plan_split(seg_tiles: Sequence[int], num_ctas: int, item_cost: int = 2,
-                     max_items: int = 640):
+                     max_items: int = 768):
     """Returns (items [(seg, t0, t1)] sorted by segment, static lists [[item
     index, ...] per CTA], queue [item index, ...]) from the C planner."""
     n = len(seg_tiles)

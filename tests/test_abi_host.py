@@ -120,8 +120,8 @@ def test_stack_and_prep_reject_bad_arguments_on_the_host():
 def test_workspace_bytes_bounds():
     assert flint.flint_attn_workspace_bytes(0, 148) == 0
     assert flint.flint_attn_workspace_bytes(65, 148) == 0
-    # room for the largest plan: 640 partials of (32*128 + 2*32) floats
-    full = 4096 + 640 * 16640
+    # room for the largest plan: 768 partials of (32*128 + 2*32) floats
+    full = 4096 + 768 * 16640
     assert flint.flint_attn_workspace_bytes(1, 148) == full
     assert flint.flint_attn_workspace_bytes(49, 148) == full
 
@@ -201,7 +201,7 @@ def test_plan_rejects_bad_arguments():
 
 # ------------------------------------------------- planner with a queue -----
 
-def check_split(seg_tiles, G, max_items=640, cost=2):
+def check_split(seg_tiles, G, max_items=768, cost=2):
     items, lists, queue = flint.flint_plan_split(seg_tiles, G, cost, max_items)
     n = len(items)
     assert n <= max_items
@@ -238,7 +238,7 @@ def test_split_stack_at_100k_queues_the_full_layers_tails():
     tiles = [3125 if (i % 7) in (3, 6) else 17 for i in range(49)]
     items, lists, queue = check_split(tiles, 148)
     queued = sum(items[i][2] - items[i][1] for i in queue)
-    assert queued == 14 * (3125 * 120 // 1000)
+    assert queued == 14 * (3125 * 200 // 1000)
     # guided sizes: ceil(remaining / 148), at least 8, largest first
     rem, prev = queued, None
     for i in queue:
@@ -248,7 +248,7 @@ def test_split_stack_at_100k_queues_the_full_layers_tails():
         rem -= size
     sizes = [items[i][2] - items[i][1] for i in queue]
     assert sizes[0] == -(-queued // 148) and min(sizes) >= 1
-    assert len(items) <= 640
+    assert len(items) <= 768
 
 
 def test_split_keeps_short_launches_static():
@@ -263,8 +263,10 @@ def test_split_keeps_short_launches_static():
 def test_split_falls_back_to_coarser_queues_then_none():
     tiles = [3125 if (i % 7) in (3, 6) else 17 for i in range(49)]
     full = check_split(tiles, 148)
-    small = check_split(tiles, 148, max_items=251)      # the no-alloc scratch
+    small = check_split(tiles, 148, max_items=500)
     assert 0 < len(small[2]) < len(full[2])
+    # the no-alloc scratch (251 partials) has no room for a useful queue
+    assert check_split(tiles, 148, max_items=251)[2] == []
     static_only = check_split(tiles, 148, max_items=148 + 49)
     assert static_only[2] == []
 
@@ -278,6 +280,6 @@ def test_split_random_cases_and_determinism():
         try:
             a = check_split(tiles, G)
         except flint.FlintError:
-            assert n + G > 640
+            assert n + G > 768
             continue
         assert a == flint.flint_plan_split(tiles, G)

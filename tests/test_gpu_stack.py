@@ -62,7 +62,7 @@ def test_stack_workspace_sizes_agree_with_the_oracle():
     err = torch.zeros(1, dtype=torch.int32, device="cuda")
     G = 148
     outs = []
-    for items in (640, 251, G + 49):
+    for items in (768, 251, G + 49):
         ws = torch.zeros(4096 + items * 16640, dtype=torch.uint8, device="cuda")
         out = torch.full((49, 32, 128), float("nan"), dtype=torch.float32, device="cuda")
         flint.flint_attn_stack(arr, L - 1, out, ws, num_ctas=G, dev_err=err)
