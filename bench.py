@@ -37,7 +37,7 @@ NOMINAL_HBM_GBS = 8000.0
 # launch from a full-size, one-pass ncu capture of the stack at context 100,000
 # (profiles/decode_kernel_stack100k_traffic.md), with the hash of the CUDA
 # sources it was taken on; reported only while the sources still hash the same.
-TRAFFIC = {("stack", 100_000): (2_910_554_624 + 9_261_056, "c72c100956b29b04")}
+TRAFFIC = {("stack", 100_000): (2_905_856_000 + 6_322_176, "58f64013b925776a")}
 
 
 def kernel_sources_hash() -> str:

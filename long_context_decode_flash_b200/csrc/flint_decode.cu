@@ -509,43 +509,6 @@ __device__ __forceinline__ void fold_partials(const DecodeParams& P, int s0, int
   }
 }
 
-// Rescales a lane's (m, l, v) to the common max M, then sums l over the warp
-// and reduce-scatters v: afterwards lane k holds the warp's sum of value k.
-__device__ __forceinline__ void warp_sum_at(float m, float M, float& l, float (&v)[32], int lane) {
-  const float sc = (m == -INFINITY) ? 0.f : exp2f(m - M);
-  l *= sc;
-#pragma unroll
-  for (int e = 0; e < 32; ++e) v[e] *= sc;
-#pragma unroll
-  for (int o = 16; o > 0; o >>= 1) l += __shfl_xor_sync(0xffffffffu, l, o);
-#pragma unroll
-  for (int o = 16; o > 0; o >>= 1) {
-    const bool up = (lane & o) != 0;
-#pragma unroll
-    for (int j = 0; j < o; ++j) {
-      const float send = up ? v[j] : v[j + o];
-      const float keep = up ? v[j + o] : v[j];
-      v[j] = keep + __shfl_xor_sync(0xffffffffu, send, o);
-    }
-  }
-}
-
-__device__ __forceinline__ float warp_max(float x) {
-#pragma unroll
-  for (int o = 16; o > 0; o >>= 1) x = fmaxf(x, __shfl_xor_sync(0xffffffffu, x, o));
-  return x;
-}
-
-// Value t of quarter c of a head, with the sink folded in.
-__device__ __forceinline__ void write_merged(const Problem& pb, int head, int c, int t, float M, float L,
-                                             float sum, float sink) {
-  const float s2 = sink * kLog2e;
-  const float Mf = fmaxf(M, s2);
-  const float a = (M == -INFINITY) ? 0.f : exp2f(M - Mf);
-  const float scale = a / (L * a + exp2f(s2 - Mf));
-  pb.out[head * kDim + 8 * (t >> 1) + 2 * c + (t & 1)] = sum * scale;
-}
-
 __device__ void run_consumer(const DecodeParams& P, const Smem& S, int warp, int lane) {
   const int g = lane >> 2, c = lane & 3;
   const int kvh = warp % kKvHeads;      // the KV head this warp serves
@@ -746,100 +709,119 @@ __device__ bool grid_barrier(unsigned int* bar, const Smem& S) {
   return S.flags[2] != 0;
 }
 
-// Merge of the deferred problems by the whole grid after the grid barrier.
-//   * Most problems: one warp per (problem, KV head g, chunk q) unit.  Lane
-//     (h, c) of the warp owns values 4q..4q+3 of head 8g + h, quarter c (the
-//     layout the consumer warps wrote), so one warp load reads 512
-//     consecutive bytes of a partial; each lane folds every partial of the
-//     problem, kMergeBatch loads in flight at a time, in item order.
-//   * A problem with many partials (a lone long problem split over every
-//     CTA) takes a whole CTA per (head, quarter c) unit instead, one thread
-//     per partial, then a block reduction; value k of a quarter is dim
-//     8(k/2) + 2c + (k & 1) of the head.
-constexpr int kMergeBatch = 16;
+// Merge of the deferred problems by the whole grid after the grid barrier, in
+// units of (problem, KV head g, chunk q).  Lane (h, c) of a warp owns values
+// 4q..4q+3 of head 8g + h, quarter c: dims 16q + 2c + {0, 1} and
+// 16q + 8 + 2c + {0, 1} of the head (the layout the consumer warps wrote), so
+// one warp load reads 512 consecutive bytes of a partial.  A lane folds its
+// partials kMergeBatch loads at a time, in item order.
+//   * Most problems take one warp per unit, every lane folding all partials.
+//   * A problem with many partials (a lone long problem split over every CTA)
+//     takes a whole CTA per unit: warp w folds partials w, w + 9, ..., then
+//     the warps' states are combined through shared memory in warp order.
+constexpr int kMergeBatch = 24;
+
+// Folds partials s0 + first, s0 + first + stride, ... (< s1) into (m, l, acc).
+__device__ __forceinline__ void fold_chunk(const DecodeParams& P, int s0, int s1, int first, int stride,
+                                           int head, int c, int q, float& m, float& l, float4& acc) {
+  for (int i0 = s0 + first; i0 < s1; i0 += kMergeBatch * stride) {
+    float mi[kMergeBatch], li[kMergeBatch];
+    float4 vi[kMergeBatch];
+#pragma unroll
+    for (int j = 0; j < kMergeBatch; ++j) {
+      const int ij = i0 + j * stride;
+      const int i = ij < s1 ? ij : i0;
+      const float* pi = P.partials + static_cast<size_t>(i) * kPartialFloats;
+      mi[j] = ij < s1 ? __ldcg(pi + kHeads * kDim + head) : -INFINITY;
+      li[j] = __ldcg(pi + kHeads * kDim + kHeads + head);
+      vi[j] = __ldcg(reinterpret_cast<const float4*>(pi) + partial_f4(head, c, q));
+    }
+    float mn = m;
+#pragma unroll
+    for (int j = 0; j < kMergeBatch; ++j) mn = fmaxf(mn, mi[j]);
+    const float sa = (m == -INFINITY) ? 0.f : exp2f(m - mn);
+    l *= sa;
+    acc = make_float4(acc.x * sa, acc.y * sa, acc.z * sa, acc.w * sa);
+    m = mn;
+#pragma unroll
+    for (int j = 0; j < kMergeBatch; ++j) {
+      const float sb = (mi[j] == -INFINITY) ? 0.f : exp2f(mi[j] - m);
+      l += sb * li[j];
+      acc.x += sb * vi[j].x;
+      acc.y += sb * vi[j].y;
+      acc.z += sb * vi[j].z;
+      acc.w += sb * vi[j].w;
+    }
+  }
+}
+
+// Writes values 4q..4q+3 of (head, c), with the sink folded in as finish_head does.
+__device__ __forceinline__ void write_chunk(const Problem& pb, int head, int c, int q, float m, float l,
+                                            float4 acc, float sink) {
+  const float s2 = sink * kLog2e;
+  const float Mf = fmaxf(m, s2);
+  const float a = (m == -INFINITY) ? 0.f : exp2f(m - Mf);
+  const float scale = a / (l * a + exp2f(s2 - Mf));
+  float* o = pb.out + head * kDim + 16 * q + 2 * c;
+  *reinterpret_cast<float2*>(o) = make_float2(acc.x * scale, acc.y * scale);
+  *reinterpret_cast<float2*>(o + 8) = make_float2(acc.z * scale, acc.w * scale);
+}
 
 __device__ void grid_merge(const DecodeParams& P, const Smem& S) {
   constexpr int kWarps = kThreads / 32;
+  constexpr int kUnits = kKvHeads * 8;  // units per problem
   const int t = threadIdx.x, lane = t & 31, warp = t >> 5;
+  const int c = lane & 3;
   {
-    const int units = (P.n_deferred - P.n_wide) * kKvHeads * 8;
+    const int units = (P.n_deferred - P.n_wide) * kUnits;
     for (int u = blockIdx.x * kWarps + warp; u < units; u += gridDim.x * kWarps) {
-      const int p = P.deferred[P.n_wide + u / (kKvHeads * 8)];
+      const int p = P.deferred[P.n_wide + u / kUnits];
       const int kvh = (u / 8) % kKvHeads, q = u % 8;
-      const int head = kvh * kGroup + (lane >> 2), c = lane & 3;
+      const int head = kvh * kGroup + (lane >> 2);
       const Problem& pb = P.prob[p];
       const float sink = pb.sinks[head];  // in flight with the partials
-      const int s0 = P.seg_item_begin[p], s1 = P.seg_item_begin[p + 1];
       float m = -INFINITY, l = 0.f;
       float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-      for (int i0 = s0; i0 < s1; i0 += kMergeBatch) {
-        float mi[kMergeBatch], li[kMergeBatch];
-        float4 vi[kMergeBatch];
-#pragma unroll
-        for (int j = 0; j < kMergeBatch; ++j) {
-          const int i = min(i0 + j, s1 - 1);
-          const float* pi = P.partials + static_cast<size_t>(i) * kPartialFloats;
-          mi[j] = i0 + j < s1 ? __ldcg(pi + kHeads * kDim + head) : -INFINITY;
-          li[j] = __ldcg(pi + kHeads * kDim + kHeads + head);
-          vi[j] = __ldcg(reinterpret_cast<const float4*>(pi) + partial_f4(head, c, q));
-        }
-        float mn = m;
-#pragma unroll
-        for (int j = 0; j < kMergeBatch; ++j) mn = fmaxf(mn, mi[j]);
-        const float sa = (m == -INFINITY) ? 0.f : exp2f(m - mn);
-        l *= sa;
-        acc = make_float4(acc.x * sa, acc.y * sa, acc.z * sa, acc.w * sa);
-        m = mn;
-#pragma unroll
-        for (int j = 0; j < kMergeBatch; ++j) {
-          const float sb = (mi[j] == -INFINITY) ? 0.f : exp2f(mi[j] - m);
-          l += sb * li[j];
-          acc.x += sb * vi[j].x;
-          acc.y += sb * vi[j].y;
-          acc.z += sb * vi[j].z;
-          acc.w += sb * vi[j].w;
-        }
-      }
-      // values 4q..4q+3 of thread (head, c) are dims 16q + 2c + {0, 1} and
-      // 16q + 8 + 2c + {0, 1}; fold in the sink as finish_head does
-      const float s2 = sink * kLog2e;
-      const float Mf = fmaxf(m, s2);
-      const float a = (m == -INFINITY) ? 0.f : exp2f(m - Mf);
-      const float scale = a / (l * a + exp2f(s2 - Mf));
-      float* o = pb.out + head * kDim + 16 * q + 2 * c;
-      *reinterpret_cast<float2*>(o) = make_float2(acc.x * scale, acc.y * scale);
-      *reinterpret_cast<float2*>(o + 8) = make_float2(acc.z * scale, acc.w * scale);
+      fold_chunk(P, P.seg_item_begin[p], P.seg_item_begin[p + 1], 0, 1, head, c, q, m, l, acc);
+      write_chunk(pb, head, c, q, m, l, acc, sink);
     }
   }
-  float* red = S.xch;  // [kWarps][34] scratch (the hand-over area is free now)
-  const int units = P.n_wide * kHeads * 4;
+  float* red = S.xch;  // [kWarps][32][6] (the hand-over area is free now)
+  const int units = P.n_wide * kUnits;
   for (int u = blockIdx.x; u < units; u += gridDim.x) {
-    const int p = P.deferred[u / (kHeads * 4)];
-    const int head = (u / 4) % kHeads, c = u % 4;
-    const float sink = P.prob[p].sinks[head];  // in flight with the partials
-    float m = -INFINITY, l = 0.f, v[32];
+    const int p = P.deferred[u / kUnits];
+    const int kvh = (u / 8) % kKvHeads, q = u % 8;
+    const int head = kvh * kGroup + (lane >> 2);
+    const Problem& pb = P.prob[p];
+    const float sink = pb.sinks[head];
+    float m = -INFINITY, l = 0.f;
+    float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+    fold_chunk(P, P.seg_item_begin[p], P.seg_item_begin[p + 1], warp, kWarps, head, c, q, m, l, acc);
+    float* mine = red + (warp * 32 + lane) * 6;
+    mine[0] = m;
+    mine[1] = l;
+    mine[2] = acc.x;
+    mine[3] = acc.y;
+    mine[4] = acc.z;
+    mine[5] = acc.w;
+    __syncthreads();
+    if (warp == 0) {
+      float M = -INFINITY;
 #pragma unroll
-    for (int e = 0; e < 32; ++e) v[e] = 0.f;
-    fold_partials(P, P.seg_item_begin[p], P.seg_item_begin[p + 1], t, kThreads, head, c, m, l, v);
-    float M = warp_max(m);
-    if (lane == 0) red[warp] = M;
-    __syncthreads();
-    M = red[0];
-#pragma unroll
-    for (int w = 1; w < kWarps; ++w) M = fmaxf(M, red[w]);
-    __syncthreads();
-    warp_sum_at(m, M, l, v, lane);
-    red[warp * 34 + lane] = v[0];
-    if (lane == 0) red[warp * 34 + 32] = l;
-    __syncthreads();
-    if (t < 32) {
-      float sum = 0.f, L = 0.f;
+      for (int w = 0; w < kWarps; ++w) M = fmaxf(M, red[(w * 32 + lane) * 6]);
+      float L = 0.f;
+      float4 A = make_float4(0.f, 0.f, 0.f, 0.f);
 #pragma unroll
       for (int w = 0; w < kWarps; ++w) {
-        sum += red[w * 34 + t];
-        L += red[w * 34 + 32];
+        const float* o = red + (w * 32 + lane) * 6;
+        const float sc = (o[0] == -INFINITY) ? 0.f : exp2f(o[0] - M);
+        L += sc * o[1];
+        A.x += sc * o[2];
+        A.y += sc * o[3];
+        A.z += sc * o[4];
+        A.w += sc * o[5];
       }
-      write_merged(P.prob[p], head, c, t, M, L, sum, sink);
+      write_chunk(pb, head, c, q, M, L, A, sink);
     }
     __syncthreads();  // red is reused by the next unit
   }
