@@ -40,6 +40,23 @@ NOMINAL_HBM_GBS = 8000.0
 TRAFFIC = {("stack", 100_000): (2_905_856_000 + 6_322_176, "58f64013b925776a")}
 
 
+def max_over_ranks(x: float, world: int, device) -> float:
+    """The largest x over all ranks: a step of the job lasts as long as its
+    slowest rank's step."""
+    if world == 1:
+        return x
+    import torch
+    t = torch.tensor([x], dtype=torch.float64, device=device)
+    torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+    return float(t.item())
+
+
+def per_token_us(ms_max: float, world: int) -> float:
+    """Whole-job time per token: every rank decodes its own token in a step,
+    so one step of the job (as long as its slowest rank) yields `world`."""
+    return ms_max * 1000.0 / world
+
+
 def kernel_sources_hash() -> str:
     import hashlib
     d = os.path.join(ROOT, "long_context_decode_flash_b200", "csrc")
@@ -419,24 +436,17 @@ def main():
             host_out.copy_(out, non_blocking=True)
             e_e[i].record(stream)
         torch.cuda.synchronize()
-        e2e_ms = statistics.mean(s.elapsed_time(e) for s, e in zip(e_s, e_e))
-        if world > 1:
-            t = torch.tensor([e2e_ms], device="cuda")
-            torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
-            e2e_ms = float(t.item())
-        e2e = {"value": e2e_ms * 1000.0 / world, "unit": "us/token" if layers is not None else "us/step",
+        e2e_ms = max_over_ranks(statistics.mean(s.elapsed_time(e) for s, e in zip(e_s, e_e)), world, "cuda")
+        e2e = {"value": per_token_us(e2e_ms, world), "unit": "us/token" if layers is not None else "us/step",
                "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h)}
 
-    if world > 1:
-        t = torch.tensor([ms], device="cuda")
-        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
-        ms = float(t.item())
+    ms = max_over_ranks(ms, world, "cuda")
 
     peak, peak_kind = measured_peak()
     achieved = algo_bytes / (ms * 1e-3) / 1e9
     line = {
         "metric": METRIC if args.workload == "stack" else f"{args.workload} decode-attention us/step",
-        "value": ms * 1000.0 / world,
+        "value": per_token_us(ms, world),
         "unit": "us/token" if args.workload == "stack" else "us/step",
         "n_gpus": world, "steps": args.steps, "warmup": max(args.warmup, 3),
         "ms_per_step": ms, "higher_is_better": False, "scaling": "weak", "vs_baseline": None,
