@@ -3,7 +3,7 @@
 with its own bf16 KV cache), on B200s.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl flint|reference]
-                    [--workload stack|full100k|swa100k|paged32]
+                    [--workload stack|full100k|full2k|swa100k|paged32|paged32swa]
 
 Prints one JSON line (rank 0).  A step is one call of flint_attn_stack: for
 every layer the fused Q/K RMSNorm (+RoPE), KV append at position 99,999 and
@@ -79,9 +79,10 @@ def parse():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=200)
-    ap.add_argument("--warmup", type=int, default=10)
+    ap.add_argument("--warmup", type=int, default=20)
     ap.add_argument("--impl", default="flint", choices=["flint", "reference"])
-    ap.add_argument("--workload", default="stack", choices=["stack", "full100k", "swa100k", "paged32"])
+    ap.add_argument("--workload", default="stack",
+                    choices=["stack", "full100k", "full2k", "swa100k", "paged32", "paged32swa"])
     ap.add_argument("--context", type=int, default=100_000,
                     help="context length (the benchmark's figure is 100,000; smaller ones serve profiling)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
@@ -135,6 +136,17 @@ def oracle_sample(layers_full, layers_window, nthreads, budget_s=10.0):
     return us, sum(tf) + sum(tw), desc
 
 
+def cpu_model() -> str:
+    try:
+        with open("/proc/cpuinfo") as f:
+            for line in f:
+                if line.startswith("model name"):
+                    return line.split(":", 1)[1].strip()
+    except OSError:
+        pass
+    return "unknown"
+
+
 def run_reference(args, rank):
     """The float64 oracle on the host cores, same metric and unit."""
     if rank != 0:
@@ -178,14 +190,15 @@ def workload_config(name):
         return dict(base, workload="49-layer decode-attention stack for one token: 35 sliding-window "
                     "(513, RoPE) + 14 full-context NoPE layers, GQA 32q/4kv x 128, sinks",
                     context=CONTEXT, layers=49, kv_layout="ring(513) + contiguous")
-    if name == "full100k":
-        return dict(base, workload="one full-context NoPE decode layer", context=CONTEXT, layers=1,
-                    kv_layout="contiguous")
+    if name in ("full100k", "full2k"):
+        return dict(base, workload="one full-context NoPE decode layer, q given (flint_attn_decode)",
+                    layers=1, kv_layout="contiguous")
     if name == "swa100k":
         return dict(base, workload="one sliding-window RoPE layer with norm+RoPE+append",
                     context=CONTEXT, layers=1, kv_layout="ring(513)")
+    kind = "sliding-window (513)" if name == "paged32swa" else "full-context"
     return dict(base, workload="32 paged requests, log-uniform lengths in [4096, 131072], "
-                "full-context layer", batch=32, kv_layout="paged(64)")
+                f"{kind} layer", batch=32, kv_layout="paged(64)")
 
 
 class ClockSampler:
@@ -297,16 +310,25 @@ def main():
     if args.workload == "stack":
         layers = I.make_stack(ctx)
         algo_bytes = flint.flint_kv_bytes(ctx)
-    elif args.workload == "full100k":
-        layers = [I.make_layer(I.W_FULL_100K, 0, ctx, 0, False, ring=False)]
-        algo_bytes = ctx * 2048
     elif args.workload == "swa100k":
         layers = [I.make_layer(I.W_SWA_100K, 0, ctx, 513, True, ring=True)]
         algo_bytes = min(ctx, 513) * 2048
+    elif args.workload in ("full100k", "full2k"):
+        # one full layer, q already normed: flint_attn_decode on a contiguous cache
+        layers = None
+        if args.workload == "full2k":
+            ctx = 2048
+        d = I.make_decode(ctx, workload=I.W_FULL_100K if args.workload == "full100k" else I.W_FULL_SMALL)
+        dec = dict(q=d.q, k=d.k_cache, v=d.v_cache, seq_lens=d.seq_lens, sinks=d.sinks, window=0,
+                   layout=flint.CONTIGUOUS, capacity=ctx, table=None)
+        algo_bytes = ctx * 2048
     else:
         layers = None
         pb = I.make_paged_batch()
-        algo_bytes = sum(pb.seq_lens) * 2048
+        window = 513 if args.workload == "paged32swa" else 0
+        dec = dict(q=pb.q, k=pb.k_pool, v=pb.v_pool, seq_lens=pb.seq_lens, sinks=pb.sinks,
+                   window=window, layout=flint.PAGED, capacity=0, table=pb.block_table)
+        algo_bytes = sum(min(L, window) if window else L for L in pb.seq_lens) * 2048
 
     cpu_baseline = None
     if rank == 0 and world == 1 and args.workload == "stack" and ctx == CONTEXT and not args.no_cpu_baseline:
@@ -317,8 +339,10 @@ def main():
         win = [layers[0], layers[1]]
         nthreads = os.cpu_count() or 1
         us, spent, desc = oracle_sample(full, win, nthreads, budget_s=10.0)
+        us1, spent1, _ = oracle_sample(full, win, 1, budget_s=5.0)
         cpu_baseline = {"value": us, "unit": "us/token", "cores": nthreads, "kind": "oracle",
-                        "sample": desc + f" ({spent:.1f} s of CPU wall time)"}
+                        "sample": desc + f" ({spent:.1f} s of CPU wall time)",
+                        "value_1_thread": us1, "cpu_model": cpu_model()}
 
     if world > 1:
         torch.distributed.init_process_group("nccl", timeout=__import__("datetime").timedelta(seconds=120))
@@ -350,16 +374,18 @@ def main():
             flint.flint_attn_stack(arr, pos, out, ws, dev_err=err)
         h2d = host_in.numel() * host_in.element_size()
     else:
-        q, k, v = pb.q.cuda(), pb.k_pool.cuda(), pb.v_pool.cuda()
-        table, sinks = pb.block_table.cuda(), pb.sinks.cuda()
-        cache = flint.kv_cache(k, v, flint.PAGED, block_table=table, num_blocks=pb.k_pool.shape[0])
-        out = torch.empty((len(pb.seq_lens), 32, 128), dtype=torch.float32, device="cuda")
-        ws = flint.workspace(len(pb.seq_lens))
-        host_in = pb.q.pin_memory()
+        q, k, v, sinks = dec["q"].cuda(), dec["k"].cuda(), dec["v"].cuda(), dec["sinks"].cuda()
+        table = dec["table"].cuda() if dec["table"] is not None else None
+        seq_lens, window = dec["seq_lens"], dec["window"]
+        cache = flint.kv_cache(k, v, dec["layout"], capacity=dec["capacity"], block_table=table,
+                               num_blocks=k.shape[0] if table is not None else 0)
+        out = torch.empty((len(seq_lens), 32, 128), dtype=torch.float32, device="cuda")
+        ws = flint.workspace(len(seq_lens))
+        host_in = dec["q"].pin_memory()
         packed = q
 
         def step():
-            flint.flint_attn_decode(q, cache, pb.seq_lens, sinks, 0, out, ws, dev_err=err)
+            flint.flint_attn_decode(q, cache, seq_lens, sinks, window, out, ws, dev_err=err)
         h2d = host_in.numel() * host_in.element_size()
     host_out = torch.empty(out.shape, dtype=torch.float32).pin_memory()
     d2h = host_out.numel() * 4
@@ -451,7 +477,9 @@ def main():
         "n_gpus": world, "steps": args.steps, "warmup": max(args.warmup, 3),
         "ms_per_step": ms, "higher_is_better": False, "scaling": "weak", "vs_baseline": None,
         "dtype": "bf16", "data": "synthetic (seeded bf16 N(0,1) q/k/v/KV, N(0,1) sinks, 1+N(0,0.1) norm weights)",
-        "config": dict(workload_config(args.workload), context=ctx, parallelism=f"replicas x{world}",
+        "config": dict(workload_config(args.workload),
+                       context=ctx if not args.workload.startswith("paged") else "per request",
+                       parallelism=f"replicas x{world}",
                        launch=launch),
         "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
                      "frac": achieved / peak, "peak_kind": peak_kind,
