@@ -6,7 +6,8 @@ its Python binding) never imports it and shares no code with it.
 
 ``flint_oracle.c`` holds the arithmetic; this module builds it with gcc and
 marshals numpy arrays through ctypes.  bf16 values travel as uint16 bit
-patterns.  Every function is pinned by tests in ``tests/test_oracle_pins.py``.
+patterns, e4m3 (fp8) cache values as uint8 codes.  Every function is pinned by
+tests in ``tests/test_oracle_pins.py``.
 """
 from __future__ import annotations
 
@@ -58,6 +59,19 @@ def _load():
             lib.fo_decode_layer.argtypes = [P, P, P, P, P, P, I, I, I, P, P, I, I, P,
                                             I, L, I, I, D, D, P, I]
             lib.fo_decode_layer.restype = I
+            U8, F = ctypes.c_uint8, ctypes.c_float
+            lib.fo_e4m3_to_f64.argtypes = [U8]
+            lib.fo_e4m3_to_f64.restype = D
+            lib.fo_f64_to_e4m3.argtypes = [D]
+            lib.fo_f64_to_e4m3.restype = U8
+            lib.fo_quantize_e4m3.argtypes = [D, F]
+            lib.fo_quantize_e4m3.restype = U8
+            lib.fo_kv_append_fp8.argtypes = [P, P, I, I, P, I, I, I, L, P, P, P, P]
+            lib.fo_attn_decode_fp8.argtypes = [P, I, I, I, P, P, P, P, I, I, P, I, L, I, P, P, I]
+            lib.fo_attn_decode_fp8.restype = I
+            lib.fo_decode_layer_fp8.argtypes = [P, P, P, P, P, P, I, I, I, P, P, P, P, I, I, P,
+                                                I, L, I, I, D, D, P, I]
+            lib.fo_decode_layer_fp8.restype = I
             lib.fo_kv_bytes.argtypes = [L, I, I, I, I, I, I]
             lib.fo_kv_bytes.restype = D
             lib.fo_num_threads.restype = I
@@ -204,3 +218,100 @@ def decode_layer(q_raw, k_raw, v_raw, w_q, w_k, sinks, k_cache, v_cache, L: int,
 def kv_bytes(ctx: int, n_full: int = 14, n_window: int = 35, window: int = 513,
              nkv: int = 4, d: int = 128, elem_bytes: int = 2) -> float:
     return _load().fo_kv_bytes(int(ctx), n_full, n_window, window, nkv, d, elem_bytes)
+
+
+# ---- FP8 (e4m3) KV cache --------------------------------------------------
+
+def e4m3_to_f64(codes) -> np.ndarray:
+    """Values of e4m3 codes (uint8 array), float64; NaN for S.1111.111."""
+    c = np.asarray(codes, np.uint8)
+    lib = _load()
+    return np.array([lib.fo_e4m3_to_f64(int(x)) for x in c.ravel()], np.float64).reshape(c.shape)
+
+
+def f64_to_e4m3(x) -> np.ndarray:
+    """Nearest e4m3 codes (ties to even, saturating at 448) of float64 values."""
+    x = np.asarray(x, np.float64)
+    lib = _load()
+    return np.array([lib.fo_f64_to_e4m3(float(v)) for v in x.ravel()], np.uint8).reshape(x.shape)
+
+
+def quantize_e4m3(x, scale: float) -> np.ndarray:
+    """Cache codes of x with one scale: float32(x) / float32(scale) in float32,
+    then the nearest e4m3 code."""
+    x = np.asarray(x, np.float64)
+    lib = _load()
+    return np.array([lib.fo_quantize_e4m3(float(v), float(scale)) for v in x.ravel()],
+                    np.uint8).reshape(x.shape)
+
+
+def _u8c(c):
+    if c.dtype != np.uint8 or not c.flags["C_CONTIGUOUS"]:
+        raise TypeError("fp8 caches must be C-contiguous uint8 arrays")
+    return c
+
+
+def _scales(s, nkv):
+    s = np.ascontiguousarray(np.asarray(s, np.float32).reshape(-1))
+    if s.shape[0] != nkv:
+        raise ValueError("one scale per KV head")
+    return s
+
+
+def kv_append_fp8(k_cache, v_cache, layout: int, pos: int, k, v, k_scale, v_scale,
+                  capacity: int = 0, block_table=None, block_size: int = 64):
+    """In place: quantizes k ([nkv, d] float64) and v ([nkv, d] bf16 bits) into
+    uint8 e4m3 caches at pos."""
+    _u8c(k_cache), _u8c(v_cache)
+    k, v = _f64(k), _u16(v)
+    nkv, d = k.shape
+    ks, vs = _scales(k_scale, nkv), _scales(v_scale, nkv)
+    bt = None if block_table is None else np.ascontiguousarray(block_table, np.int32)
+    _load().fo_kv_append_fp8(_ptr(k_cache), _ptr(v_cache), layout, int(capacity), _ptr(bt),
+                             int(block_size), nkv, d, int(pos), _ptr(k), _ptr(v), _ptr(ks),
+                             _ptr(vs))
+
+
+def attn_decode_fp8(q, k_cache, v_cache, k_scale, v_scale, L: int, sinks, window: int = 0,
+                    layout: int = CONTIGUOUS, capacity: int = 0, block_table=None,
+                    block_size: int = 64, nthreads: int = 0) -> np.ndarray:
+    """attn_decode over uint8 e4m3 caches with per-KV-head scales."""
+    q = bf16_to_f64(q) if np.asarray(q).dtype == np.uint16 else _f64(q)
+    nq, d = q.shape
+    _u8c(k_cache), _u8c(v_cache)
+    nkv = k_cache.shape[-2]
+    ks, vs = _scales(k_scale, nkv), _scales(v_scale, nkv)
+    sinks = _f64(sinks)
+    bt = None if block_table is None else np.ascontiguousarray(block_table, np.int32)
+    out = np.empty((nq, d), np.float64)
+    rc = _load().fo_attn_decode_fp8(_ptr(q), nq, nkv, d, _ptr(k_cache), _ptr(v_cache), _ptr(ks),
+                                    _ptr(vs), layout, int(capacity), _ptr(bt), int(block_size),
+                                    int(L), int(window), _ptr(sinks), _ptr(out), int(nthreads))
+    if rc != 0:
+        raise ValueError("oracle rejected the arguments")
+    return out
+
+
+def decode_layer_fp8(q_raw, k_raw, v_raw, w_q, w_k, sinks, k_cache, v_cache, k_scale, v_scale,
+                     L: int, window: int, apply_rope: bool, layout: int = CONTIGUOUS,
+                     capacity: int = 0, block_table=None, block_size: int = 64,
+                     eps: float = 1e-6, theta: float = 10000.0, nthreads: int = 0):
+    """norm (+RoPE) -> quantized append at L-1 -> attend over e4m3 caches."""
+    q_raw, k_raw, v_raw = _u16(q_raw), _u16(k_raw), _u16(v_raw)
+    w_q = None if w_q is None else _u16(w_q)
+    w_k = None if w_k is None else _u16(w_k)
+    _u8c(k_cache), _u8c(v_cache)
+    nq, d = q_raw.shape
+    nkv = k_raw.shape[0]
+    ks, vs = _scales(k_scale, nkv), _scales(v_scale, nkv)
+    sinks = _f64(sinks)
+    bt = None if block_table is None else np.ascontiguousarray(block_table, np.int32)
+    out = np.empty((nq, d), np.float64)
+    rc = _load().fo_decode_layer_fp8(_ptr(q_raw), _ptr(k_raw), _ptr(v_raw), _ptr(w_q), _ptr(w_k),
+                                     _ptr(sinks), nq, nkv, d, _ptr(k_cache), _ptr(v_cache),
+                                     _ptr(ks), _ptr(vs), layout, int(capacity), _ptr(bt),
+                                     int(block_size), int(L), int(window), int(bool(apply_rope)),
+                                     float(eps), float(theta), _ptr(out), int(nthreads))
+    if rc != 0:
+        raise ValueError("oracle rejected the arguments")
+    return out

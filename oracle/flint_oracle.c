@@ -15,6 +15,8 @@
  *     `architecture` ("GQA 4 KV x 128") and `kvCacheGiBPerRequest`.
  *   - "Day-0 Support for Flint on vLLM" (newruntime.com), "What happened":
  *     BF16 KV cache, fused normalization / rotary-position / cache operations.
+ *   - "Recursive Flint" model JSON, the "fp8" column of kvCacheGiBPerRequest:
+ *     a one-byte cache variant (format reading in the FP8 section below).
  * The pages print no formula.  The numeric definitions this library adopts
  * are: softmax over [q.k_j / sqrt(d) for j in window, sink_h], where the sink
  * logit carries no value; window at position t = max(0, t-512) .. t; RMSNorm
@@ -262,6 +264,147 @@ int fo_decode_layer(const uint16_t* q_raw, const uint16_t* k_raw,
                             block_table, block_size, L, window, sinks, out,
                             nthreads);
     free(q); free(k); free(kb);
+    return rc;
+}
+
+/* ---- FP8 (e4m3) KV cache ------------------------------------------------ */
+
+/* The "fp8" column of kvCacheGiBPerRequest ("Recursive Flint" model JSON)
+ * stores one byte per cached value, half of bf16; the pages give no format.
+ * Reading adopted: OCP 8-bit floating point E4M3 -- 1 sign bit, 4 exponent
+ * bits with bias 7, 3 mantissa bits; exponent field 0 holds subnormals
+ * m * 2^-9; the code S.1111.111 is NaN; no infinities; largest magnitude
+ * 448 (S.1111.110).  Each (layer, KV head) has one float32 scale for K and
+ * one for V: the cache holds e4m3(x / scale), read back as value * scale.
+ * The division and the rounding decision are taken in float32 (the
+ * precision the GPU takes them in): code = rne_satfinite(float(x) / scale). */
+
+double fo_e4m3_to_f64(uint8_t c)
+{
+    int sgn = c >> 7, e = (c >> 3) & 15, m = c & 7;
+    if (e == 15 && m == 7) return NAN;
+    double mag = e == 0 ? ldexp((double)m, -9) : ldexp((double)(8 + m), e - 10);
+    return sgn ? -mag : mag;
+}
+
+/* Nearest e4m3 code to x, ties to even; magnitudes at or above 448 (and
+ * infinities) saturate to +-448; NaN gives 0x7f. */
+uint8_t fo_f64_to_e4m3(double x)
+{
+    if (isnan(x)) return 0x7f;
+    uint8_t sgn = signbit(x) ? 0x80 : 0x00;
+    double a = fabs(x);
+    if (a >= 448.0) return sgn | 0x7e;
+    /* quantum: 2^(e-3) for a in [2^e, 2^(e+1)), e >= -6; 2^-9 below 2^-6 */
+    int e2;
+    frexp(a, &e2);               /* a = f * 2^e2, f in [0.5, 1) */
+    int e = e2 - 1;
+    if (e < -6) e = -6;
+    double q = ldexp(1.0, e - 3);
+    double r = nearbyint(a / q) * q;   /* round half to even (default mode) */
+    if (r == 0.0) return sgn;
+    frexp(r, &e2);
+    e = e2 - 1;                  /* r may have moved up one binade */
+    if (e < -6) return sgn | (uint8_t)(r / ldexp(1.0, -9));       /* subnormal */
+    int mant = (int)(r / ldexp(1.0, e - 3)) - 8;                  /* 0..7 */
+    return sgn | (uint8_t)(((e + 7) << 3) | mant);
+}
+
+/* The cache code of x with the given scale: float32 division, then e4m3. */
+uint8_t fo_quantize_e4m3(double x, float scale)
+{
+    float t = (float)x / scale;
+    return fo_f64_to_e4m3((double)t);
+}
+
+/* Write k ([nkv][d] float64, the normed/roped values) and v ([nkv][d] bf16
+ * bits) at position pos of byte caches laid out like the bf16 ones. */
+void fo_kv_append_fp8(uint8_t* k_cache, uint8_t* v_cache, int layout,
+                      int capacity, const int32_t* block_table, int block_size,
+                      int nkv, int d, long pos, const double* k,
+                      const uint16_t* v, const float* k_scale,
+                      const float* v_scale)
+{
+    long row = fo_storage_row(layout, pos, capacity, block_table, block_size);
+    for (int g = 0; g < nkv; ++g)
+        for (int i = 0; i < d; ++i) {
+            k_cache[(row * nkv + g) * d + i] = fo_quantize_e4m3(k[g * d + i], k_scale[g]);
+            v_cache[(row * nkv + g) * d + i] =
+                fo_quantize_e4m3(fo_bf16_to_f64(v[g * d + i]), v_scale[g]);
+        }
+}
+
+/* fo_attn_decode over e4m3 caches: K[j] = decode(code) * k_scale[g],
+ * V[j] = decode(code) * v_scale[g], everything else as there. */
+int fo_attn_decode_fp8(const double* q, int nq, int nkv, int d,
+                       const uint8_t* k_cache, const uint8_t* v_cache,
+                       const float* k_scale, const float* v_scale,
+                       int layout, int capacity, const int32_t* block_table,
+                       int block_size, long L, int window, const double* sinks,
+                       double* out, int nthreads)
+{
+    if (L < 1 || nq <= 0 || nkv <= 0 || nq % nkv != 0 || d <= 0) return -1;
+    long t = L - 1;
+    long lo = (window > 0 && t - (window - 1) > 0) ? t - (window - 1) : 0;
+    long n = t - lo + 1;
+    int group = nq / nkv;
+    double scale = 1.0 / sqrt((double)d);
+#ifdef _OPENMP
+    if (nthreads > 0) omp_set_num_threads(nthreads);
+#else
+    (void)nthreads;
+#endif
+#pragma omp parallel for schedule(static)
+    for (int h = 0; h < nq; ++h) {
+        int g = h / group;
+        const double* qh = q + (long)h * d;
+        double* s = (double*)malloc(sizeof(double) * (size_t)n);
+        double mx = sinks[h];
+        for (long j = 0; j < n; ++j) {
+            long row = fo_storage_row(layout, lo + j, capacity, block_table, block_size);
+            const uint8_t* kr = k_cache + (row * nkv + g) * d;
+            double dot = 0.0;
+            for (int i = 0; i < d; ++i) dot += qh[i] * (fo_e4m3_to_f64(kr[i]) * (double)k_scale[g]);
+            s[j] = dot * scale;
+            if (s[j] > mx) mx = s[j];
+        }
+        double den = exp(sinks[h] - mx);
+        double* o = out + (long)h * d;
+        for (int i = 0; i < d; ++i) o[i] = 0.0;
+        for (long j = 0; j < n; ++j) {
+            long row = fo_storage_row(layout, lo + j, capacity, block_table, block_size);
+            const uint8_t* vr = v_cache + (row * nkv + g) * d;
+            double p = exp(s[j] - mx);
+            den += p;
+            for (int i = 0; i < d; ++i) o[i] += p * (fo_e4m3_to_f64(vr[i]) * (double)v_scale[g]);
+        }
+        for (int i = 0; i < d; ++i) o[i] /= den;
+        free(s);
+    }
+    return 0;
+}
+
+/* fo_decode_layer with e4m3 caches: norm (+RoPE) -> quantized append -> attend. */
+int fo_decode_layer_fp8(const uint16_t* q_raw, const uint16_t* k_raw,
+                        const uint16_t* v_raw, const uint16_t* w_q,
+                        const uint16_t* w_k, const double* sinks, int nq,
+                        int nkv, int d, uint8_t* k_cache, uint8_t* v_cache,
+                        const float* k_scale, const float* v_scale, int layout,
+                        int capacity, const int32_t* block_table,
+                        int block_size, long L, int window, int apply_rope,
+                        double eps, double theta, double* out, int nthreads)
+{
+    if (L < 1) return -1;
+    double* q = (double*)malloc(sizeof(double) * (size_t)nq * d);
+    double* k = (double*)malloc(sizeof(double) * (size_t)nkv * d);
+    fo_qk_norm_rope(q_raw, k_raw, w_q, w_k, nq, nkv, d, L - 1, eps, theta,
+                    apply_rope, q, k, NULL);
+    fo_kv_append_fp8(k_cache, v_cache, layout, capacity, block_table,
+                     block_size, nkv, d, L - 1, k, v_raw, k_scale, v_scale);
+    int rc = fo_attn_decode_fp8(q, nq, nkv, d, k_cache, v_cache, k_scale,
+                                v_scale, layout, capacity, block_table,
+                                block_size, L, window, sinks, out, nthreads);
+    free(q); free(k);
     return rc;
 }
 

@@ -350,3 +350,144 @@ def test_kv_bytes_reproduce_the_model_json_table():
         assert round(oracle.kv_bytes(ctx, elem_bytes=1) / 2 ** 30, 3) == gib_fp8
     # "28 KiB per token" over the full layers (Model architecture)
     assert oracle.kv_bytes(1000, n_window=0) - oracle.kv_bytes(999, n_window=0) == 28 * 1024
+
+
+# ------------------------------------------------------ fp8 (e4m3) cache ----
+# The "fp8" column of the model JSON's kvCacheGiBPerRequest (one byte per
+# value, pinned above) is read as OCP E4M3 with a float32 scale per
+# (layer, KV head).  torch's float8_e4m3fn is an independent implementation
+# of the same format.
+
+def _torch_e4m3_values():
+    codes = torch.arange(256, dtype=torch.int32).to(torch.uint8)
+    return codes.view(torch.float8_e4m3fn).to(torch.float64).numpy()
+
+
+def test_e4m3_decode_matches_torch_for_all_codes():
+    got = oracle.e4m3_to_f64(np.arange(256, dtype=np.uint8))
+    want = _torch_e4m3_values()
+    nan = np.isnan(want)
+    assert np.array_equal(np.isnan(got), nan) and nan.sum() == 2       # 0x7f, 0xff
+    assert np.array_equal(got[~nan], want[~nan])
+    assert got[0x7E] == 448.0 and got[0x01] == 2.0 ** -9 and got[0x38] == 1.0
+
+
+def test_e4m3_encode_matches_torch_in_range():
+    r = np.random.default_rng(11)
+    x = np.concatenate([
+        r.normal(0, 30, 20000),                       # normals of both signs
+        r.uniform(-2 ** -6, 2 ** -6, 5000),           # subnormal range
+        _torch_e4m3_values()[:126] * 1.0,             # every finite code exactly
+        # midpoints between neighbouring codes: ties go to the even code
+        (_torch_e4m3_values()[1:126] + _torch_e4m3_values()[:125]) / 2,
+        np.array([463.9, -463.9, 0.0, -0.0]),
+    ])
+    x = x[np.abs(x) < 464]
+    want = torch.from_numpy(x).to(torch.float8_e4m3fn).view(torch.uint8).numpy()
+    got = oracle.f64_to_e4m3(x)
+    assert np.array_equal(got, want)
+
+
+def test_e4m3_saturates_and_round_trips():
+    big = np.array([464.0, 1e6, np.inf, -500.0, -np.inf])
+    assert list(oracle.f64_to_e4m3(big)) == [0x7E, 0x7E, 0x7E, 0xFE, 0xFE]
+    assert oracle.f64_to_e4m3(np.array([np.nan]))[0] == 0x7F
+    codes = np.array([c for c in range(256) if c not in (0x7F, 0xFF)], np.uint8)
+    assert np.array_equal(oracle.f64_to_e4m3(oracle.e4m3_to_f64(codes)), codes)
+
+
+def test_quantize_divides_in_float32_then_rounds():
+    r = np.random.default_rng(12)
+    x = r.normal(0, 3, 4000)
+    for scale in (0.0123, 1.0 / 112, 3.7):
+        t = torch.from_numpy(x).to(torch.float32) / torch.tensor(scale, dtype=torch.float32)
+        keep = t.abs() < 464
+        want = t[keep].to(torch.float8_e4m3fn).view(torch.uint8).numpy()
+        got = oracle.quantize_e4m3(x[keep.numpy()], scale)
+        assert np.array_equal(got, want)
+
+
+def _fp8_cache(L, nkv, d, seed):
+    r = np.random.default_rng(seed)
+    k = r.integers(0, 256, size=(L, nkv, d), dtype=np.uint8)
+    v = r.integers(0, 256, size=(L, nkv, d), dtype=np.uint8)
+    k[(k & 0x7F) == 0x7F] = 0x01     # no NaN codes
+    v[(v & 0x7F) == 0x7F] = 0x02
+    return k, v
+
+
+def test_fp8_attention_equals_bf16_attention_on_the_same_values():
+    # With power-of-two scales every dequantized value (4 significant bits)
+    # is exact in bf16, so the fp8 path must equal the pinned bf16 path.
+    L, nq, nkv, d = 300, 8, 2, 32
+    k8, v8 = _fp8_cache(L, nkv, d, 13)
+    ks, vs = np.array([2.0 ** -5, 2.0 ** -3], np.float32), np.array([2.0 ** -4, 0.5], np.float32)
+    kf = oracle.e4m3_to_f64(k8) * ks[None, :, None]
+    vf = oracle.e4m3_to_f64(v8) * vs[None, :, None]
+    kb, vb = oracle.f64_to_bf16(kf), oracle.f64_to_bf16(vf)
+    assert np.array_equal(oracle.bf16_to_f64(kb), kf) and np.array_equal(oracle.bf16_to_f64(vb), vf)
+    q = rng.normal(size=(nq, d))
+    sinks = rng.normal(size=nq)
+    for window in (0, 64):
+        want = oracle.attn_decode(q, kb, vb, L, sinks, window)
+        got = oracle.attn_decode_fp8(q, k8, v8, ks, vs, L, sinks, window)
+        np.testing.assert_allclose(got, want, rtol=1e-12, atol=1e-14)
+
+
+def test_fp8_attention_with_one_code_everywhere_is_closed_form():
+    L, nq, nkv, d = 50, 4, 1, 16
+    k8 = np.full((L, nkv, d), 0x30, np.uint8)     # 0.5
+    v8 = np.full((L, nkv, d), 0x4B, np.uint8)     # 3.5 * 2^... decoded below
+    vs = np.array([0.25], np.float32)
+    q = rng.normal(size=(nq, d))
+    sinks = np.array([0.3, -1.0, 2.0, -np.inf])
+    out = oracle.attn_decode_fp8(q, k8, v8, np.array([1.0], np.float32), vs, L, sinks)
+    val = oracle.e4m3_to_f64(np.array([0x4B], np.uint8))[0] * 0.25
+    s = q.sum(axis=1) * 0.5 / math.sqrt(d)          # every score of a head is equal
+    w = L * np.exp(s) / (L * np.exp(s) + np.exp(sinks))
+    np.testing.assert_allclose(out, (w * val)[:, None] * np.ones((1, d)), rtol=1e-12)
+
+
+@pytest.mark.parametrize("layout", [oracle.CONTIGUOUS, oracle.RING, oracle.PAGED])
+def test_fp8_append_places_torch_codes(layout):
+    nkv, d, bs = 4, 128, 64
+    cap = 513 if layout == oracle.RING else 256
+    table = np.array([3, 0, 2, 1], np.int32) if layout == oracle.PAGED else None
+    shape = (4 * bs, nkv, d) if layout == oracle.PAGED else (cap, nkv, d)
+    kc, vc = np.zeros(shape, np.uint8), np.zeros(shape, np.uint8)
+    k = rng.normal(0, 2, size=(nkv, d))
+    v = bf16_bits((nkv, d), 99)
+    ks = np.array([0.01, 0.02, 0.005, 1.0], np.float32)
+    vs = np.array([0.015, 0.25, 0.004, 2.0], np.float32)
+    pos = 700 if layout == oracle.RING else 130
+    oracle.kv_append_fp8(kc, vc, layout, pos, k, v, ks, vs, capacity=cap, block_table=table)
+    if layout == oracle.PAGED:
+        row = table[pos // bs] * bs + pos % bs
+    else:
+        row = pos % 513 if layout == oracle.RING else pos
+    tk = torch.from_numpy(k).to(torch.float32) / torch.from_numpy(ks)[:, None]
+    tv = torch.from_numpy(f64(v)).to(torch.float32) / torch.from_numpy(vs)[:, None]
+    sat = lambda t: t.clamp(-448, 448).to(torch.float8_e4m3fn).view(torch.uint8).numpy()
+    assert np.array_equal(kc[row], sat(tk)) and np.array_equal(vc[row], sat(tv))
+    others = np.ones(shape[0], bool)
+    others[row] = False
+    assert not kc[others].any() and not vc[others].any()
+
+
+def test_fp8_decode_layer_is_norm_rope_then_quantized_append_then_attention():
+    nq, nkv, d, L, cap = 32, 4, 128, 700, 513
+    q_raw, k_raw, v_raw = bf16_bits((nq, d), 201), bf16_bits((nkv, d), 202), bf16_bits((nkv, d), 203)
+    w_q, w_k = bf16_bits((d,), 204, 1.0, 0.1), bf16_bits((d,), 205, 1.0, 0.1)
+    sinks = rng.normal(size=nq)
+    ks = np.array([0.011, 0.009, 0.013, 0.01], np.float32)
+    vs = np.array([0.008, 0.012, 0.01, 0.009], np.float32)
+    k0, v0 = _fp8_cache(cap, nkv, d, 206)
+    kc, vc = k0.copy(), v0.copy()
+    got = oracle.decode_layer_fp8(q_raw, k_raw, v_raw, w_q, w_k, sinks, kc, vc, ks, vs, L, 513,
+                                  True, layout=oracle.RING, capacity=cap)
+    q, k, _ = oracle.qk_norm_rope(q_raw, k_raw, w_q, w_k, L - 1)
+    kw, vw = k0.copy(), v0.copy()
+    oracle.kv_append_fp8(kw, vw, oracle.RING, L - 1, k, v_raw, ks, vs, capacity=cap)
+    assert np.array_equal(kc, kw) and np.array_equal(vc, vw)
+    want = oracle.attn_decode_fp8(q, kw, vw, ks, vs, L, sinks, 513, layout=oracle.RING, capacity=cap)
+    np.testing.assert_array_equal(got, want)
