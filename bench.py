@@ -85,6 +85,8 @@ def parse():
                     choices=["stack", "full100k", "full2k", "swa100k", "paged32", "paged32swa"])
     ap.add_argument("--context", type=int, default=100_000,
                     help="context length (the benchmark's figure is 100,000; smaller ones serve profiling)")
+    ap.add_argument("--kv", default="bf16", choices=["bf16", "fp8"],
+                    help="KV-cache element: bf16, or E4M3 codes with per-head scales")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-graph", action="store_true", help="time direct launches instead of graph replays")
@@ -284,7 +286,8 @@ def build_stack_device(torch, flint, I, layers):
         d.w_q, d.w_k, d.sinks = lay.w_q.cuda(), lay.w_k.cuda(), lay.sinks.cuda()
         d.k_cache, d.v_cache = lay.k_cache.cuda(), lay.v_cache.cuda()
         d.window, d.rope = lay.window, lay.rope
-        d.cache = flint.kv_cache(d.k_cache, d.v_cache, lay.layout, capacity=lay.capacity)
+        d.cache = flint.kv_cache(d.k_cache, d.v_cache, lay.layout, capacity=lay.capacity,
+                                 k_scale=lay.k_scale, v_scale=lay.v_scale)
         dls.append(d)
     host_in = torch.cat([torch.cat([l.q_raw.reshape(-1), l.k_raw.reshape(-1), l.v_raw.reshape(-1)])
                          for l in layers]).reshape(n, per).pin_memory()
@@ -307,31 +310,37 @@ def main():
 
     # Host inputs first; the CPU baseline runs before any CUDA call.
     ctx = args.context
+    fp8 = args.kv == "fp8"
+    eb = 1 if fp8 else 2                       # bytes per cached value
+    tok_bytes = 2 * 4 * 128 * eb               # K and V of one token of one layer
     if args.workload == "stack":
-        layers = I.make_stack(ctx)
-        algo_bytes = flint.flint_kv_bytes(ctx)
+        layers = I.make_stack(ctx, fp8=fp8)
+        algo_bytes = flint.flint_kv_bytes(ctx, elem_bytes=eb)
     elif args.workload == "swa100k":
-        layers = [I.make_layer(I.W_SWA_100K, 0, ctx, 513, True, ring=True)]
-        algo_bytes = min(ctx, 513) * 2048
+        layers = [I.make_layer(I.W_SWA_100K, 0, ctx, 513, True, ring=True, fp8=fp8)]
+        algo_bytes = min(ctx, 513) * tok_bytes
     elif args.workload in ("full100k", "full2k"):
         # one full layer, q already normed: flint_attn_decode on a contiguous cache
         layers = None
         if args.workload == "full2k":
             ctx = 2048
-        d = I.make_decode(ctx, workload=I.W_FULL_100K if args.workload == "full100k" else I.W_FULL_SMALL)
+        d = I.make_decode(ctx, workload=I.W_FULL_100K if args.workload == "full100k" else I.W_FULL_SMALL,
+                          fp8=fp8)
         dec = dict(q=d.q, k=d.k_cache, v=d.v_cache, seq_lens=d.seq_lens, sinks=d.sinks, window=0,
-                   layout=flint.CONTIGUOUS, capacity=ctx, table=None)
-        algo_bytes = ctx * 2048
+                   layout=flint.CONTIGUOUS, capacity=ctx, table=None, ks=d.k_scale, vs=d.v_scale)
+        algo_bytes = ctx * tok_bytes
     else:
         layers = None
-        pb = I.make_paged_batch()
+        pb = I.make_paged_batch(fp8=fp8)
         window = 513 if args.workload == "paged32swa" else 0
         dec = dict(q=pb.q, k=pb.k_pool, v=pb.v_pool, seq_lens=pb.seq_lens, sinks=pb.sinks,
-                   window=window, layout=flint.PAGED, capacity=0, table=pb.block_table)
-        algo_bytes = sum(min(L, window) if window else L for L in pb.seq_lens) * 2048
+                   window=window, layout=flint.PAGED, capacity=0, table=pb.block_table,
+                   ks=pb.k_scale, vs=pb.v_scale)
+        algo_bytes = sum(min(L, window) if window else L for L in pb.seq_lens) * tok_bytes
 
     cpu_baseline = None
-    if rank == 0 and world == 1 and args.workload == "stack" and ctx == CONTEXT and not args.no_cpu_baseline:
+    if (rank == 0 and world == 1 and args.workload == "stack" and ctx == CONTEXT and not fp8
+            and not args.no_cpu_baseline):
         import oracle
         oracle.build()
         kinds = I.layer_kinds()
@@ -378,7 +387,8 @@ def main():
         table = dec["table"].cuda() if dec["table"] is not None else None
         seq_lens, window = dec["seq_lens"], dec["window"]
         cache = flint.kv_cache(k, v, dec["layout"], capacity=dec["capacity"], block_table=table,
-                               num_blocks=k.shape[0] if table is not None else 0)
+                               num_blocks=k.shape[0] if table is not None else 0,
+                               k_scale=dec["ks"], v_scale=dec["vs"])
         out = torch.empty((len(seq_lens), 32, 128), dtype=torch.float32, device="cuda")
         ws = flint.workspace(len(seq_lens))
         host_in = dec["q"].pin_memory()
@@ -476,16 +486,19 @@ def main():
         "unit": "us/token" if args.workload == "stack" else "us/step",
         "n_gpus": world, "steps": args.steps, "warmup": max(args.warmup, 3),
         "ms_per_step": ms, "higher_is_better": False, "scaling": "weak", "vs_baseline": None,
-        "dtype": "bf16", "data": "synthetic (seeded bf16 N(0,1) q/k/v/KV, N(0,1) sinks, 1+N(0,0.1) norm weights)",
+        "dtype": "fp8-e4m3 KV, f16 mma" if fp8 else "bf16",
+        "data": "synthetic (seeded bf16 N(0,1) q/k/v/KV, N(0,1) sinks, 1+N(0,0.1) norm weights"
+                + (", KV as E4M3 codes of x / per-head scale" if fp8 else "") + ")",
         "config": dict(workload_config(args.workload),
                        context=ctx if not args.workload.startswith("paged") else "per request",
+                       kv_dtype="e4m3" if fp8 else "bf16",
                        parallelism=f"replicas x{world}",
                        launch=launch),
         "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
                      "frac": achieved / peak, "peak_kind": peak_kind,
                      "frac_of_nominal_8000": achieved / NOMINAL_HBM_GBS,
                      "algorithmic_bytes": int(algo_bytes), "kernel": "flint decode_kernel",
-                     "traffic": traffic_for(args.workload, ctx)},
+                     "traffic": None if fp8 else traffic_for(args.workload, ctx)},
         "cpu_baseline": cpu_baseline,
         "e2e": e2e,
         "gpu_launches": args.steps,

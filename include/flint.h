@@ -76,8 +76,17 @@ typedef enum {
                                 block_table[b][t / 64], row t mod 64                 */
 } flint_kv_layout;
 
-/* One layer's KV cache for a batch of requests.  k and v are bf16 device
- * buffers of identical geometry. */
+typedef enum {
+    FLINT_KV_BF16 = 0,       /* one bf16 per cached value */
+    FLINT_KV_FP8_E4M3 = 1    /* one byte per value: an OCP E4M3 code of value / scale
+                                ("Recursive Flint" model JSON, the fp8 column of
+                                kvCacheGiBPerRequest; the format is this library's
+                                reading: the pages give only the byte count) */
+} flint_kv_dtype;
+
+/* One layer's KV cache for a batch of requests.  k and v are device buffers
+ * of identical geometry, with elements of the given dtype (the geometry below
+ * counts elements, so an E4M3 row of 4 x 128 values is 512 bytes). */
 typedef struct {
     void* k;
     void* v;
@@ -89,6 +98,11 @@ typedef struct {
     int32_t max_blocks_per_req;  /* PAGED */
     int32_t block_size;          /* PAGED: must be 64 */
     int32_t num_blocks;          /* PAGED: blocks in the pool */
+    int32_t dtype;               /* flint_kv_dtype; 0 (bf16) for zero-filled structs */
+    float k_scale[4];            /* FP8_E4M3: per KV head, stored code = e4m3(k / k_scale)
+                                    rounded to nearest even, saturated at +-448, with
+                                    the division in float32; value read = code * k_scale */
+    float v_scale[4];            /* FP8_E4M3: the same for v */
 } flint_kv_cache;
 
 /* One layer of one decoded token, for flint_attn_stack (batch 1). */

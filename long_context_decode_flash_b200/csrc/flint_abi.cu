@@ -89,48 +89,53 @@ struct MapKey {
   int dev;
   uintptr_t base;
   int64_t d2, d3, stride2;
+  int dtype;
   bool operator==(const MapKey& o) const {
-    return dev == o.dev && base == o.base && d2 == o.d2 && d3 == o.d3 && stride2 == o.stride2;
+    return dev == o.dev && base == o.base && d2 == o.d2 && d3 == o.d3 && stride2 == o.stride2 &&
+           dtype == o.dtype;
   }
 };
 struct MapKeyHash {
   size_t operator()(const MapKey& k) const {
     size_t h = std::hash<uintptr_t>()(k.base);
     h ^= std::hash<int64_t>()(k.d2 * 1000003 + k.d3) + 0x9e3779b97f4a7c15ull + (h << 6) + (h >> 2);
-    h ^= std::hash<int64_t>()(k.stride2 * 31 + k.dev) + 0x9e3779b97f4a7c15ull + (h << 6) + (h >> 2);
+    h ^= std::hash<int64_t>()(k.stride2 * 31 + k.dev * 2 + k.dtype) + 0x9e3779b97f4a7c15ull + (h << 6) + (h >> 2);
     return h;
   }
 };
 
-// A K or V cache seen as a 4-D bf16 tensor (dims innermost first):
+// A K or V cache seen as a 4-D tensor (dims innermost first):
 //   CONTIGUOUS/RING: [128 dims][4 heads][capacity tokens][B requests]
 //   PAGED:           [128 dims][4 heads][64 tokens][num_blocks]
-// read in boxes of 64 dims x 1 head x kTile (32) tokens x 1 with the 128-byte
-// swizzle.
+// read with the 128-byte swizzle in boxes of 64 dims x 1 head x kTile (32)
+// tokens x 1 for bf16, and of 128 dims x 1 head x 64 tokens x 1 for E4M3
+// (one byte per value); either way a box row is 128 bytes.
 flint_status encode_cache_map(CUtensorMap* map, void* base, const flint_kv_cache& c, int B) {
   EncodeTiledFn fn = encode_fn();
   if (!fn) return fail(FLINT_ERR_CUDA, "cuTensorMapEncodeTiled is not available from the driver");
+  const bool fp8 = c.dtype == FLINT_KV_FP8_E4M3;
+  const cuuint64_t eb = fp8 ? 1 : 2;  // bytes per element
   cuuint64_t dims[4], strides[3];
   dims[0] = kDim;
   dims[1] = kKvHeads;
-  strides[0] = kDim * 2;
-  strides[1] = kKvHeads * kDim * 2;
+  strides[0] = kDim * eb;
+  strides[1] = kKvHeads * kDim * eb;
   if (c.layout == FLINT_KV_PAGED) {
     dims[2] = kBlock;
     dims[3] = static_cast<cuuint64_t>(c.num_blocks);
-    strides[2] = static_cast<cuuint64_t>(kBlock) * kKvHeads * kDim * 2;
+    strides[2] = static_cast<cuuint64_t>(kBlock) * kKvHeads * kDim * eb;
   } else {
     const int64_t rs = c.req_stride ? c.req_stride : static_cast<int64_t>(c.capacity) * kKvHeads * kDim;
     dims[2] = static_cast<cuuint64_t>(c.capacity);
     dims[3] = static_cast<cuuint64_t>(B);
-    strides[2] = static_cast<cuuint64_t>(rs) * 2;
+    strides[2] = static_cast<cuuint64_t>(rs) * eb;
   }
   static std::mutex mu;
   static std::unordered_map<MapKey, CUtensorMap, MapKeyHash> cache;
   int dev = 0;
   cudaGetDevice(&dev);
   const MapKey key{dev, reinterpret_cast<uintptr_t>(base), static_cast<int64_t>(dims[2]),
-                   static_cast<int64_t>(dims[3]), static_cast<int64_t>(strides[2])};
+                   static_cast<int64_t>(dims[3]), static_cast<int64_t>(strides[2]), c.dtype};
   {
     std::lock_guard<std::mutex> lock(mu);
     auto it = cache.find(key);
@@ -139,9 +144,11 @@ flint_status encode_cache_map(CUtensorMap* map, void* base, const flint_kv_cache
       return FLINT_OK;
     }
   }
-  const cuuint32_t box[4] = {64, 1, static_cast<cuuint32_t>(kTile), 1};
+  const cuuint32_t box[4] = {fp8 ? static_cast<cuuint32_t>(kDim) : 64u, 1,
+                            static_cast<cuuint32_t>(fp8 ? kTileFp8 : kTile), 1};
   const cuuint32_t estr[4] = {1, 1, 1, 1};
-  CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, base, dims, strides, box, estr,
+  CUresult r = fn(map, fp8 ? CU_TENSOR_MAP_DATA_TYPE_UINT8 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, base, dims,
+                  strides, box, estr,
                   CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
                   static_cast<CUtensorMapL2promotion>(FLINT_L2_PROMOTION),
                   CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
@@ -157,6 +164,12 @@ flint_status encode_cache_map(CUtensorMap* map, void* base, const flint_kv_cache
 flint_status check_cache(const flint_kv_cache* c, int B, const char* who) {
   if (!c) return fail(FLINT_ERR_INVALID_ARG, "%s: cache is NULL", who);
   if (!c->k || !c->v) return fail(FLINT_ERR_INVALID_ARG, "%s: cache k/v is NULL", who);
+  if (c->dtype != FLINT_KV_BF16 && c->dtype != FLINT_KV_FP8_E4M3)
+    return fail(FLINT_ERR_INVALID_ARG, "%s: unknown cache dtype %d", who, c->dtype);
+  if (c->dtype == FLINT_KV_FP8_E4M3)
+    for (int g = 0; g < kKvHeads; ++g)
+      if (!(c->k_scale[g] > 0.f && c->k_scale[g] < 3.0e38f) || !(c->v_scale[g] > 0.f && c->v_scale[g] < 3.0e38f))
+        return fail(FLINT_ERR_INVALID_ARG, "%s: E4M3 scales must be finite and > 0", who);
   if (!aligned16(c->k) || !aligned16(c->v))
     return fail(FLINT_ERR_INVALID_ARG, "%s: cache k/v must be 16-byte aligned", who);
   switch (c->layout) {
@@ -167,9 +180,10 @@ flint_status check_cache(const flint_kv_cache* c, int B, const char* who) {
       if (c->layout == FLINT_KV_RING && c->capacity != kWindow)
         return fail(FLINT_ERR_UNSUPPORTED, "%s: a ring cache must have %d slots", who, kWindow);
       const int64_t dense = static_cast<int64_t>(c->capacity) * kKvHeads * kDim;
-      if (c->req_stride != 0 && (c->req_stride < dense || c->req_stride % 8 != 0))
-        return fail(FLINT_ERR_INVALID_ARG, "%s: req_stride %lld must be 0 or a multiple of 8 >= %lld",
-                    who, (long long)c->req_stride, (long long)dense);
+      const int64_t mult = c->dtype == FLINT_KV_FP8_E4M3 ? 16 : 8;  // 16-byte TMA strides
+      if (c->req_stride != 0 && (c->req_stride < dense || c->req_stride % mult != 0))
+        return fail(FLINT_ERR_INVALID_ARG, "%s: req_stride %lld must be 0 or a multiple of %lld >= %lld",
+                    who, (long long)c->req_stride, (long long)mult, (long long)dense);
       (void)B;
       return FLINT_OK;
     }
@@ -191,6 +205,7 @@ struct Range {
 };
 
 Range attended_range(const flint_kv_cache& c, int L, int window) {
+  const int T = c.dtype == FLINT_KV_FP8_E4M3 ? kTileFp8 : kTile;  // tokens per tile
   Range r;
   if (c.layout == FLINT_KV_RING) {
     r.lo = 0;
@@ -199,10 +214,10 @@ Range attended_range(const flint_kv_cache& c, int L, int window) {
   } else {
     r.lo = window > 0 ? std::max(0, L - window) : 0;
     r.hi = L;
-    // paged tiles must not straddle a block: start them on a multiple of kTile
-    r.tile_base = c.layout == FLINT_KV_PAGED ? (r.lo / kTile) * kTile : r.lo;
+    // paged tiles must not straddle a block: start them on a multiple of T
+    r.tile_base = c.layout == FLINT_KV_PAGED ? (r.lo / T) * T : r.lo;
   }
-  r.tiles = (r.hi - r.tile_base + kTile - 1) / kTile;
+  r.tiles = (r.hi - r.tile_base + T - 1) / T;
   return r;
 }
 
@@ -294,6 +309,24 @@ flint_status plan(DecodeParams& P, const int* tiles, int n_problems, int num_cta
   P.ws_items = cap;
   *grid = P.n_queue > 0 ? G : last;
   return FLINT_OK;
+}
+
+// E4M3 scales of the cache behind map pair `pair` (read by the kernel as
+// kv_scales[map_k / 2]); zero for a bf16 cache.
+void set_scales(DecodeParams& P, int pair, const flint_kv_cache& c) {
+  for (int g = 0; g < kKvHeads; ++g) {
+    const bool fp8 = c.dtype == FLINT_KV_FP8_E4M3;
+    P.kv_scales[pair][g] = fp8 ? c.k_scale[g] : 0.f;
+    P.kv_scales[pair][4 + g] = fp8 ? c.v_scale[g] : 0.f;
+  }
+}
+
+void set_prep_fp8(PrepParams& p, const flint_kv_cache& c) {
+  p.fp8 = c.dtype == FLINT_KV_FP8_E4M3 ? 1 : 0;
+  for (int g = 0; g < kKvHeads; ++g) {
+    p.k_scale[g] = p.fp8 ? c.k_scale[g] : 0.f;
+    p.v_scale[g] = p.fp8 ? c.v_scale[g] : 0.f;
+  }
 }
 
 flint_status launch_result(cudaError_t e, const char* who) {
@@ -404,6 +437,7 @@ flint_status flint_qk_norm_rope(const uint16_t* q_raw, const uint16_t* k_raw, co
                                      : static_cast<int64_t>(cache->capacity) * kKvHeads * kDim;
     p.max_blocks = cache->max_blocks_per_req;
     p.num_blocks = cache->num_blocks;
+    set_prep_fp8(p, *cache);
   }
   return launch_result(launch_prep(p, B, static_cast<cudaStream_t>(stream)), who);
 }
@@ -441,6 +475,7 @@ flint_status flint_kv_append(const uint16_t* k, const uint16_t* v, const int32_t
                                    : static_cast<int64_t>(cache->capacity) * kKvHeads * kDim;
   p.max_blocks = cache->max_blocks_per_req;
   p.num_blocks = cache->num_blocks;
+  set_prep_fp8(p, *cache);
   return launch_result(launch_prep(p, B, static_cast<cudaStream_t>(stream)), who);
 }
 
@@ -492,11 +527,13 @@ flint_status flint_attn_decode(const void* q, int32_t q_is_fp32, const flint_kv_
     pb.req = static_cast<int16_t>(cache->layout == FLINT_KV_PAGED ? 0 : b);
     pb.layout = static_cast<int8_t>(cache->layout);
     pb.q_fp32 = static_cast<int8_t>(q_is_fp32);
+    pb.fp8 = static_cast<int8_t>(cache->dtype == FLINT_KV_FP8_E4M3);
     tiles[b] = r.tiles;
   }
   int grid = 0;
   s = plan(P, tiles, B, num_ctas, ws_bytes, who, &grid);
   if (s != FLINT_OK) return s;
+  set_scales(P, 0, *cache);
   s = encode_cache_map(&P.maps[0], cache->k, *cache, B);
   if (s != FLINT_OK) return s;
   s = encode_cache_map(&P.maps[1], cache->v, *cache, B);
@@ -567,6 +604,8 @@ flint_status flint_attn_stack(const flint_layer* layers, int32_t n_layers, int32
     pb.layout = static_cast<int8_t>(ly.cache.layout);
     pb.q_fp32 = 0;
     pb.rope = static_cast<int8_t>(ly.rope);
+    pb.fp8 = static_cast<int8_t>(ly.cache.dtype == FLINT_KV_FP8_E4M3);
+    set_scales(P, i, ly.cache);
     tiles[i] = r.tiles;
     s = encode_cache_map(&P.maps[2 * i], ly.cache.k, ly.cache, 1);
     if (s != FLINT_OK) return s;

@@ -103,6 +103,10 @@ __device__ __forceinline__ Smem carve(uint8_t* raw) {
 __device__ __forceinline__ uint32_t box_offset(int kv, int head, int half) {
   return static_cast<uint32_t>(((kv * kKvHeads + head) * 2 + half) * kBoxBytes);
 }
+// E4M3 stage: one box of 64 tokens x 128 dims per (K/V, head).
+__device__ __forceinline__ uint32_t box_offset_fp8(int kv, int head) {
+  return static_cast<uint32_t>((kv * kKvHeads + head) * kBoxBytesFp8);
+}
 
 __device__ __forceinline__ void consumer_bar() {
   asm volatile("bar.sync 1, %0;" ::"n"(kConsumerWarps * 32) : "memory");
@@ -142,12 +146,24 @@ __device__ void append_new_token(const DecodeParams& P, const Problem& pb, const
   for (int g = 0; g < kKvHeads; ++g) {
     float y[4];
     norm_rope_row_warp(k_raw + g * kDim, w_k, P.eps, true, pb.rope != 0, cs, lane, y);
-    uint32_t* kd = reinterpret_cast<uint32_t*>(pb.k_rows + row + g * kDim);
-    uint32_t* vd = reinterpret_cast<uint32_t*>(pb.v_rows + row + g * kDim);
-    kd[lane] = pack_bf16x2(y[0], y[1]);
-    kd[32 + lane] = pack_bf16x2(y[2], y[3]);
-    vd[lane] = v_raw[g * 64 + lane];
-    vd[32 + lane] = v_raw[g * 64 + 32 + lane];
+    const uint32_t va = v_raw[g * 64 + lane], vb = v_raw[g * 64 + 32 + lane];
+    if (!pb.fp8) {
+      uint32_t* kd = reinterpret_cast<uint32_t*>(pb.k_rows + row + g * kDim);
+      uint32_t* vd = reinterpret_cast<uint32_t*>(pb.v_rows + row + g * kDim);
+      kd[lane] = pack_bf16x2(y[0], y[1]);
+      kd[32 + lane] = pack_bf16x2(y[2], y[3]);
+      vd[lane] = va;
+      vd[32 + lane] = vb;
+    } else {
+      // E4M3: code = e4m3(x / scale), the division in float32 (IEEE, nearest)
+      const float ks = P.kv_scales[pb.map_k >> 1][g], vs = P.kv_scales[pb.map_k >> 1][4 + g];
+      uint16_t* kd = reinterpret_cast<uint16_t*>(reinterpret_cast<uint8_t*>(pb.k_rows) + row + g * kDim);
+      uint16_t* vd = reinterpret_cast<uint16_t*>(reinterpret_cast<uint8_t*>(pb.v_rows) + row + g * kDim);
+      kd[lane] = static_cast<uint16_t>(f32x2_to_e4m3x2(__fdiv_rn(y[0], ks), __fdiv_rn(y[1], ks)));
+      kd[32 + lane] = static_cast<uint16_t>(f32x2_to_e4m3x2(__fdiv_rn(y[2], ks), __fdiv_rn(y[3], ks)));
+      vd[lane] = static_cast<uint16_t>(f32x2_to_e4m3x2(__fdiv_rn(bf16_lo(va), vs), __fdiv_rn(bf16_hi(va), vs)));
+      vd[32 + lane] = static_cast<uint16_t>(f32x2_to_e4m3x2(__fdiv_rn(bf16_lo(vb), vs), __fdiv_rn(bf16_hi(vb), vs)));
+    }
   }
   fence_proxy_async_global();
 }
@@ -220,14 +236,21 @@ __device__ ProducerCount run_producer(const DecodeParams& P, const Smem& S, int 
     }
     const Item item = P.items[it];
     const Problem& pb = P.prob[item.seg];
-    const CUtensorMap* map = &P.maps[my_kv ? pb.map_v : pb.map_k];
+    const bool fp8 = pb.fp8 != 0;
+    const int tile_tok = fp8 ? kTileFp8 : kTile;
+    // bf16: lane i < 16 loads box (K/V, head, dim half); E4M3: lane i < 8 loads box (K/V, head)
+    const int b_kv = fp8 ? (lane >> 2) & 1 : my_kv, b_head = fp8 ? lane & 3 : my_head;
+    const int n_boxes = fp8 ? 2 * kKvHeads : kBoxes;
+    const uint32_t b_off = fp8 ? box_offset_fp8(b_kv, b_head) : box_offset(my_kv, my_head, my_half);
+    const int b_x = fp8 ? 0 : 64 * my_half;
+    const CUtensorMap* map = &P.maps[b_kv ? pb.map_v : pb.map_k];
     const bool paged = pb.layout == FLINT_KV_PAGED;
-    const int app_tile = (P.prep && pb.append_tok >= 0) ? (pb.append_tok - pb.tile_base) / kTile : -1;
+    const int app_tile = (P.prep && pb.append_tok >= 0) ? (pb.append_tok - pb.tile_base) / tile_tok : -1;
     for (int t = item.t0; t < item.t1; t += 32) {
       const int n = min(32, item.t1 - t);
       int blk = 0;
       if (paged && lane < n) {
-        const int idx = (pb.tile_base + (t + lane) * kTile) / kBlock;
+        const int idx = (pb.tile_base + (t + lane) * tile_tok) / kBlock;
         if (FLINT_CHECK(P.dev_err, idx >= 0 && idx < pb.table_len, 3, idx, pb.table_len, it)) blk = __ldg(pb.table + idx);
         // An out-of-range coordinate makes TMA fill zeros; flag it for the caller.
         if (blk < 0 || blk >= pb.num_blocks) report_error(P.dev_err, FLINT_ERR_INVALID_ARG);
@@ -264,7 +287,7 @@ __device__ ProducerCount run_producer(const DecodeParams& P, const Smem& S, int 
         }
         const uint32_t fb = smem_u32(&S.full[stage]);
         const uint32_t base = smem_u32(S.stages + stage * kStageBytes);
-        const int tok = pb.tile_base + tile * kTile;
+        const int tok = pb.tile_base + tile * tile_tok;
         const int c2 = paged ? tok % kBlock : tok;
         const int c3 = paged ? b : pb.req;
         bool fine = true;
@@ -279,12 +302,11 @@ __device__ ProducerCount run_producer(const DecodeParams& P, const Smem& S, int 
         }
         fine = __shfl_sync(0xffffffffu, fine, 0);
         __syncwarp();
-        if (fine && lane < kBoxes) {
+        if (fine && lane < n_boxes) {
 #if FLINT_KV_EVICT_FIRST
-          tma_load_4d_hint(base + box_offset(my_kv, my_head, my_half), map, fb, 64 * my_half, my_head, c2,
-                           c3, kv_policy);
+          tma_load_4d_hint(base + b_off, map, fb, b_x, b_head, c2, c3, kv_policy);
 #else
-          tma_load_4d(base + box_offset(my_kv, my_head, my_half), map, fb, 64 * my_half, my_head, c2, c3);
+          tma_load_4d(base + b_off, map, fb, b_x, b_head, c2, c3);
 #endif
         }
         __syncwarp();
@@ -293,18 +315,30 @@ __device__ ProducerCount run_producer(const DecodeParams& P, const Smem& S, int 
   }
 }
 
-// q fragments for query head h: thread (g = lane/4, c = lane%4) holds dims
-// 16kk + 2c + {0,1} and 16kk + 2c + 8 + {0,1} for kk = 0..7 as the A operand
-// rows g (bf16 hi part) and g + 8 (bf16 lo part), prescaled by log2(e)/sqrt(128).
+// Dims of the values a consumer thread with quad index c holds, 16 at a time:
+// within each 16-dim chunk q, its values 0-1 are dims 16q + d0 + {0, 1} and
+// values 2-3 are 16q + d2 + {0, 1}.  For a bf16 cache (d0, d2) = (2c, 2c + 8),
+// the mma.sync fragment layout; for an E4M3 cache (4c, 4c + 2), the 4
+// consecutive bytes ldmatrix gives a thread from a row of fp8 values.  The q
+// fragment, the O accumulator and the outputs all follow the same map.
+__device__ __forceinline__ int dim_d0(int c, bool fp8) { return fp8 ? 4 * c : 2 * c; }
+__device__ __forceinline__ int dim_d2(int c, bool fp8) { return fp8 ? 4 * c + 2 : 2 * c + 8; }
+
+// q fragments for query head h: thread (g = lane/4, c = lane%4) holds, for
+// each 16-dim chunk kk, the dims above as the A operand rows g (hi part) and
+// g + 8 (lo part), prescaled by log2(e)/sqrt(128); bf16 parts for a bf16
+// cache, f16 parts for an E4M3 cache (the operands of one mma share a type).
 __device__ __forceinline__ void load_q(const DecodeParams& P, const Problem& pb, const uint8_t* in,
                                        int h, int c, const float2* cs, uint32_t (&qa)[8][4]) {
+  const bool fp8 = pb.fp8 != 0;
+  const int d0 = dim_d0(c, fp8), d2 = dim_d2(c, fp8);
   float x[8][4];
   if (P.prep || !pb.q_fp32) {
     const uint16_t* q = reinterpret_cast<const uint16_t*>(in + kInQ) + h * kDim;
 #pragma unroll
     for (int kk = 0; kk < 8; ++kk) {
-      const uint32_t a = *reinterpret_cast<const uint32_t*>(q + 16 * kk + 2 * c);
-      const uint32_t b = *reinterpret_cast<const uint32_t*>(q + 16 * kk + 2 * c + 8);
+      const uint32_t a = *reinterpret_cast<const uint32_t*>(q + 16 * kk + d0);
+      const uint32_t b = *reinterpret_cast<const uint32_t*>(q + 16 * kk + d2);
       x[kk][0] = bf16_lo(a);
       x[kk][1] = bf16_hi(a);
       x[kk][2] = bf16_lo(b);
@@ -314,8 +348,8 @@ __device__ __forceinline__ void load_q(const DecodeParams& P, const Problem& pb,
     const float* q = static_cast<const float*>(pb.q) + h * kDim;
 #pragma unroll
     for (int kk = 0; kk < 8; ++kk) {
-      const float2 a = *reinterpret_cast<const float2*>(q + 16 * kk + 2 * c);
-      const float2 b = *reinterpret_cast<const float2*>(q + 16 * kk + 2 * c + 8);
+      const float2 a = *reinterpret_cast<const float2*>(q + 16 * kk + d0);
+      const float2 b = *reinterpret_cast<const float2*>(q + 16 * kk + d2);
       x[kk][0] = a.x;
       x[kk][1] = a.y;
       x[kk][2] = b.x;
@@ -336,8 +370,8 @@ __device__ __forceinline__ void load_q(const DecodeParams& P, const Problem& pb,
 #pragma unroll
     for (int kk = 0; kk < 8; ++kk) {
       const uint16_t* w_q = reinterpret_cast<const uint16_t*>(in + kInWq);
-      const uint32_t a = *reinterpret_cast<const uint32_t*>(w_q + 16 * kk + 2 * c);
-      const uint32_t b = *reinterpret_cast<const uint32_t*>(w_q + 16 * kk + 2 * c + 8);
+      const uint32_t a = *reinterpret_cast<const uint32_t*>(w_q + 16 * kk + d0);
+      const uint32_t b = *reinterpret_cast<const uint32_t*>(w_q + 16 * kk + d2);
       x[kk][0] = x[kk][0] * r * bf16_lo(a);
       x[kk][1] = x[kk][1] * r * bf16_hi(a);
       x[kk][2] = x[kk][2] * r * bf16_lo(b);
@@ -348,17 +382,25 @@ __device__ __forceinline__ void load_q(const DecodeParams& P, const Problem& pb,
       for (int kk = 0; kk < 4; ++kk)
 #pragma unroll
         for (int e = 0; e < 4; ++e) {
-          const float2 t = cs[16 * kk + 2 * c + (e & 1) + ((e >> 1) << 3)];
+          const float2 t = cs[16 * kk + ((e >> 1) ? d2 : d0) + (e & 1)];
           const float a = x[kk][e], b = x[kk + 4][e];
           x[kk][e] = a * t.x - b * t.y;
           x[kk + 4][e] = b * t.x + a * t.y;
         }
     }
   }
+  if (fp8) {
 #pragma unroll
-  for (int kk = 0; kk < 8; ++kk) {
-    split_bf16x2(x[kk][0] * kQScale, x[kk][1] * kQScale, qa[kk][0], qa[kk][1]);
-    split_bf16x2(x[kk][2] * kQScale, x[kk][3] * kQScale, qa[kk][2], qa[kk][3]);
+    for (int kk = 0; kk < 8; ++kk) {
+      split_f16x2(x[kk][0] * kQScale, x[kk][1] * kQScale, qa[kk][0], qa[kk][1]);
+      split_f16x2(x[kk][2] * kQScale, x[kk][3] * kQScale, qa[kk][2], qa[kk][3]);
+    }
+  } else {
+#pragma unroll
+    for (int kk = 0; kk < 8; ++kk) {
+      split_bf16x2(x[kk][0] * kQScale, x[kk][1] * kQScale, qa[kk][0], qa[kk][1]);
+      split_bf16x2(x[kk][2] * kQScale, x[kk][3] * kQScale, qa[kk][2], qa[kk][3]);
+    }
   }
 }
 
@@ -450,6 +492,111 @@ __device__ __forceinline__ void consume_slice(uint32_t sK, uint32_t sV, int tok0
   }
 }
 
+// consume_slice for an E4M3 cache.  sK / sV point at row r0 of the head's K /
+// V boxes (kTileFp8 rows of 128 one-byte dims, 128-byte swizzle, r0 a
+// multiple of 8).  ldmatrix gives thread (g, c) 4 consecutive bytes of a row:
+// dims 16u + 4c .. 16u + 4c + 3, widened to f16.
+//   * QK: those bytes are the B fragment of K^T for the logical k order in
+//     which q was loaded (dims d0 = 4c, d2 = 4c + 2); the scores are then
+//     multiplied by the head's k scale.
+//   * PV: the widened V rows form two 8x8 f16 matrices per 16-dim chunk (dims
+//     16u + {0,1,4,5,8,9,12,13} and 16u + {2,3,6,7,10,11,14,15}); their
+//     transposes (movmatrix) are the B fragments of V for 8 tokens each, and
+//     O n-tile 2u + h holds dims 16u + 4c + 2h + {0, 1} in thread (g, c).
+// The caller multiplies O by the head's v scale at the item's end.
+__device__ __forceinline__ void consume_slice_fp8(uint32_t sK, uint32_t sV, int tok0, int lo, int hi,
+                                                  int lane, const uint32_t (&qa)[8][4], float k_scale,
+                                                  float& m_run, float& l_run, float (&o)[16][4]) {
+  const int c = lane & 3;
+  const int l7 = lane & 7;
+  const bool whole = (tok0 >= lo) && (tok0 + kSlice <= hi);
+
+  float sc[4];
+#pragma unroll
+  for (int jj = 0; jj < 2; ++jj) {
+    float a0[4] = {0.f, 0.f, 0.f, 0.f}, a1[4] = {0.f, 0.f, 0.f, 0.f};
+    const uint32_t row = sK + (8 * jj + l7) * 128;
+#pragma unroll
+    for (int kk = 0; kk < 8; kk += 4) {
+      const int u = kk + (lane >> 3);  // lanes 8i..8i+7 address 16-dim chunk kk + i
+      uint32_t r[4];
+      ldsm_x4(row + ((u ^ l7) << 4), r[0], r[1], r[2], r[3]);
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        const uint32_t b0 = e4m3x2_to_f16x2(r[i]), b1 = e4m3x2_to_f16x2(r[i] >> 16);
+        if (i & 1)
+          mma_f16_16816(a1, qa[kk + i], b0, b1);
+        else
+          mma_f16_16816(a0, qa[kk + i], b0, b1);
+      }
+    }
+    sc[2 * jj] = ((a0[0] + a1[0]) + (a0[2] + a1[2])) * k_scale;
+    sc[2 * jj + 1] = ((a0[1] + a1[1]) + (a0[3] + a1[3])) * k_scale;
+  }
+  if (!whole) {
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const int tok = tok0 + 8 * (i >> 1) + 2 * c + (i & 1);
+      if (tok < lo || tok >= hi) sc[i] = -INFINITY;
+    }
+  }
+
+  float mx = fmaxf(fmaxf(sc[0], sc[1]), fmaxf(sc[2], sc[3]));
+  mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 1));
+  mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 2));
+  const bool grow = mx > m_run + kRescaleSlack;
+  if (__any_sync(0xffffffffu, grow)) {
+    const float alpha = grow ? exp2f(m_run - mx) : 1.0f;
+    l_run *= alpha;
+#pragma unroll
+    for (int n = 0; n < 16; ++n)
+#pragma unroll
+      for (int e = 0; e < 4; ++e) o[n][e] *= alpha;
+    if (grow) m_run = mx;
+  }
+  const float mu = (m_run == -INFINITY) ? 0.f : m_run;
+
+  const float p0 = exp2f(sc[0] - mu), p1 = exp2f(sc[1] - mu);
+  const float p2 = exp2f(sc[2] - mu), p3 = exp2f(sc[3] - mu);
+  l_run += (p0 + p1) + (p2 + p3);
+  uint32_t pa[4];
+  split_f16x2(p0, p1, pa[0], pa[1]);
+  split_f16x2(p2, p3, pa[2], pa[3]);
+
+  uint32_t m01 = 0xffffffffu, m23 = 0xffffffffu;
+  if (!whole) {
+    const int t = tok0 + 2 * c;
+    m01 = ((t >= lo && t < hi) ? 0x0000ffffu : 0u) | ((t + 1 >= lo && t + 1 < hi) ? 0xffff0000u : 0u);
+    m23 = ((t + 8 >= lo && t + 8 < hi) ? 0x0000ffffu : 0u) |
+          ((t + 9 >= lo && t + 9 < hi) ? 0xffff0000u : 0u);
+  }
+  // lanes 8i..8i+7 address tokens 8(i & 1) + l7 of chunk u = up + (i >> 1)
+  const uint32_t row = sV + (((lane >> 3) & 1) * 8 + l7) * 128;
+#pragma unroll
+  for (int up = 0; up < 8; up += 2) {
+    const int u = up + (lane >> 4);
+    uint32_t x[4];
+    ldsm_x4(row + ((u ^ l7) << 4), x[0], x[1], x[2], x[3]);
+#pragma unroll
+    for (int half = 0; half < 2; ++half) {  // chunk up + half: x[2 half] tokens 0-7, x[2 half + 1] tokens 8-15
+      const uint32_t t0 = x[2 * half], t1 = x[2 * half + 1];
+      uint32_t v0 = movmatrix_trans(e4m3x2_to_f16x2(t0));          // dims 4c, 4c+1 of 8 tokens
+      uint32_t v1 = movmatrix_trans(e4m3x2_to_f16x2(t1));
+      uint32_t v2 = movmatrix_trans(e4m3x2_to_f16x2(t0 >> 16));    // dims 4c+2, 4c+3
+      uint32_t v3 = movmatrix_trans(e4m3x2_to_f16x2(t1 >> 16));
+      if (!whole) {  // rows outside the range may hold anything (even NaN codes)
+        v0 &= m01;
+        v2 &= m01;
+        v1 &= m23;
+        v3 &= m23;
+      }
+      const int nt = 2 * (up + half);
+      mma_f16_16816(o[nt], pa, v0, v1);
+      mma_f16_16816(o[nt + 1], pa, v2, v3);
+    }
+  }
+}
+
 // Float4 slot of values 4q..4q+3 of consumer thread (head, c)'s 32 O values
 // inside a partial.  The 32 threads of a KV head's warp (lane = 4(head % 8) + c)
 // hold chunk q in 512 consecutive bytes, so a warp's load or store of one
@@ -467,10 +614,13 @@ __device__ __forceinline__ void finish_head(const Problem& pb, int head, int c, 
   const float Mf = fmaxf(M, s2);
   const float a = (M == -INFINITY) ? 0.f : exp2f(M - Mf);
   const float scale = a / (L * a + exp2f(s2 - Mf));
-  float* dst = pb.out + head * kDim + 2 * c;
+  float* dst = pb.out + head * kDim;
+  const int d0 = dim_d0(c, pb.fp8 != 0), d2 = dim_d2(c, pb.fp8 != 0);
 #pragma unroll
-  for (int n = 0; n < 16; ++n)
-    *reinterpret_cast<float2*>(dst + 8 * n) = make_float2(v[2 * n] * scale, v[2 * n + 1] * scale);
+  for (int q = 0; q < 8; ++q) {
+    *reinterpret_cast<float2*>(dst + 16 * q + d0) = make_float2(v[4 * q] * scale, v[4 * q + 1] * scale);
+    *reinterpret_cast<float2*>(dst + 16 * q + d2) = make_float2(v[4 * q + 2] * scale, v[4 * q + 3] * scale);
+  }
 }
 
 // Folds partials i = s0 + r, s0 + r + stride, ... (< s1) of (head, quarter c)
@@ -533,10 +683,13 @@ __device__ void run_consumer(const DecodeParams& P, const Smem& S, int warp, int
     const Problem& pb = P.prob[item.seg];
     // this head's sink logit, needed only at the item's end: load it now
     const float sink = pb.sinks[head];
+    // E4M3 cache: the KV head's scales (unused for bf16)
+    const float k_scale = P.kv_scales[pb.map_k >> 1][kvh];
+    const float v_scale = P.kv_scales[pb.map_k >> 1][4 + kvh];
     {
       load_q(P, pb, S.in, head, c, S.cs, qa);
       if (P.prep && warp == kAppendWarp && pb.append_tok >= 0) {
-        const int app_tile = (pb.append_tok - pb.tile_base) / kTile;
+        const int app_tile = (pb.append_tok - pb.tile_base) / (pb.fp8 ? kTileFp8 : kTile);
         if (app_tile >= item.t0 && app_tile < item.t1) {
           append_new_token(P, pb, S.in, lane, S.cs);
           __syncwarp();
@@ -569,10 +722,21 @@ __device__ void run_consumer(const DecodeParams& P, const Smem& S, int warp, int
         continue;  // keep walking so that every warp meets the same barriers
       }
       const uint32_t base = smem_u32(S.stages + stage * kStageBytes);
-      const int r0 = group * kSlice;
-      const int tok0 = pb.tile_base + (item.t0 + k) * kTile + r0;
-      consume_slice(base + box_offset(0, kvh, 0) + r0 * 128, base + box_offset(1, kvh, 0) + r0 * 128,
-                    tok0, pb.lo, pb.hi, lane, qa, m_run, l_run, o);
+      if (!pb.fp8) {
+        const int r0 = group * kSlice;
+        const int tok0 = pb.tile_base + (item.t0 + k) * kTile + r0;
+        consume_slice(base + box_offset(0, kvh, 0) + r0 * 128, base + box_offset(1, kvh, 0) + r0 * 128,
+                      tok0, pb.lo, pb.hi, lane, qa, m_run, l_run, o);
+      } else {
+        // 64-token E4M3 tile: group q takes tokens 32q .. 32q + 31, two slices
+#pragma unroll 1
+        for (int sl = 0; sl < kTileFp8 / (kConsumerGroups * kSlice); ++sl) {
+          const int r0 = (group * (kTileFp8 / kConsumerGroups)) + sl * kSlice;
+          const int tok0 = pb.tile_base + (item.t0 + k) * kTileFp8 + r0;
+          consume_slice_fp8(base + box_offset_fp8(0, kvh) + r0 * 128, base + box_offset_fp8(1, kvh) + r0 * 128,
+                            tok0, pb.lo, pb.hi, lane, qa, k_scale, m_run, l_run, o);
+        }
+      }
       __syncwarp();
       if (lane == 0) mbar_arrive(smem_u32(&S.empty[stage]));
     }
@@ -581,10 +745,11 @@ __device__ void run_consumer(const DecodeParams& P, const Smem& S, int warp, int
     l_run += __shfl_xor_sync(0xffffffffu, l_run, 1);
     l_run += __shfl_xor_sync(0xffffffffu, l_run, 2);
     float v[32];
+    const float o_scale = pb.fp8 ? v_scale : 1.0f;  // E4M3: V was read as codes
 #pragma unroll
     for (int n = 0; n < 16; ++n) {
-      v[2 * n] = o[n][0] + o[n][2];
-      v[2 * n + 1] = o[n][1] + o[n][3];
+      v[2 * n] = (o[n][0] + o[n][2]) * o_scale;
+      v[2 * n + 1] = (o[n][1] + o[n][3]) * o_scale;
     }
     if (kConsumerGroups > 1) {
       // the other groups hand their states to group 0, which merges them
@@ -711,9 +876,9 @@ __device__ bool grid_barrier(unsigned int* bar, const Smem& S) {
 
 // Merge of the deferred problems by the whole grid after the grid barrier, in
 // units of (problem, KV head g, chunk q).  Lane (h, c) of a warp owns values
-// 4q..4q+3 of head 8g + h, quarter c: dims 16q + 2c + {0, 1} and
-// 16q + 8 + 2c + {0, 1} of the head (the layout the consumer warps wrote), so
-// one warp load reads 512 consecutive bytes of a partial.  A lane folds its
+// 4q..4q+3 of head 8g + h, quarter c: dims 16q + d0 + {0, 1} and
+// 16q + d2 + {0, 1} of the head (see dim_d0; the layout the consumer warps
+// wrote), so one warp load reads 512 consecutive bytes of a partial.  A lane folds its
 // partials kMergeBatch loads at a time, in item order.
 //   * Most problems take one warp per unit, every lane folding all partials.
 //   * A problem with many partials (a lone long problem split over every CTA)
@@ -762,9 +927,10 @@ __device__ __forceinline__ void write_chunk(const Problem& pb, int head, int c, 
   const float Mf = fmaxf(m, s2);
   const float a = (m == -INFINITY) ? 0.f : exp2f(m - Mf);
   const float scale = a / (l * a + exp2f(s2 - Mf));
-  float* o = pb.out + head * kDim + 16 * q + 2 * c;
-  *reinterpret_cast<float2*>(o) = make_float2(acc.x * scale, acc.y * scale);
-  *reinterpret_cast<float2*>(o + 8) = make_float2(acc.z * scale, acc.w * scale);
+  float* o = pb.out + head * kDim + 16 * q;
+  const int d0 = dim_d0(c, pb.fp8 != 0), d2 = dim_d2(c, pb.fp8 != 0);
+  *reinterpret_cast<float2*>(o + d0) = make_float2(acc.x * scale, acc.y * scale);
+  *reinterpret_cast<float2*>(o + d2) = make_float2(acc.z * scale, acc.w * scale);
 }
 
 __device__ void grid_merge(const DecodeParams& P, const Smem& S) {

@@ -93,7 +93,13 @@ struct Problem {
   int16_t req;              // 4th tensor coordinate (request) for CONTIGUOUS/RING
   int8_t layout, q_fp32, rope;
   int8_t deferred;          // 1: merged by the whole grid after a grid barrier
+  int8_t fp8;               // 1: E4M3 cache, 64-token tiles, scales in kv_scales[map_k / 2]
+  int8_t pad_;
 };
+static_assert(sizeof(Problem) == 128, "Problem stays 128 bytes");
+
+constexpr int kTileFp8 = 64;                  // tokens per stage for an E4M3 cache
+constexpr int kBoxBytesFp8 = kTileFp8 * 128;  // one box: 128 dims x 64 tokens, 8 KiB
 
 struct Item {
   int16_t seg;              // problem
@@ -114,6 +120,7 @@ struct DecodeParams {
   float* partials;          // workspace: one partial per item
   int32_t* dev_err;         // [0] status; debug builds also record a failed check in [2..7]
   float2 rope_cs[kDim / 2]; // prep: cos, sin of pos * theta^(-2i/128), from the host in double
+  float kv_scales[kMaxMaps / 2][8];  // per cache (map pair): k_scale[4], v_scale[4] for E4M3
   float eps;
   int32_t n_problems;
   int32_t prep;             // 1: q/k norm (+RoPE) and append fused in (layer stack)
@@ -149,6 +156,8 @@ struct PrepParams {
   float eps;
   int32_t apply_rope;
   int32_t do_norm;          // 0: k is already final (plain append)
+  int32_t fp8;              // 1: E4M3 cache (k_rows / v_rows are byte rows)
+  float k_scale[4], v_scale[4];
 };
 
 // Launchers (return cudaGetLastError() after the launch).

@@ -8,7 +8,9 @@
 // rows, then 4 k rows) with RoPE pairs (i, i+64) in one lane.  k is rounded
 // to bf16 (nearest even) once and the same bits go to k_out and the cache; v
 // is copied bit for bit.  With do_norm = 0 and no RoPE the kernel is a plain
-// bit-exact append of final k and v.
+// bit-exact append of final k and v.  An E4M3 cache receives, for k and v,
+// the codes of float32 (value / scale) (nearest even, saturating), where k is
+// the float32 normed (roped) value.
 #include "flint_device.cuh"
 
 namespace flint {
@@ -62,17 +64,32 @@ __global__ void __launch_bounds__(kPrepThreads) prep_kernel(const __grid_constan
         o[lane] = ka;
         o[32 + lane] = kb;
       }
-      if (row >= 0) {
+      if (row >= 0 && !p.fp8) {
         uint32_t* o = reinterpret_cast<uint32_t*>(p.k_rows + row + hk * kDim);
         o[lane] = ka;
         o[32 + lane] = kb;
+      } else if (row >= 0) {
+        const float s = p.k_scale[hk];
+        uint16_t* o = reinterpret_cast<uint16_t*>(reinterpret_cast<uint8_t*>(p.k_rows) + row + hk * kDim);
+        o[lane] = static_cast<uint16_t>(f32x2_to_e4m3x2(__fdiv_rn(y[0], s), __fdiv_rn(y[1], s)));
+        o[32 + lane] = static_cast<uint16_t>(f32x2_to_e4m3x2(__fdiv_rn(y[2], s), __fdiv_rn(y[3], s)));
       }
     }
   }
   if (row >= 0 && warp < kKvHeads) {
     const uint2* src = reinterpret_cast<const uint2*>(p.v_raw + (static_cast<long long>(b) * kKvHeads + warp) * kDim);
-    uint2* dst = reinterpret_cast<uint2*>(p.v_rows + row + warp * kDim);
-    dst[lane] = src[lane];
+    if (!p.fp8) {
+      uint2* dst = reinterpret_cast<uint2*>(p.v_rows + row + warp * kDim);
+      dst[lane] = src[lane];
+    } else {
+      // lane: dims 4l .. 4l+3
+      const uint2 x = src[lane];
+      const float s = p.v_scale[warp];
+      const uint32_t lo = f32x2_to_e4m3x2(__fdiv_rn(bf16_lo(x.x), s), __fdiv_rn(bf16_hi(x.x), s));
+      const uint32_t hi = f32x2_to_e4m3x2(__fdiv_rn(bf16_lo(x.y), s), __fdiv_rn(bf16_hi(x.y), s));
+      uint32_t* dst = reinterpret_cast<uint32_t*>(reinterpret_cast<uint8_t*>(p.v_rows) + row + warp * kDim);
+      dst[lane] = (lo & 0xffffu) | (hi << 16);
+    }
   }
 }
 

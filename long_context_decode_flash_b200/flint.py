@@ -24,6 +24,7 @@ FLINT_ERR_CUDA = 4
 FLINT_ERR_TIMEOUT = 5
 
 CONTIGUOUS, RING, PAGED = 0, 1, 2
+KV_BF16, KV_FP8_E4M3 = 0, 1
 NUM_Q_HEADS, NUM_KV_HEADS, HEAD_DIM = 32, 4, 128
 WINDOW, BLOCK_SIZE, MAX_CONTEXT = 513, 64, 262144
 MAX_BATCH, MAX_LAYERS = 64, 49
@@ -46,7 +47,9 @@ class KVCache(ctypes.Structure):
     _fields_ = [("k", ctypes.c_void_p), ("v", ctypes.c_void_p), ("layout", ctypes.c_int32),
                 ("capacity", ctypes.c_int32), ("req_stride", ctypes.c_int64),
                 ("block_table", ctypes.c_void_p), ("max_blocks_per_req", ctypes.c_int32),
-                ("block_size", ctypes.c_int32), ("num_blocks", ctypes.c_int32)]
+                ("block_size", ctypes.c_int32), ("num_blocks", ctypes.c_int32),
+                ("dtype", ctypes.c_int32), ("k_scale", ctypes.c_float * 4),
+                ("v_scale", ctypes.c_float * 4)]
 
 
 class StackLayer(ctypes.Structure):
@@ -132,10 +135,21 @@ def flint_kv_bytes(ctx_len: int, n_full: int = 14, n_window: int = 35, window: i
 
 def kv_cache(k: torch.Tensor, v: torch.Tensor, layout: int, capacity: int = 0,
              req_stride: int = 0, block_table: Optional[torch.Tensor] = None,
-             num_blocks: int = 0) -> KVCache:
-    """A flint_kv_cache over bf16 tensors k, v (CONTIGUOUS/RING: [B, cap, 4, 128]
-    or [cap, 4, 128]; PAGED: [num_blocks, 64, 4, 128] with an int32 table)."""
+             num_blocks: int = 0, k_scale: Optional[Sequence[float]] = None,
+             v_scale: Optional[Sequence[float]] = None) -> KVCache:
+    """A flint_kv_cache over tensors k, v (CONTIGUOUS/RING: [B, cap, 4, 128]
+    or [cap, 4, 128]; PAGED: [num_blocks, 64, 4, 128] with an int32 table):
+    bf16 tensors, or uint8 tensors of E4M3 codes with k_scale and v_scale
+    (4 floats each, one per KV head)."""
     c = KVCache()
+    if k.dtype == torch.uint8:
+        if k_scale is None or v_scale is None or len(k_scale) != 4 or len(v_scale) != 4:
+            raise FlintError(FLINT_ERR_INVALID_ARG, "an E4M3 cache needs 4 k_scale and 4 v_scale values")
+        c.dtype = KV_FP8_E4M3
+        c.k_scale[:] = [float(x) for x in k_scale]
+        c.v_scale[:] = [float(x) for x in v_scale]
+    elif k.dtype != torch.bfloat16:
+        raise FlintError(FLINT_ERR_INVALID_ARG, f"cache tensors must be bf16 or uint8, not {k.dtype}")
     c.k, c.v = k.data_ptr(), v.data_ptr()
     c.layout = int(layout)
     c.capacity = int(capacity)

@@ -84,14 +84,36 @@ class Layer:
     w_q: torch.Tensor                # bf16 [128]
     w_k: torch.Tensor                # bf16 [128]
     sinks: torch.Tensor              # f32 [32]
-    k_cache: torch.Tensor            # bf16 [capacity,4,128]
+    k_cache: torch.Tensor            # bf16 [capacity,4,128], or uint8 E4M3 codes
     v_cache: torch.Tensor
     layout: int                      # CONTIGUOUS or RING
     capacity: int
+    k_scale: Optional[List[float]] = None   # E4M3 cache: per KV head
+    v_scale: Optional[List[float]] = None
+
+
+# E4M3 (fp8) caches hold the same N(0, 1) history as the bf16 ones, divided by
+# a per-KV-head scale and cast to torch.float8_e4m3fn (torch's conversion,
+# nearest even, after a clamp to the largest code): the scales put |x| = 6 near
+# the top code 448.  Scales are drawn per (workload, layer, K/V).
+_T_KS, _T_VS = 8, 9
+
+
+def fp8_scales(seed: int) -> List[float]:
+    u = torch.rand(NUM_KV_HEADS, generator=_gen(seed), dtype=torch.float64)
+    return [float(6.0 / 448.0 * (0.9 + 0.2 * x)) for x in u]
+
+
+def to_e4m3_codes(x: torch.Tensor, scales: List[float]) -> torch.Tensor:
+    """uint8 E4M3 codes of x [..., 4, 128] / scales[kv head], via torch's cast."""
+    s = torch.tensor(scales, dtype=torch.float32).reshape(NUM_KV_HEADS, 1)
+    y = (x.to(torch.float32) / s).clamp(-448.0, 448.0)
+    return y.to(torch.float8_e4m3fn).view(torch.uint8)
 
 
 def make_layer(workload: int, layer: int, L: int, window: int, rope: bool,
-               ring: Optional[bool] = None, capacity: Optional[int] = None) -> Layer:
+               ring: Optional[bool] = None, capacity: Optional[int] = None,
+               fp8: bool = False) -> Layer:
     """A layer whose cache holds random history for positions < L-1.
 
     Window layers use a 513-slot ring unless ring=False; full layers use a
@@ -103,6 +125,12 @@ def make_layer(workload: int, layer: int, L: int, window: int, rope: bool,
     else:
         layout, cap = CONTIGUOUS, (capacity if capacity is not None else L)
     s = lambda t: seed_for(workload, layer, t)  # noqa: E731
+    k_cache = bf16_normal((cap, NUM_KV_HEADS, HEAD_DIM), s(_T_KC))
+    v_cache = bf16_normal((cap, NUM_KV_HEADS, HEAD_DIM), s(_T_VC))
+    k_scale = v_scale = None
+    if fp8:
+        k_scale, v_scale = fp8_scales(s(_T_KS)), fp8_scales(s(_T_VS))
+        k_cache, v_cache = to_e4m3_codes(k_cache, k_scale), to_e4m3_codes(v_cache, v_scale)
     return Layer(
         window=window, rope=rope, L=L,
         q_raw=bf16_normal((NUM_Q_HEADS, HEAD_DIM), s(_T_Q)),
@@ -111,9 +139,8 @@ def make_layer(workload: int, layer: int, L: int, window: int, rope: bool,
         w_q=bf16_normal((HEAD_DIM,), s(_T_WQ), 1.0, 0.1),
         w_k=bf16_normal((HEAD_DIM,), s(_T_WK), 1.0, 0.1),
         sinks=f32_normal((NUM_Q_HEADS,), s(_T_SINK)),
-        k_cache=bf16_normal((cap, NUM_KV_HEADS, HEAD_DIM), s(_T_KC)),
-        v_cache=bf16_normal((cap, NUM_KV_HEADS, HEAD_DIM), s(_T_VC)),
-        layout=layout, capacity=cap)
+        k_cache=k_cache, v_cache=v_cache,
+        layout=layout, capacity=cap, k_scale=k_scale, v_scale=v_scale)
 
 
 def layer_kinds(n_layers: int = N_LAYERS) -> List[bool]:
@@ -125,16 +152,16 @@ def layer_kinds(n_layers: int = N_LAYERS) -> List[bool]:
 
 
 def make_stack(L: int, n_layers: int = N_LAYERS, workload: int = W_STACK_100K,
-               full_capacity: Optional[int] = None) -> List[Layer]:
+               full_capacity: Optional[int] = None, fp8: bool = False) -> List[Layer]:
     """49-layer stack for one token at context L: window layers with RoPE on
-    513-slot rings, full NoPE layers on contiguous caches."""
+    513-slot rings, full NoPE layers on contiguous caches (E4M3 caches if fp8)."""
     out = []
     for i, full in enumerate(layer_kinds(n_layers)):
         if full:
             out.append(make_layer(workload, i, L, 0, False, ring=False,
-                                  capacity=full_capacity))
+                                  capacity=full_capacity, fp8=fp8))
         else:
-            out.append(make_layer(workload, i, L, WINDOW, True, ring=True))
+            out.append(make_layer(workload, i, L, WINDOW, True, ring=True, fp8=fp8))
     return out
 
 
@@ -142,21 +169,28 @@ def make_stack(L: int, n_layers: int = N_LAYERS, workload: int = W_STACK_100K,
 class DecodeInputs:
     """Already-normed q over a contiguous cache (no append)."""
     q: torch.Tensor          # bf16 [B,32,128]
-    k_cache: torch.Tensor    # bf16 [B,cap,4,128]
+    k_cache: torch.Tensor    # bf16 [B,cap,4,128], or uint8 E4M3 codes
     v_cache: torch.Tensor
     sinks: torch.Tensor      # f32 [32]
     seq_lens: List[int]
+    k_scale: Optional[List[float]] = None
+    v_scale: Optional[List[float]] = None
 
 
 def make_decode(L: int, workload: int = W_FULL_100K, B: int = 1,
-                capacity: Optional[int] = None) -> DecodeInputs:
+                capacity: Optional[int] = None, fp8: bool = False) -> DecodeInputs:
     cap = capacity if capacity is not None else L
+    k = bf16_normal((B, cap, NUM_KV_HEADS, HEAD_DIM), seed_for(workload, 0, _T_KC))
+    v = bf16_normal((B, cap, NUM_KV_HEADS, HEAD_DIM), seed_for(workload, 0, _T_VC))
+    ks = vs = None
+    if fp8:
+        ks, vs = fp8_scales(seed_for(workload, 0, _T_KS)), fp8_scales(seed_for(workload, 0, _T_VS))
+        k, v = to_e4m3_codes(k, ks), to_e4m3_codes(v, vs)
     return DecodeInputs(
         q=bf16_normal((B, NUM_Q_HEADS, HEAD_DIM), seed_for(workload, 0, _T_Q)),
-        k_cache=bf16_normal((B, cap, NUM_KV_HEADS, HEAD_DIM), seed_for(workload, 0, _T_KC)),
-        v_cache=bf16_normal((B, cap, NUM_KV_HEADS, HEAD_DIM), seed_for(workload, 0, _T_VC)),
+        k_cache=k, v_cache=v,
         sinks=f32_normal((NUM_Q_HEADS,), seed_for(workload, 0, _T_SINK)),
-        seq_lens=[L] * B)
+        seq_lens=[L] * B, k_scale=ks, v_scale=vs)
 
 
 @dataclasses.dataclass
@@ -167,6 +201,8 @@ class PagedBatch:
     block_table: torch.Tensor  # int32 [B,max_blocks]
     seq_lens: List[int]
     sinks: torch.Tensor        # f32 [32] (shared by all requests)
+    k_scale: Optional[List[float]] = None   # E4M3 pools
+    v_scale: Optional[List[float]] = None
 
 
 def log_uniform_lengths(B: int, lo: int, hi: int, seed: int) -> List[int]:
@@ -178,7 +214,7 @@ def log_uniform_lengths(B: int, lo: int, hi: int, seed: int) -> List[int]:
 
 def make_paged_batch(B: int = 32, lo: int = 4096, hi: int = 131072,
                      workload: int = W_PAGED_BATCH, spare_blocks: int = 0,
-                     seq_lens: Optional[List[int]] = None) -> PagedBatch:
+                     seq_lens: Optional[List[int]] = None, fp8: bool = False) -> PagedBatch:
     """Requests with log-uniform lengths in [lo, hi]; each request's blocks are
     drawn from one randomly permuted pool (block ids shuffled)."""
     if seq_lens is None:
@@ -193,11 +229,14 @@ def make_paged_batch(B: int = 32, lo: int = 4096, hi: int = 131072,
     for b, n in enumerate(nblk):
         table[b, :n] = perm[k:k + n].to(torch.int32)
         k += n
+    k = bf16_normal((num_blocks, BLOCK_SIZE, NUM_KV_HEADS, HEAD_DIM), seed_for(workload, 0, _T_KC))
+    v = bf16_normal((num_blocks, BLOCK_SIZE, NUM_KV_HEADS, HEAD_DIM), seed_for(workload, 0, _T_VC))
+    ks = vs = None
+    if fp8:
+        ks, vs = fp8_scales(seed_for(workload, 0, _T_KS)), fp8_scales(seed_for(workload, 0, _T_VS))
+        k, v = to_e4m3_codes(k, ks), to_e4m3_codes(v, vs)
     return PagedBatch(
         q=bf16_normal((B, NUM_Q_HEADS, HEAD_DIM), seed_for(workload, 0, _T_Q)),
-        k_pool=bf16_normal((num_blocks, BLOCK_SIZE, NUM_KV_HEADS, HEAD_DIM),
-                           seed_for(workload, 0, _T_KC)),
-        v_pool=bf16_normal((num_blocks, BLOCK_SIZE, NUM_KV_HEADS, HEAD_DIM),
-                           seed_for(workload, 0, _T_VC)),
-        block_table=table, seq_lens=list(seq_lens),
-        sinks=f32_normal((NUM_Q_HEADS,), seed_for(workload, 0, _T_SINK)))
+        k_pool=k, v_pool=v, block_table=table, seq_lens=list(seq_lens),
+        sinks=f32_normal((NUM_Q_HEADS,), seed_for(workload, 0, _T_SINK)),
+        k_scale=ks, v_scale=vs)

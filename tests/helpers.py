@@ -38,9 +38,28 @@ def bf16_ulp_diff(a_bits: np.ndarray, b_bits: np.ndarray) -> np.ndarray:
     return np.abs(ordered(a_bits) - ordered(b_bits))
 
 
+def e4m3_code_distance(a: np.ndarray, b: np.ndarray) -> np.ndarray:
+    """Distance between E4M3 codes in steps of the format (+0 and -0 coincide)."""
+    def ordered(x):
+        x = x.astype(np.int32)
+        return np.where(x & 0x80, -(x & 0x7F), x & 0x7F)
+    return np.abs(ordered(a) - ordered(b))
+
+
 def oracle_layer(layer: I.Layer, nthreads: int = 0):
     """Oracle for one synthetic layer: norm (+RoPE) -> append -> attend.
-    Returns (out f64 [32,128], k cache bits, v cache bits) after the append."""
+    Returns (out f64 [32,128], k cache, v cache) after the append: bf16 bits,
+    or uint8 codes for an E4M3 layer."""
+    if layer.k_scale is not None:
+        kc = layer.k_cache.numpy().copy()
+        vc = layer.v_cache.numpy().copy()
+        out = oracle.decode_layer_fp8(I.bits(layer.q_raw), I.bits(layer.k_raw), I.bits(layer.v_raw),
+                                      I.bits(layer.w_q), I.bits(layer.w_k),
+                                      layer.sinks.numpy().astype(np.float64), kc, vc,
+                                      layer.k_scale, layer.v_scale, layer.L, layer.window,
+                                      layer.rope, layout=layer.layout, capacity=layer.capacity,
+                                      nthreads=nthreads)
+        return out, kc, vc
     kc = I.bits(layer.k_cache).copy()
     vc = I.bits(layer.v_cache).copy()
     out = oracle.decode_layer(I.bits(layer.q_raw), I.bits(layer.k_raw), I.bits(layer.v_raw),
@@ -67,7 +86,8 @@ class DeviceLayer:
         self.window = layer.window
         self.rope = layer.rope
         self.cache = flint.kv_cache(self.k_cache, self.v_cache, layer.layout,
-                                    capacity=layer.capacity)
+                                    capacity=layer.capacity, k_scale=layer.k_scale,
+                                    v_scale=layer.v_scale)
 
 
 def stack_on_gpu(layers, pos, num_ctas=0):
