@@ -492,28 +492,29 @@ __device__ __forceinline__ void consume_slice(uint32_t sK, uint32_t sV, int tok0
   }
 }
 
-// consume_slice for an E4M3 cache.  sK / sV point at row r0 of the head's K /
-// V boxes (kTileFp8 rows of 128 one-byte dims, 128-byte swizzle, r0 a
-// multiple of 8).  ldmatrix gives thread (g, c) 4 consecutive bytes of a row:
-// dims 16u + 4c .. 16u + 4c + 3, widened to f16.
-//   * QK: those bytes are the B fragment of K^T for the logical k order in
-//     which q was loaded (dims d0 = 4c, d2 = 4c + 2); the scores are then
-//     multiplied by the head's k scale.
-//   * PV: the widened V rows form two 8x8 f16 matrices per 16-dim chunk (dims
-//     16u + {0,1,4,5,8,9,12,13} and 16u + {2,3,6,7,10,11,14,15}); their
-//     transposes (movmatrix) are the B fragments of V for 8 tokens each, and
-//     O n-tile 2u + h holds dims 16u + 4c + 2h + {0, 1} in thread (g, c).
+// The E4M3 counterpart of consume_slice, for a 32-token block (one softmax
+// step for the block).  sK / sV point at row r0 of the head's K / V boxes
+// (kTileFp8 rows of 128 one-byte dims, 128-byte swizzle, r0 a multiple of 8).
+//   * QK: ldmatrix gives thread (g, c) 4 consecutive bytes of a row (dims
+//     16u + 4c .. 16u + 4c + 3), widened to f16: the B fragment of K^T for
+//     the logical k order q was loaded in (d0 = 4c, d2 = 4c + 2).  Scores
+//     are then multiplied by the head's k scale.
+//   * PV: ldmatrix.trans on byte pairs gives a thread tokens 2c, 2c + 1 of
+//     dims 2p, 2p + 1 (p = g) of a 16-dim chunk; one byte permute splits them
+//     into the B fragments of the chunk's even-dim and odd-dim n-tiles.  O
+//     n-tile 2u holds dims 16u + 4c + {0, 2} and n-tile 2u + 1 dims
+//     16u + 4c + {1, 3} of thread (g, c) (see fp8_o_to_values).
 // The caller multiplies O by the head's v scale at the item's end.
-__device__ __forceinline__ void consume_slice_fp8(uint32_t sK, uint32_t sV, int tok0, int lo, int hi,
-                                                  int lane, const uint32_t (&qa)[8][4], float k_scale,
-                                                  float& m_run, float& l_run, float (&o)[16][4]) {
+__device__ __forceinline__ void consume_block32_fp8(uint32_t sK, uint32_t sV, int tok0, int lo, int hi,
+                                                    int lane, const uint32_t (&qa)[8][4], float k_scale,
+                                                    float& m_run, float& l_run, float (&o)[16][4]) {
   const int c = lane & 3;
   const int l7 = lane & 7;
-  const bool whole = (tok0 >= lo) && (tok0 + kSlice <= hi);
+  const bool whole = (tok0 >= lo) && (tok0 + 32 <= hi);
 
-  float sc[4];
+  float sc[8];
 #pragma unroll
-  for (int jj = 0; jj < 2; ++jj) {
+  for (int jj = 0; jj < 4; ++jj) {
     float a0[4] = {0.f, 0.f, 0.f, 0.f}, a1[4] = {0.f, 0.f, 0.f, 0.f};
     const uint32_t row = sK + (8 * jj + l7) * 128;
 #pragma unroll
@@ -535,13 +536,15 @@ __device__ __forceinline__ void consume_slice_fp8(uint32_t sK, uint32_t sV, int 
   }
   if (!whole) {
 #pragma unroll
-    for (int i = 0; i < 4; ++i) {
+    for (int i = 0; i < 8; ++i) {
       const int tok = tok0 + 8 * (i >> 1) + 2 * c + (i & 1);
       if (tok < lo || tok >= hi) sc[i] = -INFINITY;
     }
   }
 
-  float mx = fmaxf(fmaxf(sc[0], sc[1]), fmaxf(sc[2], sc[3]));
+  float mx = sc[0];
+#pragma unroll
+  for (int i = 1; i < 8; ++i) mx = fmaxf(mx, sc[i]);
   mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 1));
   mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 2));
   const bool grow = mx > m_run + kRescaleSlack;
@@ -556,45 +559,59 @@ __device__ __forceinline__ void consume_slice_fp8(uint32_t sK, uint32_t sV, int 
   }
   const float mu = (m_run == -INFINITY) ? 0.f : m_run;
 
-  const float p0 = exp2f(sc[0] - mu), p1 = exp2f(sc[1] - mu);
-  const float p2 = exp2f(sc[2] - mu), p3 = exp2f(sc[3] - mu);
-  l_run += (p0 + p1) + (p2 + p3);
-  uint32_t pa[4];
-  split_f16x2(p0, p1, pa[0], pa[1]);
-  split_f16x2(p2, p3, pa[2], pa[3]);
-
-  uint32_t m01 = 0xffffffffu, m23 = 0xffffffffu;
-  if (!whole) {
-    const int t = tok0 + 2 * c;
-    m01 = ((t >= lo && t < hi) ? 0x0000ffffu : 0u) | ((t + 1 >= lo && t + 1 < hi) ? 0xffff0000u : 0u);
-    m23 = ((t + 8 >= lo && t + 8 < hi) ? 0x0000ffffu : 0u) |
-          ((t + 9 >= lo && t + 9 < hi) ? 0xffff0000u : 0u);
+  float p[8];
+#pragma unroll
+  for (int i = 0; i < 8; ++i) p[i] = exp2f(sc[i] - mu);
+  l_run += ((p[0] + p[1]) + (p[2] + p[3])) + ((p[4] + p[5]) + (p[6] + p[7]));
+  uint32_t pa[2][4];  // k-steps of 16 tokens
+#pragma unroll
+  for (int s2 = 0; s2 < 2; ++s2) {
+    split_f16x2(p[4 * s2], p[4 * s2 + 1], pa[s2][0], pa[s2][1]);
+    split_f16x2(p[4 * s2 + 2], p[4 * s2 + 3], pa[s2][2], pa[s2][3]);
   }
-  // lanes 8i..8i+7 address tokens 8(i & 1) + l7 of chunk u = up + (i >> 1)
-  const uint32_t row = sV + (((lane >> 3) & 1) * 8 + l7) * 128;
+
+  // masks of a thread's token pairs (2c, 2c + 1) + 8 i, i = 0..3
+  uint32_t msk[4] = {0xffffffffu, 0xffffffffu, 0xffffffffu, 0xffffffffu};
+  if (!whole) {
 #pragma unroll
-  for (int up = 0; up < 8; up += 2) {
-    const int u = up + (lane >> 4);
-    uint32_t x[4];
-    ldsm_x4(row + ((u ^ l7) << 4), x[0], x[1], x[2], x[3]);
-#pragma unroll
-    for (int half = 0; half < 2; ++half) {  // chunk up + half: x[2 half] tokens 0-7, x[2 half + 1] tokens 8-15
-      const uint32_t t0 = x[2 * half], t1 = x[2 * half + 1];
-      uint32_t v0 = movmatrix_trans(e4m3x2_to_f16x2(t0));          // dims 4c, 4c+1 of 8 tokens
-      uint32_t v1 = movmatrix_trans(e4m3x2_to_f16x2(t1));
-      uint32_t v2 = movmatrix_trans(e4m3x2_to_f16x2(t0 >> 16));    // dims 4c+2, 4c+3
-      uint32_t v3 = movmatrix_trans(e4m3x2_to_f16x2(t1 >> 16));
-      if (!whole) {  // rows outside the range may hold anything (even NaN codes)
-        v0 &= m01;
-        v2 &= m01;
-        v1 &= m23;
-        v3 &= m23;
-      }
-      const int nt = 2 * (up + half);
-      mma_f16_16816(o[nt], pa, v0, v1);
-      mma_f16_16816(o[nt + 1], pa, v2, v3);
+    for (int i = 0; i < 4; ++i) {
+      const int t = tok0 + 8 * i + 2 * c;
+      msk[i] = ((t >= lo && t < hi) ? 0x0000ffffu : 0u) | ((t + 1 >= lo && t + 1 < hi) ? 0xffff0000u : 0u);
     }
   }
+  // lanes 8i..8i+7 address tokens 8i + l7 of the chunk (all four 8-token groups)
+  const uint32_t row = sV + (8 * (lane >> 3) + l7) * 128;
+#pragma unroll
+  for (int u = 0; u < 8; ++u) {
+    uint32_t x[4];
+    ldsm_x4_t(row + ((u ^ l7) << 4), x[0], x[1], x[2], x[3]);
+    uint32_t ev[4], od[4];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      // x[i]: bytes (t 2c: d 2g, d 2g+1), (t 2c+1: d 2g, d 2g+1) of token group i
+      const uint32_t y = __byte_perm(x[i], 0u, 0x3120);  // (t2c d2g, t2c+1 d2g, t2c d2g+1, t2c+1 d2g+1)
+      ev[i] = e4m3x2_to_f16x2(y) & msk[i];              // dim 2g of tokens 2c, 2c+1
+      od[i] = e4m3x2_to_f16x2(y >> 16) & msk[i];        // dim 2g+1
+    }
+#pragma unroll
+    for (int s2 = 0; s2 < 2; ++s2) {
+      mma_f16_16816(o[2 * u], pa[s2], ev[2 * s2], ev[2 * s2 + 1]);
+      mma_f16_16816(o[2 * u + 1], pa[s2], od[2 * s2], od[2 * s2 + 1]);
+    }
+  }
+}
+
+// The 32 O values of thread (g, c) in the order of the dim map (values 4q..4q+3
+// = dims 16q + 4c + 0..3), from consume_block32_fp8's accumulators, rows g
+// (P hi) and g + 8 (P lo) summed.
+__device__ __forceinline__ void fp8_o_to_values(const float (&o)[16][4], float scale, float (&v)[32]) {
+#pragma unroll
+  for (int q = 0; q < 8; ++q)
+#pragma unroll
+    for (int e = 0; e < 2; ++e) {
+      v[4 * q + 2 * e] = (o[2 * q][e] + o[2 * q][e + 2]) * scale;          // even n-tile: dim 4c + 2e
+      v[4 * q + 2 * e + 1] = (o[2 * q + 1][e] + o[2 * q + 1][e + 2]) * scale;  // odd: 4c + 2e + 1
+    }
 }
 
 // Float4 slot of values 4q..4q+3 of consumer thread (head, c)'s 32 O values
@@ -728,14 +745,11 @@ __device__ void run_consumer(const DecodeParams& P, const Smem& S, int warp, int
         consume_slice(base + box_offset(0, kvh, 0) + r0 * 128, base + box_offset(1, kvh, 0) + r0 * 128,
                       tok0, pb.lo, pb.hi, lane, qa, m_run, l_run, o);
       } else {
-        // 64-token E4M3 tile: group q takes tokens 32q .. 32q + 31, two slices
-#pragma unroll 1
-        for (int sl = 0; sl < kTileFp8 / (kConsumerGroups * kSlice); ++sl) {
-          const int r0 = (group * (kTileFp8 / kConsumerGroups)) + sl * kSlice;
-          const int tok0 = pb.tile_base + (item.t0 + k) * kTileFp8 + r0;
-          consume_slice_fp8(base + box_offset_fp8(0, kvh) + r0 * 128, base + box_offset_fp8(1, kvh) + r0 * 128,
+        // 64-token E4M3 tile: group q takes tokens 32q .. 32q + 31 as one block
+        const int r0 = group * (kTileFp8 / kConsumerGroups);
+        const int tok0 = pb.tile_base + (item.t0 + k) * kTileFp8 + r0;
+        consume_block32_fp8(base + box_offset_fp8(0, kvh) + r0 * 128, base + box_offset_fp8(1, kvh) + r0 * 128,
                             tok0, pb.lo, pb.hi, lane, qa, k_scale, m_run, l_run, o);
-        }
       }
       __syncwarp();
       if (lane == 0) mbar_arrive(smem_u32(&S.empty[stage]));
@@ -745,11 +759,14 @@ __device__ void run_consumer(const DecodeParams& P, const Smem& S, int warp, int
     l_run += __shfl_xor_sync(0xffffffffu, l_run, 1);
     l_run += __shfl_xor_sync(0xffffffffu, l_run, 2);
     float v[32];
-    const float o_scale = pb.fp8 ? v_scale : 1.0f;  // E4M3: V was read as codes
+    if (pb.fp8) {
+      fp8_o_to_values(o, v_scale, v);  // E4M3: V was read as codes
+    } else {
 #pragma unroll
-    for (int n = 0; n < 16; ++n) {
-      v[2 * n] = (o[n][0] + o[n][2]) * o_scale;
-      v[2 * n + 1] = (o[n][1] + o[n][3]) * o_scale;
+      for (int n = 0; n < 16; ++n) {
+        v[2 * n] = o[n][0] + o[n][2];
+        v[2 * n + 1] = o[n][1] + o[n][3];
+      }
     }
     if (kConsumerGroups > 1) {
       // the other groups hand their states to group 0, which merges them
