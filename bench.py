@@ -82,7 +82,7 @@ def parse():
     ap.add_argument("--warmup", type=int, default=20)
     ap.add_argument("--impl", default="flint", choices=["flint", "reference"])
     ap.add_argument("--workload", default="stack",
-                    choices=["stack", "full100k", "full2k", "swa100k", "paged32", "paged32swa"])
+                    choices=["stack", "serial", "full100k", "full2k", "swa100k", "paged32", "paged32swa"])
     ap.add_argument("--context", type=int, default=100_000,
                     help="context length (the benchmark's figure is 100,000; smaller ones serve profiling)")
     ap.add_argument("--kv", default="bf16", choices=["bf16", "fp8"],
@@ -191,6 +191,10 @@ def workload_config(name):
     if name == "stack":
         return dict(base, workload="49-layer decode-attention stack for one token: 35 sliding-window "
                     "(513, RoPE) + 14 full-context NoPE layers, GQA 32q/4kv x 128, sinks",
+                    context=CONTEXT, layers=49, kv_layout="ring(513) + contiguous")
+    if name == "serial":
+        return dict(base, workload="the same 49 layers as 49 serially dependent launches "
+                    "(programmatic dependent launch), one layer each",
                     context=CONTEXT, layers=49, kv_layout="ring(513) + contiguous")
     if name in ("full100k", "full2k"):
         return dict(base, workload="one full-context NoPE decode layer, q given (flint_attn_decode)",
@@ -313,7 +317,7 @@ def main():
     fp8 = args.kv == "fp8"
     eb = 1 if fp8 else 2                       # bytes per cached value
     tok_bytes = 2 * 4 * 128 * eb               # K and V of one token of one layer
-    if args.workload == "stack":
+    if args.workload in ("stack", "serial"):
         layers = I.make_stack(ctx, fp8=fp8)
         algo_bytes = flint.flint_kv_bytes(ctx, elem_bytes=eb)
     elif args.workload == "swa100k":
@@ -379,8 +383,12 @@ def main():
         ws = flint.workspace(len(dls))
         arr = flint.stack_layers(dls)
 
-        def step():
-            flint.flint_attn_stack(arr, pos, out, ws, dev_err=err)
+        if args.workload == "serial":
+            def step():
+                flint.flint_attn_layers_serial(arr, pos, out, ws, dev_err=err)
+        else:
+            def step():
+                flint.flint_attn_stack(arr, pos, out, ws, dev_err=err)
         h2d = host_in.numel() * host_in.element_size()
     else:
         q, k, v, sinks = dec["q"].cuda(), dec["k"].cuda(), dec["v"].cuda(), dec["sinks"].cuda()
@@ -481,9 +489,11 @@ def main():
     peak, peak_kind = measured_peak()
     achieved = algo_bytes / (ms * 1e-3) / 1e9
     line = {
-        "metric": METRIC if args.workload == "stack" else f"{args.workload} decode-attention us/step",
+        "metric": (METRIC if args.workload == "stack" else
+                   "49-layer decode-attention µs/token @100K ctx bs=1, as 49 dependent launches"
+                   if args.workload == "serial" else f"{args.workload} decode-attention us/step"),
         "value": per_token_us(ms, world),
-        "unit": "us/token" if args.workload == "stack" else "us/step",
+        "unit": "us/token" if args.workload in ("stack", "serial") else "us/step",
         "n_gpus": world, "steps": args.steps, "warmup": max(args.warmup, 3),
         "ms_per_step": ms, "higher_is_better": False, "scaling": "weak", "vs_baseline": None,
         "dtype": "fp8-e4m3 KV, f16 mma" if fp8 else "bf16",
@@ -501,7 +511,7 @@ def main():
                      "traffic": None if fp8 else traffic_for(args.workload, ctx)},
         "cpu_baseline": cpu_baseline,
         "e2e": e2e,
-        "gpu_launches": args.steps,
+        "gpu_launches": args.steps * (49 if args.workload == "serial" else 1),
         "host_us_per_call": host_us,
         "clocks": clocks.summary(),
         "per_step_us": {"min": min(per_step_ms) * 1000.0, "median": statistics.median(per_step_ms) * 1000.0,

@@ -214,6 +214,23 @@ flint_status flint_attn_stack(const flint_layer* layers, int32_t n_layers, int32
                               size_t ws_bytes, int32_t num_ctas, int32_t* dev_err,
                               void* stream);
 
+/* The same n_layers layers of one token as flint_attn_stack, run as n_layers
+ * serially dependent launches, one layer each, as a model whose layers feed
+ * one another must run them.  Each launch after the first is a programmatic
+ * dependent of the one before (CUDA programmatic dependent launch): its launch
+ * and on-chip set-up overlap the previous layer's tail, and it waits for the
+ * previous launch to complete before it touches any memory.  The layers here
+ * are independent problems (the synthetic dependence is the ordering), so the
+ * outputs equal flint_attn_stack's up to rounding order.  No counterpart
+ * kernel in the pages: their serving path launches per-layer kernels ("Day-0
+ * Support for Flint on vLLM", newruntime.com, "What happened": the kernel
+ * count per forward step).  Arguments, workspace and errors as
+ * flint_attn_stack; the workspace is reused by every layer in turn. */
+flint_status flint_attn_layers_serial(const flint_layer* layers, int32_t n_layers,
+                                      int32_t pos, float eps, double theta, float* out,
+                                      void* workspace, size_t ws_bytes, int32_t num_ctas,
+                                      int32_t* dev_err, void* stream);
+
 /* flint_attn_stack without a workspace argument, for callers that cannot
  * allocate device memory (a runtime that owns all of it through its own pool,
  * a plug-in handed buffers but no allocator).  No counterpart in the paper: it

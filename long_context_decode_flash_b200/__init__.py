@@ -8,7 +8,7 @@ _BINDING_NAMES = (
     "FlintError", "load_library", "flint_status_string", "flint_last_error",
     "flint_kv_bytes", "flint_qk_norm_rope", "flint_kv_append",
     "flint_attn_workspace_bytes", "flint_attn_decode", "flint_attn_stack",
-    "flint_attn_stack_noalloc",
+    "flint_attn_stack_noalloc", "flint_attn_layers_serial",
     "flint_plan_items", "flint_plan_split", "KVCache", "StackLayer",
 )
 

@@ -336,6 +336,93 @@ flint_status launch_result(cudaError_t e, const char* who) {
 
 }  // namespace
 
+namespace {
+
+flint_status run_stack(const flint_layer* layers, int32_t n_layers, int32_t pos, float eps, double theta,
+                       float* out, void* workspace, size_t ws_bytes, int32_t num_ctas, int32_t* dev_err,
+                       void* stream, int pdl, const char* who) {
+  if (!layers || !out || !workspace) return fail(FLINT_ERR_INVALID_ARG, "%s: NULL pointer argument", who);
+  if (n_layers < 1 || n_layers > FLINT_MAX_LAYERS)
+    return fail(FLINT_ERR_INVALID_ARG, "%s: n_layers=%d outside [1, %d]", who, n_layers, FLINT_MAX_LAYERS);
+  if (pos < 0 || pos >= FLINT_MAX_CONTEXT) return fail(FLINT_ERR_INVALID_ARG, "%s: pos=%d outside [0, %d)", who, pos, FLINT_MAX_CONTEXT);
+  if (!(eps >= 0.f) || !(theta > 0.0)) return fail(FLINT_ERR_INVALID_ARG, "%s: eps must be >= 0, theta > 0", who);
+  if (num_ctas < 0 || num_ctas > kMaxCtas) return fail(FLINT_ERR_INVALID_ARG, "%s: num_ctas %d outside [0, %d]", who, num_ctas, kMaxCtas);
+  if (!aligned16(out) || !aligned16(workspace)) return fail(FLINT_ERR_INVALID_ARG, "%s: out/workspace must be 16-byte aligned", who);
+  const int L = pos + 1;
+  int tiles[kMaxProblems];
+  static thread_local DecodeParams P;
+  memset(&P, 0, sizeof P);
+  for (int i = 0; i < n_layers; ++i) {
+    const flint_layer& ly = layers[i];
+    if (!ly.q_raw || !ly.k_raw || !ly.v_raw || !ly.w_q || !ly.w_k || !ly.sinks)
+      return fail(FLINT_ERR_INVALID_ARG, "%s: layer %d has a NULL pointer", who, i);
+    const void* ptrs[] = {ly.q_raw, ly.k_raw, ly.v_raw, ly.w_q, ly.w_k};
+    for (const void* p : ptrs)
+      if (!aligned16(p)) return fail(FLINT_ERR_INVALID_ARG, "%s: layer %d pointers must be 16-byte aligned", who, i);
+    if (ly.window != 0 && ly.window != kWindow)
+      return fail(FLINT_ERR_UNSUPPORTED, "%s: layer %d window must be 0 or %d", who, i, kWindow);
+    if (ly.rope != 0 && ly.rope != 1) return fail(FLINT_ERR_INVALID_ARG, "%s: layer %d rope must be 0 or 1", who, i);
+    flint_status s = check_cache(&ly.cache, 1, who);
+    if (s != FLINT_OK) return s;
+    s = check_len(ly.cache, L, ly.window, who, i);
+    if (s != FLINT_OK) return s;
+    const Range r = attended_range(ly.cache, L, ly.window);
+    Problem& pb = P.prob[i];
+    pb.q = ly.q_raw;
+    pb.k_raw = ly.k_raw;
+    pb.v_raw = ly.v_raw;
+    pb.w_q = ly.w_q;
+    pb.w_k = ly.w_k;
+    pb.sinks = ly.sinks;
+    pb.out = out + static_cast<size_t>(i) * kHeads * kDim;
+    pb.k_rows = static_cast<uint16_t*>(ly.cache.k);
+    pb.v_rows = static_cast<uint16_t*>(ly.cache.v);
+    pb.table = ly.cache.layout == FLINT_KV_PAGED ? ly.cache.block_table : nullptr;
+    pb.lo = r.lo;
+    pb.hi = r.hi;
+    pb.tile_base = r.tile_base;
+    pb.pos = pos;
+    pb.append_tok = ly.cache.layout == FLINT_KV_RING ? pos % ly.cache.capacity : pos;
+    pb.num_blocks = ly.cache.num_blocks;
+    pb.ext2 = ly.cache.layout == FLINT_KV_PAGED ? kBlock : ly.cache.capacity;
+    pb.ext3 = ly.cache.layout == FLINT_KV_PAGED ? ly.cache.num_blocks : 1;
+    pb.table_len = ly.cache.layout == FLINT_KV_PAGED ? ly.cache.max_blocks_per_req : 0;
+    pb.map_k = static_cast<int16_t>(2 * i);
+    pb.map_v = static_cast<int16_t>(2 * i + 1);
+    pb.req = 0;
+    pb.layout = static_cast<int8_t>(ly.cache.layout);
+    pb.q_fp32 = 0;
+    pb.rope = static_cast<int8_t>(ly.rope);
+    pb.fp8 = static_cast<int8_t>(ly.cache.dtype == FLINT_KV_FP8_E4M3);
+    set_scales(P, i, ly.cache);
+    tiles[i] = r.tiles;
+    s = encode_cache_map(&P.maps[2 * i], ly.cache.k, ly.cache, 1);
+    if (s != FLINT_OK) return s;
+    s = encode_cache_map(&P.maps[2 * i + 1], ly.cache.v, ly.cache, 1);
+    if (s != FLINT_OK) return s;
+  }
+  int grid = 0;
+  flint_status s = plan(P, tiles, n_layers, num_ctas, ws_bytes, who, &grid);
+  if (s != FLINT_OK) return s;
+  P.smem_bytes = static_cast<int32_t>(decode_smem_bytes());
+  P.counters = static_cast<int32_t*>(workspace);
+  P.partials = reinterpret_cast<float*>(static_cast<uint8_t*>(workspace) + kCounterBytes);
+  P.dev_err = dev_err;
+  P.n_problems = n_layers;
+  P.prep = 1;
+  P.pdl = pdl;
+  P.eps = eps;
+  // RoPE angles of the new token, pos * theta^(-2i/128) for i < 64, in double
+  // on the host (one position for every layer of the call)
+  for (int i = 0; i < kDim / 2; ++i) {
+    const double a = static_cast<double>(pos) * std::pow(theta, -2.0 * i / kDim);
+    P.rope_cs[i] = make_float2(static_cast<float>(std::cos(a)), static_cast<float>(std::sin(a)));
+  }
+  return launch_result(launch_decode(P, grid, static_cast<cudaStream_t>(stream)), who);
+}
+
+}  // namespace
+
 namespace flint {
 
 size_t workspace_min_bytes(int n_problems, int num_ctas) {
@@ -551,84 +638,26 @@ flint_status flint_attn_decode(const void* q, int32_t q_is_fp32, const flint_kv_
 flint_status flint_attn_stack(const flint_layer* layers, int32_t n_layers, int32_t pos, float eps,
                               double theta, float* out, void* workspace, size_t ws_bytes,
                               int32_t num_ctas, int32_t* dev_err, void* stream) {
-  const char* who = "flint_attn_stack";
-  if (!layers || !out || !workspace) return fail(FLINT_ERR_INVALID_ARG, "%s: NULL pointer argument", who);
+  return run_stack(layers, n_layers, pos, eps, theta, out, workspace, ws_bytes, num_ctas, dev_err, stream, 0,
+                   "flint_attn_stack");
+}
+
+flint_status flint_attn_layers_serial(const flint_layer* layers, int32_t n_layers, int32_t pos, float eps,
+                                      double theta, float* out, void* workspace, size_t ws_bytes,
+                                      int32_t num_ctas, int32_t* dev_err, void* stream) {
+  const char* who = "flint_attn_layers_serial";
+  if (!layers || !out) return fail(FLINT_ERR_INVALID_ARG, "%s: NULL pointer argument", who);
   if (n_layers < 1 || n_layers > FLINT_MAX_LAYERS)
     return fail(FLINT_ERR_INVALID_ARG, "%s: n_layers=%d outside [1, %d]", who, n_layers, FLINT_MAX_LAYERS);
-  if (pos < 0 || pos >= FLINT_MAX_CONTEXT) return fail(FLINT_ERR_INVALID_ARG, "%s: pos=%d outside [0, %d)", who, pos, FLINT_MAX_CONTEXT);
-  if (!(eps >= 0.f) || !(theta > 0.0)) return fail(FLINT_ERR_INVALID_ARG, "%s: eps must be >= 0, theta > 0", who);
-  if (num_ctas < 0 || num_ctas > kMaxCtas) return fail(FLINT_ERR_INVALID_ARG, "%s: num_ctas %d outside [0, %d]", who, num_ctas, kMaxCtas);
-  if (!aligned16(out) || !aligned16(workspace)) return fail(FLINT_ERR_INVALID_ARG, "%s: out/workspace must be 16-byte aligned", who);
-  const int L = pos + 1;
-  int tiles[kMaxProblems];
-  static thread_local DecodeParams P;
-  memset(&P, 0, sizeof P);
+  // One launch per layer, each after the first a programmatic dependent of
+  // the one before: it waits for that launch to complete before it touches
+  // memory, while its launch and set-up overlap the previous layer.
   for (int i = 0; i < n_layers; ++i) {
-    const flint_layer& ly = layers[i];
-    if (!ly.q_raw || !ly.k_raw || !ly.v_raw || !ly.w_q || !ly.w_k || !ly.sinks)
-      return fail(FLINT_ERR_INVALID_ARG, "%s: layer %d has a NULL pointer", who, i);
-    const void* ptrs[] = {ly.q_raw, ly.k_raw, ly.v_raw, ly.w_q, ly.w_k};
-    for (const void* p : ptrs)
-      if (!aligned16(p)) return fail(FLINT_ERR_INVALID_ARG, "%s: layer %d pointers must be 16-byte aligned", who, i);
-    if (ly.window != 0 && ly.window != kWindow)
-      return fail(FLINT_ERR_UNSUPPORTED, "%s: layer %d window must be 0 or %d", who, i, kWindow);
-    if (ly.rope != 0 && ly.rope != 1) return fail(FLINT_ERR_INVALID_ARG, "%s: layer %d rope must be 0 or 1", who, i);
-    flint_status s = check_cache(&ly.cache, 1, who);
-    if (s != FLINT_OK) return s;
-    s = check_len(ly.cache, L, ly.window, who, i);
-    if (s != FLINT_OK) return s;
-    const Range r = attended_range(ly.cache, L, ly.window);
-    Problem& pb = P.prob[i];
-    pb.q = ly.q_raw;
-    pb.k_raw = ly.k_raw;
-    pb.v_raw = ly.v_raw;
-    pb.w_q = ly.w_q;
-    pb.w_k = ly.w_k;
-    pb.sinks = ly.sinks;
-    pb.out = out + static_cast<size_t>(i) * kHeads * kDim;
-    pb.k_rows = static_cast<uint16_t*>(ly.cache.k);
-    pb.v_rows = static_cast<uint16_t*>(ly.cache.v);
-    pb.table = ly.cache.layout == FLINT_KV_PAGED ? ly.cache.block_table : nullptr;
-    pb.lo = r.lo;
-    pb.hi = r.hi;
-    pb.tile_base = r.tile_base;
-    pb.pos = pos;
-    pb.append_tok = ly.cache.layout == FLINT_KV_RING ? pos % ly.cache.capacity : pos;
-    pb.num_blocks = ly.cache.num_blocks;
-    pb.ext2 = ly.cache.layout == FLINT_KV_PAGED ? kBlock : ly.cache.capacity;
-    pb.ext3 = ly.cache.layout == FLINT_KV_PAGED ? ly.cache.num_blocks : 1;
-    pb.table_len = ly.cache.layout == FLINT_KV_PAGED ? ly.cache.max_blocks_per_req : 0;
-    pb.map_k = static_cast<int16_t>(2 * i);
-    pb.map_v = static_cast<int16_t>(2 * i + 1);
-    pb.req = 0;
-    pb.layout = static_cast<int8_t>(ly.cache.layout);
-    pb.q_fp32 = 0;
-    pb.rope = static_cast<int8_t>(ly.rope);
-    pb.fp8 = static_cast<int8_t>(ly.cache.dtype == FLINT_KV_FP8_E4M3);
-    set_scales(P, i, ly.cache);
-    tiles[i] = r.tiles;
-    s = encode_cache_map(&P.maps[2 * i], ly.cache.k, ly.cache, 1);
-    if (s != FLINT_OK) return s;
-    s = encode_cache_map(&P.maps[2 * i + 1], ly.cache.v, ly.cache, 1);
+    flint_status s = run_stack(layers + i, 1, pos, eps, theta, out + static_cast<size_t>(i) * kHeads * kDim,
+                               workspace, ws_bytes, num_ctas, dev_err, stream, i > 0 ? 1 : 0, who);
     if (s != FLINT_OK) return s;
   }
-  int grid = 0;
-  flint_status s = plan(P, tiles, n_layers, num_ctas, ws_bytes, who, &grid);
-  if (s != FLINT_OK) return s;
-  P.smem_bytes = static_cast<int32_t>(decode_smem_bytes());
-  P.counters = static_cast<int32_t*>(workspace);
-  P.partials = reinterpret_cast<float*>(static_cast<uint8_t*>(workspace) + kCounterBytes);
-  P.dev_err = dev_err;
-  P.n_problems = n_layers;
-  P.prep = 1;
-  P.eps = eps;
-  // RoPE angles of the new token, pos * theta^(-2i/128) for i < 64, in double
-  // on the host (one position for every layer of the call)
-  for (int i = 0; i < kDim / 2; ++i) {
-    const double a = static_cast<double>(pos) * std::pow(theta, -2.0 * i / kDim);
-    P.rope_cs[i] = make_float2(static_cast<float>(std::cos(a)), static_cast<float>(std::sin(a)));
-  }
-  return launch_result(launch_decode(P, grid, static_cast<cudaStream_t>(stream)), who);
+  return ok();
 }
 
 }  // extern "C"

@@ -1011,6 +1011,10 @@ __device__ void grid_merge(const DecodeParams& P, const Smem& S) {
 }
 
 __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const __grid_constant__ DecodeParams P) {
+  // A launch that follows this one in the stream with programmatic
+  // dependence may be scheduled from now on (it waits for this grid's
+  // completion before it touches global memory, see below).
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
   extern __shared__ uint8_t smem_raw[];
   const Smem S = carve(smem_raw);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -1041,6 +1045,10 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const __grid_consta
   }
   if (P.prep && threadIdx.x < kDim / 2) S.cs[threadIdx.x] = P.rope_cs[threadIdx.x];
   __syncthreads();
+  // Programmatic dependent launch: everything above overlapped the previous
+  // kernel of the stream; wait for it to complete (and its memory to be
+  // visible) before any access to the workspace, the caches or the inputs.
+  if (P.pdl) asm volatile("griddepcontrol.wait;" ::: "memory");
 
   ProducerCount pc{0, 0};
   if (warp == kConsumerWarps) {
@@ -1098,15 +1106,27 @@ cudaError_t launch_decode(const DecodeParams& p, int grid, cudaStream_t stream) 
     if (e != cudaSuccess) return e;
     configured_device = dev;
   }
-  if (p.grid_merge) {
-    // the grid barrier needs every CTA resident at once
-    void* args[] = {const_cast<DecodeParams*>(&p)};
-    e = cudaLaunchCooperativeKernel(reinterpret_cast<const void*>(decode_kernel), dim3(grid),
-                                    dim3(kThreads), args, decode_smem_bytes(), stream);
-    if (e != cudaSuccess) return e;
-  } else {
-    decode_kernel<<<grid, kThreads, decode_smem_bytes(), stream>>>(p);
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(grid);
+  cfg.blockDim = dim3(kThreads);
+  cfg.dynamicSmemBytes = decode_smem_bytes();
+  cfg.stream = stream;
+  cudaLaunchAttribute attrs[2];
+  int n = 0;
+  if (p.grid_merge) {  // the grid barrier needs every CTA resident at once
+    attrs[n].id = cudaLaunchAttributeCooperative;
+    attrs[n].val.cooperative = 1;
+    ++n;
   }
+  if (p.pdl) {
+    attrs[n].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attrs[n].val.programmaticStreamSerializationAllowed = 1;
+    ++n;
+  }
+  cfg.attrs = attrs;
+  cfg.numAttrs = n;
+  e = cudaLaunchKernelEx(&cfg, decode_kernel, p);
+  if (e != cudaSuccess) return e;
   return cudaGetLastError();
 }
 

@@ -131,6 +131,8 @@ struct DecodeParams {
   int32_t n_deferred;
   int32_t n_wide;           // deferred[0, n_wide): merged a CTA per unit, the rest a warp per unit
   int32_t ws_items;         // partial slots in the workspace
+  int32_t pdl;              // 1: programmatic dependent launch on the previous kernel of the
+                            // stream: wait for it before touching global memory
   int32_t smem_bytes;       // dynamic shared memory of the launch
 };
 

@@ -32,7 +32,7 @@ MAX_BATCH, MAX_LAYERS = 64, 49
 EXPORTED = (
     "flint_status_string", "flint_last_error", "flint_kv_bytes", "flint_qk_norm_rope",
     "flint_kv_append", "flint_attn_workspace_bytes", "flint_attn_decode", "flint_attn_stack",
-    "flint_attn_stack_noalloc", "flint_plan_items", "flint_plan_split",
+    "flint_attn_stack_noalloc", "flint_attn_layers_serial", "flint_plan_items", "flint_plan_split",
 )
 
 
@@ -86,6 +86,8 @@ def load_library() -> ctypes.CDLL:
                                               I32, P, P]
             lib.flint_attn_stack.argtypes = [P, I32, I32, ctypes.c_float, ctypes.c_double, P, P,
                                              ctypes.c_size_t, I32, P, P]
+            lib.flint_attn_layers_serial.argtypes = [P, I32, I32, ctypes.c_float, ctypes.c_double, P, P,
+                                                     ctypes.c_size_t, I32, P, P]
             lib.flint_attn_stack_noalloc.argtypes = [P, I32, I32, ctypes.c_float, ctypes.c_double,
                                                      P, I32, P, P]
             lib.flint_plan_items.argtypes = [P, I32, I32, I32, P, P, P, P, I32]
@@ -93,7 +95,7 @@ def load_library() -> ctypes.CDLL:
             lib.flint_plan_split.argtypes = [P, I32, I32, I32, I32, P, P, P, P, P]
             lib.flint_plan_split.restype = I32
             for name in ("flint_qk_norm_rope", "flint_kv_append", "flint_attn_decode",
-                         "flint_attn_stack", "flint_attn_stack_noalloc"):
+                         "flint_attn_stack", "flint_attn_stack_noalloc", "flint_attn_layers_serial"):
                 getattr(lib, name).restype = ctypes.c_int
             _lib = lib
     return _lib
@@ -230,6 +232,18 @@ def flint_attn_stack(layers, pos: int, out, ws: torch.Tensor, eps: float = 1e-6,
     _check(lib.flint_attn_stack(arr, len(arr), int(pos), eps, theta, _ptr(out), _ptr(ws),
                                 ws.numel() * ws.element_size(), int(num_ctas), _ptr(dev_err),
                                 _stream(stream)))
+    return out
+
+
+def flint_attn_layers_serial(layers, pos: int, out, ws: torch.Tensor, eps: float = 1e-6,
+                             theta: float = 10000.0, num_ctas: int = 0, dev_err=None, stream=None):
+    """flint_attn_stack as one dependent launch per layer (programmatic
+    dependent launch); layers: a ctypes array from stack_layers() or a list."""
+    arr = layers if isinstance(layers, ctypes.Array) else stack_layers(layers)
+    lib = load_library()
+    _check(lib.flint_attn_layers_serial(arr, len(arr), int(pos), eps, theta, _ptr(out), _ptr(ws),
+                                        ws.numel() * ws.element_size(), int(num_ctas), _ptr(dev_err),
+                                        _stream(stream)))
     return out
 
 
