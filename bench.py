@@ -35,9 +35,10 @@ NOMINAL_HBM_GBS = 8000.0
 
 # DRAM traffic (dram__bytes_read.sum + dram__bytes_write.sum) of one decode_kernel
 # launch from a full-size, one-pass ncu capture of the stack at context 100,000
-# (profiles/decode_kernel_stack100k_traffic.md), with the hash of the CUDA
+# (profiles/decode_kernel_stack100k_traffic.md), per KV dtype, with the hash of the CUDA
 # sources it was taken on; reported only while the sources still hash the same.
-TRAFFIC = {("stack", 100_000): (2_905_856_000 + 6_322_176, "58f64013b925776a")}
+TRAFFIC = {("stack", 100_000, "bf16"): (2_905_824_256 + 6_814_208, "207da7376fd4f092"),
+           ("stack", 100_000, "fp8"): (1_453_987_328 + 6_094_848, "207da7376fd4f092")}
 
 
 def max_over_ranks(x: float, world: int, device) -> float:
@@ -69,8 +70,8 @@ def kernel_sources_hash() -> str:
     return m.hexdigest()[:16]
 
 
-def traffic_for(workload: str, ctx: int):
-    t = TRAFFIC.get((workload, ctx))
+def traffic_for(workload: str, ctx: int, kv: str = "bf16"):
+    t = TRAFFIC.get((workload, ctx, kv))
     return t[0] if t is not None and t[1] == kernel_sources_hash() else None
 FALLBACK_HBM_GBS = 6650.0
 
@@ -508,7 +509,7 @@ def main():
                      "frac": achieved / peak, "peak_kind": peak_kind,
                      "frac_of_nominal_8000": achieved / NOMINAL_HBM_GBS,
                      "algorithmic_bytes": int(algo_bytes), "kernel": "flint decode_kernel",
-                     "traffic": None if fp8 else traffic_for(args.workload, ctx)},
+                     "traffic": traffic_for(args.workload, ctx, args.kv)},
         "cpu_baseline": cpu_baseline,
         "e2e": e2e,
         "gpu_launches": args.steps * (49 if args.workload == "serial" else 1),
