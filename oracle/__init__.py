@@ -315,3 +315,31 @@ def decode_layer_fp8(q_raw, k_raw, v_raw, w_q, w_k, sinks, k_cache, v_cache, k_s
     if rc != 0:
         raise ValueError("oracle rejected the arguments")
     return out
+
+
+# ---- prefill of a prompt ----------------------------------------------------
+
+def prefill(q_raw, k_raw, v_raw, w_q, w_k, sinks, window: int, apply_rope: bool, rows,
+            eps: float = 1e-6, theta: float = 10000.0, nthreads: int = 0):
+    """Prefill of a prompt of T tokens at positions 0..T-1 with nothing cached
+    before it: per token, norm (+RoPE) of q and k; k rounded to bf16 (the cache
+    value) and q rounded to bf16 too (prefill activations are bf16); then query
+    row t attends the keys of positions max(0, t - window + 1) .. t (window > 0)
+    or 0 .. t, with the head's sink -- the decode attention of position t
+    with L = t + 1.  q_raw [T, 32, 128], k_raw / v_raw [T, 4, 128] bf16 bits.
+    Returns (out float64 [len(rows), 32, 128] for the requested rows,
+    q bf16 bits [T, 32, 128], k bf16 bits [T, 4, 128])."""
+    q_raw, k_raw, v_raw = _u16(q_raw), _u16(k_raw), _u16(v_raw)
+    T, nq, d = q_raw.shape
+    nkv = k_raw.shape[1]
+    qb = np.empty((T, nq, d), np.uint16)
+    kb = np.empty((T, nkv, d), np.uint16)
+    for t in range(T):
+        q, _, k16 = qk_norm_rope(q_raw[t], k_raw[t], w_q, w_k, t, eps, theta, apply_rope)
+        qb[t] = f64_to_bf16(q)
+        kb[t] = k16
+    sinks = _f64(sinks)
+    out = np.empty((len(rows), nq, d), np.float64)
+    for i, t in enumerate(rows):
+        out[i] = attn_decode(qb[t], kb, v_raw, int(t) + 1, sinks, window, nthreads=nthreads)
+    return out, qb, kb

@@ -491,3 +491,34 @@ def test_fp8_decode_layer_is_norm_rope_then_quantized_append_then_attention():
     assert np.array_equal(kc, kw) and np.array_equal(vc, vw)
     want = oracle.attn_decode_fp8(q, kw, vw, ks, vs, L, sinks, 513, layout=oracle.RING, capacity=cap)
     np.testing.assert_array_equal(got, want)
+
+
+# ---------------------------------------------------------------- prefill ----
+
+@pytest.mark.parametrize("window,rope", [(0, False), (8, True)])
+def test_prefill_rows_match_causal_sdpa_with_a_sink_column(window, rope):
+    """Prefill of a T-token prompt: every row of the oracle equals one
+    torch SDPA call over the whole prompt with a causal (and sliding-window)
+    mask, GQA heads expanded, and the sink as an extra key whose value is
+    zero -- the same q, k, v bits on both sides."""
+    T, nq, nkv, d = 40, 8, 2, 32
+    q_raw, k_raw, v_raw = bf16_bits((T, nq, d), 301), bf16_bits((T, nkv, d), 302), bf16_bits((T, nkv, d), 303)
+    w_q, w_k = bf16_bits((d,), 304, 1.0, 0.1), bf16_bits((d,), 305, 1.0, 0.1)
+    sinks = rng.normal(size=nq)
+    out, qb, kb = oracle.prefill(q_raw, k_raw, v_raw, w_q, w_k, sinks, window, rope, rows=range(T))
+    q = torch.from_numpy(f64(qb)).permute(1, 0, 2)                            # [nq, T, d]
+    k = torch.from_numpy(f64(kb)).permute(1, 0, 2).repeat_interleave(nq // nkv, 0)
+    v = torch.from_numpy(f64(v_raw)).permute(1, 0, 2).repeat_interleave(nq // nkv, 0)
+    zero = torch.zeros(nq, 1, d, dtype=torch.float64)
+    k = torch.cat([k, zero], dim=1)                                           # sink key at T
+    v = torch.cat([v, zero], dim=1)
+    t = torch.arange(T)[:, None]
+    j = torch.arange(T)[None, :]
+    allowed = (j <= t) & ((j > t - window) if window else torch.ones_like(j <= t))
+    bias = torch.where(allowed, 0.0, float("-inf")).to(torch.float64)
+    bias = bias[None].repeat(nq, 1, 1)
+    # the sink column: q . 0 = 0 plus a bias equal to the head's sink logit
+    sink_col = torch.from_numpy(sinks).to(torch.float64)[:, None, None].expand(nq, T, 1)
+    bias = torch.cat([bias, sink_col * math.sqrt(d)], dim=2) / math.sqrt(d)
+    want = F.scaled_dot_product_attention(q, k, v, attn_mask=bias, scale=1.0 / math.sqrt(d))
+    np.testing.assert_allclose(out, want.permute(1, 0, 2).numpy(), rtol=1e-10, atol=1e-12)
