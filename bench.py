@@ -3,7 +3,7 @@
 with its own bf16 KV cache), on B200s.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl flint|reference]
-                    [--workload stack|full100k|full2k|swa100k|paged32|paged32swa]
+                    [--workload stack|full100k|full2k|swa100k|paged32|paged32swa|prefill8k]
 
 Prints one JSON line (rank 0).  A step is one call of flint_attn_stack: for
 every layer the fused Q/K RMSNorm (+RoPE), KV append at position 99,999 and
@@ -74,6 +74,7 @@ def traffic_for(workload: str, ctx: int, kv: str = "bf16"):
     t = TRAFFIC.get((workload, ctx, kv))
     return t[0] if t is not None and t[1] == kernel_sources_hash() else None
 FALLBACK_HBM_GBS = 6650.0
+FALLBACK_BF16_TFLOPS = 1400.0   # sustained, under the power cap
 
 
 def parse():
@@ -83,15 +84,27 @@ def parse():
     ap.add_argument("--warmup", type=int, default=20)
     ap.add_argument("--impl", default="flint", choices=["flint", "reference"])
     ap.add_argument("--workload", default="stack",
-                    choices=["stack", "serial", "full100k", "full2k", "swa100k", "paged32", "paged32swa"])
-    ap.add_argument("--context", type=int, default=100_000,
-                    help="context length (the benchmark's figure is 100,000; smaller ones serve profiling)")
+                    choices=["stack", "serial", "full100k", "full2k", "swa100k", "paged32", "paged32swa",
+                             "prefill8k"])
+    ap.add_argument("--context", type=int, default=None,
+                    help="context length (decode: 100,000; prefill8k: the prompt length, 8,192; "
+                         "smaller ones serve profiling)")
     ap.add_argument("--kv", default="bf16", choices=["bf16", "fp8"],
                     help="KV-cache element: bf16, or E4M3 codes with per-head scales")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-graph", action="store_true", help="time direct launches instead of graph replays")
     return ap.parse_args()
+
+
+def measured_tensor_peak():
+    """Dense bf16 tensor throughput: the sustained figure (the attention
+    kernels run inside a step of tens of milliseconds)."""
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+            return float(json.load(f)["bf16_tflops_sustained"]), "measured (sustained)"
+    except Exception:
+        return FALLBACK_BF16_TFLOPS, "fallback"
 
 
 def measured_peak():
@@ -159,6 +172,27 @@ def run_reference(args, rank):
 
     oracle.build()
     nthreads = os.cpu_count() or 1
+    if args.workload == "prefill8k":
+        T = args.context
+        prompts = prefill_inputs(I, T, kinds_only=True)
+        oracle_prefill_sample(prompts, T, nthreads, budget_s=2.0)  # warm-up
+        budget = max(5.0, min(30.0, 150.0 / max(1, args.steps)))
+        vals, sample = [], ""
+        for _ in range(args.steps):
+            ms, _, sample = oracle_prefill_sample(prompts, T, nthreads, budget_s=budget)
+            vals.append(ms)
+        ms = statistics.mean(vals)
+        line = {
+            "impl": "reference", "metric": PREFILL_METRIC, "value": ms, "unit": "ms/prompt",
+            "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms,
+            "higher_is_better": False, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+            "data": "synthetic", "config": prefill_config(T),
+            "cpu_baseline": {"value": ms, "unit": "ms/prompt", "cores": nthreads, "kind": "oracle",
+                             "sample": sample},
+            "e2e": {"value": ms, "unit": "ms/prompt", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+        }
+        print(json.dumps(line), flush=True)
+        return
     kinds = I.layer_kinds()
     full_i = kinds.index(True)
     layers_full = [I.make_layer(I.W_STACK_100K, full_i, CONTEXT, 0, False, ring=False)]
@@ -182,6 +216,248 @@ def run_reference(args, rank):
         "e2e": {"value": us, "unit": "us/token", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
     print(json.dumps(line), flush=True)
+
+
+# ------------------------------------------------------------- prefill ----
+
+PREFILL_T = 8192
+PREFILL_METRIC = ("49-layer prefill-attention ms per 8,192-token prompt (norm+RoPE+cache write+causal "
+                  "attention with sinks); achieved TFLOP/s vs peak")
+
+
+def prefill_keys(T: int, window: int) -> int:
+    """Keys attended by all T rows of one head (row t: min(t + 1, window) or t + 1)."""
+    if window == 0:
+        return T * (T + 1) // 2
+    w = min(window, T)
+    return w * (w + 1) // 2 + (T - w) * w
+
+
+def prefill_flops(T: int, window: int) -> int:
+    # q.k and p.v: 2 x 128 multiply-adds per (row, head, key), 32 heads
+    return prefill_keys(T, window) * 32 * 128 * 4
+
+
+def prefill_config(T):
+    return {"workload": "prefill of one prompt through Flint's 49 attention layers: per layer "
+                        "Q/K RMSNorm (+RoPE), KV-cache write and causal GQA attention with sinks; "
+                        "35 sliding-window (513, RoPE, ring cache) + 14 full-context NoPE layers "
+                        "(contiguous cache)",
+            "prompt_tokens": T, "layers": 49, "batch": 1,
+            "l2": "flushed before every step (256 MiB write, then 256 MiB read of another buffer)"}
+
+
+def prefill_inputs(I, T, kinds_only=False):
+    """The 49 layers' prompts (window 513 or 0 per layer kind); kinds_only: one
+    window and one full layer (the oracle sample)."""
+    kinds = I.layer_kinds()
+    if kinds_only:
+        return [I.make_prefill(T, 513, layer=0), I.make_prefill(T, 0, layer=kinds.index(True))]
+    return [I.make_prefill(T, 0 if full else 513, layer=i) for i, full in enumerate(kinds)]
+
+
+def oracle_prefill_sample(prompts, T, nthreads, budget_s=10.0):
+    """Time the oracle's prefill of one window and one full layer on a bounded
+    sample: its norm (+RoPE) pass over all T tokens, then the attention of as
+    many uniformly drawn rows as the budget allows, whose mean time is scaled
+    to all T rows.  Returns (ms per prompt scaled to 35 window + 14 full
+    layers, seconds spent, description)."""
+    import numpy as np
+    import oracle
+    from long_context_decode_flash_b200 import inputs as I
+
+    rng = np.random.default_rng(1)
+    est, spent, desc = [], 0.0, []
+    for p, share in zip(prompts, (0.3, 0.7)):
+        sinks, v = p.sinks.numpy().astype(np.float64), I.bits(p.v_raw)
+        t0 = time.perf_counter()
+        _, qb, kb = oracle.prefill(I.bits(p.q_raw), I.bits(p.k_raw), v, I.bits(p.w_q), I.bits(p.w_k),
+                                   sinks, p.window, p.rope, rows=[], nthreads=nthreads)
+        t_prep = time.perf_counter() - t0
+        rows, t_rows, t_end = 0, 0.0, time.perf_counter() + share * budget_s
+        while rows == 0 or time.perf_counter() < t_end:
+            t = int(rng.integers(0, T))
+            t0 = time.perf_counter()
+            oracle.attn_decode(qb[t], kb, v, t + 1, sinks, p.window, nthreads=nthreads)
+            t_rows += time.perf_counter() - t0
+            rows += 1
+        est.append(t_prep + t_rows / rows * T)
+        spent += t_prep + t_rows
+        desc.append(f"{rows} random rows of a {'window' if p.window else 'full'} layer")
+    ms = (35 * est[0] + 14 * est[1]) * 1e3
+    return ms, spent, (", ".join(desc) + f" of the {T}-token prompt after the oracle's norm (+RoPE) of "
+                       "all its tokens, all 32 heads; row time scaled to all rows and to 35 + 14 layers")
+
+
+def run_prefill(args, rank, world, local):
+    """The prefill8k workload: every step prefills one prompt through all 49
+    layers (flint_prefill_qk_norm_rope with the cache write, then
+    flint_prefill_attn, per layer)."""
+    import torch
+    from long_context_decode_flash_b200 import flint
+    from long_context_decode_flash_b200 import inputs as I
+
+    T = args.context
+    prompts = prefill_inputs(I, T)
+    cpu_baseline = None
+    if rank == 0 and world == 1 and T == PREFILL_T and not args.no_cpu_baseline:
+        import oracle
+        oracle.build()
+        sample = prefill_inputs(I, T, kinds_only=True)
+        nthreads = os.cpu_count() or 1
+        ms_cpu, spent, desc = oracle_prefill_sample(sample, T, nthreads, budget_s=15.0)
+        cpu_baseline = {"value": ms_cpu, "unit": "ms/prompt", "cores": nthreads, "kind": "oracle",
+                        "sample": desc + f" ({spent:.1f} s of CPU wall time)", "cpu_model": cpu_model()}
+
+    if world > 1:
+        torch.distributed.init_process_group("nccl", timeout=__import__("datetime").timedelta(seconds=120))
+    torch.cuda.set_device(local)
+    dev_index = torch.cuda.current_device()
+    stream = torch.cuda.current_stream()
+    flush = torch.empty(256 * 1024 * 1024 // 4, dtype=torch.float32, device="cuda")
+    flush_rd = torch.ones(256 * 1024 * 1024 // 4, dtype=torch.float32, device="cuda")
+    flush_acc = torch.zeros(1, dtype=torch.float32, device="cuda")
+
+    def flush_l2(i):
+        flush.fill_(float(i))
+        torch.sum(flush_rd, dim=0, keepdim=True, out=flush_acc)
+
+    # one packed device buffer (and its pinned host twin) holds every layer's
+    # raw q, k, v, so a step's inputs arrive with one copy
+    nq, nk = T * 32 * 128, T * 4 * 128
+    per = nq + 2 * nk
+    packed = torch.empty((len(prompts), per), dtype=torch.bfloat16, device="cuda")
+    host_in = torch.empty((len(prompts), per), dtype=torch.bfloat16).pin_memory()
+    layers = []
+    for i, p in enumerate(prompts):
+        host_in[i, :nq].copy_(p.q_raw.reshape(-1))
+        host_in[i, nq:nq + nk].copy_(p.k_raw.reshape(-1))
+        host_in[i, nq + nk:].copy_(p.v_raw.reshape(-1))
+
+        class L:
+            pass
+        d = L()
+        row = packed[i]
+        d.q_raw, d.k_raw, d.v_raw = row[:nq].view(T, 32, 128), row[nq:nq + nk].view(T, 4, 128), row[nq + nk:].view(T, 4, 128)
+        d.w_q, d.w_k, d.sinks = p.w_q.cuda(), p.w_k.cuda(), p.sinks.cuda()
+        d.window, d.rope = p.window, p.rope
+        if p.window:
+            d.kc = torch.empty((513, 4, 128), dtype=torch.bfloat16, device="cuda")
+            d.cache = None
+            layout, cap = flint.RING, 513
+        else:
+            d.kc = torch.empty((T + 1, 4, 128), dtype=torch.bfloat16, device="cuda")
+            layout, cap = flint.CONTIGUOUS, T + 1
+        d.vc = torch.empty_like(d.kc)
+        d.cache = flint.kv_cache(d.kc, d.vc, layout, capacity=cap)
+        layers.append(d)
+    packed.copy_(host_in)
+    del prompts
+    q = torch.empty((T, 32, 128), dtype=torch.bfloat16, device="cuda")
+    k = torch.empty((T, 4, 128), dtype=torch.bfloat16, device="cuda")
+    out = torch.empty((len(layers), T, 32, 128), dtype=torch.float32, device="cuda")
+    host_out = torch.empty(out.shape, dtype=torch.float32).pin_memory()
+    err = torch.zeros(1, dtype=torch.int32, device="cuda")
+    n_layers = len(layers)
+    a0 = [torch.cuda.Event(enable_timing=True) for _ in range(n_layers)]
+    a1 = [torch.cuda.Event(enable_timing=True) for _ in range(n_layers)]
+
+    def step(attn_events=False):
+        for i, d in enumerate(layers):
+            flint.flint_prefill_qk_norm_rope(d.q_raw, d.k_raw, d.w_q, d.w_k, apply_rope=d.rope, q_out=q,
+                                             k_out=k, v_raw=d.v_raw, cache=d.cache, dev_err=err)
+            if attn_events:
+                a0[i].record(stream)
+            flint.flint_prefill_attn(q, k, d.v_raw, d.sinks, d.window, out[i])
+            if attn_events:
+                a1[i].record(stream)
+
+    for _ in range(max(args.warmup, 3)):
+        flush_l2(1)
+        step()
+    torch.cuda.synchronize()
+    if int(err.item()) != 0:
+        raise SystemExit(f"device error {int(err.item())} during warm-up")
+    t0 = time.perf_counter()
+    step()
+    host_us = (time.perf_counter() - t0) * 1e6 / n_layers
+    torch.cuda.synchronize()
+
+    starts = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    ends = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    attn_ms = []
+    if world > 1:
+        torch.distributed.barrier()
+    torch.cuda.synchronize()
+    with ClockSampler(dev_index) as clocks:
+        t_wall = time.perf_counter()
+        for i in range(args.steps):
+            flush_l2(i)
+            starts[i].record(stream)
+            step(attn_events=True)
+            ends[i].record(stream)
+            torch.cuda.synchronize()  # the attention events are reused next step
+            attn_ms.append([s.elapsed_time(e) for s, e in zip(a0, a1)])
+        t_wall = time.perf_counter() - t_wall
+    if world > 1:
+        torch.distributed.barrier()
+    per_step_ms = [s.elapsed_time(e) for s, e in zip(starts, ends)]
+    ms = statistics.mean(per_step_ms)
+    if int(err.item()) != 0:
+        raise SystemExit(f"device error {int(err.item())} in the timed region")
+
+    e2e = None
+    if not args.no_e2e:
+        e_s = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+        e_e = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+        if world > 1:
+            torch.distributed.barrier()
+        torch.cuda.synchronize()
+        for i in range(args.steps):
+            flush_l2(i)
+            e_s[i].record(stream)
+            packed.copy_(host_in, non_blocking=True)
+            step()
+            host_out.copy_(out, non_blocking=True)
+            e_e[i].record(stream)
+        torch.cuda.synchronize()
+        e2e_ms = max_over_ranks(statistics.mean(s.elapsed_time(e) for s, e in zip(e_s, e_e)), world, "cuda")
+        e2e = {"value": e2e_ms / world, "unit": "ms/prompt",
+               "h2d_bytes_per_step": int(host_in.numel() * 2), "d2h_bytes_per_step": int(host_out.numel() * 4)}
+    ms = max_over_ranks(ms, world, "cuda")
+
+    kinds = I.layer_kinds()
+    flops = sum(prefill_flops(T, 0 if full else 513) for full in kinds)
+    attn_total_ms = statistics.mean(sum(x) for x in attn_ms)
+    full_ms = statistics.mean(sum(x[i] for i, f in enumerate(kinds) if f) for x in attn_ms) / sum(kinds)
+    win_ms = statistics.mean(sum(x[i] for i, f in enumerate(kinds) if not f) for x in attn_ms) / (49 - sum(kinds))
+    achieved = flops / (attn_total_ms * 1e-3) / 1e12
+    peak, peak_kind = measured_tensor_peak()
+    line = {
+        "metric": PREFILL_METRIC, "value": ms / world, "unit": "ms/prompt",
+        "n_gpus": world, "steps": args.steps, "warmup": max(args.warmup, 3), "ms_per_step": ms,
+        "higher_is_better": False, "scaling": "weak", "vs_baseline": None,
+        "dtype": "bf16 (mma.sync bf16, fp32 accumulate and softmax)",
+        "data": "synthetic (seeded bf16 N(0,1) raw q/k/v, N(0,1) sinks, 1+N(0,0.1) norm weights)",
+        "config": dict(prefill_config(T), parallelism=f"replicas x{world}", launch="direct launches"),
+        "roofline": {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
+                     "frac": achieved / peak, "peak_kind": peak_kind, "kernel": "flint prefill_kernel",
+                     "algorithmic_flops": int(flops), "attn_ms_per_prompt": attn_total_ms,
+                     "full_layer_attn_us": full_ms * 1e3, "window_layer_attn_us": win_ms * 1e3,
+                     "traffic": None},
+        "cpu_baseline": cpu_baseline,
+        "e2e": e2e,
+        "gpu_launches": args.steps * 2 * n_layers,
+        "host_us_per_call": host_us,
+        "clocks": clocks.summary(),
+        "per_step_ms": {"min": min(per_step_ms), "median": statistics.median(per_step_ms),
+                        "max": max(per_step_ms)},
+        "timed_region_wall_s": t_wall,
+    }
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        torch.distributed.destroy_process_group()
 
 
 # ------------------------------------------------------------- GPU side ----
@@ -304,8 +580,13 @@ def main():
     rank = int(os.environ.get("RANK", "0"))
     world = int(os.environ.get("WORLD_SIZE", "1"))
     local = int(os.environ.get("LOCAL_RANK", "0"))
+    if args.context is None:
+        args.context = PREFILL_T if args.workload == "prefill8k" else CONTEXT
     if args.impl == "reference":
         run_reference(args, rank)
+        return
+    if args.workload == "prefill8k":
+        run_prefill(args, rank, world, local)
         return
 
     import torch

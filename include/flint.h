@@ -254,6 +254,49 @@ flint_status flint_attn_stack_noalloc(const flint_layer* layers, int32_t n_layer
                                       int32_t pos, float eps, double theta, float* out,
                                       int32_t num_ctas, int32_t* dev_err, void* stream);
 
+/* Prefill, step 1: per-head Q/K RMSNorm, optional RoPE and the cache write
+ * for the T tokens of one prompt at positions 0 .. T-1, with nothing cached
+ * before it (the 8,192-token prefill of "Day-0 Support for Flint on vLLM",
+ * newruntime.com, "What happened"; norm and RoPE as in flint_qk_norm_rope,
+ * token t at position t).
+ *   q_raw  bf16 [T][32][128], k_raw / v_raw bf16 [T][4][128]   (device, in)
+ *   w_q, w_k  bf16 [128] (device, in)
+ *   q_out  bf16 [T][32][128] (device, out): q after norm/RoPE, rounded to
+ *          nearest even (prefill activations are bf16), or NULL
+ *   k_out  bf16 [T][4][128]  (device, out): k after norm/RoPE, rounded to
+ *          nearest even (the cache value), or NULL
+ *   cache  NULL, or the cache of this one request (request 0 of a
+ *          CONTIGUOUS / RING cache, row 0 of a PAGED block table): token t
+ *          goes to slot t (ring: t % 513, and only the last 513 tokens are
+ *          written); an E4M3 cache gets the codes of flint_qk_norm_rope.
+ * T in [1, FLINT_MAX_CONTEXT]; T must fit the cache (contiguous capacity,
+ * block table).  Errors as for flint_qk_norm_rope. */
+flint_status flint_prefill_qk_norm_rope(const uint16_t* q_raw, const uint16_t* k_raw,
+                                        const uint16_t* v_raw, const uint16_t* w_q,
+                                        const uint16_t* w_k, int32_t T, float eps,
+                                        double theta, int32_t apply_rope, uint16_t* q_out,
+                                        uint16_t* k_out, const flint_kv_cache* cache,
+                                        int32_t* dev_err, void* stream);
+
+/* Prefill, step 2: causal attention of a T-token prompt over itself, with the
+ * head's sink ("Model architecture": GQA 32/4, learned sinks, 513-token
+ * windows on the RoPE layers, full context on the NoPE layers).  Query row t
+ * of head h attends the keys of positions max(0, t - window + 1) .. t
+ * (window > 0) or 0 .. t of KV head h / 8, as flint_attn_decode does for the
+ * token at position t with L = t + 1:
+ *   out[t][h] = sum_j e^(s_j - M) v[j] / (sum_j e^(s_j - M) + e^(sink_h - M)),
+ *   s_j = q[t][h] . k[j] / sqrt(128), M = max(max_j s_j, sink_h).
+ *   q  bf16 [T][32][128]; k, v  bf16 [T][4][128] (device, in; flint_prefill_
+ *      qk_norm_rope's q_out and k_out, and v_raw)
+ *   sinks  fp32 [32] (device, in); window  0 or FLINT_WINDOW
+ *   out  fp32 [T][32][128] (device, out)
+ * T in [1, FLINT_MAX_CONTEXT].  Products on bf16 tensor-core MMAs with fp32
+ * accumulation; softmax in fp32.  Host-side errors only; dev_err is unused
+ * and may be NULL. */
+flint_status flint_prefill_attn(const uint16_t* q, const uint16_t* k, const uint16_t* v,
+                                int32_t T, const float* sinks, int32_t window, float* out,
+                                int32_t* dev_err, void* stream);
+
 /* The split planner behind both attention calls (pure host code, exposed for
  * tests).  Work is n_segs segments (one per problem, all four KV heads
  * together) of seg_tiles[s] 32-token tiles; it is cut into items (segment, tile range)

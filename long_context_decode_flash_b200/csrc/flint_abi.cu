@@ -566,6 +566,85 @@ flint_status flint_kv_append(const uint16_t* k, const uint16_t* v, const int32_t
   return launch_result(launch_prep(p, B, static_cast<cudaStream_t>(stream)), who);
 }
 
+flint_status flint_prefill_qk_norm_rope(const uint16_t* q_raw, const uint16_t* k_raw,
+                                        const uint16_t* v_raw, const uint16_t* w_q,
+                                        const uint16_t* w_k, int32_t T, float eps,
+                                        double theta, int32_t apply_rope, uint16_t* q_out,
+                                        uint16_t* k_out, const flint_kv_cache* cache,
+                                        int32_t* dev_err, void* stream) {
+  const char* who = "flint_prefill_qk_norm_rope";
+  if (!q_raw || !k_raw || !w_q || !w_k) return fail(FLINT_ERR_INVALID_ARG, "%s: NULL input pointer", who);
+  if (T < 1 || T > FLINT_MAX_CONTEXT)
+    return fail(FLINT_ERR_INVALID_ARG, "%s: T=%d outside [1, %d]", who, T, FLINT_MAX_CONTEXT);
+  if (apply_rope != 0 && apply_rope != 1) return fail(FLINT_ERR_INVALID_ARG, "%s: apply_rope must be 0 or 1", who);
+  if (!(eps >= 0.f) || !(theta > 0.0)) return fail(FLINT_ERR_INVALID_ARG, "%s: eps must be >= 0, theta > 0", who);
+  if (!q_out && !k_out && !cache) return fail(FLINT_ERR_INVALID_ARG, "%s: no output requested", who);
+  const void* ptrs[] = {q_raw, k_raw, w_q, w_k, q_out, k_out, v_raw};
+  for (const void* p : ptrs)
+    if (p && !aligned16(p)) return fail(FLINT_ERR_INVALID_ARG, "%s: pointers must be 16-byte aligned", who);
+  PrepParams p;
+  memset(&p, 0, sizeof p);
+  p.q_raw = q_raw;
+  p.k_raw = k_raw;
+  p.v_raw = v_raw;
+  p.w_q = w_q;
+  p.w_k = w_k;
+  p.q_out_bf16 = q_out;
+  p.k_out = k_out;
+  p.eps = eps;
+  p.theta = theta;
+  p.apply_rope = apply_rope;
+  p.do_norm = 1;
+  p.dev_err = dev_err;
+  p.prefill = 1;
+  p.n_tokens = T;
+  if (cache) {
+    if (!v_raw) return fail(FLINT_ERR_INVALID_ARG, "%s: writing the cache needs v_raw", who);
+    flint_status s = check_cache(cache, 1, who);
+    if (s != FLINT_OK) return s;
+    const flint_kv_cache& c = *cache;
+    if (c.layout == FLINT_KV_CONTIGUOUS && T > c.capacity)
+      return fail(FLINT_ERR_INVALID_ARG, "%s: T=%d exceeds the cache capacity %d", who, T, c.capacity);
+    if (c.layout == FLINT_KV_PAGED && static_cast<int64_t>(T) > static_cast<int64_t>(c.max_blocks_per_req) * kBlock)
+      return fail(FLINT_ERR_INVALID_ARG, "%s: T=%d exceeds the block table (%d blocks)", who, T, c.max_blocks_per_req);
+    p.k_rows = static_cast<uint16_t*>(c.k);
+    p.v_rows = static_cast<uint16_t*>(c.v);
+    p.table = c.block_table;
+    p.layout = c.layout;
+    p.capacity = c.capacity;
+    p.req_stride = c.req_stride ? c.req_stride : static_cast<int64_t>(c.capacity) * kKvHeads * kDim;
+    p.max_blocks = c.max_blocks_per_req;
+    p.num_blocks = c.num_blocks;
+    set_prep_fp8(p, c);
+  }
+  return launch_result(launch_prep(p, T, static_cast<cudaStream_t>(stream)), who);
+}
+
+flint_status flint_prefill_attn(const uint16_t* q, const uint16_t* k, const uint16_t* v, int32_t T,
+                                const float* sinks, int32_t window, float* out, int32_t* dev_err,
+                                void* stream) {
+  const char* who = "flint_prefill_attn";
+  if (!q || !k || !v || !sinks || !out) return fail(FLINT_ERR_INVALID_ARG, "%s: NULL pointer", who);
+  const void* ptrs[] = {q, k, v, sinks, out};
+  for (const void* p : ptrs)
+    if (!aligned16(p)) return fail(FLINT_ERR_INVALID_ARG, "%s: pointers must be 16-byte aligned", who);
+  if (T < 1 || T > FLINT_MAX_CONTEXT)
+    return fail(FLINT_ERR_INVALID_ARG, "%s: T=%d outside [1, %d]", who, T, FLINT_MAX_CONTEXT);
+  if (window != 0 && window != kWindow)
+    return fail(FLINT_ERR_UNSUPPORTED, "%s: window must be 0 or %d", who, kWindow);
+  PrefillParams p;
+  memset(&p, 0, sizeof p);
+  p.q = q;
+  p.k = k;
+  p.v = v;
+  p.sinks = sinks;
+  p.out = out;
+  p.dev_err = dev_err;
+  p.T = T;
+  p.window = window;
+  return launch_result(launch_prefill(p, static_cast<cudaStream_t>(stream)), who);
+}
+
 size_t flint_attn_workspace_bytes(int32_t n_problems, int32_t num_ctas) {
   if (n_problems < 1 || n_problems > kMaxProblems || num_ctas < 0 || num_ctas > kMaxCtas) return 0;
   return kCounterBytes + static_cast<size_t>(kMaxItems) * kPartialBytes;

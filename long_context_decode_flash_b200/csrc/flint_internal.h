@@ -160,11 +160,31 @@ struct PrepParams {
   int32_t do_norm;          // 0: k is already final (plain append)
   int32_t fp8;              // 1: E4M3 cache (k_rows / v_rows are byte rows)
   float k_scale[4], v_scale[4];
+  // prefill: block b is token b of one prompt (position b, cache request 0);
+  // a ring cache receives only the last `capacity` tokens
+  int32_t prefill;
+  int32_t n_tokens;
+  uint16_t* q_out_bf16;     // q rounded to bf16 [T][32][128], or nullptr
+};
+
+// Prompt attention (prefill): q bf16 [T][32][128], k / v bf16 [T][4][128],
+// out fp32 [T][32][128]; query t attends keys max(0, t - window + 1) .. t
+// (window > 0) or 0 .. t.
+struct PrefillParams {
+  const uint16_t* q;
+  const uint16_t* k;
+  const uint16_t* v;
+  const float* sinks;
+  float* out;
+  int32_t* dev_err;
+  int32_t T;
+  int32_t window;
 };
 
 // Launchers (return cudaGetLastError() after the launch).
 cudaError_t launch_decode(const DecodeParams& p, int grid, cudaStream_t stream);  // cooperative if p.grid_merge
 cudaError_t launch_prep(const PrepParams& p, int B, cudaStream_t stream);
+cudaError_t launch_prefill(const PrefillParams& p, cudaStream_t stream);
 
 size_t decode_smem_bytes();
 

@@ -8,7 +8,8 @@
 // rows, then 4 k rows) with RoPE pairs (i, i+64) in one lane.  k is rounded
 // to bf16 (nearest even) once and the same bits go to k_out and the cache; v
 // is copied bit for bit.  With do_norm = 0 and no RoPE the kernel is a plain
-// bit-exact append of final k and v.  An E4M3 cache receives, for k and v,
+// bit-exact append of final k and v.  In prefill mode the blocks are the T
+// tokens of one prompt at positions 0 .. T-1 and q is written rounded to bf16.  An E4M3 cache receives, for k and v,
 // the codes of float32 (value / scale) (nearest even, saturating), where k is
 // the float32 normed (roped) value.
 #include "flint_device.cuh"
@@ -23,15 +24,19 @@ __global__ void __launch_bounds__(kPrepThreads) prep_kernel(const __grid_constan
   __shared__ float2 cs[64];
   const int b = blockIdx.x;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int pos = p.pos[b];
+  const int pos = p.prefill ? b : p.pos[b];
+  const int req = p.prefill ? 0 : b;
   if (p.apply_rope && threadIdx.x < 64) cs[threadIdx.x] = rope_cos_sin(threadIdx.x, pos, p.theta);
   __syncthreads();
 
   // element offset of this request's new-token row (KV head 0), or -1
   long long row = -1;
-  if (p.k_rows) {
+  // (a prompt longer than a ring writes only its last `capacity` tokens, so
+  // that no two blocks write one slot)
+  const bool ring_skip = p.prefill && p.layout == FLINT_KV_RING && b < p.n_tokens - p.capacity;
+  if (p.k_rows && !ring_skip) {
     if (p.layout == FLINT_KV_PAGED) {
-      const int blk = p.table[static_cast<long long>(b) * p.max_blocks + pos / kBlock];
+      const int blk = p.table[static_cast<long long>(req) * p.max_blocks + pos / kBlock];
       if (blk >= 0 && blk < p.num_blocks) {
         row = (static_cast<long long>(blk) * kBlock + pos % kBlock) * kKvHeads * kDim;
       } else if (threadIdx.x == 0) {
@@ -39,7 +44,7 @@ __global__ void __launch_bounds__(kPrepThreads) prep_kernel(const __grid_constan
       }
     } else {
       const int slot = p.layout == FLINT_KV_RING ? pos % p.capacity : pos;
-      row = static_cast<long long>(b) * p.req_stride + static_cast<long long>(slot) * kKvHeads * kDim;
+      row = static_cast<long long>(req) * p.req_stride + static_cast<long long>(slot) * kKvHeads * kDim;
     }
   }
 
@@ -56,6 +61,11 @@ __global__ void __launch_bounds__(kPrepThreads) prep_kernel(const __grid_constan
         float* o = p.q_out + (static_cast<long long>(b) * kHeads + r) * kDim;
         reinterpret_cast<float2*>(o)[lane] = make_float2(y[0], y[1]);
         reinterpret_cast<float2*>(o + 64)[lane] = make_float2(y[2], y[3]);
+      }
+      if (p.q_out_bf16) {
+        uint32_t* o = reinterpret_cast<uint32_t*>(p.q_out_bf16 + (static_cast<long long>(b) * kHeads + r) * kDim);
+        o[lane] = pack_bf16x2(y[0], y[1]);
+        o[32 + lane] = pack_bf16x2(y[2], y[3]);
       }
     } else {
       const uint32_t ka = pack_bf16x2(y[0], y[1]), kb = pack_bf16x2(y[2], y[3]);

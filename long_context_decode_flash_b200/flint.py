@@ -33,6 +33,7 @@ EXPORTED = (
     "flint_status_string", "flint_last_error", "flint_kv_bytes", "flint_qk_norm_rope",
     "flint_kv_append", "flint_attn_workspace_bytes", "flint_attn_decode", "flint_attn_stack",
     "flint_attn_stack_noalloc", "flint_attn_layers_serial", "flint_plan_items", "flint_plan_split",
+    "flint_prefill_qk_norm_rope", "flint_prefill_attn",
 )
 
 
@@ -90,12 +91,16 @@ def load_library() -> ctypes.CDLL:
                                                      ctypes.c_size_t, I32, P, P]
             lib.flint_attn_stack_noalloc.argtypes = [P, I32, I32, ctypes.c_float, ctypes.c_double,
                                                      P, I32, P, P]
+            lib.flint_prefill_qk_norm_rope.argtypes = [P, P, P, P, P, I32, ctypes.c_float,
+                                                       ctypes.c_double, I32, P, P, P, P, P]
+            lib.flint_prefill_attn.argtypes = [P, P, P, I32, P, I32, P, P, P]
             lib.flint_plan_items.argtypes = [P, I32, I32, I32, P, P, P, P, I32]
             lib.flint_plan_items.restype = I32
             lib.flint_plan_split.argtypes = [P, I32, I32, I32, I32, P, P, P, P, P]
             lib.flint_plan_split.restype = I32
             for name in ("flint_qk_norm_rope", "flint_kv_append", "flint_attn_decode",
-                         "flint_attn_stack", "flint_attn_stack_noalloc", "flint_attn_layers_serial"):
+                         "flint_attn_stack", "flint_attn_stack_noalloc", "flint_attn_layers_serial",
+                         "flint_prefill_qk_norm_rope", "flint_prefill_attn"):
                 getattr(lib, name).restype = ctypes.c_int
             _lib = lib
     return _lib
@@ -193,6 +198,30 @@ def flint_kv_append(k, v, pos: Sequence[int], cache: KVCache, dev_err=None, stre
     lib = load_library()
     _check(lib.flint_kv_append(_ptr(k), _ptr(v), _i32_host(pos), len(pos), ctypes.byref(cache),
                                _ptr(dev_err), _stream(stream)))
+
+
+def flint_prefill_qk_norm_rope(q_raw, k_raw, w_q, w_k, eps: float = 1e-6, theta: float = 10000.0,
+                               apply_rope: bool = True, q_out=None, k_out=None, v_raw=None,
+                               cache: Optional[KVCache] = None, dev_err=None, stream=None):
+    """Norm (+RoPE) of the T tokens of one prompt at positions 0..T-1, q and k
+    out in bf16, optional cache write (request 0 of `cache`)."""
+    T = int(q_raw.shape[0])
+    lib = load_library()
+    _check(lib.flint_prefill_qk_norm_rope(_ptr(q_raw), _ptr(k_raw), _ptr(v_raw), _ptr(w_q), _ptr(w_k),
+                                          T, eps, theta, int(bool(apply_rope)), _ptr(q_out),
+                                          _ptr(k_out),
+                                          ctypes.byref(cache) if cache is not None else None,
+                                          _ptr(dev_err), _stream(stream)))
+    return q_out, k_out
+
+
+def flint_prefill_attn(q, k, v, sinks, window: int, out, dev_err=None, stream=None):
+    """Causal attention (with sinks) of a T-token prompt over itself:
+    q bf16 [T, 32, 128], k / v bf16 [T, 4, 128], out fp32 [T, 32, 128]."""
+    lib = load_library()
+    _check(lib.flint_prefill_attn(_ptr(q), _ptr(k), _ptr(v), int(q.shape[0]), _ptr(sinks), int(window),
+                                  _ptr(out), _ptr(dev_err), _stream(stream)))
+    return out
 
 
 def flint_attn_decode(q, cache: KVCache, seq_lens: Sequence[int], sinks, window: int, out,

@@ -36,7 +36,7 @@ BLOCK_SIZE = 64
 N_LAYERS = 49
 
 # workload ids used in seeds
-W_FULL_SMALL, W_SWA_100K, W_FULL_100K, W_STACK_100K, W_PAGED_BATCH = 0, 1, 2, 3, 4
+W_FULL_SMALL, W_SWA_100K, W_FULL_100K, W_STACK_100K, W_PAGED_BATCH, W_PREFILL = 0, 1, 2, 3, 4, 5
 
 # tensor ids inside a layer
 _T_Q, _T_K, _T_V, _T_WQ, _T_WK, _T_SINK, _T_KC, _T_VC = range(8)
@@ -240,3 +240,30 @@ def make_paged_batch(B: int = 32, lo: int = 4096, hi: int = 131072,
         k_pool=k, v_pool=v, block_table=table, seq_lens=list(seq_lens),
         sinks=f32_normal((NUM_Q_HEADS,), seed_for(workload, 0, _T_SINK)),
         k_scale=ks, v_scale=vs)
+
+
+@dataclasses.dataclass
+class PrefillInputs:
+    """The raw activations of one layer for a T-token prompt."""
+    q_raw: torch.Tensor        # bf16 [T,32,128]
+    k_raw: torch.Tensor        # bf16 [T,4,128]
+    v_raw: torch.Tensor        # bf16 [T,4,128]
+    w_q: torch.Tensor          # bf16 [128]
+    w_k: torch.Tensor          # bf16 [128]
+    sinks: torch.Tensor        # f32 [32]
+    window: int
+    rope: bool
+
+
+def make_prefill(T: int, window: int, workload: int = W_PREFILL, layer: int = 0) -> PrefillInputs:
+    """A prompt of T tokens for one layer (window 513 with RoPE, or 0 without),
+    with the value distributions of make_layer."""
+    s = lambda t: seed_for(workload, layer, t)  # noqa: E731
+    return PrefillInputs(
+        q_raw=bf16_normal((T, NUM_Q_HEADS, HEAD_DIM), s(_T_Q)),
+        k_raw=bf16_normal((T, NUM_KV_HEADS, HEAD_DIM), s(_T_K)),
+        v_raw=bf16_normal((T, NUM_KV_HEADS, HEAD_DIM), s(_T_V)),
+        w_q=bf16_normal((HEAD_DIM,), s(_T_WQ), 1.0, 0.1),
+        w_k=bf16_normal((HEAD_DIM,), s(_T_WK), 1.0, 0.1),
+        sinks=f32_normal((NUM_Q_HEADS,), s(_T_SINK)),
+        window=window, rope=window > 0)

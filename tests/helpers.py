@@ -16,8 +16,9 @@ def dev(t: torch.Tensor) -> torch.Tensor:
     return t.to("cuda", non_blocking=False).contiguous()
 
 
-def parity(got, want, what=""):
-    """Max-abs and relative-L2 bar over the whole output and per head."""
+def parity(got, want, what="", per_head=True):
+    """Max-abs and relative-L2 bar over the whole output and (per_head) for
+    every 128-value row."""
     got = np.asarray(got, np.float64).reshape(-1, want.shape[-1])
     want = np.asarray(want, np.float64).reshape(-1, want.shape[-1])
     assert np.isfinite(got).all(), f"{what}: non-finite output"
@@ -26,7 +27,8 @@ def parity(got, want, what=""):
     rel_head = np.linalg.norm(got - want, axis=1) / np.linalg.norm(want, axis=1)
     assert err.max() <= MAX_ABS, f"{what}: max abs err {err.max():.3e}"
     assert rel <= REL_L2, f"{what}: rel L2 err {rel:.3e}"
-    assert rel_head.max() <= REL_L2, f"{what}: worst head rel L2 {rel_head.max():.3e}"
+    if per_head:
+        assert rel_head.max() <= REL_L2, f"{what}: worst head rel L2 {rel_head.max():.3e}"
     return float(err.max()), float(rel)
 
 

@@ -117,6 +117,28 @@ def test_stack_and_prep_reject_bad_arguments_on_the_host():
     assert st == flint.FLINT_ERR_INVALID_ARG                        # slot 7 beyond capacity 4
 
 
+def test_prefill_rejects_bad_arguments_on_the_host():
+    lib = flint.load_library()
+    p = ctypes.c_void_p(0x10000)
+    eps, theta = ctypes.c_float(1e-6), ctypes.c_double(1e4)
+    E, U = flint.FLINT_ERR_INVALID_ARG, flint.FLINT_ERR_UNSUPPORTED
+    assert lib.flint_prefill_attn(p, p, p, 0, p, 0, p, None, None) == E              # T = 0
+    assert lib.flint_prefill_attn(p, p, p, flint.MAX_CONTEXT + 1, p, 0, p, None, None) == E
+    assert lib.flint_prefill_attn(p, p, p, 16, p, 100, p, None, None) == U           # window 100
+    assert lib.flint_prefill_attn(p, None, p, 16, p, 0, p, None, None) == E           # NULL k
+    assert lib.flint_prefill_attn(p, p, ctypes.c_void_p(0x10008), 16, p, 0, p, None, None) == E  # unaligned v
+    assert lib.flint_prefill_qk_norm_rope(p, p, p, p, p, 0, eps, theta, 1, p, p, None, None, None) == E
+    assert lib.flint_prefill_qk_norm_rope(p, p, p, p, p, 16, eps, theta, 2, p, p, None, None, None) == E
+    assert lib.flint_prefill_qk_norm_rope(p, p, p, p, p, 16, eps, theta, 1, None, None, None, None,
+                                          None) == E                                   # no output
+    c = _fake_cache(capacity=100)
+    assert lib.flint_prefill_qk_norm_rope(p, p, p, p, p, 101, eps, theta, 1, p, p, ctypes.byref(c), None,
+                                          None) == E                                   # 101 tokens, 100 slots
+    assert "capacity" in lib.flint_last_error().decode()
+    assert lib.flint_prefill_qk_norm_rope(p, p, None, p, p, 50, eps, theta, 1, p, p, ctypes.byref(c), None,
+                                          None) == E                                   # cache without v
+
+
 def test_workspace_bytes_bounds():
     assert flint.flint_attn_workspace_bytes(0, 148) == 0
     assert flint.flint_attn_workspace_bytes(65, 148) == 0
