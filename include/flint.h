@@ -290,9 +290,9 @@ flint_status flint_prefill_qk_norm_rope(const uint16_t* q_raw, const uint16_t* k
  *      qk_norm_rope's q_out and k_out, and v_raw)
  *   sinks  fp32 [32] (device, in); window  0 or FLINT_WINDOW
  *   out  fp32 [T][32][128] (device, out)
- * T in [1, FLINT_MAX_CONTEXT].  Products on bf16 tensor-core MMAs with fp32
- * accumulation; softmax in fp32.  Host-side errors only; dev_err is unused
- * and may be NULL. */
+ * T in [1, FLINT_MAX_CONTEXT].  Products on bf16 tensor-core MMAs (tcgen05)
+ * with fp32 accumulation; softmax in fp32.  A pipeline wait that runs past
+ * its time limit sets *dev_err = FLINT_ERR_TIMEOUT (dev_err may be NULL). */
 flint_status flint_prefill_attn(const uint16_t* q, const uint16_t* k, const uint16_t* v,
                                 int32_t T, const float* sinks, int32_t window, float* out,
                                 int32_t* dev_err, void* stream);

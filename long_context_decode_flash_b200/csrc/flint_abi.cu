@@ -634,9 +634,24 @@ flint_status flint_prefill_attn(const uint16_t* q, const uint16_t* k, const uint
     return fail(FLINT_ERR_UNSUPPORTED, "%s: window must be 0 or %d", who, kWindow);
   PrefillParams p;
   memset(&p, 0, sizeof p);
-  p.q = q;
-  p.k = k;
-  p.v = v;
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) return fail(FLINT_ERR_CUDA, "%s: cuTensorMapEncodeTiled is not available from the driver", who);
+  // [128 dims][heads][T tokens][1] bf16, 128-byte swizzle, boxes of 64 dims
+  auto encode = [&](CUtensorMap* map, const void* base, int heads, int box_heads, int box_tokens) {
+    const cuuint64_t dims[4] = {static_cast<cuuint64_t>(kDim), static_cast<cuuint64_t>(heads),
+                                static_cast<cuuint64_t>(T), 1};
+    const cuuint64_t strides[3] = {kDim * 2ull, static_cast<cuuint64_t>(heads) * kDim * 2ull,
+                                   static_cast<cuuint64_t>(T) * heads * kDim * 2ull};
+    const cuuint32_t box[4] = {64, static_cast<cuuint32_t>(box_heads), static_cast<cuuint32_t>(box_tokens), 1};
+    const cuuint32_t estr[4] = {1, 1, 1, 1};
+    return fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void*>(base), dims, strides, box, estr,
+              CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  };
+  if (encode(&p.q_map, q, kHeads, kGroup, 16) != CUDA_SUCCESS ||
+      encode(&p.k_map, k, kKvHeads, 1, 128) != CUDA_SUCCESS ||
+      encode(&p.v_map, v, kKvHeads, 1, 128) != CUDA_SUCCESS)
+    return fail(FLINT_ERR_CUDA, "%s: cuTensorMapEncodeTiled failed", who);
   p.sinks = sinks;
   p.out = out;
   p.dev_err = dev_err;

@@ -171,9 +171,10 @@ struct PrepParams {
 // out fp32 [T][32][128]; query t attends keys max(0, t - window + 1) .. t
 // (window > 0) or 0 .. t.
 struct PrefillParams {
-  const uint16_t* q;
-  const uint16_t* k;
-  const uint16_t* v;
+  // TMA maps, 128-byte swizzle, boxes of 64 dims:
+  //   q_map  [128 dims][32 heads][T tokens][1], box 64 x 8 heads x 16 tokens
+  //   k_map, v_map  [128 dims][4 heads][T tokens][1], box 64 x 1 x 128 tokens
+  CUtensorMap q_map, k_map, v_map;
   const float* sinks;
   float* out;
   int32_t* dev_err;

@@ -8,15 +8,23 @@
 // ("Day-0 Support for Flint on vLLM", hnkhoi.com, "Model architecture"; the
 // 8,192-token prefill of newruntime.com, "What happened").
 //
-// How: one CTA per (block of 16 query tokens, KV head g); warp w of the CTA
-// serves query head 8g + w, so the 8 heads of a GQA group share every K/V
-// tile.  64-token K and V tiles of the KV head stream through two shared-
-// memory stages with cp.async (16-byte chunks, XOR-swizzled so that ldmatrix
-// reads are conflict-free); blocks run from the last (longest) to the first.
-// Per tile and warp: S = Q K^T on bf16 mma.sync m16n8k16 (rows = the 16 query
-// tokens), the causal / window mask on boundary tiles, an fp32 online softmax
-// per row in log2 units, and O += P V with P split into bf16 hi and lo parts
-// (two products), so that P keeps ~16 bits.
+// How (5th-generation tensor cores, tcgen05): one CTA per (block of 16 query
+// tokens, KV head g).  Its 128 query rows are the 16 tokens x the 8 heads of
+// the group (row r = 8 * token + head), so every K/V tile serves all 8 heads.
+// Six warps:
+//   warp 4     TMA producer: the Q tile once, then 128-key K and V tiles
+//              through 3-stage rings (128-byte swizzle, two 64-dim boxes).
+//   warp 5     allocates the 512 TMEM columns; its lane 0 issues the MMAs:
+//              S = Q K^T (M 128, N 128, K 128) into one of two TMEM S buffers,
+//              and O += P V with P read from TMEM (bf16 hi and lo parts, two
+//              products) and V from shared memory (dims-major operand).
+//   warps 0-3  softmax, one thread per row (TMEM lane): S from TMEM, the
+//              causal / window mask on boundary tiles, an fp32 online softmax
+//              in log2 units whose running maximum moves only when a tile
+//              exceeds it by more than 2^8 (then O is rescaled in TMEM), P
+//              back to TMEM; at the end O, the sink and the store.
+// TMEM columns: S0 [0,128), S1 [128,256), P hi [256,320), P lo [320,384),
+// O [384,512).  Every wait is bounded; a timeout raises FLINT_ERR_TIMEOUT.
 #include <math.h>
 
 #include "flint_device.cuh"
@@ -25,198 +33,384 @@ namespace flint {
 
 namespace {
 
-constexpr int kPfQ = 16;                        // query tokens per CTA
-constexpr int kPfKv = 64;                       // key tokens per tile
-constexpr int kPfThreads = kGroup * 32;         // one warp per query head of the group
-constexpr int kPfRow = kDim * 2;                // bytes of one token's 128 dims of one KV head
-constexpr int kPfTile = kPfKv * kPfRow;         // 16 KiB
-constexpr int kPfStages = 2;
-constexpr size_t kPfSmem = static_cast<size_t>(kPfStages) * 2 * kPfTile;  // K and V: 64 KiB
+constexpr int kPq = 16;                    // query tokens per CTA
+constexpr int kRows = kPq * kGroup;        // 128 query rows (token, head)
+constexpr int kPkv = 128;                  // keys per tile
+constexpr int kKs = 3, kVs = 3;            // K and V ring stages
+constexpr int kPfThreads = 192;            // warps 0-3 softmax, 4 TMA, 5 MMA
+constexpr uint32_t kHalfBytes = kPkv * 128;            // one 64-dim box of a tile: 16 KiB
+constexpr uint32_t kTileBytes = 2 * kHalfBytes;        // 32 KiB
+constexpr uint32_t kQBytes = 2 * kRows * 128;          // 32 KiB
+constexpr uint32_t kOffK = kQBytes;
+constexpr uint32_t kOffV = kOffK + kKs * kTileBytes;
+constexpr uint32_t kOffBar = kOffV + kVs * kTileBytes;  // 229,376
+constexpr size_t kPfSmem = kOffBar + 256 + 1024;        // barriers, TMEM address, flags; alignment slack
 constexpr float kPfLog2e = 1.4426950408889634f;
 constexpr float kPfScale = static_cast<float>(1.4426950408889634 * 0.08838834764831845);
+constexpr float kTau = 8.0f;               // lazy-rescale threshold (log2 units)
+constexpr uint32_t kColS = 0, kColP = 256, kColPlo = 320, kColO = 384;
 
-__device__ __forceinline__ void cp_async16(uint32_t dst, const void* src, bool valid) {
-  // a chunk past the prompt is zero-filled (source size 0; the address stays in bounds)
-  asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(dst), "l"(src), "r"(valid ? 16 : 0)
+// Instruction descriptors (kind::f16): fp32 D, bf16 A and B, M 128, N 128;
+// S: both operands K-major; PV: B (V) dims-major.
+constexpr uint32_t kIdescS = (1u << 4) | (1u << 7) | (1u << 10) | ((kPkv >> 3) << 17) | ((128 >> 4) << 24);
+constexpr uint32_t kIdescPV = (1u << 4) | (1u << 7) | (1u << 10) | (1u << 16) | ((kDim >> 3) << 17) |
+                              ((128 >> 4) << 24);
+
+struct Bars {  // at kOffBar
+  uint64_t q_full;
+  uint64_t k_full[kKs], k_empty[kKs];
+  uint64_t v_full[kVs], v_empty[kVs];
+  uint64_t s_full[2];
+  uint64_t p_full;
+  uint64_t pv_done;
+  uint64_t mma_done;
+  uint32_t tmem_base;
+  int abort;
+};
+static_assert(sizeof(Bars) <= 256, "barrier block");
+
+// Shared-memory matrix descriptor, 128-byte swizzle (sm_100 version 1).
+__device__ __forceinline__ uint64_t sw128_desc(uint32_t saddr, uint32_t lbo, uint32_t sbo) {
+  return static_cast<uint64_t>((saddr >> 4) & 0x3FFFu) | (static_cast<uint64_t>((lbo >> 4) & 0x3FFFu) << 16) |
+         (static_cast<uint64_t>((sbo >> 4) & 0x3FFFu) << 32) | (1ull << 46) | (2ull << 61);
+}
+
+__device__ __forceinline__ void umma_ss(uint32_t d, uint64_t a, uint64_t b, uint32_t idesc, uint32_t acc) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d),
+      "l"(a), "l"(b), "r"(idesc), "r"(acc)
+      : "memory");
+}
+__device__ __forceinline__ void umma_ts(uint32_t d, uint32_t a_tmem, uint64_t b, uint32_t idesc, uint32_t acc) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}" ::"r"(d),
+      "r"(a_tmem), "l"(b), "r"(idesc), "r"(acc)
+      : "memory");
+}
+// Arrive once on `bar` when every tcgen05 operation this thread issued so far
+// has completed.
+__device__ __forceinline__ void umma_commit(uint32_t bar) {
+  asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(bar)
                : "memory");
 }
-__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
-template <int N>
-__device__ __forceinline__ void cp_async_wait() { asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory"); }
+__device__ __forceinline__ void tc_fence_before() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
+__device__ __forceinline__ void tc_fence_after() { asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory"); }
+__device__ __forceinline__ void tmem_wait_ld() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }
+__device__ __forceinline__ void tmem_wait_st() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
 
-// Loads tile j of KV head g (keys 64j .. 64j + 63) into stage buffers sK, sV:
-// row r, 16-byte chunk u goes to r * 256 + ((u ^ (r & 7)) << 4).
-__device__ __forceinline__ void load_tile(const PrefillParams& p, int g, int j, uint32_t sK, uint32_t sV) {
-  for (int ch = threadIdx.x; ch < kPfKv * (kPfRow / 16); ch += kPfThreads) {
-    const int r = ch >> 4, u = ch & 15;
-    const int key = j * kPfKv + r;
-    const bool valid = key < p.T;
-    const long long off = (static_cast<long long>(valid ? key : 0) * kKvHeads + g) * kDim + u * 8;
-    const uint32_t so = static_cast<uint32_t>(r * kPfRow + ((u ^ (r & 7)) << 4));
-    cp_async16(sK + so, p.k + off, valid);
-    cp_async16(sV + so, p.v + off, valid);
+#define FLINT_R8(i) "=r"(r[i]), "=r"(r[i + 1]), "=r"(r[i + 2]), "=r"(r[i + 3]), "=r"(r[i + 4]), \
+                    "=r"(r[i + 5]), "=r"(r[i + 6]), "=r"(r[i + 7])
+#define FLINT_W8(i) "r"(r[i]), "r"(r[i + 1]), "r"(r[i + 2]), "r"(r[i + 3]), "r"(r[i + 4]), \
+                    "r"(r[i + 5]), "r"(r[i + 6]), "r"(r[i + 7])
+
+// 32 consecutive columns of this warp's 32 lanes: lane i gets row i.
+__device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t (&r)[32]) {
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,"
+      "%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%32];"
+      : FLINT_R8(0), FLINT_R8(8), FLINT_R8(16), FLINT_R8(24)
+      : "r"(taddr));
+}
+__device__ __forceinline__ void tmem_st32(uint32_t taddr, const uint32_t (&r)[32]) {
+  asm volatile(
+      "tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,"
+      "%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31,%32};" ::"r"(taddr),
+      FLINT_W8(0), FLINT_W8(8), FLINT_W8(16), FLINT_W8(24)
+      : "memory");
+}
+
+// Bounded wait shared by all lanes of a warp: true only if every lane saw
+// the phase complete.
+__device__ __forceinline__ bool warp_wait(uint32_t bar, uint32_t parity, Bars* B) {
+  const bool ok = mbar_wait(bar, parity, &B->abort);
+  return __all_sync(0xffffffffu, ok);
+}
+
+__device__ __forceinline__ void raise_abort(const PrefillParams& p, Bars* B) {
+  if (!B->abort) report_error(p.dev_err, FLINT_ERR_TIMEOUT);
+  B->abort = 1;
+}
+
+struct Work {
+  int t0, g, j_first, n;
+  __device__ bool interior(int jj, int window) const {
+    const int k0 = (j_first + jj) * kPkv;
+    const int t_hi = t0 + kPq - 1;
+    return k0 + kPkv - 1 <= t0 && (window == 0 || k0 > t_hi - window);
+  }
+};
+
+__device__ __forceinline__ Work work_of(const PrefillParams& p) {
+  const int nblk = (p.T + kPq - 1) / kPq;
+  const int qb = nblk - 1 - static_cast<int>(blockIdx.x) / kKvHeads;  // longest blocks first
+  Work w;
+  w.g = static_cast<int>(blockIdx.x) % kKvHeads;
+  w.t0 = qb * kPq;
+  const int t_last = min(w.t0 + kPq - 1, p.T - 1);
+  w.j_first = p.window > 0 ? max(0, w.t0 - (p.window - 1)) / kPkv : 0;
+  w.n = t_last / kPkv - w.j_first + 1;
+  return w;
+}
+
+__device__ void run_tma(const PrefillParams& p, const Work& w, uint8_t* smem, Bars* B) {
+  const uint32_t base = smem_u32(smem);
+  mbar_expect_tx(smem_u32(&B->q_full), kQBytes);
+  tma_load_4d(base, &p.q_map, smem_u32(&B->q_full), 0, w.g * kGroup, w.t0, 0);
+  tma_load_4d(base + kRows * 128, &p.q_map, smem_u32(&B->q_full), 64, w.g * kGroup, w.t0, 0);
+  for (int jj = 0; jj < w.n; ++jj) {
+    const int k0 = (w.j_first + jj) * kPkv;
+    const int sk = jj % kKs, sv = jj % kVs;
+    if (jj >= kKs && !mbar_wait(smem_u32(&B->k_empty[sk]), static_cast<uint32_t>(jj / kKs - 1) & 1u, &B->abort)) {
+      raise_abort(p, B);
+      return;
+    }
+    const uint32_t dk = base + kOffK + sk * kTileBytes;
+    mbar_expect_tx(smem_u32(&B->k_full[sk]), kTileBytes);
+    tma_load_4d(dk, &p.k_map, smem_u32(&B->k_full[sk]), 0, w.g, k0, 0);
+    tma_load_4d(dk + kHalfBytes, &p.k_map, smem_u32(&B->k_full[sk]), 64, w.g, k0, 0);
+    if (jj >= kVs && !mbar_wait(smem_u32(&B->v_empty[sv]), static_cast<uint32_t>(jj / kVs - 1) & 1u, &B->abort)) {
+      raise_abort(p, B);
+      return;
+    }
+    const uint32_t dv = base + kOffV + sv * kTileBytes;
+    mbar_expect_tx(smem_u32(&B->v_full[sv]), kTileBytes);
+    tma_load_4d(dv, &p.v_map, smem_u32(&B->v_full[sv]), 0, w.g, k0, 0);
+    tma_load_4d(dv + kHalfBytes, &p.v_map, smem_u32(&B->v_full[sv]), 64, w.g, k0, 0);
+  }
+}
+
+// After an abort: let the copies still in flight land before the CTA's shared
+// memory goes away (bounded; the last kKs K and kVs V phases are the only ones
+// that can be pending).  A normal run returns at once.
+__device__ void drain_tma(const Work& w, Bars* B) {
+  const unsigned long long t0 = globaltimer_ns();
+  auto wait = [&](uint32_t bar, uint32_t parity) {
+    while (!mbar_try_wait(bar, parity))
+      if (globaltimer_ns() - t0 > kWaitLimitNs) return;
+  };
+  wait(smem_u32(&B->q_full), 0);
+  for (int jj = max(0, w.n - kKs); jj < w.n; ++jj)
+    wait(smem_u32(&B->k_full[jj % kKs]), static_cast<uint32_t>(jj / kKs) & 1u);
+  for (int jj = max(0, w.n - kVs); jj < w.n; ++jj)
+    wait(smem_u32(&B->v_full[jj % kVs]), static_cast<uint32_t>(jj / kVs) & 1u);
+}
+
+// S[jj & 1] = Q K_jj^T: 8 MMAs of K = 16 dims (32 bytes inside a swizzled
+// 128-byte row; the second 64 dims in the second box).
+__device__ __forceinline__ bool issue_s(const PrefillParams& p, int jj, uint32_t base, uint32_t tmem, Bars* B) {
+  const int sk = jj % kKs;
+  if (!mbar_wait(smem_u32(&B->k_full[sk]), static_cast<uint32_t>(jj / kKs) & 1u, &B->abort)) return false;
+  tc_fence_after();
+  const uint32_t qa = base, kb = base + kOffK + sk * kTileBytes;
+#pragma unroll
+  for (int kk = 0; kk < 8; ++kk) {
+    const uint32_t off = (kk >> 2) * (kRows * 128) + (kk & 3) * 32;
+    const uint32_t offk = (kk >> 2) * kHalfBytes + (kk & 3) * 32;
+    umma_ss(tmem + kColS + (jj & 1) * kPkv, sw128_desc(qa + off, 16, 1024), sw128_desc(kb + offk, 16, 1024),
+            kIdescS, kk > 0 ? 1u : 0u);
+  }
+  umma_commit(smem_u32(&B->k_empty[sk]));
+  umma_commit(smem_u32(&B->s_full[jj & 1]));
+  return true;
+}
+
+__device__ void run_mma(const PrefillParams& p, const Work& w, uint32_t base, uint32_t tmem, Bars* B) {
+  bool ok = mbar_wait(smem_u32(&B->q_full), 0, &B->abort);
+  if (ok) ok = issue_s(p, 0, base, tmem, B);
+  if (ok && w.n > 1) ok = issue_s(p, 1, base, tmem, B);
+  for (int jj = 0; ok && jj < w.n; ++jj) {
+    const int sv = jj % kVs;
+    ok = mbar_wait(smem_u32(&B->p_full), static_cast<uint32_t>(jj) & 1u, &B->abort) &&
+         mbar_wait(smem_u32(&B->v_full[sv]), static_cast<uint32_t>(jj / kVs) & 1u, &B->abort);
+    if (!ok) break;
+    tc_fence_after();
+    const uint32_t vb = base + kOffV + sv * kTileBytes;
+    // O += P V: K = 16 keys per MMA (rows 16kk.. of both 64-dim boxes)
+#pragma unroll
+    for (int part = 0; part < 2; ++part)
+#pragma unroll
+      for (int kk = 0; kk < 8; ++kk)
+        umma_ts(tmem + kColO, tmem + (part ? kColPlo : kColP) + kk * 8,
+                sw128_desc(vb + kk * 16 * 128, kHalfBytes, 1024), kIdescPV, (jj > 0 || part > 0 || kk > 0) ? 1u : 0u);
+    umma_commit(smem_u32(&B->v_empty[sv]));
+    umma_commit(smem_u32(&B->pv_done));
+    if (jj + 2 < w.n) ok = issue_s(p, jj + 2, base, tmem, B);
+  }
+  if (!ok) raise_abort(p, B);
+  // let every issued MMA finish before the CTA ends (its TMEM is freed)
+  umma_commit(smem_u32(&B->mma_done));
+  const unsigned long long t0 = globaltimer_ns();
+  while (!mbar_try_wait(smem_u32(&B->mma_done), 0)) {
+    if (globaltimer_ns() - t0 > kWaitLimitNs) break;
+  }
+}
+
+__device__ void run_softmax(const PrefillParams& p, const Work& w, uint32_t tmem, Bars* B, int warp, int lane) {
+  const int r = warp * 32 + lane;         // TMEM lane = query row
+  const int t = w.t0 + (r >> 3);          // its token
+  const int h = w.g * kGroup + (r & 7);   // its query head
+  const uint32_t lane_base = tmem + (static_cast<uint32_t>(warp * 32) << 16);
+  float m = -INFINITY, l = 0.f;
+  bool ok = true;
+  for (int jj = 0; jj < w.n; ++jj) {
+    if (!warp_wait(smem_u32(&B->s_full[jj & 1]), static_cast<uint32_t>(jj >> 1) & 1u, B)) {
+      ok = false;
+      break;
+    }
+    tc_fence_after();
+    float s[kPkv];
+#pragma unroll
+    for (int c = 0; c < kPkv / 32; ++c) {
+      uint32_t v[32];
+      tmem_ld32(lane_base + kColS + (jj & 1) * kPkv + 32 * c, v);
+      tmem_wait_ld();
+#pragma unroll
+      for (int i = 0; i < 32; ++i) s[32 * c + i] = __uint_as_float(v[i]) * kPfScale;
+    }
+    if (!w.interior(jj, p.window)) {
+      const int k0 = (w.j_first + jj) * kPkv;
+#pragma unroll
+      for (int i = 0; i < kPkv; ++i) {
+        const int key = k0 + i;
+        if (key > t || (p.window > 0 && key <= t - p.window)) s[i] = -INFINITY;
+      }
+    }
+    float mx = s[0];
+#pragma unroll
+    for (int i = 1; i < kPkv; ++i) mx = fmaxf(mx, s[i]);
+    const bool need = mx > m + kTau || (m == -INFINITY && mx > -INFINITY);
+    float factor = 1.f;
+    if (need) {
+      factor = (m == -INFINITY) ? 0.f : exp2f(m - mx);
+      m = mx;
+      l *= factor;
+    }
+    const float mu = (m == -INFINITY) ? 0.f : m;
+    uint32_t hi[kPkv / 2], lo[kPkv / 2];
+#pragma unroll
+    for (int c = 0; c < kPkv / 2; ++c) {
+      const float p0 = exp2f(s[2 * c] - mu), p1 = exp2f(s[2 * c + 1] - mu);
+      l += p0 + p1;
+      split_bf16x2(p0, p1, hi[c], lo[c]);
+    }
+    if (jj > 0) {
+      // P's columns and O are free once the previous tile's PV has completed
+      if (!warp_wait(smem_u32(&B->pv_done), static_cast<uint32_t>(jj - 1) & 1u, B)) {
+        ok = false;
+        break;
+      }
+      tc_fence_after();
+      if (__any_sync(0xffffffffu, need)) {
+#pragma unroll
+        for (int c = 0; c < kDim / 32; ++c) {
+          uint32_t v[32];
+          tmem_ld32(lane_base + kColO + 32 * c, v);
+          tmem_wait_ld();
+#pragma unroll
+          for (int i = 0; i < 32; ++i) v[i] = __float_as_uint(__uint_as_float(v[i]) * factor);
+          tmem_st32(lane_base + kColO + 32 * c, v);
+        }
+      }
+    }
+#pragma unroll
+    for (int c = 0; c < 2; ++c) {
+      uint32_t v[32];
+#pragma unroll
+      for (int i = 0; i < 32; ++i) v[i] = hi[32 * c + i];
+      tmem_st32(lane_base + kColP + 32 * c, v);
+#pragma unroll
+      for (int i = 0; i < 32; ++i) v[i] = lo[32 * c + i];
+      tmem_st32(lane_base + kColPlo + 32 * c, v);
+    }
+    tmem_wait_st();
+    tc_fence_before();
+    __syncwarp();
+    if (lane == 0) mbar_arrive(smem_u32(&B->p_full));
+  }
+  if (ok && !warp_wait(smem_u32(&B->pv_done), static_cast<uint32_t>(w.n - 1) & 1u, B)) ok = false;
+  if (!ok) {
+    if (lane == 0) raise_abort(p, B);
+    return;
+  }
+  tc_fence_after();
+  // out = O e^(m - M) / (l e^(m - M) + e^(sink - M)), M = max(m, sink), in log2 units
+  const float s2 = p.sinks[h] * kPfLog2e;
+  const float M = fmaxf(m, s2);
+  const float a = (m == -INFINITY) ? 0.f : exp2f(m - M);
+  const float sc = a / (l * a + exp2f(s2 - M));
+  float* out = p.out + (static_cast<long long>(t < p.T ? t : 0) * kHeads + h) * kDim;
+#pragma unroll
+  for (int c = 0; c < kDim / 32; ++c) {
+    uint32_t v[32];
+    tmem_ld32(lane_base + kColO + 32 * c, v);
+    tmem_wait_ld();
+    if (t < p.T) {
+#pragma unroll
+      for (int i = 0; i < 32; i += 4)
+        *reinterpret_cast<float4*>(out + 32 * c + i) =
+            make_float4(__uint_as_float(v[i]) * sc, __uint_as_float(v[i + 1]) * sc,
+                        __uint_as_float(v[i + 2]) * sc, __uint_as_float(v[i + 3]) * sc);
+    }
   }
 }
 
 __global__ void __launch_bounds__(kPfThreads, 1) prefill_kernel(const __grid_constant__ PrefillParams p) {
-  extern __shared__ __align__(1024) uint8_t pf_smem[];
+  extern __shared__ uint8_t pf_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(pf_raw) + 1023) & ~uintptr_t(1023));
+  Bars* B = reinterpret_cast<Bars*>(smem + kOffBar);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int gq = lane >> 2, c = lane & 3, l7 = lane & 7;
-  const int qb = gridDim.x - 1 - blockIdx.x;  // longest blocks first
-  const int g = blockIdx.y;
-  const int h = g * kGroup + warp;
-  const int t0 = qb * kPfQ;
-  const int ta = t0 + gq, tb = t0 + gq + 8;    // this thread's two query rows
+  const Work w = work_of(p);
 
-  // Q fragments (A operand rows: tokens ta and tb), straight from global memory
-  uint32_t qa[8][4];
-#pragma unroll
-  for (int kk = 0; kk < 8; ++kk) {
-    const int d0 = 16 * kk + 2 * c;
-    const uint16_t* qa_row = p.q + (static_cast<long long>(ta < p.T ? ta : 0) * kHeads + h) * kDim;
-    const uint16_t* qb_row = p.q + (static_cast<long long>(tb < p.T ? tb : 0) * kHeads + h) * kDim;
-    qa[kk][0] = ta < p.T ? *reinterpret_cast<const uint32_t*>(qa_row + d0) : 0u;
-    qa[kk][1] = tb < p.T ? *reinterpret_cast<const uint32_t*>(qb_row + d0) : 0u;
-    qa[kk][2] = ta < p.T ? *reinterpret_cast<const uint32_t*>(qa_row + d0 + 8) : 0u;
-    qa[kk][3] = tb < p.T ? *reinterpret_cast<const uint32_t*>(qb_row + d0 + 8) : 0u;
+  if (threadIdx.x == 0) {
+    mbar_init(smem_u32(&B->q_full), 1);
+    for (int s = 0; s < kKs; ++s) {
+      mbar_init(smem_u32(&B->k_full[s]), 1);
+      mbar_init(smem_u32(&B->k_empty[s]), 1);
+    }
+    for (int s = 0; s < kVs; ++s) {
+      mbar_init(smem_u32(&B->v_full[s]), 1);
+      mbar_init(smem_u32(&B->v_empty[s]), 1);
+    }
+    mbar_init(smem_u32(&B->s_full[0]), 1);
+    mbar_init(smem_u32(&B->s_full[1]), 1);
+    mbar_init(smem_u32(&B->p_full), 4);
+    mbar_init(smem_u32(&B->pv_done), 1);
+    mbar_init(smem_u32(&B->mma_done), 1);
+    B->abort = 0;
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
   }
-
-  const int t_last = min(t0 + kPfQ - 1, p.T - 1);
-  const int j_first = p.window > 0 ? max(0, t0 - (p.window - 1)) / kPfKv : 0;
-  const int j_last = t_last / kPfKv;
-  const uint32_t base = smem_u32(pf_smem);
-
-  float o[16][4];
-#pragma unroll
-  for (int n = 0; n < 16; ++n)
-#pragma unroll
-    for (int e = 0; e < 4; ++e) o[n][e] = 0.f;
-  float m_a = -INFINITY, m_b = -INFINITY, l_a = 0.f, l_b = 0.f;
-
-  load_tile(p, g, j_first, base, base + kPfTile);
-  cp_async_commit();
-  for (int j = j_first; j <= j_last; ++j) {
-    const int st = (j - j_first) & 1;
-    if (j < j_last) {
-      const uint32_t nb = base + static_cast<uint32_t>(((j + 1 - j_first) & 1) * 2 * kPfTile);
-      load_tile(p, g, j + 1, nb, nb + kPfTile);
-      cp_async_commit();
-      cp_async_wait<1>();
-    } else {
-      cp_async_wait<0>();
-    }
-    __syncthreads();
-    const uint32_t sK = base + static_cast<uint32_t>(st * 2 * kPfTile), sV = sK + kPfTile;
-
-    // S = Q K^T for the tile's 64 keys: 8 n-tiles of 8 keys
-    float s[8][4];
-#pragma unroll
-    for (int nt = 0; nt < 8; ++nt) {
-#pragma unroll
-      for (int e = 0; e < 4; ++e) s[nt][e] = 0.f;
-      const uint32_t row = sK + (8 * nt + l7) * kPfRow;
-#pragma unroll
-      for (int kk = 0; kk < 8; kk += 2) {
-        const int u = 2 * kk + (lane >> 3);  // 16-byte chunk: dims 8u .. 8u + 7
-        uint32_t b0, b1, b2, b3;
-        ldsm_x4(row + ((u ^ l7) << 4), b0, b1, b2, b3);
-        mma_bf16_16816(s[nt], qa[kk], b0, b1);
-        mma_bf16_16816(s[nt], qa[kk + 1], b2, b3);
-      }
-    }
-    // scale to log2 units; mask keys past a row's position, before its window or past the prompt
-    const int k0 = j * kPfKv;
-    const bool interior = (k0 + kPfKv - 1 <= t0) && (k0 + kPfKv <= p.T) &&
-                          (p.window == 0 || k0 > t_last - p.window);
-#pragma unroll
-    for (int nt = 0; nt < 8; ++nt)
-#pragma unroll
-      for (int e = 0; e < 4; ++e) {
-        s[nt][e] *= kPfScale;
-        if (!interior) {
-          const int key = k0 + 8 * nt + 2 * c + (e & 1);
-          const int t = (e < 2) ? ta : tb;
-          const bool ok = key <= t && key < p.T && (p.window == 0 || key > t - p.window);
-          if (!ok) s[nt][e] = -INFINITY;
-        }
-      }
-    // online softmax, rows ta (e = 0, 1) and tb (e = 2, 3)
-    float mx_a = -INFINITY, mx_b = -INFINITY;
-#pragma unroll
-    for (int nt = 0; nt < 8; ++nt) {
-      mx_a = fmaxf(mx_a, fmaxf(s[nt][0], s[nt][1]));
-      mx_b = fmaxf(mx_b, fmaxf(s[nt][2], s[nt][3]));
-    }
-    mx_a = fmaxf(mx_a, __shfl_xor_sync(0xffffffffu, mx_a, 1));
-    mx_a = fmaxf(mx_a, __shfl_xor_sync(0xffffffffu, mx_a, 2));
-    mx_b = fmaxf(mx_b, __shfl_xor_sync(0xffffffffu, mx_b, 1));
-    mx_b = fmaxf(mx_b, __shfl_xor_sync(0xffffffffu, mx_b, 2));
-    const float mn_a = fmaxf(m_a, mx_a), mn_b = fmaxf(m_b, mx_b);
-    const float al_a = (m_a == -INFINITY) ? 0.f : exp2f(m_a - mn_a);
-    const float al_b = (m_b == -INFINITY) ? 0.f : exp2f(m_b - mn_b);
-    m_a = mn_a;
-    m_b = mn_b;
-    l_a *= al_a;
-    l_b *= al_b;
-#pragma unroll
-    for (int n = 0; n < 16; ++n) {
-      o[n][0] *= al_a;
-      o[n][1] *= al_a;
-      o[n][2] *= al_b;
-      o[n][3] *= al_b;
-    }
-    const float mu_a = (m_a == -INFINITY) ? 0.f : m_a, mu_b = (m_b == -INFINITY) ? 0.f : m_b;
-#pragma unroll
-    for (int nt = 0; nt < 8; ++nt) {
-      s[nt][0] = exp2f(s[nt][0] - mu_a);
-      s[nt][1] = exp2f(s[nt][1] - mu_a);
-      s[nt][2] = exp2f(s[nt][2] - mu_b);
-      s[nt][3] = exp2f(s[nt][3] - mu_b);
-      l_a += s[nt][0] + s[nt][1];
-      l_b += s[nt][2] + s[nt][3];
-    }
-
-    // O += P V: 4 k-steps of 16 keys, 16 n-tiles of 8 dims, P as bf16 hi + lo
-#pragma unroll
-    for (int kt = 0; kt < 4; ++kt) {
-      uint32_t ph[4], pl[4];
-      split_bf16x2(s[2 * kt][0], s[2 * kt][1], ph[0], pl[0]);
-      split_bf16x2(s[2 * kt][2], s[2 * kt][3], ph[1], pl[1]);
-      split_bf16x2(s[2 * kt + 1][0], s[2 * kt + 1][1], ph[2], pl[2]);
-      split_bf16x2(s[2 * kt + 1][2], s[2 * kt + 1][3], ph[3], pl[3]);
-      const uint32_t rowv = sV + (16 * kt + ((lane >> 3) & 1) * 8 + l7) * kPfRow;
-#pragma unroll
-      for (int np = 0; np < 8; ++np) {
-        const int u = 2 * np + (lane >> 4);
-        uint32_t v0, v1, v2, v3;
-        ldsm_x4_t(rowv + ((u ^ l7) << 4), v0, v1, v2, v3);
-        mma_bf16_16816(o[2 * np], ph, v0, v1);
-        mma_bf16_16816(o[2 * np], pl, v0, v1);
-        mma_bf16_16816(o[2 * np + 1], ph, v2, v3);
-        mma_bf16_16816(o[2 * np + 1], pl, v2, v3);
-      }
-    }
-    __syncthreads();  // the stage is refilled two tiles later
+  if (warp == 4 && lane == 0) {
+    prefetch_tensormap(&p.q_map);
+    prefetch_tensormap(&p.k_map);
+    prefetch_tensormap(&p.v_map);
   }
-
-  // finish: quad-reduce l, fold in the sink, write both rows
-  l_a += __shfl_xor_sync(0xffffffffu, l_a, 1);
-  l_a += __shfl_xor_sync(0xffffffffu, l_a, 2);
-  l_b += __shfl_xor_sync(0xffffffffu, l_b, 1);
-  l_b += __shfl_xor_sync(0xffffffffu, l_b, 2);
-  const float s2 = p.sinks[h] * kPfLog2e;
-  const float Ma = fmaxf(m_a, s2), Mb = fmaxf(m_b, s2);
-  const float aa = (m_a == -INFINITY) ? 0.f : exp2f(m_a - Ma), ab = (m_b == -INFINITY) ? 0.f : exp2f(m_b - Mb);
-  const float sca = aa / (l_a * aa + exp2f(s2 - Ma)), scb = ab / (l_b * ab + exp2f(s2 - Mb));
-  if (ta < p.T) {
-    float* out = p.out + (static_cast<long long>(ta) * kHeads + h) * kDim + 2 * c;
-#pragma unroll
-    for (int n = 0; n < 16; ++n) *reinterpret_cast<float2*>(out + 8 * n) = make_float2(o[n][0] * sca, o[n][1] * sca);
+  if (warp == 5) {
+    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], 512;" ::"r"(smem_u32(&B->tmem_base))
+                 : "memory");
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
   }
-  if (tb < p.T) {
-    float* out = p.out + (static_cast<long long>(tb) * kHeads + h) * kDim + 2 * c;
-#pragma unroll
-    for (int n = 0; n < 16; ++n) *reinterpret_cast<float2*>(out + 8 * n) = make_float2(o[n][2] * scb, o[n][3] * scb);
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = B->tmem_base;
+
+  if (warp < 4) {
+    run_softmax(p, w, tmem, B, warp, lane);
+  } else if (warp == 4) {
+    if (lane == 0) run_tma(p, w, smem, B);
+  } else if (lane == 0) {
+    run_mma(p, w, smem_u32(smem), tmem, B);
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 4 && lane == 0 && B->abort) drain_tma(w, B);
+  if (warp == 5) {
+    __syncwarp();
+    tc_fence_after();
+    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, 512;" ::"r"(tmem) : "memory");
   }
 }
 
@@ -233,7 +427,7 @@ cudaError_t launch_prefill(const PrefillParams& p, cudaStream_t stream) {
     if (e != cudaSuccess) return e;
     configured_device = dev;
   }
-  const dim3 grid((p.T + kPfQ - 1) / kPfQ, kKvHeads);
+  const int grid = (p.T + kPq - 1) / kPq * kKvHeads;
   prefill_kernel<<<grid, kPfThreads, kPfSmem, stream>>>(p);
   return cudaGetLastError();
 }
