@@ -11,18 +11,23 @@
 // How (5th-generation tensor cores, tcgen05): one CTA per (block of 16 query
 // tokens, KV head g).  Its 128 query rows are the 16 tokens x the 8 heads of
 // the group (row r = 8 * token + head), so every K/V tile serves all 8 heads.
-// Six warps:
-//   warp 4     TMA producer: the Q tile once, then 128-key K and V tiles
-//              through 3-stage rings (128-byte swizzle, two 64-dim boxes).
-//   warp 5     allocates the 512 TMEM columns; its lane 0 issues the MMAs:
+// Ten warps:
+//   warp 8     TMA producer: the Q tile once, then 128-key K and V tiles
+//              through 3- and 2-stage rings (128-byte swizzle, two 64-dim
+//              boxes per tile).
+//   warp 9     allocates the 512 TMEM columns; its lane 0 issues the MMAs:
 //              S = Q K^T (M 128, N 128, K 128) into one of two TMEM S buffers,
 //              and O += P V with P read from TMEM (bf16 hi and lo parts, two
 //              products) and V from shared memory (dims-major operand).
-//   warps 0-3  softmax, one thread per row (TMEM lane): S from TMEM, the
-//              causal / window mask on boundary tiles, an fp32 online softmax
-//              in log2 units whose running maximum moves only when a tile
-//              exceeds it by more than 2^8 (then O is rescaled in TMEM), P
-//              back to TMEM; at the end O, the sink and the store.
+//   warps 0-7  softmax in two warpgroups; thread (wg, r) owns row r (TMEM
+//              lane r) and the 64 keys 64 wg .. 64 wg + 63 of every tile, and
+//              the 64 output dims 64 wg .. 64 wg + 63.  Per tile: S from TMEM,
+//              the causal / window mask on boundary tiles, the row maximum
+//              exchanged between the two warpgroups through shared memory, an
+//              fp32 online softmax in log2 units whose running maximum moves
+//              only when a tile exceeds it by more than 2^8 (then O is
+//              rescaled in TMEM), P back to TMEM; at the end O, the sink and
+//              the store.
 // TMEM columns: S0 [0,128), S1 [128,256), P hi [256,320), P lo [320,384),
 // O [384,512).  Every wait is bounded; a timeout raises FLINT_ERR_TIMEOUT.
 #include <math.h>
@@ -36,14 +41,17 @@ namespace {
 constexpr int kPq = 16;                    // query tokens per CTA
 constexpr int kRows = kPq * kGroup;        // 128 query rows (token, head)
 constexpr int kPkv = 128;                  // keys per tile
-constexpr int kKs = 3, kVs = 3;            // K and V ring stages
-constexpr int kPfThreads = 192;            // warps 0-3 softmax, 4 TMA, 5 MMA
+constexpr int kKs = 3, kVs = 2;            // K and V ring stages
+constexpr int kSoftWarps = 8;              // two warpgroups
+constexpr int kTmaWarp = 8, kMmaWarp = 9;
+constexpr int kPfThreads = 320;
 constexpr uint32_t kHalfBytes = kPkv * 128;            // one 64-dim box of a tile: 16 KiB
 constexpr uint32_t kTileBytes = 2 * kHalfBytes;        // 32 KiB
 constexpr uint32_t kQBytes = 2 * kRows * 128;          // 32 KiB
 constexpr uint32_t kOffK = kQBytes;
 constexpr uint32_t kOffV = kOffK + kKs * kTileBytes;
-constexpr uint32_t kOffBar = kOffV + kVs * kTileBytes;  // 229,376
+constexpr uint32_t kOffRed = kOffV + kVs * kTileBytes;  // row-maximum exchange [2 tiles][2 wg][128]
+constexpr uint32_t kOffBar = kOffRed + 2 * 2 * kRows * 4;
 constexpr size_t kPfSmem = kOffBar + 256 + 1024;        // barriers, TMEM address, flags; alignment slack
 constexpr float kPfLog2e = 1.4426950408889634f;
 constexpr float kPfScale = static_cast<float>(1.4426950408889634 * 0.08838834764831845);
@@ -64,6 +72,8 @@ struct Bars {  // at kOffBar
   uint64_t p_full;
   uint64_t pv_done;
   uint64_t mma_done;
+  uint64_t red_full[2];   // both softmax warpgroups wrote their row maxima (per tile parity)
+  uint64_t l_full;        // ... their row sums (once, at the end)
   uint32_t tmem_base;
   int abort;
 };
@@ -119,6 +129,12 @@ __device__ __forceinline__ void tmem_st32(uint32_t taddr, const uint32_t (&r)[32
       "%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31,%32};" ::"r"(taddr),
       FLINT_W8(0), FLINT_W8(8), FLINT_W8(16), FLINT_W8(24)
       : "memory");
+}
+
+__device__ __forceinline__ float ex2(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
 }
 
 // Bounded wait shared by all lanes of a warp: true only if every lane saw
@@ -247,54 +263,72 @@ __device__ void run_mma(const PrefillParams& p, const Work& w, uint32_t base, ui
   }
 }
 
-__device__ void run_softmax(const PrefillParams& p, const Work& w, uint32_t tmem, Bars* B, int warp, int lane) {
-  const int r = warp * 32 + lane;         // TMEM lane = query row
+__device__ void run_softmax(const PrefillParams& p, const Work& w, uint32_t tmem, uint8_t* smem, Bars* B,
+                            int warp, int lane) {
+  const int wg = warp >> 2;               // key half of every tile, dims half of O
+  const int r = (warp & 3) * 32 + lane;   // TMEM lane = query row
   const int t = w.t0 + (r >> 3);          // its token
   const int h = w.g * kGroup + (r & 7);   // its query head
-  const uint32_t lane_base = tmem + (static_cast<uint32_t>(warp * 32) << 16);
-  float m = -INFINITY, l = 0.f;
+  const uint32_t lane_base = tmem + (static_cast<uint32_t>((warp & 3) * 32) << 16);
+  float* red = reinterpret_cast<float*>(smem + kOffRed);  // [tile parity][wg][row]
+  float m = -INFINITY, l = 0.f;           // m in log2 units
   bool ok = true;
+  constexpr int kH = kPkv / 2;            // keys of this thread per tile
   for (int jj = 0; jj < w.n; ++jj) {
     if (!warp_wait(smem_u32(&B->s_full[jj & 1]), static_cast<uint32_t>(jj >> 1) & 1u, B)) {
       ok = false;
       break;
     }
     tc_fence_after();
-    float s[kPkv];
+    float s[kH];  // raw scores q.k
 #pragma unroll
-    for (int c = 0; c < kPkv / 32; ++c) {
+    for (int c = 0; c < kH / 32; ++c) {
       uint32_t v[32];
-      tmem_ld32(lane_base + kColS + (jj & 1) * kPkv + 32 * c, v);
+      tmem_ld32(lane_base + kColS + (jj & 1) * kPkv + kH * wg + 32 * c, v);
       tmem_wait_ld();
 #pragma unroll
-      for (int i = 0; i < 32; ++i) s[32 * c + i] = __uint_as_float(v[i]) * kPfScale;
+      for (int i = 0; i < 32; ++i) s[32 * c + i] = __uint_as_float(v[i]);
     }
     if (!w.interior(jj, p.window)) {
-      const int k0 = (w.j_first + jj) * kPkv;
+      const int k0 = (w.j_first + jj) * kPkv + kH * wg;
 #pragma unroll
-      for (int i = 0; i < kPkv; ++i) {
+      for (int i = 0; i < kH; ++i) {
         const int key = k0 + i;
         if (key > t || (p.window > 0 && key <= t - p.window)) s[i] = -INFINITY;
       }
     }
-    float mx = s[0];
+    float mq[8];
 #pragma unroll
-    for (int i = 1; i < kPkv; ++i) mx = fmaxf(mx, s[i]);
+    for (int q = 0; q < 8; ++q) mq[q] = s[q];
+#pragma unroll
+    for (int i = 8; i < kH; ++i) mq[i & 7] = fmaxf(mq[i & 7], s[i]);
+    float mh = fmaxf(fmaxf(fmaxf(mq[0], mq[1]), fmaxf(mq[2], mq[3])), fmaxf(fmaxf(mq[4], mq[5]), fmaxf(mq[6], mq[7])));
+    // exchange the half-row maxima (every thread arrives; bounded wait)
+    float* slot = red + (jj & 1) * 2 * kRows;
+    slot[wg * kRows + r] = mh;
+    mbar_arrive(smem_u32(&B->red_full[jj & 1]));
+    if (!warp_wait(smem_u32(&B->red_full[jj & 1]), static_cast<uint32_t>(jj >> 1) & 1u, B)) {
+      ok = false;
+      break;
+    }
+    const float mx = fmaxf(slot[r], slot[kRows + r]) * kPfScale;  // the row's tile maximum, log2 units
     const bool need = mx > m + kTau || (m == -INFINITY && mx > -INFINITY);
     float factor = 1.f;
     if (need) {
-      factor = (m == -INFINITY) ? 0.f : exp2f(m - mx);
+      factor = (m == -INFINITY) ? 0.f : ex2(m - mx);
       m = mx;
       l *= factor;
     }
     const float mu = (m == -INFINITY) ? 0.f : m;
-    uint32_t hi[kPkv / 2], lo[kPkv / 2];
+    uint32_t hi[kH / 2], lo[kH / 2];
+    float ls[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-    for (int c = 0; c < kPkv / 2; ++c) {
-      const float p0 = exp2f(s[2 * c] - mu), p1 = exp2f(s[2 * c + 1] - mu);
-      l += p0 + p1;
+    for (int c = 0; c < kH / 2; ++c) {
+      const float p0 = ex2(fmaf(s[2 * c], kPfScale, -mu)), p1 = ex2(fmaf(s[2 * c + 1], kPfScale, -mu));
+      ls[c & 3] += p0 + p1;
       split_bf16x2(p0, p1, hi[c], lo[c]);
     }
+    l += (ls[0] + ls[1]) + (ls[2] + ls[3]);
     if (jj > 0) {
       // P's columns and O are free once the previous tile's PV has completed
       if (!warp_wait(smem_u32(&B->pv_done), static_cast<uint32_t>(jj - 1) & 1u, B)) {
@@ -304,32 +338,31 @@ __device__ void run_softmax(const PrefillParams& p, const Work& w, uint32_t tmem
       tc_fence_after();
       if (__any_sync(0xffffffffu, need)) {
 #pragma unroll
-        for (int c = 0; c < kDim / 32; ++c) {
+        for (int c = 0; c < 2; ++c) {
           uint32_t v[32];
-          tmem_ld32(lane_base + kColO + 32 * c, v);
+          tmem_ld32(lane_base + kColO + 64 * wg + 32 * c, v);
           tmem_wait_ld();
 #pragma unroll
           for (int i = 0; i < 32; ++i) v[i] = __float_as_uint(__uint_as_float(v[i]) * factor);
-          tmem_st32(lane_base + kColO + 32 * c, v);
+          tmem_st32(lane_base + kColO + 64 * wg + 32 * c, v);
         }
       }
     }
-#pragma unroll
-    for (int c = 0; c < 2; ++c) {
-      uint32_t v[32];
-#pragma unroll
-      for (int i = 0; i < 32; ++i) v[i] = hi[32 * c + i];
-      tmem_st32(lane_base + kColP + 32 * c, v);
-#pragma unroll
-      for (int i = 0; i < 32; ++i) v[i] = lo[32 * c + i];
-      tmem_st32(lane_base + kColPlo + 32 * c, v);
-    }
+    tmem_st32(lane_base + kColP + 32 * wg, hi);
+    tmem_st32(lane_base + kColPlo + 32 * wg, lo);
     tmem_wait_st();
     tc_fence_before();
     __syncwarp();
     if (lane == 0) mbar_arrive(smem_u32(&B->p_full));
   }
   if (ok && !warp_wait(smem_u32(&B->pv_done), static_cast<uint32_t>(w.n - 1) & 1u, B)) ok = false;
+  // both halves of l, through the slot pair the last tile did not use (the
+  // other warpgroup is done reading it); every thread arrives on every path
+  float* lslot = red + (w.n & 1) * 2 * kRows;
+  lslot[wg * kRows + r] = l;
+  mbar_arrive(smem_u32(&B->l_full));
+  if (ok && !warp_wait(smem_u32(&B->l_full), 0, B)) ok = false;
+  l = lslot[r] + lslot[kRows + r];
   if (!ok) {
     if (lane == 0) raise_abort(p, B);
     return;
@@ -338,13 +371,13 @@ __device__ void run_softmax(const PrefillParams& p, const Work& w, uint32_t tmem
   // out = O e^(m - M) / (l e^(m - M) + e^(sink - M)), M = max(m, sink), in log2 units
   const float s2 = p.sinks[h] * kPfLog2e;
   const float M = fmaxf(m, s2);
-  const float a = (m == -INFINITY) ? 0.f : exp2f(m - M);
-  const float sc = a / (l * a + exp2f(s2 - M));
-  float* out = p.out + (static_cast<long long>(t < p.T ? t : 0) * kHeads + h) * kDim;
+  const float a = (m == -INFINITY) ? 0.f : ex2(m - M);
+  const float sc = a / (l * a + ex2(s2 - M));
+  float* out = p.out + (static_cast<long long>(t < p.T ? t : 0) * kHeads + h) * kDim + 64 * wg;
 #pragma unroll
-  for (int c = 0; c < kDim / 32; ++c) {
+  for (int c = 0; c < 2; ++c) {
     uint32_t v[32];
-    tmem_ld32(lane_base + kColO + 32 * c, v);
+    tmem_ld32(lane_base + kColO + 64 * wg + 32 * c, v);
     tmem_wait_ld();
     if (t < p.T) {
 #pragma unroll
@@ -375,19 +408,22 @@ __global__ void __launch_bounds__(kPfThreads, 1) prefill_kernel(const __grid_con
     }
     mbar_init(smem_u32(&B->s_full[0]), 1);
     mbar_init(smem_u32(&B->s_full[1]), 1);
-    mbar_init(smem_u32(&B->p_full), 4);
+    mbar_init(smem_u32(&B->p_full), kSoftWarps);
     mbar_init(smem_u32(&B->pv_done), 1);
     mbar_init(smem_u32(&B->mma_done), 1);
+    mbar_init(smem_u32(&B->red_full[0]), kSoftWarps * 32);
+    mbar_init(smem_u32(&B->red_full[1]), kSoftWarps * 32);
+    mbar_init(smem_u32(&B->l_full), kSoftWarps * 32);
     B->abort = 0;
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
     asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
   }
-  if (warp == 4 && lane == 0) {
+  if (warp == kTmaWarp && lane == 0) {
     prefetch_tensormap(&p.q_map);
     prefetch_tensormap(&p.k_map);
     prefetch_tensormap(&p.v_map);
   }
-  if (warp == 5) {
+  if (warp == kMmaWarp) {
     asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], 512;" ::"r"(smem_u32(&B->tmem_base))
                  : "memory");
     asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
@@ -397,17 +433,17 @@ __global__ void __launch_bounds__(kPfThreads, 1) prefill_kernel(const __grid_con
   tc_fence_after();
   const uint32_t tmem = B->tmem_base;
 
-  if (warp < 4) {
-    run_softmax(p, w, tmem, B, warp, lane);
-  } else if (warp == 4) {
+  if (warp < kSoftWarps) {
+    run_softmax(p, w, tmem, smem, B, warp, lane);
+  } else if (warp == kTmaWarp) {
     if (lane == 0) run_tma(p, w, smem, B);
   } else if (lane == 0) {
     run_mma(p, w, smem_u32(smem), tmem, B);
   }
   tc_fence_before();
   __syncthreads();
-  if (warp == 4 && lane == 0 && B->abort) drain_tma(w, B);
-  if (warp == 5) {
+  if (warp == kTmaWarp && lane == 0 && B->abort) drain_tma(w, B);
+  if (warp == kMmaWarp) {
     __syncwarp();
     tc_fence_after();
     asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, 512;" ::"r"(tmem) : "memory");

@@ -56,7 +56,8 @@ def u16(t: torch.Tensor) -> np.ndarray:
 
 
 def bf16_values(bits: np.ndarray) -> np.ndarray:
-    return (bits.astype(np.uint32) << 16).view(np.float32).astype(np.float64)
+    with np.errstate(invalid="ignore"):  # sentinel slots may hold NaN patterns
+        return (bits.astype(np.uint32) << 16).view(np.float32).astype(np.float64)
 
 
 def close_bits(got, want, what):
