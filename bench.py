@@ -355,6 +355,7 @@ def run_prefill(args, rank, world, local):
     del prompts
     q = torch.empty((T, 32, 128), dtype=torch.bfloat16, device="cuda")
     k = torch.empty((T, 4, 128), dtype=torch.bfloat16, device="cuda")
+    v16 = torch.empty((T, 4, 128), dtype=torch.float16, device="cuda")
     out = torch.empty((len(layers), T, 32, 128), dtype=torch.float32, device="cuda")
     host_out = torch.empty(out.shape, dtype=torch.float32).pin_memory()
     err = torch.zeros(1, dtype=torch.int32, device="cuda")
@@ -365,10 +366,10 @@ def run_prefill(args, rank, world, local):
     def step(attn_events=False):
         for i, d in enumerate(layers):
             flint.flint_prefill_qk_norm_rope(d.q_raw, d.k_raw, d.w_q, d.w_k, apply_rope=d.rope, q_out=q,
-                                             k_out=k, v_raw=d.v_raw, cache=d.cache, dev_err=err)
+                                             k_out=k, v_raw=d.v_raw, v_out=v16, cache=d.cache, dev_err=err)
             if attn_events:
                 a0[i].record(stream)
-            flint.flint_prefill_attn(q, k, d.v_raw, d.sinks, d.window, out[i])
+            flint.flint_prefill_attn(q, k, v16, d.sinks, d.window, out[i])
             if attn_events:
                 a1[i].record(stream)
 
@@ -437,7 +438,7 @@ def run_prefill(args, rank, world, local):
         "metric": PREFILL_METRIC, "value": ms / world, "unit": "ms/prompt",
         "n_gpus": world, "steps": args.steps, "warmup": max(args.warmup, 3), "ms_per_step": ms,
         "higher_is_better": False, "scaling": "weak", "vs_baseline": None,
-        "dtype": "bf16 (mma.sync bf16, fp32 accumulate and softmax)",
+        "dtype": "bf16 q.k, fp16 p.v (tcgen05 MMAs, fp32 accumulate and softmax)",
         "data": "synthetic (seeded bf16 N(0,1) raw q/k/v, N(0,1) sinks, 1+N(0,0.1) norm weights)",
         "config": dict(prefill_config(T), parallelism=f"replicas x{world}", launch="direct launches"),
         "roofline": {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",

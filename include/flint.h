@@ -265,6 +265,9 @@ flint_status flint_attn_stack_noalloc(const flint_layer* layers, int32_t n_layer
  *          nearest even (prefill activations are bf16), or NULL
  *   k_out  bf16 [T][4][128]  (device, out): k after norm/RoPE, rounded to
  *          nearest even (the cache value), or NULL
+ *   v_out  fp16 [T][4][128]  (device, out): v_raw converted to fp16 (nearest,
+ *          saturating at +-65504; exact for bf16 values in the fp16 normal
+ *          range), the v operand of flint_prefill_attn, or NULL
  *   cache  NULL, or the cache of this one request (request 0 of a
  *          CONTIGUOUS / RING cache, row 0 of a PAGED block table): token t
  *          goes to slot t (ring: t % 513, and only the last 513 tokens are
@@ -275,8 +278,9 @@ flint_status flint_prefill_qk_norm_rope(const uint16_t* q_raw, const uint16_t* k
                                         const uint16_t* v_raw, const uint16_t* w_q,
                                         const uint16_t* w_k, int32_t T, float eps,
                                         double theta, int32_t apply_rope, uint16_t* q_out,
-                                        uint16_t* k_out, const flint_kv_cache* cache,
-                                        int32_t* dev_err, void* stream);
+                                        uint16_t* k_out, uint16_t* v_out,
+                                        const flint_kv_cache* cache, int32_t* dev_err,
+                                        void* stream);
 
 /* Prefill, step 2: causal attention of a T-token prompt over itself, with the
  * head's sink ("Model architecture": GQA 32/4, learned sinks, 513-token
@@ -286,12 +290,13 @@ flint_status flint_prefill_qk_norm_rope(const uint16_t* q_raw, const uint16_t* k
  * token at position t with L = t + 1:
  *   out[t][h] = sum_j e^(s_j - M) v[j] / (sum_j e^(s_j - M) + e^(sink_h - M)),
  *   s_j = q[t][h] . k[j] / sqrt(128), M = max(max_j s_j, sink_h).
- *   q  bf16 [T][32][128]; k, v  bf16 [T][4][128] (device, in; flint_prefill_
- *      qk_norm_rope's q_out and k_out, and v_raw)
+ *   q  bf16 [T][32][128], k  bf16 [T][4][128], v  fp16 [T][4][128] (device,
+ *      in; flint_prefill_qk_norm_rope's q_out, k_out and v_out)
  *   sinks  fp32 [32] (device, in); window  0 or FLINT_WINDOW
  *   out  fp32 [T][32][128] (device, out)
- * T in [1, FLINT_MAX_CONTEXT].  Products on bf16 tensor-core MMAs (tcgen05)
- * with fp32 accumulation; softmax in fp32.  A pipeline wait that runs past
+ * T in [1, FLINT_MAX_CONTEXT].  Products on tensor-core MMAs (tcgen05) with
+ * fp32 accumulation: q.k in bf16, p.v in fp16 (p rounded to fp16 after an
+ * fp32 softmax).  A pipeline wait that runs past
  * its time limit sets *dev_err = FLINT_ERR_TIMEOUT (dev_err may be NULL). */
 flint_status flint_prefill_attn(const uint16_t* q, const uint16_t* k, const uint16_t* v,
                                 int32_t T, const float* sinks, int32_t window, float* out,

@@ -570,16 +570,18 @@ flint_status flint_prefill_qk_norm_rope(const uint16_t* q_raw, const uint16_t* k
                                         const uint16_t* v_raw, const uint16_t* w_q,
                                         const uint16_t* w_k, int32_t T, float eps,
                                         double theta, int32_t apply_rope, uint16_t* q_out,
-                                        uint16_t* k_out, const flint_kv_cache* cache,
-                                        int32_t* dev_err, void* stream) {
+                                        uint16_t* k_out, uint16_t* v_out,
+                                        const flint_kv_cache* cache, int32_t* dev_err,
+                                        void* stream) {
   const char* who = "flint_prefill_qk_norm_rope";
   if (!q_raw || !k_raw || !w_q || !w_k) return fail(FLINT_ERR_INVALID_ARG, "%s: NULL input pointer", who);
   if (T < 1 || T > FLINT_MAX_CONTEXT)
     return fail(FLINT_ERR_INVALID_ARG, "%s: T=%d outside [1, %d]", who, T, FLINT_MAX_CONTEXT);
   if (apply_rope != 0 && apply_rope != 1) return fail(FLINT_ERR_INVALID_ARG, "%s: apply_rope must be 0 or 1", who);
   if (!(eps >= 0.f) || !(theta > 0.0)) return fail(FLINT_ERR_INVALID_ARG, "%s: eps must be >= 0, theta > 0", who);
-  if (!q_out && !k_out && !cache) return fail(FLINT_ERR_INVALID_ARG, "%s: no output requested", who);
-  const void* ptrs[] = {q_raw, k_raw, w_q, w_k, q_out, k_out, v_raw};
+  if (!q_out && !k_out && !v_out && !cache) return fail(FLINT_ERR_INVALID_ARG, "%s: no output requested", who);
+  if (v_out && !v_raw) return fail(FLINT_ERR_INVALID_ARG, "%s: v_out needs v_raw", who);
+  const void* ptrs[] = {q_raw, k_raw, w_q, w_k, q_out, k_out, v_out, v_raw};
   for (const void* p : ptrs)
     if (p && !aligned16(p)) return fail(FLINT_ERR_INVALID_ARG, "%s: pointers must be 16-byte aligned", who);
   PrepParams p;
@@ -590,6 +592,7 @@ flint_status flint_prefill_qk_norm_rope(const uint16_t* q_raw, const uint16_t* k
   p.w_q = w_q;
   p.w_k = w_k;
   p.q_out_bf16 = q_out;
+  p.v_out_f16 = v_out;
   p.k_out = k_out;
   p.eps = eps;
   p.theta = theta;
@@ -637,20 +640,21 @@ flint_status flint_prefill_attn(const uint16_t* q, const uint16_t* k, const uint
   EncodeTiledFn fn = encode_fn();
   if (!fn) return fail(FLINT_ERR_CUDA, "%s: cuTensorMapEncodeTiled is not available from the driver", who);
   // [128 dims][heads][T tokens][1] bf16, 128-byte swizzle, boxes of 64 dims
-  auto encode = [&](CUtensorMap* map, const void* base, int heads, int box_heads, int box_tokens) {
+  auto encode = [&](CUtensorMap* map, const void* base, int heads, int box_heads, int box_tokens,
+                    CUtensorMapDataType dtype) {
     const cuuint64_t dims[4] = {static_cast<cuuint64_t>(kDim), static_cast<cuuint64_t>(heads),
                                 static_cast<cuuint64_t>(T), 1};
     const cuuint64_t strides[3] = {kDim * 2ull, static_cast<cuuint64_t>(heads) * kDim * 2ull,
                                    static_cast<cuuint64_t>(T) * heads * kDim * 2ull};
     const cuuint32_t box[4] = {64, static_cast<cuuint32_t>(box_heads), static_cast<cuuint32_t>(box_tokens), 1};
     const cuuint32_t estr[4] = {1, 1, 1, 1};
-    return fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void*>(base), dims, strides, box, estr,
+    return fn(map, dtype, 4, const_cast<void*>(base), dims, strides, box, estr,
               CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   };
-  if (encode(&p.q_map, q, kHeads, kGroup, 16) != CUDA_SUCCESS ||
-      encode(&p.k_map, k, kKvHeads, 1, 128) != CUDA_SUCCESS ||
-      encode(&p.v_map, v, kKvHeads, 1, 128) != CUDA_SUCCESS)
+  if (encode(&p.q_map, q, kHeads, kGroup, 16, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16) != CUDA_SUCCESS ||
+      encode(&p.k_map, k, kKvHeads, 1, 128, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16) != CUDA_SUCCESS ||
+      encode(&p.v_map, v, kKvHeads, 1, 128, CU_TENSOR_MAP_DATA_TYPE_FLOAT16) != CUDA_SUCCESS)
     return fail(FLINT_ERR_CUDA, "%s: cuTensorMapEncodeTiled failed", who);
   p.sinks = sinks;
   p.out = out;

@@ -165,15 +165,17 @@ struct PrepParams {
   int32_t prefill;
   int32_t n_tokens;
   uint16_t* q_out_bf16;     // q rounded to bf16 [T][32][128], or nullptr
+  uint16_t* v_out_f16;      // v converted to fp16 [T][4][128] (saturating), or nullptr
 };
 
-// Prompt attention (prefill): q bf16 [T][32][128], k / v bf16 [T][4][128],
-// out fp32 [T][32][128]; query t attends keys max(0, t - window + 1) .. t
-// (window > 0) or 0 .. t.
+// Prompt attention (prefill): q bf16 [T][32][128], k bf16 [T][4][128], v fp16
+// [T][4][128], out fp32 [T][32][128]; query t attends keys
+// max(0, t - window + 1) .. t (window > 0) or 0 .. t.
 struct PrefillParams {
   // TMA maps, 128-byte swizzle, boxes of 64 dims:
   //   q_map  [128 dims][32 heads][T tokens][1], box 64 x 8 heads x 16 tokens
   //   k_map, v_map  [128 dims][4 heads][T tokens][1], box 64 x 1 x 128 tokens
+  //   (k bf16, v fp16)
   CUtensorMap q_map, k_map, v_map;
   const float* sinks;
   float* out;

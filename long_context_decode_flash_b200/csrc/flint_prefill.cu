@@ -16,9 +16,9 @@
 //              through 3- and 2-stage rings (128-byte swizzle, two 64-dim
 //              boxes per tile).
 //   warp 9     allocates the 512 TMEM columns; its lane 0 issues the MMAs:
-//              S = Q K^T (M 128, N 128, K 128) into one of two TMEM S buffers,
-//              and O += P V with P read from TMEM (bf16 hi and lo parts, two
-//              products) and V from shared memory (dims-major operand).
+//              S = Q K^T (bf16, M 128, N 128, K 128) into one of two TMEM S
+//              buffers, and O += P V (fp16, K 128) with P read from TMEM and V
+//              from shared memory (dims-major operand).
 //   warps 0-7  softmax in two warpgroups; thread (wg, r) owns row r (TMEM
 //              lane r) and the 64 keys 64 wg .. 64 wg + 63 of every tile, and
 //              the 64 output dims 64 wg .. 64 wg + 63.  Per tile: S from TMEM,
@@ -28,8 +28,12 @@
 //              only when a tile exceeds it by more than 2^8 (then O is
 //              rescaled in TMEM), P back to TMEM; at the end O, the sink and
 //              the store.
-// TMEM columns: S0 [0,128), S1 [128,256), P hi [256,320), P lo [320,384),
-// O [384,512).  Every wait is bounded; a timeout raises FLINT_ERR_TIMEOUT.
+// P is rounded to fp16 (P <= 2^8 under the lazy maximum, relative error
+// 2^-12) and V arrives in fp16 (exact for bf16 values in the fp16 normal
+// range), so one PV product keeps the output within a few 1e-4 of the exact
+// attention for unit-scale values.
+// TMEM columns: S0 [0,128), S1 [128,256), P [256,320) (fp16 pairs), O
+// [384,512).  Every wait is bounded; a timeout raises FLINT_ERR_TIMEOUT.
 #include <math.h>
 
 #include "flint_device.cuh"
@@ -56,13 +60,12 @@ constexpr size_t kPfSmem = kOffBar + 256 + 1024;        // barriers, TMEM addres
 constexpr float kPfLog2e = 1.4426950408889634f;
 constexpr float kPfScale = static_cast<float>(1.4426950408889634 * 0.08838834764831845);
 constexpr float kTau = 8.0f;               // lazy-rescale threshold (log2 units)
-constexpr uint32_t kColS = 0, kColP = 256, kColPlo = 320, kColO = 384;
+constexpr uint32_t kColS = 0, kColP = 256, kColO = 384;
 
-// Instruction descriptors (kind::f16): fp32 D, bf16 A and B, M 128, N 128;
-// S: both operands K-major; PV: B (V) dims-major.
+// Instruction descriptors (kind::f16), fp32 D, M 128, N 128.  S: bf16 A and
+// B, both K-major.  PV: fp16 A and B, B (V) dims-major.
 constexpr uint32_t kIdescS = (1u << 4) | (1u << 7) | (1u << 10) | ((kPkv >> 3) << 17) | ((128 >> 4) << 24);
-constexpr uint32_t kIdescPV = (1u << 4) | (1u << 7) | (1u << 10) | (1u << 16) | ((kDim >> 3) << 17) |
-                              ((128 >> 4) << 24);
+constexpr uint32_t kIdescPV = (1u << 4) | (1u << 16) | ((kDim >> 3) << 17) | ((128 >> 4) << 24);
 
 struct Bars {  // at kOffBar
   uint64_t q_full;
@@ -243,13 +246,12 @@ __device__ void run_mma(const PrefillParams& p, const Work& w, uint32_t base, ui
     if (!ok) break;
     tc_fence_after();
     const uint32_t vb = base + kOffV + sv * kTileBytes;
-    // O += P V: K = 16 keys per MMA (rows 16kk.. of both 64-dim boxes)
+    // O += P V: K = 16 keys per MMA (rows 16kk.. of both 64-dim boxes; the
+    // fp16 pairs of keys 16kk .. 16kk + 15 are columns 8kk .. 8kk + 7 of P)
 #pragma unroll
-    for (int part = 0; part < 2; ++part)
-#pragma unroll
-      for (int kk = 0; kk < 8; ++kk)
-        umma_ts(tmem + kColO, tmem + (part ? kColPlo : kColP) + kk * 8,
-                sw128_desc(vb + kk * 16 * 128, kHalfBytes, 1024), kIdescPV, (jj > 0 || part > 0 || kk > 0) ? 1u : 0u);
+    for (int kk = 0; kk < 8; ++kk)
+      umma_ts(tmem + kColO, tmem + kColP + kk * 8, sw128_desc(vb + kk * 16 * 128, kHalfBytes, 1024), kIdescPV,
+              (jj > 0 || kk > 0) ? 1u : 0u);
     umma_commit(smem_u32(&B->v_empty[sv]));
     umma_commit(smem_u32(&B->pv_done));
     if (jj + 2 < w.n) ok = issue_s(p, jj + 2, base, tmem, B);
@@ -320,13 +322,14 @@ __device__ void run_softmax(const PrefillParams& p, const Work& w, uint32_t tmem
       l *= factor;
     }
     const float mu = (m == -INFINITY) ? 0.f : m;
-    uint32_t hi[kH / 2], lo[kH / 2];
+    uint32_t pk[kH / 2];  // fp16 pairs
     float ls[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
     for (int c = 0; c < kH / 2; ++c) {
       const float p0 = ex2(fmaf(s[2 * c], kPfScale, -mu)), p1 = ex2(fmaf(s[2 * c + 1], kPfScale, -mu));
       ls[c & 3] += p0 + p1;
-      split_bf16x2(p0, p1, hi[c], lo[c]);
+      const __half2 hp = __floats2half2_rn(p0, p1);
+      pk[c] = *reinterpret_cast<const uint32_t*>(&hp);
     }
     l += (ls[0] + ls[1]) + (ls[2] + ls[3]);
     if (jj > 0) {
@@ -348,8 +351,7 @@ __device__ void run_softmax(const PrefillParams& p, const Work& w, uint32_t tmem
         }
       }
     }
-    tmem_st32(lane_base + kColP + 32 * wg, hi);
-    tmem_st32(lane_base + kColPlo + 32 * wg, lo);
+    tmem_st32(lane_base + kColP + 32 * wg, pk);
     tmem_wait_st();
     tc_fence_before();
     __syncwarp();

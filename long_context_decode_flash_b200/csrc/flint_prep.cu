@@ -9,7 +9,8 @@
 // to bf16 (nearest even) once and the same bits go to k_out and the cache; v
 // is copied bit for bit.  With do_norm = 0 and no RoPE the kernel is a plain
 // bit-exact append of final k and v.  In prefill mode the blocks are the T
-// tokens of one prompt at positions 0 .. T-1 and q is written rounded to bf16.  An E4M3 cache receives, for k and v,
+// tokens of one prompt at positions 0 .. T-1, q is written rounded to bf16
+// and v, for the prefill attention's PV product, converted to fp16.  An E4M3 cache receives, for k and v,
 // the codes of float32 (value / scale) (nearest even, saturating), where k is
 // the float32 normed (roped) value.
 #include "flint_device.cuh"
@@ -85,6 +86,17 @@ __global__ void __launch_bounds__(kPrepThreads) prep_kernel(const __grid_constan
         o[32 + lane] = static_cast<uint16_t>(f32x2_to_e4m3x2(__fdiv_rn(y[2], s), __fdiv_rn(y[3], s)));
       }
     }
+  }
+  if (p.v_out_f16 && warp < kKvHeads) {
+    // lane: dims 4l .. 4l+3; bf16 -> fp16 to nearest, saturating at +-65504
+    const uint2 x = reinterpret_cast<const uint2*>(p.v_raw + (static_cast<long long>(b) * kKvHeads + warp) * kDim)[lane];
+    auto sat = [](float f) { return fminf(fmaxf(f, -65504.f), 65504.f); };
+    const __half2 a = __floats2half2_rn(sat(bf16_lo(x.x)), sat(bf16_hi(x.x)));
+    const __half2 c = __floats2half2_rn(sat(bf16_lo(x.y)), sat(bf16_hi(x.y)));
+    uint2 y;
+    y.x = *reinterpret_cast<const uint32_t*>(&a);
+    y.y = *reinterpret_cast<const uint32_t*>(&c);
+    reinterpret_cast<uint2*>(p.v_out_f16 + (static_cast<long long>(b) * kKvHeads + warp) * kDim)[lane] = y;
   }
   if (row >= 0 && warp < kKvHeads) {
     const uint2* src = reinterpret_cast<const uint2*>(p.v_raw + (static_cast<long long>(b) * kKvHeads + warp) * kDim);

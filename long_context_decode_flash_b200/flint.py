@@ -92,7 +92,7 @@ def load_library() -> ctypes.CDLL:
             lib.flint_attn_stack_noalloc.argtypes = [P, I32, I32, ctypes.c_float, ctypes.c_double,
                                                      P, I32, P, P]
             lib.flint_prefill_qk_norm_rope.argtypes = [P, P, P, P, P, I32, ctypes.c_float,
-                                                       ctypes.c_double, I32, P, P, P, P, P]
+                                                       ctypes.c_double, I32, P, P, P, P, P, P]
             lib.flint_prefill_attn.argtypes = [P, P, P, I32, P, I32, P, P, P]
             lib.flint_plan_items.argtypes = [P, I32, I32, I32, P, P, P, P, I32]
             lib.flint_plan_items.restype = I32
@@ -201,23 +201,25 @@ def flint_kv_append(k, v, pos: Sequence[int], cache: KVCache, dev_err=None, stre
 
 
 def flint_prefill_qk_norm_rope(q_raw, k_raw, w_q, w_k, eps: float = 1e-6, theta: float = 10000.0,
-                               apply_rope: bool = True, q_out=None, k_out=None, v_raw=None,
+                               apply_rope: bool = True, q_out=None, k_out=None, v_raw=None, v_out=None,
                                cache: Optional[KVCache] = None, dev_err=None, stream=None):
-    """Norm (+RoPE) of the T tokens of one prompt at positions 0..T-1, q and k
-    out in bf16, optional cache write (request 0 of `cache`)."""
+    """Norm (+RoPE) of the T tokens of one prompt at positions 0..T-1: q and k
+    out in bf16, v out in fp16 (the attention's v operand), optional cache
+    write (request 0 of `cache`)."""
     T = int(q_raw.shape[0])
     lib = load_library()
     _check(lib.flint_prefill_qk_norm_rope(_ptr(q_raw), _ptr(k_raw), _ptr(v_raw), _ptr(w_q), _ptr(w_k),
                                           T, eps, theta, int(bool(apply_rope)), _ptr(q_out),
-                                          _ptr(k_out),
+                                          _ptr(k_out), _ptr(v_out),
                                           ctypes.byref(cache) if cache is not None else None,
                                           _ptr(dev_err), _stream(stream)))
-    return q_out, k_out
+    return q_out, k_out, v_out
 
 
 def flint_prefill_attn(q, k, v, sinks, window: int, out, dev_err=None, stream=None):
     """Causal attention (with sinks) of a T-token prompt over itself:
-    q bf16 [T, 32, 128], k / v bf16 [T, 4, 128], out fp32 [T, 32, 128]."""
+    q bf16 [T, 32, 128], k bf16 [T, 4, 128], v fp16 [T, 4, 128],
+    out fp32 [T, 32, 128]."""
     lib = load_library()
     _check(lib.flint_prefill_attn(_ptr(q), _ptr(k), _ptr(v), int(q.shape[0]), _ptr(sinks), int(window),
                                   _ptr(out), _ptr(dev_err), _stream(stream)))

@@ -127,16 +127,18 @@ def test_prefill_rejects_bad_arguments_on_the_host():
     assert lib.flint_prefill_attn(p, p, p, 16, p, 100, p, None, None) == U           # window 100
     assert lib.flint_prefill_attn(p, None, p, 16, p, 0, p, None, None) == E           # NULL k
     assert lib.flint_prefill_attn(p, p, ctypes.c_void_p(0x10008), 16, p, 0, p, None, None) == E  # unaligned v
-    assert lib.flint_prefill_qk_norm_rope(p, p, p, p, p, 0, eps, theta, 1, p, p, None, None, None) == E
-    assert lib.flint_prefill_qk_norm_rope(p, p, p, p, p, 16, eps, theta, 2, p, p, None, None, None) == E
-    assert lib.flint_prefill_qk_norm_rope(p, p, p, p, p, 16, eps, theta, 1, None, None, None, None,
+    assert lib.flint_prefill_qk_norm_rope(p, p, p, p, p, 0, eps, theta, 1, p, p, None, None, None, None) == E
+    assert lib.flint_prefill_qk_norm_rope(p, p, p, p, p, 16, eps, theta, 2, p, p, None, None, None, None) == E
+    assert lib.flint_prefill_qk_norm_rope(p, p, p, p, p, 16, eps, theta, 1, None, None, None, None, None,
                                           None) == E                                   # no output
+    assert lib.flint_prefill_qk_norm_rope(p, p, None, p, p, 16, eps, theta, 1, None, None, p, None, None,
+                                          None) == E                                   # v_out without v_raw
     c = _fake_cache(capacity=100)
-    assert lib.flint_prefill_qk_norm_rope(p, p, p, p, p, 101, eps, theta, 1, p, p, ctypes.byref(c), None,
-                                          None) == E                                   # 101 tokens, 100 slots
+    assert lib.flint_prefill_qk_norm_rope(p, p, p, p, p, 101, eps, theta, 1, p, p, None, ctypes.byref(c),
+                                          None, None) == E                             # 101 tokens, 100 slots
     assert "capacity" in lib.flint_last_error().decode()
-    assert lib.flint_prefill_qk_norm_rope(p, p, None, p, p, 50, eps, theta, 1, p, p, ctypes.byref(c), None,
-                                          None) == E                                   # cache without v
+    assert lib.flint_prefill_qk_norm_rope(p, p, None, p, p, 50, eps, theta, 1, p, p, None, ctypes.byref(c),
+                                          None, None) == E                             # cache without v
 
 
 def test_workspace_bytes_bounds():

@@ -1,6 +1,6 @@
 """Parity of the prefill path (the T tokens of one prompt, positions 0..T-1)
 against the float64 oracle's prefill: q and k after norm (+RoPE) rounded to
-bf16, the cache they fill (bf16 and E4M3; contiguous, ring and paged), the
+bf16, v converted to fp16 for the PV product, the cache they fill (bf16 and E4M3; contiguous, ring and paged), the
 causal attention with sinks on window (513, RoPE) and full (NoPE) layers, and
 a decode step that continues from the prefilled cache."""
 import numpy as np
@@ -27,15 +27,22 @@ class Dev:
         self.T, self.window, self.rope = p.q_raw.shape[0], p.window, p.rope
 
 
-def prep_gpu(d: Dev, cache=None):
+def prep_gpu(d: Dev, cache=None, with_v=False):
     q = torch.empty((d.T, 32, 128), dtype=torch.bfloat16, device="cuda")
     k = torch.empty((d.T, 4, 128), dtype=torch.bfloat16, device="cuda")
+    v = torch.empty((d.T, 4, 128), dtype=torch.float16, device="cuda")
     err = torch.zeros(1, dtype=torch.int32, device="cuda")
     flint.flint_prefill_qk_norm_rope(d.q_raw, d.k_raw, d.w_q, d.w_k, apply_rope=d.rope, q_out=q, k_out=k,
-                                     v_raw=d.v_raw, cache=cache, dev_err=err)
+                                     v_raw=d.v_raw, v_out=v, cache=cache, dev_err=err)
     torch.cuda.synchronize()
     assert int(err.item()) == 0
-    return q, k
+    return (q, k, v) if with_v else (q, k)
+
+
+def f16(v_bf16: torch.Tensor) -> torch.Tensor:
+    """The fp16 v operand of the attention-only tests (nearest, as the prep
+    kernel converts)."""
+    return dev(v_bf16.to(torch.float16))
 
 
 def attn_gpu(q, k, v, sinks, window):
@@ -78,10 +85,12 @@ def close_bits(got, want, what):
 def test_prefill_q_and_k_match_the_oracle(window):
     p = I.make_prefill(300, window, workload=W_PF)
     d = Dev(p)
-    q, k = prep_gpu(d)
+    q, k, v = prep_gpu(d, with_v=True)
     _, qb, kb = oracle_prefill(p, rows=[])
     close_bits(u16(q), qb, "q")
     close_bits(u16(k), kb, "k")
+    # v: bf16 -> fp16 to nearest, bit for bit the host conversion
+    np.testing.assert_array_equal(v.cpu().view(torch.int16).numpy(), p.v_raw.to(torch.float16).view(torch.int16).numpy())
 
 
 @pytest.mark.parametrize("T", [1, 2, 15, 16, 17, 64, 65, 200, 700])
@@ -92,7 +101,7 @@ def test_prefill_attention_every_row(T, window):
     want, qb, kb = oracle_prefill(p, rows=range(T))
     q = dev(torch.from_numpy(qb.view(np.int16)).view(torch.bfloat16))
     k = dev(torch.from_numpy(kb.view(np.int16)).view(torch.bfloat16))
-    got = attn_gpu(q, k, dev(p.v_raw), dev(p.sinks), window)
+    got = attn_gpu(q, k, f16(p.v_raw), dev(p.sinks), window)
     parity(got, want, f"T={T} window={window}")
 
 
@@ -121,8 +130,8 @@ def test_prefill_composed_small(window):
     T = 1000
     p = I.make_prefill(T, window, workload=W_PF + 2)
     d = Dev(p)
-    q, k = prep_gpu(d)
-    got = attn_gpu(q, k, d.v_raw, d.sinks, window)
+    q, k, v = prep_gpu(d, with_v=True)
+    got = attn_gpu(q, k, v, d.sinks, window)
     check_composed(p, got, q, k, list(range(T)), f"window={window}")
 
 
@@ -140,8 +149,8 @@ def test_prefill_8192_sampled_rows(window):
     T = 8192
     p = I.make_prefill(T, window, workload=W_PF + 3)
     d = Dev(p)
-    q, k = prep_gpu(d)
-    got = attn_gpu(q, k, d.v_raw, d.sinks, window)
+    q, k, v = prep_gpu(d, with_v=True)
+    got = attn_gpu(q, k, v, d.sinks, window)
     assert np.isfinite(got).all()
     check_composed(p, got, q, k, sample_rows(T, 7), f"T=8192 window={window}")
 
@@ -152,10 +161,10 @@ def test_prefill_attention_ignores_keys_past_the_prompt_and_reruns_identically()
     for bit (the same tiles and order of work), and two launches agree."""
     p = I.make_prefill(300, 0, workload=W_PF + 4)
     d = Dev(p)
-    q, k = prep_gpu(d)
-    a = attn_gpu(q, k, d.v_raw, d.sinks, 0)
-    b = attn_gpu(q[:100].contiguous(), k[:100].contiguous(), d.v_raw[:100].contiguous(), d.sinks, 0)
-    c = attn_gpu(q, k, d.v_raw, d.sinks, 0)
+    q, k, v = prep_gpu(d, with_v=True)
+    a = attn_gpu(q, k, v, d.sinks, 0)
+    b = attn_gpu(q[:100].contiguous(), k[:100].contiguous(), v[:100].contiguous(), d.sinks, 0)
+    c = attn_gpu(q, k, v, d.sinks, 0)
     np.testing.assert_array_equal(a, c)
     np.testing.assert_array_equal(a[:96], b[:96])  # whole 16-row blocks: the same work
     parity(b, a[:100], "prefix")
