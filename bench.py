@@ -91,6 +91,8 @@ def parse():
                          "smaller ones serve profiling)")
     ap.add_argument("--kv", default="bf16", choices=["bf16", "fp8"],
                     help="KV-cache element: bf16, or E4M3 codes with per-head scales")
+    ap.add_argument("--layers", type=int, default=49,
+                    help="prefill8k: run the first N of the 49 layers (profiling; the benchmark's figure is 49)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-graph", action="store_true", help="time direct launches instead of graph replays")
@@ -247,13 +249,13 @@ def prefill_config(T):
             "l2": "flushed before every step (256 MiB write, then 256 MiB read of another buffer)"}
 
 
-def prefill_inputs(I, T, kinds_only=False):
-    """The 49 layers' prompts (window 513 or 0 per layer kind); kinds_only: one
-    window and one full layer (the oracle sample)."""
+def prefill_inputs(I, T, kinds_only=False, n_layers=49):
+    """The first n_layers of the 49 layers' prompts (window 513 or 0 per layer
+    kind); kinds_only: one window and one full layer (the oracle sample)."""
     kinds = I.layer_kinds()
     if kinds_only:
         return [I.make_prefill(T, 513, layer=0), I.make_prefill(T, 0, layer=kinds.index(True))]
-    return [I.make_prefill(T, 0 if full else 513, layer=i) for i, full in enumerate(kinds)]
+    return [I.make_prefill(T, 0 if full else 513, layer=i) for i, full in enumerate(kinds[:n_layers])]
 
 
 def oracle_prefill_sample(prompts, T, nthreads, budget_s=10.0):
@@ -298,9 +300,10 @@ def run_prefill(args, rank, world, local):
     from long_context_decode_flash_b200 import inputs as I
 
     T = args.context
-    prompts = prefill_inputs(I, T)
+    n_layers = max(1, min(49, args.layers))
+    prompts = prefill_inputs(I, T, n_layers=n_layers)
     cpu_baseline = None
-    if rank == 0 and world == 1 and T == PREFILL_T and not args.no_cpu_baseline:
+    if rank == 0 and world == 1 and T == PREFILL_T and n_layers == 49 and not args.no_cpu_baseline:
         import oracle
         oracle.build()
         sample = prefill_inputs(I, T, kinds_only=True)
@@ -427,11 +430,13 @@ def run_prefill(args, rank, world, local):
                "h2d_bytes_per_step": int(host_in.numel() * 2), "d2h_bytes_per_step": int(host_out.numel() * 4)}
     ms = max_over_ranks(ms, world, "cuda")
 
-    kinds = I.layer_kinds()
+    kinds = I.layer_kinds()[:n_layers]
     flops = sum(prefill_flops(T, 0 if full else 513) for full in kinds)
     attn_total_ms = statistics.mean(sum(x) for x in attn_ms)
-    full_ms = statistics.mean(sum(x[i] for i, f in enumerate(kinds) if f) for x in attn_ms) / sum(kinds)
-    win_ms = statistics.mean(sum(x[i] for i, f in enumerate(kinds) if not f) for x in attn_ms) / (49 - sum(kinds))
+    n_full = sum(kinds)
+    full_ms = (statistics.mean(sum(x[i] for i, f in enumerate(kinds) if f) for x in attn_ms) / n_full
+               if n_full else None)
+    win_ms = statistics.mean(sum(x[i] for i, f in enumerate(kinds) if not f) for x in attn_ms) / (n_layers - n_full)
     achieved = flops / (attn_total_ms * 1e-3) / 1e12
     peak, peak_kind = measured_tensor_peak()
     line = {
@@ -440,11 +445,13 @@ def run_prefill(args, rank, world, local):
         "higher_is_better": False, "scaling": "weak", "vs_baseline": None,
         "dtype": "bf16 q.k, fp16 p.v (tcgen05 MMAs, fp32 accumulate and softmax)",
         "data": "synthetic (seeded bf16 N(0,1) raw q/k/v, N(0,1) sinks, 1+N(0,0.1) norm weights)",
-        "config": dict(prefill_config(T), parallelism=f"replicas x{world}", launch="direct launches"),
+        "config": dict(prefill_config(T), layers=n_layers, parallelism=f"replicas x{world}",
+                       launch="direct launches"),
         "roofline": {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
                      "frac": achieved / peak, "peak_kind": peak_kind, "kernel": "flint prefill_kernel",
                      "algorithmic_flops": int(flops), "attn_ms_per_prompt": attn_total_ms,
-                     "full_layer_attn_us": full_ms * 1e3, "window_layer_attn_us": win_ms * 1e3,
+                     "full_layer_attn_us": full_ms * 1e3 if full_ms is not None else None,
+                     "window_layer_attn_us": win_ms * 1e3,
                      "traffic": None},
         "cpu_baseline": cpu_baseline,
         "e2e": e2e,
