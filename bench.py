@@ -37,8 +37,11 @@ NOMINAL_HBM_GBS = 8000.0
 # launch from a full-size, one-pass ncu capture of the stack at context 100,000
 # (profiles/decode_kernel_stack100k_traffic.md), per KV dtype, with the hash of the CUDA
 # sources it was taken on; reported only while the sources still hash the same.
-TRAFFIC = {("stack", 100_000, "bf16"): (2_905_824_256 + 6_814_208, "207da7376fd4f092"),
-           ("stack", 100_000, "fp8"): (1_453_987_328 + 6_094_848, "207da7376fd4f092")}
+TRAFFIC = {("stack", 100_000, "bf16"): (2_905_827_072 + 6_852_864, "cde382082669d367"),
+           ("stack", 100_000, "fp8"): (1_453_981_440 + 6_602_496, "cde382082669d367")}
+# The same for one prefill_kernel launch of a full (NoPE) layer on the
+# 8,192-token prompt (profiles/prefill_kernel_prefill8k_full.md).
+PREFILL_TRAFFIC = {8192: (84_186_368 + 80_689_152, "cde382082669d367")}
 
 
 def max_over_ranks(x: float, world: int, device) -> float:
@@ -72,6 +75,11 @@ def kernel_sources_hash() -> str:
 
 def traffic_for(workload: str, ctx: int, kv: str = "bf16"):
     t = TRAFFIC.get((workload, ctx, kv))
+    return t[0] if t is not None and t[1] == kernel_sources_hash() else None
+
+
+def prefill_traffic(T: int):
+    t = PREFILL_TRAFFIC.get(T)
     return t[0] if t is not None and t[1] == kernel_sources_hash() else None
 FALLBACK_HBM_GBS = 6650.0
 FALLBACK_BF16_TFLOPS = 1400.0   # sustained, under the power cap
@@ -452,7 +460,7 @@ def run_prefill(args, rank, world, local):
                      "algorithmic_flops": int(flops), "attn_ms_per_prompt": attn_total_ms,
                      "full_layer_attn_us": full_ms * 1e3 if full_ms is not None else None,
                      "window_layer_attn_us": win_ms * 1e3,
-                     "traffic": None},
+                     "traffic": prefill_traffic(T), "traffic_launch": "one full-layer launch"},
         "cpu_baseline": cpu_baseline,
         "e2e": e2e,
         "gpu_launches": args.steps * 2 * n_layers,
