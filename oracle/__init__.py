@@ -189,6 +189,55 @@ def attn_decode(q, k_cache, v_cache, L: int, sinks, window: int = 0,
     return out
 
 
+_LOG2E = 1.4426950408889634
+
+
+def attn_partial(q, k, v):
+    """The unnormalised attention of one query over the keys k / v given
+    ([n, nkv, d] bf16 bits; no window, no sink), in log2 units, for a later
+    merge across ranks ("Day-0 Support for Flint on vLLM", hnkhoi.com, "Model
+    architecture": GQA, query head h reads KV head h / (nq / nkv)):
+    s'_j = q_h . k_j / sqrt(d) log2(e), m_h = max_j s'_j,
+    l_h = sum_j 2^(s'_j - m_h), O_h = sum_j 2^(s'_j - m_h) v_j.
+    q [nq, d] float64 (or bf16 bits).  Returns (O [nq, d], m [nq], l [nq]),
+    float64; with no keys m = -inf, l = 0, O = 0."""
+    q = bf16_to_f64(q) if np.asarray(q).dtype == np.uint16 else _f64(q)
+    nq, d = q.shape
+    k, v = bf16_to_f64(k), bf16_to_f64(v)
+    n, nkv = k.shape[0], k.shape[1]
+    O = np.zeros((nq, d))
+    m = np.full(nq, -np.inf)
+    lsum = np.zeros(nq)
+    if n == 0:
+        return O, m, lsum
+    for h in range(nq):
+        g = h // (nq // nkv)
+        s = (k[:, g, :] @ q[h]) / np.sqrt(d) * _LOG2E
+        m[h] = s.max()
+        w = np.exp2(s - m[h])
+        lsum[h] = w.sum()
+        O[h] = w @ v[:, g, :]
+    return O, m, lsum
+
+
+def merge_partials(parts, sinks):
+    """The log-sum-exp merge of partials (O_r, m_r, l_r) from attn_partial with
+    each head's sink logit, which joins the softmax with no value (same page,
+    "Learned attention sinks"): M = max(sink log2(e), max_r m_r),
+    out = sum_r 2^(m_r - M) O_r / (2^(sink log2(e) - M) + sum_r 2^(m_r - M) l_r)."""
+    sinks = _f64(sinks) * _LOG2E
+    M = sinks.copy()
+    for _, m, _ in parts:
+        M = np.maximum(M, m)
+    num = 0.0
+    den = np.exp2(sinks - M)
+    for O, m, lsum in parts:
+        w = np.where(np.isneginf(m), 0.0, np.exp2(np.where(np.isneginf(m), 0.0, m) - M))
+        num = num + w[:, None] * O
+        den = den + w * lsum
+    return num / den[:, None]
+
+
 def decode_layer(q_raw, k_raw, v_raw, w_q, w_k, sinks, k_cache, v_cache, L: int,
                  window: int, apply_rope: bool, layout: int = CONTIGUOUS,
                  capacity: int = 0, block_table=None, block_size: int = 64,

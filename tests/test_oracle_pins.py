@@ -522,3 +522,39 @@ def test_prefill_rows_match_causal_sdpa_with_a_sink_column(window, rope):
     bias = torch.cat([bias, sink_col * math.sqrt(d)], dim=2) / math.sqrt(d)
     want = F.scaled_dot_product_attention(q, k, v, attn_mask=bias, scale=1.0 / math.sqrt(d))
     np.testing.assert_allclose(out, want.permute(1, 0, 2).numpy(), rtol=1e-10, atol=1e-12)
+
+
+# ------------------------------------------------------ context parallel ----
+
+def test_partials_over_any_split_merge_to_the_whole_decode():
+    """Context-parallel split-KV: the merge of the partials of consecutive
+    token ranges equals the decode attention over all of them (the sink
+    folded in once), for splits into 1, 2, 3 and 7 uneven ranges."""
+    L, nq, nkv, d = 300, 8, 2, 32
+    q = rng.normal(size=(nq, d))
+    K, V = bf16_bits((L, nkv, d), 411), bf16_bits((L, nkv, d), 412)
+    sinks = rng.normal(size=nq)
+    want = oracle.attn_decode(q, K, V, L, sinks, 0)
+    for cuts in ([], [150], [1, 299], [10, 11, 50, 120, 121, 280]):
+        edges = [0] + cuts + [L]
+        parts = [oracle.attn_partial(q, K[a:b], V[a:b]) for a, b in zip(edges[:-1], edges[1:])]
+        np.testing.assert_allclose(oracle.merge_partials(parts, sinks), want, rtol=1e-12, atol=1e-13)
+
+
+def test_partial_is_unnormalised_softmax_and_merge_without_sink_is_sdpa():
+    """One partial: O / l is plain softmax attention (torch SDPA, no sink),
+    m is the row maximum of the log2-scaled scores, and an empty range merges
+    as nothing."""
+    L, nq, nkv, d = 64, 4, 1, 16
+    q = rng.normal(size=(nq, d))
+    K, V = bf16_bits((L, nkv, d), 421), bf16_bits((L, nkv, d), 422)
+    O, m, lsum = oracle.attn_partial(q, K, V)
+    k, v = torch.from_numpy(f64(K)[:, 0, :]), torch.from_numpy(f64(V)[:, 0, :])
+    qt = torch.from_numpy(q)
+    sdpa = F.scaled_dot_product_attention(qt[None], k[None], v[None]).numpy()[0]
+    np.testing.assert_allclose(O / lsum[:, None], sdpa, rtol=1e-12, atol=1e-13)
+    np.testing.assert_allclose(m, (qt @ k.T).numpy().max(axis=1) / math.sqrt(d) * math.log2(math.e), rtol=1e-13)
+    empty = oracle.attn_partial(q, K[:0], V[:0])
+    assert np.isneginf(empty[1]).all() and (empty[2] == 0).all()
+    sinks = np.full(nq, -np.inf)
+    np.testing.assert_allclose(oracle.merge_partials([empty, (O, m, lsum)], sinks), sdpa, rtol=1e-12, atol=1e-13)
