@@ -93,10 +93,10 @@ def parse():
     ap.add_argument("--impl", default="flint", choices=["flint", "reference"])
     ap.add_argument("--workload", default="stack",
                     choices=["stack", "serial", "full100k", "full2k", "swa100k", "paged32", "paged32swa",
-                             "prefill8k"])
+                             "prefill8k", "cp262k"])
     ap.add_argument("--context", type=int, default=None,
                     help="context length (decode: 100,000; prefill8k: the prompt length, 8,192; "
-                         "smaller ones serve profiling)")
+                         "cp262k: 262,144; smaller ones serve profiling)")
     ap.add_argument("--kv", default="bf16", choices=["bf16", "fp8"],
                     help="KV-cache element: bf16, or E4M3 codes with per-head scales")
     ap.add_argument("--layers", type=int, default=49,
@@ -476,6 +476,120 @@ def run_prefill(args, rank, world, local):
         torch.distributed.destroy_process_group()
 
 
+# ---------------------------------------------------- context parallel ----
+
+CP_T = 262_144
+
+
+def run_cp(args, rank, world, local):
+    """The cp262k workload: one decode step of a full NoPE layer at the
+    262,144-token maximum context, its tokens split over the ranks (strong
+    scaling): per rank flint_attn_decode_partial over its range, an
+    all-gather of the partials, flint_merge_partials."""
+    import numpy as np
+    import torch
+    from long_context_decode_flash_b200 import cp, flint
+    from long_context_decode_flash_b200 import inputs as I
+
+    L = args.context
+    d = I.make_decode(L, workload=I.W_FULL_100K)
+    lo, hi = cp.rank_ranges(L, world)[rank]
+    cpu_baseline = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        import oracle
+        oracle.build()
+        nthreads = os.cpu_count() or 1
+        t0 = time.perf_counter()
+        oracle.attn_decode(I.bits(d.q[0]), I.bits(d.k_cache[0]), I.bits(d.v_cache[0]), L,
+                           d.sinks.numpy().astype(np.float64), 0, capacity=L, nthreads=nthreads)
+        us = (time.perf_counter() - t0) * 1e6
+        cpu_baseline = {"value": us, "unit": "us/token", "cores": nthreads, "kind": "oracle",
+                        "sample": f"one full oracle decode of the layer at context {L}"}
+    if world > 1:
+        torch.distributed.init_process_group("nccl", timeout=__import__("datetime").timedelta(seconds=120))
+    torch.cuda.set_device(local)
+    stream = torch.cuda.current_stream()
+    q = d.q.cuda()
+    kc, vc = d.k_cache[:, lo:hi].contiguous().cuda(), d.v_cache[:, lo:hi].contiguous().cuda()
+    del d.k_cache, d.v_cache
+    cache = flint.kv_cache(kc, vc, flint.CONTIGUOUS, capacity=hi - lo)
+    sinks = d.sinks.cuda()
+    out = torch.empty((1, 32, 128), dtype=torch.float32, device="cuda")
+    ws = flint.workspace(1)
+    err = torch.zeros(1, dtype=torch.int32, device="cuda")
+    flush = torch.empty(256 * 1024 * 1024 // 4, dtype=torch.float32, device="cuda")
+    flush_rd = torch.ones(256 * 1024 * 1024 // 4, dtype=torch.float32, device="cuda")
+    flush_acc = torch.zeros(1, dtype=torch.float32, device="cuda")
+
+    def flush_l2(i):
+        flush.fill_(float(i))
+        torch.sum(flush_rd, dim=0, keepdim=True, out=flush_acc)
+
+    def step():
+        cp.cp_decode(q, cache, [hi - lo], sinks, out, ws, dev_err=err)
+
+    for _ in range(max(args.warmup, 3)):
+        flush_l2(1)
+        step()
+    torch.cuda.synchronize()
+    starts = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    ends = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    if world > 1:
+        torch.distributed.barrier()
+    torch.cuda.synchronize()
+    with ClockSampler(torch.cuda.current_device()) as clocks:
+        for i in range(args.steps):
+            flush_l2(i)
+            starts[i].record(stream)
+            step()
+            ends[i].record(stream)
+        torch.cuda.synchronize()
+    if world > 1:
+        torch.distributed.barrier()
+    if int(err.item()) != 0:
+        raise SystemExit(f"device error {int(err.item())}")
+    ms = max_over_ranks(statistics.mean(s.elapsed_time(e) for s, e in zip(starts, ends)), world, "cuda")
+    host_q = d.q.pin_memory()
+    host_out = torch.empty(out.shape, dtype=torch.float32).pin_memory()
+    e_s = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    e_e = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    for i in range(args.steps):
+        flush_l2(i)
+        e_s[i].record(stream)
+        q.copy_(host_q, non_blocking=True)
+        step()
+        host_out.copy_(out, non_blocking=True)
+        e_e[i].record(stream)
+    torch.cuda.synchronize()
+    e2e_ms = max_over_ranks(statistics.mean(s.elapsed_time(e) for s, e in zip(e_s, e_e)), world, "cuda")
+    algo = L * 2 * 4 * 128 * 2
+    peak, peak_kind = measured_peak()
+    achieved = algo / (ms * 1e-3) / 1e9
+    line = {
+        "metric": "full-layer decode-attention us/token @262,144 ctx, context-parallel over the GPUs",
+        "value": ms * 1000.0, "unit": "us/token", "n_gpus": world, "steps": args.steps,
+        "warmup": max(args.warmup, 3), "ms_per_step": ms, "higher_is_better": False, "scaling": "strong",
+        "vs_baseline": None, "dtype": "bf16", "data": "synthetic (seeded bf16 N(0,1) q/KV, N(0,1) sinks)",
+        "config": {"workload": "one full-context NoPE layer, one token, its 262,144 cached tokens split "
+                               "evenly over the ranks; per rank split-KV partial, all-gather, merge with sinks",
+                   "context": L, "tokens_per_rank": hi - lo, "parallelism": f"context-parallel x{world}",
+                   "l2": "flushed before every step (256 MiB write, then 256 MiB read of another buffer)"},
+        "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak * world, "unit": "GB/s",
+                     "frac": achieved / (peak * world), "peak_kind": f"{peak_kind} x {world} GPUs",
+                     "algorithmic_bytes": algo, "kernel": "flint decode_kernel (partial) + merge",
+                     "traffic": None},
+        "cpu_baseline": cpu_baseline,
+        "e2e": {"value": e2e_ms * 1000.0, "unit": "us/token", "h2d_bytes_per_step": int(host_q.numel() * 2),
+                "d2h_bytes_per_step": int(host_out.numel() * 4)},
+        "gpu_launches": args.steps * 2,
+        "clocks": clocks.summary(),
+    }
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        torch.distributed.destroy_process_group()
+
+
 # ------------------------------------------------------------- GPU side ----
 
 def workload_config(name):
@@ -597,12 +711,15 @@ def main():
     world = int(os.environ.get("WORLD_SIZE", "1"))
     local = int(os.environ.get("LOCAL_RANK", "0"))
     if args.context is None:
-        args.context = PREFILL_T if args.workload == "prefill8k" else CONTEXT
+        args.context = {"prefill8k": PREFILL_T, "cp262k": CP_T}.get(args.workload, CONTEXT)
     if args.impl == "reference":
         run_reference(args, rank)
         return
     if args.workload == "prefill8k":
         run_prefill(args, rank, world, local)
+        return
+    if args.workload == "cp262k":
+        run_cp(args, rank, world, local)
         return
 
     import torch

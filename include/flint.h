@@ -58,6 +58,8 @@ extern "C" {
 #define FLINT_MAX_CONTEXT 262144  /* "maxContext" of the model JSON */
 #define FLINT_MAX_BATCH 64        /* requests per flint_attn_decode launch */
 #define FLINT_MAX_LAYERS 49       /* layers per flint_attn_stack call */
+#define FLINT_CP_PARTIAL_FLOATS 4160  /* 32*128 + 32 + 32: one context-parallel partial */
+#define FLINT_MAX_CP_PARTS 1024       /* partials per flint_merge_partials call */
 #define FLINT_NOALLOC_SCRATCH_BYTES (4u << 20)  /* flint_attn_stack_noalloc's fixed scratch */
 
 typedef enum {
@@ -301,6 +303,35 @@ flint_status flint_prefill_qk_norm_rope(const uint16_t* q_raw, const uint16_t* k
 flint_status flint_prefill_attn(const uint16_t* q, const uint16_t* k, const uint16_t* v,
                                 int32_t T, const float* sinks, int32_t window, float* out,
                                 int32_t* dev_err, void* stream);
+
+/* Context-parallel decode, step 1 (multi-GPU split-KV of a full layer: each
+ * rank owns a range of the layer's tokens; the pages serve on one GPU, so
+ * this follows the split-KV arithmetic of flint_attn_decode).  The attention
+ * of q over tokens [0, seq_lens[b]) of this rank's `cache` (no window, no
+ * sink), returned unnormalised so that the ranks' results can be merged:
+ *   partials  fp32 [B][FLINT_CP_PARTIAL_FLOATS] (device, out): for request b,
+ *             O [32][128], then m [32], then l [32], with scores in log2
+ *             units (s'_j = q_h . k_j / sqrt(128) * log2(e)):
+ *             m_h = max_j s'_j, l_h = sum_j 2^(s'_j - m_h),
+ *             O_h = sum_j 2^(s'_j - m_h) v_j (up to rounding order).
+ * Other arguments, the workspace and errors as flint_attn_decode. */
+flint_status flint_attn_decode_partial(const void* q, int32_t q_is_fp32,
+                                       const flint_kv_cache* cache, const int32_t* seq_lens,
+                                       int32_t B, float* partials, void* workspace,
+                                       size_t ws_bytes, int32_t num_ctas, int32_t* dev_err,
+                                       void* stream);
+
+/* Context-parallel decode, step 2: the log-sum-exp merge of n_parts partials
+ * per request (the ranks' flint_attn_decode_partial results after an
+ * all-gather) with the head's sink logit, as flint_attn_decode folds its own
+ * split partials:  M = max(sink_h log2(e), max_r m_r),
+ *   out_h = sum_r 2^(m_r - M) O_r / (2^(sink_h log2(e) - M) + sum_r 2^(m_r - M) l_r).
+ *   partials  fp32 [n_parts][B][FLINT_CP_PARTIAL_FLOATS] (device, in)
+ *   sinks     fp32 [32] (device, in);  out  fp32 [B][32][128] (device, out)
+ * n_parts in [1, FLINT_MAX_CP_PARTS], B in [1, FLINT_MAX_BATCH].  A partial
+ * with m = -inf (no tokens) contributes nothing. */
+flint_status flint_merge_partials(const float* partials, int32_t n_parts, int32_t B,
+                                  const float* sinks, float* out, void* stream);
 
 /* The split planner behind both attention calls (pure host code, exposed for
  * tests).  Work is n_segs segments (one per problem, all four KV heads

@@ -13,7 +13,7 @@ HERE = os.path.dirname(os.path.abspath(__file__))
 ROOT = os.path.dirname(HERE)
 CSRC = os.path.join(HERE, "csrc")
 LIB = os.path.join(HERE, "libflint.so")
-SOURCES = ["flint_abi.cu", "flint_decode.cu", "flint_prep.cu", "flint_prefill.cu", "flint_plan.cpp", "flint_noalloc.cu"]
+SOURCES = ["flint_abi.cu", "flint_decode.cu", "flint_prep.cu", "flint_prefill.cu", "flint_cp.cu", "flint_plan.cpp", "flint_noalloc.cu"]
 HEADERS = ["flint_internal.h", "flint_device.cuh"]
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 

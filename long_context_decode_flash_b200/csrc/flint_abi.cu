@@ -669,12 +669,11 @@ size_t flint_attn_workspace_bytes(int32_t n_problems, int32_t num_ctas) {
   return kCounterBytes + static_cast<size_t>(kMaxItems) * kPartialBytes;
 }
 
-flint_status flint_attn_decode(const void* q, int32_t q_is_fp32, const flint_kv_cache* cache,
-                               const int32_t* seq_lens, int32_t B, const float* sinks,
-                               int32_t window, float* out, void* workspace, size_t ws_bytes,
-                               int32_t num_ctas, int32_t* dev_err, void* stream) {
-  const char* who = "flint_attn_decode";
-  if (!q || !seq_lens || !sinks || !out || !workspace)
+static flint_status decode_impl(const void* q, int32_t q_is_fp32, const flint_kv_cache* cache,
+                                const int32_t* seq_lens, int32_t B, const float* sinks, int32_t window,
+                                float* out, void* workspace, size_t ws_bytes, int32_t num_ctas,
+                                int32_t* dev_err, void* stream, bool partial, const char* who) {
+  if (!q || !seq_lens || (!sinks && !partial) || !out || !workspace)
     return fail(FLINT_ERR_INVALID_ARG, "%s: NULL pointer argument", who);
   if (B < 1 || B > FLINT_MAX_BATCH) return fail(FLINT_ERR_INVALID_ARG, "%s: B=%d outside [1, %d]", who, B, FLINT_MAX_BATCH);
   if (q_is_fp32 != 0 && q_is_fp32 != 1) return fail(FLINT_ERR_INVALID_ARG, "%s: q_is_fp32 must be 0 or 1", who);
@@ -693,8 +692,9 @@ flint_status flint_attn_decode(const void* q, int32_t q_is_fp32, const flint_kv_
     const Range r = attended_range(*cache, seq_lens[b], window);
     Problem& pb = P.prob[b];
     pb.q = static_cast<const uint8_t*>(q) + static_cast<size_t>(b) * kHeads * kDim * (q_is_fp32 ? 4 : 2);
-    pb.sinks = sinks;
-    pb.out = out + static_cast<size_t>(b) * kHeads * kDim;
+    pb.sinks = partial ? nullptr : sinks;
+    pb.out = out + static_cast<size_t>(b) * (partial ? kCpPartialFloats : kHeads * kDim);
+    pb.partial = static_cast<int8_t>(partial);
     pb.table = cache->layout == FLINT_KV_PAGED
                    ? cache->block_table + static_cast<size_t>(b) * cache->max_blocks_per_req
                    : nullptr;
@@ -731,6 +731,35 @@ flint_status flint_attn_decode(const void* q, int32_t q_is_fp32, const flint_kv_
   P.prep = 0;
   P.eps = 0.f;
   return launch_result(launch_decode(P, grid, static_cast<cudaStream_t>(stream)), who);
+}
+
+flint_status flint_attn_decode(const void* q, int32_t q_is_fp32, const flint_kv_cache* cache,
+                               const int32_t* seq_lens, int32_t B, const float* sinks,
+                               int32_t window, float* out, void* workspace, size_t ws_bytes,
+                               int32_t num_ctas, int32_t* dev_err, void* stream) {
+  return decode_impl(q, q_is_fp32, cache, seq_lens, B, sinks, window, out, workspace, ws_bytes, num_ctas,
+                     dev_err, stream, false, "flint_attn_decode");
+}
+
+flint_status flint_attn_decode_partial(const void* q, int32_t q_is_fp32, const flint_kv_cache* cache,
+                                       const int32_t* seq_lens, int32_t B, float* partials,
+                                       void* workspace, size_t ws_bytes, int32_t num_ctas,
+                                       int32_t* dev_err, void* stream) {
+  return decode_impl(q, q_is_fp32, cache, seq_lens, B, nullptr, 0, partials, workspace, ws_bytes, num_ctas,
+                     dev_err, stream, true, "flint_attn_decode_partial");
+}
+
+flint_status flint_merge_partials(const float* partials, int32_t n_parts, int32_t B, const float* sinks,
+                                  float* out, void* stream) {
+  const char* who = "flint_merge_partials";
+  if (!partials || !sinks || !out) return fail(FLINT_ERR_INVALID_ARG, "%s: NULL pointer argument", who);
+  if (n_parts < 1 || n_parts > FLINT_MAX_CP_PARTS)
+    return fail(FLINT_ERR_INVALID_ARG, "%s: n_parts=%d outside [1, %d]", who, n_parts, FLINT_MAX_CP_PARTS);
+  if (B < 1 || B > FLINT_MAX_BATCH) return fail(FLINT_ERR_INVALID_ARG, "%s: B=%d outside [1, %d]", who, B, FLINT_MAX_BATCH);
+  if (!aligned16(partials) || !aligned16(out) || (reinterpret_cast<uintptr_t>(sinks) & 3u))
+    return fail(FLINT_ERR_INVALID_ARG, "%s: partials/out must be 16-byte aligned", who);
+  return launch_result(launch_merge_partials(partials, n_parts, B, sinks, out, static_cast<cudaStream_t>(stream)),
+                       who);
 }
 
 flint_status flint_attn_stack(const flint_layer* layers, int32_t n_layers, int32_t pos, float eps,

@@ -627,6 +627,21 @@ __device__ __forceinline__ int partial_f4(int head, int c, int q) {
 // 8n + 2c + {0,1} of head `head`.
 __device__ __forceinline__ void finish_head(const Problem& pb, int head, int c, float M, float L,
                                             const float (&v)[32], float sink) {
+  if (pb.partial) {
+    // unnormalised partial for a later merge across ranks: O, m, l
+    float* dst = pb.out + head * kDim;
+    const int d0 = dim_d0(c, pb.fp8 != 0), d2 = dim_d2(c, pb.fp8 != 0);
+#pragma unroll
+    for (int q = 0; q < 8; ++q) {
+      *reinterpret_cast<float2*>(dst + 16 * q + d0) = make_float2(v[4 * q], v[4 * q + 1]);
+      *reinterpret_cast<float2*>(dst + 16 * q + d2) = make_float2(v[4 * q + 2], v[4 * q + 3]);
+    }
+    if (c == 0) {
+      pb.out[kHeads * kDim + head] = M;
+      pb.out[kHeads * kDim + kHeads + head] = L;
+    }
+    return;
+  }
   const float s2 = sink * kLog2e;
   const float Mf = fmaxf(M, s2);
   const float a = (M == -INFINITY) ? 0.f : exp2f(M - Mf);
@@ -699,7 +714,7 @@ __device__ void run_consumer(const DecodeParams& P, const Smem& S, int warp, int
     const Item item = P.items[it];
     const Problem& pb = P.prob[item.seg];
     // this head's sink logit, needed only at the item's end: load it now
-    const float sink = pb.sinks[head];
+    const float sink = pb.sinks ? pb.sinks[head] : 0.f;
     // E4M3 cache: the KV head's scales (unused for bf16)
     const float k_scale = P.kv_scales[pb.map_k >> 1][kvh];
     const float v_scale = P.kv_scales[pb.map_k >> 1][4 + kvh];
@@ -940,6 +955,17 @@ __device__ __forceinline__ void fold_chunk(const DecodeParams& P, int s0, int s1
 // Writes values 4q..4q+3 of (head, c), with the sink folded in as finish_head does.
 __device__ __forceinline__ void write_chunk(const Problem& pb, int head, int c, int q, float m, float l,
                                             float4 acc, float sink) {
+  if (pb.partial) {
+    float* o = pb.out + head * kDim + 16 * q;
+    const int d0 = dim_d0(c, pb.fp8 != 0), d2 = dim_d2(c, pb.fp8 != 0);
+    *reinterpret_cast<float2*>(o + d0) = make_float2(acc.x, acc.y);
+    *reinterpret_cast<float2*>(o + d2) = make_float2(acc.z, acc.w);
+    if (c == 0 && q == 0) {
+      pb.out[kHeads * kDim + head] = m;
+      pb.out[kHeads * kDim + kHeads + head] = l;
+    }
+    return;
+  }
   const float s2 = sink * kLog2e;
   const float Mf = fmaxf(m, s2);
   const float a = (m == -INFINITY) ? 0.f : exp2f(m - Mf);
@@ -962,7 +988,7 @@ __device__ void grid_merge(const DecodeParams& P, const Smem& S) {
       const int kvh = (u / 8) % kKvHeads, q = u % 8;
       const int head = kvh * kGroup + (lane >> 2);
       const Problem& pb = P.prob[p];
-      const float sink = pb.sinks[head];  // in flight with the partials
+      const float sink = pb.sinks ? pb.sinks[head] : 0.f;  // in flight with the partials
       float m = -INFINITY, l = 0.f;
       float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
       fold_chunk(P, P.seg_item_begin[p], P.seg_item_begin[p + 1], 0, 1, head, c, q, m, l, acc);
@@ -976,7 +1002,7 @@ __device__ void grid_merge(const DecodeParams& P, const Smem& S) {
     const int kvh = (u / 8) % kKvHeads, q = u % 8;
     const int head = kvh * kGroup + (lane >> 2);
     const Problem& pb = P.prob[p];
-    const float sink = pb.sinks[head];
+    const float sink = pb.sinks ? pb.sinks[head] : 0.f;
     float m = -INFINITY, l = 0.f;
     float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
     fold_chunk(P, P.seg_item_begin[p], P.seg_item_begin[p + 1], warp, kWarps, head, c, q, m, l, acc);

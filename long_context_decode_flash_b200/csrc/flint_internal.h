@@ -94,7 +94,8 @@ struct Problem {
   int8_t layout, q_fp32, rope;
   int8_t deferred;          // 1: merged by the whole grid after a grid barrier
   int8_t fp8;               // 1: E4M3 cache, 64-token tiles, scales in kv_scales[map_k / 2]
-  int8_t pad_;
+  int8_t partial;           // 1: out receives the unnormalised partial (O [32][128], m [32],
+                            //    l [32]; log2 units) and no sink is folded in (sinks may be NULL)
 };
 static_assert(sizeof(Problem) == 128, "Problem stays 128 bytes");
 
@@ -184,10 +185,16 @@ struct PrefillParams {
   int32_t window;
 };
 
+// A partial as the context-parallel calls exchange it: O [32][128] (natural
+// dims), m [32], l [32], fp32.
+constexpr int kCpPartialFloats = kHeads * kDim + 2 * kHeads;
+
 // Launchers (return cudaGetLastError() after the launch).
 cudaError_t launch_decode(const DecodeParams& p, int grid, cudaStream_t stream);  // cooperative if p.grid_merge
 cudaError_t launch_prep(const PrepParams& p, int B, cudaStream_t stream);
 cudaError_t launch_prefill(const PrefillParams& p, cudaStream_t stream);
+cudaError_t launch_merge_partials(const float* partials, int n_parts, int B, const float* sinks, float* out,
+                                  cudaStream_t stream);
 
 size_t decode_smem_bytes();
 

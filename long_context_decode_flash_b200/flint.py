@@ -33,8 +33,10 @@ EXPORTED = (
     "flint_status_string", "flint_last_error", "flint_kv_bytes", "flint_qk_norm_rope",
     "flint_kv_append", "flint_attn_workspace_bytes", "flint_attn_decode", "flint_attn_stack",
     "flint_attn_stack_noalloc", "flint_attn_layers_serial", "flint_plan_items", "flint_plan_split",
-    "flint_prefill_qk_norm_rope", "flint_prefill_attn",
+    "flint_prefill_qk_norm_rope", "flint_prefill_attn", "flint_attn_decode_partial",
+    "flint_merge_partials",
 )
+CP_PARTIAL_FLOATS = 32 * 128 + 2 * 32
 
 
 class FlintError(RuntimeError):
@@ -94,13 +96,16 @@ def load_library() -> ctypes.CDLL:
             lib.flint_prefill_qk_norm_rope.argtypes = [P, P, P, P, P, I32, ctypes.c_float,
                                                        ctypes.c_double, I32, P, P, P, P, P, P]
             lib.flint_prefill_attn.argtypes = [P, P, P, I32, P, I32, P, P, P]
+            lib.flint_attn_decode_partial.argtypes = [P, I32, P, P, I32, P, P, ctypes.c_size_t, I32, P, P]
+            lib.flint_merge_partials.argtypes = [P, I32, I32, P, P, P]
             lib.flint_plan_items.argtypes = [P, I32, I32, I32, P, P, P, P, I32]
             lib.flint_plan_items.restype = I32
             lib.flint_plan_split.argtypes = [P, I32, I32, I32, I32, P, P, P, P, P]
             lib.flint_plan_split.restype = I32
             for name in ("flint_qk_norm_rope", "flint_kv_append", "flint_attn_decode",
                          "flint_attn_stack", "flint_attn_stack_noalloc", "flint_attn_layers_serial",
-                         "flint_prefill_qk_norm_rope", "flint_prefill_attn"):
+                         "flint_prefill_qk_norm_rope", "flint_prefill_attn", "flint_attn_decode_partial",
+                         "flint_merge_partials"):
                 getattr(lib, name).restype = ctypes.c_int
             _lib = lib
     return _lib
@@ -235,6 +240,29 @@ def flint_attn_decode(q, cache: KVCache, seq_lens: Sequence[int], sinks, window:
                                  _i32_host(seq_lens), len(seq_lens), _ptr(sinks), int(window),
                                  _ptr(out), _ptr(ws), ws.numel() * ws.element_size(), int(num_ctas),
                                  _ptr(dev_err), _stream(stream)))
+    return out
+
+
+def flint_attn_decode_partial(q, cache: KVCache, seq_lens: Sequence[int], partials, ws: torch.Tensor,
+                              num_ctas: int = 0, dev_err=None, stream=None):
+    """This rank's unnormalised attention over tokens [0, seq_lens[b]) of its
+    cache: partials fp32 [B, CP_PARTIAL_FLOATS] (O [32,128], m [32], l [32])."""
+    if q.dtype not in (torch.bfloat16, torch.float32):
+        raise FlintError(FLINT_ERR_INVALID_ARG, "q must be bf16 or fp32")
+    lib = load_library()
+    _check(lib.flint_attn_decode_partial(_ptr(q), int(q.dtype == torch.float32), ctypes.byref(cache),
+                                         _i32_host(seq_lens), len(seq_lens), _ptr(partials), _ptr(ws),
+                                         ws.numel() * ws.element_size(), int(num_ctas), _ptr(dev_err),
+                                         _stream(stream)))
+    return partials
+
+
+def flint_merge_partials(partials, sinks, out, stream=None):
+    """Merge partials fp32 [n_parts, B, CP_PARTIAL_FLOATS] with the sinks into
+    out fp32 [B, 32, 128]."""
+    n, B = int(partials.shape[0]), int(partials.shape[1])
+    lib = load_library()
+    _check(lib.flint_merge_partials(_ptr(partials), n, B, _ptr(sinks), _ptr(out), _stream(stream)))
     return out
 
 

@@ -141,6 +141,23 @@ def test_prefill_rejects_bad_arguments_on_the_host():
                                           None, None) == E                             # cache without v
 
 
+def test_context_parallel_calls_reject_bad_arguments_on_the_host():
+    lib = flint.load_library()
+    p = ctypes.c_void_p(0x10000)
+    E = flint.FLINT_ERR_INVALID_ARG
+    assert lib.flint_merge_partials(p, 0, 1, p, p, None) == E                       # no partials
+    assert lib.flint_merge_partials(p, 1025, 1, p, p, None) == E                    # above the maximum
+    assert lib.flint_merge_partials(p, 2, 65, p, p, None) == E                      # B too large
+    assert lib.flint_merge_partials(ctypes.c_void_p(0x10004), 2, 1, p, p, None) == E  # unaligned
+    assert lib.flint_merge_partials(p, 2, 1, None, p, None) == E                    # no sinks
+    c = _fake_cache(capacity=100)
+    lens = (ctypes.c_int32 * 1)(101)
+    st = lib.flint_attn_decode_partial(p, 0, ctypes.byref(c), lens, 1, p, p, 1 << 30, 0, None, None)
+    assert st == E and "capacity" in lib.flint_last_error().decode()                 # 101 tokens, 100 slots
+    lens = (ctypes.c_int32 * 1)(0)
+    assert lib.flint_attn_decode_partial(p, 0, ctypes.byref(c), lens, 1, p, p, 1 << 30, 0, None, None) == E
+
+
 def test_workspace_bytes_bounds():
     assert flint.flint_attn_workspace_bytes(0, 148) == 0
     assert flint.flint_attn_workspace_bytes(65, 148) == 0
