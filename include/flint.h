@@ -312,8 +312,11 @@ flint_status flint_prefill_attn(const uint16_t* q, const uint16_t* k, const uint
  *   partials  fp32 [B][FLINT_CP_PARTIAL_FLOATS] (device, out): for request b,
  *             O [32][128], then m [32], then l [32], with scores in log2
  *             units (s'_j = q_h . k_j / sqrt(128) * log2(e)):
- *             m_h = max_j s'_j, l_h = sum_j 2^(s'_j - m_h),
- *             O_h = sum_j 2^(s'_j - m_h) v_j (up to rounding order).
+ *             l_h = sum_j 2^(s'_j - m_h), O_h = sum_j 2^(s'_j - m_h) v_j (up
+ *             to rounding order), where m_h is the reference the kernel
+ *             scaled by: its running maximum, which moves only by steps of
+ *             more than 8, so max_j s'_j - 8 <= m_h <= max_j s'_j.  The triple
+ *             is defined up to the common factor 2^m_h.
  * Other arguments, the workspace and errors as flint_attn_decode. */
 flint_status flint_attn_decode_partial(const void* q, int32_t q_is_fp32,
                                        const flint_kv_cache* cache, const int32_t* seq_lens,

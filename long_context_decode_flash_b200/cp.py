@@ -33,8 +33,9 @@ def rank_ranges(L: int, world: int) -> List[Tuple[int, int]]:
 
 
 def gather_partials(part: torch.Tensor, group=None) -> torch.Tensor:
-    """All ranks' partials [B, F] stacked in rank order: [world, B, F]."""
-    world = dist.get_world_size(group)
+    """All ranks' partials [B, F] stacked in rank order: [world, B, F]; a
+    process without a process group is a single rank."""
+    world = dist.get_world_size(group) if dist.is_initialized() else 1
     if world == 1:
         return part.unsqueeze(0)
     bufs = [torch.empty_like(part) for _ in range(world)]

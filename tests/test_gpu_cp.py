@@ -80,7 +80,9 @@ def test_one_rank_partial_matches_the_oracle_partial_and_merges_to_decode():
     p = parts[0, 0].cpu().numpy().astype(np.float64)
     O, m, lsum = p[:4096].reshape(32, 128), p[4096:4128], p[4128:]
     Ow, mw, lw = oracle.attn_partial(I.bits(d.q[0]), I.bits(d.k_cache[0]), I.bits(d.v_cache[0]))
-    assert np.abs(m - mw).max() <= 1e-3
+    # the kernel's reference m is its running maximum, which moves only by
+    # steps of more than 8: within 8 below the true maximum
+    assert (m <= mw + 1e-3).all() and (m >= mw - 8 - 1e-3).all()
     # the triple is defined up to the common factor 2^m: compare at the oracle's m
     f = np.exp2(m - mw)
     np.testing.assert_allclose(lsum * f, lw, rtol=1e-4)
