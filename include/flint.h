@@ -1,6 +1,13 @@
 /*
- * flint.h -- C ABI of libflint.so: one decode step of Flint attention on a
- * B200 (sm_100a), batch 1 or a batch of paged requests.
+ * flint.h -- C ABI of libflint.so: Flint attention on a B200 (sm_100a).
+ *   - decode: one step for batch 1 or a batch of paged requests
+ *     (flint_qk_norm_rope, flint_kv_append, flint_attn_decode), all 49 layers
+ *     of a token in one launch (flint_attn_stack, flint_attn_stack_noalloc)
+ *     or as 49 dependent launches (flint_attn_layers_serial); bf16 or E4M3
+ *     caches;
+ *   - prefill of a prompt (flint_prefill_qk_norm_rope, flint_prefill_attn);
+ *   - context-parallel decode across GPUs (flint_attn_decode_partial,
+ *     flint_merge_partials).
  *
  * Model facts the operations follow (page title, section):
  *   - "Day-0 Support for Flint on vLLM" (hnkhoi.com/news/1467), "Model
