@@ -182,6 +182,32 @@ def run_reference(args, rank):
 
     oracle.build()
     nthreads = os.cpu_count() or 1
+    if args.workload == "cp262k":
+        import numpy as np
+        L = args.context
+        d = I.make_decode(L, workload=I.W_FULL_100K)
+        qb, kb, vb = I.bits(d.q[0]), I.bits(d.k_cache[0]), I.bits(d.v_cache[0])
+        sinks = d.sinks.numpy().astype(np.float64)
+        vals = []
+        for i in range(max(1, args.steps) + 1):
+            t0 = time.perf_counter()
+            oracle.attn_decode(qb, kb, vb, L, sinks, 0, capacity=L, nthreads=nthreads)
+            if i > 0:  # the first run warms the caches
+                vals.append((time.perf_counter() - t0) * 1e6)
+        us = statistics.mean(vals)
+        sample = f"{len(vals)} whole-context oracle decodes of the layer at context {L}"
+        line = {
+            "impl": "reference", "metric": "full-layer decode-attention us/token @262,144 ctx, context-parallel "
+                                          "over the GPUs",
+            "value": us, "unit": "us/token", "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": us / 1000.0, "higher_is_better": False, "scaling": "strong", "vs_baseline": None,
+            "dtype": "f64", "data": "synthetic", "config": {"workload": "one full-context NoPE layer, one token",
+                                                             "context": L},
+            "cpu_baseline": {"value": us, "unit": "us/token", "cores": nthreads, "kind": "oracle", "sample": sample},
+            "e2e": {"value": us, "unit": "us/token", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+        }
+        print(json.dumps(line), flush=True)
+        return
     if args.workload == "prefill8k":
         T = args.context
         prompts = prefill_inputs(I, T, kinds_only=True)
