@@ -61,3 +61,18 @@ def test_single_rank_needs_no_process_group():
     import bench
     assert bench.max_over_ranks(0.5, 1, "cpu") == 0.5
     assert bench.per_token_us(0.5, 1) == pytest.approx(500.0)
+
+
+def test_prefill_work_counts_match_brute_force():
+    """The prefill roofline's algorithmic work: keys attended summed row by
+    row (row t attends min(t + 1, window) keys, or t + 1), 4 x 128 FLOP per
+    (row, key, head) over 32 heads."""
+    import bench
+    for T in (1, 2, 100, 512, 513, 514, 2000, 8192):
+        for window in (0, 513):
+            brute = sum(min(t + 1, window) if window else t + 1 for t in range(T))
+            assert bench.prefill_keys(T, window) == brute
+            assert bench.prefill_flops(T, window) == brute * 32 * 128 * 4
+    # the 49-layer prompt of the benchmark: 14 full and 35 window layers
+    total = 14 * bench.prefill_flops(8192, 0) + 35 * bench.prefill_flops(8192, 513)
+    assert total == 10_032_091_496_448
