@@ -211,11 +211,12 @@ def run_reference(args, rank):
     if args.workload == "prefill8k":
         T = args.context
         prompts = prefill_inputs(I, T, kinds_only=True)
-        oracle_prefill_sample(prompts, T, nthreads, budget_s=2.0)  # warm-up
-        budget = max(5.0, min(30.0, 150.0 / max(1, args.steps)))
+        cache = {}
+        oracle_prefill_sample(prompts, T, nthreads, budget_s=2.0, prep_cache=cache)  # warm-up, norm passes
+        budget = max(0.5, min(30.0, 150.0 / max(1, args.steps)))
         vals, sample = [], ""
         for _ in range(args.steps):
-            ms, _, sample = oracle_prefill_sample(prompts, T, nthreads, budget_s=budget)
+            ms, _, sample = oracle_prefill_sample(prompts, T, nthreads, budget_s=budget, prep_cache=cache)
             vals.append(ms)
         ms = statistics.mean(vals)
         line = {
@@ -235,7 +236,7 @@ def run_reference(args, rank):
     layers_win = [I.make_layer(I.W_STACK_100K, 0, CONTEXT, 513, True, ring=True)]
     oracle_sample(layers_full, layers_win, nthreads, budget_s=1.0)  # warm-up
     # each step is a bounded sample; the whole run stays within a few minutes
-    budget = max(2.0, min(20.0, 120.0 / max(1, args.steps)))
+    budget = max(0.5, min(20.0, 120.0 / max(1, args.steps)))
     vals = []
     for _ in range(args.steps):
         us_step, _, sample = oracle_sample(layers_full, layers_win, nthreads, budget_s=budget)
@@ -292,24 +293,31 @@ def prefill_inputs(I, T, kinds_only=False, n_layers=49):
     return [I.make_prefill(T, 0 if full else 513, layer=i) for i, full in enumerate(kinds[:n_layers])]
 
 
-def oracle_prefill_sample(prompts, T, nthreads, budget_s=10.0):
+def oracle_prefill_sample(prompts, T, nthreads, budget_s=10.0, prep_cache=None):
     """Time the oracle's prefill of one window and one full layer on a bounded
     sample: its norm (+RoPE) pass over all T tokens, then the attention of as
     many uniformly drawn rows as the budget allows, whose mean time is scaled
-    to all T rows.  Returns (ms per prompt scaled to 35 window + 14 full
-    layers, seconds spent, description)."""
+    to all T rows.  prep_cache (a dict) keeps each layer's norm pass and its
+    time across calls, so repeated samples time only rows.  Returns (ms per
+    prompt scaled to 35 window + 14 full layers, seconds spent, description)."""
     import numpy as np
     import oracle
     from long_context_decode_flash_b200 import inputs as I
 
     rng = np.random.default_rng(1)
     est, spent, desc = [], 0.0, []
-    for p, share in zip(prompts, (0.3, 0.7)):
+    for i, (p, share) in enumerate(zip(prompts, (0.3, 0.7))):
         sinks, v = p.sinks.numpy().astype(np.float64), I.bits(p.v_raw)
-        t0 = time.perf_counter()
-        _, qb, kb = oracle.prefill(I.bits(p.q_raw), I.bits(p.k_raw), v, I.bits(p.w_q), I.bits(p.w_k),
-                                   sinks, p.window, p.rope, rows=[], nthreads=nthreads)
-        t_prep = time.perf_counter() - t0
+        if prep_cache is not None and i in prep_cache:
+            qb, kb, t_prep = prep_cache[i]
+        else:
+            t0 = time.perf_counter()
+            _, qb, kb = oracle.prefill(I.bits(p.q_raw), I.bits(p.k_raw), v, I.bits(p.w_q), I.bits(p.w_k),
+                                       sinks, p.window, p.rope, rows=[], nthreads=nthreads)
+            t_prep = time.perf_counter() - t0
+            spent += t_prep
+            if prep_cache is not None:
+                prep_cache[i] = (qb, kb, t_prep)
         rows, t_rows, t_end = 0, 0.0, time.perf_counter() + share * budget_s
         while rows == 0 or time.perf_counter() < t_end:
             t = int(rng.integers(0, T))
@@ -318,7 +326,7 @@ def oracle_prefill_sample(prompts, T, nthreads, budget_s=10.0):
             t_rows += time.perf_counter() - t0
             rows += 1
         est.append(t_prep + t_rows / rows * T)
-        spent += t_prep + t_rows
+        spent += t_rows
         desc.append(f"{rows} random rows of a {'window' if p.window else 'full'} layer")
     ms = (35 * est[0] + 14 * est[1]) * 1e3
     return ms, spent, (", ".join(desc) + f" of the {T}-token prompt after the oracle's norm (+RoPE) of "
