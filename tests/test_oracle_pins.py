@@ -558,3 +558,15 @@ def test_partial_is_unnormalised_softmax_and_merge_without_sink_is_sdpa():
     assert np.isneginf(empty[1]).all() and (empty[2] == 0).all()
     sinks = np.full(nq, -np.inf)
     np.testing.assert_allclose(oracle.merge_partials([empty, (O, m, lsum)], sinks), sdpa, rtol=1e-12, atol=1e-13)
+
+
+def test_storage_row_follows_each_layout():
+    """Slot of a logical position: contiguous t, ring t mod capacity, paged
+    table[t // 64] * 64 + t mod 64 ("Model architecture": window layers keep
+    513 tokens; the paged layout is a block table of 64-token blocks)."""
+    table = np.array([5, 0, 7, 2], np.int32)
+    for t in (0, 1, 63, 64, 100, 255):
+        assert oracle.storage_row(oracle.CONTIGUOUS, t) == t
+        assert oracle.storage_row(oracle.PAGED, t, block_table=table, block_size=64) == table[t // 64] * 64 + t % 64
+    for t in (0, 512, 513, 1025, 100_000):
+        assert oracle.storage_row(oracle.RING, t, capacity=513) == t % 513
