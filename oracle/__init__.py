@@ -224,18 +224,24 @@ def merge_partials(parts, sinks):
     """The log-sum-exp merge of partials (O_r, m_r, l_r) from attn_partial with
     each head's sink logit, which joins the softmax with no value (same page,
     "Learned attention sinks"): M = max(sink log2(e), max_r m_r),
-    out = sum_r 2^(m_r - M) O_r / (2^(sink log2(e) - M) + sum_r 2^(m_r - M) l_r)."""
+    out = sum_r 2^(m_r - M) O_r / (2^(sink log2(e) - M) + sum_r 2^(m_r - M) l_r).
+    A head with no key in any partial and a sink of -inf has no softmax mass
+    at all (M = -inf); its output is taken as 0, since nothing carries a value
+    (the reading that an empty split adds nothing, never a NaN)."""
     sinks = _f64(sinks) * _LOG2E
     M = sinks.copy()
     for _, m, _ in parts:
         M = np.maximum(M, m)
+    empty = np.isneginf(M)
+    Mz = np.where(empty, 0.0, M)
     num = 0.0
-    den = np.exp2(sinks - M)
+    den = np.where(np.isneginf(sinks), 0.0, np.exp2(np.where(np.isneginf(sinks), 0.0, sinks) - Mz))
     for O, m, lsum in parts:
-        w = np.where(np.isneginf(m), 0.0, np.exp2(np.where(np.isneginf(m), 0.0, m) - M))
+        w = np.where(np.isneginf(m), 0.0, np.exp2(np.where(np.isneginf(m), 0.0, m) - Mz))
         num = num + w[:, None] * O
         den = den + w * lsum
-    return num / den[:, None]
+    num = num * np.ones((len(M), 1))
+    return np.where(empty[:, None], 0.0, num / np.where(empty, 1.0, den)[:, None])
 
 
 def decode_layer(q_raw, k_raw, v_raw, w_q, w_k, sinks, k_cache, v_cache, L: int,

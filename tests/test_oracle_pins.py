@@ -560,6 +560,24 @@ def test_partial_is_unnormalised_softmax_and_merge_without_sink_is_sdpa():
     np.testing.assert_allclose(oracle.merge_partials([empty, (O, m, lsum)], sinks), sdpa, rtol=1e-12, atol=1e-13)
 
 
+def test_merge_of_only_empty_partials_with_a_minus_inf_sink_is_zero():
+    """No key in any partial and a sink of -inf: no softmax mass anywhere, and
+    the merge gives 0 for those heads (not 0/0); heads with a finite sink give
+    0 too (the sink carries no value), and a head whose sink is -inf next to
+    a non-empty partial is plain softmax attention."""
+    nq, d = 4, 16
+    q = rng.normal(size=(nq, d))
+    K, V = bf16_bits((8, 1, d), 431), bf16_bits((8, 1, d), 432)
+    empty = oracle.attn_partial(q, K[:0], V[:0])
+    sinks = np.array([-np.inf, -np.inf, 0.5, -3.0])
+    out = oracle.merge_partials([empty, empty, empty], sinks)
+    assert np.isfinite(out).all() and (out == 0).all()
+    full = oracle.attn_partial(q, K, V)
+    sinks = np.full(nq, -np.inf)
+    want = full[0] / full[2][:, None]
+    np.testing.assert_allclose(oracle.merge_partials([empty, full, empty], sinks), want, rtol=1e-12, atol=1e-13)
+
+
 def test_storage_row_follows_each_layout():
     """Slot of a logical position: contiguous t, ring t mod capacity, paged
     table[t // 64] * 64 + t mod 64 ("Model architecture": window layers keep
