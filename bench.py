@@ -34,13 +34,14 @@ CONTEXT = 100_000
 NOMINAL_HBM_GBS = 8000.0
 
 # DRAM traffic (dram__bytes_read.sum + dram__bytes_write.sum) of one decode_kernel
-# launch from a full-size, one-pass ncu capture of the stack at context 100,000
-# (profiles/decode_kernel_stack100k_traffic.md), per KV dtype, with the hash of the CUDA
-# sources it was taken on; reported only while the sources still hash the same.
+# launch from a full-size, one-pass ncu capture (those two metrics and the
+# launch duration, --clock-control none, one launch after the warm-up) of each
+# workload, per KV dtype, with the hash of the CUDA sources it was taken on;
+# reported only while the sources still hash the same.
 TRAFFIC = {("stack", 100_000, "bf16"): (2_906_088_192 + 6_870_528, "38ee5c4a48fcdd23"),
            ("stack", 100_000, "fp8"): (1_453_981_440 + 6_602_496, "cde382082669d367")}
 # The same for one prefill_kernel launch of a full (NoPE) layer on the
-# 8,192-token prompt (profiles/prefill_kernel_prefill8k_full.md).
+# 8,192-token prompt (a --set full capture of that one launch).
 PREFILL_TRAFFIC = {8192: (83_963_648 + 80_508_928, "38ee5c4a48fcdd23")}
 
 

@@ -190,7 +190,12 @@ size_t flint_attn_workspace_bytes(int32_t n_problems, int32_t num_ctas);
 /* Split-KV flash-decode over a batch of B requests of one layer: q already
  * normed (and roped).  The new token is already in the cache; request b
  * attends positions [max(0, L_b - window), L_b) (window 513) or [0, L_b)
- * (window 0), L_b = seq_lens[b].
+ * (window 0), L_b = seq_lens[b].  What it computes is the attention of
+ * "Day-0 Support for Flint on vLLM" (hnkhoi.com), "Model architecture": GQA
+ * with 32 query over 4 KV heads of 128 dims, a learned sink logit per query
+ * head that joins the softmax without a value, and either a 513-token window
+ * or the whole context; the batch-1 decode at 100,000 tokens it serves is the
+ * one of the same page on newruntime.com, "What happened".
  *   q         bf16 or fp32 [B][32][128] (device); q_is_fp32 selects
  *   cache     any layout; RING requires window == 513 and capacity 513
  *   seq_lens  HOST int32 [B], 1 <= L_b <= FLINT_MAX_CONTEXT (and <= capacity
@@ -202,7 +207,12 @@ size_t flint_attn_workspace_bytes(int32_t n_problems, int32_t num_ctas);
  *   num_ctas  0 = one CTA per SM (the tuned default)
  * B in [1, FLINT_MAX_BATCH].  Result is deterministic run to run for a given
  * workspace size and num_ctas: queued chunks have fixed bounds, whichever CTA
- * takes them, and partials are merged in a fixed order. */
+ * takes them, and partials are merged in a fixed order.  A PAGED block id
+ * outside [0, num_blocks) is never handed to a load: that tile is skipped, the
+ * output is meaningless, and *dev_err = FLINT_ERR_INVALID_ARG.  A pipeline
+ * wait that runs past its time limit sets *dev_err = FLINT_ERR_TIMEOUT; the
+ * kernel then lets its copies in flight land and returns (zero the workspace
+ * before the next call). */
 flint_status flint_attn_decode(const void* q, int32_t q_is_fp32,
                                const flint_kv_cache* cache, const int32_t* seq_lens,
                                int32_t B, const float* sinks, int32_t window,
@@ -212,7 +222,12 @@ flint_status flint_attn_decode(const void* q, int32_t q_is_fp32,
 /* One decoded token through n_layers attention layers in ONE launch: for each
  * layer, per-head Q/K RMSNorm (+RoPE if layer.rope), append of k and v_raw at
  * position pos, and decode attention over the layer's window, all scheduled
- * together across the GPU (the layers are independent problems here).
+ * together across the GPU (the layers are independent problems here).  The
+ * layer stack is Flint's ("Day-0 Support for Flint on vLLM", hnkhoi.com,
+ * "Model architecture"): 49 layers, 35 with a 513-token window and RoPE, 14
+ * over the full context without positional encoding, each with per-head Q/K
+ * RMSNorm and sinks; the norm, rotary and cache steps fused with attention
+ * follow the same page on newruntime.com, "What happened".
  *   layers    HOST array [n_layers], 1 <= n_layers <= FLINT_MAX_LAYERS;
  *             window layers usually RING caches, full layers CONTIGUOUS
  *   pos       position of the new token (context pos + 1 after the append)
@@ -249,11 +264,16 @@ flint_status flint_attn_layers_serial(const flint_layer* layers, int32_t n_layer
  *   device memory of every device its device code is loaded on, until the
  *   process exits.  Calls whose smallest workspace,
  *   4096 + (CTAs + n_layers) * 16640 bytes, exceeds it are refused with
- *   FLINT_ERR_WORKSPACE (49 layers fit with up to 202 CTAs).  The scratch is
+ *   FLINT_ERR_WORKSPACE; CTAs counts the CTAs a launch uses, num_ctas (0: one
+ *   per SM) but never more than the device has SMs.  49 layers fit with up to
+ *   202 CTAs, so on a device of 202 SMs or fewer (a 148-SM B200) no call is
+ *   refused for its size.  The scratch is
  *   below flint_attn_workspace_bytes, so the run-time balancing queue is
  *   coarser than with a full workspace (same results up to rounding order).
  *   Set-up: the first call on a device, with that device current, looks up the
- *   scratch's address; make it before any stream capture.
+ *   scratch's address; make it before any stream capture.  The address
+ *   belongs to the device's CUDA context: after a device reset the first call
+ *   looks it up again, and must again come before any capture.
  *   Sharing: every call on a device uses the same scratch, which keeps the last
  *   call's contents; each call clears the counters it needs on `stream` first.
  *   Calls that overlap on the GPU (other streams, other threads) race.
@@ -339,7 +359,8 @@ flint_status flint_attn_decode_partial(const void* q, int32_t q_is_fp32,
  *   partials  fp32 [n_parts][B][FLINT_CP_PARTIAL_FLOATS] (device, in)
  *   sinks     fp32 [32] (device, in);  out  fp32 [B][32][128] (device, out)
  * n_parts in [1, FLINT_MAX_CP_PARTS], B in [1, FLINT_MAX_BATCH].  A partial
- * with m = -inf (no tokens) contributes nothing. */
+ * with m = -inf (no tokens) contributes nothing; a head with no token in any
+ * partial and a sink of -inf (M = -inf) gets the output 0. */
 flint_status flint_merge_partials(const float* partials, int32_t n_parts, int32_t B,
                                   const float* sinks, float* out, void* stream);
 

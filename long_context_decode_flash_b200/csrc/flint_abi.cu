@@ -13,6 +13,7 @@
 #include <mutex>
 #include <string>
 #include <unordered_map>
+#include <vector>
 
 #include "flint_internal.h"
 
@@ -427,10 +428,39 @@ namespace flint {
 
 size_t workspace_min_bytes(int n_problems, int num_ctas) {
   if (n_problems < 1 || n_problems > kMaxProblems || num_ctas < 0 || num_ctas > kMaxCtas) return 0;
-  int g = num_ctas;
-  if (g == 0 && device_num_sms(&g) != 0) g = kMaxCtas;
-  g = std::min(g, kMaxCtas);
+  // the CTAs plan() launches: num_ctas (0: one per SM), never more than the
+  // device's SMs (kMaxCtas if the count cannot be read)
+  int sms = kMaxCtas;
+  if (device_num_sms(&sms) != 0) sms = kMaxCtas;
+  const int g = std::min(num_ctas == 0 ? sms : std::min(num_ctas, sms), kMaxCtas);
   return kCounterBytes + static_cast<size_t>(std::min(kMaxItems, g + n_problems)) * kPartialBytes;
+}
+
+void* current_context() {
+  typedef CUresult (*GetCtxFn)(CUcontext*);
+  static GetCtxFn fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<GetCtxFn>(p);
+  });
+  CUcontext ctx = nullptr;
+  if (!fn || fn(&ctx) != CUDA_SUCCESS) return nullptr;
+  return ctx;
+}
+
+cudaError_t configure_once(ContextSet& done, const void* kernel, int bytes) {
+  void* ctx = current_context();
+  std::lock_guard<std::mutex> lock(done.mu);
+  if (ctx && std::find(done.ctxs.begin(), done.ctxs.end(), ctx) != done.ctxs.end()) return cudaSuccess;
+  const cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+  if (e != cudaSuccess) return e;
+  // with no context yet the call above made one; the next launch records it
+  if (ctx) done.ctxs.push_back(ctx);
+  return cudaSuccess;
 }
 
 flint_status record_error(flint_status s, const char* fmt, ...) {
@@ -475,6 +505,7 @@ flint_status flint_qk_norm_rope(const uint16_t* q_raw, const uint16_t* k_raw, co
                                 int32_t B, float eps, double theta, int32_t apply_rope,
                                 float* q_out, uint16_t* k_out, const flint_kv_cache* cache,
                                 int32_t* dev_err, void* stream) {
+  FLINT_NVTX_RANGE("flint_qk_norm_rope");
   const char* who = "flint_qk_norm_rope";
   if (!q_raw || !k_raw || !w_q || !w_k || !pos)
     return fail(FLINT_ERR_INVALID_ARG, "%s: NULL input pointer", who);
@@ -531,6 +562,7 @@ flint_status flint_qk_norm_rope(const uint16_t* q_raw, const uint16_t* k_raw, co
 
 flint_status flint_kv_append(const uint16_t* k, const uint16_t* v, const int32_t* pos, int32_t B,
                              const flint_kv_cache* cache, int32_t* dev_err, void* stream) {
+  FLINT_NVTX_RANGE("flint_kv_append");
   const char* who = "flint_kv_append";
   if (!k || !v || !pos) return fail(FLINT_ERR_INVALID_ARG, "%s: NULL input pointer", who);
   if (!aligned16(k) || !aligned16(v)) return fail(FLINT_ERR_INVALID_ARG, "%s: k/v must be 16-byte aligned", who);
@@ -573,6 +605,7 @@ flint_status flint_prefill_qk_norm_rope(const uint16_t* q_raw, const uint16_t* k
                                         uint16_t* k_out, uint16_t* v_out,
                                         const flint_kv_cache* cache, int32_t* dev_err,
                                         void* stream) {
+  FLINT_NVTX_RANGE("flint_prefill_qk_norm_rope");
   const char* who = "flint_prefill_qk_norm_rope";
   if (!q_raw || !k_raw || !w_q || !w_k) return fail(FLINT_ERR_INVALID_ARG, "%s: NULL input pointer", who);
   if (T < 1 || T > FLINT_MAX_CONTEXT)
@@ -626,6 +659,7 @@ flint_status flint_prefill_qk_norm_rope(const uint16_t* q_raw, const uint16_t* k
 flint_status flint_prefill_attn(const uint16_t* q, const uint16_t* k, const uint16_t* v, int32_t T,
                                 const float* sinks, int32_t window, float* out, int32_t* dev_err,
                                 void* stream) {
+  FLINT_NVTX_RANGE("flint_prefill_attn");
   const char* who = "flint_prefill_attn";
   if (!q || !k || !v || !sinks || !out) return fail(FLINT_ERR_INVALID_ARG, "%s: NULL pointer", who);
   const void* ptrs[] = {q, k, v, sinks, out};
@@ -737,6 +771,7 @@ flint_status flint_attn_decode(const void* q, int32_t q_is_fp32, const flint_kv_
                                const int32_t* seq_lens, int32_t B, const float* sinks,
                                int32_t window, float* out, void* workspace, size_t ws_bytes,
                                int32_t num_ctas, int32_t* dev_err, void* stream) {
+  FLINT_NVTX_RANGE("flint_attn_decode");
   return decode_impl(q, q_is_fp32, cache, seq_lens, B, sinks, window, out, workspace, ws_bytes, num_ctas,
                      dev_err, stream, false, "flint_attn_decode");
 }
@@ -745,12 +780,14 @@ flint_status flint_attn_decode_partial(const void* q, int32_t q_is_fp32, const f
                                        const int32_t* seq_lens, int32_t B, float* partials,
                                        void* workspace, size_t ws_bytes, int32_t num_ctas,
                                        int32_t* dev_err, void* stream) {
+  FLINT_NVTX_RANGE("flint_attn_decode_partial");
   return decode_impl(q, q_is_fp32, cache, seq_lens, B, nullptr, 0, partials, workspace, ws_bytes, num_ctas,
                      dev_err, stream, true, "flint_attn_decode_partial");
 }
 
 flint_status flint_merge_partials(const float* partials, int32_t n_parts, int32_t B, const float* sinks,
                                   float* out, void* stream) {
+  FLINT_NVTX_RANGE("flint_merge_partials");
   const char* who = "flint_merge_partials";
   if (!partials || !sinks || !out) return fail(FLINT_ERR_INVALID_ARG, "%s: NULL pointer argument", who);
   if (n_parts < 1 || n_parts > FLINT_MAX_CP_PARTS)
@@ -765,6 +802,7 @@ flint_status flint_merge_partials(const float* partials, int32_t n_parts, int32_
 flint_status flint_attn_stack(const flint_layer* layers, int32_t n_layers, int32_t pos, float eps,
                               double theta, float* out, void* workspace, size_t ws_bytes,
                               int32_t num_ctas, int32_t* dev_err, void* stream) {
+  FLINT_NVTX_RANGE("flint_attn_stack");
   return run_stack(layers, n_layers, pos, eps, theta, out, workspace, ws_bytes, num_ctas, dev_err, stream, 0,
                    "flint_attn_stack");
 }
@@ -772,6 +810,7 @@ flint_status flint_attn_stack(const flint_layer* layers, int32_t n_layers, int32
 flint_status flint_attn_layers_serial(const flint_layer* layers, int32_t n_layers, int32_t pos, float eps,
                                       double theta, float* out, void* workspace, size_t ws_bytes,
                                       int32_t num_ctas, int32_t* dev_err, void* stream) {
+  FLINT_NVTX_RANGE("flint_attn_layers_serial");
   const char* who = "flint_attn_layers_serial";
   if (!layers || !out) return fail(FLINT_ERR_INVALID_ARG, "%s: NULL pointer argument", who);
   if (n_layers < 1 || n_layers > FLINT_MAX_LAYERS)

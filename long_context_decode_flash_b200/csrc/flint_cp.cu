@@ -8,7 +8,8 @@
 //     out = sum_r 2^(m_r - M) O_r / (2^(s - M) + sum_r 2^(m_r - M) l_r),
 // the log-sum-exp merge of split-KV decoding with the sink as one more
 // logit that carries no value ("Day-0 Support for Flint on vLLM",
-// hnkhoi.com, "Model architecture": learned attention sinks).
+// hnkhoi.com, "Model architecture": learned attention sinks).  With no key
+// anywhere and s = -inf (M = -inf) the output is 0.
 #include "flint_device.cuh"
 
 namespace flint {
@@ -25,6 +26,12 @@ __global__ void __launch_bounds__(kDim) merge_kernel(const float* __restrict__ p
   float M = s2;
   for (int r = 0; r < n; ++r)
     M = fmaxf(M, parts[(static_cast<size_t>(r) * B + b) * kCpPartialFloats + kHeads * kDim + h]);
+  // No key in any partial and a sink of -inf: the softmax has no mass at all;
+  // the output is 0 (nothing carries a value), not 0/0.
+  if (M == -INFINITY) {
+    out[(static_cast<size_t>(b) * kHeads + h) * kDim + d] = 0.f;
+    return;
+  }
   float L = exp2f(s2 - M), o = 0.f;
   for (int r = 0; r < n; ++r) {
     const float* pr = parts + (static_cast<size_t>(r) * B + b) * kCpPartialFloats;

@@ -46,6 +46,26 @@
 
 namespace flint {
 
+// Device-side timeline tracing, compiled in only with -DFLINT_TRACE: thread
+// (0, lane 0 of a role) of every CTA stores %globaltimer at fixed points of
+// its life into g_trace[block][slot]; flint_trace_read copies the table out.
+// Release builds carry no trace code.
+#ifdef FLINT_TRACE
+constexpr int kTraceSlots = 16;
+__device__ unsigned long long g_trace[kMaxCtas][kTraceSlots];
+#define FLINT_TRACE_MARK(slot) (::flint::g_trace[blockIdx.x][(slot)] = ::flint::globaltimer_ns())
+#define FLINT_TRACE_SET(slot, v) (::flint::g_trace[blockIdx.x][(slot)] = (v))
+#else
+#define FLINT_TRACE_MARK(slot) ((void)0)
+#define FLINT_TRACE_SET(slot, v) ((void)0)
+#endif
+
+#ifdef FLINT_TEST_HOOKS
+// {block, tile sequence number}: that CTA's producer leaves that tile's stage
+// unarmed (no load, no expected bytes); {-1, -1} = off.
+__device__ int g_stall_decode[2] = {-1, -1};
+#endif
+
 namespace {
 
 constexpr float kLog2e = 1.4426950408889634f;
@@ -216,7 +236,8 @@ __device__ ProducerCount run_producer(const DecodeParams& P, const Smem& S, int 
     {  // pick the next item once the consumers released the last inputs, and
        // stage its small inputs (or, with no item left, tell them to stop)
       bool ok = mbar_wait(smem_u32(S.in_empty), (static_cast<uint32_t>(k) & 1u) ^ 1u, S.flags);
-      ok = __all_sync(0xffffffffu, ok);
+      // once the CTA aborted, nothing more is staged or loaded
+      ok = __all_sync(0xffffffffu, ok && !S.flags[0]);
       if (!ok) {
         if (lane == 0) abort_cta(P, S);
         return {seq, k};
@@ -252,7 +273,8 @@ __device__ ProducerCount run_producer(const DecodeParams& P, const Smem& S, int 
       if (paged && lane < n) {
         const int idx = (pb.tile_base + (t + lane) * tile_tok) / kBlock;
         if (FLINT_CHECK(P.dev_err, idx >= 0 && idx < pb.table_len, 3, idx, pb.table_len, it)) blk = __ldg(pb.table + idx);
-        // An out-of-range coordinate makes TMA fill zeros; flag it for the caller.
+        // A block id outside the pool: flag it for the caller; its tile's
+        // loads are skipped below.
         if (blk < 0 || blk >= pb.num_blocks) report_error(P.dev_err, FLINT_ERR_INVALID_ARG);
       }
       for (int j = 0; j < n; ++j, ++seq) {
@@ -260,7 +282,10 @@ __device__ ProducerCount run_producer(const DecodeParams& P, const Smem& S, int 
         const int stage = seq % kStages;
         const uint32_t phase = static_cast<uint32_t>(seq / kStages) & 1u;
         bool ok = mbar_wait(smem_u32(&S.empty[stage]), phase ^ 1u, S.flags);
-        ok = __all_sync(0xffffffffu, ok);
+        // After an abort a consumer warp may have skipped a phase of this
+        // stage, so the barrier's parity no longer says which tile it freed:
+        // arm nothing more (the drain below waits for what was issued).
+        ok = __all_sync(0xffffffffu, ok && !S.flags[0]);
         if (!ok) {
           if (lane == 0) abort_cta(P, S);
           return {seq, k + 1};
@@ -294,7 +319,16 @@ __device__ ProducerCount run_producer(const DecodeParams& P, const Smem& S, int 
         if (lane == 0) {
           fine = FLINT_CHECK(P.dev_err, (base & 1023u) == 0 && base + kStageBytes <= smem_u32(S.full), 6,
                              static_cast<int>(base), stage, seq);
-          fine = fine && FLINT_CHECK(P.dev_err, c2 >= 0 && c2 < pb.ext2 && c3 >= 0 && c3 < pb.ext3, 5, c2, c3, it);
+          // Every coordinate handed to TMA lies inside the tensor: a tile
+          // outside it (only a bad paged block id can make one; reported
+          // above) loads nothing.
+          const bool in_range = c2 >= 0 && c2 < pb.ext2 && c3 >= 0 && c3 < pb.ext3;
+          fine = fine && FLINT_CHECK(P.dev_err, in_range || paged, 5, c2, c3, it) && in_range;
+#ifdef FLINT_TEST_HOOKS
+          if (static_cast<int>(blockIdx.x) == g_stall_decode[0] && seq == g_stall_decode[1]) {
+            fine = false;  // leave the stage unarmed: its waiters run out of time
+          } else
+#endif
           if (fine)
             mbar_expect_tx(fb, kStageBytes);
           else
@@ -302,6 +336,9 @@ __device__ ProducerCount run_producer(const DecodeParams& P, const Smem& S, int 
         }
         fine = __shfl_sync(0xffffffffu, fine, 0);
         __syncwarp();
+#ifdef FLINT_TRACE
+        if (seq == 0 && lane == 0) FLINT_TRACE_MARK(2);
+#endif
         if (fine && lane < n_boxes) {
 #if FLINT_KV_EVICT_FIRST
           tma_load_4d_hint(base + b_off, map, fb, b_x, b_head, c2, c3, kv_policy);
@@ -622,6 +659,19 @@ __device__ __forceinline__ int partial_f4(int head, int c, int q) {
   return ((head >> 3) * 8 + q) * 32 + (head & 7) * 4 + c;
 }
 
+// The factor that turns an unnormalised O (with running max M and sum L, log2
+// units) into the output with the head's sink logit folded into the softmax:
+// 2^(M - Mf) / (L 2^(M - Mf) + 2^(s - Mf)), s = sink log2(e), Mf = max(M, s).
+// With no key (M = -inf) the output is 0, whatever the sink (also for a sink
+// of -inf, where the formula would read 0/0).
+__device__ __forceinline__ float sink_scale(float M, float L, float sink) {
+  if (M == -INFINITY) return 0.f;
+  const float s2 = sink * kLog2e;
+  const float Mf = fmaxf(M, s2);
+  const float a = exp2f(M - Mf);
+  return a / (L * a + exp2f(s2 - Mf));
+}
+
 // out[head][8n + 2c + e] = O * 2^(M - Mf) / (L 2^(M - Mf) + 2^(sink - Mf)), the
 // sink logit of this head folded into the softmax; thread (g, c) owns dims
 // 8n + 2c + {0,1} of head `head`.
@@ -642,10 +692,7 @@ __device__ __forceinline__ void finish_head(const Problem& pb, int head, int c, 
     }
     return;
   }
-  const float s2 = sink * kLog2e;
-  const float Mf = fmaxf(M, s2);
-  const float a = (M == -INFINITY) ? 0.f : exp2f(M - Mf);
-  const float scale = a / (L * a + exp2f(s2 - Mf));
+  const float scale = sink_scale(M, L, sink);
   float* dst = pb.out + head * kDim;
   const int d0 = dim_d0(c, pb.fp8 != 0), d2 = dim_d2(c, pb.fp8 != 0);
 #pragma unroll
@@ -744,6 +791,11 @@ __device__ void run_consumer(const DecodeParams& P, const Smem& S, int warp, int
 
     const int ntiles = item.t1 - item.t0;
     for (int k = 0; k < ntiles; ++k, ++seq) {
+      // Once the CTA aborted, a warp neither waits, reads nor releases a
+      // stage: a warp that gave up on a phase would otherwise pass the parity
+      // wait of the same stage's next tile on an older phase.  It keeps
+      // walking so that every warp meets the same barriers.
+      if (__any_sync(0xffffffffu, S.flags[0] != 0)) continue;
       const int stage = seq % kStages;
       const uint32_t phase = static_cast<uint32_t>(seq / kStages) & 1u;
       // every lane observes the phase completion (acquire) before reading the stage
@@ -751,8 +803,11 @@ __device__ void run_consumer(const DecodeParams& P, const Smem& S, int warp, int
       ok = __all_sync(0xffffffffu, ok);
       if (!ok) {
         if (lane == 0) abort_cta(P, S);
-        continue;  // keep walking so that every warp meets the same barriers
+        continue;
       }
+#ifdef FLINT_TRACE
+      if (seq == 0 && warp == 0 && lane == 0) FLINT_TRACE_MARK(3);
+#endif
       const uint32_t base = smem_u32(S.stages + stage * kStageBytes);
       if (!pb.fp8) {
         const int r0 = group * kSlice;
@@ -771,6 +826,7 @@ __device__ void run_consumer(const DecodeParams& P, const Smem& S, int warp, int
     }
 
     // ---- item end: this warp holds (m, l, O) of its 8 heads over the item
+    if (warp == 0 && lane == 0) FLINT_TRACE_MARK(4);
     l_run += __shfl_xor_sync(0xffffffffu, l_run, 1);
     l_run += __shfl_xor_sync(0xffffffffu, l_run, 2);
     float v[32];
@@ -830,6 +886,7 @@ __device__ void run_consumer(const DecodeParams& P, const Smem& S, int warp, int
     }
     __syncwarp();
     consumer_bar();
+    if (threadIdx.x == 0) FLINT_TRACE_MARK(5);
     // A deferred problem is merged after the grid barrier, whose fence
     // releases these partials.  Otherwise one thread releases them (the
     // barrier above orders every consumer's stores before its fence) and
@@ -870,6 +927,7 @@ __device__ void run_consumer(const DecodeParams& P, const Smem& S, int warp, int
         for (int e = 0; e < 32; ++e) v[e] = v[e] * sa + mine[e] * sb;
         finish_head(pb, head, c, M, ll * sa + lo_ * sb, v, sink);
         if (threadIdx.x == 0) P.counters[item.seg] = 0;  // ready for the next call
+        if (threadIdx.x == 0) FLINT_TRACE_MARK(12);
       }
     }
     __syncwarp();
@@ -966,10 +1024,7 @@ __device__ __forceinline__ void write_chunk(const Problem& pb, int head, int c, 
     }
     return;
   }
-  const float s2 = sink * kLog2e;
-  const float Mf = fmaxf(m, s2);
-  const float a = (m == -INFINITY) ? 0.f : exp2f(m - Mf);
-  const float scale = a / (l * a + exp2f(s2 - Mf));
+  const float scale = sink_scale(m, l, sink);
   float* o = pb.out + head * kDim + 16 * q;
   const int d0 = dim_d0(c, pb.fp8 != 0), d2 = dim_d2(c, pb.fp8 != 0);
   *reinterpret_cast<float2*>(o + d0) = make_float2(acc.x * scale, acc.y * scale);
@@ -1041,6 +1096,14 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const __grid_consta
   // dependence may be scheduled from now on (it waits for this grid's
   // completion before it touches global memory, see below).
   asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+#ifdef FLINT_TRACE
+  if (threadIdx.x == 0) {
+    unsigned int smid;
+    asm volatile("mov.u32 %0, %%smid;" : "=r"(smid));
+    FLINT_TRACE_MARK(0);
+    FLINT_TRACE_SET(10, smid);
+  }
+#endif
   extern __shared__ uint8_t smem_raw[];
   const Smem S = carve(smem_raw);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -1075,14 +1138,20 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const __grid_consta
   // kernel of the stream; wait for it to complete (and its memory to be
   // visible) before any access to the workspace, the caches or the inputs.
   if (P.pdl) asm volatile("griddepcontrol.wait;" ::: "memory");
+  if (threadIdx.x == 0) FLINT_TRACE_MARK(1);
 
   ProducerCount pc{0, 0};
   if (warp == kConsumerWarps) {
     pc = run_producer(P, S, c0, c1, claim, lane);
+    if (lane == 0) {
+      FLINT_TRACE_MARK(6);
+      FLINT_TRACE_SET(11, pc.staged);
+    }
   } else {
     run_consumer(P, S, warp, lane);
   }
   __syncthreads();
+  if (threadIdx.x == 0) FLINT_TRACE_MARK(7);
   // After an abort, let every issued copy land before the CTA's shared memory
   // goes away (bounded as well; a normal run returns at once).  Only the last
   // armed input phase can still have copies in flight: the producer arms the
@@ -1106,7 +1175,12 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const __grid_consta
     if (grid_barrier(reinterpret_cast<unsigned int*>(P.counters + kBarrierWord), S)) {
       // every CTA has made its last claim: ready the queue for the next call
       if (blockIdx.x == 0 && threadIdx.x == 0) P.counters[kQueueHead] = 0;
+      if (threadIdx.x == 0) FLINT_TRACE_MARK(8);
       grid_merge(P, S);
+#ifdef FLINT_TRACE
+      __syncthreads();
+      if (threadIdx.x == 0) FLINT_TRACE_MARK(9);
+#endif
     } else if (threadIdx.x == 0) {
       report_error(P.dev_err, FLINT_ERR_TIMEOUT);
     }
@@ -1121,17 +1195,30 @@ size_t decode_smem_bytes() {
          kInBytes;
 }
 
+#ifdef FLINT_TRACE
+// Copies the trace table (kMaxCtas x kTraceSlots uint64) to host memory.
+extern "C" int flint_trace_read(unsigned long long* host) {
+  return static_cast<int>(cudaMemcpyFromSymbol(host, g_trace, sizeof(g_trace)));
+}
+extern "C" int flint_trace_clear() {
+  static unsigned long long zero[kMaxCtas][kTraceSlots];
+  return static_cast<int>(cudaMemcpyToSymbol(g_trace, zero, sizeof(zero)));
+}
+#endif
+
+#ifdef FLINT_TEST_HOOKS
+// Test builds only: CTA `block` leaves the stage of its tile number `seq`
+// (counted over its whole run) unarmed; block = -1 turns the hook off.
+extern "C" int flint_test_stall_decode(int block, int seq) {
+  const int v[2] = {block, seq};
+  return static_cast<int>(cudaMemcpyToSymbol(g_stall_decode, v, sizeof v));
+}
+#endif
+
 cudaError_t launch_decode(const DecodeParams& p, int grid, cudaStream_t stream) {
-  static int configured_device = -1;
-  int dev = 0;
-  cudaError_t e = cudaGetDevice(&dev);
+  static ContextSet configured;
+  cudaError_t e = configure_once(configured, reinterpret_cast<const void*>(decode_kernel), static_cast<int>(decode_smem_bytes()));
   if (e != cudaSuccess) return e;
-  if (configured_device != dev) {
-    e = cudaFuncSetAttribute(decode_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             static_cast<int>(decode_smem_bytes()));
-    if (e != cudaSuccess) return e;
-    configured_device = dev;
-  }
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(grid);
   cfg.blockDim = dim3(kThreads);

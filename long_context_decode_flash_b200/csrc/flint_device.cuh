@@ -12,8 +12,19 @@
 namespace flint {
 
 // A pipeline wait gives up after this long (the whole decode step takes well
-// under a millisecond); the kernel then reports FLINT_ERR_TIMEOUT.
-constexpr unsigned long long kWaitLimitNs = 2000000000ull;
+// under a millisecond); the kernel then reports FLINT_ERR_TIMEOUT.  A build
+// for the time-out tests sets a short limit (FLINT_WAIT_LIMIT_NS).
+#ifndef FLINT_WAIT_LIMIT_NS
+#define FLINT_WAIT_LIMIT_NS 2000000000ull
+#endif
+constexpr unsigned long long kWaitLimitNs = FLINT_WAIT_LIMIT_NS;
+
+// Test hooks (FLINT_TEST_HOOKS, only together with FLINT_DEBUG_CHECKS): a
+// kernel can be told to leave one pipeline stage of one CTA unarmed, so that
+// the waits on it run out and the abort path runs without any fault.
+#if defined(FLINT_TEST_HOOKS) && !defined(FLINT_DEBUG_CHECKS)
+#error "FLINT_TEST_HOOKS needs FLINT_DEBUG_CHECKS"
+#endif
 
 __device__ __forceinline__ uint32_t smem_u32(const void* p) {
   return static_cast<uint32_t>(__cvta_generic_to_shared(p));

@@ -6,7 +6,26 @@
 #include <cuda_runtime.h>
 #include <stdint.h>
 
+#include <mutex>
+#include <vector>
+
 #include "flint.h"
+
+// NVTX ranges around every entry point, for timelines in Nsight Systems or
+// any NVTX consumer: compiled in with -DFLINT_NVTX (header-only NVTX 3, which
+// costs nothing unless a tool is attached); release builds carry none.
+#ifdef FLINT_NVTX
+#include <nvtx3/nvToolsExt.h>
+namespace flint {
+struct NvtxRange {
+  explicit NvtxRange(const char* name) { nvtxRangePushA(name); }
+  ~NvtxRange() { nvtxRangePop(); }
+};
+}  // namespace flint
+#define FLINT_NVTX_RANGE(name) ::flint::NvtxRange flint_nvtx_range_(name)
+#else
+#define FLINT_NVTX_RANGE(name) ((void)0)
+#endif
 
 namespace flint {
 
@@ -204,5 +223,21 @@ size_t workspace_min_bytes(int n_problems, int num_ctas);
 
 // Sets the message that flint_last_error() returns on this thread; returns s.
 flint_status record_error(flint_status s, const char* fmt, ...);
+
+// The CUDA context current on the calling thread (a driver handle), or
+// nullptr if there is none yet.  Per-context state (a kernel's shared-memory
+// attribute, the address of a module variable) is keyed on it: after a device
+// reset the runtime makes a new context, and state kept for the old one is void.
+void* current_context();
+
+// The contexts in which a kernel's launch attribute has been set.
+struct ContextSet {
+  std::mutex mu;
+  std::vector<void*> ctxs;
+};
+
+// Sets the dynamic shared-memory limit of `kernel` to `bytes` once per
+// context (thread-safe; `done` is the caller's record of configured contexts).
+cudaError_t configure_once(ContextSet& done, const void* kernel, int bytes);
 
 }  // namespace flint

@@ -19,6 +19,9 @@
 // Set-up: the first call on a device, made with that device current, looks up
 // the address of the device's copy of the scratch (cudaGetSymbolAddress) and
 // keeps it for later calls.  Make that first call before any stream capture.
+// The address belongs to the device's current CUDA context: after a device
+// reset the runtime makes a new context, the next call looks the address up
+// again, and that call too must come before any capture.
 #include <cuda_runtime.h>
 #include <stdio.h>
 
@@ -41,9 +44,12 @@ static __device__ __align__(256) unsigned char g_scratch[FLINT_NOALLOC_SCRATCH_B
 constexpr int kMaxDevices = 64;
 std::mutex g_mu;
 void* g_scratch_addr[kMaxDevices] = {};
+void* g_scratch_ctx[kMaxDevices] = {};  // the context each address was looked up in
 
 // Address of the current device's copy of g_scratch.  The first call on a
-// device looks it up (with that device current) and keeps it.
+// device looks it up (with that device current) and keeps it together with the
+// current context; a call in another context (after a device reset) looks it
+// up again.
 flint_status scratch_address(void** out, const char* who) {
   int dev = -1;
   cudaError_t e = cudaGetDevice(&dev);
@@ -51,13 +57,15 @@ flint_status scratch_address(void** out, const char* who) {
   if (dev < 0 || dev >= kMaxDevices)
     return record_error(FLINT_ERR_UNSUPPORTED, "%s: device %d outside the %d devices supported", who, dev, kMaxDevices);
   std::lock_guard<std::mutex> lock(g_mu);
-  if (!g_scratch_addr[dev]) {
+  void* ctx = current_context();
+  if (!g_scratch_addr[dev] || !ctx || ctx != g_scratch_ctx[dev]) {
     void* p = nullptr;
     e = cudaGetSymbolAddress(&p, g_scratch);
     if (e != cudaSuccess || !p)
       return record_error(FLINT_ERR_CUDA, "%s: cudaGetSymbolAddress of the scratch failed on device %d: %s",
                           who, dev, cudaGetErrorString(e));
     g_scratch_addr[dev] = p;
+    g_scratch_ctx[dev] = current_context();  // the lookup above made one if there was none
   }
   *out = g_scratch_addr[dev];
   return FLINT_OK;
@@ -69,6 +77,7 @@ extern "C" flint_status flint_attn_stack_noalloc(const flint_layer* layers, int3
                                                  int32_t pos, float eps, double theta, float* out,
                                                  int32_t num_ctas, int32_t* dev_err, void* stream) {
   const char* who = "flint_attn_stack_noalloc";
+  FLINT_NVTX_RANGE(who);
   // Size check first: the scratch cannot grow.  It must hold the static plan;
   // the run-time queue then gets the part of it that is left.
   const size_t need = workspace_min_bytes(n_layers, num_ctas);

@@ -93,11 +93,23 @@ extern "C" int32_t flint_plan_items(const int32_t* seg_tiles, int32_t n_segs, in
 
 namespace {
 
-constexpr int kDynMinTiles = 64;  // smaller segments stay wholly static
+#ifndef FLINT_DYN_MIN_TILES
+#define FLINT_DYN_MIN_TILES 64
+#endif
+#ifndef FLINT_DYN_MIN_SHARE
+#define FLINT_DYN_MIN_SHARE 64
+#endif
+#ifndef FLINT_DYN_SMALL_PERMILLE
+#define FLINT_DYN_SMALL_PERMILLE 200
+#endif
+#ifndef FLINT_DYN_SMALL_CHUNK
+#define FLINT_DYN_SMALL_CHUNK 8
+#endif
+constexpr int kDynMinTiles = FLINT_DYN_MIN_TILES;  // smaller segments stay wholly static
 // Below this many tiles per CTA the whole launch stays static: a CTA's share
 // is then short next to a chunk, and the few SMs that stream slower cost less
 // than the queue's extra items.
-constexpr int kDynMinShare = 64;
+constexpr int kDynMinShare = FLINT_DYN_MIN_SHARE;
 
 struct Variant {
   int permille;   // share of a large segment's tiles put in the queue
@@ -105,8 +117,14 @@ struct Variant {
 };
 // Tried in order until the plan fits max_items; the last one is static only.
 // A variant whose smallest chunk exceeds an eighth of a CTA's share is
-// skipped: a chunk that large taken late would itself be the tail.
-constexpr Variant kVariants[] = {{200, 8}, {200, 16}, {200, 32}, {100, 32}, {0, 0}};
+// skipped: a chunk that large taken late would itself be the tail.  The
+// variant before the static one serves short shares (few tiles per CTA).
+constexpr Variant kVariants[] = {{200, 8},
+                                 {200, 16},
+                                 {200, 32},
+                                 {100, 32},
+                                 {FLINT_DYN_SMALL_PERMILLE, FLINT_DYN_SMALL_CHUNK},
+                                 {0, 0}};
 
 }  // namespace
 

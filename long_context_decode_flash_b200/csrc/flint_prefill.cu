@@ -152,6 +152,20 @@ __device__ __forceinline__ void raise_abort(const PrefillParams& p, Bars* B) {
   B->abort = 1;
 }
 
+#ifdef FLINT_TEST_HOOKS
+// {block, K tile}: that CTA's producer leaves that K tile unarmed; {-1, -1} = off.
+__device__ int g_stall_prefill[2] = {-1, -1};
+#endif
+
+// K and V tiles whose loads the producer issued (the drain's bound).
+struct Issued {
+  int k, v;
+};
+
+__device__ __forceinline__ bool aborted(const Bars* B) {
+  return *reinterpret_cast<const volatile int*>(&B->abort) != 0;
+}
+
 struct Work {
   int t0, g, j_first, n;
   __device__ bool interior(int jj, int window) const {
@@ -173,8 +187,11 @@ __device__ __forceinline__ Work work_of(const PrefillParams& p) {
   return w;
 }
 
-__device__ void run_tma(const PrefillParams& p, const Work& w, uint8_t* smem, Bars* B) {
+// Returns the K and V tiles it issued.  Once the CTA aborted it issues
+// nothing more.
+__device__ Issued run_tma(const PrefillParams& p, const Work& w, uint8_t* smem, Bars* B) {
   const uint32_t base = smem_u32(smem);
+  Issued n{0, 0};
   mbar_expect_tx(smem_u32(&B->q_full), kQBytes);
   tma_load_4d(base, &p.q_map, smem_u32(&B->q_full), 0, w.g * kGroup, w.t0, 0);
   tma_load_4d(base + kRows * 128, &p.q_map, smem_u32(&B->q_full), 64, w.g * kGroup, w.t0, 0);
@@ -183,36 +200,49 @@ __device__ void run_tma(const PrefillParams& p, const Work& w, uint8_t* smem, Ba
     const int sk = jj % kKs, sv = jj % kVs;
     if (jj >= kKs && !mbar_wait(smem_u32(&B->k_empty[sk]), static_cast<uint32_t>(jj / kKs - 1) & 1u, &B->abort)) {
       raise_abort(p, B);
-      return;
+      return n;
     }
+    if (aborted(B)) return n;
     const uint32_t dk = base + kOffK + sk * kTileBytes;
-    mbar_expect_tx(smem_u32(&B->k_full[sk]), kTileBytes);
-    tma_load_4d(dk, &p.k_map, smem_u32(&B->k_full[sk]), 0, w.g, k0, 0);
-    tma_load_4d(dk + kHalfBytes, &p.k_map, smem_u32(&B->k_full[sk]), 64, w.g, k0, 0);
+#ifdef FLINT_TEST_HOOKS
+    if (!(static_cast<int>(blockIdx.x) == g_stall_prefill[0] && jj == g_stall_prefill[1]))
+#endif
+    {
+      mbar_expect_tx(smem_u32(&B->k_full[sk]), kTileBytes);
+      tma_load_4d(dk, &p.k_map, smem_u32(&B->k_full[sk]), 0, w.g, k0, 0);
+      tma_load_4d(dk + kHalfBytes, &p.k_map, smem_u32(&B->k_full[sk]), 64, w.g, k0, 0);
+    }
+    n.k = jj + 1;
     if (jj >= kVs && !mbar_wait(smem_u32(&B->v_empty[sv]), static_cast<uint32_t>(jj / kVs - 1) & 1u, &B->abort)) {
       raise_abort(p, B);
-      return;
+      return n;
     }
+    if (aborted(B)) return n;
     const uint32_t dv = base + kOffV + sv * kTileBytes;
     mbar_expect_tx(smem_u32(&B->v_full[sv]), kTileBytes);
     tma_load_4d(dv, &p.v_map, smem_u32(&B->v_full[sv]), 0, w.g, k0, 0);
     tma_load_4d(dv + kHalfBytes, &p.v_map, smem_u32(&B->v_full[sv]), 64, w.g, k0, 0);
+    n.v = jj + 1;
   }
+  return n;
 }
 
 // After an abort: let the copies still in flight land before the CTA's shared
-// memory goes away (bounded; the last kKs K and kVs V phases are the only ones
-// that can be pending).  A normal run returns at once.
-__device__ void drain_tma(const Work& w, Bars* B) {
+// memory goes away (bounded).  Only the last kKs K and kVs V tiles the
+// producer issued can be pending: it issues tile j into a stage only after the
+// stage's tile j - kKs (or j - kVs) was consumed, which needed it landed.  The
+// waits must be on those issued phases: a parity wait on a later, never armed
+// phase of the same stage would pass on an older one while a copy still lands.
+__device__ void drain_tma(Issued n, Bars* B) {
   const unsigned long long t0 = globaltimer_ns();
   auto wait = [&](uint32_t bar, uint32_t parity) {
     while (!mbar_try_wait(bar, parity))
       if (globaltimer_ns() - t0 > kWaitLimitNs) return;
   };
   wait(smem_u32(&B->q_full), 0);
-  for (int jj = max(0, w.n - kKs); jj < w.n; ++jj)
+  for (int jj = max(0, n.k - kKs); jj < n.k; ++jj)
     wait(smem_u32(&B->k_full[jj % kKs]), static_cast<uint32_t>(jj / kKs) & 1u);
-  for (int jj = max(0, w.n - kVs); jj < w.n; ++jj)
+  for (int jj = max(0, n.v - kVs); jj < n.v; ++jj)
     wait(smem_u32(&B->v_full[jj % kVs]), static_cast<uint32_t>(jj / kVs) & 1u);
 }
 
@@ -435,16 +465,17 @@ __global__ void __launch_bounds__(kPfThreads, 1) prefill_kernel(const __grid_con
   tc_fence_after();
   const uint32_t tmem = B->tmem_base;
 
+  Issued issued{0, 0};
   if (warp < kSoftWarps) {
     run_softmax(p, w, tmem, smem, B, warp, lane);
   } else if (warp == kTmaWarp) {
-    if (lane == 0) run_tma(p, w, smem, B);
+    if (lane == 0) issued = run_tma(p, w, smem, B);
   } else if (lane == 0) {
     run_mma(p, w, smem_u32(smem), tmem, B);
   }
   tc_fence_before();
   __syncthreads();
-  if (warp == kTmaWarp && lane == 0 && B->abort) drain_tma(w, B);
+  if (warp == kTmaWarp && lane == 0 && aborted(B)) drain_tma(issued, B);
   if (warp == kMmaWarp) {
     __syncwarp();
     tc_fence_after();
@@ -454,17 +485,19 @@ __global__ void __launch_bounds__(kPfThreads, 1) prefill_kernel(const __grid_con
 
 }  // namespace
 
+#ifdef FLINT_TEST_HOOKS
+// Test builds only: CTA `block` leaves its K tile `tile` unarmed; block = -1
+// turns the hook off.
+extern "C" int flint_test_stall_prefill(int block, int tile) {
+  const int v[2] = {block, tile};
+  return static_cast<int>(cudaMemcpyToSymbol(g_stall_prefill, v, sizeof v));
+}
+#endif
+
 cudaError_t launch_prefill(const PrefillParams& p, cudaStream_t stream) {
-  static int configured_device = -1;
-  int dev = 0;
-  cudaError_t e = cudaGetDevice(&dev);
+  static ContextSet configured;
+  cudaError_t e = configure_once(configured, reinterpret_cast<const void*>(prefill_kernel), static_cast<int>(kPfSmem));
   if (e != cudaSuccess) return e;
-  if (configured_device != dev) {
-    e = cudaFuncSetAttribute(prefill_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             static_cast<int>(kPfSmem));
-    if (e != cudaSuccess) return e;
-    configured_device = dev;
-  }
   const int grid = (p.T + kPq - 1) / kPq * kKvHeads;
   prefill_kernel<<<grid, kPfThreads, kPfSmem, stream>>>(p);
   return cudaGetLastError();

@@ -66,48 +66,60 @@ _lock = threading.Lock()
 _lib = None
 
 
+def open_library(path: str) -> ctypes.CDLL:
+    """Load a build of the library from `path` with its signatures declared
+    (load_library() does this for the package's libflint.so; tests use it for
+    the test builds)."""
+    if not os.path.exists(path):
+        raise FlintError(FLINT_ERR_CUDA, f"{path} is not built "
+                         "(python -m long_context_decode_flash_b200.build)")
+    lib = ctypes.CDLL(path)
+    P, I32, I64 = ctypes.c_void_p, ctypes.c_int32, ctypes.c_int64
+    lib.flint_status_string.argtypes = [ctypes.c_int]
+    lib.flint_status_string.restype = ctypes.c_char_p
+    lib.flint_last_error.restype = ctypes.c_char_p
+    lib.flint_kv_bytes.argtypes = [I64, I32, I32, I32, I32]
+    lib.flint_kv_bytes.restype = ctypes.c_uint64
+    lib.flint_qk_norm_rope.argtypes = [P, P, P, P, P, P, I32, ctypes.c_float, ctypes.c_double,
+                                       I32, P, P, P, P, P]
+    lib.flint_kv_append.argtypes = [P, P, P, I32, P, P, P]
+    lib.flint_attn_workspace_bytes.argtypes = [I32, I32]
+    lib.flint_attn_workspace_bytes.restype = ctypes.c_size_t
+    lib.flint_attn_decode.argtypes = [P, I32, P, P, I32, P, I32, P, P, ctypes.c_size_t,
+                                      I32, P, P]
+    lib.flint_attn_stack.argtypes = [P, I32, I32, ctypes.c_float, ctypes.c_double, P, P,
+                                     ctypes.c_size_t, I32, P, P]
+    lib.flint_attn_layers_serial.argtypes = [P, I32, I32, ctypes.c_float, ctypes.c_double, P, P,
+                                             ctypes.c_size_t, I32, P, P]
+    lib.flint_attn_stack_noalloc.argtypes = [P, I32, I32, ctypes.c_float, ctypes.c_double,
+                                             P, I32, P, P]
+    lib.flint_prefill_qk_norm_rope.argtypes = [P, P, P, P, P, I32, ctypes.c_float,
+                                               ctypes.c_double, I32, P, P, P, P, P, P]
+    lib.flint_prefill_attn.argtypes = [P, P, P, I32, P, I32, P, P, P]
+    lib.flint_attn_decode_partial.argtypes = [P, I32, P, P, I32, P, P, ctypes.c_size_t, I32, P, P]
+    lib.flint_merge_partials.argtypes = [P, I32, I32, P, P, P]
+    lib.flint_plan_items.argtypes = [P, I32, I32, I32, P, P, P, P, I32]
+    lib.flint_plan_items.restype = I32
+    lib.flint_plan_split.argtypes = [P, I32, I32, I32, I32, P, P, P, P, P]
+    lib.flint_plan_split.restype = I32
+    for name in ("flint_qk_norm_rope", "flint_kv_append", "flint_attn_decode",
+                 "flint_attn_stack", "flint_attn_stack_noalloc", "flint_attn_layers_serial",
+                 "flint_prefill_qk_norm_rope", "flint_prefill_attn", "flint_attn_decode_partial",
+                 "flint_merge_partials"):
+        getattr(lib, name).restype = ctypes.c_int
+    # test builds only (libflint_hooks.so): leave one pipeline stage unarmed
+    for name in ("flint_test_stall_decode", "flint_test_stall_prefill"):
+        if hasattr(lib, name):
+            getattr(lib, name).argtypes = [ctypes.c_int, ctypes.c_int]
+            getattr(lib, name).restype = ctypes.c_int
+    return lib
+
+
 def load_library() -> ctypes.CDLL:
     global _lib
     with _lock:
         if _lib is None:
-            if not os.path.exists(LIB_PATH):
-                raise FlintError(FLINT_ERR_CUDA, f"{LIB_PATH} is not built "
-                                 "(python -m long_context_decode_flash_b200.build)")
-            lib = ctypes.CDLL(LIB_PATH)
-            P, I32, I64 = ctypes.c_void_p, ctypes.c_int32, ctypes.c_int64
-            lib.flint_status_string.argtypes = [ctypes.c_int]
-            lib.flint_status_string.restype = ctypes.c_char_p
-            lib.flint_last_error.restype = ctypes.c_char_p
-            lib.flint_kv_bytes.argtypes = [I64, I32, I32, I32, I32]
-            lib.flint_kv_bytes.restype = ctypes.c_uint64
-            lib.flint_qk_norm_rope.argtypes = [P, P, P, P, P, P, I32, ctypes.c_float, ctypes.c_double,
-                                               I32, P, P, P, P, P]
-            lib.flint_kv_append.argtypes = [P, P, P, I32, P, P, P]
-            lib.flint_attn_workspace_bytes.argtypes = [I32, I32]
-            lib.flint_attn_workspace_bytes.restype = ctypes.c_size_t
-            lib.flint_attn_decode.argtypes = [P, I32, P, P, I32, P, I32, P, P, ctypes.c_size_t,
-                                              I32, P, P]
-            lib.flint_attn_stack.argtypes = [P, I32, I32, ctypes.c_float, ctypes.c_double, P, P,
-                                             ctypes.c_size_t, I32, P, P]
-            lib.flint_attn_layers_serial.argtypes = [P, I32, I32, ctypes.c_float, ctypes.c_double, P, P,
-                                                     ctypes.c_size_t, I32, P, P]
-            lib.flint_attn_stack_noalloc.argtypes = [P, I32, I32, ctypes.c_float, ctypes.c_double,
-                                                     P, I32, P, P]
-            lib.flint_prefill_qk_norm_rope.argtypes = [P, P, P, P, P, I32, ctypes.c_float,
-                                                       ctypes.c_double, I32, P, P, P, P, P, P]
-            lib.flint_prefill_attn.argtypes = [P, P, P, I32, P, I32, P, P, P]
-            lib.flint_attn_decode_partial.argtypes = [P, I32, P, P, I32, P, P, ctypes.c_size_t, I32, P, P]
-            lib.flint_merge_partials.argtypes = [P, I32, I32, P, P, P]
-            lib.flint_plan_items.argtypes = [P, I32, I32, I32, P, P, P, P, I32]
-            lib.flint_plan_items.restype = I32
-            lib.flint_plan_split.argtypes = [P, I32, I32, I32, I32, P, P, P, P, P]
-            lib.flint_plan_split.restype = I32
-            for name in ("flint_qk_norm_rope", "flint_kv_append", "flint_attn_decode",
-                         "flint_attn_stack", "flint_attn_stack_noalloc", "flint_attn_layers_serial",
-                         "flint_prefill_qk_norm_rope", "flint_prefill_attn", "flint_attn_decode_partial",
-                         "flint_merge_partials"):
-                getattr(lib, name).restype = ctypes.c_int
-            _lib = lib
+            _lib = open_library(LIB_PATH)
     return _lib
 
 

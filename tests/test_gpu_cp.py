@@ -127,3 +127,19 @@ def test_cp_decode_single_process_group_of_one():
         parity(out.cpu().numpy()[0], oracle_full(d, 0, L), "cp_decode")
     finally:
         dist.destroy_process_group()
+
+
+def test_merge_of_only_empty_partials_is_zero_not_nan():
+    """Partials with no key at all (m = -inf, l = 0, O = 0), some heads with a
+    sink of -inf: the merge has no softmax mass for those heads and gives 0,
+    as the oracle's merge does; finite sinks give 0 as well."""
+    B = 2
+    parts = torch.zeros((3, B, flint.CP_PARTIAL_FLOATS), dtype=torch.float32)
+    parts[:, :, 32 * 128:32 * 128 + 32] = float("-inf")
+    sinks = torch.randn(32, dtype=torch.float32)
+    sinks[::2] = float("-inf")
+    got = merge(dev(parts), dev(sinks))
+    empty = (np.zeros((32, 128)), np.full(32, -np.inf), np.zeros(32))
+    want = oracle.merge_partials([empty] * 3, sinks.numpy().astype(np.float64))
+    assert np.isfinite(got).all()
+    assert np.array_equal(got[0], want) and np.array_equal(got[1], want)

@@ -193,7 +193,10 @@ def test_paged_equals_contiguous_bitwise_shape():
 def test_paged_block_id_out_of_range_sets_device_error():
     pb = I.make_paged_batch(seq_lens=[300], workload=I.W_PAGED_BATCH)
     table = pb.block_table.clone()
-    table[0, 2] = pb.k_pool.shape[0] + 5          # beyond the pool: TMA reads zeros
+    # a block id beyond the pool: the tiles of that block are never loaded (no
+    # coordinate outside the tensor reaches TMA), the error is flagged, and the
+    # output is meaningless
+    table[0, 2] = pb.k_pool.shape[0] + 5
     cache = flint.kv_cache(dev(pb.k_pool), dev(pb.v_pool), flint.PAGED, block_table=dev(table),
                            num_blocks=pb.k_pool.shape[0])
     out = torch.empty((1, 32, 128), dtype=torch.float32, device="cuda")
@@ -202,7 +205,6 @@ def test_paged_block_id_out_of_range_sets_device_error():
     flint.flint_attn_decode(dev(pb.q), cache, [300], dev(pb.sinks), 0, out, ws, dev_err=err)
     torch.cuda.synchronize()
     assert int(err.item()) == flint.FLINT_ERR_INVALID_ARG
-    assert torch.isfinite(out).all()
 
 
 def test_workspace_too_small_is_rejected():

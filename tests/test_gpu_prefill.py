@@ -93,6 +93,32 @@ def test_prefill_q_and_k_match_the_oracle(window):
     np.testing.assert_array_equal(v.cpu().view(torch.int16).numpy(), p.v_raw.to(torch.float16).view(torch.int16).numpy())
 
 
+def test_prefill_v_fp16_at_the_edges_of_the_format():
+    """v_out is v_raw converted to fp16 to nearest even, saturating at
+    +-65,504 (as documented for flint_prefill_qk_norm_rope): bf16 values
+    beyond the fp16 range clamp to the largest finite fp16, values below the
+    smallest normal fp16 (6.1e-5) become subnormals or round to zero, signed
+    zeros keep their sign; bit for bit a host conversion with the same rule."""
+    T = 64
+    p = I.make_prefill(T, 0, workload=W_PF + 9)
+    edges = torch.tensor([65504.0, 65536.0, -65536.0, 1.0e5, -3.0e38, 3.0e38, 2.0 ** -14, -(2.0 ** -14),
+                          2.0 ** -15, 1.5 * 2.0 ** -20, 2.0 ** -24, 2.0 ** -25, 3.0 * 2.0 ** -25,
+                          2.0 ** -26, 1e-30, -1e-30, 0.0, -0.0, 6.0e-5, -5.9e-5], dtype=torch.float32)
+    v = p.v_raw.clone().reshape(-1)
+    idx = torch.arange(edges.numel()) * 97 % v.numel()
+    v[idx] = edges.to(torch.bfloat16)
+    p.v_raw = v.reshape(T, 4, 128)
+    d = Dev(p)
+    _, _, v16 = prep_gpu(d, with_v=True)
+    want = p.v_raw.float().clamp(-65504.0, 65504.0).to(torch.float16)
+    got_bits = v16.cpu().view(torch.int16).numpy()
+    want_bits = want.view(torch.int16).numpy()
+    np.testing.assert_array_equal(got_bits, want_bits)
+    flat = want.reshape(-1)[idx]
+    assert (flat[:6].abs() == 65504).all()           # saturated
+    assert flat[13].item() == 0.0 and flat[14].item() == 0.0  # below half the smallest subnormal
+
+
 @pytest.mark.parametrize("T", [1, 2, 15, 16, 17, 64, 65, 200, 700])
 @pytest.mark.parametrize("window", [flint.WINDOW, 0])
 def test_prefill_attention_every_row(T, window):

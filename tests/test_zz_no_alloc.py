@@ -14,7 +14,7 @@ import torch
 from long_context_decode_flash_b200 import flint
 from long_context_decode_flash_b200 import inputs as I
 
-from helpers import MAX_ABS, REL_L2, DeviceLayer
+from helpers import MAX_ABS, REL_L2, DeviceLayer, oracle_layer
 
 WORKLOAD = I.W_STACK_100K + 30
 
@@ -51,9 +51,16 @@ def test_noalloc_stack_matches_stack_twice():
     # 49 layers at context 20,000: full layers are split over a few CTAs each
     # and merged by their last-arriving CTA through the scratch counters
     L = 20_000
-    ref, outs = run_both(I.make_stack(L, workload=WORKLOAD), L - 1)
+    layers = I.make_stack(L, workload=WORKLOAD)
+    ref, outs = run_both(layers, L - 1)
     for k, o in enumerate(outs):
         close(o, ref, f"call {k + 1}")
+    # and against the float64 oracle directly: one full and two window layers
+    kinds = I.layer_kinds()
+    for i in (kinds.index(True), 0, 48):
+        want, _, _ = oracle_layer(layers[i])
+        for k, o in enumerate(outs):
+            close(o[i], want, f"call {k + 1}, layer {i} against the oracle")
 
 
 @pytest.mark.gpu
@@ -73,17 +80,24 @@ def min_workspace(n_layers, ctas):
     return 4096 + (ctas + n_layers) * 16640
 
 
-def test_noalloc_refuses_more_than_its_scratch():
-    # 49 layers on 296 CTAs need more than the fixed scratch: refused on the
-    # host before any device work, with the sizes in the message
-    need = min_workspace(49, 296)
-    assert need > 4 << 20
+def test_noalloc_size_check_counts_the_ctas_launched():
+    """The size check counts the CTAs a launch would use: num_ctas, but never
+    more than the device has SMs (296, the launch limit, when the count cannot
+    be read, as on a machine without a GPU).  Too large a request is refused on
+    the host before any device work, with the sizes in the message; one that
+    fits goes on to the argument checks (here it is refused for its NULL layer
+    pointers)."""
+    sms = torch.cuda.get_device_properties(0).multi_processor_count if torch.cuda.is_available() else 296
+    need = min_workspace(49, min(296, sms))
     arr = (flint.StackLayer * 49)()
     out = ctypes.c_void_p(16)
     lib = flint.load_library()
     st = lib.flint_attn_stack_noalloc(arr, 49, 0, 1e-6, 1e4, out, 296, None, None)
-    assert st == flint.FLINT_ERR_WORKSPACE
     msg = lib.flint_last_error().decode()
-    assert str(need) in msg and str(4 << 20) in msg, msg
-    # and 49 layers on 202 CTAs, the most that fit, pass the size check
+    if need > 4 << 20:
+        assert st == flint.FLINT_ERR_WORKSPACE, msg
+        assert str(need) in msg and str(4 << 20) in msg, msg
+    else:
+        assert st == flint.FLINT_ERR_INVALID_ARG and "NULL" in msg, msg
+    # 49 layers on 202 CTAs, the most that fit, pass the size check
     assert min_workspace(49, 202) <= 4 << 20 < min_workspace(49, 203)
