@@ -44,6 +44,10 @@
 
 #include "flint_device.cuh"
 
+#ifndef FLINT_PREFETCH_MAPS
+#define FLINT_PREFETCH_MAPS 0
+#endif
+
 namespace flint {
 
 // Device-side timeline tracing, compiled in only with -DFLINT_TRACE: thread
@@ -541,13 +545,16 @@ __device__ __forceinline__ void consume_slice(uint32_t sK, uint32_t sV, int tok0
 //     into the B fragments of the chunk's even-dim and odd-dim n-tiles.  O
 //     n-tile 2u holds dims 16u + 4c + {0, 2} and n-tile 2u + 1 dims
 //     16u + 4c + {1, 3} of thread (g, c) (see fp8_o_to_values).
-// The caller multiplies O by the head's v scale at the item's end.
+// The caller multiplies O by the head's v scale at the item's end.  kWhole:
+// every token of the block lies in [lo, hi), so no row needs a mask (the
+// caller picks the instance; the masks are ALU work on every value).
+template <bool kWhole>
 __device__ __forceinline__ void consume_block32_fp8(uint32_t sK, uint32_t sV, int tok0, int lo, int hi,
                                                     int lane, const uint32_t (&qa)[8][4], float k_scale,
                                                     float& m_run, float& l_run, float (&o)[16][4]) {
   const int c = lane & 3;
   const int l7 = lane & 7;
-  const bool whole = (tok0 >= lo) && (tok0 + 32 <= hi);
+  constexpr bool whole = kWhole;
 
   float sc[8];
 #pragma unroll
@@ -561,7 +568,8 @@ __device__ __forceinline__ void consume_block32_fp8(uint32_t sK, uint32_t sV, in
       ldsm_x4(row + ((u ^ l7) << 4), r[0], r[1], r[2], r[3]);
 #pragma unroll
       for (int i = 0; i < 4; ++i) {
-        const uint32_t b0 = e4m3x2_to_f16x2(r[i]), b1 = e4m3x2_to_f16x2(r[i] >> 16);
+        uint32_t b0, b1;
+        e4m3x4_to_f16x2x2(r[i], b0, b1);
         if (i & 1)
           mma_f16_16816(a1, qa[kk + i], b0, b1);
         else
@@ -627,8 +635,11 @@ __device__ __forceinline__ void consume_block32_fp8(uint32_t sK, uint32_t sV, in
     for (int i = 0; i < 4; ++i) {
       // x[i]: bytes (t 2c: d 2g, d 2g+1), (t 2c+1: d 2g, d 2g+1) of token group i
       const uint32_t y = __byte_perm(x[i], 0u, 0x3120);  // (t2c d2g, t2c+1 d2g, t2c d2g+1, t2c+1 d2g+1)
-      ev[i] = e4m3x2_to_f16x2(y) & msk[i];              // dim 2g of tokens 2c, 2c+1
-      od[i] = e4m3x2_to_f16x2(y >> 16) & msk[i];        // dim 2g+1
+      e4m3x4_to_f16x2x2(y, ev[i], od[i]);               // dims 2g, 2g+1 of tokens 2c, 2c+1
+      if (!whole) {
+        ev[i] &= msk[i];
+        od[i] &= msk[i];
+      }
     }
 #pragma unroll
     for (int s2 = 0; s2 < 2; ++s2) {
@@ -818,8 +829,14 @@ __device__ void run_consumer(const DecodeParams& P, const Smem& S, int warp, int
         // 64-token E4M3 tile: group q takes tokens 32q .. 32q + 31 as one block
         const int r0 = group * (kTileFp8 / kConsumerGroups);
         const int tok0 = pb.tile_base + (item.t0 + k) * kTileFp8 + r0;
-        consume_block32_fp8(base + box_offset_fp8(0, kvh) + r0 * 128, base + box_offset_fp8(1, kvh) + r0 * 128,
-                            tok0, pb.lo, pb.hi, lane, qa, k_scale, m_run, l_run, o);
+        if (tok0 >= pb.lo && tok0 + 32 <= pb.hi)
+          consume_block32_fp8<true>(base + box_offset_fp8(0, kvh) + r0 * 128,
+                                    base + box_offset_fp8(1, kvh) + r0 * 128, tok0, pb.lo, pb.hi, lane, qa,
+                                    k_scale, m_run, l_run, o);
+        else
+          consume_block32_fp8<false>(base + box_offset_fp8(0, kvh) + r0 * 128,
+                                     base + box_offset_fp8(1, kvh) + r0 * 128, tok0, pb.lo, pb.hi, lane, qa,
+                                     k_scale, m_run, l_run, o);
       }
       __syncwarp();
       if (lane == 0) mbar_arrive(smem_u32(&S.empty[stage]));
@@ -939,25 +956,39 @@ __device__ void run_consumer(const DecodeParams& P, const Smem& S, int warp, int
 // the others add 1, so bit 31 of the word flips once all G blocks arrived and
 // its low bits return to their start value (zero in a fresh workspace).
 // Bounded: returns false after the time limit.
+#ifndef FLINT_BARRIER_RELEASE
+#define FLINT_BARRIER_RELEASE 0
+#endif
 __device__ bool grid_barrier(unsigned int* bar, const Smem& S) {
   __syncthreads();
   if (threadIdx.x == 0) {
-    __threadfence();
     const unsigned int add = blockIdx.x == 0 ? 0x80000000u - (gridDim.x - 1) : 1u;
+#if FLINT_BARRIER_RELEASE
+    // the arrival publishes this CTA's writes (release); the CTA's other
+    // threads' writes are ordered before it by the __syncthreads above
+    unsigned int old;
+    asm volatile("atom.add.release.gpu.global.u32 %0, [%1], %2;" : "=r"(old) : "l"(bar), "r"(add) : "memory");
+#else
+    __threadfence();
     const unsigned int old = atomicAdd(bar, add);
+#endif
     const unsigned long long t0 = globaltimer_ns();
     int ok = 1;
-    for (;;) {
+    for (int spin = 0;; ++spin) {
       unsigned int cur;
       asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(cur) : "l"(bar) : "memory");
       if ((cur ^ old) & 0x80000000u) break;
-      if (globaltimer_ns() - t0 > kWaitLimitNs) {
+      if ((spin & 15) == 15 && globaltimer_ns() - t0 > kWaitLimitNs) {
         ok = 0;
         break;
       }
+#if !FLINT_BARRIER_RELEASE
       __nanosleep(20);
+#endif
     }
+#if !FLINT_BARRIER_RELEASE
     __threadfence();
+#endif
     S.flags[2] = ok;
   }
   __syncthreads();
@@ -974,7 +1005,10 @@ __device__ bool grid_barrier(unsigned int* bar, const Smem& S) {
 //   * A problem with many partials (a lone long problem split over every CTA)
 //     takes a whole CTA per unit: warp w folds partials w, w + 9, ..., then
 //     the warps' states are combined through shared memory in warp order.
-constexpr int kMergeBatch = 24;
+#ifndef FLINT_MERGE_BATCH
+#define FLINT_MERGE_BATCH 24
+#endif
+constexpr int kMergeBatch = FLINT_MERGE_BATCH;
 
 // Folds partials s0 + first, s0 + first + stride, ... (< s1) into (m, l, acc).
 __device__ __forceinline__ void fold_chunk(const DecodeParams& P, int s0, int s1, int first, int stride,
@@ -1133,6 +1167,14 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const __grid_consta
     asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
   }
   if (P.prep && threadIdx.x < kDim / 2) S.cs[threadIdx.x] = P.rope_cs[threadIdx.x];
+#if FLINT_PREFETCH_MAPS
+  if (warp == kConsumerWarps) {
+    // the tensor maps are read by TMA from parameter memory: fetch their lines
+    // now, while the plan is still being read, not at the first load
+    const int n_maps = P.prep ? 2 * P.n_problems : 2;
+    for (int i = lane; i < n_maps; i += 32) prefetch_tensormap(&P.maps[i]);
+  }
+#endif
   __syncthreads();
   // Programmatic dependent launch: everything above overlapped the previous
   // kernel of the stream; wait for it to complete (and its memory to be

@@ -194,12 +194,14 @@ __device__ __forceinline__ uint32_t movmatrix_trans(uint32_t x) {
 
 // ---- E4M3 helpers -----------------------------------------------------------
 
-// Two E4M3 codes (first in the low byte) -> packed f16x2 (first in the low
-// half); every E4M3 value is exact in f16.
-__device__ __forceinline__ uint32_t e4m3x2_to_f16x2(uint32_t two_codes) {
-  const __half2_raw h = __nv_cvt_fp8x2_to_halfraw2(static_cast<__nv_fp8x2_storage_t>(two_codes & 0xffffu),
-                                                   __NV_E4M3);
-  return static_cast<uint32_t>(h.x) | (static_cast<uint32_t>(h.y) << 16);
+// Four E4M3 codes (byte i = code i) -> two packed f16x2: codes 0, 1 in `lo`,
+// codes 2, 3 in `hi` (first of each pair in the low half); the two 16-bit
+// halves of the word feed the conversions directly.
+__device__ __forceinline__ void e4m3x4_to_f16x2x2(uint32_t four, uint32_t& lo, uint32_t& hi) {
+  asm("{\n\t.reg .b16 a, b;\n\tmov.b32 {a, b}, %2;\n\t"
+      "cvt.rn.f16x2.e4m3x2 %0, a;\n\tcvt.rn.f16x2.e4m3x2 %1, b;\n\t}"
+      : "=r"(lo), "=r"(hi)
+      : "r"(four));
 }
 
 // Two floats -> two E4M3 codes (first in the low byte), nearest even,
