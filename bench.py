@@ -38,8 +38,13 @@ NOMINAL_HBM_GBS = 8000.0
 # launch duration, --clock-control none, one launch after the warm-up) of each
 # workload, per KV dtype, with the hash of the CUDA sources it was taken on;
 # reported only while the sources still hash the same.
-TRAFFIC = {("stack", 100_000, "bf16"): (2_906_088_192 + 6_870_528, "38ee5c4a48fcdd23"),
-           ("stack", 100_000, "fp8"): (1_453_981_440 + 6_602_496, "cde382082669d367")}
+TRAFFIC = {("stack", 100_000, "bf16"): (2_905_866_240 + 7_171_584, "f0faa7f388d2e1d4"),
+           ("stack", 100_000, "fp8"): (1_453_846_016 + 6_466_560, "f0faa7f388d2e1d4"),
+           ("full100k", 100_000, "bf16"): (204_910_592 + 3_482_368, "f0faa7f388d2e1d4"),
+           ("full2k", 2048, "bf16"): (4_285_696 + 0, "f0faa7f388d2e1d4"),
+           ("swa100k", 100_000, "bf16"): (1_143_552 + 0, "f0faa7f388d2e1d4"),
+           ("paged32", 100_000, "bf16"): (2_271_119_872 + 6_297_600, "f0faa7f388d2e1d4"),
+           ("paged32swa", 100_000, "bf16"): (36_023_296 + 46_336, "f0faa7f388d2e1d4")}
 # The same for one prefill_kernel launch of a full (NoPE) layer on the
 # 8,192-token prompt (a --set full capture of that one launch).
 PREFILL_TRAFFIC = {8192: (83_963_648 + 80_508_928, "38ee5c4a48fcdd23")}
