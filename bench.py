@@ -36,15 +36,16 @@ NOMINAL_HBM_GBS = 8000.0
 # DRAM traffic (dram__bytes_read.sum + dram__bytes_write.sum) of one decode_kernel
 # launch from a full-size, one-pass ncu capture (those two metrics and the
 # launch duration, --clock-control none, one launch after the warm-up) of each
-# workload, per KV dtype, with the hash of the CUDA sources it was taken on;
-# reported only while the sources still hash the same.
-TRAFFIC = {("stack", 100_000, "bf16"): (2_905_866_240 + 7_171_584, "f0faa7f388d2e1d4"),
-           ("stack", 100_000, "fp8"): (1_453_846_016 + 6_466_560, "f0faa7f388d2e1d4"),
-           ("full100k", 100_000, "bf16"): (204_910_592 + 3_482_368, "f0faa7f388d2e1d4"),
-           ("full2k", 2048, "bf16"): (4_285_696 + 0, "f0faa7f388d2e1d4"),
-           ("swa100k", 100_000, "bf16"): (1_143_552 + 0, "f0faa7f388d2e1d4"),
-           ("paged32", 100_000, "bf16"): (2_271_119_872 + 6_297_600, "f0faa7f388d2e1d4"),
-           ("paged32swa", 100_000, "bf16"): (36_023_296 + 46_336, "f0faa7f388d2e1d4")}
+# workload, per KV dtype, with the hash of the decode kernel's sources
+# (DECODE_SOURCES below) it was taken on; reported only while they still hash
+# the same.  The captures were taken on the whole-source hash f0faa7f388d2e1d4.
+TRAFFIC = {("stack", 100_000, "bf16"): (2_905_866_240 + 7_171_584, "b851b12eb2899e83"),
+           ("stack", 100_000, "fp8"): (1_453_846_016 + 6_466_560, "b851b12eb2899e83"),
+           ("full100k", 100_000, "bf16"): (204_910_592 + 3_482_368, "b851b12eb2899e83"),
+           ("full2k", 2048, "bf16"): (4_285_696 + 0, "b851b12eb2899e83"),
+           ("swa100k", 100_000, "bf16"): (1_143_552 + 0, "b851b12eb2899e83"),
+           ("paged32", 100_000, "bf16"): (2_271_119_872 + 6_297_600, "b851b12eb2899e83"),
+           ("paged32swa", 100_000, "bf16"): (36_023_296 + 46_336, "b851b12eb2899e83")}
 # The same for one prefill_kernel launch of a full (NoPE) layer on the
 # 8,192-token prompt (a --set full capture of that one launch).
 PREFILL_TRAFFIC = {8192: (83_963_648 + 80_508_928, "38ee5c4a48fcdd23")}
@@ -67,26 +68,41 @@ def per_token_us(ms_max: float, world: int) -> float:
     return ms_max * 1000.0 / world
 
 
-def kernel_sources_hash() -> str:
+# The sources each kernel's launch is built from (its device code and the
+# host code that plans and launches it); a recorded DRAM-traffic figure is
+# reported only while these still hash to the value recorded with it.
+DECODE_SOURCES = ("csrc/flint_decode.cu", "csrc/flint_device.cuh", "csrc/flint_internal.h",
+                  "csrc/flint_abi.cu", "csrc/flint_plan.cpp")
+PREFILL_SOURCES = ("csrc/flint_prefill.cu", "csrc/flint_device.cuh", "csrc/flint_internal.h",
+                   "csrc/flint_abi.cu")
+
+
+def kernel_sources_hash(files=None) -> str:
+    """sha256 (16 hex digits) of the named package sources plus include/flint.h,
+    or of every CUDA/C++ source under csrc/ with files=None."""
     import hashlib
-    d = os.path.join(ROOT, "long_context_decode_flash_b200", "csrc")
+    pkg = os.path.join(ROOT, "long_context_decode_flash_b200")
+    if files is None:
+        d = os.path.join(pkg, "csrc")
+        paths = [os.path.join(d, f) for f in sorted(os.listdir(d)) if f.endswith((".cu", ".cuh", ".h", ".cpp"))]
+    else:
+        paths = [os.path.join(pkg, f) for f in files] + [os.path.join(ROOT, "include", "flint.h")]
     m = hashlib.sha256()
-    for f in sorted(os.listdir(d)):
-        if f.endswith((".cu", ".cuh", ".h", ".cpp")):
-            m.update(f.encode())
-            with open(os.path.join(d, f), "rb") as fh:
-                m.update(fh.read())
+    for path in paths:
+        m.update(os.path.basename(path).encode())
+        with open(path, "rb") as fh:
+            m.update(fh.read())
     return m.hexdigest()[:16]
 
 
 def traffic_for(workload: str, ctx: int, kv: str = "bf16"):
     t = TRAFFIC.get((workload, ctx, kv))
-    return t[0] if t is not None and t[1] == kernel_sources_hash() else None
+    return t[0] if t is not None and t[1] == kernel_sources_hash(DECODE_SOURCES) else None
 
 
 def prefill_traffic(T: int):
     t = PREFILL_TRAFFIC.get(T)
-    return t[0] if t is not None and t[1] == kernel_sources_hash() else None
+    return t[0] if t is not None and t[1] == kernel_sources_hash(PREFILL_SOURCES) else None
 FALLBACK_HBM_GBS = 6650.0
 FALLBACK_BF16_TFLOPS = 1400.0   # sustained, under the power cap
 
