@@ -297,6 +297,17 @@ def prefill_flops(T: int, window: int) -> int:
     return prefill_keys(T, window) * 32 * 128 * 4
 
 
+def prefill_prep_bytes(T: int, window: int) -> int:
+    """Algorithmic HBM bytes of one flint_prefill_qk_norm_rope launch as the
+    step makes it: raw q, k, v read (10 KiB a token); q and k (bf16) and v
+    (fp16) written (10 KiB a token); the cache rows of k and v (2 KiB a
+    token; a 513-slot ring receives only the last 513 tokens)."""
+    row = 128 * 2
+    per_token = (32 + 4 + 4) * row * 2
+    cached = min(T, window) if window else T
+    return T * per_token + cached * 2 * 4 * row
+
+
 def prefill_config(T):
     return {"workload": "prefill of one prompt through Flint's 49 attention layers: per layer "
                         "Q/K RMSNorm (+RoPE), KV-cache write and causal GQA attention with sinks; "
@@ -429,9 +440,12 @@ def run_prefill(args, rank, world, local):
     n_layers = len(layers)
     a0 = [torch.cuda.Event(enable_timing=True) for _ in range(n_layers)]
     a1 = [torch.cuda.Event(enable_timing=True) for _ in range(n_layers)]
+    p0 = [torch.cuda.Event(enable_timing=True) for _ in range(n_layers)]  # the prep launch: p0[i] .. a0[i]
 
     def step(attn_events=False):
         for i, d in enumerate(layers):
+            if attn_events:
+                p0[i].record(stream)
             flint.flint_prefill_qk_norm_rope(d.q_raw, d.k_raw, d.w_q, d.w_k, apply_rope=d.rope, q_out=q,
                                              k_out=k, v_raw=d.v_raw, v_out=v16, cache=d.cache, dev_err=err)
             if attn_events:
@@ -454,6 +468,7 @@ def run_prefill(args, rank, world, local):
     starts = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
     ends = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
     attn_ms = []
+    prep_ms = []
     if world > 1:
         torch.distributed.barrier()
     torch.cuda.synchronize()
@@ -466,6 +481,7 @@ def run_prefill(args, rank, world, local):
             ends[i].record(stream)
             torch.cuda.synchronize()  # the attention events are reused next step
             attn_ms.append([s.elapsed_time(e) for s, e in zip(a0, a1)])
+            prep_ms.append([s.elapsed_time(e) for s, e in zip(p0, a0)])
         t_wall = time.perf_counter() - t_wall
     if world > 1:
         torch.distributed.barrier()
@@ -503,6 +519,20 @@ def run_prefill(args, rank, world, local):
     win_ms = statistics.mean(sum(x[i] for i, f in enumerate(kinds) if not f) for x in attn_ms) / (n_layers - n_full)
     achieved = flops / (attn_total_ms * 1e-3) / 1e12
     peak, peak_kind = measured_tensor_peak()
+    # the norm/RoPE/cache pass (prefill_prep_kernel), HBM-bound: its own events
+    prep_layer_ms = [statistics.mean(x[i] for x in prep_ms) for i in range(n_layers)]
+    prep_bytes = sum(prefill_prep_bytes(T, 0 if full else 513) for full in kinds)
+    prep_gbs = prep_bytes / (sum(prep_layer_ms) * 1e-3) / 1e9
+    hbm_peak, hbm_kind = measured_peak()
+    prep = {"kernel": "flint prefill_prep_kernel", "bound": "hbm",
+            "us_per_layer": sum(prep_layer_ms) * 1e3 / n_layers,
+            "full_layer_us": (statistics.mean(prep_layer_ms[i] for i, f in enumerate(kinds) if f) * 1e3
+                              if n_full else None),
+            "window_layer_us": statistics.mean(prep_layer_ms[i] for i, f in enumerate(kinds) if not f) * 1e3,
+            "algorithmic_bytes_per_prompt": int(prep_bytes), "achieved": prep_gbs, "peak": hbm_peak,
+            "unit": "GB/s", "frac": prep_gbs / hbm_peak, "peak_kind": hbm_kind,
+            "note": "events around each launch; the previous layer's attention output (134 MB fp32) "
+                    "is still being written back from L2 when it starts"}
     line = {
         "metric": PREFILL_METRIC, "value": ms / world, "unit": "ms/prompt",
         "n_gpus": world, "steps": args.steps, "warmup": max(args.warmup, 3), "ms_per_step": ms,
@@ -517,6 +547,7 @@ def run_prefill(args, rank, world, local):
                      "full_layer_attn_us": full_ms * 1e3 if full_ms is not None else None,
                      "window_layer_attn_us": win_ms * 1e3,
                      "traffic": prefill_traffic(T), "traffic_launch": "one full-layer launch"},
+        "prep": prep,
         "cpu_baseline": cpu_baseline,
         "e2e": e2e,
         "gpu_launches": args.steps * 2 * n_layers,

@@ -301,8 +301,16 @@ flint_status flint_attn_stack_noalloc(const flint_layer* layers, int32_t n_layer
  *          CONTIGUOUS / RING cache, row 0 of a PAGED block table): token t
  *          goes to slot t (ring: t % 513, and only the last 513 tokens are
  *          written); an E4M3 cache gets the codes of flint_qk_norm_rope.
+ * Arithmetic in float32 as in flint_qk_norm_rope (the angles formed and
+ * rounded from double), except that the sum of squares runs in another order
+ * and the reciprocal square root is the hardware's (within 2 ulp): q and k
+ * may differ from flint_qk_norm_rope's by one bf16 ulp where a value lies
+ * next to a rounding boundary.
  * T in [1, FLINT_MAX_CONTEXT]; T must fit the cache (contiguous capacity,
- * block table).  Errors as for flint_qk_norm_rope. */
+ * block table).  Every pointer 16-byte aligned.  Errors as for
+ * flint_qk_norm_rope; the kernel streams the tokens through shared memory,
+ * and a copy wait that runs past its time limit sets *dev_err =
+ * FLINT_ERR_TIMEOUT. */
 flint_status flint_prefill_qk_norm_rope(const uint16_t* q_raw, const uint16_t* k_raw,
                                         const uint16_t* v_raw, const uint16_t* w_q,
                                         const uint16_t* w_k, int32_t T, float eps,

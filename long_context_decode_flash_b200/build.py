@@ -23,7 +23,7 @@ LIB = os.path.join(HERE, "libflint.so")
 # wait limit, so that a wait on a stage nobody arms runs out quickly.
 HOOKS_LIB = os.path.join(HERE, "libflint_hooks.so")
 HOOKS_WAIT_LIMIT_NS = 5_000_000
-SOURCES = ["flint_abi.cu", "flint_decode.cu", "flint_prep.cu", "flint_prefill.cu", "flint_cp.cu", "flint_plan.cpp", "flint_noalloc.cu"]
+SOURCES = ["flint_abi.cu", "flint_decode.cu", "flint_prep.cu", "flint_prefill.cu", "flint_prefill_prep.cu", "flint_cp.cu", "flint_plan.cpp", "flint_noalloc.cu"]
 HEADERS = ["flint_internal.h", "flint_device.cuh"]
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 

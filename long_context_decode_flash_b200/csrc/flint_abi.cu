@@ -653,7 +653,9 @@ flint_status flint_prefill_qk_norm_rope(const uint16_t* q_raw, const uint16_t* k
     p.num_blocks = c.num_blocks;
     set_prep_fp8(p, c);
   }
-  return launch_result(launch_prep(p, T, static_cast<cudaStream_t>(stream)), who);
+  int sms = 0;
+  if (device_num_sms(&sms) != 0) return fail(FLINT_ERR_CUDA, "%s: cannot read the device's SM count", who);
+  return launch_result(launch_prefill_prep(p, prefill_prep_grid(T, sms), static_cast<cudaStream_t>(stream)), who);
 }
 
 flint_status flint_prefill_attn(const uint16_t* q, const uint16_t* k, const uint16_t* v, int32_t T,

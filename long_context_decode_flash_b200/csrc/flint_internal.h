@@ -180,8 +180,8 @@ struct PrepParams {
   int32_t do_norm;          // 0: k is already final (plain append)
   int32_t fp8;              // 1: E4M3 cache (k_rows / v_rows are byte rows)
   float k_scale[4], v_scale[4];
-  // prefill: block b is token b of one prompt (position b, cache request 0);
-  // a ring cache receives only the last `capacity` tokens
+  // prefill (prefill_prep_kernel): token t of one prompt at position t, cache
+  // request 0; a ring cache receives only the last `capacity` tokens
   int32_t prefill;
   int32_t n_tokens;
   uint16_t* q_out_bf16;     // q rounded to bf16 [T][32][128], or nullptr
@@ -211,6 +211,10 @@ constexpr int kCpPartialFloats = kHeads * kDim + 2 * kHeads;
 // Launchers (return cudaGetLastError() after the launch).
 cudaError_t launch_decode(const DecodeParams& p, int grid, cudaStream_t stream);  // cooperative if p.grid_merge
 cudaError_t launch_prep(const PrepParams& p, int B, cudaStream_t stream);
+// The prefill pass of one prompt (p.prefill = 1): a persistent grid of
+// `grid` CTAs, each streaming a contiguous range of the p.n_tokens tokens.
+int prefill_prep_grid(int T, int num_sms);
+cudaError_t launch_prefill_prep(const PrepParams& p, int grid, cudaStream_t stream);
 cudaError_t launch_prefill(const PrefillParams& p, cudaStream_t stream);
 cudaError_t launch_merge_partials(const float* partials, int n_parts, int B, const float* sinks, float* out,
                                   cudaStream_t stream);

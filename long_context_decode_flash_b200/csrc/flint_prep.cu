@@ -8,11 +8,10 @@
 // rows, then 4 k rows) with RoPE pairs (i, i+64) in one lane.  k is rounded
 // to bf16 (nearest even) once and the same bits go to k_out and the cache; v
 // is copied bit for bit.  With do_norm = 0 and no RoPE the kernel is a plain
-// bit-exact append of final k and v.  In prefill mode the blocks are the T
-// tokens of one prompt at positions 0 .. T-1, q is written rounded to bf16
-// and v, for the prefill attention's PV product, converted to fp16.  An E4M3 cache receives, for k and v,
+// bit-exact append of final k and v.  An E4M3 cache receives, for k and v,
 // the codes of float32 (value / scale) (nearest even, saturating), where k is
-// the float32 normed (roped) value.
+// the float32 normed (roped) value.  (A prompt's tokens, in prefill, go
+// through prefill_prep_kernel instead.)
 #include "flint_device.cuh"
 
 namespace flint {
@@ -25,17 +24,14 @@ __global__ void __launch_bounds__(kPrepThreads) prep_kernel(const __grid_constan
   __shared__ float2 cs[64];
   const int b = blockIdx.x;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int pos = p.prefill ? b : p.pos[b];
-  const int req = p.prefill ? 0 : b;
+  const int pos = p.pos[b];
+  const int req = b;
   if (p.apply_rope && threadIdx.x < 64) cs[threadIdx.x] = rope_cos_sin(threadIdx.x, pos, p.theta);
   __syncthreads();
 
   // element offset of this request's new-token row (KV head 0), or -1
   long long row = -1;
-  // (a prompt longer than a ring writes only its last `capacity` tokens, so
-  // that no two blocks write one slot)
-  const bool ring_skip = p.prefill && p.layout == FLINT_KV_RING && b < p.n_tokens - p.capacity;
-  if (p.k_rows && !ring_skip) {
+  if (p.k_rows) {
     if (p.layout == FLINT_KV_PAGED) {
       const int blk = p.table[static_cast<long long>(req) * p.max_blocks + pos / kBlock];
       if (blk >= 0 && blk < p.num_blocks) {
@@ -63,11 +59,6 @@ __global__ void __launch_bounds__(kPrepThreads) prep_kernel(const __grid_constan
         reinterpret_cast<float2*>(o)[lane] = make_float2(y[0], y[1]);
         reinterpret_cast<float2*>(o + 64)[lane] = make_float2(y[2], y[3]);
       }
-      if (p.q_out_bf16) {
-        uint32_t* o = reinterpret_cast<uint32_t*>(p.q_out_bf16 + (static_cast<long long>(b) * kHeads + r) * kDim);
-        o[lane] = pack_bf16x2(y[0], y[1]);
-        o[32 + lane] = pack_bf16x2(y[2], y[3]);
-      }
     } else {
       const uint32_t ka = pack_bf16x2(y[0], y[1]), kb = pack_bf16x2(y[2], y[3]);
       if (p.k_out) {
@@ -86,17 +77,6 @@ __global__ void __launch_bounds__(kPrepThreads) prep_kernel(const __grid_constan
         o[32 + lane] = static_cast<uint16_t>(f32x2_to_e4m3x2(__fdiv_rn(y[2], s), __fdiv_rn(y[3], s)));
       }
     }
-  }
-  if (p.v_out_f16 && warp < kKvHeads) {
-    // lane: dims 4l .. 4l+3; bf16 -> fp16 to nearest, saturating at +-65504
-    const uint2 x = reinterpret_cast<const uint2*>(p.v_raw + (static_cast<long long>(b) * kKvHeads + warp) * kDim)[lane];
-    auto sat = [](float f) { return fminf(fmaxf(f, -65504.f), 65504.f); };
-    const __half2 a = __floats2half2_rn(sat(bf16_lo(x.x)), sat(bf16_hi(x.x)));
-    const __half2 c = __floats2half2_rn(sat(bf16_lo(x.y)), sat(bf16_hi(x.y)));
-    uint2 y;
-    y.x = *reinterpret_cast<const uint32_t*>(&a);
-    y.y = *reinterpret_cast<const uint32_t*>(&c);
-    reinterpret_cast<uint2*>(p.v_out_f16 + (static_cast<long long>(b) * kKvHeads + warp) * kDim)[lane] = y;
   }
   if (row >= 0 && warp < kKvHeads) {
     const uint2* src = reinterpret_cast<const uint2*>(p.v_raw + (static_cast<long long>(b) * kKvHeads + warp) * kDim);

@@ -108,7 +108,7 @@ def open_library(path: str) -> ctypes.CDLL:
                  "flint_merge_partials"):
         getattr(lib, name).restype = ctypes.c_int
     # test builds only (libflint_hooks.so): leave one pipeline stage unarmed
-    for name in ("flint_test_stall_decode", "flint_test_stall_prefill"):
+    for name in ("flint_test_stall_decode", "flint_test_stall_prefill", "flint_test_stall_prefill_prep"):
         if hasattr(lib, name):
             getattr(lib, name).argtypes = [ctypes.c_int, ctypes.c_int]
             getattr(lib, name).restype = ctypes.c_int

@@ -460,3 +460,111 @@ def test_prefill_drain_keyed_on_the_tile_count_is_caught():
         cta = prefill_run(rng.randint(6, 12), rng, 0.05, drain="count")
         caught += cta.in_flight_at_exit > 0
     assert caught > 0
+
+
+# ---------------------------------------------------------------------------
+# prefill_prep_kernel: one producer warp fills a ring of token slots (the
+# expected bytes raised first, the copies issued, then the warp's arrivals);
+# every consumer warp reads every token's slot and releases it.
+
+def prep_run(n, slots, warps, rng, p_timeout, stall_k=None, drain="handed_out"):
+    """n: tokens of the CTA's range.  stall_k: token whose slot the producer
+    never arms (the test hook).  drain: "handed_out" (the kernel: the last
+    `slots` tokens the producer got to) or "range" (the last `slots` tokens
+    of the whole range, a mistake the tests below catch)."""
+    cta = Cta(rng, p_timeout)
+    full = [Bar(1) for _ in range(slots)]
+    empty = [Bar(warps) for _ in range(slots)]
+    slot_tok = [None] * slots
+    res = {}
+
+    def producer():
+        k = 0
+        while k < n:
+            s = k % slots
+            if k >= slots:
+                ok = yield from cta.wait(empty[s], (k // slots - 1) & 1)
+                if not ok:
+                    cta.raise_abort()
+                    break
+            if cta.abort:
+                break
+            if k != stall_k:
+                old = slot_tok[s]
+                assert old is None or old["landed"], f"slot {s} re-armed while token {old['k']} is landing"
+                tag = {"landed": False, "k": k}
+                slot_tok[s] = tag
+                full[s].tx += 1                        # expect_tx, no arrival
+                cta.landing.append((full[s], 1, tag))  # the bulk copies
+                yield
+                full[s].arrive()                       # after the angles and the row
+            k += 1
+        res["handed_out"] = k
+
+    def consumer(w):
+        for k in range(n):
+            s = k % slots
+            ok = yield from cta.wait(full[s], (k // slots) & 1)
+            if not ok:
+                cta.raise_abort()
+                return
+            tag = slot_tok[s]
+            assert tag is not None and tag["k"] == k and tag["landed"], \
+                f"warp {w} read slot {s} for token {k} before it landed"
+            empty[s].arrive()
+            yield
+
+    actors = {"producer": producer()}
+    for w in range(warps):
+        actors[f"c{w}"] = consumer(w)
+    run_actors(cta, actors)
+
+    # __syncthreads, then the drain (producer lane 0) after an abort
+    if cta.abort:
+        last = res["handed_out"] if drain == "handed_out" else n
+        for k in range(max(0, last - slots), last):
+            if k == stall_k:
+                continue
+            bar, parity = full[k % slots], (k // slots) & 1
+            while not bar.parity_ok(parity):
+                if not any(b is bar for b, _, _ in cta.landing):
+                    break
+                cta.land_one()
+    cta.in_flight_at_exit = len(cta.landing)
+    return cta
+
+
+@pytest.mark.parametrize("slots", [2, 6, 8])
+def test_prefill_prep_abort_leaves_nothing_in_flight(slots):
+    rng = random.Random(700 + slots)
+    for trial in range(400):
+        n = rng.randint(1, 30)
+        p = rng.choice([0.0, 0.001, 0.01, 0.05, 0.3])
+        cta = prep_run(n, slots, 8, rng, p)
+        assert cta.in_flight_at_exit == 0, f"trial {trial}: a copy is in flight at exit (n={n}, p={p})"
+        assert (cta.status == 5) == (cta.gave_up > 0), f"trial {trial}: status {cta.status}, gave up {cta.gave_up}"
+
+
+def test_prefill_prep_stalled_slot_times_out_and_drains():
+    """The GPU test hook: the producer never arms one token's slot; the
+    consumers give up on it, the producer (waiting for that slot to come
+    free) sees the abort, the status is TIMEOUT and nothing is in flight."""
+    rng = random.Random(77)
+    for trial in range(300):
+        n = rng.randint(2, 30)
+        stall = rng.randrange(n)
+        cta = prep_run(n, 6, 8, rng, p_timeout=0.0005, stall_k=stall)
+        assert cta.status == 5 and cta.in_flight_at_exit == 0, f"trial {trial}"
+
+
+def test_prefill_prep_drain_keyed_on_the_range_is_caught():
+    """Waiting on the last slots of the token range instead of the tokens the
+    producer handed out: after an early abort those phases were never armed,
+    and a parity wait on one passes on an older phase while a copy lands."""
+    rng = random.Random(78)
+    caught = 0
+    for trial in range(600):
+        n = rng.randint(12, 30)
+        cta = prep_run(n, 6, 8, rng, 0.05, drain="range")
+        caught += cta.in_flight_at_exit > 0
+    assert caught > 0

@@ -11,7 +11,7 @@ import oracle
 from long_context_decode_flash_b200 import flint
 from long_context_decode_flash_b200 import inputs as I
 
-from helpers import bf16_ulp_diff, dev, e4m3_code_distance, parity
+from helpers import close_bits, dev, e4m3_code_distance, parity, u16
 
 pytestmark = pytest.mark.gpu
 
@@ -56,29 +56,6 @@ def attn_gpu(q, k, v, sinks, window):
 def oracle_prefill(p: I.PrefillInputs, rows):
     return oracle.prefill(I.bits(p.q_raw), I.bits(p.k_raw), I.bits(p.v_raw), I.bits(p.w_q), I.bits(p.w_k),
                           p.sinks.numpy().astype(np.float64), p.window, p.rope, rows=rows)
-
-
-def u16(t: torch.Tensor) -> np.ndarray:
-    return t.cpu().view(torch.int16).numpy().view(np.uint16)
-
-
-def bf16_values(bits: np.ndarray) -> np.ndarray:
-    with np.errstate(invalid="ignore"):  # sentinel slots may hold NaN patterns
-        return (bits.astype(np.uint32) << 16).view(np.float32).astype(np.float64)
-
-
-def close_bits(got, want, what):
-    """bf16 values after norm (+RoPE): float32 on the device, float64 in the
-    oracle, each rounded once to bf16.  They differ rarely, and then by one
-    ulp -- or, where RoPE's x cos - y sin cancels to near zero, by a few 1e-7
-    in absolute terms, which is many ulps of so small a value (the inputs are
-    O(1) after the norm); 1e-5 absolute bounds that case."""
-    d = bf16_ulp_diff(got, want)
-    a, b = bf16_values(got), bf16_values(want)
-    with np.errstate(invalid="ignore"):  # sentinel slots may hold inf / NaN patterns (equal bits)
-        ok = (d <= 1) | (np.abs(a - b) <= 1e-5)
-    assert ok.all(), f"{what}: {int((~ok).sum())} values apart by more than 1 ulp and 1e-5"
-    assert (d > 0).mean() <= 0.01, f"{what}: {(d > 0).mean():.4f} of the values differ"
 
 
 @pytest.mark.parametrize("window", [flint.WINDOW, 0])

@@ -22,7 +22,7 @@ from long_context_decode_flash_b200 import build as cuda_build
 from long_context_decode_flash_b200 import flint
 from long_context_decode_flash_b200 import inputs as I
 
-from helpers import DeviceLayer, dev, oracle_layer, parity
+from helpers import DeviceLayer, close_bits, dev, oracle_layer, parity, u16
 
 pytestmark = pytest.mark.gpu
 
@@ -145,3 +145,42 @@ def test_prefill_stalled_k_tile_times_out_then_recovers(hooks):
         torch.cuda.synchronize()
         assert int(err.item()) == 0
     parity(out.cpu().numpy(), want, "prefill after a time-out", per_head=True)
+
+
+def test_prefill_prep_stalled_slot_times_out_then_recovers(hooks):
+    """The prefill's norm/RoPE pass: CTA 0 leaves the slot of its second token
+    unarmed, so its consumer warps' waits run out and its producer, waiting
+    for a slot to come free, sees the abort."""
+    T = 1000
+    p = I.make_prefill(T, flint.WINDOW, workload=I.W_PREFILL + 31)
+    _, qb, kb = oracle.prefill(I.bits(p.q_raw), I.bits(p.k_raw), I.bits(p.v_raw), I.bits(p.w_q),
+                               I.bits(p.w_k), p.sinks.numpy().astype(np.float64), flint.WINDOW, p.rope, rows=[])
+    q_raw, k_raw, v_raw, w_q, w_k = dev(p.q_raw), dev(p.k_raw), dev(p.v_raw), dev(p.w_q), dev(p.w_k)
+    q = torch.empty((T, 32, 128), dtype=torch.bfloat16, device="cuda")
+    k = torch.empty((T, 4, 128), dtype=torch.bfloat16, device="cuda")
+    v16 = torch.empty((T, 4, 128), dtype=torch.float16, device="cuda")
+    err = torch.zeros(1, dtype=torch.int32, device="cuda")
+
+    def call():
+        flint.flint_prefill_qk_norm_rope(q_raw, k_raw, w_q, w_k, apply_rope=p.rope, q_out=q, k_out=k,
+                                         v_raw=v_raw, v_out=v16, dev_err=err)
+
+    with using(hooks):
+        assert hooks.flint_test_stall_prefill_prep(-1, -1) == 0
+        call()
+        torch.cuda.synchronize()
+        assert int(err.item()) == 0
+        assert hooks.flint_test_stall_prefill_prep(0, 1) == 0
+        dt = timed(call)
+        assert int(err.item()) == flint.FLINT_ERR_TIMEOUT
+        assert dt < 6 * LIMIT_S + 0.25, f"the timed-out call took {dt:.3f} s"
+        assert hooks.flint_test_stall_prefill_prep(-1, -1) == 0
+        err.zero_()
+        for t in (q, k, v16):
+            t.fill_(float("nan"))
+        call()
+        torch.cuda.synchronize()
+        assert int(err.item()) == 0
+    close_bits(u16(q), qb, "q after a time-out")
+    close_bits(u16(k), kb, "k after a time-out")
+    np.testing.assert_array_equal(u16(v16), u16(p.v_raw.to(torch.float16)))
