@@ -312,14 +312,18 @@ __device__ void run_softmax(const PrefillParams& p, const Work& w, uint32_t tmem
       break;
     }
     tc_fence_after();
+    static_assert(kH == 64, "two 32-column loads per tile");
     float s[kH];  // raw scores q.k
-#pragma unroll
-    for (int c = 0; c < kH / 32; ++c) {
-      uint32_t v[32];
-      tmem_ld32(lane_base + kColS + (jj & 1) * kPkv + kH * wg + 32 * c, v);
+    {
+      uint32_t v0[32], v1[32];
+      tmem_ld32(lane_base + kColS + (jj & 1) * kPkv + kH * wg, v0);
+      tmem_ld32(lane_base + kColS + (jj & 1) * kPkv + kH * wg + 32, v1);
       tmem_wait_ld();
 #pragma unroll
-      for (int i = 0; i < 32; ++i) s[32 * c + i] = __uint_as_float(v[i]);
+      for (int i = 0; i < 32; ++i) {
+        s[i] = __uint_as_float(v0[i]);
+        s[32 + i] = __uint_as_float(v1[i]);
+      }
     }
     if (!w.interior(jj, p.window)) {
       const int k0 = (w.j_first + jj) * kPkv + kH * wg;
@@ -333,8 +337,8 @@ __device__ void run_softmax(const PrefillParams& p, const Work& w, uint32_t tmem
 #pragma unroll
     for (int q = 0; q < 8; ++q) mq[q] = s[q];
 #pragma unroll
-    for (int i = 8; i < kH; ++i) mq[i & 7] = fmaxf(mq[i & 7], s[i]);
-    float mh = fmaxf(fmaxf(fmaxf(mq[0], mq[1]), fmaxf(mq[2], mq[3])), fmaxf(fmaxf(mq[4], mq[5]), fmaxf(mq[6], mq[7])));
+    for (int i = 8; i < kH; i += 2) mq[(i >> 1) & 7] = max3(mq[(i >> 1) & 7], s[i], s[i + 1]);
+    const float mh = max3(max3(mq[0], mq[1], mq[2]), max3(mq[3], mq[4], mq[5]), fmaxf(mq[6], mq[7]));
     // exchange the half-row maxima (every thread arrives; bounded wait)
     float* slot = red + (jj & 1) * 2 * kRows;
     slot[wg * kRows + r] = mh;
@@ -353,15 +357,19 @@ __device__ void run_softmax(const PrefillParams& p, const Work& w, uint32_t tmem
     }
     const float mu = (m == -INFINITY) ? 0.f : m;
     uint32_t pk[kH / 2];  // fp16 pairs
-    float ls[4] = {0.f, 0.f, 0.f, 0.f};
+    // scale, shift and sum a pair of scores per paired-fp32 instruction
+    const float2 scale2 = make_float2(kPfScale, kPfScale), nmu2 = make_float2(-mu, -mu);
+    float2 ls[2] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
 #pragma unroll
     for (int c = 0; c < kH / 2; ++c) {
-      const float p0 = ex2(fmaf(s[2 * c], kPfScale, -mu)), p1 = ex2(fmaf(s[2 * c + 1], kPfScale, -mu));
-      ls[c & 3] += p0 + p1;
-      const __half2 hp = __floats2half2_rn(p0, p1);
+      const float2 x = fma2(make_float2(s[2 * c], s[2 * c + 1]), scale2, nmu2);
+      const float2 pp = make_float2(ex2(x.x), ex2(x.y));
+      ls[c & 1] = add2(ls[c & 1], pp);
+      const __half2 hp = __floats2half2_rn(pp.x, pp.y);
       pk[c] = *reinterpret_cast<const uint32_t*>(&hp);
     }
-    l += (ls[0] + ls[1]) + (ls[2] + ls[3]);
+    const float2 lsum = add2(ls[0], ls[1]);
+    l += lsum.x + lsum.y;
     if (jj > 0) {
       // P's columns and O are free once the previous tile's PV has completed
       if (!warp_wait(smem_u32(&B->pv_done), static_cast<uint32_t>(jj - 1) & 1u, B)) {
@@ -376,7 +384,12 @@ __device__ void run_softmax(const PrefillParams& p, const Work& w, uint32_t tmem
           tmem_ld32(lane_base + kColO + 64 * wg + 32 * c, v);
           tmem_wait_ld();
 #pragma unroll
-          for (int i = 0; i < 32; ++i) v[i] = __float_as_uint(__uint_as_float(v[i]) * factor);
+          for (int i = 0; i < 32; i += 2) {
+            const float2 o2 = mul2(make_float2(__uint_as_float(v[i]), __uint_as_float(v[i + 1])),
+                                   make_float2(factor, factor));
+            v[i] = __float_as_uint(o2.x);
+            v[i + 1] = __float_as_uint(o2.y);
+          }
           tmem_st32(lane_base + kColO + 64 * wg + 32 * c, v);
         }
       }
