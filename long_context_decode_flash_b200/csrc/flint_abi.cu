@@ -697,7 +697,9 @@ flint_status flint_prefill_attn(const uint16_t* q, const uint16_t* k, const uint
   p.dev_err = dev_err;
   p.T = T;
   p.window = window;
-  return launch_result(launch_prefill(p, static_cast<cudaStream_t>(stream)), who);
+  int sms = 0;
+  if (device_num_sms(&sms) != 0) return fail(FLINT_ERR_CUDA, "%s: cannot read the device's SM count", who);
+  return launch_result(launch_prefill(p, sms, static_cast<cudaStream_t>(stream)), who);
 }
 
 size_t flint_attn_workspace_bytes(int32_t n_problems, int32_t num_ctas) {

@@ -215,7 +215,9 @@ cudaError_t launch_prep(const PrepParams& p, int B, cudaStream_t stream);
 // `grid` CTAs, each streaming a contiguous range of the p.n_tokens tokens.
 int prefill_prep_grid(int T, int num_sms);
 cudaError_t launch_prefill_prep(const PrepParams& p, int grid, cudaStream_t stream);
-cudaError_t launch_prefill(const PrefillParams& p, cudaStream_t stream);
+// One persistent CTA per SM (num_sms), each over a share of the (query block,
+// KV head) units.
+cudaError_t launch_prefill(const PrefillParams& p, int num_sms, cudaStream_t stream);
 cudaError_t launch_merge_partials(const float* partials, int n_parts, int B, const float* sinks, float* out,
                                   cudaStream_t stream);
 

@@ -36,6 +36,8 @@
 // [384,512).  Every wait is bounded; a timeout raises FLINT_ERR_TIMEOUT.
 #include <math.h>
 
+#include <algorithm>
+
 #include "flint_device.cuh"
 
 namespace flint {
@@ -55,7 +57,10 @@ constexpr uint32_t kQBytes = 2 * kRows * 128;          // 32 KiB
 constexpr uint32_t kOffK = kQBytes;
 constexpr uint32_t kOffV = kOffK + kKs * kTileBytes;
 constexpr uint32_t kOffRed = kOffV + kVs * kTileBytes;  // row-maximum exchange [2 tiles][2 wg][128]
-constexpr uint32_t kOffBar = kOffRed + 2 * 2 * kRows * 4;
+constexpr uint32_t kOffL = kOffRed + 2 * 2 * kRows * 4;    // row-sum exchange [2 wg][128], once per unit
+constexpr uint32_t kOffStage = kOffL + 2 * kRows * 4;  // output staging, [softmax warp][32 rows][16 floats]
+constexpr uint32_t kStageWarpBytes = 32 * 16 * 4;
+constexpr uint32_t kOffBar = kOffStage + kSoftWarps * kStageWarpBytes;
 constexpr size_t kPfSmem = kOffBar + 256 + 1024;        // barriers, TMEM address, flags; alignment slack
 constexpr float kPfLog2e = 1.4426950408889634f;
 constexpr float kPfScale = static_cast<float>(1.4426950408889634 * 0.08838834764831845);
@@ -68,7 +73,8 @@ constexpr uint32_t kIdescS = (1u << 4) | (1u << 7) | (1u << 10) | ((kPkv >> 3) <
 constexpr uint32_t kIdescPV = (1u << 4) | (1u << 16) | ((kDim >> 3) << 17) | ((128 >> 4) << 24);
 
 struct Bars {  // at kOffBar
-  uint64_t q_full;
+  uint64_t q_full;        // the unit's Q tile landed (phase = unit)
+  uint64_t q_empty;       // every S MMA of the unit completed: Q may be replaced
   uint64_t k_full[kKs], k_empty[kKs];
   uint64_t v_full[kVs], v_empty[kVs];
   uint64_t s_full[2];
@@ -76,7 +82,7 @@ struct Bars {  // at kOffBar
   uint64_t pv_done;
   uint64_t mma_done;
   uint64_t red_full[2];   // both softmax warpgroups wrote their row maxima (per tile parity)
-  uint64_t l_full;        // ... their row sums (once, at the end)
+  uint64_t l_full;        // ... their row sums (once per unit)
   uint32_t tmem_base;
   int abort;
 };
@@ -157,9 +163,9 @@ __device__ __forceinline__ void raise_abort(const PrefillParams& p, Bars* B) {
 __device__ int g_stall_prefill[2] = {-1, -1};
 #endif
 
-// K and V tiles whose loads the producer issued (the drain's bound).
+// Q, K and V tiles whose loads the producer issued (the drain's bound).
 struct Issued {
-  int k, v;
+  int k, v, q;
 };
 
 __device__ __forceinline__ bool aborted(const Bars* B) {
@@ -175,11 +181,14 @@ struct Work {
   }
 };
 
-__device__ __forceinline__ Work work_of(const PrefillParams& p) {
+// Units (block of 16 query tokens, KV head), numbered longest first.
+__device__ __forceinline__ int n_units(const PrefillParams& p) { return (p.T + kPq - 1) / kPq * kKvHeads; }
+
+__device__ __forceinline__ Work work_of_unit(const PrefillParams& p, int u) {
   const int nblk = (p.T + kPq - 1) / kPq;
-  const int qb = nblk - 1 - static_cast<int>(blockIdx.x) / kKvHeads;  // longest blocks first
+  const int qb = nblk - 1 - u / kKvHeads;
   Work w;
-  w.g = static_cast<int>(blockIdx.x) % kKvHeads;
+  w.g = u % kKvHeads;
   w.t0 = qb * kPq;
   const int t_last = min(w.t0 + kPq - 1, p.T - 1);
   w.j_first = p.window > 0 ? max(0, w.t0 - (p.window - 1)) / kPkv : 0;
@@ -187,42 +196,67 @@ __device__ __forceinline__ Work work_of(const PrefillParams& p) {
   return w;
 }
 
-// Returns the K and V tiles it issued.  Once the CTA aborted it issues
-// nothing more.
-__device__ Issued run_tma(const PrefillParams& p, const Work& w, uint8_t* smem, Bars* B) {
+// The i-th unit of this CTA: rounds of gridDim.x units, dealt in alternating
+// directions so that every CTA's total is close to the mean; >= n_units(p)
+// past the CTA's last unit.
+__device__ __forceinline__ int unit_of(int i) {
+  const int G = static_cast<int>(gridDim.x), c = static_cast<int>(blockIdx.x);
+  return i * G + ((i & 1) ? G - 1 - c : c);
+}
+
+// The producer: per unit, the Q tile (once the previous unit's S MMAs are
+// done with the buffer), then the unit's K and V tiles through the rings,
+// counted across units.  Returns what it issued; once the CTA aborted it
+// issues nothing more.
+__device__ Issued run_tma(const PrefillParams& p, uint8_t* smem, Bars* B) {
   const uint32_t base = smem_u32(smem);
-  Issued n{0, 0};
-  mbar_expect_tx(smem_u32(&B->q_full), kQBytes);
-  tma_load_4d(base, &p.q_map, smem_u32(&B->q_full), 0, w.g * kGroup, w.t0, 0);
-  tma_load_4d(base + kRows * 128, &p.q_map, smem_u32(&B->q_full), 64, w.g * kGroup, w.t0, 0);
-  for (int jj = 0; jj < w.n; ++jj) {
-    const int k0 = (w.j_first + jj) * kPkv;
-    const int sk = jj % kKs, sv = jj % kVs;
-    if (jj >= kKs && !mbar_wait(smem_u32(&B->k_empty[sk]), static_cast<uint32_t>(jj / kKs - 1) & 1u, &B->abort)) {
+  Issued n{0, 0, 0};
+  const int units = n_units(p);
+  int T = 0;  // the CTA's tile count so far
+  for (int i = 0;; ++i) {
+    const int u = unit_of(i);
+    if (u >= units) break;
+    const Work w = work_of_unit(p, u);
+    if (i > 0 && !mbar_wait(smem_u32(&B->q_empty), static_cast<uint32_t>(i - 1) & 1u, &B->abort)) {
       raise_abort(p, B);
       return n;
     }
     if (aborted(B)) return n;
-    const uint32_t dk = base + kOffK + sk * kTileBytes;
+    mbar_expect_tx(smem_u32(&B->q_full), kQBytes);
+    tma_load_4d(base, &p.q_map, smem_u32(&B->q_full), 0, w.g * kGroup, w.t0, 0);
+    tma_load_4d(base + kRows * 128, &p.q_map, smem_u32(&B->q_full), 64, w.g * kGroup, w.t0, 0);
+    n.q = i + 1;
+    for (int jj = 0; jj < w.n; ++jj) {
+      const int tt = T + jj;
+      const int k0 = (w.j_first + jj) * kPkv;
+      const int sk = tt % kKs, sv = tt % kVs;
+      if (tt >= kKs && !mbar_wait(smem_u32(&B->k_empty[sk]), static_cast<uint32_t>(tt / kKs - 1) & 1u, &B->abort)) {
+        raise_abort(p, B);
+        return n;
+      }
+      if (aborted(B)) return n;
+      const uint32_t dk = base + kOffK + sk * kTileBytes;
 #ifdef FLINT_TEST_HOOKS
-    if (!(static_cast<int>(blockIdx.x) == g_stall_prefill[0] && jj == g_stall_prefill[1]))
+      if (!(static_cast<int>(blockIdx.x) == g_stall_prefill[0] && tt == g_stall_prefill[1]))
 #endif
-    {
-      mbar_expect_tx(smem_u32(&B->k_full[sk]), kTileBytes);
-      tma_load_4d(dk, &p.k_map, smem_u32(&B->k_full[sk]), 0, w.g, k0, 0);
-      tma_load_4d(dk + kHalfBytes, &p.k_map, smem_u32(&B->k_full[sk]), 64, w.g, k0, 0);
+      {
+        mbar_expect_tx(smem_u32(&B->k_full[sk]), kTileBytes);
+        tma_load_4d(dk, &p.k_map, smem_u32(&B->k_full[sk]), 0, w.g, k0, 0);
+        tma_load_4d(dk + kHalfBytes, &p.k_map, smem_u32(&B->k_full[sk]), 64, w.g, k0, 0);
+      }
+      n.k = tt + 1;
+      if (tt >= kVs && !mbar_wait(smem_u32(&B->v_empty[sv]), static_cast<uint32_t>(tt / kVs - 1) & 1u, &B->abort)) {
+        raise_abort(p, B);
+        return n;
+      }
+      if (aborted(B)) return n;
+      const uint32_t dv = base + kOffV + sv * kTileBytes;
+      mbar_expect_tx(smem_u32(&B->v_full[sv]), kTileBytes);
+      tma_load_4d(dv, &p.v_map, smem_u32(&B->v_full[sv]), 0, w.g, k0, 0);
+      tma_load_4d(dv + kHalfBytes, &p.v_map, smem_u32(&B->v_full[sv]), 64, w.g, k0, 0);
+      n.v = tt + 1;
     }
-    n.k = jj + 1;
-    if (jj >= kVs && !mbar_wait(smem_u32(&B->v_empty[sv]), static_cast<uint32_t>(jj / kVs - 1) & 1u, &B->abort)) {
-      raise_abort(p, B);
-      return n;
-    }
-    if (aborted(B)) return n;
-    const uint32_t dv = base + kOffV + sv * kTileBytes;
-    mbar_expect_tx(smem_u32(&B->v_full[sv]), kTileBytes);
-    tma_load_4d(dv, &p.v_map, smem_u32(&B->v_full[sv]), 0, w.g, k0, 0);
-    tma_load_4d(dv + kHalfBytes, &p.v_map, smem_u32(&B->v_full[sv]), 64, w.g, k0, 0);
-    n.v = jj + 1;
+    T += w.n;
   }
   return n;
 }
@@ -239,16 +273,18 @@ __device__ void drain_tma(Issued n, Bars* B) {
     while (!mbar_try_wait(bar, parity))
       if (globaltimer_ns() - t0 > kWaitLimitNs) return;
   };
-  wait(smem_u32(&B->q_full), 0);
+  if (n.q > 0) wait(smem_u32(&B->q_full), static_cast<uint32_t>(n.q - 1) & 1u);
   for (int jj = max(0, n.k - kKs); jj < n.k; ++jj)
     wait(smem_u32(&B->k_full[jj % kKs]), static_cast<uint32_t>(jj / kKs) & 1u);
   for (int jj = max(0, n.v - kVs); jj < n.v; ++jj)
     wait(smem_u32(&B->v_full[jj % kVs]), static_cast<uint32_t>(jj / kVs) & 1u);
 }
 
-// S[jj & 1] = Q K_jj^T: 8 MMAs of K = 16 dims (32 bytes inside a swizzled
-// 128-byte row; the second 64 dims in the second box).
-__device__ __forceinline__ bool issue_s(const PrefillParams& p, int jj, uint32_t base, uint32_t tmem, Bars* B) {
+// S[jj & 1] = Q K_jj^T for the CTA's tile jj: 8 MMAs of K = 16 dims (32 bytes
+// inside a swizzled 128-byte row; the second 64 dims in the second box).
+// last: the unit's last S, after which Q may be replaced.
+__device__ __forceinline__ bool issue_s(const PrefillParams& p, int jj, bool last, uint32_t base, uint32_t tmem,
+                                        Bars* B) {
   const int sk = jj % kKs;
   if (!mbar_wait(smem_u32(&B->k_full[sk]), static_cast<uint32_t>(jj / kKs) & 1u, &B->abort)) return false;
   tc_fence_after();
@@ -262,29 +298,50 @@ __device__ __forceinline__ bool issue_s(const PrefillParams& p, int jj, uint32_t
   }
   umma_commit(smem_u32(&B->k_empty[sk]));
   umma_commit(smem_u32(&B->s_full[jj & 1]));
+  if (last) umma_commit(smem_u32(&B->q_empty));
   return true;
 }
 
-__device__ void run_mma(const PrefillParams& p, const Work& w, uint32_t base, uint32_t tmem, Bars* B) {
+// The MMA thread, over the CTA's units with its tiles counted across them.
+// Per unit: S of the first two tiles, then per tile PV and the S two tiles
+// ahead within the unit.  The first PV of a unit overwrites O: every softmax
+// warp read the previous unit's O out of TMEM before it wrote its half of
+// this tile's P, so p_full already orders that PV after the reads.  The next unit's first S come after
+// this unit's last PV, so that no PV waits for the next Q tile.
+__device__ void run_mma(const PrefillParams& p, uint32_t base, uint32_t tmem, Bars* B) {
+  const int units = n_units(p);
+  int T = 0;
+  Work w = work_of_unit(p, unit_of(0));
   bool ok = mbar_wait(smem_u32(&B->q_full), 0, &B->abort);
-  if (ok) ok = issue_s(p, 0, base, tmem, B);
-  if (ok && w.n > 1) ok = issue_s(p, 1, base, tmem, B);
-  for (int jj = 0; ok && jj < w.n; ++jj) {
-    const int sv = jj % kVs;
-    ok = mbar_wait(smem_u32(&B->p_full), static_cast<uint32_t>(jj) & 1u, &B->abort) &&
-         mbar_wait(smem_u32(&B->v_full[sv]), static_cast<uint32_t>(jj / kVs) & 1u, &B->abort);
-    if (!ok) break;
-    tc_fence_after();
-    const uint32_t vb = base + kOffV + sv * kTileBytes;
-    // O += P V: K = 16 keys per MMA (rows 16kk.. of both 64-dim boxes; the
-    // fp16 pairs of keys 16kk .. 16kk + 15 are columns 8kk .. 8kk + 7 of P)
+  if (ok) ok = issue_s(p, 0, w.n == 1, base, tmem, B);
+  if (ok && w.n > 1) ok = issue_s(p, 1, w.n == 2, base, tmem, B);
+  for (int i = 0; ok; ++i) {
+    for (int jj = 0; ok && jj < w.n; ++jj) {
+      const int tt = T + jj;
+      const int sv = tt % kVs;
+      ok = mbar_wait(smem_u32(&B->p_full), static_cast<uint32_t>(tt) & 1u, &B->abort) &&
+           mbar_wait(smem_u32(&B->v_full[sv]), static_cast<uint32_t>(tt / kVs) & 1u, &B->abort);
+      if (!ok) break;
+      tc_fence_after();
+      const uint32_t vb = base + kOffV + sv * kTileBytes;
+      // O += P V: K = 16 keys per MMA (rows 16kk.. of both 64-dim boxes; the
+      // fp16 pairs of keys 16kk .. 16kk + 15 are columns 8kk .. 8kk + 7 of P)
 #pragma unroll
-    for (int kk = 0; kk < 8; ++kk)
-      umma_ts(tmem + kColO, tmem + kColP + kk * 8, sw128_desc(vb + kk * 16 * 128, kHalfBytes, 1024), kIdescPV,
-              (jj > 0 || kk > 0) ? 1u : 0u);
-    umma_commit(smem_u32(&B->v_empty[sv]));
-    umma_commit(smem_u32(&B->pv_done));
-    if (jj + 2 < w.n) ok = issue_s(p, jj + 2, base, tmem, B);
+      for (int kk = 0; kk < 8; ++kk)
+        umma_ts(tmem + kColO, tmem + kColP + kk * 8, sw128_desc(vb + kk * 16 * 128, kHalfBytes, 1024), kIdescPV,
+                (jj > 0 || kk > 0) ? 1u : 0u);
+      umma_commit(smem_u32(&B->v_empty[sv]));
+      umma_commit(smem_u32(&B->pv_done));
+      if (jj + 2 < w.n) ok = issue_s(p, tt + 2, jj + 2 == w.n - 1, base, tmem, B);
+    }
+    if (!ok) break;
+    T += w.n;
+    const int u = unit_of(i + 1);
+    if (u >= units) break;
+    w = work_of_unit(p, u);
+    ok = mbar_wait(smem_u32(&B->q_full), static_cast<uint32_t>(i + 1) & 1u, &B->abort);
+    if (ok) ok = issue_s(p, T, w.n == 1, base, tmem, B);
+    if (ok && w.n > 1) ok = issue_s(p, T + 1, w.n == 2, base, tmem, B);
   }
   if (!ok) raise_abort(p, B);
   // let every issued MMA finish before the CTA ends (its TMEM is freed)
@@ -295,8 +352,10 @@ __device__ void run_mma(const PrefillParams& p, const Work& w, uint32_t base, ui
   }
 }
 
-__device__ void run_softmax(const PrefillParams& p, const Work& w, uint32_t tmem, uint8_t* smem, Bars* B,
-                            int warp, int lane) {
+// One unit (the CTA's i-th; its tiles are the CTA's T .. T + w.n - 1).
+// Returns false if a wait ran out (the caller stops).
+__device__ bool softmax_unit(const PrefillParams& p, const Work& w, int i, int T, uint32_t tmem, uint8_t* smem,
+                             Bars* B, int warp, int lane) {
   const int wg = warp >> 2;               // key half of every tile, dims half of O
   const int r = (warp & 3) * 32 + lane;   // TMEM lane = query row
   const int t = w.t0 + (r >> 3);          // its token
@@ -307,7 +366,8 @@ __device__ void run_softmax(const PrefillParams& p, const Work& w, uint32_t tmem
   bool ok = true;
   constexpr int kH = kPkv / 2;            // keys of this thread per tile
   for (int jj = 0; jj < w.n; ++jj) {
-    if (!warp_wait(smem_u32(&B->s_full[jj & 1]), static_cast<uint32_t>(jj >> 1) & 1u, B)) {
+    const int tt = T + jj;  // the CTA's tile count: buffers and barrier phases
+    if (!warp_wait(smem_u32(&B->s_full[tt & 1]), static_cast<uint32_t>(tt >> 1) & 1u, B)) {
       ok = false;
       break;
     }
@@ -316,8 +376,8 @@ __device__ void run_softmax(const PrefillParams& p, const Work& w, uint32_t tmem
     float s[kH];  // raw scores q.k
     {
       uint32_t v0[32], v1[32];
-      tmem_ld32(lane_base + kColS + (jj & 1) * kPkv + kH * wg, v0);
-      tmem_ld32(lane_base + kColS + (jj & 1) * kPkv + kH * wg + 32, v1);
+      tmem_ld32(lane_base + kColS + (tt & 1) * kPkv + kH * wg, v0);
+      tmem_ld32(lane_base + kColS + (tt & 1) * kPkv + kH * wg + 32, v1);
       tmem_wait_ld();
 #pragma unroll
       for (int i = 0; i < 32; ++i) {
@@ -340,10 +400,10 @@ __device__ void run_softmax(const PrefillParams& p, const Work& w, uint32_t tmem
     for (int i = 8; i < kH; i += 2) mq[(i >> 1) & 7] = max3(mq[(i >> 1) & 7], s[i], s[i + 1]);
     const float mh = max3(max3(mq[0], mq[1], mq[2]), max3(mq[3], mq[4], mq[5]), fmaxf(mq[6], mq[7]));
     // exchange the half-row maxima (every thread arrives; bounded wait)
-    float* slot = red + (jj & 1) * 2 * kRows;
+    float* slot = red + (tt & 1) * 2 * kRows;
     slot[wg * kRows + r] = mh;
-    mbar_arrive(smem_u32(&B->red_full[jj & 1]));
-    if (!warp_wait(smem_u32(&B->red_full[jj & 1]), static_cast<uint32_t>(jj >> 1) & 1u, B)) {
+    mbar_arrive(smem_u32(&B->red_full[tt & 1]));
+    if (!warp_wait(smem_u32(&B->red_full[tt & 1]), static_cast<uint32_t>(tt >> 1) & 1u, B)) {
       ok = false;
       break;
     }
@@ -370,14 +430,15 @@ __device__ void run_softmax(const PrefillParams& p, const Work& w, uint32_t tmem
     }
     const float2 lsum = add2(ls[0], ls[1]);
     l += lsum.x + lsum.y;
-    if (jj > 0) {
-      // P's columns and O are free once the previous tile's PV has completed
-      if (!warp_wait(smem_u32(&B->pv_done), static_cast<uint32_t>(jj - 1) & 1u, B)) {
+    if (tt > 0) {
+      // P's columns (and O) are free once the CTA's previous PV has completed;
+      // the first tile of a unit leaves O alone (its PV overwrites it)
+      if (!warp_wait(smem_u32(&B->pv_done), static_cast<uint32_t>(tt - 1) & 1u, B)) {
         ok = false;
         break;
       }
       tc_fence_after();
-      if (__any_sync(0xffffffffu, need)) {
+      if (jj > 0 && __any_sync(0xffffffffu, need)) {
 #pragma unroll
         for (int c = 0; c < 2; ++c) {
           uint32_t v[32];
@@ -400,37 +461,76 @@ __device__ void run_softmax(const PrefillParams& p, const Work& w, uint32_t tmem
     __syncwarp();
     if (lane == 0) mbar_arrive(smem_u32(&B->p_full));
   }
-  if (ok && !warp_wait(smem_u32(&B->pv_done), static_cast<uint32_t>(w.n - 1) & 1u, B)) ok = false;
-  // both halves of l, through the slot pair the last tile did not use (the
-  // other warpgroup is done reading it); every thread arrives on every path
-  float* lslot = red + (w.n & 1) * 2 * kRows;
+  if (ok && !warp_wait(smem_u32(&B->pv_done), static_cast<uint32_t>(T + w.n - 1) & 1u, B)) ok = false;
+  // both halves of l through their own slots; every thread arrives on every
+  // path (a fast warpgroup writes these slots again only after the next
+  // unit's maximum exchanges, which the slow one joins after reading them)
+  float* lslot = reinterpret_cast<float*>(smem + kOffL);
   lslot[wg * kRows + r] = l;
   mbar_arrive(smem_u32(&B->l_full));
-  if (ok && !warp_wait(smem_u32(&B->l_full), 0, B)) ok = false;
+  if (ok && !warp_wait(smem_u32(&B->l_full), static_cast<uint32_t>(i) & 1u, B)) ok = false;
   l = lslot[r] + lslot[kRows + r];
-  if (!ok) {
-    if (lane == 0) raise_abort(p, B);
-    return;
-  }
+  if (!ok) return false;
   tc_fence_after();
+  // O out of TMEM (complete before this warp's next P store and p_full
+  // arrival, which the next unit's first PV, overwriting O, waits for)
+  uint32_t v0[32], v1[32];
+  tmem_ld32(lane_base + kColO + 64 * wg, v0);
+  tmem_ld32(lane_base + kColO + 64 * wg + 32, v1);
+  tmem_wait_ld();
   // out = O e^(m - M) / (l e^(m - M) + e^(sink - M)), M = max(m, sink), in log2 units
   const float s2 = p.sinks[h] * kPfLog2e;
   const float M = fmaxf(m, s2);
   const float a = (m == -INFINITY) ? 0.f : ex2(m - M);
   const float sc = a / (l * a + ex2(s2 - M));
-  float* out = p.out + (static_cast<long long>(t < p.T ? t : 0) * kHeads + h) * kDim + 64 * wg;
+  // The scaled O goes out through a per-warp staging tile, 16 of this
+  // warpgroup's 64 dims per round: each lane writes its row (16-byte chunks
+  // swizzled by row so that a quarter-warp hits distinct banks), then every
+  // store instruction covers 64 contiguous bytes of 8 rows (rows 8k..8k+7 are
+  // the 8 heads of one token, 512 bytes apart).  Lane-per-row stores would
+  // touch 32 lines per instruction.
+  float* stg = reinterpret_cast<float*>(smem + kOffStage + warp * kStageWarpBytes);
+  const int row0 = (warp & 3) * 32;
 #pragma unroll
-  for (int c = 0; c < 2; ++c) {
-    uint32_t v[32];
-    tmem_ld32(lane_base + kColO + 64 * wg + 32 * c, v);
-    tmem_wait_ld();
-    if (t < p.T) {
+  for (int q = 0; q < 4; ++q) {
 #pragma unroll
-      for (int i = 0; i < 32; i += 4)
-        *reinterpret_cast<float4*>(out + 32 * c + i) =
-            make_float4(__uint_as_float(v[i]) * sc, __uint_as_float(v[i + 1]) * sc,
-                        __uint_as_float(v[i + 2]) * sc, __uint_as_float(v[i + 3]) * sc);
+    for (int i4 = 0; i4 < 4; ++i4) {
+      const int e = (q & 1) * 16 + 4 * i4;
+      const float4 val = q < 2 ? make_float4(__uint_as_float(v0[e]) * sc, __uint_as_float(v0[e + 1]) * sc,
+                                             __uint_as_float(v0[e + 2]) * sc, __uint_as_float(v0[e + 3]) * sc)
+                               : make_float4(__uint_as_float(v1[e]) * sc, __uint_as_float(v1[e + 1]) * sc,
+                                             __uint_as_float(v1[e + 2]) * sc, __uint_as_float(v1[e + 3]) * sc);
+      reinterpret_cast<float4*>(stg + lane * 16)[i4 ^ ((lane >> 1) & 3)] = val;
     }
+    __syncwarp();
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+      const int rw = 8 * k + (lane >> 2), c4 = lane & 3;  // row of the warp, 16-byte chunk
+      const float4 val = reinterpret_cast<const float4*>(stg + rw * 16)[c4 ^ ((rw >> 1) & 3)];
+      const int rr = row0 + rw;
+      const int tr = w.t0 + (rr >> 3);
+      if (tr < p.T)
+        *reinterpret_cast<float4*>(p.out + (static_cast<long long>(tr) * kHeads + w.g * kGroup + (rr & 7)) * kDim +
+                                   64 * wg + 16 * q + 4 * c4) = val;
+    }
+    __syncwarp();
+  }
+  return true;
+}
+
+// The softmax warps over the CTA's units.
+__device__ void run_softmax(const PrefillParams& p, uint32_t tmem, uint8_t* smem, Bars* B, int warp, int lane) {
+  const int units = n_units(p);
+  int T = 0;
+  for (int i = 0;; ++i) {
+    const int u = unit_of(i);
+    if (u >= units) break;
+    const Work w = work_of_unit(p, u);
+    if (!softmax_unit(p, w, i, T, tmem, smem, B, warp, lane)) {
+      if (lane == 0) raise_abort(p, B);
+      return;
+    }
+    T += w.n;
   }
 }
 
@@ -439,10 +539,10 @@ __global__ void __launch_bounds__(kPfThreads, 1) prefill_kernel(const __grid_con
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(pf_raw) + 1023) & ~uintptr_t(1023));
   Bars* B = reinterpret_cast<Bars*>(smem + kOffBar);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const Work w = work_of(p);
 
   if (threadIdx.x == 0) {
     mbar_init(smem_u32(&B->q_full), 1);
+    mbar_init(smem_u32(&B->q_empty), 1);
     for (int s = 0; s < kKs; ++s) {
       mbar_init(smem_u32(&B->k_full[s]), 1);
       mbar_init(smem_u32(&B->k_empty[s]), 1);
@@ -478,13 +578,13 @@ __global__ void __launch_bounds__(kPfThreads, 1) prefill_kernel(const __grid_con
   tc_fence_after();
   const uint32_t tmem = B->tmem_base;
 
-  Issued issued{0, 0};
+  Issued issued{0, 0, 0};
   if (warp < kSoftWarps) {
-    run_softmax(p, w, tmem, smem, B, warp, lane);
+    run_softmax(p, tmem, smem, B, warp, lane);
   } else if (warp == kTmaWarp) {
-    if (lane == 0) issued = run_tma(p, w, smem, B);
+    if (lane == 0) issued = run_tma(p, smem, B);
   } else if (lane == 0) {
-    run_mma(p, w, smem_u32(smem), tmem, B);
+    run_mma(p, smem_u32(smem), tmem, B);
   }
   tc_fence_before();
   __syncthreads();
@@ -507,11 +607,12 @@ extern "C" int flint_test_stall_prefill(int block, int tile) {
 }
 #endif
 
-cudaError_t launch_prefill(const PrefillParams& p, cudaStream_t stream) {
+cudaError_t launch_prefill(const PrefillParams& p, int num_sms, cudaStream_t stream) {
   static ContextSet configured;
   cudaError_t e = configure_once(configured, reinterpret_cast<const void*>(prefill_kernel), static_cast<int>(kPfSmem));
   if (e != cudaSuccess) return e;
-  const int grid = (p.T + kPq - 1) / kPq * kKvHeads;
+  // one persistent CTA per SM (the kernel fills an SM's TMEM), at most one per unit
+  const int grid = std::min((p.T + kPq - 1) / kPq * kKvHeads, num_sms);
   prefill_kernel<<<grid, kPfThreads, kPfSmem, stream>>>(p);
   return cudaGetLastError();
 }

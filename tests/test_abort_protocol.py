@@ -9,9 +9,11 @@ that the next CTA on the SM owns, and a tensor-core MMA still running when
 the TMEM columns are freed would write into another CTA's accumulators.  So
 each kernel ends with a drain: the decode kernel's producer waits (bounded)
 for the phases of the last item inputs and of the last kStages tiles it
-issued; the prefill kernel's producer waits for the K and V phases it
-issued, and its MMA thread waits for a commit that fires once every MMA it
-issued has completed, before TMEM is freed.
+issued; the persistent prefill kernel's producer waits for the last Q, K
+and V phases it issued (a Q tile per unit), and its MMA thread waits for a
+commit that fires once every MMA it issued has completed, before TMEM is
+freed; the prefill norm/RoPE kernel's producer waits for the slots of the
+last tokens it handed out.
 
 The models below replay each kernel's protocol with random interleavings,
 random landing times of the copies and of the tensor pipe, and random
@@ -307,10 +309,17 @@ class Pipe:
             cb()
 
 
-def prefill_run(n, rng, p_timeout, stall_k=None, drain="issued"):
+def prefill_run(units, rng, p_timeout, stall_k=None, drain="issued"):
+    """units: tile counts of the persistent CTA's units (an int: one unit).
+    stall_k: the CTA's K tile (counted across units) the producer never arms.
+    drain: "issued" (the kernel: the last Q, K and V phases the producer
+    issued) or "count" (as if every tile of every unit had been issued)."""
+    if isinstance(units, int):
+        units = [units]
+    n_tiles = sum(units)
     cta = Cta(rng, p_timeout)
     pipe = Pipe(rng)
-    q_full = Bar(1)
+    q_full, q_empty = Bar(1), Bar(1)
     k_full, k_empty = [Bar(1) for _ in range(KS)], [Bar(1) for _ in range(KS)]
     v_full, v_empty = [Bar(1) for _ in range(VS)], [Bar(1) for _ in range(VS)]
     s_full = [Bar(1), Bar(1)]
@@ -318,6 +327,7 @@ def prefill_run(n, rng, p_timeout, stall_k=None, drain="issued"):
     red_full = [Bar(2), Bar(2)]
     l_full = Bar(2)
     k_tag, v_tag = [None] * KS, [None] * VS
+    q_tag = [None]
     res = {}
 
     def load(bar, tags, slot, tile):
@@ -328,55 +338,88 @@ def prefill_run(n, rng, p_timeout, stall_k=None, drain="issued"):
         cta.landing.append((bar, 1, tag))
 
     def tma():
-        nk = nv = 0
-        load(q_full, None, 0, -1)
-        for j in range(n):
-            sk, sv = j % KS, j % VS
-            if j >= KS:
-                ok = yield from cta.wait(k_empty[sk], (j // KS - 1) & 1)
+        nk = nv = nq = 0
+        j = 0
+        for i, n in enumerate(units):
+            if i > 0:
+                ok = yield from cta.wait(q_empty, (i - 1) & 1)
                 if not ok:
                     cta.raise_abort()
-                    res["tma"] = (nk, nv)
+                    res["tma"] = (nk, nv, nq)
                     return
-            if j != stall_k:
-                load(k_full[sk], k_tag, sk, j)
-            nk += 1
-            if j >= VS:
-                ok = yield from cta.wait(v_empty[sv], (j // VS - 1) & 1)
-                if not ok:
-                    cta.raise_abort()
-                    res["tma"] = (nk, nv)
-                    return
-            load(v_full[sv], v_tag, sv, j)
-            nv += 1
-        res["tma"] = (nk, nv)
+            if cta.abort:
+                res["tma"] = (nk, nv, nq)
+                return
+            old = q_tag[0]
+            assert old is None or old["landed"], f"Q of unit {i} issued while unit {i - 1}'s Q is landing"
+            load(q_full, q_tag, 0, i)
+            nq += 1
+            for _ in range(n):
+                sk, sv = j % KS, j % VS
+                if j >= KS:
+                    ok = yield from cta.wait(k_empty[sk], (j // KS - 1) & 1)
+                    if not ok:
+                        cta.raise_abort()
+                        res["tma"] = (nk, nv, nq)
+                        return
+                if j != stall_k:
+                    load(k_full[sk], k_tag, sk, j)
+                nk += 1
+                if j >= VS:
+                    ok = yield from cta.wait(v_empty[sv], (j // VS - 1) & 1)
+                    if not ok:
+                        cta.raise_abort()
+                        res["tma"] = (nk, nv, nq)
+                        return
+                load(v_full[sv], v_tag, sv, j)
+                nv += 1
+                j += 1
+        res["tma"] = (nk, nv, nq)
 
-    def issue_s(j):
+    def issue_s(j, last):
         ok = yield from cta.wait(k_full[j % KS], (j // KS) & 1)
         if not ok:
             return False
         tag = k_tag[j % KS]
         assert tag["tile"] == j and tag["landed"], f"S_{j} issued on a K stage that does not hold tile {j}"
-        pipe.issue(lambda: k_empty[j % KS].arrive(), lambda: s_full[j & 1].arrive())
+        cbs = [lambda: k_empty[j % KS].arrive(), lambda: s_full[j & 1].arrive()]
+        if last:
+            cbs.append(lambda: q_empty.arrive())
+        pipe.issue(*cbs)
         return True
 
     def mma():
+        base = 0
         ok = yield from cta.wait(q_full, 0)
         if ok:
-            ok = yield from issue_s(0)
-        if ok and n > 1:
-            ok = yield from issue_s(1)
-        j = 0
-        while ok and j < n:
-            ok = yield from cta.wait(p_full, j & 1)
-            if ok:
-                ok = yield from cta.wait(v_full[j % VS], (j // VS) & 1)
+            ok = yield from issue_s(0, units[0] == 1)
+        if ok and units[0] > 1:
+            ok = yield from issue_s(1, units[0] == 2)
+        for i, n in enumerate(units):
             if not ok:
                 break
-            pipe.issue(lambda j=j: v_empty[j % VS].arrive(), lambda: pv_done.arrive())
-            if j + 2 < n:
-                ok = yield from issue_s(j + 2)
-            j += 1
+            for jj in range(n):
+                j = base + jj
+                ok = yield from cta.wait(p_full, j & 1)
+                if ok:
+                    ok = yield from cta.wait(v_full[j % VS], (j // VS) & 1)
+                if not ok:
+                    break
+                pipe.issue(lambda j=j: v_empty[j % VS].arrive(), lambda: pv_done.arrive())
+                if jj + 2 < n:
+                    ok = yield from issue_s(j + 2, jj + 2 == n - 1)
+                    if not ok:
+                        break
+            if not ok:
+                break
+            base += n
+            if i + 1 < len(units):
+                nn = units[i + 1]
+                ok = yield from cta.wait(q_full, (i + 1) & 1)
+                if ok:
+                    ok = yield from issue_s(base, nn == 1)
+                if ok and nn > 1:
+                    ok = yield from issue_s(base + 1, nn == 2)
         if not ok:
             cta.raise_abort()
         # commit: fires once every MMA issued so far has completed
@@ -387,26 +430,30 @@ def prefill_run(n, rng, p_timeout, stall_k=None, drain="issued"):
 
     def softmax(wg):
         ok = True
-        for j in range(n):
-            ok = yield from cta.wait(s_full[j & 1], (j >> 1) & 1)
-            if not ok:
-                break
-            red_full[j & 1].arrive()
-            ok = yield from cta.wait(red_full[j & 1], (j >> 1) & 1)
-            if not ok:
-                break
-            if j > 0:
-                ok = yield from cta.wait(pv_done, (j - 1) & 1)
+        j = 0
+        for i, n in enumerate(units):
+            for _ in range(n):
+                ok = yield from cta.wait(s_full[j & 1], (j >> 1) & 1)
                 if not ok:
                     break
-            p_full.arrive()
-        if ok:
-            ok = yield from cta.wait(pv_done, (n - 1) & 1)
-        l_full.arrive()
-        if ok:
-            ok = yield from cta.wait(l_full, 0)
-        if not ok:
-            cta.raise_abort()
+                red_full[j & 1].arrive()
+                ok = yield from cta.wait(red_full[j & 1], (j >> 1) & 1)
+                if not ok:
+                    break
+                if j > 0:
+                    ok = yield from cta.wait(pv_done, (j - 1) & 1)
+                    if not ok:
+                        break
+                p_full.arrive()
+                j += 1
+            if ok:
+                ok = yield from cta.wait(pv_done, (j - 1) & 1)
+            l_full.arrive()
+            if ok:
+                ok = yield from cta.wait(l_full, i & 1)
+            if not ok:
+                cta.raise_abort()
+                return
 
     run_actors(cta, {"tma": tma(), "mma": mma(), "sm0": softmax(0), "sm1": softmax(1)}, pipe)
     # after __syncthreads: the producer drains if the CTA aborted, then TMEM
@@ -422,8 +469,9 @@ def prefill_run(n, rng, p_timeout, stall_k=None, drain="issued"):
             cta.land_one()
 
     if cta.abort:
-        nk, nv = res["tma"] if drain == "issued" else (n, n)
-        bounded(q_full, 0)
+        nk, nv, nq = res["tma"] if drain == "issued" else (n_tiles, n_tiles, len(units))
+        if nq > 0:
+            bounded(q_full, (nq - 1) & 1)
         for j in range(max(0, nk - KS), nk):
             bounded(k_full[j % KS], (j // KS) & 1)
         for j in range(max(0, nv - VS), nv):
@@ -442,22 +490,35 @@ def test_prefill_abort_leaves_nothing_in_flight(n):
         assert (cta.status == 5) == (cta.gave_up > 0)
 
 
+def test_prefill_abort_across_units_leaves_nothing_in_flight():
+    """A persistent CTA's units (Q reloaded per unit): the drain also waits
+    for the last Q it issued."""
+    rng = random.Random(31)
+    for trial in range(400):
+        units = [rng.randint(1, 7) for _ in range(rng.randint(2, 5))]
+        p = rng.choice([0.0, 0.001, 0.01, 0.05, 0.3])
+        cta = prefill_run(units, rng, p)
+        assert cta.in_flight_at_exit == 0, f"trial {trial}: a copy is in flight at exit ({units}, p={p})"
+        assert (cta.status == 5) == (cta.gave_up > 0)
+
+
 def test_prefill_stalled_k_stage_times_out_and_drains():
     rng = random.Random(11)
     for trial in range(300):
-        n = rng.randint(1, 12)
-        cta = prefill_run(n, rng, 0.0005, stall_k=rng.randrange(n))
+        units = [rng.randint(1, 8) for _ in range(rng.randint(1, 3))]
+        cta = prefill_run(units, rng, 0.0005, stall_k=rng.randrange(sum(units)))
         assert cta.status == 5 and cta.in_flight_at_exit == 0, f"trial {trial}"
 
 
 def test_prefill_drain_keyed_on_the_tile_count_is_caught():
-    """A drain over the last phases of all n tiles, as if every tile had been
+    """A drain over the last phases of all tiles, as if every tile had been
     issued, passes parity waits on older phases while an issued copy is still
     landing when the producer gave up early."""
     rng = random.Random(12)
     caught = 0
     for trial in range(600):
-        cta = prefill_run(rng.randint(6, 12), rng, 0.05, drain="count")
+        units = [rng.randint(3, 8) for _ in range(rng.randint(1, 3))]
+        cta = prefill_run(units, rng, 0.05, drain="count")
         caught += cta.in_flight_at_exit > 0
     assert caught > 0
 

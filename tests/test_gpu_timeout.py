@@ -116,8 +116,14 @@ def test_decode_full_layer_stalled_stage_times_out_then_recovers(hooks):
     parity(out.cpu().numpy()[0], want, "full layer after a time-out")
 
 
-def test_prefill_stalled_k_tile_times_out_then_recovers(hooks):
-    T = 300
+@pytest.mark.parametrize("T,block,tile", [(300, 0, 1), (1000, 147, 5)])
+def test_prefill_stalled_k_tile_times_out_then_recovers(hooks, T, block, tile):
+    """(300, 0, 1): block 0 holds the last 16 query tokens, three K tiles, and
+    the second never arrives.  (1000, 147, 5): 252 units on 148 persistent
+    CTAs; CTA 147 walks units 147 and 148 (4 tiles each), and its tile 5, in
+    the second unit, never arrives (the CTA has reloaded Q by then)."""
+    if torch.cuda.get_device_properties(0).multi_processor_count != 148 and block != 0:
+        pytest.skip("the unit deal of this case assumes 148 SMs")
     p = I.make_prefill(T, 0, workload=I.W_PREFILL + 30)
     want, qb, kb = oracle.prefill(I.bits(p.q_raw), I.bits(p.k_raw), I.bits(p.v_raw), I.bits(p.w_q),
                                   I.bits(p.w_k), p.sinks.numpy().astype(np.float64), 0, p.rope,
@@ -133,8 +139,7 @@ def test_prefill_stalled_k_tile_times_out_then_recovers(hooks):
         flint.flint_prefill_attn(q, k, v16, sinks, 0, out, dev_err=err)
         torch.cuda.synchronize()
         assert int(err.item()) == 0
-        # block 0 holds the last 16 query tokens: three K tiles; the second never arrives
-        assert hooks.flint_test_stall_prefill(0, 1) == 0
+        assert hooks.flint_test_stall_prefill(block, tile) == 0
         dt = timed(lambda: flint.flint_prefill_attn(q, k, v16, sinks, 0, out, dev_err=err))
         assert int(err.item()) == flint.FLINT_ERR_TIMEOUT
         assert dt < 6 * LIMIT_S + 0.25, f"the timed-out call took {dt:.3f} s"
