@@ -146,6 +146,25 @@ __device__ __forceinline__ float ex2(float x) {
   return y;
 }
 
+// 2^x for a pair on the FMA pipe, for x <= 2^8 (the softmax's exponents):
+// x = j + f with j = rint(x) (x + 1.5 * 2^23 puts rint(x) in the low bits)
+// and f in [-1/2, 1/2]; 2^f is the degree-4 polynomial interpolating 2^f at
+// the five Chebyshev nodes of [-1/2, 1/2] (relative error below 3.6e-6 with
+// float coefficients); j joins the exponent field by an integer add.  x is
+// clamped at -127 so that the add stays in range (results below 2^-126 come
+// out as 0 or tiny values, which the fp16 P rounds to 0).
+__device__ __forceinline__ float2 ex2_fma2(float2 x) {
+  x = make_float2(fmaxf(x.x, -127.0f), fmaxf(x.y, -127.0f));
+  const float2 t = add2(x, make_float2(12582912.0f, 12582912.0f));
+  const float2 f = fma2(add2(t, make_float2(-12582912.0f, -12582912.0f)), make_float2(-1.0f, -1.0f), x);
+  float2 q = fma2(make_float2(0x1.3cbf6p-7f, 0x1.3cbf6p-7f), f, make_float2(0x1.ca1ce2p-5f, 0x1.ca1ce2p-5f));
+  q = fma2(q, f, make_float2(0x1.ebfa4cp-3f, 0x1.ebfa4cp-3f));
+  q = fma2(q, f, make_float2(0x1.62e0c2p-1f, 0x1.62e0c2p-1f));
+  q = fma2(q, f, make_float2(1.0f, 1.0f));
+  return make_float2(__int_as_float(__float_as_int(q.x) + (__float_as_int(t.x) << 23)),
+                     __int_as_float(__float_as_int(q.y) + (__float_as_int(t.y) << 23)));
+}
+
 // Bounded wait shared by all lanes of a warp: true only if every lane saw
 // the phase complete.
 __device__ __forceinline__ bool warp_wait(uint32_t bar, uint32_t parity, Bars* B) {
@@ -423,7 +442,8 @@ __device__ bool softmax_unit(const PrefillParams& p, const Work& w, int i, int T
 #pragma unroll
     for (int c = 0; c < kH / 2; ++c) {
       const float2 x = fma2(make_float2(s[2 * c], s[2 * c + 1]), scale2, nmu2);
-      const float2 pp = make_float2(ex2(x.x), ex2(x.y));
+      // one pair in four on the FMA pipe: the MUFU unit bounds this loop
+      const float2 pp = (c & 3) == 3 ? ex2_fma2(x) : make_float2(ex2(x.x), ex2(x.y));
       ls[c & 1] = add2(ls[c & 1], pp);
       const __half2 hp = __floats2half2_rn(pp.x, pp.y);
       pk[c] = *reinterpret_cast<const uint32_t*>(&hp);
@@ -599,6 +619,29 @@ __global__ void __launch_bounds__(kPfThreads, 1) prefill_kernel(const __grid_con
 }  // namespace
 
 #ifdef FLINT_TEST_HOOKS
+// Test builds only: both exponentials of the softmax, ex2_fma2 (pairs x[2i],
+// x[2i+1]; a last odd element paired with itself) and ex2.approx, of n values
+// (device pointers), for the comparison in the tests.
+__global__ void ex2_probe_kernel(const float* x, float* y_fma, float* y_mufu, int n) {
+  const int i = 2 * (blockIdx.x * blockDim.x + threadIdx.x);
+  if (i < n) {
+    const float a = x[i], b = i + 1 < n ? x[i + 1] : a;
+    const float2 y = ex2_fma2(make_float2(a, b));
+    y_fma[i] = y.x;
+    y_mufu[i] = ex2(a);
+    if (i + 1 < n) {
+      y_fma[i + 1] = y.y;
+      y_mufu[i + 1] = ex2(b);
+    }
+  }
+}
+extern "C" int flint_test_ex2(const float* x, float* y_fma, float* y_mufu, int n, void* stream) {
+  if (n < 1) return static_cast<int>(cudaErrorInvalidValue);
+  const int pairs = (n + 1) / 2;
+  ex2_probe_kernel<<<(pairs + 255) / 256, 256, 0, static_cast<cudaStream_t>(stream)>>>(x, y_fma, y_mufu, n);
+  return static_cast<int>(cudaGetLastError());
+}
+
 // Test builds only: CTA `block` leaves its K tile `tile` unarmed; block = -1
 // turns the hook off.
 extern "C" int flint_test_stall_prefill(int block, int tile) {

@@ -112,6 +112,9 @@ def open_library(path: str) -> ctypes.CDLL:
         if hasattr(lib, name):
             getattr(lib, name).argtypes = [ctypes.c_int, ctypes.c_int]
             getattr(lib, name).restype = ctypes.c_int
+    if hasattr(lib, "flint_test_ex2"):  # the prefill softmax's two exponentials, side by side
+        lib.flint_test_ex2.argtypes = [P, P, P, I32, P]
+        lib.flint_test_ex2.restype = ctypes.c_int
     return lib
 
 
