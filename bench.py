@@ -38,17 +38,20 @@ NOMINAL_HBM_GBS = 8000.0
 # launch duration, --clock-control none, one launch after the warm-up) of each
 # workload, per KV dtype, with the hash of the decode kernel's sources
 # (DECODE_SOURCES below) it was taken on; reported only while they still hash
-# the same.  The captures were taken on the whole-source hash f0faa7f388d2e1d4.
-TRAFFIC = {("stack", 100_000, "bf16"): (2_905_866_240 + 7_171_584, "b851b12eb2899e83"),
-           ("stack", 100_000, "fp8"): (1_453_846_016 + 6_466_560, "b851b12eb2899e83"),
-           ("full100k", 100_000, "bf16"): (204_910_592 + 3_482_368, "b851b12eb2899e83"),
-           ("full2k", 2048, "bf16"): (4_285_696 + 0, "b851b12eb2899e83"),
-           ("swa100k", 100_000, "bf16"): (1_143_552 + 0, "b851b12eb2899e83"),
-           ("paged32", 100_000, "bf16"): (2_271_119_872 + 6_297_600, "b851b12eb2899e83"),
-           ("paged32swa", 100_000, "bf16"): (36_023_296 + 46_336, "b851b12eb2899e83")}
+# the same.  The captures were taken on the whole-source hash 1af5b5b43635a6e3.
+TRAFFIC = {("stack", 100_000, "bf16"): (2_905_832_704 + 6_969_856, "3cc341f5f71e2a22"),
+           ("stack", 100_000, "fp8"): (1_453_909_504 + 6_871_552, "3cc341f5f71e2a22"),
+           ("full100k", 100_000, "bf16"): (204_902_656 + 3_548_160, "3cc341f5f71e2a22"),
+           ("full2k", 2048, "bf16"): (4_284_928 + 0, "3cc341f5f71e2a22"),
+           ("swa100k", 100_000, "bf16"): (1_143_808 + 0, "3cc341f5f71e2a22"),
+           ("paged32", 100_000, "bf16"): (2_271_113_984 + 7_415_296, "3cc341f5f71e2a22"),
+           ("paged32swa", 100_000, "bf16"): (36_024_320 + 13_568, "3cc341f5f71e2a22")}
 # The same for one prefill_kernel launch of a full (NoPE) layer on the
 # 8,192-token prompt (a --set full capture of that one launch).
-PREFILL_TRAFFIC = {8192: (83_963_648 + 80_508_928, "38ee5c4a48fcdd23")}
+PREFILL_TRAFFIC = {8192: (83_945_984 + 85_460_224, "52715e9f20e45c9f")}
+# The same for one prefill_prep_kernel launch of a full layer on the
+# 8,192-token prompt (one pass: the metrics above), keyed on PREP_SOURCES.
+PREP_TRAFFIC = {8192: (83_907_840 + 43_450_112, "46ca36dffb635fd5")}
 
 
 def max_over_ranks(x: float, world: int, device) -> float:
@@ -75,6 +78,8 @@ DECODE_SOURCES = ("csrc/flint_decode.cu", "csrc/flint_device.cuh", "csrc/flint_i
                   "csrc/flint_abi.cu", "csrc/flint_plan.cpp")
 PREFILL_SOURCES = ("csrc/flint_prefill.cu", "csrc/flint_device.cuh", "csrc/flint_internal.h",
                    "csrc/flint_abi.cu")
+PREP_SOURCES = ("csrc/flint_prefill_prep.cu", "csrc/flint_device.cuh", "csrc/flint_internal.h",
+                "csrc/flint_abi.cu")
 
 
 def kernel_sources_hash(files=None) -> str:
@@ -103,6 +108,11 @@ def traffic_for(workload: str, ctx: int, kv: str = "bf16"):
 def prefill_traffic(T: int):
     t = PREFILL_TRAFFIC.get(T)
     return t[0] if t is not None and t[1] == kernel_sources_hash(PREFILL_SOURCES) else None
+
+
+def prep_traffic(T: int):
+    t = PREP_TRAFFIC.get(T)
+    return t[0] if t is not None and t[1] == kernel_sources_hash(PREP_SOURCES) else None
 FALLBACK_HBM_GBS = 6650.0
 FALLBACK_BF16_TFLOPS = 1400.0   # sustained, under the power cap
 
@@ -531,6 +541,7 @@ def run_prefill(args, rank, world, local):
             "window_layer_us": statistics.mean(prep_layer_ms[i] for i, f in enumerate(kinds) if not f) * 1e3,
             "algorithmic_bytes_per_prompt": int(prep_bytes), "achieved": prep_gbs, "peak": hbm_peak,
             "unit": "GB/s", "frac": prep_gbs / hbm_peak, "peak_kind": hbm_kind,
+            "traffic": prep_traffic(T), "traffic_launch": "one full-layer launch (cold; writes still in L2 not counted)",
             "note": "events around each launch; the previous layer's attention output (134 MB fp32) "
                     "is still being written back from L2 when it starts"}
     line = {
