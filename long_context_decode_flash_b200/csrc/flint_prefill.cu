@@ -8,13 +8,16 @@
 // ("Day-0 Support for Flint on vLLM", hnkhoi.com, "Model architecture"; the
 // 8,192-token prefill of newruntime.com, "What happened").
 //
-// How (5th-generation tensor cores, tcgen05): one CTA per (block of 16 query
-// tokens, KV head g).  Its 128 query rows are the 16 tokens x the 8 heads of
-// the group (row r = 8 * token + head), so every K/V tile serves all 8 heads.
-// Ten warps:
-//   warp 8     TMA producer: the Q tile once, then 128-key K and V tiles
-//              through 3- and 2-stage rings (128-byte swizzle, two 64-dim
-//              boxes per tile).
+// How (5th-generation tensor cores, tcgen05): the work is split into units
+// (block of 16 query tokens, KV head g); a unit's 128 query rows are the 16
+// tokens x the 8 heads of the group (row r = 8 * token + head), so every K/V
+// tile serves all 8 heads.  The kernel is persistent: one CTA per SM (its 512
+// TMEM columns fill the SM) walks its share of the units, dealt longest first
+// in rounds of alternating direction; tiles, ring stages and barrier phases
+// are counted across the CTA's units.  Ten warps:
+//   warp 8     TMA producer: per unit the Q tile (once the previous unit's S
+//              MMAs are done with it), then 128-key K and V tiles through 3-
+//              and 2-stage rings (128-byte swizzle, two 64-dim boxes a tile).
 //   warp 9     allocates the 512 TMEM columns; its lane 0 issues the MMAs:
 //              S = Q K^T (bf16, M 128, N 128, K 128) into one of two TMEM S
 //              buffers, and O += P V (fp16, K 128) with P read from TMEM and V
@@ -26,8 +29,8 @@
 //              exchanged between the two warpgroups through shared memory, an
 //              fp32 online softmax in log2 units whose running maximum moves
 //              only when a tile exceeds it by more than 2^8 (then O is
-//              rescaled in TMEM), P back to TMEM; at the end O, the sink and
-//              the store.
+//              rescaled in TMEM), P back to TMEM; at the end of a unit O, the
+//              sink and the store through a per-warp staging tile.
 // P is rounded to fp16 (P <= 2^8 under the lazy maximum, relative error
 // 2^-12) and V arrives in fp16 (exact for bf16 values in the fp16 normal
 // range), so one PV product keeps the output within a few 1e-4 of the exact

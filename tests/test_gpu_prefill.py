@@ -272,3 +272,64 @@ def test_decode_continues_from_the_prefilled_cache(window):
                               p.rope, layout=layout, capacity=cap)
     parity(out.cpu().numpy()[0], dec, "decode after prefill")
 
+
+
+def _sms():
+    return torch.cuda.get_device_properties(0).multi_processor_count
+
+
+@pytest.mark.parametrize("which", ["1", "2", "g-1", "g", "g+1", "2g+1"])
+def test_prefill_prep_at_the_grid_boundaries(which):
+    """The norm/RoPE pass runs a persistent grid of g = 3 x SMs CTAs, each
+    over a contiguous share of the tokens: prompts with fewer tokens than
+    CTAs, exactly one token per CTA, and one more than that.  q and k are
+    within one bf16 ulp of the oracle's, v converts bit for bit, and every
+    cached row is the call's own k and raw v."""
+    g = 3 * _sms()
+    T = {"1": 1, "2": 2, "g-1": g - 1, "g": g, "g+1": g + 1, "2g+1": 2 * g + 1}[which]
+    p = I.make_prefill(T, flint.WINDOW, workload=W_PF + 40)
+    d = Dev(p)
+    kc = torch.zeros((T + 3, 4, 128), dtype=torch.bfloat16, device="cuda")
+    vc = torch.zeros_like(kc)
+    cache = flint.kv_cache(kc, vc, flint.CONTIGUOUS, capacity=T + 3)
+    q, k, v = prep_gpu(d, cache=cache, with_v=True)
+    _, qb, kb = oracle_prefill(p, rows=[])
+    close_bits(u16(q), qb, "q")
+    close_bits(u16(k), kb, "k")
+    np.testing.assert_array_equal(u16(v), u16(p.v_raw.to(torch.float16)))
+    np.testing.assert_array_equal(u16(kc)[:T], u16(k))
+    np.testing.assert_array_equal(u16(vc)[:T], I.bits(p.v_raw))
+    assert not u16(kc)[T:].any() and not u16(vc)[T:].any()  # no write past the prompt
+
+
+@pytest.mark.parametrize("case", ["one unit per CTA", "four CTAs with two units"])
+@pytest.mark.parametrize("window", [flint.WINDOW, 0])
+def test_prefill_attention_every_row_at_the_unit_deal(case, window):
+    """The attention's persistent grid has one CTA per SM, each over units of
+    16 query tokens x one KV head: T = 4 x SMs gives one unit per CTA, and 16
+    more tokens give four CTAs a second unit.  Every row against the oracle,
+    from its own q and k bits."""
+    T = 4 * _sms() + (16 if case.startswith("four") else 0)
+    p = I.make_prefill(T, window, workload=W_PF + 41)
+    want, qb, kb = oracle_prefill(p, rows=range(T))
+    q = dev(torch.from_numpy(qb.view(np.int16)).view(torch.bfloat16))
+    k = dev(torch.from_numpy(kb.view(np.int16)).view(torch.bfloat16))
+    got = attn_gpu(q, k, f16(p.v_raw), dev(p.sinks), window)
+    parity(got, want, f"T={T} window={window}")
+
+
+@pytest.mark.parametrize("window", [flint.WINDOW, 0])
+def test_prefill_attention_over_several_rounds_of_units(window):
+    """T = 12 x SMs + 16: every CTA walks three or four units, dealt in
+    rounds of alternating direction; rows at the edges of 16-token units and
+    of 128-key tiles, and a random draw, against the oracle."""
+    T = 12 * _sms() + 16
+    p = I.make_prefill(T, window, workload=W_PF + 42)
+    edges = [0, 1, 15, 16, 17, 127, 128, 129, 511, 512, 513, 514, T // 2, T - 17, T - 16, T - 1]
+    rng = np.random.default_rng(7)
+    rows = sorted({r for r in edges + rng.choice(T, size=24, replace=False).tolist() if 0 <= r < T})
+    want, qb, kb = oracle_prefill(p, rows=rows)
+    q = dev(torch.from_numpy(qb.view(np.int16)).view(torch.bfloat16))
+    k = dev(torch.from_numpy(kb.view(np.int16)).view(torch.bfloat16))
+    got = attn_gpu(q, k, f16(p.v_raw), dev(p.sinks), window)
+    parity(got[rows], want, f"T={T} window={window}")
