@@ -48,7 +48,7 @@ TRAFFIC = {("stack", 100_000, "bf16"): (2_905_832_704 + 6_969_856, "3cc341f5f71e
            ("paged32swa", 100_000, "bf16"): (36_024_320 + 13_568, "3cc341f5f71e2a22")}
 # The same for one prefill_kernel launch of a full (NoPE) layer on the
 # 8,192-token prompt (a --set full capture of that one launch).
-PREFILL_TRAFFIC = {8192: (83_945_984 + 85_460_224, "52715e9f20e45c9f")}
+PREFILL_TRAFFIC = {8192: (83_945_472 + 84_220_928, "5d5bf132b6f67c8e")}
 # The same for one prefill_prep_kernel launch of a full layer on the
 # 8,192-token prompt (one pass: the metrics above), keyed on PREP_SOURCES.
 PREP_TRAFFIC = {8192: (83_907_840 + 43_450_112, "46ca36dffb635fd5")}
