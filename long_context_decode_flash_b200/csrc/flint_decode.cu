@@ -72,6 +72,14 @@ __device__ int g_stall_decode[2] = {-1, -1};
 
 namespace {
 
+// 2^x from the hardware unit (ex2.approx.ftz: ~2^-22 relative error, results
+// below 2^-126 flushed to 0, which a softmax sum cannot tell apart).
+__device__ __forceinline__ float ex2_approx(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+
 constexpr float kLog2e = 1.4426950408889634f;
 // log2(e) / sqrt(128): scores come out of the tensor cores in log2 units.
 constexpr float kQScale = static_cast<float>(1.4426950408889634 * 0.08838834764831845);
@@ -490,7 +498,7 @@ __device__ __forceinline__ void consume_slice(uint32_t sK, uint32_t sV, int tok0
   // slack (always on its first valid tile); the branch is warp-uniform.
   const bool grow = mx > m_run + kRescaleSlack;
   if (__any_sync(0xffffffffu, grow)) {
-    const float alpha = grow ? exp2f(m_run - mx) : 1.0f;
+    const float alpha = grow ? ex2_approx(m_run - mx) : 1.0f;
     l_run *= alpha;
 #pragma unroll
     for (int n = 0; n < 16; ++n)
@@ -501,8 +509,8 @@ __device__ __forceinline__ void consume_slice(uint32_t sK, uint32_t sV, int tok0
   const float mu = (m_run == -INFINITY) ? 0.f : m_run;
 
   // P = 2^(s - m) split into the bf16 hi/lo rows of the A operand.
-  const float p0 = exp2f(sc[0] - mu), p1 = exp2f(sc[1] - mu);
-  const float p2 = exp2f(sc[2] - mu), p3 = exp2f(sc[3] - mu);
+  const float p0 = ex2_approx(sc[0] - mu), p1 = ex2_approx(sc[1] - mu);
+  const float p2 = ex2_approx(sc[2] - mu), p3 = ex2_approx(sc[3] - mu);
   l_run += (p0 + p1) + (p2 + p3);
   uint32_t pa[4];
   split_bf16x2(p0, p1, pa[0], pa[1]);
@@ -594,7 +602,7 @@ __device__ __forceinline__ void consume_block32_fp8(uint32_t sK, uint32_t sV, in
   mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 2));
   const bool grow = mx > m_run + kRescaleSlack;
   if (__any_sync(0xffffffffu, grow)) {
-    const float alpha = grow ? exp2f(m_run - mx) : 1.0f;
+    const float alpha = grow ? ex2_approx(m_run - mx) : 1.0f;
     l_run *= alpha;
 #pragma unroll
     for (int n = 0; n < 16; ++n)
@@ -606,7 +614,7 @@ __device__ __forceinline__ void consume_block32_fp8(uint32_t sK, uint32_t sV, in
 
   float p[8];
 #pragma unroll
-  for (int i = 0; i < 8; ++i) p[i] = exp2f(sc[i] - mu);
+  for (int i = 0; i < 8; ++i) p[i] = ex2_approx(sc[i] - mu);
   l_run += ((p[0] + p[1]) + (p[2] + p[3])) + ((p[4] + p[5]) + (p[6] + p[7]));
   uint32_t pa[2][4];  // k-steps of 16 tokens
 #pragma unroll
