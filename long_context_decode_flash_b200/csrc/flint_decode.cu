@@ -584,8 +584,12 @@ __device__ __forceinline__ void consume_block32_fp8(uint32_t sK, uint32_t sV, in
           mma_f16_16816(a0, qa[kk + i], b0, b1);
       }
     }
-    sc[2 * jj] = ((a0[0] + a1[0]) + (a0[2] + a1[2])) * k_scale;
-    sc[2 * jj + 1] = ((a0[1] + a1[1]) + (a0[3] + a1[3])) * k_scale;
+    // rows g (q hi) and g + 8 (q lo) of both accumulators, two tokens at a time
+    const float2 t = add2(add2(make_float2(a0[0], a0[1]), make_float2(a1[0], a1[1])),
+                          add2(make_float2(a0[2], a0[3]), make_float2(a1[2], a1[3])));
+    const float2 st = mul2(t, make_float2(k_scale, k_scale));
+    sc[2 * jj] = st.x;
+    sc[2 * jj + 1] = st.y;
   }
   if (!whole) {
 #pragma unroll
@@ -613,9 +617,18 @@ __device__ __forceinline__ void consume_block32_fp8(uint32_t sK, uint32_t sV, in
   const float mu = (m_run == -INFINITY) ? 0.f : m_run;
 
   float p[8];
+  const float2 nmu = make_float2(-mu, -mu);
 #pragma unroll
-  for (int i = 0; i < 8; ++i) p[i] = ex2_approx(sc[i] - mu);
-  l_run += ((p[0] + p[1]) + (p[2] + p[3])) + ((p[4] + p[5]) + (p[6] + p[7]));
+  for (int i = 0; i < 8; i += 2) {
+    const float2 x = add2(make_float2(sc[i], sc[i + 1]), nmu);
+    p[i] = ex2_approx(x.x);
+    p[i + 1] = ex2_approx(x.y);
+  }
+  {
+    const float2 s01 = add2(add2(make_float2(p[0], p[1]), make_float2(p[2], p[3])),
+                            add2(make_float2(p[4], p[5]), make_float2(p[6], p[7])));
+    l_run += s01.x + s01.y;
+  }
   uint32_t pa[2][4];  // k-steps of 16 tokens
 #pragma unroll
   for (int s2 = 0; s2 < 2; ++s2) {
