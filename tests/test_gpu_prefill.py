@@ -333,3 +333,44 @@ def test_prefill_attention_over_several_rounds_of_units(window):
     k = dev(torch.from_numpy(kb.view(np.int16)).view(torch.bfloat16))
     got = attn_gpu(q, k, f16(p.v_raw), dev(p.sinks), window)
     parity(got[rows], want, f"T={T} window={window}")
+
+
+@pytest.mark.parametrize("outputs", ["cache only", "q only", "k only", "q and v", "k, v and cache, no q"])
+@pytest.mark.parametrize("rope", [True, False])
+def test_prefill_prep_with_a_subset_of_the_outputs(outputs, rope):
+    """Each output of the norm/RoPE pass is optional; the kernel stages only
+    the rows the call needs (q for q_out, k for k_out or a cache, v for v_out
+    or a cache) and expects exactly their bytes.  Every subset must finish
+    without a device error and give the same bits as the call with every
+    output."""
+    T = 700
+    window = flint.WINDOW if rope else 0
+    p = I.make_prefill(T, window, workload=W_PF + 43)
+    d = Dev(p)
+    q_ref, k_ref, v_ref = prep_gpu(d, with_v=True)
+    want = {"q": u16(q_ref), "k": u16(k_ref), "v": u16(v_ref)}
+    use = {"cache only": {"cache"}, "q only": {"q"}, "k only": {"k"}, "q and v": {"q", "v"},
+           "k, v and cache, no q": {"k", "v", "cache"}}[outputs]
+    q = torch.full((T, 32, 128), float("nan"), dtype=torch.bfloat16, device="cuda") if "q" in use else None
+    k = torch.full((T, 4, 128), float("nan"), dtype=torch.bfloat16, device="cuda") if "k" in use else None
+    v = torch.full((T, 4, 128), float("nan"), dtype=torch.float16, device="cuda") if "v" in use else None
+    cache = None
+    if "cache" in use:
+        kc = torch.zeros((T, 4, 128), dtype=torch.bfloat16, device="cuda")
+        vc = torch.zeros_like(kc)
+        cache = flint.kv_cache(kc, vc, flint.CONTIGUOUS, capacity=T)
+    needs_v = v is not None or cache is not None
+    err = torch.zeros(1, dtype=torch.int32, device="cuda")
+    flint.flint_prefill_qk_norm_rope(d.q_raw, d.k_raw, d.w_q, d.w_k, apply_rope=d.rope, q_out=q, k_out=k,
+                                     v_raw=d.v_raw if needs_v else None, v_out=v, cache=cache, dev_err=err)
+    torch.cuda.synchronize()
+    assert int(err.item()) == 0
+    if q is not None:
+        np.testing.assert_array_equal(u16(q), want["q"])
+    if k is not None:
+        np.testing.assert_array_equal(u16(k), want["k"])
+    if v is not None:
+        np.testing.assert_array_equal(u16(v), want["v"])
+    if cache is not None:
+        np.testing.assert_array_equal(u16(kc), want["k"])
+        np.testing.assert_array_equal(u16(vc), I.bits(p.v_raw))
