@@ -38,14 +38,14 @@ NOMINAL_HBM_GBS = 8000.0
 # launch duration, --clock-control none, one launch after the warm-up) of each
 # workload, per KV dtype, with the hash of the decode kernel's sources
 # (DECODE_SOURCES below) it was taken on; reported only while they still hash
-# the same.  The captures were taken on the whole-source hash 4d785bdb2021fefa.
-TRAFFIC = {("stack", 100_000, "bf16"): (2_905_920_256 + 7_245_824, "dc1731a105ec56a1"),
-           ("stack", 100_000, "fp8"): (1_453_917_696 + 6_590_720, "dc1731a105ec56a1"),
-           ("full100k", 100_000, "bf16"): (204_907_008 + 3_603_456, "dc1731a105ec56a1"),
-           ("full2k", 2048, "bf16"): (4_283_648 + 0, "dc1731a105ec56a1"),
-           ("swa100k", 100_000, "bf16"): (1_142_016 + 0, "dc1731a105ec56a1"),
-           ("paged32", 100_000, "bf16"): (2_271_163_904 + 6_551_040, "dc1731a105ec56a1"),
-           ("paged32swa", 100_000, "bf16"): (36_022_272 + 60_160, "dc1731a105ec56a1")}
+# the same.  The captures were taken on the whole-source hash 1ab6844e5d63414e.
+TRAFFIC = {("stack", 100_000, "bf16"): (2_905_857_024 + 7_194_624, "8e3306ca89b8190c"),
+           ("stack", 100_000, "fp8"): (1_453_875_456 + 6_482_688, "8e3306ca89b8190c"),
+           ("full100k", 100_000, "bf16"): (204_924_416 + 3_562_240, "8e3306ca89b8190c"),
+           ("full2k", 2048, "bf16"): (4_283_392 + 0, "8e3306ca89b8190c"),
+           ("swa100k", 100_000, "bf16"): (1_140_992 + 0, "8e3306ca89b8190c"),
+           ("paged32", 100_000, "bf16"): (2_271_121_664 + 7_319_040, "8e3306ca89b8190c"),
+           ("paged32swa", 100_000, "bf16"): (36_022_528 + 18_688, "8e3306ca89b8190c")}
 # The same for one prefill_kernel launch of a full (NoPE) layer on the
 # 8,192-token prompt (a --set full capture of that one launch).
 PREFILL_TRAFFIC = {8192: (83_945_472 + 84_220_928, "5d5bf132b6f67c8e")}
