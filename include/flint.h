@@ -180,9 +180,11 @@ flint_status flint_kv_append(const uint16_t* k, const uint16_t* v, const int32_t
  * runs with less, down to 4096 + (CTAs + n_problems) * 16640 bytes, with a
  * coarser run-time balancing queue; below that it returns
  * FLINT_ERR_WORKSPACE.  The workspace holds split partials, per-problem
- * arrival counters, a grid-barrier word and the queue head; it must be
+ * arrival counters, a grid-barrier word, the merge-ticket word (whose upper
+ * bits count launches), per-partial ready flags and the queue head; it must be
  * zero-filled before its first use, and every call that completes without a
- * device error leaves it ready for the next call (counters back at zero).
+ * device error leaves it ready for the next call (arrival counters and queue
+ * head back at zero, flags tagged with the launch count).
  * After a device error, zero it again.  Calls that share a workspace must not
  * overlap in time.  Returns 0 for invalid arguments. */
 size_t flint_attn_workspace_bytes(int32_t n_problems, int32_t num_ctas);

@@ -41,9 +41,6 @@ flint_status ok() {
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
 constexpr int kItemCost = 2;  // per-item overhead in tile units (planner cost model)
-// A deferred problem with more partials than this is merged a CTA per unit
-// (thread per partial) instead of a warp per unit (lane per partial).
-constexpr int kWideMergeItems = 96;
 
 // ---- device properties (cached per device) --------------------------------
 
@@ -248,7 +245,7 @@ flint_status plan(DecodeParams& P, const int* tiles, int n_problems, int num_cta
   int sms = num_ctas;
   if (sms == 0 && device_num_sms(&sms) != 0)
     return fail(FLINT_ERR_CUDA, "cannot query the SM count of the current device");
-  // One CTA fits an SM, and a launch that ends in a grid barrier needs all of
+  // One CTA fits an SM, and a launch whose merging CTAs wait for the others needs all of
   // them resident: never more CTAs than the device has SMs.
   int dev_sms = 0;
   if (num_ctas > 0 && device_num_sms(&dev_sms) == 0) sms = std::min(sms, dev_sms);
@@ -292,21 +289,36 @@ flint_status plan(DecodeParams& P, const int* tiles, int n_problems, int num_cta
     P.seg_item_begin[s] = static_cast<int16_t>(i);
   }
   // Problems with queued chunks, or split more widely than kInlineMergeMax,
-  // are merged by the whole grid after the grid barrier: their last items
-  // finish near the end of the launch, where one CTA merging alone would be
-  // the tail.
+  // are merged at the launch's end by the CTAs that finish streaming first,
+  // as their items' flags come up: their last items finish near the end of
+  // the launch, where one CTA merging alone would be the tail.
   P.n_deferred = 0;
   P.n_wide = 0;
+  // When a CTA per unit covers every unit of every deferred problem at once
+  // (a lone problem on a short context), every problem is merged that way:
+  // each warp then folds a ninth of the partials.
+  int n_def = 0;
+  for (int s = 0; s < n_segs; ++s)
+    n_def += (queued[s] || P.seg_item_begin[s + 1] - P.seg_item_begin[s] > kInlineMergeMax) ? 1 : 0;
+  const bool one_round = n_def * kKvHeads * 8 <= G;
   for (int wide = 1; wide >= 0; --wide) {
     for (int s = 0; s < n_segs; ++s) {
       const int items = P.seg_item_begin[s + 1] - P.seg_item_begin[s];
       const bool deferred = queued[s] || items > kInlineMergeMax;
       P.prob[s].deferred = deferred ? 1 : 0;
-      if (deferred && (items > kWideMergeItems) == (wide == 1)) P.deferred[P.n_deferred++] = static_cast<int16_t>(s);
+      if (deferred && (items > kWideMergeItems || one_round) == (wide == 1)) P.deferred[P.n_deferred++] = static_cast<int16_t>(s);
     }
     if (wide) P.n_wide = P.n_deferred;
   }
+  for (int w = 0; w < kMaxItems / 32; ++w) P.raised[w] = 0;
+  for (int i = 0; i < n; ++i)
+    if (P.prob[seg[i]].deferred) P.raised[i / 32] |= 1u << (i % 32);
   P.grid_merge = (P.n_deferred > 0 || P.n_queue > 0) ? 1 : 0;
+  // Ready flags where a problem is split over very many items (a lone long
+  // context over every SM), the grid barrier otherwise.
+  P.merge_flags = 0;
+  for (int s = 0; s < n_segs; ++s)
+    if (P.seg_item_begin[s + 1] - P.seg_item_begin[s] > kWideMergeItems) P.merge_flags = P.grid_merge;
   P.ws_items = cap;
   *grid = P.n_queue > 0 ? G : last;
   return FLINT_OK;

@@ -36,8 +36,10 @@
 //     and the last CTA to arrive (atomic counter, no spinning) merges all
 //     partials of the problem in item order and folds in the sinks.  A
 //     problem split over many CTAs (more than kInlineMergeMax items) is
-//     instead merged after a grid barrier (cooperative launch) by every warp
-//     of the grid.  Merge orders are fixed, so results are deterministic.
+//     instead merged by the CTAs that finish streaming first (cooperative
+//     launch), each partial folded once its ready flag is up, while the
+//     other CTAs still stream.  Merge orders are fixed, so results are
+//     deterministic.
 // Every mbarrier wait is bounded in time; on timeout the kernel records
 // FLINT_ERR_TIMEOUT, lets its loads land and returns.
 #include <math.h>
@@ -108,10 +110,11 @@ struct Smem {
   uint64_t* in_full;    // item inputs landed
   uint64_t* in_empty;   // item inputs consumed
   float2* cs;
-  volatile int* flags;  // [0] abort, [1] last-arrival broadcast, [2] grid barrier,
+  volatile int* flags;  // [0] abort, [1] last-arrival broadcast, [2] merge-ticket rank,
                         // [3] item whose new token is in the cache (+1),
                         // [4] item whose inputs are staged (producer -> consumers),
-                        // [5] that item as consumer warp 0 saw it (-1: stop)
+                        // [5] that item as consumer warp 0 saw it (-1: stop),
+                        // [6] the launch's ready-flag value (merge tail)
   float* xch;           // group hand-over area
   uint8_t* in;          // item inputs
 };
@@ -148,6 +151,28 @@ __device__ __forceinline__ void consumer_bar() {
 __device__ __forceinline__ void abort_cta(const DecodeParams& P, const Smem& S) {
   if (!S.flags[0]) report_error(P.dev_err, FLINT_ERR_TIMEOUT);
   S.flags[0] = 1;
+}
+
+// Ticket word, item flags and abort word of the merge at the launch's end
+// (see merge_tail).
+constexpr int kTicketShift = 12;
+static_assert(2 * kMaxCtas < (1 << (kTicketShift - 1)), "ticket ranks stay apart from block 0's addend");
+
+__device__ __forceinline__ unsigned int ld_relaxed_u32(const int32_t* p) {
+  unsigned int v;
+  asm volatile("ld.relaxed.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+  return v;
+}
+__device__ __forceinline__ void st_release_u32(int32_t* p, unsigned int v) {
+  asm volatile("st.release.gpu.global.u32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
+}
+
+// Raises item `it`'s ready flag (thread 0, after the barrier that orders the
+// other consumers' partial stores before it); `word` is the ticket word, read
+// by the same thread at the item's end.
+__device__ __forceinline__ void publish_item(const DecodeParams& P, int it, unsigned int word) {
+  if (!FLINT_CHECK(P.dev_err, it >= 0 && it < P.n_items && it < kMaxItems, 9, it, P.n_items, 0)) return;
+  st_release_u32(P.counters + kItemFlags + it, (word >> kTicketShift) + 1);
 }
 
 // Element offset, from the cache base the problem names, of the new token's
@@ -770,6 +795,7 @@ __device__ __forceinline__ void fold_partials(const DecodeParams& P, int s0, int
   }
 }
 
+template <bool kFlags>
 __device__ void run_consumer(const DecodeParams& P, const Smem& S, int warp, int lane) {
   const int g = lane >> 2, c = lane & 3;
   const int kvh = warp % kKvHeads;      // the KV head this warp serves
@@ -865,6 +891,12 @@ __device__ void run_consumer(const DecodeParams& P, const Smem& S, int warp, int
 
     // ---- item end: this warp holds (m, l, O) of its 8 heads over the item
     if (warp == 0 && lane == 0) FLINT_TRACE_MARK(4);
+    // ready-flag mode: the epoch for a deferred item's flag, read now so that
+    // the load is in flight while the partial is stored
+    [[maybe_unused]] unsigned int ticket_word = 0u;
+    if constexpr (kFlags) {
+      if (pb.deferred && threadIdx.x == 0) ticket_word = ld_relaxed_u32(P.counters + kTicketWord);
+    }
     l_run += __shfl_xor_sync(0xffffffffu, l_run, 1);
     l_run += __shfl_xor_sync(0xffffffffu, l_run, 2);
     float v[32];
@@ -925,11 +957,20 @@ __device__ void run_consumer(const DecodeParams& P, const Smem& S, int warp, int
     __syncwarp();
     consumer_bar();
     if (threadIdx.x == 0) FLINT_TRACE_MARK(5);
-    // A deferred problem is merged after the grid barrier, whose fence
-    // releases these partials.  Otherwise one thread releases them (the
-    // barrier above orders every consumer's stores before its fence) and
-    // counts the arrival; the last CTA to arrive merges.
-    if (pb.deferred) continue;
+    // One thread releases the partial (the barrier above orders every
+    // consumer's stores before it).  A deferred problem's item raises its
+    // ready flag for the CTAs that merge at the launch's end (ready-flag
+    // mode) or waits for the grid barrier; otherwise the thread counts the
+    // arrival, and the last CTA to arrive merges.
+    if (pb.deferred) {
+      if constexpr (kFlags) {
+        if (threadIdx.x == 0) {
+          publish_item(P, it, ticket_word);
+          FLINT_TRACE_MARK(12);
+        }
+      }
+      continue;
+    }
     if (threadIdx.x == 0) {
       int prev = 0;
       __threadfence();
@@ -972,6 +1013,70 @@ __device__ void run_consumer(const DecodeParams& P, const Smem& S, int warp, int
     consumer_bar();  // flags[1] and the hand-over area are reused by the next item
   }
 }
+
+// ---- merge of the deferred problems at the launch's end --------------------
+// Two modes, chosen per launch by the planner (P.merge_flags):
+//   * Grid barrier (0): every CTA arrives once its streaming is over; then
+//     CTA b merges tasks b, b + G, ...  Cheapest where the CTAs end together
+//     (short streams, or the run-time queue evening out the end).
+//   * Ready flags (1, when a problem is split over more than kWideMergeItems
+//     items): the CTAs that finish streaming first merge while the others
+//     still stream, each batch of partials once its items' flags are up.  It
+//     pays where the CTAs' end times spread over microseconds (a lone long
+//     context: ~21 tiles per CTA, SMs differing by up to ~28 % in rate).
+//     Its protocol:
+//   * Ticket (counters[kTicketWord]): after its streaming every CTA takes
+//     exactly one.  Block 0 adds 2^12 - (G - 1), the others add 1, so the
+//     low 12 bits return to zero once all G CTAs took theirs, and the carry
+//     out of them counts launches in bits 12..31: the launch's epoch E, the
+//     same in every CTA's ticket.  A CTA's rank is the number of tickets
+//     taken before its own; rank r merges tasks r, r + G, ...
+//   * Item flags (counters[kItemFlags + item]): after the consumers' barrier
+//     at the item's end, thread 0 stores E + 1 with release order.  It reads
+//     E from the ticket word (the load issued as the item ends, so that it is
+//     in flight while the partial is stored): no carry can happen before this
+//     CTA takes its own ticket.
+//   * Abort word (counters[kAbortWord]): a CTA that aborted stores E + 1, so
+//     that the merging CTAs stop waiting for its items.
+//   * The CTA of rank G - 1 knows that every CTA has made its last claim and
+//     raised its last flag: it resets the queue head and zeroes every flag
+//     this launch did not raise.  So at a launch's start each flag holds zero
+//     or the previous such launch's value (E), never this launch's E + 1,
+//     whatever the plans of earlier launches were.
+#ifndef FLINT_MERGE_BATCH
+#define FLINT_MERGE_BATCH 8
+#endif
+constexpr int kMergeBatch = FLINT_MERGE_BATCH;
+// Takes this CTA's ticket (thread 0): returns its rank, sets *ready = E + 1.
+__device__ __forceinline__ int take_ticket(const DecodeParams& P, unsigned int* ready) {
+  const unsigned int G = gridDim.x;
+  const unsigned int add = blockIdx.x == 0 ? (1u << kTicketShift) - (G - 1) : 1u;
+  unsigned int old;
+  // acquire: the queue reset below follows every other CTA's claims;
+  // release: this CTA's claims precede its ticket
+  asm volatile("atom.add.acq_rel.gpu.global.u32 %0, [%1], %2;"
+               : "=r"(old)
+               : "l"(P.counters + kTicketWord), "r"(add)
+               : "memory");
+  *ready = (old >> kTicketShift) + 1;
+  const unsigned int lo = old & ((1u << kTicketShift) - 1);
+  if (blockIdx.x == 0 || lo < (1u << (kTicketShift - 1))) return static_cast<int>(lo);
+  return static_cast<int>(lo + G) - (1 << kTicketShift);  // block 0 came before
+}
+
+// The merge works in units of (problem, KV head g, chunk q).  Lane (h, c) of
+// a warp owns values 4q..4q+3 of head 8g + h, quarter c: dims 16q + d0 +
+// {0, 1} and 16q + d2 + {0, 1} of the head (see dim_d0; the layout the
+// consumer warps wrote), so one warp load reads 512 consecutive bytes of a
+// partial.  A lane folds its partials kMergeBatch loads at a time, a batch
+// once its items' flags are up, and combines the batch states in batch order.
+//   * A problem with many partials (a lone long problem split over every
+//     CTA), or any deferred problem when a CTA per unit covers all their units
+//     at once, takes a whole CTA per unit (a task): warp w folds partials w,
+//     w + 9, ..., then the warps' states are combined through shared memory
+//     in warp order.
+//   * The other deferred problems take one warp per unit, nine units to a
+//     task, every lane folding all partials of its unit.
 
 // Grid-wide barrier for a cooperative launch: block 0 adds 2^31 - (G - 1),
 // the others add 1, so bit 31 of the word flips once all G blocks arrived and
@@ -1019,22 +1124,76 @@ __device__ bool grid_barrier(unsigned int* bar, const Smem& S) {
   return S.flags[2] != 0;
 }
 
-// Merge of the deferred problems by the whole grid after the grid barrier, in
-// units of (problem, KV head g, chunk q).  Lane (h, c) of a warp owns values
-// 4q..4q+3 of head 8g + h, quarter c: dims 16q + d0 + {0, 1} and
-// 16q + d2 + {0, 1} of the head (see dim_d0; the layout the consumer warps
-// wrote), so one warp load reads 512 consecutive bytes of a partial.  A lane folds its
-// partials kMergeBatch loads at a time, in item order.
-//   * Most problems take one warp per unit, every lane folding all partials.
-//   * A problem with many partials (a lone long problem split over every CTA)
-//     takes a whole CTA per unit: warp w folds partials w, w + 9, ..., then
-//     the warps' states are combined through shared memory in warp order.
-#ifndef FLINT_MERGE_BATCH
-#define FLINT_MERGE_BATCH 8
-#endif
-constexpr int kMergeBatch = FLINT_MERGE_BATCH;
+__device__ __forceinline__ unsigned int ld_acquire_u32(const int32_t* p) {
+  unsigned int v;
+  asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+  return v;
+}
 
-// Folds partials s0 + first, s0 + first + stride, ... (< s1) into (m, l, acc).
+// Ready-flag mode: folds the warp's partials s0 + first + k * stride (k = 0,
+// 1, ...; < s1) into (m, l, acc) in item order, kMergeBatch loads at a time.
+// Lane j watches the flag of the j-th item not folded yet (an acquire load);
+// the warp's ballot gives the run of raised flags at the front, and every
+// whole batch of it (or the last, short batch) is folded.  Batches start at
+// fixed multiples of kMergeBatch, as in fold_chunk, so the sums do not depend
+// on the mode or on when flags came up.  False if the wait gave up (some CTA
+// aborted, or the time limit ran out); the state is then meaningless.
+__device__ __forceinline__ bool fold_chunk_wait(const DecodeParams& P, int s0, int s1, int first, int stride,
+                                                int head, int c, int q, unsigned int ready, float& m, float& l,
+                                                float4& acc) {
+  const int lane = threadIdx.x & 31;
+  const int i_first = s0 + first;
+  const int n = i_first < s1 ? (s1 - i_first + stride - 1) / stride : 0;
+  const unsigned long long t0 = globaltimer_ns();
+  int done = 0, spin = 0;
+  while (done < n) {
+    const int k = done + lane;
+    const bool up = k >= n || ld_acquire_u32(P.counters + kItemFlags + i_first + k * stride) == ready;
+    const unsigned int mask = __ballot_sync(0xffffffffu, up);
+    __syncwarp();  // orders every lane's partial loads below after the lanes' acquires
+    int take = min(mask == 0xffffffffu ? 32 : __ffs(~mask) - 1, n - done);
+    if (take < n - done) take -= take % kMergeBatch;
+    if (take == 0) {
+      if (ld_relaxed_u32(P.counters + kAbortWord) == ready) return false;
+      if ((++spin & 7) == 0 && globaltimer_ns() - t0 > kWaitLimitNs) return false;
+      continue;
+    }
+    for (int b = 0; b < take; b += kMergeBatch) {
+      const int cnt = min(kMergeBatch, take - b);
+      const int i0 = i_first + (done + b) * stride;
+      float mi[kMergeBatch], li[kMergeBatch];
+      float4 vi[kMergeBatch];
+#pragma unroll
+      for (int j = 0; j < kMergeBatch; ++j) {
+        const int i = j < cnt ? i0 + j * stride : i0;
+        const float* pi = P.partials + static_cast<size_t>(i) * kPartialFloats;
+        mi[j] = j < cnt ? __ldcg(pi + kHeads * kDim + head) : -INFINITY;
+        li[j] = __ldcg(pi + kHeads * kDim + kHeads + head);
+        vi[j] = __ldcg(reinterpret_cast<const float4*>(pi) + partial_f4(head, c, q));
+      }
+      float mn = m;
+#pragma unroll
+      for (int j = 0; j < kMergeBatch; ++j) mn = fmaxf(mn, mi[j]);
+      const float sa = (m == -INFINITY) ? 0.f : exp2f(m - mn);
+      l *= sa;
+      acc = make_float4(acc.x * sa, acc.y * sa, acc.z * sa, acc.w * sa);
+      m = mn;
+#pragma unroll
+      for (int j = 0; j < kMergeBatch; ++j) {
+        const float sb = (mi[j] == -INFINITY) ? 0.f : exp2f(mi[j] - m);
+        l += sb * li[j];
+        acc.x += sb * vi[j].x;
+        acc.y += sb * vi[j].y;
+        acc.z += sb * vi[j].z;
+        acc.w += sb * vi[j].w;
+      }
+    }
+    done += take;
+  }
+  return true;
+}
+
+// Grid-barrier mode: Folds partials s0 + first, s0 + first + stride, ... (< s1) into (m, l, acc).
 __device__ __forceinline__ void fold_chunk(const DecodeParams& P, int s0, int s1, int first, int stride,
                                            int head, int c, int q, float& m, float& l, float4& acc) {
   for (int i0 = s0 + first; i0 < s1; i0 += kMergeBatch * stride) {
@@ -1089,6 +1248,9 @@ __device__ __forceinline__ void write_chunk(const Problem& pb, int head, int c, 
   *reinterpret_cast<float2*>(o + d2) = make_float2(acc.z * scale, acc.w * scale);
 }
 
+// Grid-barrier mode: the merge of the deferred problems by the whole grid
+// after the grid barrier; CTA b takes the units of task b (its warps one
+// regular unit each, or the whole CTA a wide unit), b + G, ...
 __device__ void grid_merge(const DecodeParams& P, const Smem& S) {
   constexpr int kWarps = kThreads / 32;
   constexpr int kUnits = kKvHeads * 8;  // units per problem
@@ -1157,6 +1319,108 @@ __device__ void grid_merge(const DecodeParams& P, const Smem& S) {
   }
 }
 
+// Ready-flag mode: the launch's end for a CTA whose streaming is over: its
+// ticket, then its merge tasks.  A wait that gives up records
+// FLINT_ERR_TIMEOUT; the task's output is then left unwritten.
+__device__ void merge_tail(const DecodeParams& P, const Smem& S) {
+  constexpr int kWarps = kThreads / 32;
+  constexpr int kUnits = kKvHeads * 8;  // units per problem
+  const int t = threadIdx.x, lane = t & 31, warp = t >> 5;
+  const int c = lane & 3;
+  if (t == 0) {
+    unsigned int r;
+    const int k = take_ticket(P, &r);
+    if (S.flags[0]) st_release_u32(P.counters + kAbortWord, r);
+    if (k == static_cast<int>(gridDim.x) - 1) P.counters[kQueueHead] = 0;  // ready for the next call
+    S.flags[2] = k;
+    S.flags[6] = static_cast<int>(r);
+    FLINT_TRACE_MARK(8);
+  }
+  __syncthreads();
+  const int rank = S.flags[2];
+  const unsigned int ready = static_cast<unsigned int>(S.flags[6]);
+  if (rank == static_cast<int>(gridDim.x) - 1) {
+    // zero the flags this launch did not raise (no merging CTA reads them)
+    for (int i = t; i < kMaxItems; i += kThreads)
+      if (!((P.raised[i / 32] >> (i % 32)) & 1u)) P.counters[kItemFlags + i] = 0;
+  }
+  const int wide_tasks = P.n_wide * kUnits;
+  const int units = (P.n_deferred - P.n_wide) * kUnits;
+  const int n_tasks = wide_tasks + (units + kWarps - 1) / kWarps;
+  float* red = S.xch;  // [kWarps][32][6] (the hand-over area is free now)
+  for (int task = rank; task < n_tasks; task += gridDim.x) {
+    if (task >= wide_tasks) {
+      const int u = (task - wide_tasks) * kWarps + warp;
+      if (u < units) {
+        const int p = P.deferred[P.n_wide + u / kUnits];
+        const int kvh = (u / 8) % kKvHeads, q = u % 8;
+        const int head = kvh * kGroup + (lane >> 2);
+        const Problem& pb = P.prob[p];
+        const float sink = pb.sinks ? pb.sinks[head] : 0.f;  // in flight with the partials
+        float m = -INFINITY, l = 0.f;
+        float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+        if (threadIdx.x == 0) FLINT_TRACE_MARK(13);
+        if (fold_chunk_wait(P, P.seg_item_begin[p], P.seg_item_begin[p + 1], 0, 1, head, c, q, ready, m, l,
+                            acc))
+          write_chunk(pb, head, c, q, m, l, acc, sink);
+        else if (lane == 0)
+          report_error(P.dev_err, FLINT_ERR_TIMEOUT);
+        if (threadIdx.x == 0) FLINT_TRACE_MARK(15);
+      }
+      continue;
+    }
+    const int p = P.deferred[task / kUnits];
+    const int kvh = (task / 8) % kKvHeads, q = task % 8;
+    const int head = kvh * kGroup + (lane >> 2);
+    const Problem& pb = P.prob[p];
+    const float sink = pb.sinks ? pb.sinks[head] : 0.f;
+    float m = -INFINITY, l = 0.f;
+    float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+    const int s0 = P.seg_item_begin[p], s1 = P.seg_item_begin[p + 1];
+#ifdef FLINT_TRACE
+    if (threadIdx.x == 0) FLINT_TRACE_SET(13, globaltimer_ns() + 0ull * (s0 + s1 + sink));
+#endif
+    const bool ok = fold_chunk_wait(P, s0, s1, warp, kWarps, head, c, q, ready, m, l, acc);
+#ifdef FLINT_TRACE
+    if (threadIdx.x == 0) FLINT_TRACE_SET(14, globaltimer_ns() + 0ull * static_cast<unsigned long long>(acc.x + m + l));
+#endif
+    float* mine = red + (warp * 32 + lane) * 6;
+    mine[0] = m;
+    mine[1] = l;
+    mine[2] = acc.x;
+    mine[3] = acc.y;
+    mine[4] = acc.z;
+    mine[5] = acc.w;
+    const bool failed = __syncthreads_or(!ok);
+    if (warp == 0 && !failed) {
+      float M = -INFINITY;
+#pragma unroll
+      for (int w = 0; w < kWarps; ++w) M = fmaxf(M, red[(w * 32 + lane) * 6]);
+      float L = 0.f;
+      float4 A = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+      for (int w = 0; w < kWarps; ++w) {
+        const float* o = red + (w * 32 + lane) * 6;
+        const float sc = (o[0] == -INFINITY) ? 0.f : exp2f(o[0] - M);
+        L += sc * o[1];
+        A.x += sc * o[2];
+        A.y += sc * o[3];
+        A.z += sc * o[4];
+        A.w += sc * o[5];
+      }
+      write_chunk(pb, head, c, q, M, L, A, sink);
+    }
+    if (threadIdx.x == 0) {
+      if (failed) report_error(P.dev_err, FLINT_ERR_TIMEOUT);
+      FLINT_TRACE_MARK(15);
+    }
+    __syncthreads();  // red is reused by the next task
+  }
+}
+
+// kFlags: the launch merges its deferred problems in ready-flag mode
+// (P.merge_flags), else after the grid barrier.
+template <bool kFlags>
 __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const __grid_constant__ DecodeParams P) {
   // A launch that follows this one in the stream with programmatic
   // dependence may be scheduled from now on (it waits for this grid's
@@ -1222,7 +1486,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const __grid_consta
       FLINT_TRACE_SET(11, pc.staged);
     }
   } else {
-    run_consumer(P, S, warp, lane);
+    run_consumer<kFlags>(P, S, warp, lane);
   }
   __syncthreads();
   if (threadIdx.x == 0) FLINT_TRACE_MARK(7);
@@ -1246,7 +1510,12 @@ __global__ void __launch_bounds__(kThreads, 1) decode_kernel(const __grid_consta
     }
   }
   if (P.grid_merge) {
-    if (grid_barrier(reinterpret_cast<unsigned int*>(P.counters + kBarrierWord), S)) {
+    if constexpr (kFlags) {
+      merge_tail(P, S);
+#ifdef FLINT_TRACE
+      if (threadIdx.x == 0) FLINT_TRACE_MARK(9);
+#endif
+    } else if (grid_barrier(reinterpret_cast<unsigned int*>(P.counters + kBarrierWord), S)) {
       // every CTA has made its last claim: ready the queue for the next call
       if (blockIdx.x == 0 && threadIdx.x == 0) P.counters[kQueueHead] = 0;
       if (threadIdx.x == 0) FLINT_TRACE_MARK(8);
@@ -1290,8 +1559,11 @@ extern "C" int flint_test_stall_decode(int block, int seq) {
 #endif
 
 cudaError_t launch_decode(const DecodeParams& p, int grid, cudaStream_t stream) {
-  static ContextSet configured;
-  cudaError_t e = configure_once(configured, reinterpret_cast<const void*>(decode_kernel), static_cast<int>(decode_smem_bytes()));
+  static ContextSet configured[2];
+  const int mode = p.merge_flags ? 1 : 0;
+  const void* kernel = mode ? reinterpret_cast<const void*>(decode_kernel<true>)
+                            : reinterpret_cast<const void*>(decode_kernel<false>);
+  cudaError_t e = configure_once(configured[mode], kernel, static_cast<int>(decode_smem_bytes()));
   if (e != cudaSuccess) return e;
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(grid);
@@ -1300,7 +1572,7 @@ cudaError_t launch_decode(const DecodeParams& p, int grid, cudaStream_t stream) 
   cfg.stream = stream;
   cudaLaunchAttribute attrs[2];
   int n = 0;
-  if (p.grid_merge) {  // the grid barrier needs every CTA resident at once
+  if (p.grid_merge) {  // the merging CTAs wait for the others: every CTA resident at once
     attrs[n].id = cudaLaunchAttributeCooperative;
     attrs[n].val.cooperative = 1;
     ++n;
@@ -1312,7 +1584,7 @@ cudaError_t launch_decode(const DecodeParams& p, int grid, cudaStream_t stream) 
   }
   cfg.attrs = attrs;
   cfg.numAttrs = n;
-  e = cudaLaunchKernelEx(&cfg, decode_kernel, p);
+  e = mode ? cudaLaunchKernelEx(&cfg, decode_kernel<true>, p) : cudaLaunchKernelEx(&cfg, decode_kernel<false>, p);
   if (e != cudaSuccess) return e;
   return cudaGetLastError();
 }

@@ -76,8 +76,18 @@ constexpr int kMaxCtas = 296;
 
 // A problem split into more than kInlineMergeMax items is not merged by its
 // last-arriving CTA (one CTA reading every partial would be the tail of the
-// launch) but by all warps of the grid after a grid barrier.
+// launch) but by the CTAs that finish streaming first, as its items' ready
+// flags come up.
 constexpr int kInlineMergeMax = 16;
+
+// A deferred problem with more partials than this is merged a CTA per unit
+// (each of its 9 warps folding every 9th partial) instead of a warp per unit
+// (the warp folding all partials).  So no warp folds more than
+// kMergeWarpItems partials.
+constexpr int kWideMergeItems = 96;
+constexpr int kMergeWarpItems = 96;
+static_assert(kWideMergeItems <= kMergeWarpItems && (kMaxItems + 8) / 9 <= kMergeWarpItems,
+              "a merging warp folds at most kMergeWarpItems partials");
 
 // One split partial of a problem: O for 32 heads (in the order the consumer
 // warps hold it, chunk-interleaved across each warp's lanes), m [32] (log2
@@ -85,9 +95,17 @@ constexpr int kInlineMergeMax = 16;
 constexpr int kPartialFloats = kHeads * kDim + 2 * kHeads;
 constexpr size_t kCounterBytes = 4096;
 // int32 slots of the workspace's counter area: [0, kMaxSegs) per-problem
-// arrival counters, then the grid-barrier word and the run-time queue head.
+// arrival counters, then the grid-barrier word, the run-time queue head, the
+// abort word and the merge-ticket word, and from kItemFlags one ready flag
+// per item.
 constexpr int kBarrierWord = kMaxSegs;
 constexpr int kQueueHead = kMaxSegs + 1;
+constexpr int kAbortWord = kMaxSegs + 2;
+constexpr int kTicketWord = kMaxSegs + 3;
+constexpr int kItemFlags = 128;
+static_assert(kMaxItems % 32 == 0, "one raised-flag bit per item");
+static_assert(kTicketWord < kItemFlags && kItemFlags + kMaxItems <= static_cast<int>(kCounterBytes / 4),
+              "the counter area holds the counters and one flag per item");
 
 // One attention problem: one request of one layer.
 struct Problem {
@@ -111,7 +129,7 @@ struct Problem {
   int16_t map_k, map_v;     // tensor-map indices
   int16_t req;              // 4th tensor coordinate (request) for CONTIGUOUS/RING
   int8_t layout, q_fp32, rope;
-  int8_t deferred;          // 1: merged by the whole grid after a grid barrier
+  int8_t deferred;          // 1: merged at the launch's end (grid barrier or ready flags)
   int8_t fp8;               // 1: E4M3 cache, 64-token tiles, scales in kv_scales[map_k / 2]
   int8_t partial;           // 1: out receives the unnormalised partial (O [32][128], m [32],
                             //    l [32]; log2 units) and no sink is folded in (sinks may be NULL)
@@ -145,8 +163,9 @@ struct DecodeParams {
   int32_t n_problems;
   int32_t prep;             // 1: q/k norm (+RoPE) and append fused in (layer stack)
   int32_t n_items;          // items in the plan
-  int32_t grid_merge;       // 1: a grid barrier ends the launch (cooperative launch):
-                            // some problem is deferred or the queue is not empty
+  int32_t grid_merge;       // 1: the launch ends in a merge of the deferred problems
+                            // (cooperative launch): some problem is deferred or the
+                            // queue is not empty
   int16_t deferred[kMaxProblems];  // the deferred problems, those with many partials first
   int32_t n_deferred;
   int32_t n_wide;           // deferred[0, n_wide): merged a CTA per unit, the rest a warp per unit
@@ -154,6 +173,9 @@ struct DecodeParams {
   int32_t pdl;              // 1: programmatic dependent launch on the previous kernel of the
                             // stream: wait for it before touching global memory
   int32_t smem_bytes;       // dynamic shared memory of the launch
+  int32_t merge_flags;      // 1: the merge at the launch's end runs on ready flags and
+                            // tickets (decode_kernel<true>), 0: after a grid barrier
+  uint32_t raised[kMaxItems / 32];  // bit i: item i is a deferred problem's (it raises a ready flag)
 };
 
 static_assert(sizeof(DecodeParams) <= 32000, "kernel parameters exceed 32 KiB");

@@ -71,6 +71,26 @@ def e4m3_code_distance(a: np.ndarray, b: np.ndarray) -> np.ndarray:
     return np.abs(ordered(a) - ordered(b))
 
 
+def check_workspace_clean(ws: torch.Tensor):
+    """The counter area (the first 4096 bytes) a clean call leaves behind:
+    per-problem arrival counters [0, 64) at zero; the grid-barrier word (64)
+    with only its generation bit (31) left; queue head (65) and abort word
+    (66) at zero; the merge-ticket word (67) with its low 12 bits at zero (its
+    upper bits count the launches that ended in merge tickets, the epoch E);
+    the spare words up to 128 at zero; the item ready flags [128, 896) each
+    zero or the last ticket launch's value (E); the rest zero."""
+    w = ws[:4096].view(torch.int32).cpu().numpy().astype(np.int64) & 0xFFFFFFFF
+    assert not w[:64].any(), "arrival counters left non-zero"
+    assert w[64] & 0x7FFFFFFF == 0, f"grid-barrier word {w[64]:#x}: low bits not back at zero"
+    assert not w[65:67].any(), "queue head or abort word left non-zero"
+    assert w[67] & 0xFFF == 0, f"ticket word {w[67]:#x}: low bits not back at zero"
+    epoch = w[67] >> 12
+    assert not w[68:128].any(), "spare counter words left non-zero"
+    flags = w[128:896]
+    assert np.all((flags == 0) | (flags == epoch)), "an item flag holds another launch's value"
+    assert not w[896:].any()
+
+
 def oracle_layer(layer: I.Layer, nthreads: int = 0):
     """Oracle for one synthetic layer: norm (+RoPE) -> append -> attend.
     Returns (out f64 [32,128], k cache, v cache) after the append: bf16 bits,

@@ -8,7 +8,7 @@ import oracle
 from long_context_decode_flash_b200 import flint
 from long_context_decode_flash_b200 import inputs as I
 
-from helpers import dev, parity
+from helpers import check_workspace_clean, dev, parity
 
 pytestmark = pytest.mark.gpu
 
@@ -25,11 +25,7 @@ def run_decode(q, k, v, seq_lens, sinks, window, layout=flint.CONTIGUOUS, capaci
                             dev_err=err)
     torch.cuda.synchronize()
     assert int(err.item()) == 0
-    # the library leaves the per-problem arrival counters and the queue head at
-    # zero after a clean call (the grid-barrier word between them keeps only a
-    # generation bit)
-    assert int(ws[:256].view(torch.int32).abs().sum().item()) == 0
-    assert int(ws[256:4096].view(torch.int32)[1:].abs().sum().item()) == 0
+    check_workspace_clean(ws)  # ready for the next call
     return out.cpu().numpy()
 
 
@@ -74,6 +70,45 @@ def test_deterministic_run_to_run():
     a = run_decode(*args, capacity=20000)
     b = run_decode(*args, capacity=20000)
     assert np.array_equal(a, b)
+
+
+def test_workspace_reused_across_plans():
+    """One workspace through calls of different plans: a problem merged a CTA
+    per unit (9,000 tokens over every SM), one merged a warp per unit, a
+    ragged batch, a launch with no merge at the end, and the first call again.
+    The items' ready flags carry the launch count, so a flag left by an
+    earlier plan never passes for a new one: every call matches the oracle,
+    a repeated call gives the same bits, and the workspace is left clean."""
+    ws = flint.workspace(3)
+    err = torch.zeros(1, dtype=torch.int32, device="cuda")
+    big = I.make_decode(9000, workload=I.W_FULL_SMALL + 40)
+    small = I.make_decode(2048, workload=I.W_FULL_SMALL + 41)
+    batch = I.make_decode(5000, workload=I.W_FULL_SMALL + 42, B=3)
+    batch.seq_lens = [5000, 700, 3000]
+    want_big, want_small = oracle_contig(big, 0, 0), oracle_contig(small, 0, 0)
+    want_batch = [oracle_contig(batch, b, 0) for b in range(3)]
+
+    def call(d, num_ctas=0):
+        cache = flint.kv_cache(dev(d.k_cache), dev(d.v_cache), flint.CONTIGUOUS,
+                               capacity=d.k_cache.shape[1])
+        out = torch.full((len(d.seq_lens), 32, 128), float("nan"), dtype=torch.float32, device="cuda")
+        flint.flint_attn_decode(dev(d.q), cache, d.seq_lens, dev(d.sinks), 0, out, ws,
+                                num_ctas=num_ctas, dev_err=err)
+        torch.cuda.synchronize()
+        assert int(err.item()) == 0
+        check_workspace_clean(ws)
+        return out.cpu().numpy()
+
+    first = call(big)
+    parity(first[0], want_big, "9000 tokens, first call")
+    for n in (148, 0):
+        parity(call(small, n)[0], want_small, f"2048 tokens, num_ctas={n}")
+    got = call(batch)
+    for b in range(3):
+        parity(got[b], want_batch[b], f"batch request {b}")
+    parity(call(small, 7)[0], want_small, "2048 tokens on 7 CTAs (merged inline)")
+    again = call(big)
+    assert np.array_equal(again, first)
 
 
 def test_full_layer_100k_matches_oracle():
