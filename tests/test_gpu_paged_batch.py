@@ -39,10 +39,8 @@ def test_paged_batch_32_requests(batch, window):
     assert int(err.item()) == 0
     got = out.cpu().numpy()
     assert np.isfinite(got).all()
-    order = np.argsort(pb.seq_lens)
-    sample = [int(order[0]), int(order[len(order) // 2]), int(order[-1]), 7]
     kp, vp = I.bits(pb.k_pool), I.bits(pb.v_pool)
-    for b in sample:
+    for b in range(B):  # every request (~1.1M tokens of oracle work, ~8 s)
         want = oracle.attn_decode(I.bits(pb.q[b]), kp, vp, pb.seq_lens[b],
                                   pb.sinks.numpy().astype(np.float64), window,
                                   layout=oracle.PAGED, block_table=pb.block_table[b].numpy())
