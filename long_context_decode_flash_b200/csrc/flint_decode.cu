@@ -36,9 +36,11 @@
 //     and the last CTA to arrive (atomic counter, no spinning) merges all
 //     partials of the problem in item order and folds in the sinks.  A
 //     problem split over many CTAs (more than kInlineMergeMax items) is
-//     instead merged by the CTAs that finish streaming first (cooperative
-//     launch), each partial folded once its ready flag is up, while the
-//     other CTAs still stream.  Merge orders are fixed, so results are
+//     instead merged at the launch's end by the whole grid (cooperative
+//     launch): after a grid barrier, or, for a problem over more than
+//     kWideMergeItems items, by the CTAs that finish streaming first, each
+//     batch of partials folded once its ready flags are up while the other
+//     CTAs still stream.  Merge orders are fixed, so results are
 //     deterministic.
 // Every mbarrier wait is bounded in time; on timeout the kernel records
 // FLINT_ERR_TIMEOUT, lets its loads land and returns.
@@ -1052,8 +1054,8 @@ __device__ __forceinline__ int take_ticket(const DecodeParams& P, unsigned int* 
   const unsigned int G = gridDim.x;
   const unsigned int add = blockIdx.x == 0 ? (1u << kTicketShift) - (G - 1) : 1u;
   unsigned int old;
-  // acquire: the queue reset below follows every other CTA's claims;
-  // release: this CTA's claims precede its ticket
+  // acquire: the queue reset by the last ticket's CTA follows every other
+  // CTA's claims; release: this CTA's claims precede its ticket
   asm volatile("atom.add.acq_rel.gpu.global.u32 %0, [%1], %2;"
                : "=r"(old)
                : "l"(P.counters + kTicketWord), "r"(add)
