@@ -8,10 +8,12 @@ its streaming is over.
     The low 12 bits return to zero after the G tickets of a launch, and the
     carry out of them counts launches (the epoch E, bits 12..31).  A CTA's
     rank is the number of tickets taken before its own.
-  * A raised flag holds E + 1.  The publishing thread reads E from the
-    ticket word at the item's end and raises the flag once the CTA's next
-    item has begun (or the CTA has no item left), before its own CTA takes a
-    ticket.
+  * A raised flag holds E + 1.  At the item's end the publishing thread
+    reads E from the ticket word and then raises the flag, both before its
+    own CTA takes a ticket.
+  * A CTA that aborted (a wait ran out) stops taking items and stores E + 1
+    into the abort word with its ticket; the merging CTAs stop waiting when
+    they see it.
   * The CTA of rank G - 1 resets the queue head and zeroes every flag that
     the launch did not raise.
 
@@ -20,10 +22,11 @@ the CTAs' steps.  It checks that the ranks of a launch are 0..G-1 and the
 epoch is the same in every CTA; that the word ends each launch with its low
 bits at zero and the epoch one higher; that a merging CTA never sees a flag
 as raised before this launch raised it, even when the epoch wraps; that no
-CTA claims from the queue after the reset; and that every launch ends.
-Mutants are caught: no flag clearing (with a narrow epoch, where stale flags
-come back), the reset by a CTA other than rank G - 1, and a ticket taken
-before the CTA's last publication.
+CTA claims from the queue after the reset; and that every launch ends, an
+aborted one too.  Mutants are caught: no flag clearing (with a narrow epoch,
+where stale flags come back), the reset by a CTA other than rank G - 1, a
+ticket taken before the CTA's last publication, and an abort that leaves the
+abort word unset.
 """
 import itertools
 import random
@@ -80,13 +83,15 @@ def test_ticket_ranks_random_orders(G):
 
 
 def launch(ws, rng, G, n_items, deferred, epoch_bits=20, clear=True, reset_rank=None,
-           ticket_early=False, queue_items=0):
-    """One launch of the model.  ws: dict with 'ticket', 'flags', 'queue'.
-    deferred[i]: item i belongs to a deferred problem (it raises a flag and is
-    merged).  Items [0, n_static) are dealt round robin to the CTAs; the last
-    `queue_items` items are claimed from the queue.  Returns a list of
-    violations."""
+           ticket_early=False, queue_items=0, abort_cta=None, abort_word=True):
+    """One launch of the model.  ws: dict with 'ticket', 'flags', 'queue',
+    'abort'.  deferred[i]: item i belongs to a deferred problem (it raises a
+    flag and is merged).  Items [0, n_static) are dealt round robin to the
+    CTAs; the last `queue_items` items are claimed from the queue.  CTA
+    `abort_cta` aborts after its first item.  Returns (violations, whether a
+    merge gave up on an abort)."""
     errors = []
+    gave_up = []
     emask = (1 << epoch_bits) - 1
     reset_rank = G - 1 if reset_rank is None else reset_rank
     n_static = n_items - queue_items
@@ -96,18 +101,16 @@ def launch(ws, rng, G, n_items, deferred, epoch_bits=20, clear=True, reset_rank=
     def cta(b):
         mine = [i for i in range(n_static) if owner[i] == b]
         rank = ready = None
+        aborted = False
         if ticket_early:
             ws["ticket"], rank, ready = take_ticket(ws["ticket"], b, G)
             yield
         # stream the static items, then claim queued ones until the queue is dry
-        pending = None  # (item, epoch read at its end): raised once the next item began
-
-        def raise_pending():
-            if pending is not None:
-                ws["flags"][pending[0]] = pending[1] + 1
-                published.add(pending[0])
-
+        done = 0
         while True:
+            if b == abort_cta and done == 1:
+                aborted = True  # a wait ran out: no further item is taken
+                break
             if mine:
                 i = mine.pop(0)
             else:
@@ -119,18 +122,19 @@ def launch(ws, rng, G, n_items, deferred, epoch_bits=20, clear=True, reset_rank=
                 i = n_static + q
                 if ws.get("reset_done"):
                     errors.append(f"claim of queue slot {q} after the queue reset")
-            yield  # the item's first tile
-            raise_pending()
-            pending = None
-            yield  # the rest of the item
+            yield  # streaming the item
             if deferred[i]:
-                pending = (i, (ws["ticket"] >> SHIFT) & emask)
+                e = (ws["ticket"] >> SHIFT) & emask
                 yield
-        raise_pending()
-        yield
+                ws["flags"][i] = e + 1
+                published.add(i)
+                yield
+            done += 1
         if not ticket_early:
             ws["ticket"], rank, ready = take_ticket(ws["ticket"], b, G)
         ready = ((ready - 1) & emask) + 1  # E + 1 for an epoch of epoch_bits bits
+        if aborted and abort_word:
+            ws["abort"] = ready
         yield
         if rank == reset_rank:
             ws["queue"] = 0
@@ -147,6 +151,9 @@ def launch(ws, rng, G, n_items, deferred, epoch_bits=20, clear=True, reset_rank=
                     continue
                 spins = 0
                 while ws["flags"][i] != ready:
+                    if ws["abort"] == ready:
+                        gave_up.append(i)
+                        return
                     spins += 1
                     if spins > 10_000:
                         errors.append(f"wait on item {i} never ended")
@@ -169,23 +176,27 @@ def launch(ws, rng, G, n_items, deferred, epoch_bits=20, clear=True, reset_rank=
             errors.append("launch did not end")
             break
     ws["reset_done"] = False
-    if ws["queue"] != 0:
+    if ws["queue"] != 0 and abort_cta is None:
         errors.append("queue head not reset")
     if ws["ticket"] & LOW:
         errors.append("ticket low bits not back at zero")
-    return errors
+    return errors, bool(gave_up)
+
+
+def fresh_ws(max_items, word=0):
+    return {"ticket": word, "flags": [0] * max_items, "queue": 0, "abort": 0}
 
 
 def run_launches(seed, n_launches, max_items=24, **kw):
     rng = random.Random(seed)
-    ws = {"ticket": kw.pop("start_word", 0), "flags": [0] * max_items, "queue": 0}
+    ws = fresh_ws(max_items, kw.pop("start_word", 0))
     errors = []
     for _ in range(n_launches):
         G = rng.randint(1, 6)
         n_items = rng.randint(1, max_items)
         queue_items = rng.randint(0, n_items // 2)
         deferred = [rng.random() < 0.6 for _ in range(n_items)]
-        errors += launch(ws, rng, G, n_items, deferred, queue_items=queue_items, **kw)
+        errors += launch(ws, rng, G, n_items, deferred, queue_items=queue_items, **kw)[0]
         if errors:
             break
     return errors
@@ -228,3 +239,32 @@ def test_ticket_before_the_last_publication_is_caught():
         if errors:
             break
     assert errors, "an early ticket should break the protocol"
+
+
+def aborted_launches(seed, n_launches, abort_word=True):
+    """Launches in which one CTA aborts after its first item; the workspace is
+    zeroed after each, as the library asks after a device error."""
+    rng = random.Random(seed)
+    errors, gave_up = [], 0
+    for _ in range(n_launches):
+        ws = fresh_ws(24, rng.randrange(1 << 20) << SHIFT)
+        G = rng.randint(2, 6)
+        n_items = rng.randint(2 * G, 24)
+        deferred = [True] * n_items  # every item merged: the aborted CTA's are awaited
+        e, g = launch(ws, rng, G, n_items, deferred, abort_cta=rng.randrange(G), abort_word=abort_word)
+        errors += e
+        gave_up += g
+        if errors:
+            break
+    return errors, gave_up
+
+
+def test_an_abort_ends_every_wait():
+    errors, gave_up = aborted_launches(7, 150)
+    assert errors == []
+    assert gave_up > 0  # the merging CTAs did wait on the aborted CTA's items
+
+
+def test_abort_without_the_abort_word_is_caught():
+    errors, _ = aborted_launches(8, 150, abort_word=False)
+    assert any("never ended" in e for e in errors), errors
