@@ -43,24 +43,25 @@ NOMINAL_HBM_GBS = 8000.0
 # captured on 19a68889bfe7d421 (whole-source 674e68c590d7e033).  Two changes
 # since: a host-side rule (a launch with programmatic dependence keeps the
 # grid-barrier merge), which leaves these launches' parameters and kernel
-# unchanged, and a comment in flint_decode.cu (ed918c626bf307fb).  The stack
-# and full100k recaptures on 24d5ac5ca49d61bc match their 19a68889 figures
-# within 0.01 % of the reads.
-TRAFFIC = {("stack", 100_000, "bf16"): (2_905_872_896 + 7_185_664, "ed918c626bf307fb"),
-           ("stack", 100_000, "fp8"): (1_453_878_528 + 6_585_600, "ed918c626bf307fb"),
-           ("full100k", 100_000, "bf16"): (204_903_424 + 3_350_272, "ed918c626bf307fb"),
-           ("full2k", 2048, "bf16"): (4_287_232 + 0, "ed918c626bf307fb"),
-           ("swa100k", 100_000, "bf16"): (1_141_504 + 0, "ed918c626bf307fb"),
-           ("paged32", 100_000, "bf16"): (2_271_105_792 + 6_537_472, "ed918c626bf307fb"),
-           ("paged32swa", 100_000, "bf16"): (36_022_784 + 67_328, "ed918c626bf307fb")}
+# unchanged, and comments in flint_decode.cu, flint_abi.cu and
+# flint_internal.h (71d178cd5680e1f1).  The stack and full100k recaptures on
+# 24d5ac5ca49d61bc match their 19a68889 figures within 0.01 % of the reads.
+TRAFFIC = {("stack", 100_000, "bf16"): (2_905_872_896 + 7_185_664, "71d178cd5680e1f1"),
+           ("stack", 100_000, "fp8"): (1_453_878_528 + 6_585_600, "71d178cd5680e1f1"),
+           ("full100k", 100_000, "bf16"): (204_903_424 + 3_350_272, "71d178cd5680e1f1"),
+           ("full2k", 2048, "bf16"): (4_287_232 + 0, "71d178cd5680e1f1"),
+           ("swa100k", 100_000, "bf16"): (1_141_504 + 0, "71d178cd5680e1f1"),
+           ("paged32", 100_000, "bf16"): (2_271_105_792 + 6_537_472, "71d178cd5680e1f1"),
+           ("paged32swa", 100_000, "bf16"): (36_022_784 + 67_328, "71d178cd5680e1f1")}
 # The same for one prefill_kernel launch of a full (NoPE) layer on the
 # 8,192-token prompt (one pass: the metrics above), and for one
 # prefill_prep_kernel launch of a full layer (keyed on PREP_SOURCES).  Both
 # were captured on prefill sources 57c0c741ce570be8 and prep sources
-# 565c542954471930.  The only change since is the decode stack's host-side
-# merge-mode rule in flint_abi.cu, which no prefill call reaches.
-PREFILL_TRAFFIC = {8192: (83_956_224 + 86_484_736, "dd081a28169d247d")}
-PREP_TRAFFIC = {8192: (83_913_216 + 43_561_216, "52e8171ac9abe563")}
+# 565c542954471930.  The changes since are the decode stack's host-side
+# merge-mode rule in flint_abi.cu, which no prefill call reaches, and
+# comments in flint_abi.cu and flint_internal.h.
+PREFILL_TRAFFIC = {8192: (83_956_224 + 86_484_736, "aeb8ffda79af38f3")}
+PREP_TRAFFIC = {8192: (83_913_216 + 43_561_216, "395e12b169604c1e")}
 
 
 def max_over_ranks(x: float, world: int, device) -> float:

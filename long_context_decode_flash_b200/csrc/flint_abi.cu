@@ -289,8 +289,8 @@ flint_status plan(DecodeParams& P, const int* tiles, int n_problems, int num_cta
     P.seg_item_begin[s] = static_cast<int16_t>(i);
   }
   // Problems with queued chunks, or split more widely than kInlineMergeMax,
-  // are merged at the launch's end by the CTAs that finish streaming first,
-  // as their items' flags come up: their last items finish near the end of
+  // are merged at the launch's end by the whole grid (after a grid barrier,
+  // or on ready flags, see below): their last items finish near the end of
   // the launch, where one CTA merging alone would be the tail.
   P.n_deferred = 0;
   P.n_wide = 0;

@@ -76,8 +76,9 @@ constexpr int kMaxCtas = 296;
 
 // A problem split into more than kInlineMergeMax items is not merged by its
 // last-arriving CTA (one CTA reading every partial would be the tail of the
-// launch) but by the CTAs that finish streaming first, as its items' ready
-// flags come up.
+// launch) but by the whole grid at the launch's end: after a grid barrier,
+// or, for a problem over more than kWideMergeItems items, by the CTAs that
+// finish streaming first as its items' ready flags come up.
 constexpr int kInlineMergeMax = 16;
 
 // A deferred problem with more partials than this is merged a CTA per unit

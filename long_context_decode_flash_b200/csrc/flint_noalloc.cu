@@ -36,7 +36,8 @@ namespace {
 static_assert(FLINT_NOALLOC_SCRATCH_BYTES % 256 == 0, "scratch size is a multiple of 256 bytes");
 static_assert(FLINT_NOALLOC_SCRATCH_BYTES > kCounterBytes, "scratch holds the counters and partials");
 
-// The scratch: arrival counters and the grid-barrier word in its first
+// The scratch: the counter area (arrival counters, grid-barrier, queue,
+// abort and merge-ticket words, item ready flags) in its first
 // kCounterBytes, split partials after them (the workspace layout of
 // flint_attn_stack).
 static __device__ __align__(256) unsigned char g_scratch[FLINT_NOALLOC_SCRATCH_BYTES];
