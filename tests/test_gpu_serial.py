@@ -8,7 +8,8 @@ import torch
 from long_context_decode_flash_b200 import flint
 from long_context_decode_flash_b200 import inputs as I
 
-from helpers import DeviceLayer, bf16_ulp_diff, check_workspace_clean, e4m3_code_distance, oracle_layer, parity
+from helpers import (DeviceLayer, bf16_ulp_diff, check_workspace_clean, e4m3_code_distance, oracle_layer, parity,
+                     stack_on_gpu)
 
 pytestmark = pytest.mark.gpu
 
@@ -65,3 +66,20 @@ def test_serial_100k_sampled_layers():
     for i in (full[0], full[-1], 0, 48):
         want, _, _ = oracle_layer(layers[i])
         parity(got[i], want, f"layer {i}")
+
+
+def test_both_merge_modes_give_the_same_bits():
+    """A full layer at context 100,000, planned alone over every SM (148
+    partials), merges on ready flags when it is launched by itself
+    (flint_attn_stack of that one layer) and after the grid barrier when it
+    is the dependent second launch of the layer-serial path.  The plan, the
+    partials and the merge's batch boundaries are the same, so the outputs
+    agree bit for bit, and both match the oracle."""
+    L = 100_000
+    window = I.make_layer(I.W_STACK_100K + 61, 0, L, I.WINDOW, True, ring=True)
+    full = I.make_layer(I.W_STACK_100K + 61, 1, L, 0, False, ring=False)
+    flags, _ = stack_on_gpu([full], L - 1)
+    barrier, _ = serial_on_gpu([window, full], L - 1)
+    assert np.array_equal(flags[0], barrier[1])
+    want, _, _ = oracle_layer(full)
+    parity(flags[0], want, "full layer, ready-flag merge")
